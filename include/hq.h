@@ -1,0 +1,235 @@
+/*
+ * hq.h -- C ABI of the B200 (sm_100a) quantised-weight GEMM library.
+ *
+ * The operations follow the Humming kernel library as described in
+ * "Announcing Humming: Fast, Flexible Kernels for Quantized Inference":
+ *   - section "Unified quantization representation": weight format, scale
+ *     granularity, scale dtype, zero point and second-level scale are
+ *     independent parameters; the activation has its own format
+ *     (hq_quant_desc below);
+ *   - section "Tuning & JIT per workload": parameters are validated, dims
+ *     padded and tensors repacked into the kernel's layout (hq_pack_weights);
+ *   - section "Performance", WnA16 and W8A8/W4A8/W4A4: dense and MoE GEMMs,
+ *     MoE on "Indexed" and "Grouped" paths (hq_gemm, hq_moe_gemm);
+ * and the SGLang integration digest (PR #23754, humming_moe_runner_core_run,
+ * moe_permute_prepare, moe_permute / moe_unpermute, moe_fused_mul_sum) for
+ * the MoE call semantics (hq_moe_permute, hq_moe_gemm,
+ * hq_moe_unpermute_sum).
+ *
+ * Conventions for every call:
+ *   - All pointers are DEVICE pointers unless stated otherwise, 16-byte
+ *     aligned.  The caller allocates and owns every buffer and stream.  The
+ *     library allocates no device memory.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream) and never synchronises.
+ *   - Every call returns an hq_status and never aborts.  Argument errors are
+ *     detected on the host before any launch.  Errors that can only be seen
+ *     on the device (an expert id out of range, a pipeline wait that timed
+ *     out) are recorded in a per-device error word read by hq_device_error().
+ *   - Row-major layouts; `[a, b]` means a rows of b contiguous elements.
+ *   - Tensors the library consumes are in the "standard format":
+ *       INT4/UINT4 codes  int32 [E, N, K/8]: nibble j (bits 4j..4j+3) of word
+ *                         w is the code of k = 8w + j; INT4 two's complement.
+ *       INT4 zero points  int32 [E, N, ceil(G/8)] packed the same way along
+ *                         the group axis (G = K / w_group, or 1 per channel).
+ *       INT4 scales       bf16  [E, N, G].
+ *       E2M1 codes        uint8 [E, N, K/2], low nibble = even k.
+ *       E8M0 scales       uint8 [E, N, K/32] (MXFP4).
+ *       UE4M3 scales      uint8 [E, N, K/16] (NVFP4) + fp32 global [E].
+ *       E4M3 codes        uint8 [E, N, K] + fp32 per-channel scales [E, N].
+ *   - Decoded values: INT4 w = (q - z) * s (z = 0 when symmetric);
+ *     MXFP4 w = e2m1 * 2^(c - 127); NVFP4 w = e2m1 * ue4m3 * g;
+ *     FP8 w = e4m3 with the channel scale applied to the output.
+ *   - Accumulation is fp32; outputs are bf16 (round to nearest even).
+ */
+#ifndef HQ_H
+#define HQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define HQ_API __attribute__((visibility("default")))
+#else
+#define HQ_API
+#endif
+
+typedef struct CUstream_st *hq_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+  HQ_OK = 0,
+  HQ_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned pointer    */
+  HQ_ERR_UNSUPPORTED = 2,  /* valid description, combination not built     */
+  HQ_ERR_WORKSPACE = 3,    /* workspace smaller than *_workspace_bytes()   */
+  HQ_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed         */
+  HQ_ERR_TIMEOUT = 5,      /* a bounded device-side wait gave up           */
+  HQ_ERR_DEVICE_INDEX = 6, /* an expert id outside [0, E) seen on device   */
+  HQ_ERR_ARCH = 7          /* the current device is not sm_100             */
+} hq_status;
+
+/* Element formats used in hq_quant_desc. */
+typedef enum {
+  HQ_BF16 = 0,
+  HQ_FP32 = 1,
+  HQ_INT4 = 2,   /* signed 4-bit, two's complement                         */
+  HQ_UINT4 = 3,  /* unsigned 4-bit (asymmetric with zero points)           */
+  HQ_E2M1 = 4,   /* FP4 (OCP MX)                                           */
+  HQ_E4M3 = 5,   /* FP8 (OCP "fn"); as an activation: per-token fp32 scale */
+  HQ_E8M0 = 6,   /* power-of-two scale (OCP MX)                            */
+  HQ_UE4M3 = 7,  /* unsigned E4M3 block scale (NVFP4)                      */
+  HQ_MXFP8 = 8,  /* activation: E4M3 codes + E8M0 scale per 32 along K     */
+  HQ_NVFP4 = 9   /* activation: E2M1 codes + UE4M3 per 16 + fp32 global    */
+} hq_dtype;
+
+/*
+ * Unified quantisation description ("Announcing Humming", section "Unified
+ * quantization representation").  Supported weight descriptions:
+ *   INT4  + BF16 scales, w_group in {0 (per channel), 32, 64, 128}
+ *   UINT4 + BF16 scales + zero points, w_group in {32, 64, 128}
+ *   E2M1  + E8M0 scales, w_group = 32                       (MXFP4)
+ *   E2M1  + UE4M3 scales, w_group = 16, w_has_global = 1    (NVFP4)
+ *   E4M3  + FP32 per-channel scales, w_group = 0            (FP8)
+ * and every one of them with a_dtype in {BF16, E4M3, MXFP8, NVFP4}.
+ */
+typedef struct {
+  int32_t w_dtype;       /* HQ_INT4 | HQ_UINT4 | HQ_E2M1 | HQ_E4M3           */
+  int32_t w_group;       /* 0 = per output channel, else group size along K */
+  int32_t w_scale_dtype; /* HQ_BF16 | HQ_E8M0 | HQ_UE4M3 | HQ_FP32           */
+  int32_t w_has_zero;    /* 1: UINT4 zero points, same grouping as scales   */
+  int32_t w_has_global;  /* 1: FP32 second-level scale per expert (NVFP4)   */
+  int32_t a_dtype;       /* HQ_BF16 | HQ_E4M3 | HQ_MXFP8 | HQ_NVFP4          */
+} hq_quant_desc;
+
+typedef enum { HQ_MOE_GROUPED = 0, HQ_MOE_INDEXED = 1 } hq_moe_mode;
+
+/* Text for a status code (static storage). */
+HQ_API const char *hq_status_string(hq_status s);
+
+/* Reads and clears the current device's device-side error word after
+ * synchronising `stream`.  Returns HQ_OK, HQ_ERR_TIMEOUT or
+ * HQ_ERR_DEVICE_INDEX. */
+HQ_API hq_status hq_device_error(hq_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Weight repack ("Announcing Humming", section "Tuning & JIT per workload":
+ * validate, pad, repack into the kernel layout).
+ *
+ * hq_packed_weights_bytes: size of the opaque packed buffer for E experts of
+ *   N x K weights (0 if the description or sizes are unsupported).  N is
+ *   padded to 64 rows and K must be a multiple of 64.
+ * hq_pack_weights: standard-format codes / scales / zeros (device) and, for
+ *   NVFP4, `global_scale` (device fp32 [E]) -> `packed` (device,
+ *   hq_packed_weights_bytes).  `zeros` must be NULL unless w_has_zero;
+ *   `global_scale` NULL unless w_has_global.  Bit-exact and deterministic.
+ * hq_unpack_weights: the inverse, back to the standard format (for tests).
+ * ---------------------------------------------------------------------- */
+HQ_API size_t hq_packed_weights_bytes(const hq_quant_desc *desc, int E, int N, int K);
+HQ_API hq_status hq_pack_weights(const hq_quant_desc *desc, int E, int N, int K, const void *codes,
+                          const void *scales, const void *zeros, const float *global_scale,
+                          void *packed, hq_stream_t stream);
+HQ_API hq_status hq_unpack_weights(const hq_quant_desc *desc, int E, int N, int K, const void *packed,
+                            void *codes, void *scales, void *zeros, float *global_scale,
+                            hq_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Activation quantisation ("Announcing Humming", section "W8A8 / W4A8 /
+ * W4A4" and the MoE activation override in its usage section: tokenwise
+ * FP8, MXFP8, NVFP4 activations).  x: bf16 [M, K], K a multiple of 32.
+ *   a_dtype == HQ_E4M3: codes uint8 [M, K], scales fp32 [M];
+ *       s = amax_row / 448, q = e4m3(x / s) (s = 1 for an all-zero row).
+ *   a_dtype == HQ_MXFP8: codes uint8 [M, K], scales uint8 E8M0 [M, K/32];
+ *       e = floor(log2(amax_blk)) - 8 clamped to [-127, 127], code e + 127,
+ *       q = e4m3(x * 2^-e) (code 127 and q = 0 for an all-zero block).
+ *   a_dtype == HQ_NVFP4: codes uint8 [M, K/2] (low nibble = even k),
+ *       scales uint8 UE4M3 [M, K/16], global fp32 [1];
+ *       g = amax_tensor / 2688 (or *static_global if non-NULL; 1 for an
+ *       all-zero tensor), sb = ue4m3((amax_blk / 6) / g),
+ *       d = sb * g, q = e2m1(x / d) (q = 0 when d = 0).
+ * All conversions round to nearest even and saturate; fp32 IEEE steps in
+ * the order written.  `global_out` receives g (NVFP4 only).
+ * `workspace` (NVFP4 dynamic only): >= 16 bytes, may be NULL otherwise.
+ * ---------------------------------------------------------------------- */
+HQ_API hq_status hq_quant_act(const hq_quant_desc *desc, int M, int K, const void *x_bf16, void *codes,
+                       void *scales, float *global_out, const float *static_global,
+                       void *workspace, size_t ws_bytes, hq_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Dense GEMM: C[M, N] (bf16) = A[M, K] . W[N, K]^T with W the packed
+ * weights of one expert (E = 1) and A in desc->a_dtype:
+ *   BF16:  a = bf16 [M, K], a_scales = NULL
+ *   E4M3:  a = uint8 [M, K], a_scales = fp32 [M] (per token)
+ *   MXFP8: a = uint8 [M, K], a_scales = uint8 [M, K/32]
+ *   NVFP4: a = uint8 [M, K/2], a_scales = uint8 [M, K/16], a_global = fp32 [1]
+ * M >= 0 (M == 0 is a no-op), N >= 1, K a multiple of 64.
+ * `workspace` of hq_gemm_workspace_bytes() bytes; its split-K counters must
+ * be zero when first used (for example cudaMemset once after allocation);
+ * every completed call leaves them zero again.
+ * ---------------------------------------------------------------------- */
+HQ_API size_t hq_gemm_workspace_bytes(const hq_quant_desc *desc, int M, int N, int K);
+HQ_API hq_status hq_gemm(const hq_quant_desc *desc, int M, int N, int K, const void *packed_w,
+                  const void *a, const void *a_scales, const float *a_global, void *c_bf16,
+                  void *workspace, size_t ws_bytes, hq_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * MoE routing prepare (SGLang digest: moe_permute_prepare /
+ * moe_align_block_size).  topk_ids int32 [T, topk], values in [0, E).
+ * Slot s = t * topk + j.  Outputs (int32):
+ *   expert_offsets [E + 1]: exclusive prefix of per-expert slot counts;
+ *   perm [T * topk]: slot at each expert-sorted position (stable: slots of
+ *       one expert in increasing s);
+ *   inv_perm [T * topk]: position of each slot.
+ * An id outside [0, E) sets HQ_ERR_DEVICE_INDEX in the device error word
+ * and expert_offsets[E] = -1; hq_moe_gemm then writes nothing.
+ * ---------------------------------------------------------------------- */
+HQ_API hq_status hq_moe_permute(int T, int topk, int E, const int32_t *topk_ids, int32_t *expert_offsets,
+                         int32_t *perm, int32_t *inv_perm, hq_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * MoE expert GEMM ("Announcing Humming", section "Performance": Indexed and
+ * Grouped MoE paths; SGLang digest: humming_moe_runner_core_run with gemm
+ * types "indexed" and "grouped_contiguous").
+ *   packed_w: hq_pack_weights output for E experts of N x K.
+ *   a_bf16: activations in slot-independent token order: [T, K] when
+ *       a_per_slot == 0 (every slot of token t multiplies row t, the
+ *       gate-up case) or [T * topk, K] when a_per_slot == 1 (slot s
+ *       multiplies row s, the down case).  If desc->a_dtype is not BF16 the
+ *       activations are quantised on the fly with hq_quant_act's recipe.
+ *   expert_offsets / perm / inv_perm: hq_moe_permute outputs.
+ *   mode HQ_MOE_GROUPED: rows are first gathered expert-contiguous into the
+ *       workspace, then a grouped GEMM runs over them.
+ *   mode HQ_MOE_INDEXED: the GEMM gathers rows by index; no permuted copy.
+ *   combine == 0: out = Y bf16 [T * topk, N], Y[s] = a_row(s) . W_e(s)^T.
+ *   combine == 1: out bf16 [T, N],
+ *       out[t] = routed_scale * sum_j topk_weights[t, j] * Y[t * topk + j]
+ *       (fp32 sum over j in increasing j; Y rounded to bf16 first).
+ * The result does not depend on the mode.
+ * ---------------------------------------------------------------------- */
+HQ_API size_t hq_moe_workspace_bytes(hq_moe_mode mode, const hq_quant_desc *desc, int T, int topk, int E,
+                              int N, int K, int a_per_slot, int combine);
+HQ_API hq_status hq_moe_gemm(hq_moe_mode mode, const hq_quant_desc *desc, int T, int topk, int E, int N,
+                      int K, const void *packed_w, const void *a_bf16, int a_per_slot,
+                      const int32_t *expert_offsets, const int32_t *perm,
+                      const int32_t *inv_perm, const float *topk_weights, float routed_scale,
+                      int combine, void *out_bf16, void *workspace, size_t ws_bytes,
+                      hq_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Fused weighted top-k sum (SGLang digest: moe_fused_mul_sum, and
+ * moe_unpermute): out[t, n] = routed_scale * sum_j w[t, j] * y[r(t, j), n]
+ * with r(t, j) = inv_perm[t * topk + j] if inv_perm is non-NULL (y in
+ * expert-sorted order) else t * topk + j (y in slot order).  y bf16
+ * [T * topk, N]; out bf16 [T, N]; the sum is fp32 in increasing j.
+ * ---------------------------------------------------------------------- */
+HQ_API hq_status hq_moe_unpermute_sum(int T, int topk, int N, const void *y_bf16,
+                               const int32_t *inv_perm, const float *topk_weights,
+                               float routed_scale, void *out_bf16, hq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HQ_H */

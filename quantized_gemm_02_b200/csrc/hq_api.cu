@@ -1,0 +1,338 @@
+// C-ABI entry points of libhq: argument validation, workspace planning and
+// kernel dispatch.  Every call validates on the host, launches on the
+// caller's stream, allocates nothing and never synchronises (except
+// hq_device_error, whose job is to synchronise).
+#include <cuda_runtime.h>
+
+#include <cstring>
+
+#include "hq_internal.cuh"
+
+namespace hq {
+
+hq_status launch_pack(const Layout &L, int E, const void *codes, const void *scales, const void *zeros,
+                      const float *global_scale, void *packed, cudaStream_t st);
+hq_status launch_unpack(const Layout &L, int E, const void *packed, void *codes, void *scales, void *zeros,
+                        float *global_scale, cudaStream_t st);
+hq_status launch_quant_act(int afmt, int M, int K, const void *x, void *codes, void *scales, float *global_out,
+                           const float *static_global, void *workspace, cudaStream_t st);
+hq_status launch_act_decode(int afmt, int R, int K, const void *codes, const void *scales, const int32_t *idx,
+                            int div, void *out, cudaStream_t st);
+hq_status launch_gather_rows(int R, int K, const void *a, const int32_t *idx, int div, void *out, cudaStream_t st);
+hq_status launch_moe_permute(int T, int topk, int E, const int32_t *ids, int32_t *offsets, int32_t *perm,
+                             int32_t *inv, cudaStream_t st);
+hq_status launch_unpermute_sum(int T, int topk, int N, const void *y, const int32_t *inv, const float *w, float rs,
+                               void *out, cudaStream_t st);
+
+hq_status launch_stream_gemm(const Layout &L, const void *packed, const void *a_bf16, const float *row_scale,
+                             const float *a_global, int M, int moe, int E, const int32_t *offsets,
+                             const int32_t *perm, int a_indexed, int a_div, void *out, const StreamLaunch &s,
+                             void *workspace, cudaStream_t st);
+
+hq_status check_launch() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+}
+
+bool device_is_sm100() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return false;
+  if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return false;
+  return major == 10 && minor == 0;
+}
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Bytes of one activation row in its quantised storage and of its scales.
+static size_t act_code_bytes(int afmt, int K) { return afmt == A_NVFP4 ? (size_t)K / 2 : (size_t)K; }
+static size_t act_scale_bytes(int afmt, int K) {
+  switch (afmt) {
+    case A_FP8: return 4;
+    case A_MXFP8: return (size_t)K / 32;
+    case A_NVFP4: return (size_t)K / 16;
+    default: return 0;
+  }
+}
+
+// ---- workspace carving: regions placed in order, 256-byte aligned --------
+struct Carver {
+  uint8_t *base;
+  size_t off = 0;
+  void *take(size_t bytes) {
+    void *p = base ? base + off : nullptr;
+    off = align_up(off + bytes, 256);
+    return p;
+  }
+};
+
+// Dense GEMM plan (shared by the size query and the call).
+struct DensePlan {
+  Layout L;
+  int afmt;
+  StreamLaunch s;
+};
+
+static hq_status plan_dense(const hq_quant_desc *d, int M, int N, int K, DensePlan *pl) {
+  int fmt, afmt;
+  if (!d) return HQ_ERR_INVALID_ARG;
+  if (!weight_format(d, &fmt) || !act_format(d, &afmt)) return HQ_ERR_UNSUPPORTED;
+  if (M < 0 || N < 1 || !valid_k(d, K)) return HQ_ERR_INVALID_ARG;
+  pl->L = make_layout(fmt, d->w_group, N, K);
+  pl->afmt = afmt;
+  pl->s = plan_stream(M > 0 ? M : 1, 0, pl->L.NT, pl->L.KB, false);
+  return HQ_OK;
+}
+
+static size_t dense_ws(const DensePlan &pl, int M, int K, uint8_t *base, void **split_ws, void **a_dec) {
+  Carver c{base};
+  *split_ws = c.take(stream_workspace_bytes(pl.s, pl.L.NT));
+  *a_dec = (pl.afmt != A_BF16) ? c.take((size_t)M * K * 2) : nullptr;
+  return c.off;
+}
+
+// MoE plan.
+struct MoePlan {
+  Layout L;
+  int afmt;
+  StreamLaunch s;
+  int R;         // routed rows = T * topk
+  int src_rows;  // activation rows supplied by the caller
+};
+
+static hq_status plan_moe(const hq_quant_desc *d, int T, int topk, int E, int N, int K, int a_per_slot,
+                          MoePlan *pl) {
+  int fmt, afmt;
+  if (!d) return HQ_ERR_INVALID_ARG;
+  if (!weight_format(d, &fmt) || !act_format(d, &afmt)) return HQ_ERR_UNSUPPORTED;
+  if (T < 0 || topk < 1 || E < 1 || E > 1024 || N < 1 || !valid_k(d, K)) return HQ_ERR_INVALID_ARG;
+  if ((long)T * topk > (1L << 30)) return HQ_ERR_INVALID_ARG;
+  pl->L = make_layout(fmt, d->w_group, N, K);
+  pl->afmt = afmt;
+  pl->R = T * topk;
+  pl->src_rows = a_per_slot ? pl->R : T;
+  const int R = pl->R > 0 ? pl->R : 1;
+  const int active = R < E ? R : E;
+  const int avg = (R + active - 1) / active;
+  const int mt = avg <= 8 ? 8 : avg <= 16 ? 16 : 32;
+  long bound = (R + mt - 1) / mt + active;
+  if (bound > R) bound = R;
+  pl->s = plan_stream(avg, (int)bound, pl->L.NT, pl->L.KB, true);
+  return HQ_OK;
+}
+
+struct MoeWs {
+  void *split, *y, *a_bf16, *codes, *scales, *glob, *amax;
+};
+
+static size_t moe_ws(const MoePlan &pl, hq_moe_mode mode, int K, int N, int combine, uint8_t *base, MoeWs *w) {
+  Carver c{base};
+  w->split = c.take(stream_workspace_bytes(pl.s, pl.L.NT));
+  w->y = combine ? c.take((size_t)pl.R * N * 2) : nullptr;
+  const bool need_bf16_copy = (mode == HQ_MOE_GROUPED) || (pl.afmt != A_BF16);
+  const size_t rows_bf16 = (mode == HQ_MOE_GROUPED) ? (size_t)pl.R : (size_t)pl.src_rows;
+  w->a_bf16 = need_bf16_copy ? c.take(rows_bf16 * K * 2) : nullptr;
+  if (pl.afmt != A_BF16) {
+    w->codes = c.take((size_t)pl.src_rows * act_code_bytes(pl.afmt, K));
+    w->scales = c.take((size_t)pl.src_rows * act_scale_bytes(pl.afmt, K));
+    w->glob = c.take(16);
+    w->amax = c.take(16);
+  } else {
+    w->codes = w->scales = w->glob = w->amax = nullptr;
+  }
+  return c.off;
+}
+
+}  // namespace hq
+
+using namespace hq;
+
+extern "C" {
+
+const char *hq_status_string(hq_status s) {
+  switch (s) {
+    case HQ_OK: return "ok";
+    case HQ_ERR_INVALID_ARG: return "invalid argument";
+    case HQ_ERR_UNSUPPORTED: return "unsupported format combination or size";
+    case HQ_ERR_WORKSPACE: return "workspace too small";
+    case HQ_ERR_CUDA: return "CUDA error";
+    case HQ_ERR_TIMEOUT: return "device-side wait timed out";
+    case HQ_ERR_DEVICE_INDEX: return "expert id out of range";
+    case HQ_ERR_ARCH: return "device is not sm_100";
+    default: return "unknown status";
+  }
+}
+
+hq_status hq_device_error(hq_stream_t stream) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return HQ_ERR_CUDA;
+  int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_hq_error, sizeof(int)) != cudaSuccess) return HQ_ERR_CUDA;
+  if (v != 0 && cudaMemcpyToSymbol(g_hq_error, &zero, sizeof(int)) != cudaSuccess) return HQ_ERR_CUDA;
+  return (hq_status)v;
+}
+
+size_t hq_packed_weights_bytes(const hq_quant_desc *desc, int E, int N, int K) {
+  int fmt;
+  if (!weight_format(desc, &fmt) || E < 1 || N < 1 || !valid_k(desc, K)) return 0;
+  return make_layout(fmt, desc->w_group, N, K).stride * (size_t)E;
+}
+
+hq_status hq_pack_weights(const hq_quant_desc *desc, int E, int N, int K, const void *codes, const void *scales,
+                          const void *zeros, const float *global_scale, void *packed, hq_stream_t stream) {
+  int fmt;
+  if (!desc) return HQ_ERR_INVALID_ARG;
+  if (!weight_format(desc, &fmt)) return HQ_ERR_UNSUPPORTED;
+  if (E < 1 || N < 1 || !valid_k(desc, K)) return HQ_ERR_INVALID_ARG;
+  if (!codes || !scales || !packed) return HQ_ERR_INVALID_ARG;
+  if ((fmt == W_UINT4) != (zeros != nullptr)) return HQ_ERR_INVALID_ARG;
+  if ((fmt == W_NVFP4) != (global_scale != nullptr)) return HQ_ERR_INVALID_ARG;
+  if (!aligned16(codes) || !aligned16(packed) || ((uintptr_t)scales & 3u)) return HQ_ERR_INVALID_ARG;
+  if (!device_is_sm100()) return HQ_ERR_ARCH;
+  const Layout L = make_layout(fmt, desc->w_group, N, K);
+  return launch_pack(L, E, codes, scales, zeros, global_scale, packed, (cudaStream_t)stream);
+}
+
+hq_status hq_unpack_weights(const hq_quant_desc *desc, int E, int N, int K, const void *packed, void *codes,
+                            void *scales, void *zeros, float *global_scale, hq_stream_t stream) {
+  int fmt;
+  if (!desc) return HQ_ERR_INVALID_ARG;
+  if (!weight_format(desc, &fmt)) return HQ_ERR_UNSUPPORTED;
+  if (E < 1 || N < 1 || !valid_k(desc, K)) return HQ_ERR_INVALID_ARG;
+  if (!codes || !scales || !packed) return HQ_ERR_INVALID_ARG;
+  if ((fmt == W_UINT4) != (zeros != nullptr)) return HQ_ERR_INVALID_ARG;
+  if ((fmt == W_NVFP4) != (global_scale != nullptr)) return HQ_ERR_INVALID_ARG;
+  if (!device_is_sm100()) return HQ_ERR_ARCH;
+  const Layout L = make_layout(fmt, desc->w_group, N, K);
+  return launch_unpack(L, E, packed, codes, scales, zeros, global_scale, (cudaStream_t)stream);
+}
+
+hq_status hq_quant_act(const hq_quant_desc *desc, int M, int K, const void *x_bf16, void *codes, void *scales,
+                       float *global_out, const float *static_global, void *workspace, size_t ws_bytes,
+                       hq_stream_t stream) {
+  int afmt;
+  if (!desc) return HQ_ERR_INVALID_ARG;
+  if (!act_format(desc, &afmt)) return HQ_ERR_UNSUPPORTED;
+  if (afmt == A_BF16) return HQ_ERR_INVALID_ARG;
+  if (M < 0 || K < 32 || (K % 32) != 0) return HQ_ERR_INVALID_ARG;
+  if (M == 0) return HQ_OK;
+  if (!x_bf16 || !codes || !scales || !aligned16(x_bf16) || !aligned16(codes)) return HQ_ERR_INVALID_ARG;
+  if (afmt == A_NVFP4) {
+    if (!global_out && !static_global) return HQ_ERR_INVALID_ARG;
+    if (!static_global && (!workspace || ws_bytes < 16)) return HQ_ERR_WORKSPACE;
+  }
+  if (!device_is_sm100()) return HQ_ERR_ARCH;
+  return launch_quant_act(afmt, M, K, x_bf16, codes, scales, global_out, static_global, workspace,
+                          (cudaStream_t)stream);
+}
+
+size_t hq_gemm_workspace_bytes(const hq_quant_desc *desc, int M, int N, int K) {
+  DensePlan pl;
+  if (plan_dense(desc, M, N, K, &pl) != HQ_OK) return 0;
+  void *a, *b;
+  return dense_ws(pl, M, K, nullptr, &a, &b);
+}
+
+hq_status hq_gemm(const hq_quant_desc *desc, int M, int N, int K, const void *packed_w, const void *a,
+                  const void *a_scales, const float *a_global, void *c_bf16, void *workspace, size_t ws_bytes,
+                  hq_stream_t stream) {
+  DensePlan pl;
+  const hq_status ps = plan_dense(desc, M, N, K, &pl);
+  if (ps != HQ_OK) return ps;
+  if (M == 0) return HQ_OK;
+  if (!packed_w || !a || !c_bf16 || !aligned16(packed_w) || !aligned16(a)) return HQ_ERR_INVALID_ARG;
+  if (pl.afmt != A_BF16 && !a_scales) return HQ_ERR_INVALID_ARG;
+  if (pl.afmt == A_NVFP4 && !a_global) return HQ_ERR_INVALID_ARG;
+  void *split_ws, *a_dec;
+  const size_t need = dense_ws(pl, M, K, (uint8_t *)workspace, &split_ws, &a_dec);
+  if (!workspace || ws_bytes < need || !aligned16(workspace)) return HQ_ERR_WORKSPACE;
+  if (!device_is_sm100()) return HQ_ERR_ARCH;
+  cudaStream_t st = (cudaStream_t)stream;
+  const void *a_use = a;
+  const float *row_scale = nullptr;
+  if (pl.afmt != A_BF16) {
+    hq_status s = launch_act_decode(pl.afmt, M, K, a, a_scales, nullptr, 1, a_dec, st);
+    if (s != HQ_OK) return s;
+    a_use = a_dec;
+    if (pl.afmt == A_FP8) row_scale = (const float *)a_scales;
+  }
+  return launch_stream_gemm(pl.L, packed_w, a_use, row_scale, pl.afmt == A_NVFP4 ? a_global : nullptr, M, 0, 1,
+                            nullptr, nullptr, 0, 1, c_bf16, pl.s, split_ws, st);
+}
+
+hq_status hq_moe_permute(int T, int topk, int E, const int32_t *topk_ids, int32_t *expert_offsets, int32_t *perm,
+                         int32_t *inv_perm, hq_stream_t stream) {
+  if (T < 0 || topk < 1 || E < 1 || E > 1024) return HQ_ERR_INVALID_ARG;
+  if (!expert_offsets || (T > 0 && (!topk_ids || !perm || !inv_perm))) return HQ_ERR_INVALID_ARG;
+  if (!device_is_sm100()) return HQ_ERR_ARCH;
+  return launch_moe_permute(T, topk, E, topk_ids, expert_offsets, perm, inv_perm, (cudaStream_t)stream);
+}
+
+size_t hq_moe_workspace_bytes(hq_moe_mode mode, const hq_quant_desc *desc, int T, int topk, int E, int N, int K,
+                              int a_per_slot, int combine) {
+  MoePlan pl;
+  if (plan_moe(desc, T, topk, E, N, K, a_per_slot, &pl) != HQ_OK) return 0;
+  MoeWs w;
+  return moe_ws(pl, mode, K, N, combine, nullptr, &w);
+}
+
+hq_status hq_moe_gemm(hq_moe_mode mode, const hq_quant_desc *desc, int T, int topk, int E, int N, int K,
+                      const void *packed_w, const void *a_bf16, int a_per_slot, const int32_t *expert_offsets,
+                      const int32_t *perm, const int32_t *inv_perm, const float *topk_weights, float routed_scale,
+                      int combine, void *out_bf16, void *workspace, size_t ws_bytes, hq_stream_t stream) {
+  MoePlan pl;
+  if (mode != HQ_MOE_GROUPED && mode != HQ_MOE_INDEXED) return HQ_ERR_INVALID_ARG;
+  const hq_status ps = plan_moe(desc, T, topk, E, N, K, a_per_slot, &pl);
+  if (ps != HQ_OK) return ps;
+  if (T == 0) return HQ_OK;
+  if (!packed_w || !a_bf16 || !expert_offsets || !perm || !out_bf16) return HQ_ERR_INVALID_ARG;
+  if (!aligned16(packed_w) || !aligned16(a_bf16) || !aligned16(out_bf16)) return HQ_ERR_INVALID_ARG;
+  if (combine && (!topk_weights || (N % 8) != 0)) return HQ_ERR_INVALID_ARG;
+  (void)inv_perm;
+  MoeWs w;
+  const size_t need = moe_ws(pl, mode, K, N, combine, (uint8_t *)workspace, &w);
+  if (!workspace || ws_bytes < need || !aligned16(workspace)) return HQ_ERR_WORKSPACE;
+  if (!device_is_sm100()) return HQ_ERR_ARCH;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int div = a_per_slot ? 1 : topk;
+  const void *a_use = a_bf16;
+  const float *row_scale = nullptr;
+  const float *a_global = nullptr;
+  int a_indexed = (mode == HQ_MOE_INDEXED) ? 1 : 0;
+  hq_status s = HQ_OK;
+  if (pl.afmt != A_BF16) {
+    // quantise the caller's rows on the fly, then decode exactly to bf16
+    s = launch_quant_act(pl.afmt, pl.src_rows, K, a_bf16, w.codes, w.scales, (float *)w.glob, nullptr, w.amax, st);
+    if (s != HQ_OK) return s;
+    if (mode == HQ_MOE_GROUPED)
+      s = launch_act_decode(pl.afmt, pl.R, K, w.codes, w.scales, perm, div, w.a_bf16, st);
+    else
+      s = launch_act_decode(pl.afmt, pl.src_rows, K, w.codes, w.scales, nullptr, 1, w.a_bf16, st);
+    if (s != HQ_OK) return s;
+    a_use = w.a_bf16;
+    if (pl.afmt == A_FP8) row_scale = (const float *)w.scales;
+    if (pl.afmt == A_NVFP4) a_global = (const float *)w.glob;
+  } else if (mode == HQ_MOE_GROUPED) {
+    s = launch_gather_rows(pl.R, K, a_bf16, perm, div, w.a_bf16, st);
+    if (s != HQ_OK) return s;
+    a_use = w.a_bf16;
+  }
+  void *y = combine ? w.y : out_bf16;
+  s = launch_stream_gemm(pl.L, packed_w, a_use, row_scale, a_global, 0, 1, E, expert_offsets, perm, a_indexed, div,
+                         y, pl.s, w.split, st);
+  if (s != HQ_OK) return s;
+  if (combine) s = launch_unpermute_sum(T, topk, N, y, nullptr, topk_weights, routed_scale, out_bf16, st);
+  return s;
+}
+
+hq_status hq_moe_unpermute_sum(int T, int topk, int N, const void *y_bf16, const int32_t *inv_perm,
+                               const float *topk_weights, float routed_scale, void *out_bf16, hq_stream_t stream) {
+  if (T < 0 || topk < 1 || N < 8 || (N % 8) != 0) return HQ_ERR_INVALID_ARG;
+  if (T == 0) return HQ_OK;
+  if (!y_bf16 || !topk_weights || !out_bf16 || !aligned16(y_bf16) || !aligned16(out_bf16)) return HQ_ERR_INVALID_ARG;
+  if (!device_is_sm100()) return HQ_ERR_ARCH;
+  return launch_unpermute_sum(T, topk, N, y_bf16, inv_perm, topk_weights, routed_scale, out_bf16,
+                              (cudaStream_t)stream);
+}
+
+}  // extern "C"

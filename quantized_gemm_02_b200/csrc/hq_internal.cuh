@@ -1,0 +1,236 @@
+// Internal definitions shared by the sm_100a kernels of libhq.
+//
+// Packed weight layout (the "repack into the kernel's layout" step of
+// "Announcing Humming", section "Tuning & JIT per workload").  Per expert:
+//
+//   weights  [NT][KB][4 panels][32 lanes][16 B]           4-bit formats
+//            [NT][KB][4 panels][2 halves][32 lanes][16 B]  8-bit formats
+//   scales   [NT][G][64]   element = bf16 | E8M0 | UE4M3 (1 group = w_group
+//                          k's; per-channel scales use G = 1), FP8
+//                          per-channel scales are fp32 [NT][64]
+//   zeros    [NT][G][64]   uint8 (UINT4 only)
+//   global   fp32 (NVFP4 only)
+//
+// with NT = ceil(N / 64) row tiles, KB = K / 64 k-blocks.  One (row tile,
+// k-block) unit holds 64 rows x 64 k.  Inside it, panel p covers rows
+// 16p..16p+15; lane l of a warp reads its 16 bytes, which are exactly the
+// mma.sync m16n8k16 A-fragment values of that lane for the four k16 steps of
+// the k-block (4-bit) or two of them per half (8-bit).  Inside each 32-bit
+// word (one k16 step, 4-bit) the eight fragment values e0..e7 (e0,e1 = row
+// g, k 2t,2t+1; e2,e3 = row g+8; e4..e7 the same at k+8; g = l/4, t = l%4)
+// sit at nibble positions e0:0 e1:4 e2:1 e3:5 e4:2 e5:6 e6:3 e7:7, so
+// that (w >> 4i) & 0x000F000F yields fragment register i in both halves.
+// 8-bit words hold bytes [e0 e2 e1 e3] (first word) and [e4 e6 e5 e7].
+// INT4 codes are stored biased (u = q + 8) so every integer format decodes
+// as (u - z); signed INT4 uses z = 8.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/hq.h"
+
+namespace hq {
+
+// Internal weight formats.
+enum WFmt : int { W_INT4 = 0, W_UINT4 = 1, W_MXFP4 = 2, W_NVFP4 = 3, W_FP8 = 4, W_NFMT = 5 };
+// Internal activation formats.
+enum AFmt : int { A_BF16 = 0, A_FP8 = 1, A_MXFP8 = 2, A_NVFP4 = 3 };
+
+constexpr int TILE_N = 64;   // rows of W per tile
+constexpr int TILE_K = 64;   // k per k-block
+
+struct Layout {
+  int fmt;
+  int N, K, NT, KB, G, group;  // group = k per scale group (K for per-channel)
+  int wbits;                   // 4 or 8
+  int sbytes;                  // bytes per scale element (per-group scales)
+  size_t w_bytes, s_bytes, z_bytes, c_bytes, g_bytes;  // per expert
+  size_t w_off, s_off, z_off, c_off, g_off, stride;     // offsets inside an expert region
+  __host__ __device__ size_t unit_bytes() const { return (size_t)TILE_N * TILE_K * wbits / 8; }
+};
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Returns false if the description is not one of the supported ones.
+inline bool weight_format(const hq_quant_desc *d, int *fmt) {
+  if (!d) return false;
+  switch (d->w_dtype) {
+    case HQ_INT4:
+      if (d->w_scale_dtype != HQ_BF16 || d->w_has_zero || d->w_has_global) return false;
+      if (!(d->w_group == 0 || d->w_group == 32 || d->w_group == 64 || d->w_group == 128)) return false;
+      *fmt = W_INT4;
+      return true;
+    case HQ_UINT4:
+      if (d->w_scale_dtype != HQ_BF16 || !d->w_has_zero || d->w_has_global) return false;
+      if (!(d->w_group == 32 || d->w_group == 64 || d->w_group == 128)) return false;
+      *fmt = W_UINT4;
+      return true;
+    case HQ_E2M1:
+      if (d->w_has_zero) return false;
+      if (d->w_scale_dtype == HQ_E8M0 && d->w_group == 32 && !d->w_has_global) { *fmt = W_MXFP4; return true; }
+      if (d->w_scale_dtype == HQ_UE4M3 && d->w_group == 16 && d->w_has_global) { *fmt = W_NVFP4; return true; }
+      return false;
+    case HQ_E4M3:
+      if (d->w_scale_dtype != HQ_FP32 || d->w_group != 0 || d->w_has_zero || d->w_has_global) return false;
+      *fmt = W_FP8;
+      return true;
+    default:
+      return false;
+  }
+}
+
+// K must hold whole k-blocks and whole scale groups.
+inline bool valid_k(const hq_quant_desc *d, int K) {
+  if (K < 64 || (K % 64) != 0) return false;
+  return d->w_group == 0 || (K % d->w_group) == 0;
+}
+
+inline bool act_format(const hq_quant_desc *d, int *afmt) {
+  switch (d->a_dtype) {
+    case HQ_BF16: *afmt = A_BF16; return true;
+    case HQ_E4M3: *afmt = A_FP8; return true;
+    case HQ_MXFP8: *afmt = A_MXFP8; return true;
+    case HQ_NVFP4: *afmt = A_NVFP4; return true;
+    default: return false;
+  }
+}
+
+inline Layout make_layout(int fmt, int group, int N, int K) {
+  Layout L{};
+  L.fmt = fmt;
+  L.N = N;
+  L.K = K;
+  L.NT = (N + TILE_N - 1) / TILE_N;
+  L.KB = K / TILE_K;
+  L.group = (group == 0) ? K : group;
+  L.G = K / L.group;
+  L.wbits = (fmt == W_FP8) ? 8 : 4;
+  L.sbytes = (fmt == W_INT4 || fmt == W_UINT4) ? 2 : 1;
+  L.w_bytes = (size_t)L.NT * L.KB * L.unit_bytes();
+  L.s_bytes = (fmt == W_FP8) ? 0 : (size_t)L.NT * L.G * TILE_N * L.sbytes;
+  L.z_bytes = (fmt == W_UINT4) ? (size_t)L.NT * L.G * TILE_N : 0;
+  L.c_bytes = (fmt == W_FP8) ? (size_t)L.NT * TILE_N * 4 : 0;
+  L.g_bytes = (fmt == W_NVFP4) ? 16 : 0;
+  size_t off = 0;
+  L.w_off = off; off = align_up(off + L.w_bytes, 256);
+  L.s_off = off; off = align_up(off + L.s_bytes, 256);
+  L.z_off = off; off = align_up(off + L.z_bytes, 256);
+  L.c_off = off; off = align_up(off + L.c_bytes, 256);
+  L.g_off = off; off = align_up(off + L.g_bytes, 256);
+  L.stride = off;
+  return L;
+}
+
+// Device-side error word (one per device, module scope).  The library is
+// built as one translation unit (libhq.cu), so the definition lives here.
+__device__ int g_hq_error = 0;
+
+// Polling bound for every device-side wait: about one second.
+constexpr unsigned long long WAIT_LIMIT_NS = 1000000000ull;
+
+#ifdef __CUDACC__
+__device__ __forceinline__ void set_device_error(int code) { atomicCAS(&g_hq_error, 0, code); }
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long global_timer_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait: returns false (and records HQ_ERR_TIMEOUT) after about a
+// second without the phase completing.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_timer_ns();
+  while (true) {
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (global_timer_ns() - t0 > WAIT_LIMIT_NS) {
+      set_device_error(HQ_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// 1-D bulk copy global -> shared, completing on an mbarrier (16-byte
+// aligned addresses, size a multiple of 16).
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Same, with an L2 evict-first hint for data read exactly once (weights).
+__device__ __forceinline__ void bulk_g2s_stream(void *dst, const void *src, uint32_t bytes, uint64_t *bar,
+                                                uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], "
+      "%4;" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+#endif
+
+// Launch plan of the weight-streaming GEMM (hq_gemm_stream.cu).
+struct StreamLaunch {
+  int mt;            // token tile (8, 16, 32)
+  int mtiles;        // grid.y: token tiles (dense) or an upper bound on (expert, tile) pairs (MoE)
+  int splits;        // split-K factor
+  int kb_per_split;  // k-blocks per split
+};
+StreamLaunch plan_stream(int rows_bound, int mtiles_bound_moe, int NT, int KB, bool moe);
+size_t stream_workspace_bytes(const StreamLaunch &s, int NT);
+
+// Host-side helpers implemented in hq_api.cu.
+hq_status check_launch();
+bool device_is_sm100();
+
+}  // namespace hq

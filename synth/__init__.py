@@ -35,7 +35,7 @@ import torch
 
 __all__ = [
     "generator", "bf16_normal", "random_bytes", "int4_weights", "mxfp4_weights",
-    "nvfp4_weights_random", "routing_softmax_topk", "routing_zipf",
+    "nvfp4_weights_random", "fp8_weights_random", "routing_softmax_topk", "routing_zipf",
     "pack_nibbles_i32", "pack_nibbles_u8", "to_np_bits",
 ]
 
@@ -138,6 +138,15 @@ def nvfp4_weights_random(E: int, N: int, K: int, gen: torch.Generator, device: s
     sc = torch.randint(0x28, 0x50, (E, N, K // 16), generator=gen, dtype=torch.int32, device=device)
     g = torch.full((E,), 1.0 / 64.0, dtype=torch.float32, device=device)
     return {"codes": codes, "scales": sc.to(torch.uint8), "global": g}
+
+
+def fp8_weights_random(E: int, N: int, K: int, gen: torch.Generator, device: str = "cpu") -> dict:
+    """E4M3 codes uniform over the 254 finite codes (the two NaN codes
+    0x7F / 0xFF are never drawn); fp32 per-channel scales |N(0, 0.01)| + 1e-3."""
+    r = torch.randint(0, 254, (E, N, K), generator=gen, dtype=torch.int32, device=device)
+    codes = (r + (r >= 0x7F).to(torch.int32)).to(torch.uint8)
+    sc = torch.randn(E, N, generator=gen, dtype=torch.float32, device=device).abs() * 0.01 + 1e-3
+    return {"codes": codes, "scales": sc}
 
 
 def routing_softmax_topk(T: int, E: int, k: int, gen: torch.Generator, device: str = "cpu"):

@@ -23,3 +23,9 @@ def read_golden(name):
                 continue
             rows.append(line.split())
     return rows
+
+
+def pytest_sessionstart(session):
+    # build libhq.so in-tree if it is missing or older than its sources
+    from quantized_gemm_02_b200 import build as _b
+    _b.build()

@@ -1,0 +1,84 @@
+"""Host-side checks of the C-ABI library (no GPU needed): it loads, exports
+every entry point include/hq.h declares, and rejects bad arguments on the
+host before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import quantized_gemm_02_b200 as hq
+from hqtest import cdesc
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", h)).read()
+            names += re.findall(r"^HQ_API\s+[^(]*?\b(hq_\w+)\s*\(", txt, flags=re.M)
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    L = hq.lib()
+    names = declared_symbols()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(hq.EXPORTS) <= set(names)
+
+
+def test_status_strings():
+    for s in range(8):
+        assert hq.hq_status_string(s)
+    assert hq.hq_status_string(99) == "unknown status"
+
+
+def test_packed_size_queries():
+    # INT4 g128, N=4096, K=4096: 8 MiB codes + 32 groups x 64 rows x 2 B per tile row
+    n = hq.hq_packed_weights_bytes(cdesc("int4_g128"), 1, 4096, 4096)
+    assert n >= 4096 * 4096 // 2 + 4096 * 32 * 2
+    assert n < 4096 * 4096 // 2 * 1.05
+    # E experts scale linearly
+    assert hq.hq_packed_weights_bytes(cdesc("mxfp4"), 8, 256, 512) == 8 * hq.hq_packed_weights_bytes(cdesc("mxfp4"), 1, 256, 512)
+    # ragged N pads to 64 rows
+    assert hq.hq_packed_weights_bytes(cdesc("fp8"), 1, 65, 128) == hq.hq_packed_weights_bytes(cdesc("fp8"), 1, 128, 128)
+    # K not a multiple of 64 and unsupported descriptions give 0
+    assert hq.hq_packed_weights_bytes(cdesc("int4_g128"), 1, 64, 96) == 0
+    bad = cdesc("mxfp4")
+    bad.w_group = 16
+    assert hq.hq_packed_weights_bytes(bad, 1, 64, 128) == 0
+
+
+def test_workspace_queries_are_consistent():
+    d = cdesc("uint4_g128")
+    assert hq.hq_gemm_workspace_bytes(d, 16, 8192, 8192) > 0
+    dq = cdesc("nvfp4", "nvfp4")
+    # quantised activations need a decode buffer on top
+    assert hq.hq_gemm_workspace_bytes(dq, 32, 7168, 7168) >= 32 * 7168 * 2
+    m = hq.hq_moe_workspace_bytes(hq.HQ_MOE_GROUPED, cdesc("mxfp4"), 16, 8, 256, 4096, 7168, 0, 1)
+    assert m >= 16 * 8 * 4096 * 2 + 16 * 8 * 7168 * 2
+    assert hq.hq_moe_workspace_bytes(hq.HQ_MOE_INDEXED, cdesc("mxfp4"), 16, 8, 256, 4096, 7168, 0, 0) < m
+
+
+def test_host_validation_without_device():
+    d = cdesc("int4_g128")
+    with pytest.raises(hq.HQError) as e:
+        hq.hq_pack_weights(d, 1, 64, 100, 16, 16, None, None, 16, stream=0)
+    assert e.value.status == 1  # K not a multiple of 64
+    bad = cdesc("int4_g128")
+    bad.w_dtype = 99
+    with pytest.raises(hq.HQError) as e:
+        hq.hq_gemm(bad, 1, 64, 128, 16, 16, None, None, 16, 16, 0, stream=0)
+    assert e.value.status == 2
+    with pytest.raises(hq.HQError) as e:
+        hq.hq_gemm(d, 1, 64, 128, 16, 16, None, None, 16, None, 0, stream=0)
+    assert e.value.status == 3  # no workspace
+    with pytest.raises(hq.HQError) as e:
+        hq.hq_moe_permute(4, 2, 2000, 16, 16, 16, 16, stream=0)
+    assert e.value.status == 1  # E > 1024
+    # a zero-row GEMM is a no-op that succeeds without a device
+    hq.hq_gemm(d, 0, 64, 128, 16, 16, None, None, 16, None, 0, stream=0)

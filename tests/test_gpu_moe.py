@@ -1,0 +1,149 @@
+"""GPU parity of the MoE path: routing prepare (bit-exact), grouped and
+indexed expert GEMMs, fused weighted top-k sum, on-the-fly activation
+quantisation, and the invariants (grouped == indexed, E=1 top-1 == dense)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synth
+from hqtest import assert_close, cdesc, gpu_pack, make_weights, np_bits, oracle_decoder, oracle_quant
+
+pytestmark = pytest.mark.gpu
+
+
+def gpu_permute(ids_gpu, E):
+    import quantized_gemm_02_b200 as hq
+    T, k = ids_gpu.shape
+    off = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    inv = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    hq.hq_moe_permute(T, k, E, ids_gpu, off, perm, inv)
+    return off, perm, inv
+
+
+@pytest.mark.parametrize("T,E,k,zipf", [(1, 256, 8, False), (300, 64, 8, True), (2048, 256, 8, False),
+                                         (4096, 256, 8, True), (5, 3, 2, False)])
+def test_permute_bit_exact(T, E, k, zipf):
+    g = synth.generator(T + E)
+    ids, _ = synth.routing_zipf(T, E, k, 1.2, g) if zipf else synth.routing_softmax_topk(T, E, k, g)
+    off, perm, inv = gpu_permute(ids.cuda(), E)
+    torch.cuda.synchronize()
+    o_off, o_perm, o_inv = O.moe_permute(ids.numpy(), E)
+    assert np.array_equal(off.cpu().numpy(), o_off)
+    assert np.array_equal(perm.cpu().numpy(), o_perm)
+    assert np.array_equal(inv.cpu().numpy(), o_inv)
+
+
+def test_permute_rejects_bad_ids():
+    import quantized_gemm_02_b200 as hq
+    ids = torch.tensor([[0, 1], [2, 7]], dtype=torch.int32, device="cuda")
+    off, perm, inv = gpu_permute(ids, 4)
+    assert hq.hq_device_error() == 6
+    assert int(off[4].item()) == -1
+    assert hq.hq_device_error() == 0  # cleared
+
+
+def run_moe(mode, wname, aname, packed, T, k, E, N, K, a, a_per_slot, off, perm, inv, w, rs, combine):
+    import quantized_gemm_02_b200 as hq
+    d = cdesc(wname, aname)
+    wsb = hq.hq_moe_workspace_bytes(mode, d, T, k, E, N, K, a_per_slot, combine)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+    out = torch.empty((T if combine else T * k), N, dtype=torch.bfloat16, device="cuda")
+    hq.hq_moe_gemm(mode, d, T, k, E, N, K, packed, a, a_per_slot, off, perm, inv, w, rs, combine, out, ws, wsb)
+    return out
+
+
+def moe_case(wname, aname, T, E, k, N, K, a_per_slot, seed, zipf=False, device_weights=False):
+    """Inputs, the GPU results for both modes and both combine settings, and
+    the oracle's combined output / per-slot outputs."""
+    g = synth.generator(seed)
+    x = synth.bf16_normal((T * k if a_per_slot else T, K), g)
+    ids, wts = synth.routing_zipf(T, E, k, 1.2, g) if zipf else synth.routing_softmax_topk(T, E, k, g)
+    w = make_weights(wname, E, N, K, seed=seed + 1, device="cuda" if device_weights else "cpu")
+    packed = gpu_pack(wname, w, E, N, K)
+    off, perm, inv = gpu_permute(ids.cuda(), E)
+    res = {}
+    for mode in (0, 1):
+        for combine in (0, 1):
+            res[(mode, combine)] = run_moe(mode, wname, aname, packed, T, k, E, N, K, x.cuda(), a_per_slot, off,
+                                           perm, inv, wts.cuda(), 1.5, combine)
+    torch.cuda.synchronize()
+    xb = np_bits(x)
+    if aname == "bf16":
+        A, row = O.decode_act("bf16", xb.shape[0], K, xb)
+    else:
+        q, s, og = oracle_quant(aname, xb)
+        A, row = O.decode_act(aname, xb.shape[0], K, q, s, og)
+    slots_rows = np.arange(T * k) if a_per_slot else np.repeat(np.arange(T), k)
+    A_slots = A[slots_rows]
+    row_slots = None if row is None else row[slots_rows]
+    dec = oracle_decoder(wname, w, N, K)
+    out, bound, Y, B = O.moe(A_slots, ids.numpy(), wts.numpy(), dec, routed_scale=1.5, row_scale=row_slots)
+    return res, out, bound, Y, B, ids.numpy(), wts.numpy()
+
+
+@pytest.mark.parametrize("wname,aname", [("mxfp4", "bf16"), ("int4_g128", "bf16"), ("uint4_g64", "bf16"),
+                                         ("mxfp4", "mxfp8"), ("nvfp4", "nvfp4"), ("fp8", "fp8")])
+@pytest.mark.parametrize("a_per_slot", [0, 1])
+def test_moe_small(wname, aname, a_per_slot):
+    T, E, k, N, K = 23, 16, 4, 96, 256
+    res, out, bound, Y, B, ids, wts = moe_case(wname, aname, T, E, k, N, K, a_per_slot, seed=31, zipf=True)
+    # grouped and indexed agree bit for bit
+    assert torch.equal(res[(0, 0)], res[(1, 0)])
+    assert torch.equal(res[(0, 1)], res[(1, 1)])
+    assert_close(res[(0, 0)].cpu(), Y, B, what="per-slot Y")
+    # combine: Y is rounded to bf16 before the fp32 weighted sum, so the bound
+    # doubles (two bf16 roundings)
+    assert_close(res[(0, 1)].cpu(), out, bound, rel=8e-3, what="combined")
+
+
+def test_moe_single_expert_top1_equals_dense():
+    import quantized_gemm_02_b200 as hq
+    T, N, K = 17, 128, 512
+    g = synth.generator(3)
+    x = synth.bf16_normal((T, K), g).cuda()
+    w = make_weights("mxfp4", 1, N, K, seed=4)
+    packed = gpu_pack("mxfp4", w, 1, N, K)
+    ids = torch.zeros(T, 1, dtype=torch.int32, device="cuda")
+    wts = torch.ones(T, 1, dtype=torch.float32, device="cuda")
+    off, perm, inv = gpu_permute(ids, 1)
+    y = run_moe(0, "mxfp4", "bf16", packed, T, 1, 1, N, K, x, 0, off, perm, inv, wts, 1.0, 0)
+    d = cdesc("mxfp4")
+    wsb = hq.hq_gemm_workspace_bytes(d, T, N, K)
+    ws = torch.zeros(max(wsb, 16), dtype=torch.uint8, device="cuda")
+    c = torch.empty(T, N, dtype=torch.bfloat16, device="cuda")
+    hq.hq_gemm(d, T, N, K, packed, x, None, None, c, ws, wsb)
+    torch.cuda.synchronize()
+    assert torch.equal(y, c)
+
+
+@pytest.mark.parametrize("T", [1, 16])
+def test_config3_shapes_gate_up(T):
+    # MoE W4A16 MXFP4 gate-up GEMM at the full expert count: E=256, top-8,
+    # N=4096, K=7168; weights drawn on the GPU, oracle on sampled columns of
+    # the touched experts.
+    E, k, N, K = 256, 8, 4096, 7168
+    g = synth.generator(50 + T)
+    x = synth.bf16_normal((T, K), g)
+    ids, wts = synth.routing_softmax_topk(T, E, k, g)
+    w = make_weights("mxfp4", E, N, K, seed=60, device="cuda")
+    packed = gpu_pack("mxfp4", w, E, N, K)
+    off, perm, inv = gpu_permute(ids.cuda(), E)
+    out = {}
+    for mode in (0, 1):
+        out[mode] = run_moe(mode, "mxfp4", "bf16", packed, T, k, E, N, K, x.cuda(), 0, off, perm, inv, wts.cuda(),
+                            1.0, 1)
+    torch.cuda.synchronize()
+    assert torch.equal(out[0], out[1])
+    cols = np.sort(np.random.default_rng(T).choice(N, 128, replace=False))
+    A, _ = O.decode_act("bf16", T, K, np_bits(x))
+    codes, scales = w["codes"], w["scales"]
+
+    def dec(e):
+        c = synth.to_np_bits(codes[e][torch.as_tensor(cols, device="cuda")])
+        s = synth.to_np_bits(scales[e][torch.as_tensor(cols, device="cuda")])
+        return O.decode_weights(O.Desc("e2m1", 32, "e8m0"), len(cols), K, c, s)
+
+    ref, bound, _, _ = O.moe(np.repeat(A, k, axis=0), ids.numpy(), wts.numpy(), dec, 1.0)
+    assert_close(out[0].cpu()[:, torch.as_tensor(cols)], ref, bound, rel=8e-3, what=f"config3 T={T}")
