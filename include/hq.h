@@ -228,6 +228,31 @@ HQ_API hq_status hq_moe_unpermute_sum(int T, int topk, int N, const void *y_bf16
                                const int32_t *inv_perm, const float *topk_weights,
                                float routed_scale, void *out_bf16, hq_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Dense GEMM for callers that cannot allocate device memory (no counterpart
+ * in the pages; an addition of this library).
+ *
+ * Some callers cannot call cudaMalloc when they run a GEMM: code running
+ * inside a CUDA graph capture, embedded runtimes or allocator hooks that own
+ * all device memory, and plugins that are given no allocator.  This call
+ * computes exactly what hq_gemm computes, with the same arguments except the
+ * workspace: its scratch is one fixed array of 64 MiB inside the library's
+ * device image, which every GPU that loads the library holds until the
+ * process exits.
+ *   - Sizes whose workspace (hq_gemm_workspace_bytes) exceeds 64 MiB are
+ *     rejected with HQ_ERR_WORKSPACE before anything is launched.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current and caches it; make
+ *     that first call before any stream capture.
+ *   - The call allocates nothing; it clears the part of the array that must
+ *     start at zero (split-K tile counters) with cudaMemsetAsync on `stream`.
+ *   - Every call shares the one array and it keeps the last call's contents:
+ *     calls that overlap on the GPU (different streams, no ordering) race.
+ * ---------------------------------------------------------------------- */
+HQ_API hq_status hq_gemm_noalloc(const hq_quant_desc *desc, int M, int N, int K, const void *packed_w,
+                                 const void *a, const void *a_scales, const float *a_global, void *c_bf16,
+                                 hq_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

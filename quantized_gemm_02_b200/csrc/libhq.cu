@@ -5,3 +5,4 @@
 #include "hq_gemm_stream.cu"
 #include "hq_moe.cu"
 #include "hq_api.cu"
+#include "hq_noalloc.cu"
