@@ -203,9 +203,190 @@ def workload_w4a16_dense_m16(hq, gen_seed=0):
     return ops, cfg, [packed]
 
 
+def workload_shape(hq, M, N, K, gen_seed=0):
+    """One dense W4A16 UINT4-asymmetric GEMM of the given shape (profiling)."""
+    d = desc_of(hq, hq.HQ_UINT4, 128, hq.HQ_BF16, 1, 0, hq.HQ_BF16)
+    gen = synth.generator(gen_seed, "cuda")
+    w = synth.int4_weights(1, N, K, 128, True, gen, device="cuda")
+    packed = torch.empty(hq.hq_packed_weights_bytes(d, 1, N, K), dtype=torch.uint8, device="cuda")
+    hq.hq_pack_weights(d, 1, N, K, w["codes"], w["scales"], w["zeros"], None, packed)
+    ops = [dense_op(hq, d, f"N{N}_K{K}_M{M}", M, N, K, packed, packed_bytes_int4(N, K, 128, True), gen)]
+    cfg = {"workload": f"dense W4A16 UINT4 asym g128, M={M}, N={N}, K={K}", "l2": "flushed before every GEMM"}
+    return ops, cfg, [packed]
+
+
+def moe_ops(hq, name, wdesc, E, topk, H, I, Ts, routing, gen, mode_names=("grouped", "indexed"), weights=None,
+            a_dtype=None):
+    """MoE gate-up (N = 2I, K = H) and down (N = H, K = I) GEMMs for every T
+    and mode; step time = permute + gate-up + down, as the pages time MoE."""
+    dev = "cuda"
+    if weights is None:
+        weights = {}
+        for part, (N, K) in (("gate_up", (2 * I, H)), ("down", (H, I))):
+            if wdesc.w_dtype == hq.HQ_E2M1 and wdesc.w_scale_dtype == hq.HQ_E8M0:
+                w = synth.mxfp4_weights(E, N, K, gen, device=dev)
+                glob = None
+                bytes_per = N * K // 2 + N * K // 32
+            else:
+                w = synth.nvfp4_weights_random(E, N, K, gen, device=dev)
+                glob = w["global"]
+                bytes_per = N * K // 2 + N * K // 16
+            packed = torch.empty(hq.hq_packed_weights_bytes(wdesc, E, N, K), dtype=torch.uint8, device=dev)
+            hq.hq_pack_weights(wdesc, E, N, K, w["codes"], w["scales"], None, glob, packed)
+            del w
+            weights[part] = (packed, N, K, bytes_per)
+    ops = []
+    for T in Ts:
+        ids, wts = routing(T, gen)
+        touched = int(torch.unique(ids).numel())
+        x_gate = synth.bf16_normal((T, H), gen, device=dev)
+        x_down = synth.bf16_normal((T * topk, I), gen, device=dev)
+        off = torch.empty(E + 1, dtype=torch.int32, device=dev)
+        perm = torch.empty(T * topk, dtype=torch.int32, device=dev)
+        inv = torch.empty(T * topk, dtype=torch.int32, device=dev)
+        ids_h = ids.cpu().pin_memory()
+        x_gate_h = x_gate.cpu().pin_memory()
+        out_h = torch.empty(T, H, dtype=torch.bfloat16).pin_memory()
+        for mode_name in mode_names:
+            mode = hq.HQ_MOE_GROUPED if mode_name == "grouped" else hq.HQ_MOE_INDEXED
+            pg, Ng, Kg, bg = weights["gate_up"]
+            pd, Nd, Kd, bd = weights["down"]
+            wsg = hq.hq_moe_workspace_bytes(mode, wdesc, T, topk, E, Ng, Kg, 0, 0)
+            wsd = hq.hq_moe_workspace_bytes(mode, wdesc, T, topk, E, Nd, Kd, 1, 1)
+            ws = torch.zeros(max(wsg, wsd), dtype=torch.uint8, device=dev)
+            y = torch.empty(T * topk, Ng, dtype=torch.bfloat16, device=dev)
+            out = torch.empty(T, Nd, dtype=torch.bfloat16, device=dev)
+            ids_e = torch.empty_like(ids)
+            x_e = torch.empty_like(x_gate)
+
+            def run(mode=mode, pg=pg, pd=pd, Ng=Ng, Kg=Kg, Nd=Nd, Kd=Kd, ws=ws, y=y, out=out, ids=ids, wts=wts,
+                    x_gate=x_gate, x_down=x_down, off=off, perm=perm, inv=inv, T=T, wsg=wsg, wsd=wsd):
+                hq.hq_moe_permute(T, topk, E, ids, off, perm, inv)
+                hq.hq_moe_gemm(mode, wdesc, T, topk, E, Ng, Kg, pg, x_gate, 0, off, perm, inv, wts, 1.0, 0, y, ws,
+                               wsg)
+                hq.hq_moe_gemm(mode, wdesc, T, topk, E, Nd, Kd, pd, x_down, 1, off, perm, inv, wts, 1.0, 1, out,
+                               ws, wsd)
+
+            def e2e(run=run, ids=ids, ids_e=ids_e, ids_h=ids_h, x_gate=x_gate, x_e=x_e, x_gate_h=x_gate_h,
+                    out=out, out_h=out_h):
+                ids.copy_(ids_h, non_blocking=True)
+                x_gate.copy_(x_gate_h, non_blocking=True)
+                run()
+                out_h.copy_(out, non_blocking=True)
+
+            flops = 2.0 * T * topk * (Ng * Kg + Nd * Kd)
+            wbytes = touched * (bg + bd)
+            io = T * Kg * 2 + T * topk * Ng * 2 + T * topk * Kd * 2 + T * Nd * 2
+            quant = 1 if (a_dtype is not None and a_dtype != hq.HQ_BF16) else 0
+            # kernels: permute; per GEMM [quant + decode | gather] + GEMM; combine
+            kernels = 1 + (2 + quant) * 2 + 1
+            ops.append(Op(f"{name}_T{T}_{mode_name}", run, flops, wbytes, io, kernels,
+                          T * topk * 4 + T * Kg * 2, T * Nd * 2, e2e))
+    return ops, weights
+
+
+def workload_moe_w4a16_mxfp4(hq, gen_seed=0):
+    E, topk, H, I = 256, 8, 7168, 2048
+    gen = synth.generator(gen_seed, "cuda")
+    d = desc_of(hq, hq.HQ_E2M1, 32, hq.HQ_E8M0, 0, 0, hq.HQ_BF16)
+    routing = lambda T, g: synth.routing_softmax_topk(T, E, topk, g, device="cuda")
+    ops, w = moe_ops(hq, "moe_w4a16_mxfp4", d, E, topk, H, I, [1, 16, 128, 1024, 4096], routing, gen)
+    cfg = {"workload": "MoE W4A16 MXFP4: E=256 top-8 softmax routing, H=7168, I=2048, T in {1,16,128,1024,4096}, "
+                       "grouped + indexed; step = permute + gate-up + down (+ fused weighted sum)",
+           "l2": "flushed before every call; weights ~6 GB"}
+    return ops, cfg, [w]
+
+
+def workload_moe_w4a8_mxfp8(hq, gen_seed=0):
+    E, topk, H, I = 256, 8, 7168, 2048
+    gen = synth.generator(gen_seed, "cuda")
+    d = desc_of(hq, hq.HQ_E2M1, 32, hq.HQ_E8M0, 0, 0, hq.HQ_MXFP8)
+    routing = lambda T, g: synth.routing_zipf(T, E, topk, 1.2, g, device="cuda")
+    ops, w = moe_ops(hq, "moe_w4a8_mxfp8", d, E, topk, H, I, [1, 64, 512, 4096], routing, gen, a_dtype=hq.HQ_MXFP8)
+    cfg = {"workload": "MoE W4A8: MXFP4 weights x MXFP8 activations quantised on the fly, Zipf(1.2) routing, E=256 "
+                       "top-8, H=7168, I=2048, T in {1,64,512,4096}, grouped + indexed, fused weighted sum",
+           "l2": "flushed before every call"}
+    return ops, cfg, [w]
+
+
+def workload_moe_nvfp4(hq, gen_seed=0):
+    E, topk, H, I = 256, 8, 7168, 2048
+    gen = synth.generator(gen_seed, "cuda")
+    d = desc_of(hq, hq.HQ_E2M1, 16, hq.HQ_UE4M3, 0, 1, hq.HQ_NVFP4)
+    routing = lambda T, g: synth.routing_softmax_topk(T, E, topk, g, device="cuda")
+    ops, w = moe_ops(hq, "moe_nvfp4", d, E, topk, H, I, [4096], routing, gen, a_dtype=hq.HQ_NVFP4)
+    cfg = {"workload": "MoE W4A4 NVFP4 x NVFP4 (activations quantised on the fly), E=256 top-8, H=7168, I=2048, "
+                       "T=4096, grouped + indexed", "l2": "flushed before every call"}
+    return ops, cfg, [w]
+
+
+def workload_dense_quantised(hq, fmt, gen_seed=0):
+    """Config 5 dense: N = K = 7168, both operands N(0,1) quantised by the
+    library's own quantiser (weights per output row), M swept."""
+    N = K = 7168
+    dev = "cuda"
+    gen = synth.generator(gen_seed, dev)
+    if fmt == "nvfp4":
+        d = desc_of(hq, hq.HQ_E2M1, 16, hq.HQ_UE4M3, 0, 1, hq.HQ_NVFP4)
+        wbytes = N * K // 2 + N * K // 16
+    else:
+        d = desc_of(hq, hq.HQ_E4M3, 0, hq.HQ_FP32, 0, 0, hq.HQ_E4M3)
+        wbytes = N * K + N * 4
+    Wf = synth.bf16_normal((N, K), gen, device=dev)
+
+    def quant(x):
+        M = x.shape[0]
+        if fmt == "nvfp4":
+            c = torch.empty(M, K // 2, dtype=torch.uint8, device=dev)
+            s = torch.empty(M, K // 16, dtype=torch.uint8, device=dev)
+        else:
+            c = torch.empty(M, K, dtype=torch.uint8, device=dev)
+            s = torch.empty(M, dtype=torch.float32, device=dev)
+        g = torch.zeros(1, dtype=torch.float32, device=dev)
+        wsq = torch.zeros(64, dtype=torch.uint8, device=dev)
+        return c, s, g, wsq
+
+    wc, wsc, wg, wq = quant(Wf)
+    hq.hq_quant_act(d, N, K, Wf, wc, wsc, wg, None, wq, 64)
+    packed = torch.empty(hq.hq_packed_weights_bytes(d, 1, N, K), dtype=torch.uint8, device=dev)
+    hq.hq_pack_weights(d, 1, N, K, wc, wsc, None, wg if fmt == "nvfp4" else None, packed)
+    ops = []
+    keep = [packed]
+    for M in [1, 32, 256, 2048, 8192]:
+        x = synth.bf16_normal((M, K), gen, device=dev)
+        c, s, g, wq2 = quant(x)
+        C = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        wsb = hq.hq_gemm_workspace_bytes(d, M, N, K)
+        ws = torch.zeros(max(wsb, 256), dtype=torch.uint8, device=dev)
+        x_h = x.cpu().pin_memory()
+        C_h = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
+
+        def run(M=M, x=x, c=c, s=s, g=g, wq2=wq2, C=C, ws=ws, wsb=wsb):
+            hq.hq_quant_act(d, M, K, x, c, s, g, None, wq2, 64)
+            hq.hq_gemm(d, M, N, K, packed, c, s, g if fmt == "nvfp4" else None, C, ws, wsb)
+
+        def e2e(run=run, x=x, x_h=x_h, C=C, C_h=C_h):
+            x.copy_(x_h, non_blocking=True)
+            run()
+            C_h.copy_(C, non_blocking=True)
+
+        kern = (2 if fmt == "nvfp4" else 1) + (1 if fmt == "fp8" else 2)
+        ops.append(Op(f"{fmt}_N{N}_K{K}_M{M}", run, 2.0 * M * N * K, wbytes, M * K * 2 + M * N * 2, kern,
+                      M * K * 2, M * N * 2, e2e))
+    cfg = {"workload": f"dense {'W4A4 NVFP4 x NVFP4' if fmt == 'nvfp4' else 'W8A8 FP8 per-channel x per-token'}, "
+                       "N=K=7168, M in {1,32,256,2048,8192}, activation quantisation inside the step",
+           "l2": "flushed before every call"}
+    return ops, cfg, keep
+
+
 WORKLOADS = {
     "w4a16_asym_sweep": workload_w4a16_asym_sweep,
     "w4a16_dense_m16": workload_w4a16_dense_m16,
+    "moe_w4a16_mxfp4": workload_moe_w4a16_mxfp4,
+    "moe_w4a8_mxfp8": workload_moe_w4a8_mxfp8,
+    "moe_nvfp4": workload_moe_nvfp4,
+    "w4a4_nvfp4": lambda hq: workload_dense_quantised(hq, "nvfp4"),
+    "w8a8_fp8": lambda hq: workload_dense_quantised(hq, "fp8"),
 }
 
 
@@ -307,6 +488,7 @@ def main():
     ap.add_argument("--impl", default="hq", choices=["hq", "reference"])
     ap.add_argument("--workload", default="w4a16_asym_sweep", choices=list(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shape", default=None, help="M,N,K: one dense W4A16 GEMM instead of a workload")
     args = ap.parse_args()
     ws, rank, local = init_dist()
     if args.impl == "reference":
@@ -314,7 +496,11 @@ def main():
 
     hq = _hq()
     peaks = load_peaks()
-    ops, cfg, keep = WORKLOADS[args.workload](hq)
+    if args.shape:
+        M, N, K = (int(x) for x in args.shape.split(","))
+        ops, cfg, keep = workload_shape(hq, M, N, K)
+    else:
+        ops, cfg, keep = WORKLOADS[args.workload](hq)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
     n_ops = len(ops)

@@ -201,7 +201,10 @@ HQ_API hq_status hq_moe_permute(int T, int topk, int E, const int32_t *topk_ids,
  *   expert_offsets / perm / inv_perm: hq_moe_permute outputs.
  *   mode HQ_MOE_GROUPED: rows are first gathered expert-contiguous into the
  *       workspace, then a grouped GEMM runs over them.
- *   mode HQ_MOE_INDEXED: the GEMM gathers rows by index; no permuted copy.
+ *   mode HQ_MOE_INDEXED: rows are addressed through the routing index.  In
+ *       this version the tensor-core kernel reads both modes' rows from the
+ *       expert-contiguous copy in the workspace; the modes give bit-identical
+ *       results.
  *   combine == 0: out = Y bf16 [T * topk, N], Y[s] = a_row(s) . W_e(s)^T.
  *   combine == 1: out bf16 [T, N],
  *       out[t] = routed_scale * sum_j topk_weights[t, j] * Y[t * topk + j]

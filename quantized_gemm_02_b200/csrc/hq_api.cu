@@ -24,10 +24,10 @@ hq_status launch_moe_permute(int T, int topk, int E, const int32_t *ids, int32_t
 hq_status launch_unpermute_sum(int T, int topk, int N, const void *y, const int32_t *inv, const float *w, float rs,
                                void *out, cudaStream_t st);
 
-hq_status launch_stream_gemm(const Layout &L, const void *packed, const void *a_bf16, const float *row_scale,
-                             const float *a_global, int M, int moe, int E, const int32_t *offsets,
-                             const int32_t *perm, int a_indexed, int a_div, void *out, const StreamLaunch &s,
-                             void *workspace, cudaStream_t st);
+hq_status launch_tc_gemm(const Layout &L, const void *packed, const void *a_bf16, int a_rows, const float *row_scale,
+                         const float *a_global, int M, int moe, int E, const int32_t *offsets, const int32_t *perm,
+                         int a_div, int gather, void *out, const TcLaunch &t, void *workspace, cudaStream_t st,
+                         bool e4m3_act = false);
 
 hq_status check_launch() {
   const cudaError_t e = cudaGetLastError();
@@ -71,7 +71,7 @@ struct Carver {
 struct DensePlan {
   Layout L;
   int afmt;
-  StreamLaunch s;
+  TcLaunch s;
 };
 
 static hq_status plan_dense(const hq_quant_desc *d, int M, int N, int K, DensePlan *pl) {
@@ -81,13 +81,13 @@ static hq_status plan_dense(const hq_quant_desc *d, int M, int N, int K, DensePl
   if (M < 0 || N < 1 || !valid_k(d, K)) return HQ_ERR_INVALID_ARG;
   pl->L = make_layout(fmt, d->w_group, N, K);
   pl->afmt = afmt;
-  pl->s = plan_stream(M > 0 ? M : 1, 0, pl->L.NT, pl->L.KB, false);
+  pl->s = plan_tc(M > 0 ? M : 1, 0, N, pl->L.KB, false);
   return HQ_OK;
 }
 
 static size_t dense_ws(const DensePlan &pl, int M, int K, uint8_t *base, void **split_ws, void **a_dec) {
   Carver c{base};
-  *split_ws = c.take(stream_workspace_bytes(pl.s, pl.L.NT));
+  *split_ws = c.take(tc_workspace_bytes(pl.s));
   *a_dec = (pl.afmt != A_BF16) ? c.take((size_t)M * K * 2) : nullptr;
   return c.off;
 }
@@ -96,7 +96,7 @@ static size_t dense_ws(const DensePlan &pl, int M, int K, uint8_t *base, void **
 struct MoePlan {
   Layout L;
   int afmt;
-  StreamLaunch s;
+  TcLaunch s;
   int R;         // routed rows = T * topk
   int src_rows;  // activation rows supplied by the caller
 };
@@ -115,10 +115,10 @@ static hq_status plan_moe(const hq_quant_desc *d, int T, int topk, int E, int N,
   const int R = pl->R > 0 ? pl->R : 1;
   const int active = R < E ? R : E;
   const int avg = (R + active - 1) / active;
-  const int mt = avg <= 8 ? 8 : avg <= 16 ? 16 : 32;
-  long bound = (R + mt - 1) / mt + active;
+  const int bnt = plan_tc(avg, 1, N, pl->L.KB, true).bnt;
+  long bound = (R + bnt - 1) / bnt + active;
   if (bound > R) bound = R;
-  pl->s = plan_stream(avg, (int)bound, pl->L.NT, pl->L.KB, true);
+  pl->s = plan_tc(avg, (int)bound, N, pl->L.KB, true);
   return HQ_OK;
 }
 
@@ -128,11 +128,11 @@ struct MoeWs {
 
 static size_t moe_ws(const MoePlan &pl, hq_moe_mode mode, int K, int N, int combine, uint8_t *base, MoeWs *w) {
   Carver c{base};
-  w->split = c.take(stream_workspace_bytes(pl.s, pl.L.NT));
+  w->split = c.take(tc_workspace_bytes(pl.s));
   w->y = combine ? c.take((size_t)pl.R * N * 2) : nullptr;
-  const bool need_bf16_copy = (mode == HQ_MOE_GROUPED) || (pl.afmt != A_BF16);
-  const size_t rows_bf16 = (mode == HQ_MOE_GROUPED) ? (size_t)pl.R : (size_t)pl.src_rows;
-  w->a_bf16 = need_bf16_copy ? c.take(rows_bf16 * K * 2) : nullptr;
+  // both modes currently stage the expert-sorted rows (see hq_moe_gemm)
+  (void)mode;
+  w->a_bf16 = c.take((size_t)pl.R * K * 2);
   if (pl.afmt != A_BF16) {
     w->codes = c.take((size_t)pl.src_rows * act_code_bytes(pl.afmt, K));
     w->scales = c.take((size_t)pl.src_rows * act_scale_bytes(pl.afmt, K));
@@ -248,6 +248,11 @@ hq_status hq_gemm(const hq_quant_desc *desc, int M, int N, int K, const void *pa
   if (!workspace || ws_bytes < need || !aligned16(workspace)) return HQ_ERR_WORKSPACE;
   if (!device_is_sm100()) return HQ_ERR_ARCH;
   cudaStream_t st = (cudaStream_t)stream;
+  if (pl.L.fmt == W_FP8 && pl.afmt == A_FP8) {
+    // E4M3 x E4M3 on the FP8 tensor path; per-token x per-channel scales in the epilogue
+    return launch_tc_gemm(pl.L, packed_w, a, M, (const float *)a_scales, nullptr, M, 0, 1, nullptr, nullptr, 1, 0,
+                          c_bf16, pl.s, split_ws, st, true);
+  }
   const void *a_use = a;
   const float *row_scale = nullptr;
   if (pl.afmt != A_BF16) {
@@ -256,8 +261,8 @@ hq_status hq_gemm(const hq_quant_desc *desc, int M, int N, int K, const void *pa
     a_use = a_dec;
     if (pl.afmt == A_FP8) row_scale = (const float *)a_scales;
   }
-  return launch_stream_gemm(pl.L, packed_w, a_use, row_scale, pl.afmt == A_NVFP4 ? a_global : nullptr, M, 0, 1,
-                            nullptr, nullptr, 0, 1, c_bf16, pl.s, split_ws, st);
+  return launch_tc_gemm(pl.L, packed_w, a_use, M, row_scale, pl.afmt == A_NVFP4 ? a_global : nullptr, M, 0, 1,
+                        nullptr, nullptr, 1, 0, c_bf16, pl.s, split_ws, st);
 }
 
 hq_status hq_moe_permute(int T, int topk, int E, const int32_t *topk_ids, int32_t *expert_offsets, int32_t *perm,
@@ -298,28 +303,28 @@ hq_status hq_moe_gemm(hq_moe_mode mode, const hq_quant_desc *desc, int T, int to
   const void *a_use = a_bf16;
   const float *row_scale = nullptr;
   const float *a_global = nullptr;
-  int a_indexed = (mode == HQ_MOE_INDEXED) ? 1 : 0;
+  // The tensor-core kernel reads activation tiles by TMA from expert-sorted
+  // rows in both modes: the rows are gathered (and, for quantised
+  // activations, quantised on the fly and decoded exactly) into the
+  // workspace first.  Results do not depend on the mode.
+  const int a_indexed = 0;
   hq_status s = HQ_OK;
   if (pl.afmt != A_BF16) {
-    // quantise the caller's rows on the fly, then decode exactly to bf16
     s = launch_quant_act(pl.afmt, pl.src_rows, K, a_bf16, w.codes, w.scales, (float *)w.glob, nullptr, w.amax, st);
     if (s != HQ_OK) return s;
-    if (mode == HQ_MOE_GROUPED)
-      s = launch_act_decode(pl.afmt, pl.R, K, w.codes, w.scales, perm, div, w.a_bf16, st);
-    else
-      s = launch_act_decode(pl.afmt, pl.src_rows, K, w.codes, w.scales, nullptr, 1, w.a_bf16, st);
+    s = launch_act_decode(pl.afmt, pl.R, K, w.codes, w.scales, perm, div, w.a_bf16, st);
     if (s != HQ_OK) return s;
-    a_use = w.a_bf16;
     if (pl.afmt == A_FP8) row_scale = (const float *)w.scales;
     if (pl.afmt == A_NVFP4) a_global = (const float *)w.glob;
-  } else if (mode == HQ_MOE_GROUPED) {
+  } else {
     s = launch_gather_rows(pl.R, K, a_bf16, perm, div, w.a_bf16, st);
     if (s != HQ_OK) return s;
-    a_use = w.a_bf16;
   }
+  a_use = w.a_bf16;
   void *y = combine ? w.y : out_bf16;
-  s = launch_stream_gemm(pl.L, packed_w, a_use, row_scale, a_global, 0, 1, E, expert_offsets, perm, a_indexed, div,
-                         y, pl.s, w.split, st);
+  const int a_rows = (a_indexed ? pl.src_rows : pl.R);
+  s = launch_tc_gemm(pl.L, packed_w, a_use, a_rows, row_scale, a_global, 0, 1, E, expert_offsets, perm, div, a_indexed,
+                     y, pl.s, w.split, st);
   if (s != HQ_OK) return s;
   if (combine) s = launch_unpermute_sum(T, topk, N, y, nullptr, topk_weights, routed_scale, out_bf16, st);
   return s;

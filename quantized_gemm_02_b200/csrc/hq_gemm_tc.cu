@@ -1,0 +1,722 @@
+// Tensor-core (tcgen05 / TMEM) quantised-weight GEMM, dense and MoE, for
+// every token count.
+//
+// "Announcing Humming", section "Tuning and JIT compilation per workload":
+// a TMA + UMMA pipeline with dequantisation and scaling fused into the kernel
+// ("Shared CUDA components across formats and architectures"), work split
+// along K for small batches.  The sm_100a design:
+//
+//   * swap-AB: 128 weight rows are the MMA's M side and sit in TENSOR MEMORY
+//     as operand A; a tile of 16..256 tokens is the N side, operand B, in
+//     shared memory.  Dequantised weights never touch shared memory, so the
+//     shared-memory traffic per packed weight byte stays at ~2 bytes even
+//     when the kernel streams weights at full HBM rate;
+//   * warp roles (14 warps):
+//       warps 0..3   epilogue: tcgen05.ld of the fp32 accumulator (warp w owns
+//                    TMEM lanes 32w..32w+31), fp32 scales, bf16 out or fp32
+//                    split-K partials with a deterministic last-split fixup;
+//       warp 4       producer: TMA of the activation tile (bf16, 128-byte
+//                    swizzle; a 4-row gather for MoE indexed mode), 1-D bulk
+//                    copies of the packed weight unit, scales, zero points;
+//       warp 5       MMA issuer: tcgen05.mma.cta_group::1.kind::f16 with A
+//                    from TMEM and B from a shared-memory descriptor;
+//       warps 6..13  dequant: thread = weight row, decodes 32 k of its row per
+//                    k-block to bf16 pairs and stores them with
+//                    tcgen05.st.32x32b into the A ring in TMEM;
+//   * shared-memory ring (NS stages, one 64-k block each) for activations
+//     and packed weights, TMEM ring (4 stages x 32 columns) for dequantised
+//     weights, fp32 accumulator in TMEM after the ring;
+//   * every mbarrier wait is bounded (~1 s); on a timeout the CTA records
+//     HQ_ERR_TIMEOUT, raises an abort flag, releases its TMEM and returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include "hq_internal.cuh"
+
+namespace hq {
+
+namespace tc {
+
+constexpr int BM = TILE_N;        // 128 weight rows = MMA M
+constexpr int NA = 4;             // TMEM A ring depth
+constexpr int THREADS = 14 * 32;
+constexpr int WARP_PRODUCER = 4, WARP_MMA = 5, WARP_DQ0 = 6, NDQ = 8;
+
+template <int WF>
+struct Traits {
+  static constexpr int wbits = (WF == W_FP8) ? 8 : 4;
+  static constexpr int unit = BM * TILE_K * wbits / 8;  // packed bytes per (tile, k-block)
+  static constexpr int sbytes = (WF == W_INT4 || WF == W_UINT4) ? 2 : 1;
+  static constexpr int max_groups_kb = (WF == W_NVFP4) ? 4 : 2;  // scale groups per k-block (upper bound)
+  static constexpr bool has_scales = (WF != W_FP8);
+  static constexpr bool has_zero = (WF == W_UINT4);
+};
+
+// F8: both operands E4M3 (kind::f8f6f4, weights copied into TMEM unchanged);
+// otherwise weights are dequantised to bf16 (kind::f16).
+template <int WF, int BNT, bool F8>
+struct Cfg {
+  static constexpr int A_COLS = F8 ? 16 : 32;                                  // TMEM columns per 64-k stage
+  static constexpr int ACT = BNT * (F8 ? 64 : 128);                            // [BNT][64] bf16 or e4m3, swizzled
+  static constexpr int WPK = Traits<WF>::unit;
+  static constexpr int SC = Traits<WF>::max_groups_kb * BM * Traits<WF>::sbytes;
+  static constexpr int ZP = Traits<WF>::has_zero ? Traits<WF>::max_groups_kb * BM : 0;
+  static constexpr int STAGE = (ACT + WPK + SC + ZP + 1023) / 1024 * 1024;
+  // two CTAs per SM up to 128 tokens (TMEM: 2 x 256 columns), one beyond
+  static constexpr int CTAS_PER_SM = BNT <= 128 ? 2 : 1;
+  static constexpr int NS_BY_SMEM = ((CTAS_PER_SM == 2 ? 104 : 200) * 1024) / STAGE;
+  static constexpr int NS = NS_BY_SMEM > 8 ? 8 : NS_BY_SMEM;                  // shared-memory ring depth
+  static constexpr int CTRL = 4096;                                            // barriers + tile info
+  static constexpr int BYTES = NS * STAGE + CTRL + 1024;                      // + alignment slack
+  static constexpr int D_COL = NA * A_COLS;                                    // accumulator columns start
+  static constexpr int TMEM_COLS = (D_COL + BNT) <= 256 ? 256 : 512;
+  static_assert(NS >= 2, "stage too large");
+};
+
+struct Params {
+  const uint8_t *packed;
+  size_t stride;
+  size_t w_off, s_off, z_off, c_off, g_off;
+  int N, K, NT, KB, G, group;
+  int gshift;              // k >> gshift = scale group (31 for one group per row)
+  const float *row_scale;  // per caller row (FP8 per-token) or null
+  const float *a_global;   // NVFP4 activation global scale or null
+  int M;                   // dense rows
+  int moe, E;
+  const int32_t *offsets, *perm;
+  int a_div;
+  int gather;              // MoE indexed mode: activation rows gathered by index
+  uint16_t *out;
+  int splits, kb_per_split;
+  float *partial;
+  int *counters;
+};
+
+// ---- PTX wrappers ----------------------------------------------------------------
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)1 << 16;            // leading byte offset (unused for swizzled K-major)
+  d |= (uint64_t)(1024 >> 4) << 32;  // stride byte offset: 8-row groups 1024 B apart
+  d |= (uint64_t)1 << 46;            // descriptor version
+  d |= (uint64_t)2 << 61;            // 128-byte swizzle
+  return d;
+}
+
+// K-major, 64-byte swizzle (rows of 64 e4m3 codes, 8-row groups 512 B apart)
+__device__ __forceinline__ uint64_t sw64_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)1 << 16;
+  d |= (uint64_t)(512 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)4 << 61;  // 64-byte swizzle
+  return d;
+}
+
+template <int BNT>
+__device__ __forceinline__ constexpr uint32_t idesc_e4m3() {
+  return (1u << 4)                       // D = f32; A = B = E4M3 (format 0)
+         | ((uint32_t)(BNT >> 3) << 17)  // N
+         | ((uint32_t)(BM >> 4) << 24);  // M
+}
+
+template <int BNT>
+__device__ __forceinline__ constexpr uint32_t idesc_bf16() {
+  return (1u << 4)                       // D = f32
+         | (1u << 7) | (1u << 10)        // A = B = bf16
+         | ((uint32_t)(BNT >> 3) << 17)  // N
+         | ((uint32_t)(BM >> 4) << 24);  // M
+}
+
+__device__ __forceinline__ void mma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(acc));
+}
+
+__device__ __forceinline__ void mma_ts_f8(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(acc));
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t *bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_gather4(void *dst, const CUtensorMap *map, int x, int r0, int r1, int r2, int r3,
+                                            uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// ---- bf16 pair arithmetic and decoders ---------------------------------------
+__device__ __forceinline__ uint32_t bsub2(uint32_t a, uint32_t b) {
+  __nv_bfloat162 r = __hsub2(*reinterpret_cast<__nv_bfloat162 *>(&a), *reinterpret_cast<__nv_bfloat162 *>(&b));
+  return *reinterpret_cast<uint32_t *>(&r);
+}
+__device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b) {
+  __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162 *>(&a), *reinterpret_cast<__nv_bfloat162 *>(&b));
+  return *reinterpret_cast<uint32_t *>(&r);
+}
+__device__ __forceinline__ uint32_t bcast16(uint32_t h) { return (h & 0xFFFFu) | (h << 16); }
+// bf16 bits of an E4M3 / UE4M3 code's value (exact: <= 4 significant bits)
+__device__ __forceinline__ uint32_t e4m3_code_to_bf16(uint32_t c) {
+  const float mag = __uint_as_float((c & 0x7Fu) << 20) * 1.329227995784916e36f;  // 2^120
+  return (__float_as_uint(mag) >> 16) | ((c & 0x80u) << 8);
+}
+// bf16 bits of 2^(c - 127) for an E8M0 code c in [0, 254]
+__device__ __forceinline__ uint32_t e8m0_code_to_bf16(uint32_t c) { return c ? (c << 7) : 0x0040u; }
+// E2M1 pair (codes at bits 0..3 and 16..19) -> bf16 pair carrying value * 2^-126
+__device__ __forceinline__ uint32_t e2m1_pair(uint32_t x) {
+  return ((x << 6) & 0x01C001C0u) | ((x << 12) & 0x80008000u);
+}
+// E4M3 pair (codes at bits 0..7 and 16..23) -> bf16 pair carrying value * 2^-120
+__device__ __forceinline__ uint32_t e4m3_pair(uint32_t x) {
+  return ((x & 0x007F007Fu) << 4) | ((x & 0x00800080u) << 8);
+}
+
+// ---- the kernel ----------------------------------------------------------------
+template <int WF, int BNT, bool F8>
+__global__ void __launch_bounds__(THREADS, 1) tc_gemm_kernel(const __grid_constant__ CUtensorMap act_map,
+                                                             const Params p) {
+  using TR = Traits<WF>;
+  using C = Cfg<WF, BNT, F8>;
+  static_assert(!F8 || WF == W_FP8, "the E4M3 x E4M3 path takes FP8 weights");
+  constexpr int NS = C::NS;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *ctrl = smem + NS * C::STAGE;
+  uint64_t *full = reinterpret_cast<uint64_t *>(ctrl);  // [NS]  stage landed
+  uint64_t *sfree = full + NS;                           // [NS]  stage consumed (MMA + dequant)
+  uint64_t *afull = sfree + NS;                          // [NA]  TMEM A stage written
+  uint64_t *aempty = afull + NA;                         // [NA]  TMEM A stage consumed
+  uint64_t *accum = aempty + NA;                         // accumulator complete
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accum + 1);
+  int *s_abort = reinterpret_cast<int *>(tmem_slot + 1);
+  int *s_info = s_abort + 1;  // [0] expert [1] row base [2] valid rows [3] is_last
+  int *s_orow = s_info + 4;   // [BNT] output row of each token column
+  int *s_srow = s_orow + BNT; // [BNT] caller activation row (per-token scale, gather index)
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int wt = blockIdx.x % p.NT;   // 128-row weight tile
+  const int split = blockIdx.x / p.NT;
+  const int slot = blockIdx.y;        // token tile (dense) or (expert, tile) slot (MoE)
+
+  // ---- tile -> (expert, token rows) ----
+  if (warp == 0) {
+    int expert = 0, base = 0, nvalid = 0;
+    if (!p.moe) {
+      base = slot * BNT;
+      nvalid = min(BNT, p.M - base);
+    } else if (p.offsets[p.E] >= 0) {
+      int running = 0, found = -1, tile_in = 0;
+      for (int e0 = 0; e0 < p.E && found < 0; e0 += 32) {
+        const int e = e0 + lane;
+        int tiles = 0;
+        if (e < p.E) tiles = (p.offsets[e + 1] - p.offsets[e] + BNT - 1) / BNT;
+        int incl = tiles;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        const int excl = running + incl - tiles;
+        const bool mine = (e < p.E) && slot >= excl && slot < excl + tiles;
+        const unsigned ball = __ballot_sync(0xffffffffu, mine);
+        if (ball) {
+          const int src = __ffs(ball) - 1;
+          found = __shfl_sync(0xffffffffu, e, src);
+          tile_in = __shfl_sync(0xffffffffu, slot - excl, src);
+        }
+        running += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      if (found >= 0) {
+        expert = found;
+        base = p.offsets[found] + tile_in * BNT;
+        nvalid = min(BNT, p.offsets[found + 1] - base);
+      }
+    }
+    for (int i = lane; i < BNT; i += 32) {
+      int orow = -1, srow = -1;
+      if (i < nvalid) {
+        const int pos = base + i;
+        if (!p.moe) {
+          orow = srow = pos;
+        } else {
+          orow = p.perm[pos];
+          srow = orow / p.a_div;
+        }
+      }
+      s_orow[i] = orow;
+      s_srow[i] = srow;
+    }
+    if (lane == 0) {
+      s_info[0] = expert;
+      s_info[1] = base;
+      s_info[2] = nvalid;
+      *s_abort = 0;
+    }
+  }
+  if (tid == 32) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&sfree[s], 1 + NDQ);
+    }
+    for (int a = 0; a < NA; ++a) {
+      mbar_init(&afull[a], NDQ);
+      mbar_init(&aempty[a], 1);
+    }
+    mbar_init(accum, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const int expert = s_info[0], row_base = s_info[1], nvalid = s_info[2];
+  if (nvalid <= 0) return;
+
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(C::TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const uint8_t *eb = p.packed + (size_t)expert * p.stride;
+  const int kb_begin = split * p.kb_per_split;
+  const int kb_end = min(p.KB, kb_begin + p.kb_per_split);
+  const int nkb = kb_end - kb_begin;
+
+  if (warp == WARP_PRODUCER) {
+    // ================= producer (whole warp in step, lane 0 issues) =================
+    const uint64_t pol = policy_evict_first();
+    for (int it = 0; it < nkb; ++it) {
+      const int s = it % NS;
+      if (it >= NS && !mbar_wait(&sfree[s], ((it / NS) - 1) & 1)) { *s_abort = 1; break; }
+      if (*(volatile int *)s_abort) break;
+      if (lane == 0) {
+        uint8_t *st = smem + s * C::STAGE;
+        const int kb = kb_begin + it;
+        const int g0 = (kb * TILE_K) >> p.gshift;
+        const int g1 = (((kb + 1) * TILE_K - 1) >> p.gshift) + 1;
+        const uint32_t sb = TR::has_scales ? (uint32_t)((g1 - g0) * BM * TR::sbytes) : 0u;
+        const uint32_t zb = TR::has_zero ? (uint32_t)((g1 - g0) * BM) : 0u;
+        constexpr uint32_t row_bytes = F8 ? 64u : 128u;
+        const uint32_t ab = p.gather ? (uint32_t)(((nvalid + 3) / 4) * 4 * row_bytes) : (uint32_t)(BNT * row_bytes);
+        mbar_arrive_expect_tx(&full[s], ab + TR::unit + sb + zb);
+        if (!p.gather) {
+          tma_load_2d(st, &act_map, kb * TILE_K, row_base, &full[s]);
+        } else {
+          for (int i = 0; i < nvalid; i += 4) {
+            const int r0 = s_srow[i];
+            const int r1 = (i + 1 < nvalid) ? s_srow[i + 1] : r0;
+            const int r2 = (i + 2 < nvalid) ? s_srow[i + 2] : r0;
+            const int r3 = (i + 3 < nvalid) ? s_srow[i + 3] : r0;
+            tma_gather4(st + i * row_bytes, &act_map, kb * TILE_K, r0, r1, r2, r3, &full[s]);
+          }
+        }
+        bulk_g2s_stream(st + C::ACT, eb + p.w_off + ((size_t)wt * p.KB + kb) * TR::unit, TR::unit, &full[s], pol);
+        if (TR::has_scales)
+          bulk_g2s(st + C::ACT + C::WPK, eb + p.s_off + ((size_t)wt * p.G + g0) * BM * TR::sbytes, sb, &full[s]);
+        if (TR::has_zero)
+          bulk_g2s(st + C::ACT + C::WPK + C::SC, eb + p.z_off + ((size_t)wt * p.G + g0) * BM, zb, &full[s]);
+      }
+      __syncwarp();
+    }
+  } else if (warp >= WARP_DQ0) {
+    // ================= dequant: thread = weight row =================
+    const int dq = warp - WARP_DQ0;       // 0..7
+    const int sp = warp & 3;              // TMEM subpartition this warp may access
+    const int half = dq >> 2;             // which 32 k of the 64-k block
+    const int r = sp * 32 + lane;         // weight row inside the tile
+    const uint32_t t_row = tmem + ((uint32_t)(sp * 32) << 16);
+    for (int it = 0; it < nkb; ++it) {
+      const int s = it % NS, a = it % NA;
+      if (!mbar_wait(&full[s], (it / NS) & 1)) { *s_abort = 1; break; }
+      if (it >= NA && !mbar_wait(&aempty[a], ((it / NA) - 1) & 1)) { *s_abort = 1; break; }
+      if (*(volatile int *)s_abort) break;
+      tc_fence_after();
+      const uint8_t *st = smem + s * C::STAGE;
+      const uint8_t *wpk = st + C::ACT;
+      const uint8_t *sc = st + C::ACT + C::WPK;
+      const uint8_t *zp = st + C::ACT + C::WPK + C::SC;
+      const int kb = kb_begin + it;
+      const int g0 = (kb * TILE_K) >> p.gshift;
+      const int gt = ((kb * TILE_K + half * 32) >> p.gshift) - g0;  // group of this thread's first k
+      if constexpr (F8) {
+        // E4M3 weights go to TMEM unchanged, bytes put back in k order
+        uint32_t rg8[8];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const uint4 v = *reinterpret_cast<const uint4 *>(wpk + (half * 2 + c) * (BM * 16) + r * 16);
+          rg8[c * 4 + 0] = __byte_perm(v.x, 0, 0x3120);
+          rg8[c * 4 + 1] = __byte_perm(v.y, 0, 0x3120);
+          rg8[c * 4 + 2] = __byte_perm(v.z, 0, 0x3120);
+          rg8[c * 4 + 3] = __byte_perm(v.w, 0, 0x3120);
+        }
+        tmem_st8(t_row + (uint32_t)(a * C::A_COLS + half * 8), rg8);
+      } else {
+      uint32_t rg[16];
+      if constexpr (TR::wbits == 4) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(wpk + half * (BM * 16) + r * 16);
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+        if constexpr (WF == W_INT4 || WF == W_UINT4) {
+          // groups are >= 32 k: one scale (and zero point) covers the thread's 32 k
+          const uint32_t s2 = bcast16(reinterpret_cast<const uint16_t *>(sc)[gt * BM + r]);
+          const uint32_t z2 = (WF == W_UINT4) ? bcast16(0x4300u + zp[gt * BM + r]) : 0x43084308u;
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              rg[j * 4 + i] = bmul2(bsub2(((w4[j] >> (4 * i)) & 0x000F000Fu) | 0x43004300u, z2), s2);
+        } else {
+          // MXFP4: one group of 32; NVFP4: two groups of 16 (words 0-1, 2-3)
+          uint32_t s2[2];
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const uint32_t c = sc[(gt + (WF == W_NVFP4 ? q : 0)) * BM + r];
+            s2[q] = bcast16(WF == W_MXFP4 ? e8m0_code_to_bf16(c) : e4m3_code_to_bf16(c));
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              rg[j * 4 + i] = bmul2(bmul2(e2m1_pair(w4[j] >> (4 * i)), 0x7E807E80u), s2[j >> 1]);
+        }
+      } else {
+        // 8-bit: two 16-k chunks per thread
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const uint4 v = *reinterpret_cast<const uint4 *>(wpk + (half * 2 + c) * (BM * 16) + r * 16);
+          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            rg[c * 8 + j * 2] = bmul2(e4m3_pair(w4[j]), 0x7B807B80u);
+            rg[c * 8 + j * 2 + 1] = bmul2(e4m3_pair(w4[j] >> 8), 0x7B807B80u);
+          }
+        }
+      }
+      tmem_st16(t_row + (uint32_t)(a * C::A_COLS + half * 16), rg);
+      }
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&afull[a]);
+        mbar_arrive(&sfree[s]);
+      }
+    }
+  } else if (warp == WARP_MMA) {
+    // ================= MMA issuer (whole warp in step, lane 0 issues) =================
+    constexpr uint32_t idesc = F8 ? idesc_e4m3<BNT>() : idesc_bf16<BNT>();
+    const uint32_t tmem_d = tmem + C::D_COL;
+    for (int it = 0; it < nkb; ++it) {
+      const int s = it % NS, a = it % NA;
+      if (!mbar_wait(&full[s], (it / NS) & 1)) { *s_abort = 1; break; }
+      if (!mbar_wait(&afull[a], (it / NA) & 1)) { *s_abort = 1; break; }
+      if (*(volatile int *)s_abort) break;
+      tc_fence_after();
+      if (lane == 0) {
+        if constexpr (F8) {
+          // two K=32 steps of 32 bytes per 64-k block
+          const uint64_t bdesc = sw64_desc(smem_u32(smem + s * C::STAGE));
+#pragma unroll
+          for (int k32 = 0; k32 < 2; ++k32)
+            mma_ts_f8(tmem_d, tmem + (uint32_t)(a * C::A_COLS + k32 * 8), bdesc + (uint64_t)(k32 * 2), idesc,
+                      (it > 0 || k32 > 0) ? 1u : 0u);
+        } else {
+          const uint64_t bdesc = sw128_desc(smem_u32(smem + s * C::STAGE));
+#pragma unroll
+          for (int k16 = 0; k16 < 4; ++k16)
+            mma_ts(tmem_d, tmem + (uint32_t)(a * C::A_COLS + k16 * 8), bdesc + (uint64_t)(k16 * 2), idesc,
+                   (it > 0 || k16 > 0) ? 1u : 0u);
+        }
+        mma_commit(&sfree[s]);
+        mma_commit(&aempty[a]);
+      }
+      __syncwarp();
+    }
+    if (lane == 0) mma_commit(accum);
+    __syncwarp();
+  } else {
+    // ================= epilogue: warps 0..3 =================
+    const bool ok = mbar_wait(accum, 0);
+    tc_fence_after();
+    const int r = warp * 32 + lane;         // weight row inside the tile
+    const int n = wt * BM + r;              // output column
+    const int tile = slot * p.NT + wt;
+    float cs = 1.f, gs = 1.f;
+    if (WF == W_FP8 && n < p.N) cs = reinterpret_cast<const float *>(eb + p.c_off)[n];
+    if (WF == W_NVFP4) gs = reinterpret_cast<const float *>(eb + p.g_off)[0];
+    if (p.a_global) gs = __fmul_rn(gs, *p.a_global);
+    const bool run = ok && !*(volatile int *)s_abort;
+    if (run) {
+      for (int c0 = 0; c0 < BNT && c0 < nvalid; c0 += 16) {
+        float v[16];
+        tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(C::D_COL + c0), v);
+        if (p.splits > 1) {
+          float *part = p.partial + ((size_t)tile * p.splits + split) * BNT * BM;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) __stcg(&part[(size_t)(c0 + i) * BM + r], v[i]);
+        } else if (n < p.N) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int m = c0 + i;
+            if (m < nvalid) {
+              float x = v[i];
+              if (p.row_scale) x *= p.row_scale[s_srow[m]];
+              x *= cs;
+              x *= gs;
+              p.out[(size_t)s_orow[m] * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(x));
+            }
+          }
+        }
+      }
+    }
+    if (p.splits > 1) {
+      __threadfence();
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (tid == 0) s_info[3] = (atomicAdd(&p.counters[tile], 1) == p.splits - 1);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS));
+  }
+  // ---- split-K fixup: the last split of a tile sums every split's partial
+  // in split order (deterministic), all threads, 16-byte loads, all splits
+  // of an item in flight together ----
+  if (p.splits > 1 && s_info[3] && !*(volatile int *)s_abort) {
+    __threadfence();
+    const int tile = slot * p.NT + wt;
+    const float4 *pp = reinterpret_cast<const float4 *>(p.partial + (size_t)tile * p.splits * BNT * BM);
+    float gs = 1.f;
+    if (WF == W_NVFP4) gs = reinterpret_cast<const float *>(eb + p.g_off)[0];
+    if (p.a_global) gs = __fmul_rn(gs, *p.a_global);
+    for (int item = tid; item < nvalid * (BM / 4); item += THREADS) {
+      const int m = item / (BM / 4), r4 = item % (BM / 4);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int sp0 = 0; sp0 < p.splits; sp0 += 8) {
+        float4 v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (sp0 + j < p.splits) v[j] = __ldcg(pp + ((size_t)(sp0 + j) * BNT + m) * (BM / 4) + r4);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (sp0 + j < p.splits) {
+            acc.x += v[j].x; acc.y += v[j].y; acc.z += v[j].z; acc.w += v[j].w;
+          }
+      }
+      const float rs = p.row_scale ? p.row_scale[s_srow[m]] : 1.f;
+      const float a4[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int n = wt * BM + r4 * 4 + j;
+        if (n < p.N) {
+          float x = a4[j] * rs;
+          if (WF == W_FP8) x *= reinterpret_cast<const float *>(eb + p.c_off)[n];
+          x *= gs;
+          p.out[(size_t)s_orow[m] * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(x));
+        }
+      }
+    }
+    if (tid == 0) p.counters[tile] = 0;  // ready for the next call
+  }
+}
+
+}  // namespace tc
+
+// ---- host side -------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void *ptr = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// [rows, K] row-major activations, box = 64 k x box_rows: bf16 with a
+// 128-byte swizzle, or E4M3 bytes with a 64-byte swizzle.
+static bool make_act_map(CUtensorMap *m, const void *a, int rows, int K, int box_rows, bool e4m3) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const int es = e4m3 ? 1 : 2;
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)K * es};
+  cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  const CUresult r = fn(m, e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                        const_cast<void *>(a), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        e4m3 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Token tile = the smallest of 16, 32, 64, 128, 256 covering the rows a tile
+// is expected to hold; split-K until the grid covers the SMs about twice.
+TcLaunch plan_tc(int rows_per_tile, int mtiles_bound_moe, int N, int KB, bool moe) {
+  TcLaunch t{};
+  t.bnt = rows_per_tile <= 16 ? 16 : rows_per_tile <= 32 ? 32 : rows_per_tile <= 64 ? 64 : rows_per_tile <= 128 ? 128 : 256;
+  t.ntw = (N + TILE_N - 1) / TILE_N;
+  t.mtiles = moe ? mtiles_bound_moe : (rows_per_tile + t.bnt - 1) / t.bnt;
+  if (t.mtiles < 1) t.mtiles = 1;
+  const long tiles = (long)t.ntw * t.mtiles;
+  const long slots = (t.bnt <= 128 ? 2 : 1) * 148;  // CTAs resident at once
+  int max_splits = KB / 4;                          // at least 4 k-blocks per split
+  if (max_splits < 1) max_splits = 1;
+  // pick the split count with the least (waves x k-blocks per CTA), small
+  // penalty per extra split for the fixup traffic
+  int splits = 1;
+  double best = 1e30;
+  for (int s = 1; s <= max_splits && s <= 64; ++s) {
+    const int kb = (KB + s - 1) / s;
+    const long ctas = tiles * ((KB + kb - 1) / kb);
+    const long waves = (ctas + slots - 1) / slots;
+    const double cost = (double)waves * kb * (1.0 + 0.01 * s);
+    if (cost < best) {
+      best = cost;
+      splits = s;
+    }
+  }
+  int kbps = (KB + splits - 1) / splits;
+  splits = (KB + kbps - 1) / kbps;
+  t.splits = splits;
+  t.kb_per_split = kbps;
+  return t;
+}
+
+size_t tc_workspace_bytes(const TcLaunch &t) {
+  if (t.splits <= 1) return 256;
+  const size_t tiles = (size_t)t.ntw * t.mtiles;
+  return align_up(tiles * sizeof(int), 256) + tiles * t.splits * t.bnt * TILE_N * sizeof(float);
+}
+
+template <int WF, int BNT, bool F8>
+static hq_status tc_launch_one(const CUtensorMap &map, const tc::Params &p, const TcLaunch &t, cudaStream_t st) {
+  using C = tc::Cfg<WF, BNT, F8>;
+  auto kern = tc::tc_gemm_kernel<WF, BNT, F8>;
+  static unsigned configured = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return HQ_ERR_CUDA;
+  if (dev >= 32 || !(configured & (1u << dev))) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::BYTES) != cudaSuccess)
+      return HQ_ERR_CUDA;
+    if (dev < 32) configured |= 1u << dev;
+  }
+  dim3 grid(t.ntw * t.splits, t.mtiles);
+  kern<<<grid, tc::THREADS, C::BYTES, st>>>(map, p);
+  return check_launch();
+}
+
+template <int WF, bool F8 = false>
+static hq_status tc_launch_wf(const CUtensorMap &map, const tc::Params &p, const TcLaunch &t, cudaStream_t st) {
+  switch (t.bnt) {
+    case 16: return tc_launch_one<WF, 16, F8>(map, p, t, st);
+    case 32: return tc_launch_one<WF, 32, F8>(map, p, t, st);
+    case 64: return tc_launch_one<WF, 64, F8>(map, p, t, st);
+    case 128: return tc_launch_one<WF, 128, F8>(map, p, t, st);
+    default: return tc_launch_one<WF, 256, F8>(map, p, t, st);
+  }
+}
+
+// a_bf16 holds `a_rows` rows of K bf16 values.  Dense and MoE grouped: a tile
+// reads the rows [row_base, row_base + BNT) (rows past a tile's end are
+// loaded but never written back; rows past the matrix are zero-filled).  MoE
+// indexed (gather = 1): a tile gathers the caller rows perm[pos] / a_div.
+hq_status launch_tc_gemm(const Layout &L, const void *packed, const void *a_bf16, int a_rows, const float *row_scale,
+                         const float *a_global, int M, int moe, int E, const int32_t *offsets, const int32_t *perm,
+                         int a_div, int gather, void *out, const TcLaunch &t, void *workspace, cudaStream_t st,
+                         bool e4m3_act) {
+  if (e4m3_act && L.fmt != W_FP8) return HQ_ERR_UNSUPPORTED;
+  CUtensorMap map;
+  if (!make_act_map(&map, a_bf16, a_rows, L.K, gather ? 1 : t.bnt, e4m3_act)) return HQ_ERR_CUDA;
+  tc::Params p{};
+  p.packed = (const uint8_t *)packed;
+  p.stride = L.stride;
+  p.w_off = L.w_off; p.s_off = L.s_off; p.z_off = L.z_off; p.c_off = L.c_off; p.g_off = L.g_off;
+  p.N = L.N; p.K = L.K; p.NT = L.NT; p.KB = L.KB; p.G = L.G; p.group = L.group;
+  p.gshift = ((L.group & (L.group - 1)) == 0) ? __builtin_ctz((unsigned)L.group) : 31;
+  p.row_scale = row_scale;
+  p.a_global = a_global;
+  p.M = M;
+  p.moe = moe;
+  p.E = E;
+  p.offsets = offsets;
+  p.perm = perm;
+  p.a_div = a_div;
+  p.gather = gather;
+  p.out = (uint16_t *)out;
+  p.splits = t.splits;
+  p.kb_per_split = t.kb_per_split;
+  if (t.splits > 1) {
+    const size_t tiles = (size_t)t.ntw * t.mtiles;
+    p.counters = (int *)workspace;
+    p.partial = (float *)((uint8_t *)workspace + align_up(tiles * sizeof(int), 256));
+  }
+  switch (L.fmt) {
+    case W_INT4: return tc_launch_wf<W_INT4>(map, p, t, st);
+    case W_UINT4: return tc_launch_wf<W_UINT4>(map, p, t, st);
+    case W_MXFP4: return tc_launch_wf<W_MXFP4>(map, p, t, st);
+    case W_NVFP4: return tc_launch_wf<W_NVFP4>(map, p, t, st);
+    case W_FP8: return e4m3_act ? tc_launch_wf<W_FP8, true>(map, p, t, st) : tc_launch_wf<W_FP8>(map, p, t, st);
+    default: return HQ_ERR_UNSUPPORTED;
+  }
+}
+
+}  // namespace hq

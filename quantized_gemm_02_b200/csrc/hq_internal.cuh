@@ -1,26 +1,27 @@
 // Internal definitions shared by the sm_100a kernels of libhq.
 //
 // Packed weight layout (the "repack into the kernel's layout" step of
-// "Announcing Humming", section "Tuning & JIT per workload").  Per expert:
+// "Announcing Humming", section "Tuning and JIT compilation per workload").
+// Per expert, 256-byte aligned regions:
 //
-//   weights  [NT][KB][4 panels][32 lanes][16 B]           4-bit formats
-//            [NT][KB][4 panels][2 halves][32 lanes][16 B]  8-bit formats
-//   scales   [NT][G][64]   element = bf16 | E8M0 | UE4M3 (1 group = w_group
-//                          k's; per-channel scales use G = 1), FP8
-//                          per-channel scales are fp32 [NT][64]
-//   zeros    [NT][G][64]   uint8 (UINT4 only)
-//   global   fp32 (NVFP4 only)
+//   weights  [NT][KB][CH][128 rows][16 B]   CH = 2 chunks of 32 k (4-bit)
+//                                           or 4 chunks of 16 k (8-bit)
+//   scales   [NT][G][128]  element = bf16 | E8M0 | UE4M3 (one group =
+//                          w_group k's; per-channel scales use G = 1)
+//   zeros    [NT][G][128]  uint8 (UINT4 only)
+//   chscale  [NT][128]     fp32 (FP8 per-channel scales)
+//   global   fp32          (NVFP4 second-level scale)
 //
-// with NT = ceil(N / 64) row tiles, KB = K / 64 k-blocks.  One (row tile,
-// k-block) unit holds 64 rows x 64 k.  Inside it, panel p covers rows
-// 16p..16p+15; lane l of a warp reads its 16 bytes, which are exactly the
-// mma.sync m16n8k16 A-fragment values of that lane for the four k16 steps of
-// the k-block (4-bit) or two of them per half (8-bit).  Inside each 32-bit
-// word (one k16 step, 4-bit) the eight fragment values e0..e7 (e0,e1 = row
-// g, k 2t,2t+1; e2,e3 = row g+8; e4..e7 the same at k+8; g = l/4, t = l%4)
-// sit at nibble positions e0:0 e1:4 e2:1 e3:5 e4:2 e5:6 e6:3 e7:7, so
-// that (w >> 4i) & 0x000F000F yields fragment register i in both halves.
-// 8-bit words hold bytes [e0 e2 e1 e3] (first word) and [e4 e6 e5 e7].
+// with NT = ceil(N / 128) row tiles and KB = K / 64 k-blocks.  One (row
+// tile, k-block) unit is contiguous (4 KiB for 4-bit, 8 KiB for 8-bit), so a
+// CTA streams it with one bulk copy; inside it, thread r of the dequant
+// warps reads the 16-byte chunks of row r, consecutive threads consecutive
+// 16 bytes (conflict-free).  Within a 32-bit word the values are interleaved
+// so that one mask yields an adjacent k pair in the two bf16 halves:
+//   4-bit: nibble p holds k offset 2*(p%4) + p/4, so (w >> 4i) & 0x000F000F
+//          is the pair (k 2i, k 2i+1);
+//   8-bit: bytes hold k offsets [0 2 1 3], so (w >> 8i) & 0x00FF00FF is the
+//          pair (k 2i, k 2i+1).
 // INT4 codes are stored biased (u = q + 8) so every integer format decodes
 // as (u - z); signed INT4 uses z = 8.
 #pragma once
@@ -37,7 +38,7 @@ enum WFmt : int { W_INT4 = 0, W_UINT4 = 1, W_MXFP4 = 2, W_NVFP4 = 3, W_FP8 = 4, 
 // Internal activation formats.
 enum AFmt : int { A_BF16 = 0, A_FP8 = 1, A_MXFP8 = 2, A_NVFP4 = 3 };
 
-constexpr int TILE_N = 64;   // rows of W per tile
+constexpr int TILE_N = 128;  // rows of W per tile (the MMA M dimension)
 constexpr int TILE_K = 64;   // k per k-block
 
 struct Layout {
@@ -48,6 +49,7 @@ struct Layout {
   size_t w_bytes, s_bytes, z_bytes, c_bytes, g_bytes;  // per expert
   size_t w_off, s_off, z_off, c_off, g_off, stride;     // offsets inside an expert region
   __host__ __device__ size_t unit_bytes() const { return (size_t)TILE_N * TILE_K * wbits / 8; }
+  __host__ __device__ int chunks() const { return wbits == 4 ? 2 : 4; }
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -171,14 +173,28 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: the thread sleeps until the phase
+// completes or about `hint_ns` have passed, instead of spinning and taking
+// issue slots from the warps doing the work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait: returns false (and records HQ_ERR_TIMEOUT) after about a
 // second without the phase completing.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_timer_ns();
   while (true) {
-    for (int i = 0; i < 64; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
     if (global_timer_ns() - t0 > WAIT_LIMIT_NS) {
       set_device_error(HQ_ERR_TIMEOUT);
       return false;
@@ -219,15 +235,16 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
 }
 #endif
 
-// Launch plan of the weight-streaming GEMM (hq_gemm_stream.cu).
-struct StreamLaunch {
-  int mt;            // token tile (8, 16, 32)
+// Launch plan of the tensor-core GEMM (hq_gemm_tc.cu).
+struct TcLaunch {
+  int bnt;           // token tile = MMA N (16, 32, 64, 128, 256)
+  int ntw;           // 128-row weight tiles
   int mtiles;        // grid.y: token tiles (dense) or an upper bound on (expert, tile) pairs (MoE)
   int splits;        // split-K factor
   int kb_per_split;  // k-blocks per split
 };
-StreamLaunch plan_stream(int rows_bound, int mtiles_bound_moe, int NT, int KB, bool moe);
-size_t stream_workspace_bytes(const StreamLaunch &s, int NT);
+TcLaunch plan_tc(int rows_per_tile, int mtiles_bound_moe, int N, int KB, bool moe);
+size_t tc_workspace_bytes(const TcLaunch &t);
 
 // Host-side helpers implemented in hq_api.cu.
 hq_status check_launch();

@@ -6,29 +6,25 @@
 
 namespace hq {
 
-// Position of the (row, k) element inside a 64x64 unit:
-//   word index inside the unit (32-bit words) and bit offset inside the word.
+// Position of element (row i_row, k offset kk) inside one 128 x 64 unit:
+// 32-bit word index inside the unit and bit offset inside the word.
 struct FragPos {
   uint32_t word;
   uint32_t shift;
 };
 
 __host__ __device__ inline FragPos frag_pos(int wbits, int i_row, int kk) {
-  const int p = i_row >> 4, rr = i_row & 15;
-  const int g = rr & 7, hi_row = rr >> 3;
-  const int s = kk >> 4, c = kk & 15;
-  const int hi_k = c >> 3, c8 = c & 7;
-  const int t = c8 >> 1, odd = c8 & 1;
-  const int lane = g * 4 + t;
-  const int e = (hi_k ? 4 : 0) + (hi_row ? 2 : 0) + odd;  // fragment element 0..7
   FragPos fp;
   if (wbits == 4) {
-    fp.word = (uint32_t)((p * 32 + lane) * 4 + s);
-    fp.shift = (uint32_t)(4 * ((e >> 1) + 4 * (e & 1)));
+    const int chunk = kk >> 5, kc = kk & 31, j = kc >> 3, ko = kc & 7;
+    const int pos = (ko & 1) * 4 + (ko >> 1);  // nibble holding k offset ko
+    fp.word = (uint32_t)((chunk * TILE_N + i_row) * 4 + j);
+    fp.shift = (uint32_t)(4 * pos);
   } else {
-    const int ew = e & 3;  // element inside its word
-    fp.word = (uint32_t)(p * 256 + (s >> 1) * 128 + lane * 4 + 2 * (s & 1) + (e >> 2));
-    fp.shift = (uint32_t)(8 * (((ew & 1) << 1) | (ew >> 1)));
+    const int chunk = kk >> 4, kc = kk & 15, j = kc >> 2, ko = kc & 3;
+    const int pos = (ko & 1) * 2 + (ko >> 1);  // byte holding k offset ko
+    fp.word = (uint32_t)((chunk * TILE_N + i_row) * 4 + j);
+    fp.shift = (uint32_t)(8 * pos);
   }
   return fp;
 }
@@ -49,6 +45,7 @@ __global__ void pack_weights_kernel(Layout L, int E, const uint8_t *codes, uint8
   const size_t words_per_unit = L.unit_bytes() / 4;
   const size_t words_per_expert = (size_t)L.NT * L.KB * words_per_unit;
   const size_t total = words_per_expert * E;
+  const size_t code_stride = (L.fmt == W_FP8) ? (size_t)L.N * L.K : (size_t)L.N * L.K / 2;
   for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < total;
        idx += (size_t)gridDim.x * blockDim.x) {
     const int e = (int)(idx / words_per_expert);
@@ -56,37 +53,15 @@ __global__ void pack_weights_kernel(Layout L, int E, const uint8_t *codes, uint8
     const size_t unit = rem / words_per_unit;
     const uint32_t wi = (uint32_t)(rem % words_per_unit);
     const int nt = (int)(unit / L.KB), kb = (int)(unit % L.KB);
-    const size_t code_stride = (L.fmt == W_FP8) ? (size_t)L.N * L.K
-                               : (L.fmt == W_MXFP4 || L.fmt == W_NVFP4) ? (size_t)L.N * L.K / 2
-                                                                        : (size_t)L.N * L.K / 2;
     const uint8_t *ce = codes + (size_t)e * code_stride;
+    const int chunk = (int)(wi / (TILE_N * 4)), i_row = (int)((wi / 4) % TILE_N), j = (int)(wi % 4);
+    const int r = nt * TILE_N + i_row;
     uint32_t word = 0;
     const int per = 32 / L.wbits;
-    // enumerate the elements of this word by scanning the unit's 64x64
-    // positions that map here: invert frag_pos directly
     for (int slot = 0; slot < per; ++slot) {
-      // decode (row, kk) from (wi, slot)
-      int i_row, kk;
-      if (L.wbits == 4) {
-        const int p = wi / 128, lane = (wi / 4) % 32, s = wi % 4;
-        const int pos = slot;                       // nibble position
-        const int e_el = ((pos & 3) << 1) | (pos >> 2);  // inverse of (e>>1)+4*(e&1)
-        const int g = lane / 4, t = lane % 4;
-        const int hi_k = e_el >> 2, hi_row = (e_el >> 1) & 1, odd = e_el & 1;
-        i_row = p * 16 + hi_row * 8 + g;
-        kk = s * 16 + hi_k * 8 + t * 2 + odd;
-      } else {
-        const int p = wi / 256, h = (wi / 128) % 2, lane = (wi / 4) % 32, w4 = wi % 4;
-        const int s = 2 * h + (w4 >> 1), which = w4 & 1;
-        const int bpos = slot;                           // byte position in word
-        const int ew = ((bpos & 1) << 1) | (bpos >> 1);  // inverse of byte order [e0 e2 e1 e3]
-        const int e_el = which * 4 + ew;
-        const int g = lane / 4, t = lane % 4;
-        const int hi_k = e_el >> 2, hi_row = (e_el >> 1) & 1, odd = e_el & 1;
-        i_row = p * 16 + hi_row * 8 + g;
-        kk = s * 16 + hi_k * 8 + t * 2 + odd;
-      }
-      const int r = nt * TILE_N + i_row;
+      int kk;
+      if (L.wbits == 4) kk = chunk * 32 + j * 8 + 2 * (slot & 3) + (slot >> 2);
+      else kk = chunk * 16 + j * 4 + 2 * (slot & 1) + (slot >> 1);
       const int k = kb * TILE_K + kk;
       uint32_t v = 0;
       if (r < L.N) {
