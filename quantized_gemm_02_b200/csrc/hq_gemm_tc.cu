@@ -23,9 +23,13 @@
 //       warps 6..13  dequant: thread = weight row, decodes 32 k of its row per
 //                    k-block to bf16 pairs and stores them with
 //                    tcgen05.st.32x32b into the A ring in TMEM;
-//   * shared-memory ring (NS stages, one 64-k block each) for activations
-//     and packed weights, TMEM ring (4 stages x 32 columns) for dequantised
-//     weights, fp32 accumulator in TMEM after the ring;
+//   * persistent CTAs (one or two per SM): whole tiles round-robin when
+//     there are at least as many tiles as CTAs, else K-split units with a
+//     deterministic fp32 fixup by the last split of each tile;
+//   * shared-memory ring (NS stages of up to KPS 64-k blocks) for
+//     activations and packed weights, TMEM ring (NA blocks of 32 columns,
+//     16 for E4M3) for dequantised weights, fp32 accumulators (two where
+//     TMEM allows) after the ring;
 //   * every mbarrier wait is bounded (~1 s); on a timeout the CTA records
 //     HQ_ERR_TIMEOUT, raises an abort flag, releases its TMEM and returns.
 #include <cuda.h>
@@ -39,7 +43,6 @@ namespace hq {
 namespace tc {
 
 constexpr int BM = TILE_N;        // 128 weight rows = MMA M
-constexpr int NA = 4;             // TMEM A ring depth
 constexpr int THREADS = 14 * 32;
 constexpr int WARP_PRODUCER = 4, WARP_MMA = 5, WARP_DQ0 = 6, NDQ = 8;
 
@@ -55,23 +58,35 @@ struct Traits {
 
 // F8: both operands E4M3 (kind::f8f6f4, weights copied into TMEM unchanged);
 // otherwise weights are dequantised to bf16 (kind::f16).
+// F8: both operands E4M3 (kind::f8f6f4, weights copied into TMEM unchanged);
+// otherwise weights are dequantised to bf16 (kind::f16).
 template <int WF, int BNT, bool F8>
 struct Cfg {
-  static constexpr int A_COLS = F8 ? 16 : 32;                                  // TMEM columns per 64-k stage
-  static constexpr int ACT = BNT * (F8 ? 64 : 128);                            // [BNT][64] bf16 or e4m3, swizzled
-  static constexpr int WPK = Traits<WF>::unit;
-  static constexpr int SC = Traits<WF>::max_groups_kb * BM * Traits<WF>::sbytes;
-  static constexpr int ZP = Traits<WF>::has_zero ? Traits<WF>::max_groups_kb * BM : 0;
+  static constexpr int KPS = BNT <= 16 ? 4 : BNT <= 64 ? 2 : 1;               // 64-k blocks per stage
+  static constexpr int A_COLS = F8 ? 16 : 32;                                  // TMEM columns per 64-k block
+  static constexpr int ACT_KB = BNT * (F8 ? 64 : 128);                         // one block of activations
+  static constexpr int ACT = KPS * ACT_KB;                                     // [KPS][BNT][64], swizzled
+  static constexpr int WPK = KPS * Traits<WF>::unit;
+  static constexpr int SC = KPS * Traits<WF>::max_groups_kb * BM * Traits<WF>::sbytes;
+  static constexpr int ZP = Traits<WF>::has_zero ? KPS * Traits<WF>::max_groups_kb * BM : 0;
   static constexpr int STAGE = (ACT + WPK + SC + ZP + 1023) / 1024 * 1024;
-  // two CTAs per SM up to 128 tokens (TMEM: 2 x 256 columns), one beyond
-  static constexpr int CTAS_PER_SM = BNT <= 128 ? 2 : 1;
-  static constexpr int NS_BY_SMEM = ((CTAS_PER_SM == 2 ? 104 : 200) * 1024) / STAGE;
+  // two CTAs per SM up to 64 tokens (TMEM 2 x 256 columns), one beyond
+  static constexpr int CTAS_PER_SM = BNT <= 64 ? 2 : 1;
+  static constexpr int NS_BY_SMEM = ((CTAS_PER_SM == 2 ? 100 : 196) * 1024) / STAGE;
   static constexpr int NS = NS_BY_SMEM > 8 ? 8 : NS_BY_SMEM;                  // shared-memory ring depth
-  static constexpr int CTRL = 4096;                                            // barriers + tile info
+  static constexpr int CTRL = 8192;                                            // barriers + tile tables
   static constexpr int BYTES = NS * STAGE + CTRL + 1024;                      // + alignment slack
-  static constexpr int D_COL = NA * A_COLS;                                    // accumulator columns start
-  static constexpr int TMEM_COLS = (D_COL + BNT) <= 256 ? 256 : 512;
+  // TMEM: the CTA's share (256 columns with two CTAs per SM, else 512) holds
+  // ND accumulators of BNT columns and a ring of NA dequantised 64-k blocks.
+  // The ring must cover the MMA completion latency (~1 us), so it takes all
+  // the columns the accumulators leave.
+  static constexpr int TMEM_COLS = CTAS_PER_SM == 2 ? 256 : 512;
+  static constexpr int ND = (4 * A_COLS + 2 * BNT) <= TMEM_COLS ? 2 : 1;      // accumulator buffers
+  static constexpr int NA_FIT = (TMEM_COLS - ND * BNT) / A_COLS;
+  static constexpr int NA = NA_FIT > 12 ? 12 : NA_FIT;                         // TMEM A ring depth
+  static constexpr int D_COL = NA * A_COLS;                                    // accumulators start
   static_assert(NS >= 2, "stage too large");
+  static_assert(NA >= 2 && D_COL + ND * BNT <= TMEM_COLS, "TMEM budget");
 };
 
 struct Params {
@@ -88,9 +103,11 @@ struct Params {
   int a_div;
   int gather;              // MoE indexed mode: activation rows gathered by index
   uint16_t *out;
-  int splits, kb_per_split;
-  float *partial;
-  int *counters;
+  int ntw;                 // 128-row weight tiles
+  int mtiles;              // token tiles (dense: exact; MoE: upper bound)
+  int nctas;               // persistent CTAs (grid size)
+  float *partial;          // [tiles * S][BNT][128] fp32 split-K partial tiles
+  int *counters;           // [ntw * mtiles] per-tile arrival tickets
 };
 
 // ---- PTX wrappers ----------------------------------------------------------------
@@ -225,41 +242,99 @@ __device__ __forceinline__ uint32_t e4m3_pair(uint32_t x) {
 }
 
 // ---- the kernel ----------------------------------------------------------------
+// Persistent CTAs.  Work units are (tile, k-range) pairs; tiles are ordered
+// token-tile-major with the weight tile fastest.
+//   * at least as many tiles as CTAs: unit u of CTA c is the whole tile
+//     c + u * nctas (round-robin, so the CTAs running together share their
+//     activation tile in L2 and no tile is shared between CTAs);
+//   * fewer tiles than CTAs (decode sizes): every tile is split along K into
+//     S contiguous ranges, one unit per CTA; each split stores an fp32
+//     partial and the last split to arrive (atomic ticket) sums the S
+//     partials in split order with all its threads.
+// The TMEM accumulator is double-buffered where TMEM allows, so one unit's
+// epilogue overlaps the next unit's main loop.
+
+struct TileInfo {
+  int wt, expert, base, nvalid;
+};
+
+struct Sched {
+  int tiles;  // tiles in this call (MoE: from the routing)
+  int S;      // K splits per tile (1 in round-robin mode)
+  int kbps;   // k-blocks per split
+  bool rr;    // round-robin whole tiles
+};
+
+__device__ __forceinline__ Sched make_sched(int tiles, int nctas, int KB) {
+  Sched sc;
+  sc.tiles = tiles;
+  sc.rr = tiles >= nctas;
+  if (sc.rr || tiles == 0) {
+    sc.S = 1;
+    sc.kbps = KB;
+  } else {
+    int S = nctas / tiles;
+    const int max_s = KB / 2 > 0 ? KB / 2 : 1;  // at least two k-blocks per split
+    if (S > max_s) S = max_s;
+    sc.kbps = (KB + S - 1) / S;
+    sc.S = (KB + sc.kbps - 1) / sc.kbps;
+  }
+  return sc;
+}
+
+// Unit u of CTA c: tile t, k-blocks [kb0, kb1) and split index; false once
+// the CTA has no more work.
+__device__ __forceinline__ bool unit_at(const Sched &sc, int c, int nctas, int KB, int u, int &t, int &kb0,
+                                        int &kb1, int &split) {
+  if (sc.rr) {
+    t = c + u * nctas;
+    if (t >= sc.tiles) return false;
+    kb0 = 0;
+    kb1 = KB;
+    split = 0;
+    return true;
+  }
+  if (u > 0 || c >= sc.tiles * sc.S) return false;
+  t = c % sc.tiles;
+  split = c / sc.tiles;
+  kb0 = split * sc.kbps;
+  kb1 = min(KB, kb0 + sc.kbps);
+  return kb0 < kb1;
+}
+
 template <int WF, int BNT, bool F8>
-__global__ void __launch_bounds__(THREADS, 1) tc_gemm_kernel(const __grid_constant__ CUtensorMap act_map,
+__global__ void __launch_bounds__(THREADS, (BNT <= 64 ? 2 : 1)) tc_gemm_kernel(const __grid_constant__ CUtensorMap act_map,
                                                              const Params p) {
   using TR = Traits<WF>;
   using C = Cfg<WF, BNT, F8>;
   static_assert(!F8 || WF == W_FP8, "the E4M3 x E4M3 path takes FP8 weights");
-  constexpr int NS = C::NS;
+  constexpr int NS = C::NS, ND = C::ND, NA = C::NA;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *ctrl = smem + NS * C::STAGE;
-  uint64_t *full = reinterpret_cast<uint64_t *>(ctrl);  // [NS]  stage landed
-  uint64_t *sfree = full + NS;                           // [NS]  stage consumed (MMA + dequant)
-  uint64_t *afull = sfree + NS;                          // [NA]  TMEM A stage written
-  uint64_t *aempty = afull + NA;                         // [NA]  TMEM A stage consumed
-  uint64_t *accum = aempty + NA;                         // accumulator complete
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accum + 1);
+  uint64_t *full = reinterpret_cast<uint64_t *>(ctrl);  // [NS] stage landed
+  uint64_t *sfree = full + NS;                           // [NS] stage consumed (MMA + dequant)
+  uint64_t *afull = sfree + NS;                          // [NA] TMEM A stage written
+  uint64_t *aempty = afull + NA;                         // [NA] TMEM A stage consumed
+  uint64_t *accf = aempty + NA;                          // [ND] accumulator complete
+  uint64_t *acce = accf + ND;                            // [ND] accumulator drained
+  long long *s_total = reinterpret_cast<long long *>(acce + ND);  // 8-byte slot after the barriers
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(s_total + 1);
   int *s_abort = reinterpret_cast<int *>(tmem_slot + 1);
-  int *s_info = s_abort + 1;  // [0] expert [1] row base [2] valid rows [3] is_last
-  int *s_orow = s_info + 4;   // [BNT] output row of each token column
-  int *s_srow = s_orow + BNT; // [BNT] caller activation row (per-token scale, gather index)
+  int *s_last = s_abort + 1;
+  int *s_tpre = s_last + 1;  // [E+1] MoE: prefix of token tiles per expert
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int wt = blockIdx.x % p.NT;   // 128-row weight tile
-  const int split = blockIdx.x / p.NT;
-  const int slot = blockIdx.y;        // token tile (dense) or (expert, tile) slot (MoE)
+  const int cta = blockIdx.x;
 
-  // ---- tile -> (expert, token rows) ----
+  // ---- number of valid token tiles (MoE: from the routing offsets) ----
   if (warp == 0) {
-    int expert = 0, base = 0, nvalid = 0;
+    int tvalid = 0;
     if (!p.moe) {
-      base = slot * BNT;
-      nvalid = min(BNT, p.M - base);
+      tvalid = (p.M + BNT - 1) / BNT;
     } else if (p.offsets[p.E] >= 0) {
-      int running = 0, found = -1, tile_in = 0;
-      for (int e0 = 0; e0 < p.E && found < 0; e0 += 32) {
+      int running = 0;
+      for (int e0 = 0; e0 < p.E; e0 += 32) {
         const int e = e0 + lane;
         int tiles = 0;
         if (e < p.E) tiles = (p.offsets[e + 1] - p.offsets[e] + BNT - 1) / BNT;
@@ -269,41 +344,17 @@ __global__ void __launch_bounds__(THREADS, 1) tc_gemm_kernel(const __grid_consta
           const int v = __shfl_up_sync(0xffffffffu, incl, o);
           if (lane >= o) incl += v;
         }
-        const int excl = running + incl - tiles;
-        const bool mine = (e < p.E) && slot >= excl && slot < excl + tiles;
-        const unsigned ball = __ballot_sync(0xffffffffu, mine);
-        if (ball) {
-          const int src = __ffs(ball) - 1;
-          found = __shfl_sync(0xffffffffu, e, src);
-          tile_in = __shfl_sync(0xffffffffu, slot - excl, src);
-        }
+        if (e < p.E) s_tpre[e + 1] = running + incl;
         running += __shfl_sync(0xffffffffu, incl, 31);
       }
-      if (found >= 0) {
-        expert = found;
-        base = p.offsets[found] + tile_in * BNT;
-        nvalid = min(BNT, p.offsets[found + 1] - base);
-      }
+      if (lane == 0) s_tpre[0] = 0;
+      tvalid = running;
     }
-    for (int i = lane; i < BNT; i += 32) {
-      int orow = -1, srow = -1;
-      if (i < nvalid) {
-        const int pos = base + i;
-        if (!p.moe) {
-          orow = srow = pos;
-        } else {
-          orow = p.perm[pos];
-          srow = orow / p.a_div;
-        }
-      }
-      s_orow[i] = orow;
-      s_srow[i] = srow;
-    }
+    if (tvalid > p.mtiles) tvalid = p.mtiles;  // never beyond the sized workspace
     if (lane == 0) {
-      s_info[0] = expert;
-      s_info[1] = base;
-      s_info[2] = nvalid;
+      *s_total = (long long)tvalid * p.ntw;  // tiles
       *s_abort = 0;
+      *s_last = 0;
     }
   }
   if (tid == 32) {
@@ -315,12 +366,40 @@ __global__ void __launch_bounds__(THREADS, 1) tc_gemm_kernel(const __grid_consta
       mbar_init(&afull[a], NDQ);
       mbar_init(&aempty[a], 1);
     }
-    mbar_init(accum, 1);
+    for (int d = 0; d < ND; ++d) {
+      mbar_init(&accf[d], 1);
+      mbar_init(&acce[d], 4);
+    }
     fence_barrier_init();
   }
   __syncthreads();
-  const int expert = s_info[0], row_base = s_info[1], nvalid = s_info[2];
-  if (nvalid <= 0) return;
+  const Sched sch = make_sched((int)*s_total, p.nctas, p.KB);
+  const bool split_mode = !sch.rr && sch.S > 1;
+  int t_mine, kb0_mine, kb1_mine, sp_mine;  // first unit of this CTA
+  if (!unit_at(sch, cta, p.nctas, p.KB, 0, t_mine, kb0_mine, kb1_mine, sp_mine)) return;
+
+  // tile index -> weight tile, expert, token rows
+  auto tile_info = [&](int t) {
+    TileInfo ti;
+    const int slot = t / p.ntw;
+    ti.wt = t - slot * p.ntw;
+    if (!p.moe) {
+      ti.expert = 0;
+      ti.base = slot * BNT;
+      ti.nvalid = min(BNT, p.M - ti.base);
+    } else {
+      int lo = 0, hi = p.E;  // largest e with s_tpre[e] <= slot
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (s_tpre[mid] <= slot) lo = mid;
+        else hi = mid;
+      }
+      ti.expert = lo;
+      ti.base = p.offsets[lo] + (slot - s_tpre[lo]) * BNT;
+      ti.nvalid = min(BNT, p.offsets[lo + 1] - ti.base);
+    }
+    return ti;
+  };
 
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
@@ -331,202 +410,244 @@ __global__ void __launch_bounds__(THREADS, 1) tc_gemm_kernel(const __grid_consta
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
-  const uint8_t *eb = p.packed + (size_t)expert * p.stride;
-  const int kb_begin = split * p.kb_per_split;
-  const int kb_end = min(p.KB, kb_begin + p.kb_per_split);
-  const int nkb = kb_end - kb_begin;
-
   if (warp == WARP_PRODUCER) {
     // ================= producer (whole warp in step, lane 0 issues) =================
     const uint64_t pol = policy_evict_first();
-    for (int it = 0; it < nkb; ++it) {
-      const int s = it % NS;
-      if (it >= NS && !mbar_wait(&sfree[s], ((it / NS) - 1) & 1)) { *s_abort = 1; break; }
-      if (*(volatile int *)s_abort) break;
+    int is = 0;
+    bool stop = false;
+    for (int u = 0; !stop; ++u) {
+      int t, ukb0, ukb1, usp;
+      if (!unit_at(sch, cta, p.nctas, p.KB, u, t, ukb0, ukb1, usp)) break;
+      const TileInfo ti = tile_info(t);
+      for (int kbs = ukb0; kbs < ukb1; kbs += C::KPS, ++is) {
+      const int nblk = min(C::KPS, ukb1 - kbs);
+      const int s = is % NS;
+      if (is >= NS && !mbar_wait(&sfree[s], ((is / NS) - 1) & 1)) { *s_abort = 1; stop = true; break; }
+      if (*(volatile int *)s_abort) { stop = true; break; }
       if (lane == 0) {
+        const uint8_t *eb = p.packed + (size_t)ti.expert * p.stride;
         uint8_t *st = smem + s * C::STAGE;
-        const int kb = kb_begin + it;
-        const int g0 = (kb * TILE_K) >> p.gshift;
-        const int g1 = (((kb + 1) * TILE_K - 1) >> p.gshift) + 1;
+        const int g0 = (kbs * TILE_K) >> p.gshift;
+        const int g1 = (((kbs + nblk) * TILE_K - 1) >> p.gshift) + 1;
         const uint32_t sb = TR::has_scales ? (uint32_t)((g1 - g0) * BM * TR::sbytes) : 0u;
         const uint32_t zb = TR::has_zero ? (uint32_t)((g1 - g0) * BM) : 0u;
         constexpr uint32_t row_bytes = F8 ? 64u : 128u;
-        const uint32_t ab = p.gather ? (uint32_t)(((nvalid + 3) / 4) * 4 * row_bytes) : (uint32_t)(BNT * row_bytes);
-        mbar_arrive_expect_tx(&full[s], ab + TR::unit + sb + zb);
-        if (!p.gather) {
-          tma_load_2d(st, &act_map, kb * TILE_K, row_base, &full[s]);
-        } else {
-          for (int i = 0; i < nvalid; i += 4) {
-            const int r0 = s_srow[i];
-            const int r1 = (i + 1 < nvalid) ? s_srow[i + 1] : r0;
-            const int r2 = (i + 2 < nvalid) ? s_srow[i + 2] : r0;
-            const int r3 = (i + 3 < nvalid) ? s_srow[i + 3] : r0;
-            tma_gather4(st + i * row_bytes, &act_map, kb * TILE_K, r0, r1, r2, r3, &full[s]);
+        const uint32_t ab = p.gather ? (uint32_t)(((ti.nvalid + 3) / 4) * 4 * row_bytes) : (uint32_t)C::ACT_KB;
+        mbar_arrive_expect_tx(&full[s], ab * nblk + TR::unit * nblk + sb + zb);
+        for (int j = 0; j < nblk; ++j) {
+          const int kbj = kbs + j;
+          if (!p.gather) {
+            tma_load_2d(st + j * C::ACT_KB, &act_map, kbj * TILE_K, ti.base, &full[s]);
+          } else {
+            for (int i = 0; i < ti.nvalid; i += 4) {
+              int r[4];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) r[q] = p.perm[ti.base + min(i + q, ti.nvalid - 1)] / p.a_div;
+              tma_gather4(st + j * C::ACT_KB + i * row_bytes, &act_map, kbj * TILE_K, r[0], r[1], r[2], r[3],
+                          &full[s]);
+            }
           }
         }
-        bulk_g2s_stream(st + C::ACT, eb + p.w_off + ((size_t)wt * p.KB + kb) * TR::unit, TR::unit, &full[s], pol);
+        bulk_g2s_stream(st + C::ACT, eb + p.w_off + ((size_t)ti.wt * p.KB + kbs) * TR::unit, TR::unit * nblk,
+                        &full[s], pol);
         if (TR::has_scales)
-          bulk_g2s(st + C::ACT + C::WPK, eb + p.s_off + ((size_t)wt * p.G + g0) * BM * TR::sbytes, sb, &full[s]);
+          bulk_g2s(st + C::ACT + C::WPK, eb + p.s_off + ((size_t)ti.wt * p.G + g0) * BM * TR::sbytes, sb,
+                   &full[s]);
         if (TR::has_zero)
-          bulk_g2s(st + C::ACT + C::WPK + C::SC, eb + p.z_off + ((size_t)wt * p.G + g0) * BM, zb, &full[s]);
+          bulk_g2s(st + C::ACT + C::WPK + C::SC, eb + p.z_off + ((size_t)ti.wt * p.G + g0) * BM, zb, &full[s]);
       }
       __syncwarp();
+      }
     }
   } else if (warp >= WARP_DQ0) {
     // ================= dequant: thread = weight row =================
     const int dq = warp - WARP_DQ0;       // 0..7
     const int sp = warp & 3;              // TMEM subpartition this warp may access
-    const int half = dq >> 2;             // which 32 k of the 64-k block
+    const int half = dq >> 2;             // which 32 k of each 64-k block
     const int r = sp * 32 + lane;         // weight row inside the tile
     const uint32_t t_row = tmem + ((uint32_t)(sp * 32) << 16);
-    for (int it = 0; it < nkb; ++it) {
-      const int s = it % NS, a = it % NA;
-      if (!mbar_wait(&full[s], (it / NS) & 1)) { *s_abort = 1; break; }
-      if (it >= NA && !mbar_wait(&aempty[a], ((it / NA) - 1) & 1)) { *s_abort = 1; break; }
-      if (*(volatile int *)s_abort) break;
-      tc_fence_after();
+    int ia = 0;  // 64-k blocks decoded so far (TMEM A ring position)
+    int is = 0;
+    bool stop = false;
+    for (int u = 0; !stop; ++u) {
+      int t, ukb0, ukb1, usp;
+      if (!unit_at(sch, cta, p.nctas, p.KB, u, t, ukb0, ukb1, usp)) break;
+      for (int kbs = ukb0; kbs < ukb1 && !stop; kbs += C::KPS, ++is) {
+      const int nblk = min(C::KPS, ukb1 - kbs);
+      const int s = is % NS;
+      if (!mbar_wait(&full[s], (is / NS) & 1)) { *s_abort = 1; stop = true; break; }
       const uint8_t *st = smem + s * C::STAGE;
-      const uint8_t *wpk = st + C::ACT;
       const uint8_t *sc = st + C::ACT + C::WPK;
       const uint8_t *zp = st + C::ACT + C::WPK + C::SC;
-      const int kb = kb_begin + it;
-      const int g0 = (kb * TILE_K) >> p.gshift;
-      const int gt = ((kb * TILE_K + half * 32) >> p.gshift) - g0;  // group of this thread's first k
-      if constexpr (F8) {
-        // E4M3 weights go to TMEM unchanged, bytes put back in k order
-        uint32_t rg8[8];
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const uint4 v = *reinterpret_cast<const uint4 *>(wpk + (half * 2 + c) * (BM * 16) + r * 16);
-          rg8[c * 4 + 0] = __byte_perm(v.x, 0, 0x3120);
-          rg8[c * 4 + 1] = __byte_perm(v.y, 0, 0x3120);
-          rg8[c * 4 + 2] = __byte_perm(v.z, 0, 0x3120);
-          rg8[c * 4 + 3] = __byte_perm(v.w, 0, 0x3120);
-        }
-        tmem_st8(t_row + (uint32_t)(a * C::A_COLS + half * 8), rg8);
-      } else {
-      uint32_t rg[16];
-      if constexpr (TR::wbits == 4) {
-        const uint4 v = *reinterpret_cast<const uint4 *>(wpk + half * (BM * 16) + r * 16);
-        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-        if constexpr (WF == W_INT4 || WF == W_UINT4) {
-          // groups are >= 32 k: one scale (and zero point) covers the thread's 32 k
-          const uint32_t s2 = bcast16(reinterpret_cast<const uint16_t *>(sc)[gt * BM + r]);
-          const uint32_t z2 = (WF == W_UINT4) ? bcast16(0x4300u + zp[gt * BM + r]) : 0x43084308u;
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              rg[j * 4 + i] = bmul2(bsub2(((w4[j] >> (4 * i)) & 0x000F000Fu) | 0x43004300u, z2), s2);
+      const int g0 = (kbs * TILE_K) >> p.gshift;
+      for (int j = 0; j < nblk; ++j, ++ia) {
+        const int a = ia % NA;
+        if (ia >= NA && !mbar_wait(&aempty[a], ((ia / NA) - 1) & 1)) { *s_abort = 1; stop = true; break; }
+        if (*(volatile int *)s_abort) { stop = true; break; }
+        tc_fence_after();
+        const int kb = kbs + j;
+        const uint8_t *wpk_j = st + C::ACT + j * TR::unit;
+        const int gt = ((kb * TILE_K + half * 32) >> p.gshift) - g0;  // group of this thread's first k
+        if constexpr (F8) {
+          // E4M3 weights go to TMEM unchanged, bytes put back in k order
+          uint32_t rg8[8];
+  #pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(wpk_j + (half * 2 + c) * (BM * 16) + r * 16);
+            rg8[c * 4 + 0] = __byte_perm(v.x, 0, 0x3120);
+            rg8[c * 4 + 1] = __byte_perm(v.y, 0, 0x3120);
+            rg8[c * 4 + 2] = __byte_perm(v.z, 0, 0x3120);
+            rg8[c * 4 + 3] = __byte_perm(v.w, 0, 0x3120);
+          }
+          tmem_st8(t_row + (uint32_t)(a * C::A_COLS + half * 8), rg8);
         } else {
-          // MXFP4: one group of 32; NVFP4: two groups of 16 (words 0-1, 2-3)
-          uint32_t s2[2];
-#pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            const uint32_t c = sc[(gt + (WF == W_NVFP4 ? q : 0)) * BM + r];
-            s2[q] = bcast16(WF == W_MXFP4 ? e8m0_code_to_bf16(c) : e4m3_code_to_bf16(c));
+          uint32_t rg[16];
+          if constexpr (TR::wbits == 4) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(wpk_j + half * (BM * 16) + r * 16);
+            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+            if constexpr (WF == W_INT4 || WF == W_UINT4) {
+              // groups are >= 32 k: one scale (and zero point) covers the thread's 32 k
+              const uint32_t s2 = bcast16(reinterpret_cast<const uint16_t *>(sc)[gt * BM + r]);
+              const uint32_t z2 = (WF == W_UINT4) ? bcast16(0x4300u + zp[gt * BM + r]) : 0x43084308u;
+  #pragma unroll
+              for (int j = 0; j < 4; ++j)
+  #pragma unroll
+                for (int i = 0; i < 4; ++i)
+                  rg[j * 4 + i] = bmul2(bsub2(((w4[j] >> (4 * i)) & 0x000F000Fu) | 0x43004300u, z2), s2);
+            } else {
+              // MXFP4: one group of 32; NVFP4: two groups of 16 (words 0-1, 2-3)
+              uint32_t s2[2];
+  #pragma unroll
+              for (int q = 0; q < 2; ++q) {
+                const uint32_t c = sc[(gt + (WF == W_NVFP4 ? q : 0)) * BM + r];
+                s2[q] = bcast16(WF == W_MXFP4 ? e8m0_code_to_bf16(c) : e4m3_code_to_bf16(c));
+              }
+  #pragma unroll
+              for (int j = 0; j < 4; ++j)
+  #pragma unroll
+                for (int i = 0; i < 4; ++i)
+                  rg[j * 4 + i] = bmul2(bmul2(e2m1_pair(w4[j] >> (4 * i)), 0x7E807E80u), s2[j >> 1]);
+            }
+          } else {
+            // 8-bit weights with bf16 activations: two 16-k chunks per thread
+  #pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              const uint4 v = *reinterpret_cast<const uint4 *>(wpk_j + (half * 2 + c) * (BM * 16) + r * 16);
+              const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+  #pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                rg[c * 8 + j * 2] = bmul2(e4m3_pair(w4[j]), 0x7B807B80u);
+                rg[c * 8 + j * 2 + 1] = bmul2(e4m3_pair(w4[j] >> 8), 0x7B807B80u);
+              }
+            }
           }
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              rg[j * 4 + i] = bmul2(bmul2(e2m1_pair(w4[j] >> (4 * i)), 0x7E807E80u), s2[j >> 1]);
+          tmem_st16(t_row + (uint32_t)(a * C::A_COLS + half * 16), rg);
         }
-      } else {
-        // 8-bit: two 16-k chunks per thread
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const uint4 v = *reinterpret_cast<const uint4 *>(wpk + (half * 2 + c) * (BM * 16) + r * 16);
-          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            rg[c * 8 + j * 2] = bmul2(e4m3_pair(w4[j]), 0x7B807B80u);
-            rg[c * 8 + j * 2 + 1] = bmul2(e4m3_pair(w4[j] >> 8), 0x7B807B80u);
-          }
-        }
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&afull[a]);
       }
-      tmem_st16(t_row + (uint32_t)(a * C::A_COLS + half * 16), rg);
-      }
-      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-      tc_fence_before();
+      if (stop) break;
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&afull[a]);
-        mbar_arrive(&sfree[s]);
+      if (lane == 0) mbar_arrive(&sfree[s]);
       }
     }
   } else if (warp == WARP_MMA) {
     // ================= MMA issuer (whole warp in step, lane 0 issues) =================
     constexpr uint32_t idesc = F8 ? idesc_e4m3<BNT>() : idesc_bf16<BNT>();
-    const uint32_t tmem_d = tmem + C::D_COL;
-    for (int it = 0; it < nkb; ++it) {
-      const int s = it % NS, a = it % NA;
-      if (!mbar_wait(&full[s], (it / NS) & 1)) { *s_abort = 1; break; }
-      if (!mbar_wait(&afull[a], (it / NA) & 1)) { *s_abort = 1; break; }
-      if (*(volatile int *)s_abort) break;
-      tc_fence_after();
-      if (lane == 0) {
-        if constexpr (F8) {
-          // two K=32 steps of 32 bytes per 64-k block
-          const uint64_t bdesc = sw64_desc(smem_u32(smem + s * C::STAGE));
+    int ia = 0;  // 64-k blocks consumed
+    int is = 0;
+    bool stop = false;
+    for (int u = 0; !stop; ++u) {
+      int t, ukb0, ukb1, usp;
+      if (!unit_at(sch, cta, p.nctas, p.KB, u, t, ukb0, ukb1, usp)) break;
+      const int d = u % ND;
+      if (u >= ND && !mbar_wait(&acce[d], ((u / ND) - 1) & 1)) { *s_abort = 1; break; }
+      for (int kbs = ukb0; kbs < ukb1 && !stop; kbs += C::KPS, ++is) {
+        const int nblk = min(C::KPS, ukb1 - kbs);
+        const int s = is % NS;
+        if (!mbar_wait(&full[s], (is / NS) & 1)) { *s_abort = 1; stop = true; break; }
+        for (int j = 0; j < nblk; ++j, ++ia) {
+          const int a = ia % NA;
+          const int kb = kbs + j;
+          const bool first = (kb == ukb0);
+          const bool last = (kb == ukb1 - 1);
+          if (!mbar_wait(&afull[a], (ia / NA) & 1)) { *s_abort = 1; stop = true; break; }
+          if (*(volatile int *)s_abort) { stop = true; break; }
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t tmem_d = tmem + (uint32_t)(C::D_COL + d * BNT);
+            const uint32_t b_addr = smem_u32(smem + s * C::STAGE + j * C::ACT_KB);
+            if constexpr (F8) {
+              // two K=32 steps of 32 bytes per 64-k block
+              const uint64_t bdesc = sw64_desc(b_addr);
 #pragma unroll
-          for (int k32 = 0; k32 < 2; ++k32)
-            mma_ts_f8(tmem_d, tmem + (uint32_t)(a * C::A_COLS + k32 * 8), bdesc + (uint64_t)(k32 * 2), idesc,
-                      (it > 0 || k32 > 0) ? 1u : 0u);
-        } else {
-          const uint64_t bdesc = sw128_desc(smem_u32(smem + s * C::STAGE));
+              for (int k32 = 0; k32 < 2; ++k32)
+                mma_ts_f8(tmem_d, tmem + (uint32_t)(a * C::A_COLS + k32 * 8), bdesc + (uint64_t)(k32 * 2), idesc,
+                          (!first || k32 > 0) ? 1u : 0u);
+            } else {
+              const uint64_t bdesc = sw128_desc(b_addr);
 #pragma unroll
-          for (int k16 = 0; k16 < 4; ++k16)
-            mma_ts(tmem_d, tmem + (uint32_t)(a * C::A_COLS + k16 * 8), bdesc + (uint64_t)(k16 * 2), idesc,
-                   (it > 0 || k16 > 0) ? 1u : 0u);
+              for (int k16 = 0; k16 < 4; ++k16)
+                mma_ts(tmem_d, tmem + (uint32_t)(a * C::A_COLS + k16 * 8), bdesc + (uint64_t)(k16 * 2), idesc,
+                       (!first || k16 > 0) ? 1u : 0u);
+            }
+            mma_commit(&aempty[a]);
+            if (last) mma_commit(&accf[d]);
+          }
+          __syncwarp();
         }
-        mma_commit(&sfree[s]);
-        mma_commit(&aempty[a]);
+        if (stop) break;
+        if (lane == 0) mma_commit(&sfree[s]);
+        __syncwarp();
       }
-      __syncwarp();
     }
-    if (lane == 0) mma_commit(accum);
-    __syncwarp();
   } else {
-    // ================= epilogue: warps 0..3 =================
-    const bool ok = mbar_wait(accum, 0);
-    tc_fence_after();
-    const int r = warp * 32 + lane;         // weight row inside the tile
-    const int n = wt * BM + r;              // output column
-    const int tile = slot * p.NT + wt;
-    float cs = 1.f, gs = 1.f;
-    if (WF == W_FP8 && n < p.N) cs = reinterpret_cast<const float *>(eb + p.c_off)[n];
-    if (WF == W_NVFP4) gs = reinterpret_cast<const float *>(eb + p.g_off)[0];
-    if (p.a_global) gs = __fmul_rn(gs, *p.a_global);
-    const bool run = ok && !*(volatile int *)s_abort;
-    if (run) {
-      for (int c0 = 0; c0 < BNT && c0 < nvalid; c0 += 16) {
+    // ================= epilogue: warps 0..3, thread = weight row =================
+    const int r = warp * 32 + lane;
+    for (int u = 0;; ++u) {
+      int t, ukb0, ukb1, usp;
+      if (!unit_at(sch, cta, p.nctas, p.KB, u, t, ukb0, ukb1, usp)) break;
+      const int d = u % ND;
+      const bool ok = mbar_wait(&accf[d], (u / ND) & 1);
+      tc_fence_after();
+      if (!ok || *(volatile int *)s_abort) break;
+      const TileInfo ti = tile_info(t);
+      const uint8_t *eb = p.packed + (size_t)ti.expert * p.stride;
+      const int n = ti.wt * BM + r;
+      float cs = 1.f, gs = 1.f;
+      if (WF == W_FP8 && n < p.N) cs = reinterpret_cast<const float *>(eb + p.c_off)[n];
+      if (WF == W_NVFP4) gs = reinterpret_cast<const float *>(eb + p.g_off)[0];
+      if (p.a_global) gs = __fmul_rn(gs, *p.a_global);
+      float *part = p.partial + ((size_t)t * sch.S + usp) * BNT * BM;
+      for (int c0 = 0; c0 < BNT && c0 < ti.nvalid; c0 += 16) {
         float v[16];
-        tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(C::D_COL + c0), v);
-        if (p.splits > 1) {
-          float *part = p.partial + ((size_t)tile * p.splits + split) * BNT * BM;
+        tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(C::D_COL + d * BNT + c0), v);
+        if (split_mode) {
 #pragma unroll
           for (int i = 0; i < 16; ++i) __stcg(&part[(size_t)(c0 + i) * BM + r], v[i]);
         } else if (n < p.N) {
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const int m = c0 + i;
-            if (m < nvalid) {
+            if (m < ti.nvalid) {
+              const int pos = ti.base + m;
+              const int orow = p.moe ? p.perm[pos] : pos;
               float x = v[i];
-              if (p.row_scale) x *= p.row_scale[s_srow[m]];
+              if (p.row_scale) x *= p.row_scale[p.moe ? orow / p.a_div : pos];
               x *= cs;
               x *= gs;
-              p.out[(size_t)s_orow[m] * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(x));
+              p.out[(size_t)orow * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(x));
             }
           }
         }
       }
-    }
-    if (p.splits > 1) {
-      __threadfence();
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (tid == 0) s_info[3] = (atomicAdd(&p.counters[tile], 1) == p.splits - 1);
+      if (split_mode) __threadfence();  // partial visible before the tile ticket
+      // accumulator read: hand it back to the MMA warp
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acce[d]);
     }
   }
   tc_fence_before();
@@ -535,44 +656,60 @@ __global__ void __launch_bounds__(THREADS, 1) tc_gemm_kernel(const __grid_consta
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS));
   }
-  // ---- split-K fixup: the last split of a tile sums every split's partial
-  // in split order (deterministic), all threads, 16-byte loads, all splits
-  // of an item in flight together ----
-  if (p.splits > 1 && s_info[3] && !*(volatile int *)s_abort) {
-    __threadfence();
-    const int tile = slot * p.NT + wt;
-    const float4 *pp = reinterpret_cast<const float4 *>(p.partial + (size_t)tile * p.splits * BNT * BM);
+  if (!split_mode) return;
+  // ---- split mode: take the tile's ticket; the last split to arrive sums
+  // the S partials in split order (deterministic) with all threads, 16-byte
+  // loads and every split's load of an item in flight together.  Every split
+  // takes its ticket, so the counter is back at zero once all have arrived.
+  if (tid == 0) {
+    const int tk = atomicAdd(&p.counters[t_mine], 1);
+    const bool last = (tk == sch.S - 1);
+    if (last) p.counters[t_mine] = 0;  // ready for the next call
+    *s_last = (last && !*(volatile int *)s_abort) ? 1 : 0;
+  }
+  __syncthreads();
+  if (!*(volatile int *)s_last) return;
+  __threadfence();
+  {
+    const TileInfo ti = tile_info(t_mine);
+    const uint8_t *eb = p.packed + (size_t)ti.expert * p.stride;
+    const float4 *pp = reinterpret_cast<const float4 *>(p.partial + (size_t)t_mine * sch.S * BNT * BM);
     float gs = 1.f;
     if (WF == W_NVFP4) gs = reinterpret_cast<const float *>(eb + p.g_off)[0];
     if (p.a_global) gs = __fmul_rn(gs, *p.a_global);
-    for (int item = tid; item < nvalid * (BM / 4); item += THREADS) {
+    for (int item = tid; item < ti.nvalid * (BM / 4); item += THREADS) {
       const int m = item / (BM / 4), r4 = item % (BM / 4);
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int sp0 = 0; sp0 < p.splits; sp0 += 8) {
+      for (int s0 = 0; s0 < sch.S; s0 += 8) {
         float4 v[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j)
-          if (sp0 + j < p.splits) v[j] = __ldcg(pp + ((size_t)(sp0 + j) * BNT + m) * (BM / 4) + r4);
+          if (s0 + j < sch.S) v[j] = __ldcg(pp + ((size_t)(s0 + j) * BNT + m) * (BM / 4) + r4);
 #pragma unroll
         for (int j = 0; j < 8; ++j)
-          if (sp0 + j < p.splits) {
-            acc.x += v[j].x; acc.y += v[j].y; acc.z += v[j].z; acc.w += v[j].w;
+          if (s0 + j < sch.S) {
+            acc.x += v[j].x;
+            acc.y += v[j].y;
+            acc.z += v[j].z;
+            acc.w += v[j].w;
           }
       }
-      const float rs = p.row_scale ? p.row_scale[s_srow[m]] : 1.f;
+      const int pos = ti.base + m;
+      const int orow = p.moe ? p.perm[pos] : pos;
+      const float rs = p.row_scale ? p.row_scale[p.moe ? orow / p.a_div : pos] : 1.f;
       const float a4[4] = {acc.x, acc.y, acc.z, acc.w};
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const int n = wt * BM + r4 * 4 + j;
+        const int n = ti.wt * BM + r4 * 4 + j;
         if (n < p.N) {
-          float x = a4[j] * rs;
+          float x = a4[j];
+          if (p.row_scale) x *= rs;
           if (WF == W_FP8) x *= reinterpret_cast<const float *>(eb + p.c_off)[n];
           x *= gs;
-          p.out[(size_t)s_orow[m] * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(x));
+          p.out[(size_t)orow * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(x));
         }
       }
     }
-    if (tid == 0) p.counters[tile] = 0;  // ready for the next call
   }
 }
 
@@ -609,42 +746,27 @@ static bool make_act_map(CUtensorMap *m, const void *a, int rows, int K, int box
 }
 
 // Token tile = the smallest of 16, 32, 64, 128, 256 covering the rows a tile
-// is expected to hold; split-K until the grid covers the SMs about twice.
+// is expected to hold; persistent grid of (2 or 1) x 148 CTAs, fewer when
+// there are not at least 4 k-blocks of work per CTA.
 TcLaunch plan_tc(int rows_per_tile, int mtiles_bound_moe, int N, int KB, bool moe) {
   TcLaunch t{};
   t.bnt = rows_per_tile <= 16 ? 16 : rows_per_tile <= 32 ? 32 : rows_per_tile <= 64 ? 64 : rows_per_tile <= 128 ? 128 : 256;
   t.ntw = (N + TILE_N - 1) / TILE_N;
   t.mtiles = moe ? mtiles_bound_moe : (rows_per_tile + t.bnt - 1) / t.bnt;
   if (t.mtiles < 1) t.mtiles = 1;
-  const long tiles = (long)t.ntw * t.mtiles;
-  const long slots = (t.bnt <= 128 ? 2 : 1) * 148;  // CTAs resident at once
-  int max_splits = KB / 4;                          // at least 4 k-blocks per split
-  if (max_splits < 1) max_splits = 1;
-  // pick the split count with the least (waves x k-blocks per CTA), small
-  // penalty per extra split for the fixup traffic
-  int splits = 1;
-  double best = 1e30;
-  for (int s = 1; s <= max_splits && s <= 64; ++s) {
-    const int kb = (KB + s - 1) / s;
-    const long ctas = tiles * ((KB + kb - 1) / kb);
-    const long waves = (ctas + slots - 1) / slots;
-    const double cost = (double)waves * kb * (1.0 + 0.01 * s);
-    if (cost < best) {
-      best = cost;
-      splits = s;
-    }
-  }
-  int kbps = (KB + splits - 1) / splits;
-  splits = (KB + kbps - 1) / kbps;
-  t.splits = splits;
-  t.kb_per_split = kbps;
+  const long long iters = (long long)t.ntw * t.mtiles * KB;
+  const int slots = (t.bnt <= 64 ? 2 : 1) * 148;
+  long long n = (iters + 3) / 4;
+  if (n > slots) n = slots;
+  if (n < 1) n = 1;
+  t.nctas = (int)n;
   return t;
 }
 
 size_t tc_workspace_bytes(const TcLaunch &t) {
-  if (t.splits <= 1) return 256;
   const size_t tiles = (size_t)t.ntw * t.mtiles;
-  return align_up(tiles * sizeof(int), 256) + tiles * t.splits * t.bnt * TILE_N * sizeof(float);
+  // tile tickets, then one fp32 [bnt][128] partial per split (splits <= CTAs)
+  return align_up(tiles * sizeof(int), 256) + (size_t)t.nctas * t.bnt * TILE_N * sizeof(float);
 }
 
 template <int WF, int BNT, bool F8>
@@ -659,8 +781,7 @@ static hq_status tc_launch_one(const CUtensorMap &map, const tc::Params &p, cons
       return HQ_ERR_CUDA;
     if (dev < 32) configured |= 1u << dev;
   }
-  dim3 grid(t.ntw * t.splits, t.mtiles);
-  kern<<<grid, tc::THREADS, C::BYTES, st>>>(map, p);
+  kern<<<t.nctas, tc::THREADS, C::BYTES, st>>>(map, p);
   return check_launch();
 }
 
@@ -702,9 +823,10 @@ hq_status launch_tc_gemm(const Layout &L, const void *packed, const void *a_bf16
   p.a_div = a_div;
   p.gather = gather;
   p.out = (uint16_t *)out;
-  p.splits = t.splits;
-  p.kb_per_split = t.kb_per_split;
-  if (t.splits > 1) {
+  p.ntw = t.ntw;
+  p.mtiles = t.mtiles;
+  p.nctas = t.nctas;
+  {
     const size_t tiles = (size_t)t.ntw * t.mtiles;
     p.counters = (int *)workspace;
     p.partial = (float *)((uint8_t *)workspace + align_up(tiles * sizeof(int), 256));

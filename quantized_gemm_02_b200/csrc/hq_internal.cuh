@@ -237,11 +237,10 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
 
 // Launch plan of the tensor-core GEMM (hq_gemm_tc.cu).
 struct TcLaunch {
-  int bnt;           // token tile = MMA N (16, 32, 64, 128, 256)
-  int ntw;           // 128-row weight tiles
-  int mtiles;        // grid.y: token tiles (dense) or an upper bound on (expert, tile) pairs (MoE)
-  int splits;        // split-K factor
-  int kb_per_split;  // k-blocks per split
+  int bnt;     // token tile = MMA N (16, 32, 64, 128, 256)
+  int ntw;     // 128-row weight tiles
+  int mtiles;  // token tiles (dense) or an upper bound on (expert, tile) pairs (MoE)
+  int nctas;   // persistent CTAs
 };
 TcLaunch plan_tc(int rows_per_tile, int mtiles_bound_moe, int N, int KB, bool moe);
 size_t tc_workspace_bytes(const TcLaunch &t);

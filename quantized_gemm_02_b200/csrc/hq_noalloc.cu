@@ -59,7 +59,7 @@ extern "C" hq_status hq_gemm_noalloc(const hq_quant_desc *desc, int M, int N, in
   if (ss != HQ_OK) return ss;
   // The array keeps the previous call's contents; the split-K tile counters
   // at its head must start at zero.
-  if (pl.s.splits > 1) {
+  {
     const size_t counters = align_up((size_t)pl.s.ntw * pl.s.mtiles * sizeof(int), 256);
     if (cudaMemsetAsync(scratch, 0, counters, (cudaStream_t)stream) != cudaSuccess) return HQ_ERR_CUDA;
   }
