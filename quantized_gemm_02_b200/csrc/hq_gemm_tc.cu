@@ -302,6 +302,18 @@ __device__ __forceinline__ bool unit_at(const Sched &sc, int c, int nctas, int K
   return kb0 < kb1;
 }
 
+// A unit's k-blocks are walked in stages of KPS blocks, starting at a
+// CTA-dependent stage and wrapping around, so that the CTAs running at the
+// same time read different parts of the shared activation rows instead of
+// all hitting the same L2 lines.  Every role walks the same order; the
+// accumulation order is fixed by the CTA index, so results stay
+// deterministic.
+__device__ __forceinline__ int stage_rotation(int c, int nst) { return nst > 1 ? c % nst : 0; }
+__device__ __forceinline__ int stage_of(int i, int rot, int nst) {
+  const int s = i + rot;
+  return s >= nst ? s - nst : s;
+}
+
 template <int WF, int BNT, bool F8>
 __global__ void __launch_bounds__(THREADS, (BNT <= 64 ? 2 : 1)) tc_gemm_kernel(const __grid_constant__ CUtensorMap act_map,
                                                              const Params p) {
@@ -310,7 +322,9 @@ __global__ void __launch_bounds__(THREADS, (BNT <= 64 ? 2 : 1)) tc_gemm_kernel(c
   static_assert(!F8 || WF == W_FP8, "the E4M3 x E4M3 path takes FP8 weights");
   constexpr int NS = C::NS, ND = C::ND, NA = C::NA;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte alignment for the 128-byte swizzle, by offsetting from the
+  // shared array itself so that the compiler keeps every access an ld.shared
+  uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t *ctrl = smem + NS * C::STAGE;
   uint64_t *full = reinterpret_cast<uint64_t *>(ctrl);  // [NS] stage landed
   uint64_t *sfree = full + NS;                           // [NS] stage consumed (MMA + dequant)
@@ -419,7 +433,10 @@ __global__ void __launch_bounds__(THREADS, (BNT <= 64 ? 2 : 1)) tc_gemm_kernel(c
       int t, ukb0, ukb1, usp;
       if (!unit_at(sch, cta, p.nctas, p.KB, u, t, ukb0, ukb1, usp)) break;
       const TileInfo ti = tile_info(t);
-      for (int kbs = ukb0; kbs < ukb1; kbs += C::KPS, ++is) {
+      const int nst = (ukb1 - ukb0 + C::KPS - 1) / C::KPS;
+      const int rot = stage_rotation(cta, nst);
+      for (int i = 0; i < nst; ++i, ++is) {
+      const int kbs = ukb0 + stage_of(i, rot, nst) * C::KPS;
       const int nblk = min(C::KPS, ukb1 - kbs);
       const int s = is % NS;
       if (is >= NS && !mbar_wait(&sfree[s], ((is / NS) - 1) & 1)) { *s_abort = 1; stop = true; break; }
@@ -472,7 +489,10 @@ __global__ void __launch_bounds__(THREADS, (BNT <= 64 ? 2 : 1)) tc_gemm_kernel(c
     for (int u = 0; !stop; ++u) {
       int t, ukb0, ukb1, usp;
       if (!unit_at(sch, cta, p.nctas, p.KB, u, t, ukb0, ukb1, usp)) break;
-      for (int kbs = ukb0; kbs < ukb1 && !stop; kbs += C::KPS, ++is) {
+      const int nst = (ukb1 - ukb0 + C::KPS - 1) / C::KPS;
+      const int rot = stage_rotation(cta, nst);
+      for (int i = 0; i < nst && !stop; ++i, ++is) {
+      const int kbs = ukb0 + stage_of(i, rot, nst) * C::KPS;
       const int nblk = min(C::KPS, ukb1 - kbs);
       const int s = is % NS;
       if (!mbar_wait(&full[s], (is / NS) & 1)) { *s_abort = 1; stop = true; break; }
@@ -564,15 +584,17 @@ __global__ void __launch_bounds__(THREADS, (BNT <= 64 ? 2 : 1)) tc_gemm_kernel(c
       if (!unit_at(sch, cta, p.nctas, p.KB, u, t, ukb0, ukb1, usp)) break;
       const int d = u % ND;
       if (u >= ND && !mbar_wait(&acce[d], ((u / ND) - 1) & 1)) { *s_abort = 1; break; }
-      for (int kbs = ukb0; kbs < ukb1 && !stop; kbs += C::KPS, ++is) {
+      const int nst = (ukb1 - ukb0 + C::KPS - 1) / C::KPS;
+      const int rot = stage_rotation(cta, nst);
+      for (int i = 0; i < nst && !stop; ++i, ++is) {
+        const int kbs = ukb0 + stage_of(i, rot, nst) * C::KPS;
         const int nblk = min(C::KPS, ukb1 - kbs);
         const int s = is % NS;
         if (!mbar_wait(&full[s], (is / NS) & 1)) { *s_abort = 1; stop = true; break; }
         for (int j = 0; j < nblk; ++j, ++ia) {
           const int a = ia % NA;
-          const int kb = kbs + j;
-          const bool first = (kb == ukb0);
-          const bool last = (kb == ukb1 - 1);
+          const bool first = (i == 0 && j == 0);
+          const bool last = (i == nst - 1 && j == nblk - 1);
           if (!mbar_wait(&afull[a], (ia / NA) & 1)) { *s_abort = 1; stop = true; break; }
           if (*(volatile int *)s_abort) { stop = true; break; }
           tc_fence_after();
@@ -745,17 +767,32 @@ static bool make_act_map(CUtensorMap *m, const void *a, int rows, int K, int box
   return r == CUDA_SUCCESS;
 }
 
+static int sm_count() {
+  static int cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cached[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
 // Token tile = the smallest of 16, 32, 64, 128, 256 covering the rows a tile
-// is expected to hold; persistent grid of (2 or 1) x 148 CTAs, fewer when
-// there are not at least 4 k-blocks of work per CTA.
+// is expected to hold.  Up to 32 tokens: the decode kernel, one CTA per SM
+// (fewer when there are not 4 k-blocks of work per CTA).  Beyond: two (up to
+// 64 tokens) or one CTA per SM of the multi-stage kernel.
 TcLaunch plan_tc(int rows_per_tile, int mtiles_bound_moe, int N, int KB, bool moe) {
   TcLaunch t{};
   t.bnt = rows_per_tile <= 16 ? 16 : rows_per_tile <= 32 ? 32 : rows_per_tile <= 64 ? 64 : rows_per_tile <= 128 ? 128 : 256;
+  t.kind = t.bnt <= 32 ? 1 : 0;
   t.ntw = (N + TILE_N - 1) / TILE_N;
   t.mtiles = moe ? mtiles_bound_moe : (rows_per_tile + t.bnt - 1) / t.bnt;
   if (t.mtiles < 1) t.mtiles = 1;
   const long long iters = (long long)t.ntw * t.mtiles * KB;
-  const int slots = (t.bnt <= 64 ? 2 : 1) * 148;
+  const int sms = sm_count();
+  const int slots = t.kind == 1 ? sms : (t.bnt <= 64 ? 2 : 1) * sms;
   long long n = (iters + 3) / 4;
   if (n > slots) n = slots;
   if (n < 1) n = 1;
@@ -763,10 +800,17 @@ TcLaunch plan_tc(int rows_per_tile, int mtiles_bound_moe, int N, int KB, bool mo
   return t;
 }
 
-size_t tc_workspace_bytes(const TcLaunch &t) {
+size_t tc_counter_bytes(const TcLaunch &t) {
   const size_t tiles = (size_t)t.ntw * t.mtiles;
-  // tile tickets, then one fp32 [bnt][128] partial per split (splits <= CTAs)
-  return align_up(tiles * sizeof(int), 256) + (size_t)t.nctas * t.bnt * TILE_N * sizeof(float);
+  // decode kernel: one ticket per (tile, epilogue warp)
+  return align_up(tiles * (t.kind == 1 ? 4 : 1) * sizeof(int), 256);
+}
+
+size_t tc_workspace_bytes(const TcLaunch &t) {
+  // tile tickets, then the fp32 [bnt][128] partial tiles: one per split
+  // (splits <= CTAs), or a head and a tail slot per CTA in the decode kernel
+  const size_t parts = t.kind == 1 ? (size_t)t.nctas * 2 : (size_t)t.nctas;
+  return tc_counter_bytes(t) + parts * t.bnt * TILE_N * sizeof(float);
 }
 
 template <int WF, int BNT, bool F8>
@@ -795,6 +839,9 @@ static hq_status tc_launch_wf(const CUtensorMap &map, const tc::Params &p, const
     default: return tc_launch_one<WF, 256, F8>(map, p, t, st);
   }
 }
+
+hq_status launch_dec_gemm(const Layout &L, const tc::Params &p, const void *a, int a_rows, const TcLaunch &t,
+                          cudaStream_t st, bool e4m3_act);
 
 // a_bf16 holds `a_rows` rows of K bf16 values.  Dense and MoE grouped: a tile
 // reads the rows [row_base, row_base + BNT) (rows past a tile's end are
@@ -826,10 +873,11 @@ hq_status launch_tc_gemm(const Layout &L, const void *packed, const void *a_bf16
   p.ntw = t.ntw;
   p.mtiles = t.mtiles;
   p.nctas = t.nctas;
-  {
-    const size_t tiles = (size_t)t.ntw * t.mtiles;
-    p.counters = (int *)workspace;
-    p.partial = (float *)((uint8_t *)workspace + align_up(tiles * sizeof(int), 256));
+  p.counters = (int *)workspace;
+  p.partial = (float *)((uint8_t *)workspace + tc_counter_bytes(t));
+  if (t.kind == 1) {
+    if (gather) return HQ_ERR_UNSUPPORTED;
+    return launch_dec_gemm(L, p, a_bf16, a_rows, t, st, e4m3_act);
   }
   switch (L.fmt) {
     case W_INT4: return tc_launch_wf<W_INT4>(map, p, t, st);

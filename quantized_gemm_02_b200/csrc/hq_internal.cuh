@@ -237,6 +237,7 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
 
 // Launch plan of the tensor-core GEMM (hq_gemm_tc.cu).
 struct TcLaunch {
+  int kind;    // 0: multi-CTA-per-SM kernel (>= 64 tokens per tile); 1: decode kernel (16 or 32)
   int bnt;     // token tile = MMA N (16, 32, 64, 128, 256)
   int ntw;     // 128-row weight tiles
   int mtiles;  // token tiles (dense) or an upper bound on (expert, tile) pairs (MoE)
@@ -244,6 +245,9 @@ struct TcLaunch {
 };
 TcLaunch plan_tc(int rows_per_tile, int mtiles_bound_moe, int N, int KB, bool moe);
 size_t tc_workspace_bytes(const TcLaunch &t);
+// Bytes at the head of the workspace that must be zero before the first
+// call (tile tickets; every call leaves them zero again).
+size_t tc_counter_bytes(const TcLaunch &t);
 
 // Host-side helpers implemented in hq_api.cu.
 hq_status check_launch();

@@ -60,8 +60,7 @@ extern "C" hq_status hq_gemm_noalloc(const hq_quant_desc *desc, int M, int N, in
   // The array keeps the previous call's contents; the split-K tile counters
   // at its head must start at zero.
   {
-    const size_t counters = align_up((size_t)pl.s.ntw * pl.s.mtiles * sizeof(int), 256);
-    if (cudaMemsetAsync(scratch, 0, counters, (cudaStream_t)stream) != cudaSuccess) return HQ_ERR_CUDA;
+    if (cudaMemsetAsync(scratch, 0, tc_counter_bytes(pl.s), (cudaStream_t)stream) != cudaSuccess) return HQ_ERR_CUDA;
   }
   return hq_gemm(desc, M, N, K, packed_w, a, a_scales, a_global, c_bf16, scratch, NOALLOC_SCRATCH_BYTES, stream);
 }
