@@ -55,20 +55,59 @@ def load_peaks():
 # clocks sampler (nvidia-smi during the timed region)
 # ---------------------------------------------------------------------------
 class Clocks:
+    """Samples the SM clock and the clock-event reasons of this rank's GPU
+    during the timed region: NVML every 10 ms (read-only queries), else
+    nvidia-smi every 50 ms."""
+
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                   "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
 
     def __init__(self, index: int):
         self.index = index
         self.proc = None
+        self.nvml = None
         self.lines = []
+        self.samples = []  # (sm_mhz, max_mhz, reason bits)
+        self.stop_flag = threading.Event()
+
+    def _nvml_handle(self, pynvml):
+        try:
+            props = torch.cuda.get_device_properties(self.index)
+            bus = "%08X:%02X:%02X.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+            return pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(self.index)
 
     def start(self):
         try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = self._nvml_handle(pynvml)
+            mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.nvml = pynvml
+
+            def loop():
+                while not self.stop_flag.is_set():
+                    try:
+                        sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                        rb = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        self.samples.append((float(sm), float(mx), int(rb)))
+                    except Exception:
+                        pass
+                    time.sleep(0.01)
+
+            self.th = threading.Thread(target=loop, daemon=True)
+            self.th.start()
+            return
+        except Exception:
+            self.nvml = None
+        try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.th = threading.Thread(target=self._read, daemon=True)
             self.th.start()
         except OSError:
@@ -79,6 +118,19 @@ class Clocks:
             self.lines.append(line.strip())
 
     def stop(self):
+        if self.nvml is not None:
+            self.stop_flag.set()
+            self.th.join(timeout=2)
+            if not self.samples:
+                return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+            reasons = set()
+            for _, _, rb in self.samples:
+                for n, bit in self.REASON_BITS.items():
+                    if rb & bit:
+                        reasons.add(n)
+            return {"sm_mhz": statistics.median(x[0] for x in self.samples),
+                    "sm_max_mhz": max(x[1] for x in self.samples), "reasons": sorted(reasons),
+                    "samples": len(self.samples), "source": "nvml, 10 ms"}
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
@@ -104,7 +156,7 @@ class Clocks:
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "source": "nvidia-smi, 50 ms"}
 
 
 # ---------------------------------------------------------------------------
@@ -113,8 +165,9 @@ class Clocks:
 class Op:
     """One library call of a step, with its algorithmic cost."""
 
-    def __init__(self, name, run, flops, w_bytes, io_bytes, kernels, h2d=None, d2h=None, e2e=None):
+    def __init__(self, name, run, flops, w_bytes, io_bytes, kernels, h2d=None, d2h=None, e2e=None, kernel=None):
         self.name = name
+        self.kernel = kernel      # the library kernel that dominates the call
         self.run = run            # device-resident call
         self.flops = flops
         self.w_bytes = w_bytes    # packed weight + scale + zero bytes the call must read
@@ -161,7 +214,44 @@ def dense_op(hq, d, name, M, N, K, packed, w_bytes, gen, a_fmt="bf16", a_bits=No
         hq.hq_gemm(d, M, N, K, packed, A_e, None, None, C, ws, wsb)
         C_h.copy_(C, non_blocking=True)
 
-    return Op(name, run, 2.0 * M * N * K, w_bytes, M * K * 2 + M * N * 2, 1, M * K * 2, M * N * 2, e2e)
+    return Op(name, run, 2.0 * M * N * K, w_bytes, M * K * 2 + M * N * 2, 1, M * K * 2, M * N * 2, e2e,
+              kernel=gemm_kernel_name(M))
+
+
+def gemm_kernel_name(rows_per_tile):
+    """The GEMM kernel the library picks for a token tile of this many rows."""
+    return "dec_gemm_kernel" if rows_per_tile <= 32 else "tc_gemm_kernel"
+
+
+KERNEL_SOURCES = ("quantized_gemm_02_b200/csrc/hq_gemm_tc.cu", "quantized_gemm_02_b200/csrc/hq_gemm_small.cu",
+                  "quantized_gemm_02_b200/csrc/hq_internal.cuh")
+
+
+def kernel_source_digest():
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(op_name):
+    """DRAM bytes per launch (read + write) of the op's GEMM kernel from the
+    committed ncu capture in profiles/traffic.md, or None when there is none
+    or the kernel sources changed since it was taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.md")
+    if not os.path.exists(p):
+        return None
+    digest = kernel_source_digest()
+    for line in open(p):
+        f = [x.strip() for x in line.strip().strip("|").split("|")]
+        if len(f) >= 6 and f[0] == op_name and f[5] == digest:
+            try:
+                return float(f[4])
+            except ValueError:
+                return None
+    return None
 
 
 def packed_bytes_int4(N, K, group, zero):
@@ -557,8 +647,9 @@ def main():
     else:
         roof = {"bound": "hbm", "achieved": dom.bytes / t_dom / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = None
-    roof["kernel"] = "hq stream_gemm (" + dom.name + ")"
+    roof["traffic"] = measured_traffic(dom.name)
+    roof["algorithmic_bytes"] = dom.bytes
+    roof["kernel"] = (dom.kernel or "hq") + " (" + dom.name + ")"
     roof["peak_source"] = peaks["source"] + (" burst" if roof["bound"] == "tensor" else "")
 
     sweep = []

@@ -162,15 +162,20 @@ __device__ __forceinline__ void decode_bf16(const uint8_t *wpk, const uint8_t *s
                                             int kbase, int g0, int gshift, uint32_t (&rg)[32]) {
   using TR = Traits<WF>;
   if constexpr (TR::wbits == 4) {
+    uint32_t s2c = 0, z2c = 0;  // INT4 / UINT4: scale and zero point of the previous chunk
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
       const uint4 v = *reinterpret_cast<const uint4 *>(wpk + c * (BM * 16) + r * 16);
       const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
       const int gt = ((kbase + 32 * c) >> gshift) - g0;  // group of this chunk's first k
       if constexpr (WF == W_INT4 || WF == W_UINT4) {
-        // groups are >= 32 k: one scale (and zero point) per chunk
-        const uint32_t s2 = tc::bcast16(reinterpret_cast<const uint16_t *>(sc)[gt * BM + r]);
-        const uint32_t z2 = (WF == W_UINT4) ? tc::bcast16(0x4300u + zp[gt * BM + r]) : 0x43084308u;
+        // groups are >= 32 k: one scale (and zero point) per chunk, loaded
+        // again only when the second chunk starts a new group
+        if (c == 0 || gt != (((kbase) >> gshift) - g0)) {
+          s2c = tc::bcast16(reinterpret_cast<const uint16_t *>(sc)[gt * BM + r]);
+          z2c = (WF == W_UINT4) ? tc::bcast16(0x4300u + zp[gt * BM + r]) : 0x43084308u;
+        }
+        const uint32_t s2 = s2c, z2 = z2c;
 #pragma unroll
         for (int j = 0; j < 4; ++j)
 #pragma unroll
@@ -220,7 +225,7 @@ __global__ void __launch_bounds__(THREADS, 1) dec_gemm_kernel(const __grid_const
   uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t *ctrl = smem + NS * C::STAGE;
   uint64_t *full = reinterpret_cast<uint64_t *>(ctrl);  // [NS] stage landed
-  uint64_t *sfree = full + NS;                           // [NS] stage consumed (MMA + dequant)
+  uint64_t *sfree = full + NS;                           // [NS] stage consumed (MMA done)
   uint64_t *afull = sfree + NS;                          // [NAS] decoded stage in TMEM
   uint64_t *aempty = afull + NAS;                        // [NAS] decoded stage consumed by the MMA
   uint64_t *accf = aempty + NAS;                         // [ND] accumulator complete
@@ -265,7 +270,7 @@ __global__ void __launch_bounds__(THREADS, 1) dec_gemm_kernel(const __grid_const
   if (tid == 32) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 2);  // weight and activation producers
-      mbar_init(&sfree[s], 1 + NDQ);
+      mbar_init(&sfree[s], 1);  // MMA commit: it runs after every dequant warp is done with the stage
     }
     for (int a = 0; a < NAS; ++a) {
       mbar_init(&afull[a], NDQ);
@@ -322,7 +327,7 @@ __global__ void __launch_bounds__(THREADS, 1) dec_gemm_kernel(const __grid_const
     // Packed weights, scales and zero points of each stage: three 1-D bulk
     // copies.  The activations come from their own producer warp, so that
     // the copy engine always has the next stage's requests queued.
-    const uint64_t pol = policy_evict_first();
+    const uint64_t pol = p.weights_once ? policy_evict_first() : policy_evict_normal();
     Walk w;
     w.start(beg, end, p.KB);
     Ring rs;
@@ -421,10 +426,7 @@ __global__ void __launch_bounds__(THREADS, 1) dec_gemm_kernel(const __grid_const
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       tc::tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&afull[ra.idx]);
-        mbar_arrive(&sfree[rs.idx]);
-      }
+      if (lane == 0) mbar_arrive(&afull[ra.idx]);
     }
   } else if (warp == WARP_MMA) {
     // ================= MMA issuer (whole warp in step, one elected lane issues) =================

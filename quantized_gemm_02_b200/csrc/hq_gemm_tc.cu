@@ -106,6 +106,8 @@ struct Params {
   int ntw;                 // 128-row weight tiles
   int mtiles;              // token tiles (dense: exact; MoE: upper bound)
   int nctas;               // persistent CTAs (grid size)
+  int weights_once;        // every weight tile is read by one token tile only (stream it past L2)
+  int group_slots;         // dense: token tiles per raster group (<= 1: weight tile fastest)
   float *partial;          // [tiles * S][BNT][128] fp32 split-K partial tiles
   int *counters;           // [ntw * mtiles] per-tile arrival tickets
 };
@@ -395,8 +397,21 @@ __global__ void __launch_bounds__(THREADS, (BNT <= 64 ? 2 : 1)) tc_gemm_kernel(c
   // tile index -> weight tile, expert, token rows
   auto tile_info = [&](int t) {
     TileInfo ti;
-    const int slot = t / p.ntw;
-    ti.wt = t - slot * p.ntw;
+    int slot;
+    if (!p.moe && p.group_slots > 1) {
+      // dense: token tiles in groups of group_slots, the token tile fastest
+      // inside a group, so that the CTAs running together share each weight
+      // tile across the group and every weight byte leaves HBM once per group
+      const int per = p.group_slots * p.ntw;
+      const int grp = t / per;
+      const int rem = t - grp * per;
+      const int gs = min(p.group_slots, p.mtiles - grp * p.group_slots);
+      ti.wt = rem / gs;
+      slot = grp * p.group_slots + (rem - ti.wt * gs);
+    } else {
+      slot = t / p.ntw;
+      ti.wt = t - slot * p.ntw;
+    }
     if (!p.moe) {
       ti.expert = 0;
       ti.base = slot * BNT;
@@ -426,7 +441,7 @@ __global__ void __launch_bounds__(THREADS, (BNT <= 64 ? 2 : 1)) tc_gemm_kernel(c
   const uint32_t tmem = *tmem_slot;
   if (warp == WARP_PRODUCER) {
     // ================= producer (whole warp in step, lane 0 issues) =================
-    const uint64_t pol = policy_evict_first();
+    const uint64_t pol = p.weights_once ? policy_evict_first() : policy_evict_normal();
     int is = 0;
     bool stop = false;
     for (int u = 0; !stop; ++u) {
@@ -873,6 +888,15 @@ hq_status launch_tc_gemm(const Layout &L, const void *packed, const void *a_bf16
   p.ntw = t.ntw;
   p.mtiles = t.mtiles;
   p.nctas = t.nctas;
+  p.weights_once = (!moe && t.mtiles == 1) ? 1 : 0;
+  // raster groups of token tiles whose activations take about 32 MB of L2
+  {
+    const long long act_tile = (long long)t.bnt * L.K * (e4m3_act ? 1 : 2);
+    long long gsl = (32ll << 20) / (act_tile > 0 ? act_tile : 1);
+    if (gsl < 1) gsl = 1;
+    if (gsl > t.mtiles) gsl = t.mtiles;
+    p.group_slots = (int)gsl;
+  }
   p.counters = (int *)workspace;
   p.partial = (float *)((uint8_t *)workspace + tc_counter_bytes(t));
   if (t.kind == 1) {
