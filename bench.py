@@ -367,9 +367,14 @@ def moe_ops(hq, name, wdesc, E, topk, H, I, Ts, routing, gen, mode_names=("group
             flops = 2.0 * T * topk * (Ng * Kg + Nd * Kd)
             wbytes = touched * (bg + bd)
             io = T * Kg * 2 + T * topk * Ng * 2 + T * topk * Kd * 2 + T * Nd * 2
-            quant = 1 if (a_dtype is not None and a_dtype != hq.HQ_BF16) else 0
-            # kernels: permute; per GEMM [quant + decode | gather] + GEMM; combine
-            kernels = 1 + (2 + quant) * 2 + 1
+            quant = a_dtype is not None and a_dtype != hq.HQ_BF16
+            block_scaled = (wdesc.w_dtype == hq.HQ_E2M1 and
+                            ((wdesc.w_scale_dtype == hq.HQ_E8M0 and a_dtype == hq.HQ_MXFP8) or
+                             (wdesc.w_scale_dtype == hq.HQ_UE4M3 and a_dtype == hq.HQ_NVFP4)))
+            # kernels: permute; per GEMM: quant + gather codes + scale relayout + GEMM (block-scaled MMA),
+            # quant + decode + GEMM, or gather + GEMM (bf16); combine
+            per_gemm = 4 if block_scaled else (3 if quant else 2)
+            kernels = 1 + per_gemm * 2 + 1
             ops.append(Op(f"{name}_T{T}_{mode_name}", run, flops, wbytes, io, kernels,
                           T * topk * 4 + T * Kg * 2, T * Nd * 2, e2e))
     return ops, weights

@@ -29,6 +29,14 @@ hq_status launch_tc_gemm(const Layout &L, const void *packed, const void *a_bf16
                          int a_div, int gather, void *out, const TcLaunch &t, void *workspace, cudaStream_t st,
                          bool e4m3_act = false);
 
+hq_status launch_bs_gemm(const Layout &L, const void *packed, int E, const void *a_codes, int a_rows,
+                         const void *a_scales, int a_div, const float *a_global, int M, int moe,
+                         const int32_t *offsets, const int32_t *perm, void *out, const TcLaunch &t,
+                         void *workspace, void *sf_tiles, cudaStream_t st);
+size_t bs_sf_tiles_bytes(const Layout &L, const TcLaunch &t);
+hq_status launch_gather_bytes(int R, int row_bytes, const void *a, const int32_t *idx, int div, void *out,
+                              cudaStream_t st);
+
 hq_status check_launch() {
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
@@ -79,16 +87,20 @@ static hq_status plan_dense(const hq_quant_desc *d, int M, int N, int K, DensePl
   if (!d) return HQ_ERR_INVALID_ARG;
   if (!weight_format(d, &fmt) || !act_format(d, &afmt)) return HQ_ERR_UNSUPPORTED;
   if (M < 0 || N < 1 || !valid_k(d, K)) return HQ_ERR_INVALID_ARG;
-  pl->L = make_layout(fmt, d->w_group, N, K);
+  pl->L = layout_for(d, fmt, N, K);
   pl->afmt = afmt;
-  pl->s = plan_tc(M > 0 ? M : 1, 0, N, pl->L.KB, false);
+  pl->s = plan_tc(M > 0 ? M : 1, 0, N, pl->L.KB, false, pl->L.bs);
   return HQ_OK;
 }
 
+// Dense workspace: split-K state; then either the decoded bf16 copy of
+// quantised activations, or (block-scaled MMA) the activation scales in the
+// kernel's chunk order.
 static size_t dense_ws(const DensePlan &pl, int M, int K, uint8_t *base, void **split_ws, void **a_dec) {
   Carver c{base};
   *split_ws = c.take(tc_workspace_bytes(pl.s));
-  *a_dec = (pl.afmt != A_BF16) ? c.take((size_t)M * K * 2) : nullptr;
+  if (pl.L.bs != BS_NONE) *a_dec = c.take(bs_sf_tiles_bytes(pl.L, pl.s));
+  else *a_dec = (pl.afmt != A_BF16) ? c.take((size_t)M * K * 2) : nullptr;
   return c.off;
 }
 
@@ -108,31 +120,40 @@ static hq_status plan_moe(const hq_quant_desc *d, int T, int topk, int E, int N,
   if (!weight_format(d, &fmt) || !act_format(d, &afmt)) return HQ_ERR_UNSUPPORTED;
   if (T < 0 || topk < 1 || E < 1 || E > 1024 || N < 1 || !valid_k(d, K)) return HQ_ERR_INVALID_ARG;
   if ((long)T * topk > (1L << 30)) return HQ_ERR_INVALID_ARG;
-  pl->L = make_layout(fmt, d->w_group, N, K);
+  pl->L = layout_for(d, fmt, N, K);
   pl->afmt = afmt;
   pl->R = T * topk;
   pl->src_rows = a_per_slot ? pl->R : T;
   const int R = pl->R > 0 ? pl->R : 1;
   const int active = R < E ? R : E;
   const int avg = (R + active - 1) / active;
-  const int bnt = plan_tc(avg, 1, N, pl->L.KB, true).bnt;
+  const int bnt = plan_tc(avg, 1, N, pl->L.KB, true, pl->L.bs).bnt;
   long bound = (R + bnt - 1) / bnt + active;
   if (bound > R) bound = R;
-  pl->s = plan_tc(avg, (int)bound, N, pl->L.KB, true);
+  pl->s = plan_tc(avg, (int)bound, N, pl->L.KB, true, pl->L.bs);
   return HQ_OK;
 }
 
 struct MoeWs {
   void *split, *y, *a_bf16, *codes, *scales, *glob, *amax;
+  void *s_codes, *s_scales;  // block-scaled layouts: expert-sorted codes, scale chunks per token tile
 };
 
 static size_t moe_ws(const MoePlan &pl, hq_moe_mode mode, int K, int N, int combine, uint8_t *base, MoeWs *w) {
   Carver c{base};
   w->split = c.take(tc_workspace_bytes(pl.s));
   w->y = combine ? c.take((size_t)pl.R * N * 2) : nullptr;
-  // both modes currently stage the expert-sorted rows (see hq_moe_gemm)
+  // both modes stage the expert-sorted rows (see hq_moe_gemm): bf16 rows, or
+  // for a block-scaled layout the quantised codes and scales as they are
   (void)mode;
-  w->a_bf16 = c.take((size_t)pl.R * K * 2);
+  if (pl.L.bs == BS_NONE) {
+    w->a_bf16 = c.take((size_t)pl.R * K * 2);
+    w->s_codes = w->s_scales = nullptr;
+  } else {
+    w->a_bf16 = nullptr;
+    w->s_codes = c.take((size_t)pl.R * act_code_bytes(pl.afmt, K));
+    w->s_scales = c.take(bs_sf_tiles_bytes(pl.L, pl.s));  // scales in the kernel's chunk order
+  }
   if (pl.afmt != A_BF16) {
     w->codes = c.take((size_t)pl.src_rows * act_code_bytes(pl.afmt, K));
     w->scales = c.take((size_t)pl.src_rows * act_scale_bytes(pl.afmt, K));
@@ -175,7 +196,7 @@ hq_status hq_device_error(hq_stream_t stream) {
 size_t hq_packed_weights_bytes(const hq_quant_desc *desc, int E, int N, int K) {
   int fmt;
   if (!weight_format(desc, &fmt) || E < 1 || N < 1 || !valid_k(desc, K)) return 0;
-  return make_layout(fmt, desc->w_group, N, K).stride * (size_t)E;
+  return layout_for(desc, fmt, N, K).stride * (size_t)E;
 }
 
 hq_status hq_pack_weights(const hq_quant_desc *desc, int E, int N, int K, const void *codes, const void *scales,
@@ -189,7 +210,7 @@ hq_status hq_pack_weights(const hq_quant_desc *desc, int E, int N, int K, const 
   if ((fmt == W_NVFP4) != (global_scale != nullptr)) return HQ_ERR_INVALID_ARG;
   if (!aligned16(codes) || !aligned16(packed) || ((uintptr_t)scales & 3u)) return HQ_ERR_INVALID_ARG;
   if (!device_is_sm100()) return HQ_ERR_ARCH;
-  const Layout L = make_layout(fmt, desc->w_group, N, K);
+  const Layout L = layout_for(desc, fmt, N, K);
   return launch_pack(L, E, codes, scales, zeros, global_scale, packed, (cudaStream_t)stream);
 }
 
@@ -203,7 +224,7 @@ hq_status hq_unpack_weights(const hq_quant_desc *desc, int E, int N, int K, cons
   if ((fmt == W_UINT4) != (zeros != nullptr)) return HQ_ERR_INVALID_ARG;
   if ((fmt == W_NVFP4) != (global_scale != nullptr)) return HQ_ERR_INVALID_ARG;
   if (!device_is_sm100()) return HQ_ERR_ARCH;
-  const Layout L = make_layout(fmt, desc->w_group, N, K);
+  const Layout L = layout_for(desc, fmt, N, K);
   return launch_unpack(L, E, packed, codes, scales, zeros, global_scale, (cudaStream_t)stream);
 }
 
@@ -248,6 +269,11 @@ hq_status hq_gemm(const hq_quant_desc *desc, int M, int N, int K, const void *pa
   if (!workspace || ws_bytes < need || !aligned16(workspace)) return HQ_ERR_WORKSPACE;
   if (!device_is_sm100()) return HQ_ERR_ARCH;
   cudaStream_t st = (cudaStream_t)stream;
+  if (pl.L.bs != BS_NONE) {
+    // block-scaled MMA: the quantised activations go to the tensor core as they are
+    return launch_bs_gemm(pl.L, packed_w, 1, a, M, a_scales, 1, pl.afmt == A_NVFP4 ? a_global : nullptr, M, 0,
+                          nullptr, nullptr, c_bf16, pl.s, split_ws, a_dec, st);
+  }
   if (pl.L.fmt == W_FP8 && pl.afmt == A_FP8) {
     // E4M3 x E4M3 on the FP8 tensor path; per-token x per-channel scales in the epilogue
     return launch_tc_gemm(pl.L, packed_w, a, M, (const float *)a_scales, nullptr, M, 0, 1, nullptr, nullptr, 1, 0,
@@ -309,6 +335,20 @@ hq_status hq_moe_gemm(hq_moe_mode mode, const hq_quant_desc *desc, int T, int to
   // workspace first.  Results do not depend on the mode.
   const int a_indexed = 0;
   hq_status s = HQ_OK;
+  void *y = combine ? w.y : out_bf16;
+  if (pl.L.bs != BS_NONE) {
+    // quantise the caller rows once, gather codes and scales into expert order
+    s = launch_quant_act(pl.afmt, pl.src_rows, K, a_bf16, w.codes, w.scales, (float *)w.glob, nullptr, w.amax, st);
+    if (s != HQ_OK) return s;
+    s = launch_gather_bytes(pl.R, (int)act_code_bytes(pl.afmt, K), w.codes, perm, div, w.s_codes, st);
+    if (s != HQ_OK) return s;
+    s = launch_bs_gemm(pl.L, packed_w, E, w.s_codes, pl.R, w.scales, div,
+                       pl.afmt == A_NVFP4 ? (const float *)w.glob : nullptr, 0, 1, expert_offsets, perm, y, pl.s,
+                       w.split, w.s_scales, st);
+    if (s != HQ_OK) return s;
+    if (combine) s = launch_unpermute_sum(T, topk, N, y, nullptr, topk_weights, routed_scale, out_bf16, st);
+    return s;
+  }
   if (pl.afmt != A_BF16) {
     s = launch_quant_act(pl.afmt, pl.src_rows, K, a_bf16, w.codes, w.scales, (float *)w.glob, nullptr, w.amax, st);
     if (s != HQ_OK) return s;
@@ -321,7 +361,6 @@ hq_status hq_moe_gemm(hq_moe_mode mode, const hq_quant_desc *desc, int T, int to
     if (s != HQ_OK) return s;
   }
   a_use = w.a_bf16;
-  void *y = combine ? w.y : out_bf16;
   const int a_rows = (a_indexed ? pl.src_rows : pl.R);
   s = launch_tc_gemm(pl.L, packed_w, a_use, a_rows, row_scale, a_global, 0, 1, E, expert_offsets, perm, div, a_indexed,
                      y, pl.s, w.split, st);

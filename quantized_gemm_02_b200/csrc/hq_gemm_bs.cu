@@ -1,0 +1,645 @@
+// Block-scaled tensor-core GEMM: MXFP4 weights x MXFP8 activations and
+// NVFP4 weights x NVFP4 activations, with the block scales applied by the
+// tensor core itself (no dequantisation anywhere).
+//
+// "Announcing Humming", section "Shared CUDA components across formats and
+// architectures": the microscaling formats feed block-scaled MMAs directly on
+// hardware that has them; OCP Microscaling Formats (MX) v1.0 specification,
+// sections 5.1-5.3 (shared E8M0 scale per 32 elements) and the NVFP4 format
+// (E4M3 scale per 16 elements and an FP32 tensor scale).  The sm_100a design:
+//
+//   * tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale (MX, K = 32 per
+//     instruction, E2M1 weights expanded to one byte per code in shared
+//     memory by the TMA) or kind::mxf4nvf4.block_scale.scale_vec::4X (NV,
+//     K = 64, both operands packed E2M1); 128 weight rows are operand A,
+//     16..128 tokens operand B, both in shared memory with a 128-byte swizzle;
+//   * the scale chunks (128 rows x 4 scales, 512 bytes) go shared memory ->
+//     tensor memory with tcgen05.cp.32x128b.warpx4; the weight scales are
+//     stored in that order by the repack, the activation scales are gathered
+//     into it by the activation producer;
+//   * warps: 0..3 epilogue, 4 weight producer (3-D TMA of the codes, bulk copy
+//     of the scale chunks), 5 MMA issuer, 6 activation producer (2-D TMA of
+//     the codes, bulk copy of the scale chunks);
+//   * the activation scales are put in chunk order per token tile by a small
+//     kernel first (bs_sf_tiles_kernel; for MoE it also follows the
+//     permutation, so the expert-sorted scales are never stored row-wise);
+//   * persistent CTAs, one per SM, Stream-K over (tile, stage) iterations with
+//     the decode kernel's deterministic last-arriver fixup;
+//   * every mbarrier wait is bounded; a timeout records HQ_ERR_TIMEOUT.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include "hq_internal.cuh"
+
+namespace hq {
+
+namespace bs {
+
+using tc::BM;
+using tc::Params;
+using tc::TileInfo;
+
+constexpr int WARP_W = 4, WARP_MMA = 5, WARP_ACT = 6;
+constexpr int THREADS = 7 * 32;
+constexpr int TMEM_COLS = 512;
+constexpr int SFA_COL = 256;  // TMEM columns of the weight scales (after two 128-column accumulators)
+constexpr int SFB_COL = 288;  // TMEM columns of the activation scales
+
+// KIND: BS_MX or BS_NV.  A stage is one 128-byte row of each operand: 128 k
+// (MX: E2M1 expanded to bytes / E4M3) or 256 k (NV: packed E2M1), four MMAs.
+template <int KIND, int BNT>
+struct Cfg {
+  static constexpr int KSTAGE = KIND == BS_MX ? 128 : 256;
+  static constexpr int SF_CH = KIND == BS_MX ? 1 : 4;  // scale chunks (4 columns) per stage
+  static constexpr int W_SMEM = BM * 128;                  // weight tile in shared memory
+  static constexpr int W_GLOBAL = KIND == BS_MX ? BM * 64 : BM * 128;  // packed bytes it is read from
+  static constexpr int A_SMEM = BNT * 128;
+  static constexpr int SFA_OFF = W_SMEM + A_SMEM;
+  static constexpr int SFB_OFF = SFA_OFF + SF_CH * 512;
+  static constexpr int STAGE = (SFB_OFF + SF_CH * 512 + 1023) / 1024 * 1024;
+  static constexpr int NS_FIT = (200 * 1024) / STAGE;
+  static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;
+  static constexpr int CTRL = 8192;
+  static constexpr int BYTES = NS * STAGE + CTRL + 1024;
+  static constexpr int ND = 2;
+  static_assert(BNT <= 128 && ND * BNT <= SFA_COL, "accumulators fit before the scale columns");
+  static_assert(SFB_COL + 4 * SF_CH <= TMEM_COLS, "TMEM budget");
+  static_assert(NS >= 3, "stage too large");
+};
+
+// Instruction descriptor of the block-scaled kinds (M = 128, K-major A and B).
+template <int KIND, int BNT>
+__device__ __forceinline__ constexpr uint32_t idesc_bs(uint32_t sf_id) {
+  return (sf_id << 4)                                            // B scale id (byte of the scale column)
+         | ((KIND == BS_MX ? 5u : 1u) << 7)                      // A = E2M1
+         | ((KIND == BS_MX ? 0u : 1u) << 10)                     // B = E4M3 (MX) / E2M1 (NV)
+         | ((uint32_t)(BNT >> 3) << 17)                          // N
+         | ((KIND == BS_MX ? 1u : 0u) << 23)                     // scales: UE8M0 (MX) / UE4M3 (NV)
+         | ((uint32_t)(BM >> 4) << 24)                           // M
+         | (sf_id << 29);                                        // A scale id
+}
+
+// Shared-memory descriptor of a 32-row x 16-byte scale chunk (no swizzle,
+// 8-row core matrices 128 bytes apart).
+__device__ __forceinline__ uint64_t sf_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)(128 >> 4) << 16;
+  d |= (uint64_t)(128 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  return d;
+}
+
+__device__ __forceinline__ void sf_copy(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+template <int KIND>
+__device__ __forceinline__ void mma_bs(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t sfa,
+                                       uint32_t sfb, uint32_t acc) {
+  if constexpr (KIND == BS_MX) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb));
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+            tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb));
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Walks a CTA's iterations one stage at a time; a segment is a run inside
+// one tile.  Every role walks the same sequence.
+struct Walk {
+  int t, ks, left;
+  bool seg_first, seg_last;
+  __device__ __forceinline__ void start(long long beg, long long end, int ki) {
+    t = (int)(beg / ki);
+    ks = (int)(beg - (long long)t * ki);
+    left = (int)(end - beg);
+    seg_first = true;
+    seg_last = (ks + 1 == ki) || (left == 1);
+  }
+  __device__ __forceinline__ void next(int ki) {
+    --left;
+    ++ks;
+    seg_first = (ks == ki);
+    if (ks == ki) {
+      ks = 0;
+      ++t;
+    }
+    seg_last = (ks + 1 == ki) || (left == 1);
+  }
+};
+
+// The epilogue of one segment, 32 token columns at a time (the accumulator
+// columns of a 128-token tile do not fit in registers at once).  Whole tiles
+// are written directly; a Stream-K piece is stored as an fp32 partial and the
+// last of the CTAs sharing the tile sums the parts in k order.
+template <int BNT>
+__device__ __forceinline__ void epilogue_segment(const Params &p, const TileInfo &ti, int t, bool whole, bool head,
+                                                 uint32_t tacc, uint64_t *acce, float gs, int cta, int warp, int lane,
+                                                 long long total) {
+  constexpr int CW = BNT < 32 ? BNT : 32;
+  const int r = warp * 32 + lane;
+  const int n = ti.wt * BM + r;
+  float *part = p.partial + ((size_t)cta * 2 + (head ? 0 : 1)) * BNT * BM;
+  auto write = [&](int c0, const float *x) {
+    if (n >= p.N) return;
+#pragma unroll
+    for (int i = 0; i < CW; ++i) {
+      const int m = c0 + i;
+      if (m < ti.nvalid) {
+        const int pos = ti.base + m;
+        const int orow = p.moe ? p.perm[pos] : pos;
+        p.out[(size_t)orow * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(x[i] * gs));
+      }
+    }
+  };
+#pragma unroll 1
+  for (int c0 = 0; c0 < BNT; c0 += CW) {
+    float v[CW];
+#pragma unroll
+    for (int h = 0; h < CW; h += 16) {
+      float v16[16];
+      tc::tmem_ld16(tacc + ((uint32_t)(warp * 32) << 16) + (uint32_t)(c0 + h), v16);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) v[h + i] = v16[i];
+    }
+    if (whole) {
+      write(c0, v);
+    } else {
+#pragma unroll
+      for (int i = 0; i < CW; ++i) __stcg(&part[(size_t)(c0 + i) * BM + r], v[i]);
+    }
+  }
+  // accumulator read: hand it back to the MMA warp
+  tc::tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(acce);
+  if (whole) return;
+  __threadfence();
+  __syncwarp();
+  const long long t_first = (long long)t * p.KB;
+  const int c_first = dec::cta_of(t_first, total, p.nctas);
+  const int c_last = dec::cta_of(t_first + p.KB - 1, total, p.nctas);
+  int last = 0;
+  if (lane == 0) {
+    int *ctr = p.counters + (size_t)t * 4 + warp;
+    last = (atomicAdd(ctr, 1) == c_last - c_first);
+    if (last) *ctr = 0;  // ready for the next call
+  }
+  last = __shfl_sync(0xffffffffu, last, 0);
+  if (!last) return;
+  __threadfence();
+#pragma unroll 1
+  for (int c0 = 0; c0 < BNT; c0 += CW) {
+    float x[CW];
+#pragma unroll
+    for (int i = 0; i < CW; ++i) x[i] = 0.f;
+    for (int c = c_first; c <= c_last; ++c) {
+      const float *pc = p.partial + ((size_t)c * 2 + (c == c_first ? 1 : 0)) * BNT * BM + (size_t)c0 * BM + r;
+      float y[CW];
+#pragma unroll
+      for (int i = 0; i < CW; ++i) y[i] = __ldcg(pc + (size_t)i * BM);
+#pragma unroll
+      for (int i = 0; i < CW; ++i) x[i] += y[i];
+    }
+    write(c0, x);
+  }
+}
+
+template <int KIND, int BNT>
+__global__ void __launch_bounds__(THREADS, 1)
+    bs_gemm_kernel(const __grid_constant__ CUtensorMap w_map, const __grid_constant__ CUtensorMap a_map,
+                   const Params p) {
+  using C = Cfg<KIND, BNT>;
+  constexpr int NS = C::NS, ND = C::ND;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t *ctrl = smem + NS * C::STAGE;
+  uint64_t *full = reinterpret_cast<uint64_t *>(ctrl);  // [NS] weights + activations + scales landed
+  uint64_t *sfree = full + NS;                           // [NS] stage consumed by the MMAs
+  uint64_t *accf = sfree + NS;                           // [ND] accumulator complete
+  uint64_t *acce = accf + ND;                            // [ND] accumulator drained
+  long long *s_total = reinterpret_cast<long long *>(acce + ND);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(s_total + 1);
+  int *s_abort = reinterpret_cast<int *>(tmem_slot + 1);
+  int *s_tpre = s_abort + 1;  // [E+1] MoE: prefix of token tiles per expert
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int cta = blockIdx.x;
+
+  if (warp == 0) {
+    int tvalid = 0;
+    if (!p.moe) {
+      tvalid = (p.M + BNT - 1) / BNT;
+    } else if (p.offsets[p.E] >= 0) {
+      int running = 0;
+      for (int e0 = 0; e0 < p.E; e0 += 32) {
+        const int e = e0 + lane;
+        int tiles = 0;
+        if (e < p.E) tiles = (p.offsets[e + 1] - p.offsets[e] + BNT - 1) / BNT;
+        int incl = tiles;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        if (e < p.E) s_tpre[e + 1] = running + incl;
+        running += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      if (lane == 0) s_tpre[0] = 0;
+      tvalid = running;
+    }
+    if (tvalid > p.mtiles) tvalid = p.mtiles;
+    if (lane == 0) {
+      *s_total = (long long)tvalid * p.ntw * p.KB;  // (tile, stage) iterations
+      *s_abort = 0;
+    }
+  }
+  if (tid == 32) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 2);  // weight producer and activation producer
+      mbar_init(&sfree[s], 1);
+    }
+    for (int d = 0; d < ND; ++d) {
+      mbar_init(&accf[d], 1);
+      mbar_init(&acce[d], 4);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const long long total = __shfl_sync(0xffffffffu, *s_total, 0);
+  const long long beg = dec::range_begin(cta, total, p.nctas);
+  const long long end = dec::range_begin(cta + 1, total, p.nctas);
+  if (beg >= end) return;
+
+  auto tile_info = [&](int t) {
+    TileInfo ti;
+    const int slot = t / p.ntw;
+    ti.wt = t - slot * p.ntw;
+    if (!p.moe) {
+      ti.expert = 0;
+      ti.base = slot * BNT;
+      ti.nvalid = min(BNT, p.M - ti.base);
+    } else {
+      int lo = 0, hi = p.E;
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (s_tpre[mid] <= slot) lo = mid;
+        else hi = mid;
+      }
+      ti.expert = lo;
+      ti.base = p.offsets[lo] + (slot - s_tpre[lo]) * BNT;
+      ti.nvalid = min(BNT, p.offsets[lo + 1] - ti.base);
+    }
+    return ti;
+  };
+
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = __shfl_sync(0xffffffffu, *tmem_slot, 0);
+  const int chunks_per_tile = p.K / (4 * p.group);  // scale chunks per 128-row weight tile
+
+  if (warp == WARP_W) {
+    // ================= weight producer: codes (3-D TMA) + scale chunks (bulk) =================
+    const uint64_t pol = p.weights_once ? policy_evict_first() : policy_evict_normal();
+    Walk w;
+    w.start(beg, end, p.KB);
+    int cur_t = -1, wrow = 0, expert = 0;
+    const uint8_t *sfsrc = nullptr;
+    for (int is = 0, s = 0, ph = 0; w.left > 0; ++is, w.next(p.KB)) {
+      if (w.t != cur_t) {
+        const TileInfo ti = tile_info(w.t);
+        expert = ti.expert;
+        wrow = ti.wt * BM;
+        sfsrc = p.packed + (size_t)ti.expert * p.stride + p.s_off + (size_t)ti.wt * chunks_per_tile * 512;
+        cur_t = w.t;
+      }
+      if (is >= NS && !mbar_wait(&sfree[s], ph ^ 1)) { *s_abort = 1; break; }
+      if (*(volatile int *)s_abort) break;
+      if (lane == 0) {
+        uint8_t *st = smem + s * C::STAGE;
+        // the transaction count of the expanding (MX) copy is the packed bytes read
+        mbar_arrive_expect_tx(&full[s], (uint32_t)(C::W_GLOBAL + C::SF_CH * 512));
+        // MX: coordinates in 4-bit elements (expanded to bytes in shared memory); NV: bytes
+        const int x = KIND == BS_MX ? w.ks * C::KSTAGE : w.ks * 128;
+        asm volatile(
+            "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint "
+            "[%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(st)),
+            "l"(&w_map), "r"(x), "r"(wrow), "r"(expert), "r"(smem_u32(&full[s])), "l"(pol)
+            : "memory");
+        bulk_g2s(st + C::SFA_OFF, sfsrc + (size_t)w.ks * C::SF_CH * 512, C::SF_CH * 512, &full[s]);
+      }
+      __syncwarp();
+      if (++s == NS) { s = 0; ph ^= 1; }
+    }
+  } else if (warp == WARP_ACT) {
+    // ================= activation producer: codes (2-D TMA) + scale chunks (bulk) =================
+    Walk w;
+    w.start(beg, end, p.KB);
+    int cur_t = -1, base = 0;
+    const uint8_t *sfsrc = nullptr;
+    for (int is = 0, s = 0, ph = 0; w.left > 0; ++is, w.next(p.KB)) {
+      if (w.t != cur_t) {
+        base = tile_info(w.t).base;
+        // scale chunks of this tile's token slot, laid out by bs_sf_tiles_kernel
+        sfsrc = p.a_sf + (size_t)(w.t / p.ntw) * p.KB * (C::SF_CH * 512);
+        cur_t = w.t;
+      }
+      if (is >= NS && !mbar_wait(&sfree[s], ph ^ 1)) { *s_abort = 1; break; }
+      if (*(volatile int *)s_abort) break;
+      if (lane == 0) {
+        uint8_t *st = smem + s * C::STAGE;
+        mbar_arrive_expect_tx(&full[s], (uint32_t)(C::A_SMEM + C::SF_CH * 512));
+        tma_load_2d(st + C::W_SMEM, &a_map, w.ks * 128, base, &full[s]);
+        bulk_g2s(st + C::SFB_OFF, sfsrc + (size_t)w.ks * C::SF_CH * 512, C::SF_CH * 512, &full[s]);
+      }
+      __syncwarp();
+      if (++s == NS) { s = 0; ph ^= 1; }
+    }
+  } else if (warp == WARP_MMA) {
+    // ================= MMA issuer (one elected lane) =================
+    Walk w;
+    w.start(beg, end, p.KB);
+    int q = 0, d = 0, dph = 0;
+    for (int is = 0, s = 0, ph = 0; w.left > 0; ++is, w.next(p.KB)) {
+      if (w.seg_first) {
+        if (q > 0 && ++d == ND) { d = 0; dph ^= 1; }
+        if (q >= ND && !mbar_wait(&acce[d], dph ^ 1)) { *s_abort = 1; break; }
+        ++q;
+      }
+      if (!mbar_wait(&full[s], ph)) { *s_abort = 1; break; }
+      if (*(volatile int *)s_abort) break;
+      tc::tc_fence_after();
+      const uint32_t st = smem_u32(smem + s * C::STAGE);
+      const uint64_t adesc = tc::sw128_desc(st);
+      const uint64_t bdesc = tc::sw128_desc(st + C::W_SMEM);
+      const uint32_t tmem_d = tmem + (uint32_t)(d * BNT);
+      const uint32_t acc0 = w.seg_first ? 0u : 1u;
+      if (dec::elect_one()) {
+        // scale chunks -> TMEM; the copies and the MMAs below execute in issue
+        // order, so the previous stage's MMAs have read the old scales
+#pragma unroll
+        for (int c = 0; c < C::SF_CH; ++c) {
+          sf_copy(tmem + (uint32_t)(SFA_COL + 4 * c), sf_desc(st + C::SFA_OFF + c * 512));
+          sf_copy(tmem + (uint32_t)(SFB_COL + 4 * c), sf_desc(st + C::SFB_OFF + c * 512));
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          // MX: one scale per 32 k = byte j of the chunk's column; NV: chunk j, all 4 bytes
+          const uint32_t sf_id = KIND == BS_MX ? (uint32_t)j : 0u;
+          const uint32_t col = KIND == BS_MX ? 0u : (uint32_t)(4 * j);
+          mma_bs<KIND>(tmem_d, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(2 * j), idesc_bs<KIND, BNT>(sf_id),
+                       (tmem + SFA_COL + col) | (sf_id << 30), (tmem + SFB_COL + col) | (sf_id << 30),
+                       j > 0 ? 1u : acc0);
+        }
+        tc::mma_commit(&sfree[s]);
+        if (w.seg_last) tc::mma_commit(&accf[d]);
+      }
+      __syncwarp();
+      if (++s == NS) { s = 0; ph ^= 1; }
+    }
+  } else if (warp < 4) {
+    // ================= epilogue: warps 0..3, thread = weight row =================
+    int t = (int)(beg / p.KB);
+    int ks0 = (int)(beg - (long long)t * p.KB);
+    int left = (int)(end - beg);
+    for (int d = 0, dph = 0; left > 0;) {
+      const int seg_len = min(p.KB - ks0, left);
+      const bool whole = (ks0 == 0) && (seg_len == p.KB);
+      const bool ok = mbar_wait(&accf[d], dph);
+      tc::tc_fence_after();
+      if (!ok || *(volatile int *)s_abort) break;
+      const TileInfo ti = tile_info(t);
+      float gs = 1.f;
+      if (KIND == BS_NV) {
+        gs = reinterpret_cast<const float *>(p.packed + (size_t)ti.expert * p.stride + p.g_off)[0];
+        if (p.a_global) gs = __fmul_rn(gs, *p.a_global);
+      }
+      epilogue_segment<BNT>(p, ti, t, whole, ks0 > 0, tmem + (uint32_t)(d * BNT), &acce[d], gs, cta, warp, lane,
+                            total);
+      left -= seg_len;
+      ++t;
+      ks0 = 0;
+      if (++d == ND) { d = 0; dph ^= 1; }
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc::tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+  }
+}
+
+// Activation scales in the order the block-scaled kernel copies them: for
+// token slot q, stage ks and chunk c, 512 bytes with 4 scales of each of the
+// slot's rows n at (n % 32) * 16 + (n / 32) * 4 (rows past the slot's valid
+// rows, and n >= bnt, are zero).  Dense: slot q = rows [q * bnt, q * bnt +
+// bnt) of the activations.  MoE: slots enumerate the experts' token tiles in
+// expert order (rows offsets[e] + i * bnt, ...) and expert-sorted row r reads
+// caller row perm[r] / div.  One thread per 4-byte word.
+__global__ void bs_sf_tiles_kernel(int slots, int bnt, int kst, int sf_ch, int ld, const uint8_t *__restrict__ sf,
+                                   int M, int moe, int E, const int32_t *__restrict__ offsets,
+                                   const int32_t *__restrict__ perm, int div, uint32_t *__restrict__ out) {
+  extern __shared__ int tpre[];  // [E + 1] MoE: prefix of token tiles per expert
+  bool routed_ok = true;
+  if (moe) {
+    routed_ok = offsets[E] >= 0;
+    if (threadIdx.x < 32) {
+      const int lane = threadIdx.x;
+      int running = 0;
+      for (int e0 = 0; e0 < E; e0 += 32) {
+        const int e = e0 + lane;
+        int tiles = 0;
+        if (e < E && routed_ok) tiles = (offsets[e + 1] - offsets[e] + bnt - 1) / bnt;
+        int incl = tiles;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        if (e < E) tpre[e + 1] = running + incl;
+        running += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      if (lane == 0) tpre[0] = 0;
+    }
+    __syncthreads();
+  }
+  const size_t total = (size_t)slots * kst * sf_ch * 128;
+  for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < total;
+       idx += (size_t)gridDim.x * blockDim.x) {
+    const int n = (int)(idx & 127);
+    const size_t rest = idx >> 7;
+    const int c = (int)(rest % sf_ch);
+    const size_t rest2 = rest / sf_ch;
+    const int ks = (int)(rest2 % kst);
+    const int q = (int)(rest2 / kst);
+    uint32_t v = 0;
+    if (n < bnt) {
+      int src = -1;
+      if (!moe) {
+        const int row = q * bnt + n;
+        if (row < M) src = row;
+      } else if (routed_ok && q < tpre[E]) {
+        int lo = 0, hi = E;  // largest e with tpre[e] <= q
+        while (hi - lo > 1) {
+          const int mid = (lo + hi) >> 1;
+          if (tpre[mid] <= q) lo = mid;
+          else hi = mid;
+        }
+        const int row = offsets[lo] + (q - tpre[lo]) * bnt + n;
+        if (row < offsets[lo + 1]) src = perm[row] / div;
+      }
+      if (src >= 0) v = *reinterpret_cast<const uint32_t *>(sf + (size_t)src * ld + ((size_t)ks * sf_ch + c) * 4);
+    }
+    out[(((size_t)q * kst + ks) * sf_ch + c) * 128 + (n & 31) * 4 + (n >> 5)] = v;
+  }
+}
+
+}  // namespace bs
+
+// ---- host side -------------------------------------------------------------------
+
+// Weight codes of all experts: rows NT*128 per expert, experts `stride` bytes
+// apart.  MX: 4-bit elements expanded to one byte each in shared memory
+// (box 128 codes x 128 rows); NV: packed bytes (box 128 bytes x 128 rows).
+static bool make_bs_weight_map(CUtensorMap *m, const Layout &L, const void *packed, int E) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const bool mx = L.bs == BS_MX;
+  cuuint64_t dims[3] = {(cuuint64_t)(mx ? L.K : L.K / 2), (cuuint64_t)L.NT * TILE_N, (cuuint64_t)E};
+  cuuint64_t strides[2] = {(cuuint64_t)(L.K / 2), (cuuint64_t)L.stride};
+  cuuint32_t box[3] = {128u, 128u, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUresult r = fn(m, mx ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B : CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
+                        const_cast<uint8_t *>((const uint8_t *)packed + L.w_off), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Activation codes [rows][row_bytes] (E4M3 bytes or packed E2M1), box 128 bytes x bnt rows.
+static bool make_bs_act_map(CUtensorMap *m, const void *a, int rows, int row_bytes, int bnt) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+  cuuint32_t box[2] = {128u, (cuuint32_t)bnt};
+  cuuint32_t estr[2] = {1u, 1u};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(a), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int KIND, int BNT>
+static hq_status bs_launch_one(const CUtensorMap &wm, const CUtensorMap &am, const tc::Params &p, const TcLaunch &t,
+                               cudaStream_t st) {
+  using C = bs::Cfg<KIND, BNT>;
+  auto kern = bs::bs_gemm_kernel<KIND, BNT>;
+  static unsigned configured = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return HQ_ERR_CUDA;
+  if (dev >= 32 || !(configured & (1u << dev))) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::BYTES) != cudaSuccess)
+      return HQ_ERR_CUDA;
+    if (dev < 32) configured |= 1u << dev;
+  }
+  kern<<<t.nctas, bs::THREADS, C::BYTES, st>>>(wm, am, p);
+  return check_launch();
+}
+
+template <int KIND>
+static hq_status bs_launch_kind(const CUtensorMap &wm, const CUtensorMap &am, const tc::Params &p,
+                                const TcLaunch &t, cudaStream_t st) {
+  switch (t.bnt) {
+    case 16: return bs_launch_one<KIND, 16>(wm, am, p, t, st);
+    case 32: return bs_launch_one<KIND, 32>(wm, am, p, t, st);
+    case 64: return bs_launch_one<KIND, 64>(wm, am, p, t, st);
+    default: return bs_launch_one<KIND, 128>(wm, am, p, t, st);
+  }
+}
+
+size_t bs_sf_tiles_bytes(const Layout &L, const TcLaunch &t) {
+  if (L.bs == BS_NONE) return 0;
+  const int kstage = L.bs == BS_MX ? 128 : 256;
+  const int sf_ch = L.bs == BS_MX ? 1 : 4;
+  return (size_t)t.mtiles * (L.K / kstage) * sf_ch * 512;
+}
+
+// a_codes: `a_rows` activation rows (MXFP8: K E4M3 bytes per row; NVFP4: K/2
+// packed bytes) in the order the tiles read them: dense rows of a, or MoE
+// expert-sorted rows.  a_scales: the caller's scale rows (MXFP8: K/32 E8M0,
+// NVFP4: K/16 UE4M3 per row), read through perm / div for MoE.  Outputs go to
+// row perm[r] for MoE.  sf_tiles: bs_sf_tiles_bytes() of scratch.
+hq_status launch_bs_gemm(const Layout &L, const void *packed, int E, const void *a_codes, int a_rows,
+                         const void *a_scales, int a_div, const float *a_global, int M, int moe,
+                         const int32_t *offsets, const int32_t *perm, void *out, const TcLaunch &t,
+                         void *workspace, void *sf_tiles, cudaStream_t st) {
+  if (L.bs == BS_NONE || t.kind != 2) return HQ_ERR_UNSUPPORTED;
+  if (((uintptr_t)packed & 31) != 0 || ((uintptr_t)a_scales & 3) != 0) return HQ_ERR_INVALID_ARG;
+  const int kstage = L.bs == BS_MX ? 128 : 256;
+  const int sf_ch = L.bs == BS_MX ? 1 : 4;
+  const int row_bytes = L.bs == BS_MX ? L.K : L.K / 2;
+  CUtensorMap wm, am;
+  if (!make_bs_weight_map(&wm, L, packed, E)) return HQ_ERR_CUDA;
+  if (!make_bs_act_map(&am, a_codes, a_rows, row_bytes, t.bnt)) return HQ_ERR_CUDA;
+  {
+    const size_t words = (size_t)t.mtiles * (L.K / kstage) * sf_ch * 128;
+    size_t blocks = (words + 255) / 256;
+    if (blocks > 148 * 8) blocks = 148 * 8;
+    bs::bs_sf_tiles_kernel<<<(int)blocks, 256, moe ? (E + 1) * sizeof(int) : 0, st>>>(
+        t.mtiles, t.bnt, L.K / kstage, sf_ch, L.K / L.group, (const uint8_t *)a_scales, M, moe, E, offsets, perm,
+        a_div, (uint32_t *)sf_tiles);
+    const hq_status s = check_launch();
+    if (s != HQ_OK) return s;
+  }
+  tc::Params p{};
+  p.packed = (const uint8_t *)packed;
+  p.stride = L.stride;
+  p.w_off = L.w_off; p.s_off = L.s_off; p.z_off = L.z_off; p.c_off = L.c_off; p.g_off = L.g_off;
+  p.N = L.N; p.K = L.K; p.NT = L.NT; p.G = L.G; p.group = L.group;
+  p.KB = L.K / kstage;  // iterations (stages) per tile
+  p.a_global = a_global;
+  p.M = M;
+  p.moe = moe;
+  p.E = E;
+  p.offsets = offsets;
+  p.perm = perm;
+  p.a_div = 1;
+  p.out = (uint16_t *)out;
+  p.ntw = t.ntw;
+  p.mtiles = t.mtiles;
+  p.nctas = t.nctas;
+  p.weights_once = (!moe && t.mtiles == 1) ? 1 : 0;
+  p.a_sf = (const uint8_t *)sf_tiles;
+  p.a_sf_ld = 0;
+  p.a_rows = a_rows;
+  p.counters = (int *)workspace;
+  p.partial = (float *)((uint8_t *)workspace + tc_counter_bytes(t));
+  if (L.bs == BS_MX) return bs_launch_kind<BS_MX>(wm, am, p, t, st);
+  return bs_launch_kind<BS_NV>(wm, am, p, t, st);
+}
+
+}  // namespace hq

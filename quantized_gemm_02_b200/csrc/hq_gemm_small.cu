@@ -212,6 +212,73 @@ __device__ __forceinline__ void decode_bf16(const uint8_t *wpk, const uint8_t *s
   }
 }
 
+// One epilogue warp's end of a segment (Stream-K piece of a tile): v[m] is
+// the fp32 accumulator of weight row n for the tile's token m.  A whole tile
+// is scaled and written as bf16; a piece is stored as an fp32 partial
+// (slot 0 for a head piece that starts mid-tile, else slot 1) and the warp
+// takes its ticket for the tile: the last of the CTAs sharing the tile sums
+// every part in k order and writes the rows.  `ki` = iterations per tile,
+// `total` = iterations of the launch.
+template <int BNT>
+__device__ __forceinline__ void store_rows(const Params &p, const TileInfo &ti, int n, const float (&x)[BNT],
+                                           float cs, float gs) {
+  if (n >= p.N) return;
+#pragma unroll
+  for (int m = 0; m < BNT; ++m) {
+    if (m < ti.nvalid) {
+      const int pos = ti.base + m;
+      const int orow = p.moe ? p.perm[pos] : pos;
+      float z = x[m];
+      if (p.row_scale) z *= p.row_scale[p.moe ? orow / p.a_div : pos];
+      z *= cs;
+      z *= gs;
+      p.out[(size_t)orow * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(z));
+    }
+  }
+}
+
+template <int BNT>
+__device__ __forceinline__ void finish_segment(const Params &p, const TileInfo &ti, int t, bool whole, bool head,
+                                               const float (&v)[BNT], float cs, float gs, int cta, int warp,
+                                               int lane, long long total, int ki) {
+  const int r = warp * 32 + lane;
+  const int n = ti.wt * BM + r;
+  if (whole) {
+    store_rows<BNT>(p, ti, n, v, cs, gs);
+    return;
+  }
+  float *part = p.partial + ((size_t)cta * 2 + (head ? 0 : 1)) * BNT * BM;
+#pragma unroll
+  for (int m = 0; m < BNT; ++m) __stcg(&part[(size_t)m * BM + r], v[m]);
+  __threadfence();
+  __syncwarp();
+  const long long t_first = (long long)t * ki;
+  const int c_first = cta_of(t_first, total, p.nctas);
+  const int c_last = cta_of(t_first + ki - 1, total, p.nctas);
+  int last = 0;
+  if (lane == 0) {
+    int *ctr = p.counters + (size_t)t * 4 + warp;
+    last = (atomicAdd(ctr, 1) == c_last - c_first);
+    if (last) *ctr = 0;  // ready for the next call
+  }
+  last = __shfl_sync(0xffffffffu, last, 0);
+  if (!last) return;
+  __threadfence();
+  // contributors in k order; each one's BNT loads are in flight together
+  float x[BNT];
+#pragma unroll
+  for (int m = 0; m < BNT; ++m) x[m] = 0.f;
+  for (int c = c_first; c <= c_last; ++c) {
+    const float *pc = p.partial + ((size_t)c * 2 + (c == c_first ? 1 : 0)) * BNT * BM + r;
+    float y[BNT];
+#pragma unroll
+    for (int m = 0; m < BNT; ++m) y[m] = __ldcg(pc + (size_t)m * BM);
+#pragma unroll
+    for (int m = 0; m < BNT; ++m) x[m] += y[m];
+  }
+  store_rows<BNT>(p, ti, n, x, cs, gs);
+}
+
 template <int WF, int BNT, bool F8>
 __global__ void __launch_bounds__(THREADS, 1) dec_gemm_kernel(const __grid_constant__ CUtensorMap act_map,
                                                                const Params p) {
@@ -500,9 +567,6 @@ __global__ void __launch_bounds__(THREADS, 1) dec_gemm_kernel(const __grid_const
       if (WF == W_FP8 && n < p.N) cs = reinterpret_cast<const float *>(eb + p.c_off)[n];
       if (WF == W_NVFP4) gs = reinterpret_cast<const float *>(eb + p.g_off)[0];
       if (p.a_global) gs = __fmul_rn(gs, *p.a_global);
-      // a head segment (starts mid-tile) takes partial slot 0, any other slot 1
-      const int pslot = (kb0 > 0) ? 0 : 1;
-      float *part = p.partial + ((size_t)cta * 2 + pslot) * BNT * BM;
       float v[BNT];
 #pragma unroll
       for (int c0 = 0; c0 < BNT; c0 += 16) {
@@ -515,68 +579,7 @@ __global__ void __launch_bounds__(THREADS, 1) dec_gemm_kernel(const __grid_const
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acce[rd.idx]);
-      if (whole) {
-        if (n < p.N) {
-#pragma unroll
-          for (int m = 0; m < BNT; ++m) {
-            if (m < ti.nvalid) {
-              const int pos = ti.base + m;
-              const int orow = p.moe ? p.perm[pos] : pos;
-              float x = v[m];
-              if (p.row_scale) x *= p.row_scale[p.moe ? orow / p.a_div : pos];
-              x *= cs;
-              x *= gs;
-              p.out[(size_t)orow * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(x));
-            }
-          }
-        }
-      } else {
-        // store the partial, take this warp's ticket for the tile; the last of
-        // the CTAs sharing the tile sums every part in k order
-#pragma unroll
-        for (int m = 0; m < BNT; ++m) __stcg(&part[(size_t)m * BM + r], v[m]);
-        __threadfence();
-        __syncwarp();
-        const long long t_first = (long long)t * p.KB;
-        const int c_first = cta_of(t_first, total, p.nctas);
-        const int c_last = cta_of(t_first + p.KB - 1, total, p.nctas);
-        int last = 0;
-        if (lane == 0) {
-          int *ctr = p.counters + (size_t)t * 4 + warp;
-          last = (atomicAdd(ctr, 1) == c_last - c_first);
-          if (last) *ctr = 0;  // ready for the next call
-        }
-        last = __shfl_sync(0xffffffffu, last, 0);
-        if (last) {
-          __threadfence();
-          // contributors in k order; each one's BNT loads are in flight together
-          float x[BNT];
-#pragma unroll
-          for (int m = 0; m < BNT; ++m) x[m] = 0.f;
-          for (int c = c_first; c <= c_last; ++c) {
-            const float *pc = p.partial + ((size_t)c * 2 + (c == c_first ? 1 : 0)) * BNT * BM + r;
-            float y[BNT];
-#pragma unroll
-            for (int m = 0; m < BNT; ++m) y[m] = __ldcg(pc + (size_t)m * BM);
-#pragma unroll
-            for (int m = 0; m < BNT; ++m) x[m] += y[m];
-          }
-          if (n < p.N) {
-#pragma unroll
-            for (int m = 0; m < BNT; ++m) {
-              if (m < ti.nvalid) {
-                const int pos = ti.base + m;
-                const int orow = p.moe ? p.perm[pos] : pos;
-                float z = x[m];
-                if (p.row_scale) z *= p.row_scale[p.moe ? orow / p.a_div : pos];
-                z *= cs;
-                z *= gs;
-                p.out[(size_t)orow * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(z));
-              }
-            }
-          }
-        }
-      }
+      finish_segment<BNT>(p, ti, t, whole, kb0 > 0, v, cs, gs, cta, warp, lane, total, p.KB);
       left -= seg_len;
       ++t;
       kb0 = 0;

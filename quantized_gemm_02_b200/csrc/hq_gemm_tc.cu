@@ -108,6 +108,9 @@ struct Params {
   int nctas;               // persistent CTAs (grid size)
   int weights_once;        // every weight tile is read by one token tile only (stream it past L2)
   int group_slots;         // dense: token tiles per raster group (<= 1: weight tile fastest)
+  const uint8_t *a_sf;     // block-scaled kernel: activation block scales, a_sf_ld bytes per row
+  int a_sf_ld;
+  int a_rows;              // block-scaled kernel: rows of the activation matrix
   float *partial;          // [tiles * S][BNT][128] fp32 split-K partial tiles
   int *counters;           // [ntw * mtiles] per-tile arrival tickets
 };
@@ -798,16 +801,23 @@ static int sm_count() {
 // is expected to hold.  Up to 32 tokens: the decode kernel, one CTA per SM
 // (fewer when there are not 4 k-blocks of work per CTA).  Beyond: two (up to
 // 64 tokens) or one CTA per SM of the multi-stage kernel.
-TcLaunch plan_tc(int rows_per_tile, int mtiles_bound_moe, int N, int KB, bool moe) {
+TcLaunch plan_tc(int rows_per_tile, int mtiles_bound_moe, int N, int KB, bool moe, int bs) {
   TcLaunch t{};
   t.bnt = rows_per_tile <= 16 ? 16 : rows_per_tile <= 32 ? 32 : rows_per_tile <= 64 ? 64 : rows_per_tile <= 128 ? 128 : 256;
   t.kind = t.bnt <= 32 ? 1 : 0;
+  if (bs != BS_NONE) {
+    // block-scaled kernel: up to 128 tokens per tile, one CTA per SM, a
+    // stage is 2 (MX) or 4 (NV) 64-k blocks
+    t.kind = 2;
+    if (t.bnt > 128) t.bnt = 128;
+    KB /= (bs == BS_MX ? 2 : 4);
+  }
   t.ntw = (N + TILE_N - 1) / TILE_N;
   t.mtiles = moe ? mtiles_bound_moe : (rows_per_tile + t.bnt - 1) / t.bnt;
   if (t.mtiles < 1) t.mtiles = 1;
   const long long iters = (long long)t.ntw * t.mtiles * KB;
   const int sms = sm_count();
-  const int slots = t.kind == 1 ? sms : (t.bnt <= 64 ? 2 : 1) * sms;
+  const int slots = t.kind != 0 ? sms : (t.bnt <= 64 ? 2 : 1) * sms;
   long long n = (iters + 3) / 4;
   if (n > slots) n = slots;
   if (n < 1) n = 1;
@@ -817,14 +827,14 @@ TcLaunch plan_tc(int rows_per_tile, int mtiles_bound_moe, int N, int KB, bool mo
 
 size_t tc_counter_bytes(const TcLaunch &t) {
   const size_t tiles = (size_t)t.ntw * t.mtiles;
-  // decode kernel: one ticket per (tile, epilogue warp)
-  return align_up(tiles * (t.kind == 1 ? 4 : 1) * sizeof(int), 256);
+  // decode and block-scaled kernels: one ticket per (tile, epilogue warp)
+  return align_up(tiles * (t.kind != 0 ? 4 : 1) * sizeof(int), 256);
 }
 
 size_t tc_workspace_bytes(const TcLaunch &t) {
   // tile tickets, then the fp32 [bnt][128] partial tiles: one per split
-  // (splits <= CTAs), or a head and a tail slot per CTA in the decode kernel
-  const size_t parts = t.kind == 1 ? (size_t)t.nctas * 2 : (size_t)t.nctas;
+  // (splits <= CTAs), or a head and a tail slot per CTA (Stream-K kernels)
+  const size_t parts = t.kind != 0 ? (size_t)t.nctas * 2 : (size_t)t.nctas;
   return tc_counter_bytes(t) + parts * t.bnt * TILE_N * sizeof(float);
 }
 

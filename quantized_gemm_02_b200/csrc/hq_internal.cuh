@@ -41,8 +41,13 @@ enum AFmt : int { A_BF16 = 0, A_FP8 = 1, A_MXFP8 = 2, A_NVFP4 = 3 };
 constexpr int TILE_N = 128;  // rows of W per tile (the MMA M dimension)
 constexpr int TILE_K = 64;   // k per k-block
 
+// Block-scaled layouts: weights that the tensor core consumes as they are
+// (no dequantisation), with the block scales next to them.
+enum { BS_NONE = 0, BS_MX = 1, BS_NV = 2 };
+
 struct Layout {
   int fmt;
+  int bs;                      // BS_*: block-scaled MMA layout, or the dequantisation layout
   int N, K, NT, KB, G, group;  // group = k per scale group (K for per-channel)
   int wbits;                   // 4 or 8
   int sbytes;                  // bytes per scale element (per-group scales)
@@ -98,9 +103,21 @@ inline bool act_format(const hq_quant_desc *d, int *afmt) {
   }
 }
 
-inline Layout make_layout(int fmt, int group, int N, int K) {
+// Packed layouts.
+//  * Dequantisation layout (bs == BS_NONE): see the unit description above.
+//  * Block-scaled layouts, chosen when the activation format makes the pair
+//    one the tensor core multiplies with block scales itself:
+//      BS_MX  MXFP4 weights x MXFP8 activations (kind::mxf8f6f4, K % 128 == 0)
+//      BS_NV  NVFP4 weights x NVFP4 activations (kind::mxf4nvf4, K % 256 == 0)
+//    codes: row-major [NT*128][K/2] bytes, two E2M1 codes per byte (even k in
+//    the low nibble), rows past N zero; scales: per 128-row tile, chunks of
+//    4 scale columns x 128 rows in the order the tensor-memory copy expects
+//    (row i, scale column j of the chunk at byte (i%32)*16 + (i/32)*4 + j),
+//    [NT][K / (4 * scale group)][512 B]; NVFP4 global scale as fp32.
+inline Layout make_layout(int fmt, int group, int N, int K, int bs = BS_NONE) {
   Layout L{};
   L.fmt = fmt;
+  L.bs = bs;
   L.N = N;
   L.K = K;
   L.NT = (N + TILE_N - 1) / TILE_N;
@@ -114,6 +131,12 @@ inline Layout make_layout(int fmt, int group, int N, int K) {
   L.z_bytes = (fmt == W_UINT4) ? (size_t)L.NT * L.G * TILE_N : 0;
   L.c_bytes = (fmt == W_FP8) ? (size_t)L.NT * TILE_N * 4 : 0;
   L.g_bytes = (fmt == W_NVFP4) ? 16 : 0;
+  if (bs != BS_NONE) {
+    L.w_bytes = (size_t)L.NT * TILE_N * (K / 2);
+    L.s_bytes = (size_t)L.NT * (K / (4 * L.group)) * 512;
+    L.z_bytes = 0;
+    L.c_bytes = 0;
+  }
   size_t off = 0;
   L.w_off = off; off = align_up(off + L.w_bytes, 256);
   L.s_off = off; off = align_up(off + L.s_bytes, 256);
@@ -122,6 +145,18 @@ inline Layout make_layout(int fmt, int group, int N, int K) {
   L.g_off = off; off = align_up(off + L.g_bytes, 256);
   L.stride = off;
   return L;
+}
+
+// The packed layout of a description: block-scaled when the weight and
+// activation formats pair up for a block-scaled MMA and K fits its stage.
+inline Layout layout_for(const hq_quant_desc *d, int fmt, int N, int K) {
+  int afmt = -1;
+  int bs = BS_NONE;
+  if (act_format(d, &afmt)) {
+    if (fmt == W_MXFP4 && afmt == A_MXFP8 && (K % 128) == 0) bs = BS_MX;
+    if (fmt == W_NVFP4 && afmt == A_NVFP4 && (K % 256) == 0) bs = BS_NV;
+  }
+  return make_layout(fmt, d->w_group, N, K, bs);
 }
 
 // Device-side error word (one per device, module scope).  The library is
@@ -243,13 +278,14 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
 
 // Launch plan of the tensor-core GEMM (hq_gemm_tc.cu).
 struct TcLaunch {
-  int kind;    // 0: multi-CTA-per-SM kernel (>= 64 tokens per tile); 1: decode kernel (16 or 32)
+  int kind;    // 0: multi-CTA-per-SM kernel (>= 64 tokens per tile); 1: decode kernel (16 or 32);
+               // 2: block-scaled kernel (16..128)
   int bnt;     // token tile = MMA N (16, 32, 64, 128, 256)
   int ntw;     // 128-row weight tiles
   int mtiles;  // token tiles (dense) or an upper bound on (expert, tile) pairs (MoE)
   int nctas;   // persistent CTAs
 };
-TcLaunch plan_tc(int rows_per_tile, int mtiles_bound_moe, int N, int KB, bool moe);
+TcLaunch plan_tc(int rows_per_tile, int mtiles_bound_moe, int N, int KB, bool moe, int bs = BS_NONE);
 size_t tc_workspace_bytes(const TcLaunch &t);
 // Bytes at the head of the workspace that must be zero before the first
 // call (tile tickets; every call leaves them zero again).

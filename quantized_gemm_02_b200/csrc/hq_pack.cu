@@ -180,6 +180,76 @@ __global__ void unpack_side_kernel(Layout L, int E, const uint8_t *packed, uint8
   }
 }
 
+// ---- block-scaled layouts ----------------------------------------------------------
+// Byte offset of scale column j (0..3 inside its chunk) of tile row i in a
+// 512-byte scale chunk: the row's 32-row group picks the 4-byte column
+// inside the row's 16-byte line, so that one tensor-memory copy of the chunk
+// (32 lanes x 16 bytes, replicated to the four lane quadrants) puts the
+// scales of rows i, i + 32, i + 64, i + 96 in four consecutive columns.
+__host__ __device__ inline uint32_t bs_sf_offset(int i, int j) { return (uint32_t)((i & 31) * 16 + (i >> 5) * 4 + j); }
+
+// Codes: row-major copy with the rows past N zeroed; 16 bytes per thread.
+__global__ void pack_bs_codes_kernel(Layout L, int E, const uint8_t *codes, uint8_t *packed) {
+  const size_t row16 = (size_t)L.K / 32;  // 16-byte pieces per row (K/2 bytes)
+  const size_t rows = (size_t)L.NT * TILE_N;
+  const size_t total = (size_t)E * rows * row16;
+  for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < total;
+       idx += (size_t)gridDim.x * blockDim.x) {
+    const int e = (int)(idx / (rows * row16));
+    const size_t rem = idx % (rows * row16);
+    const int r = (int)(rem / row16);
+    const size_t c = rem % row16;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (r < L.N) v = reinterpret_cast<const uint4 *>(codes + ((size_t)e * L.N + r) * (L.K / 2))[c];
+    reinterpret_cast<uint4 *>(packed + (size_t)e * L.stride + L.w_off + (size_t)r * (L.K / 2))[c] = v;
+  }
+}
+
+// Scales into 512-byte chunks (one thread per scale byte) and the global scale.
+__global__ void pack_bs_side_kernel(Layout L, int E, const uint8_t *scales, const float *global_scale,
+                                    uint8_t *packed) {
+  const int R = L.NT * TILE_N;
+  const size_t total = (size_t)E * R * L.G;
+  for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < total;
+       idx += (size_t)gridDim.x * blockDim.x) {
+    const int e = (int)(idx / ((size_t)R * L.G));
+    const int rem = (int)(idx % ((size_t)R * L.G));
+    const int r = rem / L.G, gi = rem % L.G;
+    const int nt = r / TILE_N, i = r % TILE_N;
+    uint8_t *base = packed + (size_t)e * L.stride;
+    const uint8_t sv = (r < L.N) ? scales[((size_t)e * L.N + r) * L.G + gi] : (uint8_t)0;
+    base[L.s_off + ((size_t)nt * (L.G / 4) + gi / 4) * 512 + bs_sf_offset(i, gi & 3)] = sv;
+    if (L.fmt == W_NVFP4 && r == 0 && gi == 0) reinterpret_cast<float *>(base + L.g_off)[0] = global_scale[e];
+  }
+}
+
+__global__ void unpack_bs_kernel(Layout L, int E, const uint8_t *packed, uint8_t *codes, uint8_t *scales,
+                                 float *global_scale) {
+  const size_t row16 = (size_t)L.K / 32;
+  const size_t total_c = (size_t)E * L.N * row16;
+  const size_t total_s = (size_t)E * L.N * L.G;
+  for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < total_c + total_s;
+       idx += (size_t)gridDim.x * blockDim.x) {
+    if (idx < total_c) {
+      const int e = (int)(idx / ((size_t)L.N * row16));
+      const size_t rem = idx % ((size_t)L.N * row16);
+      const int r = (int)(rem / row16);
+      const size_t c = rem % row16;
+      reinterpret_cast<uint4 *>(codes + ((size_t)e * L.N + r) * (L.K / 2))[c] =
+          reinterpret_cast<const uint4 *>(packed + (size_t)e * L.stride + L.w_off + (size_t)r * (L.K / 2))[c];
+    } else {
+      const size_t j = idx - total_c;
+      const int e = (int)(j / ((size_t)L.N * L.G));
+      const int rem = (int)(j % ((size_t)L.N * L.G));
+      const int r = rem / L.G, gi = rem % L.G;
+      const int nt = r / TILE_N, i = r % TILE_N;
+      const uint8_t *base = packed + (size_t)e * L.stride;
+      scales[j] = base[L.s_off + ((size_t)nt * (L.G / 4) + gi / 4) * 512 + bs_sf_offset(i, gi & 3)];
+      if (L.fmt == W_NVFP4 && r == 0 && gi == 0) global_scale[e] = reinterpret_cast<const float *>(base + L.g_off)[0];
+    }
+  }
+}
+
 static int pack_grid(size_t total, int threads) {
   size_t b = (total + threads - 1) / threads;
   if (b > 148 * 64) b = 148 * 64;
@@ -189,6 +259,14 @@ static int pack_grid(size_t total, int threads) {
 
 hq_status launch_pack(const Layout &L, int E, const void *codes, const void *scales, const void *zeros,
                       const float *global_scale, void *packed, cudaStream_t st) {
+  if (L.bs != BS_NONE) {
+    const size_t n16 = (size_t)E * L.NT * TILE_N * (L.K / 32);
+    pack_bs_codes_kernel<<<pack_grid(n16, 256), 256, 0, st>>>(L, E, (const uint8_t *)codes, (uint8_t *)packed);
+    const size_t ns = (size_t)E * L.NT * TILE_N * L.G;
+    pack_bs_side_kernel<<<pack_grid(ns, 256), 256, 0, st>>>(L, E, (const uint8_t *)scales, global_scale,
+                                                             (uint8_t *)packed);
+    return check_launch();
+  }
   const size_t words = (size_t)E * L.NT * L.KB * (L.unit_bytes() / 4);
   pack_weights_kernel<<<pack_grid(words, 256), 256, 0, st>>>(L, E, (const uint8_t *)codes, (uint8_t *)packed);
   const size_t side = (size_t)E * L.NT * TILE_N * L.G;
@@ -199,6 +277,12 @@ hq_status launch_pack(const Layout &L, int E, const void *codes, const void *sca
 
 hq_status launch_unpack(const Layout &L, int E, const void *packed, void *codes, void *scales, void *zeros,
                         float *global_scale, cudaStream_t st) {
+  if (L.bs != BS_NONE) {
+    const size_t n = (size_t)E * L.N * (L.K / 32) + (size_t)E * L.N * L.G;
+    unpack_bs_kernel<<<pack_grid(n, 256), 256, 0, st>>>(L, E, (const uint8_t *)packed, (uint8_t *)codes,
+                                                         (uint8_t *)scales, global_scale);
+    return check_launch();
+  }
   const int per = (L.fmt == W_FP8) ? 1 : (L.fmt == W_MXFP4 || L.fmt == W_NVFP4) ? 2 : 8;
   const size_t n = (size_t)E * L.N * (L.K / per);
   unpack_codes_kernel<<<pack_grid(n, 256), 256, 0, st>>>(L, E, (const uint8_t *)packed, (uint8_t *)codes);

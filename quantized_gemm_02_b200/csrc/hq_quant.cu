@@ -253,6 +253,20 @@ __global__ void gather_rows_kernel(int R, int K, const uint16_t *__restrict__ a,
   }
 }
 
+// Row gather of raw bytes (quantised codes or scales): out row r = a row
+// idx[r] / div; row_bytes is a multiple of 4.
+__global__ void gather_bytes_kernel(int R, int row_bytes, const uint8_t *__restrict__ a,
+                                    const int32_t *__restrict__ idx, int div, uint8_t *__restrict__ out) {
+  const int per_row = row_bytes / 4;
+  const size_t total = (size_t)R * per_row;
+  for (size_t c = blockIdx.x * (size_t)blockDim.x + threadIdx.x; c < total; c += (size_t)gridDim.x * blockDim.x) {
+    const int r = (int)(c / per_row), ch = (int)(c % per_row);
+    const int src = idx[r] / div;
+    reinterpret_cast<uint32_t *>(out + (size_t)r * row_bytes)[ch] =
+        reinterpret_cast<const uint32_t *>(a + (size_t)src * row_bytes)[ch];
+  }
+}
+
 static int quant_grid(size_t total, int threads) {
   size_t b = (total + threads - 1) / threads;
   if (b > 148 * 16) b = 148 * 16;
@@ -304,6 +318,16 @@ hq_status launch_gather_rows(int R, int K, const void *a, const int32_t *idx, in
   if (R == 0) return HQ_OK;
   const size_t n = (size_t)R * (K / 8);
   gather_rows_kernel<<<quant_grid(n, 256), 256, 0, st>>>(R, K, (const uint16_t *)a, idx, div, (uint16_t *)out);
+  return check_launch();
+}
+
+hq_status launch_gather_bytes(int R, int row_bytes, const void *a, const int32_t *idx, int div, void *out,
+                              cudaStream_t st) {
+  if (R == 0) return HQ_OK;
+  if (row_bytes % 4) return HQ_ERR_INVALID_ARG;
+  const size_t n = (size_t)R * (row_bytes / 4);
+  gather_bytes_kernel<<<quant_grid(n, 256), 256, 0, st>>>(R, row_bytes, (const uint8_t *)a, idx, div,
+                                                           (uint8_t *)out);
   return check_launch();
 }
 

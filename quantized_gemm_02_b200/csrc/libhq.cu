@@ -4,6 +4,7 @@
 #include "hq_pack.cu"
 #include "hq_gemm_tc.cu"
 #include "hq_gemm_small.cu"
+#include "hq_gemm_bs.cu"
 #include "hq_moe.cu"
 #include "hq_api.cu"
 #include "hq_noalloc.cu"

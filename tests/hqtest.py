@@ -86,9 +86,12 @@ def oracle_decoder(wname: str, w: dict, N: int, K: int):
     return dec
 
 
-def gpu_pack(wname: str, w: dict, E: int, N: int, K: int):
+def gpu_pack(wname: str, w: dict, E: int, N: int, K: int, aname: str = "bf16"):
+    """Packs for the description the GEMM will use: the packed layout depends
+    on the activation format (block-scaled layouts for MXFP4 x MXFP8 and
+    NVFP4 x NVFP4)."""
     import quantized_gemm_02_b200 as hq
-    d = cdesc(wname)
+    d = cdesc(wname, aname)
     nbytes = hq.hq_packed_weights_bytes(d, E, N, K)
     assert nbytes > 0
     packed = torch.empty(nbytes, dtype=torch.uint8, device="cuda")

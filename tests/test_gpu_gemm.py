@@ -30,7 +30,7 @@ def parity(wname, aname, M, N, K, seed=0, cols=None, rows=None):
     """Runs one GEMM on the GPU and checks it against the oracle (optionally on
     sampled output columns / rows).  Returns the max err/bound ratio."""
     w = make_weights(wname, 1, N, K, seed=seed)
-    packed = gpu_pack(wname, w, 1, N, K)
+    packed = gpu_pack(wname, w, 1, N, K, aname)
     x = synth.bf16_normal((M, K), synth.generator(seed + 1))
     xb = np_bits(x)
     if aname == "bf16":
@@ -102,7 +102,7 @@ def test_config5_quantised_weights(aname):
     assert np.array_equal(wc.cpu().numpy(), q)
     wname = "nvfp4" if aname == "nvfp4" else "fp8"
     w = {"codes": wc[None], "scales": ws[None], "zeros": None, "global": (wg if aname == "nvfp4" else None)}
-    packed = gpu_pack(wname, w, 1, N, K)
+    packed = gpu_pack(wname, w, 1, N, K, aname)
     ac, asc, ag = gpu_quant(aname, x.cuda())
     c = run_gemm(wname, aname, packed, M, N, K, ac, asc, ag if aname == "nvfp4" else None)
     torch.cuda.synchronize()

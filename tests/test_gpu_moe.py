@@ -61,7 +61,7 @@ def moe_case(wname, aname, T, E, k, N, K, a_per_slot, seed, zipf=False, device_w
     x = synth.bf16_normal((T * k if a_per_slot else T, K), g)
     ids, wts = synth.routing_zipf(T, E, k, 1.2, g) if zipf else synth.routing_softmax_topk(T, E, k, g)
     w = make_weights(wname, E, N, K, seed=seed + 1, device="cuda" if device_weights else "cpu")
-    packed = gpu_pack(wname, w, E, N, K)
+    packed = gpu_pack(wname, w, E, N, K, aname)
     off, perm, inv = gpu_permute(ids.cuda(), E)
     res = {}
     for mode in (0, 1):

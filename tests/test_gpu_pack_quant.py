@@ -27,6 +27,31 @@ def test_pack_unpack_identity(wname):
         assert np.array_equal(np_bits(out[k]), np_bits(v)), k
 
 
+@pytest.mark.parametrize("wname,aname", [("mxfp4", "mxfp8"), ("nvfp4", "nvfp4")])
+def test_pack_unpack_identity_block_scaled(wname, aname):
+    # block-scaled layouts (chosen by the activation format): codes row-major,
+    # scales in 512-byte chunks
+    import quantized_gemm_02_b200 as hq
+    E, N, K = 2, 80, 512
+    w = make_weights(wname, E, N, K, seed=5)
+    packed = gpu_pack(wname, w, E, N, K, aname)
+    out = {k: (None if v is None else torch.empty_like(v, device="cuda")) for k, v in w.items()}
+    hq.hq_unpack_weights(cdesc(wname, aname), E, N, K, packed, out["codes"], out["scales"], out["zeros"],
+                         out["global"])
+    torch.cuda.synchronize()
+    for k, v in w.items():
+        if v is None:
+            continue
+        assert np.array_equal(np_bits(out[k]), np_bits(v)), k
+    # the codes sit row-major (two per byte, even k low), padded rows zero
+    d = cdesc(wname, aname)
+    per_e = hq.hq_packed_weights_bytes(d, 1, N, K)
+    p0 = packed[:per_e].cpu().numpy()
+    codes = w["codes"][0].numpy() if hasattr(w["codes"], "numpy") else w["codes"][0].cpu().numpy()
+    assert np.array_equal(p0[: N * K // 2].reshape(N, K // 2), codes.reshape(N, K // 2))
+    assert not p0[N * K // 2: 128 * K // 2].any()
+
+
 def test_pack_is_deterministic_and_pads_with_zero():
     E, N, K = 1, 70, 128
     w = make_weights("int4_g128", E, N, K, seed=4)

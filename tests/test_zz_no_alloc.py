@@ -34,13 +34,14 @@ def _reference_and_bound(wname, aname, w, x, M, N, K):
 
 @pytest.mark.parametrize("wname,aname,M,N,K", [
     ("mxfp4", "bf16", 4, 512, 8192),        # split-K: tile counters at the head of the scratch
-    ("nvfp4", "nvfp4", 24, 320, 1024),      # quantised activations: decoded copy in the scratch
+    ("nvfp4", "nvfp4", 24, 320, 1024),      # block-scaled MMA, Stream-K tickets in the scratch
+    ("nvfp4", "fp8", 24, 320, 1024),        # quantised activations: decoded copy in the scratch
     ("uint4_g128", "bf16", 40, 200, 2048),  # several token tiles
 ])
 def test_noalloc_matches_hq_gemm_twice(wname, aname, M, N, K):
     import quantized_gemm_02_b200 as hq
     w = make_weights(wname, 1, N, K, seed=M + N)
-    packed = gpu_pack(wname, w, 1, N, K)
+    packed = gpu_pack(wname, w, 1, N, K, aname)
     x = synth.bf16_normal((M, K), synth.generator(M))
     d = cdesc(wname, aname)
     if aname == "bf16":
@@ -71,8 +72,9 @@ def test_noalloc_matches_hq_gemm_twice(wname, aname, M, N, K):
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
     import quantized_gemm_02_b200 as hq
-    # NVFP4 activations need a decoded bf16 copy of A: 4096 x 16384 x 2 B = 128 MiB > 64 MiB
-    d = cdesc("nvfp4", "nvfp4")
+    # FP8 activations with NVFP4 weights need a decoded bf16 copy of A:
+    # 4096 x 16384 x 2 B = 128 MiB > 64 MiB
+    d = cdesc("nvfp4", "fp8")
     assert hq.hq_gemm_workspace_bytes(d, 4096, 256, 16384) > (64 << 20)
     with pytest.raises(hq.HQError) as e:
         hq.hq_gemm_noalloc(d, 4096, 256, 16384, 16, 16, 16, 16, 16)
