@@ -415,10 +415,9 @@ def workload_moe_nvfp4(hq, gen_seed=0):
     return ops, cfg, [w]
 
 
-def workload_dense_quantised(hq, fmt, gen_seed=0):
+def workload_dense_quantised(hq, fmt, gen_seed=0, N=7168, K=7168, Ms=(1, 32, 256, 2048, 8192)):
     """Config 5 dense: N = K = 7168, both operands N(0,1) quantised by the
     library's own quantiser (weights per output row), M swept."""
-    N = K = 7168
     dev = "cuda"
     gen = synth.generator(gen_seed, dev)
     if fmt == "nvfp4":
@@ -447,7 +446,7 @@ def workload_dense_quantised(hq, fmt, gen_seed=0):
     hq.hq_pack_weights(d, 1, N, K, wc, wsc, None, wg if fmt == "nvfp4" else None, packed)
     ops = []
     keep = [packed]
-    for M in [1, 32, 256, 2048, 8192]:
+    for M in Ms:
         x = synth.bf16_normal((M, K), gen, device=dev)
         c, s, g, wq2 = quant(x)
         C = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
@@ -469,7 +468,7 @@ def workload_dense_quantised(hq, fmt, gen_seed=0):
         ops.append(Op(f"{fmt}_N{N}_K{K}_M{M}", run, 2.0 * M * N * K, wbytes, M * K * 2 + M * N * 2, kern,
                       M * K * 2, M * N * 2, e2e))
     cfg = {"workload": f"dense {'W4A4 NVFP4 x NVFP4' if fmt == 'nvfp4' else 'W8A8 FP8 per-channel x per-token'}, "
-                       "N=K=7168, M in {1,32,256,2048,8192}, activation quantisation inside the step",
+                       f"N={N}, K={K}, M in {{{','.join(str(m) for m in Ms)}}}, activation quantisation inside the step",
            "l2": "flushed before every call"}
     return ops, cfg, keep
 
@@ -583,7 +582,10 @@ def main():
     ap.add_argument("--impl", default="hq", choices=["hq", "reference"])
     ap.add_argument("--workload", default="w4a16_asym_sweep", choices=list(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--shape", default=None, help="M,N,K: one dense W4A16 GEMM instead of a workload")
+    ap.add_argument("--eager", action="store_true", help="time plain calls instead of replayed CUDA graphs")
+    ap.add_argument("--shape", default=None, help="M,N,K: one dense GEMM instead of a workload")
+    ap.add_argument("--shape-fmt", default="uint4", choices=["uint4", "nvfp4", "fp8"],
+                    help="--shape weights: W4A16 UINT4 asym g128, or NVFP4 x NVFP4 / FP8 x FP8 quantised in the step")
     args = ap.parse_args()
     ws, rank, local = init_dist()
     if args.impl == "reference":
@@ -593,7 +595,10 @@ def main():
     peaks = load_peaks()
     if args.shape:
         M, N, K = (int(x) for x in args.shape.split(","))
-        ops, cfg, keep = workload_shape(hq, M, N, K)
+        if args.shape_fmt == "uint4":
+            ops, cfg, keep = workload_shape(hq, M, N, K)
+        else:
+            ops, cfg, keep = workload_dense_quantised(hq, args.shape_fmt, N=N, K=K, Ms=(M,))
     else:
         ops, cfg, keep = WORKLOADS[args.workload](hq)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
@@ -601,13 +606,40 @@ def main():
     n_ops = len(ops)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in ops]
 
+    # Each device-resident call is captured once in a CUDA graph and replayed,
+    # as a serving loop would, so that the timed region holds the GPU work and
+    # not the Python launch path; --eager times the plain calls instead.
+    graphs = [None] * n_ops
+    if not args.eager:
+        try:
+            for op in ops:  # first calls (per-device kernel attributes) happen outside capture
+                op.run()
+            torch.cuda.synchronize()
+            for i, op in enumerate(ops):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    op.run()
+                graphs[i] = g
+            torch.cuda.synchronize()
+            cfg["launch"] = "one CUDA graph per call, replayed"
+        except Exception as exc:  # capture unsupported: fall back to eager calls
+            graphs = [None] * n_ops
+            cfg["launch"] = "eager (graph capture failed: %s)" % type(exc).__name__
+    else:
+        cfg["launch"] = "eager"
+
     def one_step(timed: bool, e2e: bool = False):
         times = []
         for i, op in enumerate(ops):
             flush.zero_()
             a, b = ev[i]
             a.record(stream)
-            (op.e2e if e2e else op.run)()
+            if e2e:
+                op.e2e()
+            elif graphs[i] is not None:
+                graphs[i].replay()
+            else:
+                op.run()
             b.record(stream)
         torch.cuda.synchronize()
         for a, b in ev:

@@ -206,16 +206,28 @@ __device__ __forceinline__ void epilogue_segment(const Params &p, const TileInfo
   __threadfence();
 #pragma unroll 1
   for (int c0 = 0; c0 < BNT; c0 += CW) {
+    // contributors in k order; the loads of U contributors are in flight together
+    constexpr int U = CW <= 16 ? 4 : 2;
     float x[CW];
 #pragma unroll
     for (int i = 0; i < CW; ++i) x[i] = 0.f;
-    for (int c = c_first; c <= c_last; ++c) {
-      const float *pc = p.partial + ((size_t)c * 2 + (c == c_first ? 1 : 0)) * BNT * BM + (size_t)c0 * BM + r;
-      float y[CW];
+    for (int cb = c_first; cb <= c_last; cb += U) {
+      float y[U][CW];
 #pragma unroll
-      for (int i = 0; i < CW; ++i) y[i] = __ldcg(pc + (size_t)i * BM);
+      for (int u = 0; u < U; ++u) {
+        const int c = cb + u;
+        if (c <= c_last) {
+          const float *pc = p.partial + ((size_t)c * 2 + (c == c_first ? 1 : 0)) * BNT * BM + (size_t)c0 * BM + r;
 #pragma unroll
-      for (int i = 0; i < CW; ++i) x[i] += y[i];
+          for (int i = 0; i < CW; ++i) y[u][i] = __ldcg(pc + (size_t)i * BM);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (cb + u <= c_last) {
+#pragma unroll
+          for (int i = 0; i < CW; ++i) x[i] += y[u][i];
+        }
     }
     write(c0, x);
   }
@@ -309,15 +321,24 @@ __global__ void __launch_bounds__(THREADS, 1)
     return ti;
   };
 
-  if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                 "r"(TMEM_COLS));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  // The producer warps start loading at once; the warps that use tensor
+  // memory wait (named barrier 1) for warp 0's allocation.
+  const bool producer = (warp == WARP_W || warp == WARP_ACT);
+  uint32_t tmem = 0;
+  if (producer) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&w_map) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&a_map) : "memory");
+  } else {
+    if (warp == 0) {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                   "r"(TMEM_COLS));
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc::tc_fence_before();
+    asm volatile("bar.sync 1, %0;" ::"r"(THREADS - 64) : "memory");
+    tc::tc_fence_after();
+    tmem = __shfl_sync(0xffffffffu, *tmem_slot, 0);
   }
-  tc::tc_fence_before();
-  __syncthreads();
-  tc::tc_fence_after();
-  const uint32_t tmem = __shfl_sync(0xffffffffu, *tmem_slot, 0);
   const int chunks_per_tile = p.K / (4 * p.group);  // scale chunks per 128-row weight tile
 
   if (warp == WARP_W) {

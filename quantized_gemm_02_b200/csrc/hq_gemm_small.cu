@@ -264,17 +264,28 @@ __device__ __forceinline__ void finish_segment(const Params &p, const TileInfo &
   last = __shfl_sync(0xffffffffu, last, 0);
   if (!last) return;
   __threadfence();
-  // contributors in k order; each one's BNT loads are in flight together
+  // contributors in k order; the loads of U contributors are in flight together
+  constexpr int U = BNT <= 16 ? 2 : 1;  // within the 80-register budget of this kernel
   float x[BNT];
 #pragma unroll
   for (int m = 0; m < BNT; ++m) x[m] = 0.f;
-  for (int c = c_first; c <= c_last; ++c) {
-    const float *pc = p.partial + ((size_t)c * 2 + (c == c_first ? 1 : 0)) * BNT * BM + r;
-    float y[BNT];
+  for (int c0 = c_first; c0 <= c_last; c0 += U) {
+    float y[U][BNT];
 #pragma unroll
-    for (int m = 0; m < BNT; ++m) y[m] = __ldcg(pc + (size_t)m * BM);
+    for (int u = 0; u < U; ++u) {
+      const int c = c0 + u;
+      if (c <= c_last) {
+        const float *pc = p.partial + ((size_t)c * 2 + (c == c_first ? 1 : 0)) * BNT * BM + r;
 #pragma unroll
-    for (int m = 0; m < BNT; ++m) x[m] += y[m];
+        for (int m = 0; m < BNT; ++m) y[u][m] = __ldcg(pc + (size_t)m * BM);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (c0 + u <= c_last) {
+#pragma unroll
+        for (int m = 0; m < BNT; ++m) x[m] += y[u][m];
+      }
   }
   store_rows<BNT>(p, ti, n, x, cs, gs);
 }
@@ -379,15 +390,23 @@ __global__ void __launch_bounds__(THREADS, 1) dec_gemm_kernel(const __grid_const
     return ti;
   };
 
-  if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                 "r"(TMEM_COLS));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  // The producer warps start loading at once; the warps that use tensor
+  // memory wait (named barrier 1) for warp 0's allocation.
+  const bool producer = (warp == WARP_PRODUCER || warp == WARP_ACT);
+  uint32_t tmem = 0;
+  if (producer) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&act_map) : "memory");
+  } else {
+    if (warp == 0) {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                   "r"(TMEM_COLS));
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc::tc_fence_before();
+    asm volatile("bar.sync 1, %0;" ::"r"(THREADS - 64) : "memory");
+    tc::tc_fence_after();
+    tmem = __shfl_sync(0xffffffffu, *tmem_slot, 0);
   }
-  tc::tc_fence_before();
-  __syncthreads();
-  tc::tc_fence_after();
-  const uint32_t tmem = __shfl_sync(0xffffffffu, *tmem_slot, 0);
 
   if (warp == WARP_PRODUCER) {
     // ================= weight producer (whole warp in step, lane 0 issues) =================
