@@ -1,6 +1,7 @@
 """Benchmark of the quantised-weight GEMM path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl hq|reference] [--workload NAME]
+                    [--shape M,N,K [--shape-fmt uint4|nvfp4|fp8]] [--eager] [--no-cpu-baseline]
 
 Metric: quantised GEMM TFLOPS (and weight GB/s, % of roofline) versus M.
 Default workload ``w4a16_asym_sweep``: dense W4A16 with UINT4 weights, UINT4
@@ -8,9 +9,15 @@ zero points and bf16 scales per 128-K group, (N, K) in {(8192, 8192),
 (28672, 8192), (8192, 28672)}, M swept over 1, 4, 16, 64, 256, 1024, 4096,
 8192; A bf16 N(0, 1).  One step runs every (shape, M) GEMM once; the L2 is
 flushed (a 512 MiB memset, untimed) before each GEMM and each GEMM is timed
-with CUDA events on its stream.  ``value`` = total flops of a step / summed
-GEMM time.  Other workloads (``--workload``): ``w4a16_dense_m16``,
-``moe_w4a16_mxfp4``, ``moe_w4a8_mxfp8``, ``w4a4_nvfp4``, ``w8a8_fp8``.
+with CUDA events on its stream.  Each call is captured once in a CUDA graph
+and replayed (``--eager`` times the plain calls).  ``value`` = total flops of
+a step / summed GEMM time.  Other workloads (``--workload``):
+``w4a16_dense_m16``, ``moe_w4a16_mxfp4``, ``moe_w4a8_mxfp8``, ``moe_nvfp4``,
+``w4a4_nvfp4``, ``w8a8_fp8``.  The roofline object describes the dominant
+call: HBM-bound calls against the measured copy bandwidth, tensor-bound ones
+against the measured bf16 peak times the nominal ratio of the call's MMA kind
+(FP8 and MXFP8 x FP4 weights 2, FP4 x FP4 4); ``traffic`` is the committed ncu
+DRAM figure when the kernel sources still match it.
 
 Multi-GPU (torchrun): replicas only, every rank runs the same workload on
 its own GPU; the timed region is bracketed by a barrier and a synchronise,
@@ -36,6 +43,15 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 import synth  # noqa: E402
+
+METRIC = "quantized GEMM TFLOPS and weight GB/s vs M (dense+MoE), % of roofline, 1xB200"
+
+# Workload titles shared by the library arm's config and the reference arm's config.
+WORKLOAD_TITLE = {
+    "w4a16_asym_sweep": "dense W4A16 UINT4 asym g128 bf16-scale, (N,K) in {(8192,8192),(28672,8192),(8192,28672)}, "
+                        "M in {1,4,16,64,256,1024,4096,8192}",
+    "w4a16_dense_m16": "dense W4A16 INT4 sym g128, M=16, N=K=4096",
+}
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -165,9 +181,13 @@ class Clocks:
 class Op:
     """One library call of a step, with its algorithmic cost."""
 
-    def __init__(self, name, run, flops, w_bytes, io_bytes, kernels, h2d=None, d2h=None, e2e=None, kernel=None):
+    def __init__(self, name, run, flops, w_bytes, io_bytes, kernels, h2d=None, d2h=None, e2e=None, kernel=None,
+                 peak_ratio=1.0):
         self.name = name
         self.kernel = kernel      # the library kernel that dominates the call
+        # dense tensor peak of the call's MMA kind relative to bf16 (nominal ratios: FP8 and
+        # MXFP8-with-FP4-weights 2, FP4 x FP4 4), applied to the measured bf16 peak
+        self.peak_ratio = peak_ratio
         self.run = run            # device-resident call
         self.flops = flops
         self.w_bytes = w_bytes    # packed weight + scale + zero bytes the call must read
@@ -274,9 +294,7 @@ def workload_w4a16_asym_sweep(hq, gen_seed=0):
         wb = packed_bytes_int4(N, K, 128, True)
         for M in Ms:
             ops.append(dense_op(hq, d, f"N{N}_K{K}_M{M}", M, N, K, packed, wb, gen))
-    cfg = {"workload": "dense W4A16 UINT4 asym g128 bf16-scale, (N,K) in {(8192,8192),(28672,8192),(8192,28672)}, "
-                       "M in {1,4,16,64,256,1024,4096,8192}",
-           "shapes": shapes, "M": Ms, "l2": "flushed before every GEMM (512 MiB memset, untimed)"}
+    cfg = {"workload": WORKLOAD_TITLE["w4a16_asym_sweep"], "shapes": shapes, "M": Ms, "l2": "flushed before every GEMM (512 MiB memset, untimed)"}
     return ops, cfg, keep
 
 
@@ -289,7 +307,7 @@ def workload_w4a16_dense_m16(hq, gen_seed=0):
     packed = torch.empty(hq.hq_packed_weights_bytes(d, 1, N, K), dtype=torch.uint8, device="cuda")
     hq.hq_pack_weights(d, 1, N, K, w["codes"], w["scales"], None, None, packed)
     ops = [dense_op(hq, d, "N4096_K4096_M16", M, N, K, packed, packed_bytes_int4(N, K, 128, False), gen)]
-    cfg = {"workload": "dense W4A16 INT4 sym g128, M=16, N=K=4096", "l2": "flushed before every GEMM"}
+    cfg = {"workload": WORKLOAD_TITLE["w4a16_dense_m16"], "l2": "flushed before every GEMM"}
     return ops, cfg, [packed]
 
 
@@ -375,8 +393,12 @@ def moe_ops(hq, name, wdesc, E, topk, H, I, Ts, routing, gen, mode_names=("group
             # quant + decode + GEMM, or gather + GEMM (bf16); combine
             per_gemm = 4 if block_scaled else (3 if quant else 2)
             kernels = 1 + per_gemm * 2 + 1
+            ratio = 1.0
+            if block_scaled:
+                ratio = 2.0 if wdesc.w_scale_dtype == hq.HQ_E8M0 else 4.0
             ops.append(Op(f"{name}_T{T}_{mode_name}", run, flops, wbytes, io, kernels,
-                          T * topk * 4 + T * Kg * 2, T * Nd * 2, e2e))
+                          T * topk * 4 + T * Kg * 2, T * Nd * 2, e2e,
+                          kernel="bs_gemm_kernel" if block_scaled else "MoE GEMM kernels", peak_ratio=ratio))
     return ops, weights
 
 
@@ -466,7 +488,9 @@ def workload_dense_quantised(hq, fmt, gen_seed=0, N=7168, K=7168, Ms=(1, 32, 256
 
         kern = (2 if fmt == "nvfp4" else 1) + (1 if fmt == "fp8" else 2)
         ops.append(Op(f"{fmt}_N{N}_K{K}_M{M}", run, 2.0 * M * N * K, wbytes, M * K * 2 + M * N * 2, kern,
-                      M * K * 2, M * N * 2, e2e))
+                      M * K * 2, M * N * 2, e2e,
+                      kernel="bs_gemm_kernel" if fmt == "nvfp4" else gemm_kernel_name(M),
+                      peak_ratio=4.0 if fmt == "nvfp4" else 2.0))
     cfg = {"workload": f"dense {'W4A4 NVFP4 x NVFP4' if fmt == 'nvfp4' else 'W8A8 FP8 per-channel x per-token'}, "
                        f"N={N}, K={K}, M in {{{','.join(str(m) for m in Ms)}}}, activation quantisation inside the step",
            "l2": "flushed before every call"}
@@ -562,11 +586,12 @@ def run_reference(args, ws, rank):
         if i >= args.warmup:
             steps.append(cb)
     v = statistics.median([s["value"] for s in steps])
-    line = {"impl": "reference", "metric": "quantized GEMM TFLOPS (CPU fp64 oracle)", "value": v, "unit": "TFLOPS",
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOPS",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": statistics.median([s["seconds"] for s in steps]) * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": args.workload, "sample": cb["sample"]},
+            "config": {"workload": WORKLOAD_TITLE.get(args.workload, args.workload), "sample": cb["sample"],
+                       "note": "CPU fp64 oracle on the host cores, a bounded sample of the workload"},
             "cpu_baseline": {"value": v, "unit": "TFLOPS", "cores": cb["cores"], "kind": "oracle",
                              "sample": cb["sample"]},
             "e2e": {"value": v, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -677,17 +702,19 @@ def main():
     dom = ops[i_dom]
     t_dom = per_op[i_dom] / 1e3
     hbm_t = dom.bytes / (peaks["hbm_gbs"] * 1e9)
-    flop_t = dom.flops / (peaks["bf16_tflops"] * 1e12)
+    peak_fmt = peaks["bf16_tflops"] * dom.peak_ratio
+    flop_t = dom.flops / (peak_fmt * 1e12)
     if flop_t >= hbm_t:
-        roof = {"bound": "tensor", "achieved": dom.flops / t_dom / 1e12, "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s"}
+        roof = {"bound": "tensor", "achieved": dom.flops / t_dom / 1e12, "peak": peak_fmt, "unit": "TFLOP/s"}
     else:
         roof = {"bound": "hbm", "achieved": dom.bytes / t_dom / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = measured_traffic(dom.name)
     roof["algorithmic_bytes"] = dom.bytes
     roof["kernel"] = (dom.kernel or "hq") + " (" + dom.name + ")"
-    roof["peak_source"] = peaks["source"] + (" burst" if roof["bound"] == "tensor" else "")
+    roof["peak_source"] = peaks["source"] + (" burst" if roof["bound"] == "tensor" else "") + (
+        " bf16 x %g (nominal ratio of the MMA kind)" % dom.peak_ratio if roof["bound"] == "tensor" and dom.peak_ratio != 1
+        else "")
 
     sweep = []
     for op, t in zip(ops, per_op):
@@ -695,9 +722,9 @@ def main():
         hb = op.bytes / s / 1e9
         sweep.append({"op": op.name, "us": round(t * 1e3, 2), "tflops": round(op.flops / s / 1e12, 2),
                       "weight_gbs": round(op.w_bytes / s / 1e9, 1), "hbm_frac": round(hb / peaks["hbm_gbs"], 3),
-                      "tensor_frac": round(op.flops / s / 1e12 / peaks["bf16_tflops"], 3)})
+                      "tensor_frac": round(op.flops / s / 1e12 / (peaks["bf16_tflops"] * op.peak_ratio), 3)})
     line = {
-        "metric": "quantized GEMM TFLOPS and weight GB/s vs M (dense+MoE), % of roofline, 1xB200",
+        "metric": METRIC,
         "value": value, "unit": "TFLOPS", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic", "config": cfg,

@@ -120,7 +120,14 @@ HQ_API hq_status hq_device_error(hq_stream_t stream);
  *
  * hq_packed_weights_bytes: size of the opaque packed buffer for E experts of
  *   N x K weights (0 if the description or sizes are unsupported).  N is
- *   padded to 64 rows and K must be a multiple of 64.
+ *   padded to 128 rows and K must be a multiple of 64.
+ * The packed layout depends on the whole description, the activation
+ *   format included: MXFP4 weights with a_dtype MXFP8 (K a multiple of 128)
+ *   and NVFP4 weights with a_dtype NVFP4 (K a multiple of 256) are stored
+ *   for the block-scaled tensor-core MMA (codes as they are, scales in the
+ *   MMA's chunk order); every other pair for in-kernel dequantisation.  Pack,
+ *   unpack, hq_gemm and hq_moe_gemm must be given the same description.
+ *   The packed buffer must be 32-byte aligned (cudaMalloc's 256 is).
  * hq_pack_weights: standard-format codes / scales / zeros (device) and, for
  *   NVFP4, `global_scale` (device fp32 [E]) -> `packed` (device,
  *   hq_packed_weights_bytes).  `zeros` must be NULL unless w_has_zero;
@@ -168,6 +175,10 @@ HQ_API hq_status hq_quant_act(const hq_quant_desc *desc, int M, int K, const voi
  * `workspace` of hq_gemm_workspace_bytes() bytes; its split-K counters must
  * be zero when first used (for example cudaMemset once after allocation);
  * every completed call leaves them zero again.
+ * Block-scaled pairs (MXFP4 x MXFP8, NVFP4 x NVFP4, see hq_pack_weights)
+ * multiply the quantised activations as they are (a_scales 4-byte aligned);
+ * other quantised activations are decoded exactly to bf16 in the workspace
+ * and multiplied with the dequantised weights.
  * ---------------------------------------------------------------------- */
 HQ_API size_t hq_gemm_workspace_bytes(const hq_quant_desc *desc, int M, int N, int K);
 HQ_API hq_status hq_gemm(const hq_quant_desc *desc, int M, int N, int K, const void *packed_w,
