@@ -114,6 +114,14 @@ HQ_API const char *hq_status_string(hq_status s);
  * HQ_ERR_DEVICE_INDEX. */
 HQ_API hq_status hq_device_error(hq_stream_t stream);
 
+/* Diagnostics (no counterpart in the pages): launches one warp that waits
+ * on an mbarrier nothing arrives on, with the same bounded wait every GEMM
+ * pipeline uses, limited to `limit_ns` (0 < limit_ns <= 1e9).  The wait
+ * gives up, records HQ_ERR_TIMEOUT in the device error word (read it with
+ * hq_device_error) and the kernel returns; the context stays usable.  This
+ * is how the device-side failure path is tested without faulting a GPU. */
+HQ_API hq_status hq_selftest_wait_timeout(unsigned long long limit_ns, hq_stream_t stream);
+
 /* ------------------------------------------------------------------------
  * Weight repack ("Announcing Humming", section "Tuning & JIT per workload":
  * validate, pad, repack into the kernel layout).

@@ -17,7 +17,7 @@ __all__ = [
     "HQ_NVFP4", "HQ_MOE_GROUPED", "HQ_MOE_INDEXED",
     "hq_status_string", "hq_device_error", "hq_packed_weights_bytes", "hq_pack_weights", "hq_unpack_weights",
     "hq_quant_act", "hq_gemm_workspace_bytes", "hq_gemm", "hq_moe_permute", "hq_moe_workspace_bytes",
-    "hq_moe_gemm", "hq_moe_unpermute_sum", "hq_gemm_noalloc",
+    "hq_moe_gemm", "hq_moe_unpermute_sum", "hq_gemm_noalloc", "hq_selftest_wait_timeout",
 ]
 
 HQ_BF16, HQ_FP32, HQ_INT4, HQ_UINT4, HQ_E2M1, HQ_E4M3, HQ_E8M0, HQ_UE4M3, HQ_MXFP8, HQ_NVFP4 = range(10)
@@ -32,7 +32,7 @@ STATUS = {
 EXPORTS = (
     "hq_status_string", "hq_device_error", "hq_packed_weights_bytes", "hq_pack_weights", "hq_unpack_weights",
     "hq_quant_act", "hq_gemm_workspace_bytes", "hq_gemm", "hq_moe_permute", "hq_moe_workspace_bytes",
-    "hq_moe_gemm", "hq_moe_unpermute_sum", "hq_gemm_noalloc",
+    "hq_moe_gemm", "hq_moe_unpermute_sum", "hq_gemm_noalloc", "hq_selftest_wait_timeout",
 )
 
 
@@ -87,6 +87,7 @@ def _lib() -> ctypes.CDLL:
             "hq_moe_gemm": (I, [I, D, I, I, I, I, I, P, P, I, P, P, P, P, F, I, P, P, Z, P]),
             "hq_moe_unpermute_sum": (I, [I, I, I, P, P, P, F, P, P]),
             "hq_gemm_noalloc": (I, [D, I, I, I, P, P, P, P, P, P]),
+            "hq_selftest_wait_timeout": (I, [ctypes.c_ulonglong, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -192,3 +193,10 @@ def hq_gemm_noalloc(desc, M, N, K, packed_w, a, a_scales, a_global, c, stream=No
     _check("hq_gemm_noalloc", _lib().hq_gemm_noalloc(
         ctypes.byref(desc), M, N, K, _ptr(packed_w), _ptr(a), _ptr(a_scales), _ptr(a_global), _ptr(c),
         _stream(stream)))
+
+
+def hq_selftest_wait_timeout(limit_ns: int, stream=None):
+    """Runs the bounded-wait self-test (a wait nothing satisfies, limited to
+    limit_ns); afterwards hq_device_error() reports HQ_ERR_TIMEOUT."""
+    _check("hq_selftest_wait_timeout", _lib().hq_selftest_wait_timeout(int(limit_ns), _stream(stream)))
+

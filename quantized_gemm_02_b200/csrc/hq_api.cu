@@ -185,6 +185,26 @@ const char *hq_status_string(hq_status s) {
   }
 }
 
+// Self-test of the device-side failure path: one warp waits on an mbarrier
+// that nothing arrives on, with the bounded wait every pipeline uses; the
+// wait gives up after limit_ns, records HQ_ERR_TIMEOUT and the kernel returns.
+__global__ void selftest_wait_kernel(unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  mbar_wait(&bar, 0, limit_ns);  // nothing arrives
+}
+
+hq_status hq_selftest_wait_timeout(unsigned long long limit_ns, hq_stream_t stream) {
+  if (limit_ns == 0 || limit_ns > WAIT_LIMIT_NS) return HQ_ERR_INVALID_ARG;
+  if (!device_is_sm100()) return HQ_ERR_ARCH;
+  selftest_wait_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(limit_ns);
+  return check_launch();
+}
+
 hq_status hq_device_error(hq_stream_t stream) {
   if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return HQ_ERR_CUDA;
   int v = 0, zero = 0;

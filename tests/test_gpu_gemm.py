@@ -72,6 +72,12 @@ def test_gemm_large_token_count():
     parity("uint4_g128", "bf16", 300, 96, 384, seed=5)
 
 
+def test_gemm_many_token_tiles():
+    # 2100 tokens: eleven 256-token tiles (ragged last), grouped raster of token tiles
+    parity("uint4_g128", "bf16", 2100, 136, 256, seed=6)
+    parity("fp8", "fp8", 2100, 136, 256, seed=7)
+
+
 def test_config1_full():
     # Dense W4A16: M=16, N=K=4096, INT4 symmetric, bf16 scales per 128 group
     r = parity("int4_g128", "bf16", 16, 4096, 4096, seed=0)
