@@ -78,6 +78,14 @@ def test_gemm_many_token_tiles():
     parity("fp8", "fp8", 2100, 136, 256, seed=7)
 
 
+@pytest.mark.parametrize("wname,aname", [("mxfp4", "mxfp8"), ("nvfp4", "nvfp4")])
+@pytest.mark.parametrize("M", [129, 300])
+def test_gemm_block_scaled_many_token_tiles(wname, aname, M):
+    # more than 128 tokens: several 128-token tiles of the block-scaled
+    # kernel (scale chunks of each token slot), ragged last tile
+    parity(wname, aname, M, 136, 512, seed=20 + M)
+
+
 def test_config1_full():
     # Dense W4A16: M=16, N=K=4096, INT4 symmetric, bf16 scales per 128 group
     r = parity("int4_g128", "bf16", 16, 4096, 4096, seed=0)
