@@ -489,7 +489,7 @@ def workload_dense_quantised(hq, fmt, gen_seed=0, N=7168, K=7168, Ms=(1, 32, 256
         kern = (2 if fmt == "nvfp4" else 1) + (1 if fmt == "fp8" else 2)
         ops.append(Op(f"{fmt}_N{N}_K{K}_M{M}", run, 2.0 * M * N * K, wbytes, M * K * 2 + M * N * 2, kern,
                       M * K * 2, M * N * 2, e2e,
-                      kernel="bs_gemm_kernel" if fmt == "nvfp4" else gemm_kernel_name(M),
+                      kernel="bs_gemm_kernel",
                       peak_ratio=4.0 if fmt == "nvfp4" else 2.0))
     cfg = {"workload": f"dense {'W4A4 NVFP4 x NVFP4' if fmt == 'nvfp4' else 'W8A8 FP8 per-channel x per-token'}, "
                        f"N={N}, K={K}, M in {{{','.join(str(m) for m in Ms)}}}, activation quantisation inside the step",

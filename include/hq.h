@@ -133,7 +133,9 @@ HQ_API hq_status hq_selftest_wait_timeout(unsigned long long limit_ns, hq_stream
  *   format included: MXFP4 weights with a_dtype MXFP8 (K a multiple of 128)
  *   and NVFP4 weights with a_dtype NVFP4 (K a multiple of 256) are stored
  *   for the block-scaled tensor-core MMA (codes as they are, scales in the
- *   MMA's chunk order); every other pair for in-kernel dequantisation.  Pack,
+ *   MMA's chunk order), FP8 weights with a_dtype E4M3 (K a multiple of 128)
+ *   as row-major E4M3 bytes with per-row fp32 scales for the FP8 MMA; every
+ *   other pair for in-kernel dequantisation.  Pack,
  *   unpack, hq_gemm and hq_moe_gemm must be given the same description.
  *   The packed buffer must be 32-byte aligned (cudaMalloc's 256 is).
  * hq_pack_weights: standard-format codes / scales / zeros (device) and, for
@@ -183,10 +185,12 @@ HQ_API hq_status hq_quant_act(const hq_quant_desc *desc, int M, int K, const voi
  * `workspace` of hq_gemm_workspace_bytes() bytes; its split-K counters must
  * be zero when first used (for example cudaMemset once after allocation);
  * every completed call leaves them zero again.
- * Block-scaled pairs (MXFP4 x MXFP8, NVFP4 x NVFP4, see hq_pack_weights)
- * multiply the quantised activations as they are (a_scales 4-byte aligned);
- * other quantised activations are decoded exactly to bf16 in the workspace
- * and multiplied with the dequantised weights.
+ * Block-scaled pairs (MXFP4 x MXFP8, NVFP4 x NVFP4) and FP8 x E4M3 with K a
+ * multiple of 128 (see hq_pack_weights) multiply the quantised activations
+ * as they are (a_scales 4-byte aligned); other quantised activations are
+ * decoded exactly to bf16 in the workspace and multiplied with the
+ * dequantised weights (FP8 x E4M3 otherwise: E4M3 weights and activations on
+ * the FP8 MMA with the weights staged through tensor memory).
  * ---------------------------------------------------------------------- */
 HQ_API size_t hq_gemm_workspace_bytes(const hq_quant_desc *desc, int M, int N, int K);
 HQ_API hq_status hq_gemm(const hq_quant_desc *desc, int M, int N, int K, const void *packed_w,

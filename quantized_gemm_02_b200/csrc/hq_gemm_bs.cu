@@ -46,12 +46,13 @@ constexpr int TMEM_COLS = 512;
 constexpr int SFA_COL = 256;  // TMEM columns of the weight scales (after two 128-column accumulators)
 constexpr int SFB_COL = 288;  // TMEM columns of the activation scales
 
-// KIND: BS_MX or BS_NV.  A stage is one 128-byte row of each operand: 128 k
-// (MX: E2M1 expanded to bytes / E4M3) or 256 k (NV: packed E2M1), four MMAs.
+// KIND: BS_MX, BS_NV or BS_F8.  A stage is one 128-byte row of each operand:
+// 128 k (MX: E2M1 expanded to bytes / E4M3; F8: E4M3) or 256 k (NV: packed
+// E2M1), four MMAs.
 template <int KIND, int BNT>
 struct Cfg {
-  static constexpr int KSTAGE = KIND == BS_MX ? 128 : 256;
-  static constexpr int SF_CH = KIND == BS_MX ? 1 : 4;  // scale chunks (4 columns) per stage
+  static constexpr int KSTAGE = KIND == BS_NV ? 256 : 128;
+  static constexpr int SF_CH = KIND == BS_MX ? 1 : KIND == BS_NV ? 4 : 0;  // scale chunks (4 columns) per stage
   static constexpr int W_SMEM = BM * 128;                  // weight tile in shared memory
   static constexpr int W_GLOBAL = KIND == BS_MX ? BM * 64 : BM * 128;  // packed bytes it is read from
   static constexpr int A_SMEM = BNT * 128;
@@ -63,14 +64,17 @@ struct Cfg {
   static constexpr int CTRL = 8192;
   static constexpr int BYTES = NS * STAGE + CTRL + 1024;
   static constexpr int ND = 2;
-  static_assert(BNT <= 128 && ND * BNT <= SFA_COL, "accumulators fit before the scale columns");
+  // the accumulators fit before the scale columns (FP8 has none)
+  static_assert(SF_CH == 0 ? ND * BNT <= TMEM_COLS : (BNT <= 128 && ND * BNT <= SFA_COL), "TMEM budget");
   static_assert(SFB_COL + 4 * SF_CH <= TMEM_COLS, "TMEM budget");
   static_assert(NS >= 3, "stage too large");
 };
 
-// Instruction descriptor of the block-scaled kinds (M = 128, K-major A and B).
+// Instruction descriptor of the block-scaled kinds (M = 128, K-major A and B);
+// FP8: kind::f8f6f4, fp32 accumulator, E4M3 x E4M3.
 template <int KIND, int BNT>
 __device__ __forceinline__ constexpr uint32_t idesc_bs(uint32_t sf_id) {
+  if (KIND == BS_F8) return tc::idesc_e4m3<BNT>();
   return (sf_id << 4)                                            // B scale id (byte of the scale column)
          | ((KIND == BS_MX ? 5u : 1u) << 7)                      // A = E2M1
          | ((KIND == BS_MX ? 0u : 1u) << 10)                     // B = E4M3 (MX) / E2M1 (NV)
@@ -98,7 +102,14 @@ __device__ __forceinline__ void sf_copy(uint32_t taddr, uint64_t sdesc) {
 template <int KIND>
 __device__ __forceinline__ void mma_bs(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t sfa,
                                        uint32_t sfb, uint32_t acc) {
-  if constexpr (KIND == BS_MX) {
+  if constexpr (KIND == BS_F8) {
+    (void)sfa;
+    (void)sfb;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc));
+  } else if constexpr (KIND == BS_MX) {
     asm volatile(
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(tmem_d),
@@ -150,8 +161,8 @@ struct Walk {
 // last of the CTAs sharing the tile sums the parts in k order.
 template <int BNT>
 __device__ __forceinline__ void epilogue_segment(const Params &p, const TileInfo &ti, int t, bool whole, bool head,
-                                                 uint32_t tacc, uint64_t *acce, float gs, int cta, int warp, int lane,
-                                                 long long total) {
+                                                 uint32_t tacc, uint64_t *acce, float cs, float gs, int cta, int warp,
+                                                 int lane, long long total) {
   constexpr int CW = BNT < 32 ? BNT : 32;
   const int r = warp * 32 + lane;
   const int n = ti.wt * BM + r;
@@ -164,7 +175,12 @@ __device__ __forceinline__ void epilogue_segment(const Params &p, const TileInfo
       if (m < ti.nvalid) {
         const int pos = ti.base + m;
         const int orow = p.moe ? p.perm[pos] : pos;
-        p.out[(size_t)orow * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(x[i] * gs));
+        // FP8: per-token x per-row scales; block-scaled kinds: global scales
+        float z = x[i];
+        if (p.row_scale) z *= p.row_scale[p.moe ? orow / p.a_div : pos];
+        z *= cs;
+        z *= gs;
+        p.out[(size_t)orow * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(z));
       }
     }
   };
@@ -362,14 +378,15 @@ __global__ void __launch_bounds__(THREADS, 1)
         uint8_t *st = smem + s * C::STAGE;
         // the transaction count of the expanding (MX) copy is the packed bytes read
         mbar_arrive_expect_tx(&full[s], (uint32_t)(C::W_GLOBAL + C::SF_CH * 512));
-        // MX: coordinates in 4-bit elements (expanded to bytes in shared memory); NV: bytes
+        // MX: coordinates in 4-bit elements (expanded to bytes in shared memory); NV, F8: bytes
         const int x = KIND == BS_MX ? w.ks * C::KSTAGE : w.ks * 128;
         asm volatile(
             "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint "
             "[%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(st)),
             "l"(&w_map), "r"(x), "r"(wrow), "r"(expert), "r"(smem_u32(&full[s])), "l"(pol)
             : "memory");
-        bulk_g2s(st + C::SFA_OFF, sfsrc + (size_t)w.ks * C::SF_CH * 512, C::SF_CH * 512, &full[s]);
+        if constexpr (C::SF_CH > 0)
+          bulk_g2s(st + C::SFA_OFF, sfsrc + (size_t)w.ks * C::SF_CH * 512, C::SF_CH * 512, &full[s]);
       }
       __syncwarp();
       if (++s == NS) { s = 0; ph ^= 1; }
@@ -393,7 +410,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         uint8_t *st = smem + s * C::STAGE;
         mbar_arrive_expect_tx(&full[s], (uint32_t)(C::A_SMEM + C::SF_CH * 512));
         tma_load_2d(st + C::W_SMEM, &a_map, w.ks * 128, base, &full[s]);
-        bulk_g2s(st + C::SFB_OFF, sfsrc + (size_t)w.ks * C::SF_CH * 512, C::SF_CH * 512, &full[s]);
+        if constexpr (C::SF_CH > 0)
+          bulk_g2s(st + C::SFB_OFF, sfsrc + (size_t)w.ks * C::SF_CH * 512, C::SF_CH * 512, &full[s]);
       }
       __syncwarp();
       if (++s == NS) { s = 0; ph ^= 1; }
@@ -452,12 +470,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc::tc_fence_after();
       if (!ok || *(volatile int *)s_abort) break;
       const TileInfo ti = tile_info(t);
-      float gs = 1.f;
+      const uint8_t *eb = p.packed + (size_t)ti.expert * p.stride;
+      float cs = 1.f, gs = 1.f;
       if (KIND == BS_NV) {
-        gs = reinterpret_cast<const float *>(p.packed + (size_t)ti.expert * p.stride + p.g_off)[0];
+        gs = reinterpret_cast<const float *>(eb + p.g_off)[0];
         if (p.a_global) gs = __fmul_rn(gs, *p.a_global);
       }
-      epilogue_segment<BNT>(p, ti, t, whole, ks0 > 0, tmem + (uint32_t)(d * BNT), &acce[d], gs, cta, warp, lane,
+      if (KIND == BS_F8) cs = reinterpret_cast<const float *>(eb + p.c_off)[ti.wt * BM + warp * 32 + lane];
+      epilogue_segment<BNT>(p, ti, t, whole, ks0 > 0, tmem + (uint32_t)(d * BNT), &acce[d], cs, gs, cta, warp, lane,
                             total);
       left -= seg_len;
       ++t;
@@ -544,13 +564,14 @@ __global__ void bs_sf_tiles_kernel(int slots, int bnt, int kst, int sf_ch, int l
 
 // Weight codes of all experts: rows NT*128 per expert, experts `stride` bytes
 // apart.  MX: 4-bit elements expanded to one byte each in shared memory
-// (box 128 codes x 128 rows); NV: packed bytes (box 128 bytes x 128 rows).
+// (box 128 codes x 128 rows); NV, F8: bytes (box 128 bytes x 128 rows).
 static bool make_bs_weight_map(CUtensorMap *m, const Layout &L, const void *packed, int E) {
   auto fn = encode_fn();
   if (!fn) return false;
   const bool mx = L.bs == BS_MX;
-  cuuint64_t dims[3] = {(cuuint64_t)(mx ? L.K : L.K / 2), (cuuint64_t)L.NT * TILE_N, (cuuint64_t)E};
-  cuuint64_t strides[2] = {(cuuint64_t)(L.K / 2), (cuuint64_t)L.stride};
+  const size_t rb = L.bs_row_bytes();
+  cuuint64_t dims[3] = {(cuuint64_t)(mx ? L.K : rb), (cuuint64_t)L.NT * TILE_N, (cuuint64_t)E};
+  cuuint64_t strides[2] = {(cuuint64_t)rb, (cuuint64_t)L.stride};
   cuuint32_t box[3] = {128u, 128u, 1u};
   cuuint32_t estr[3] = {1u, 1u, 1u};
   const CUresult r = fn(m, mx ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B : CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
@@ -598,35 +619,39 @@ static hq_status bs_launch_kind(const CUtensorMap &wm, const CUtensorMap &am, co
     case 16: return bs_launch_one<KIND, 16>(wm, am, p, t, st);
     case 32: return bs_launch_one<KIND, 32>(wm, am, p, t, st);
     case 64: return bs_launch_one<KIND, 64>(wm, am, p, t, st);
-    default: return bs_launch_one<KIND, 128>(wm, am, p, t, st);
+    case 128: return bs_launch_one<KIND, 128>(wm, am, p, t, st);
+    default:
+      if constexpr (KIND == BS_F8) return bs_launch_one<KIND, 256>(wm, am, p, t, st);
+      return HQ_ERR_UNSUPPORTED;
   }
 }
 
 size_t bs_sf_tiles_bytes(const Layout &L, const TcLaunch &t) {
-  if (L.bs == BS_NONE) return 0;
+  if (L.bs == BS_NONE || L.bs == BS_F8) return 0;
   const int kstage = L.bs == BS_MX ? 128 : 256;
   const int sf_ch = L.bs == BS_MX ? 1 : 4;
   return (size_t)t.mtiles * (L.K / kstage) * sf_ch * 512;
 }
 
-// a_codes: `a_rows` activation rows (MXFP8: K E4M3 bytes per row; NVFP4: K/2
-// packed bytes) in the order the tiles read them: dense rows of a, or MoE
+// a_codes: `a_rows` activation rows (MXFP8, FP8: K E4M3 bytes per row; NVFP4:
+// K/2 packed bytes) in the order the tiles read them: dense rows of a, or MoE
 // expert-sorted rows.  a_scales: the caller's scale rows (MXFP8: K/32 E8M0,
-// NVFP4: K/16 UE4M3 per row), read through perm / div for MoE.  Outputs go to
-// row perm[r] for MoE.  sf_tiles: bs_sf_tiles_bytes() of scratch.
+// NVFP4: K/16 UE4M3, FP8: one fp32 per row), read through perm / div for MoE.
+// Outputs go to row perm[r] for MoE.  sf_tiles: bs_sf_tiles_bytes() of
+// scratch (none for FP8).
 hq_status launch_bs_gemm(const Layout &L, const void *packed, int E, const void *a_codes, int a_rows,
                          const void *a_scales, int a_div, const float *a_global, int M, int moe,
                          const int32_t *offsets, const int32_t *perm, void *out, const TcLaunch &t,
                          void *workspace, void *sf_tiles, cudaStream_t st) {
   if (L.bs == BS_NONE || t.kind != 2) return HQ_ERR_UNSUPPORTED;
   if (((uintptr_t)packed & 31) != 0 || ((uintptr_t)a_scales & 3) != 0) return HQ_ERR_INVALID_ARG;
-  const int kstage = L.bs == BS_MX ? 128 : 256;
+  const int kstage = L.bs == BS_NV ? 256 : 128;
   const int sf_ch = L.bs == BS_MX ? 1 : 4;
-  const int row_bytes = L.bs == BS_MX ? L.K : L.K / 2;
+  const int row_bytes = L.bs == BS_NV ? L.K / 2 : L.K;
   CUtensorMap wm, am;
   if (!make_bs_weight_map(&wm, L, packed, E)) return HQ_ERR_CUDA;
   if (!make_bs_act_map(&am, a_codes, a_rows, row_bytes, t.bnt)) return HQ_ERR_CUDA;
-  {
+  if (L.bs != BS_F8) {
     const size_t words = (size_t)t.mtiles * (L.K / kstage) * sf_ch * 128;
     size_t blocks = (words + 255) / 256;
     if (blocks > 148 * 8) blocks = 148 * 8;
@@ -648,7 +673,10 @@ hq_status launch_bs_gemm(const Layout &L, const void *packed, int E, const void 
   p.E = E;
   p.offsets = offsets;
   p.perm = perm;
-  p.a_div = 1;
+  // FP8: per-token scales in the epilogue, caller row perm[r] / div for MoE;
+  // the block scales were laid out per token tile above
+  p.row_scale = L.bs == BS_F8 ? (const float *)a_scales : nullptr;
+  p.a_div = L.bs == BS_F8 ? a_div : 1;
   p.out = (uint16_t *)out;
   p.ntw = t.ntw;
   p.mtiles = t.mtiles;
@@ -660,6 +688,7 @@ hq_status launch_bs_gemm(const Layout &L, const void *packed, int E, const void 
   p.counters = (int *)workspace;
   p.partial = (float *)((uint8_t *)workspace + tc_counter_bytes(t));
   if (L.bs == BS_MX) return bs_launch_kind<BS_MX>(wm, am, p, t, st);
+  if (L.bs == BS_F8) return bs_launch_kind<BS_F8>(wm, am, p, t, st);
   return bs_launch_kind<BS_NV>(wm, am, p, t, st);
 }
 

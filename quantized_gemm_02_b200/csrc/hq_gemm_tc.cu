@@ -806,11 +806,12 @@ TcLaunch plan_tc(int rows_per_tile, int mtiles_bound_moe, int N, int KB, bool mo
   t.bnt = rows_per_tile <= 16 ? 16 : rows_per_tile <= 32 ? 32 : rows_per_tile <= 64 ? 64 : rows_per_tile <= 128 ? 128 : 256;
   t.kind = t.bnt <= 32 ? 1 : 0;
   if (bs != BS_NONE) {
-    // block-scaled kernel: up to 128 tokens per tile, one CTA per SM, a
-    // stage is 2 (MX) or 4 (NV) 64-k blocks
+    // block-scaled kernel: one CTA per SM, a stage is 2 (MX, FP8) or 4 (NV)
+    // 64-k blocks; up to 128 tokens per tile next to the scale columns in
+    // tensor memory, 256 without scales (FP8)
     t.kind = 2;
-    if (t.bnt > 128) t.bnt = 128;
-    KB /= (bs == BS_MX ? 2 : 4);
+    if (t.bnt > 128 && bs != BS_F8) t.bnt = 128;
+    KB /= (bs == BS_NV ? 4 : 2);
   }
   t.ntw = (N + TILE_N - 1) / TILE_N;
   t.mtiles = moe ? mtiles_bound_moe : (rows_per_tile + t.bnt - 1) / t.bnt;

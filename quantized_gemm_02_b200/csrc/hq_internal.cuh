@@ -43,7 +43,7 @@ constexpr int TILE_K = 64;   // k per k-block
 
 // Block-scaled layouts: weights that the tensor core consumes as they are
 // (no dequantisation), with the block scales next to them.
-enum { BS_NONE = 0, BS_MX = 1, BS_NV = 2 };
+enum { BS_NONE = 0, BS_MX = 1, BS_NV = 2, BS_F8 = 3 };
 
 struct Layout {
   int fmt;
@@ -55,6 +55,8 @@ struct Layout {
   size_t w_off, s_off, z_off, c_off, g_off, stride;     // offsets inside an expert region
   __host__ __device__ size_t unit_bytes() const { return (size_t)TILE_N * TILE_K * wbits / 8; }
   __host__ __device__ int chunks() const { return wbits == 4 ? 2 : 4; }
+  // row-major code bytes per weight row of the block-scaled / FP8 layouts
+  __host__ __device__ size_t bs_row_bytes() const { return bs == BS_F8 ? (size_t)K : (size_t)K / 2; }
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -114,6 +116,9 @@ inline bool act_format(const hq_quant_desc *d, int *afmt) {
 //    4 scale columns x 128 rows in the order the tensor-memory copy expects
 //    (row i, scale column j of the chunk at byte (i%32)*16 + (i/32)*4 + j),
 //    [NT][K / (4 * scale group)][512 B]; NVFP4 global scale as fp32.
+//  * BS_F8: FP8 weights x FP8 activations with K % 128 == 0 (kind::f8f6f4,
+//    both operands straight from TMA): codes row-major [NT*128][K] E4M3
+//    bytes, rows past N zero; per-row fp32 scales [NT*128] (zero past N).
 inline Layout make_layout(int fmt, int group, int N, int K, int bs = BS_NONE) {
   Layout L{};
   L.fmt = fmt;
@@ -132,10 +137,10 @@ inline Layout make_layout(int fmt, int group, int N, int K, int bs = BS_NONE) {
   L.c_bytes = (fmt == W_FP8) ? (size_t)L.NT * TILE_N * 4 : 0;
   L.g_bytes = (fmt == W_NVFP4) ? 16 : 0;
   if (bs != BS_NONE) {
-    L.w_bytes = (size_t)L.NT * TILE_N * (K / 2);
-    L.s_bytes = (size_t)L.NT * (K / (4 * L.group)) * 512;
+    L.w_bytes = (size_t)L.NT * TILE_N * L.bs_row_bytes();
+    L.s_bytes = bs == BS_F8 ? 0 : (size_t)L.NT * (K / (4 * L.group)) * 512;
     L.z_bytes = 0;
-    L.c_bytes = 0;
+    L.c_bytes = bs == BS_F8 ? (size_t)L.NT * TILE_N * 4 : 0;
   }
   size_t off = 0;
   L.w_off = off; off = align_up(off + L.w_bytes, 256);
@@ -155,6 +160,7 @@ inline Layout layout_for(const hq_quant_desc *d, int fmt, int N, int K) {
   if (act_format(d, &afmt)) {
     if (fmt == W_MXFP4 && afmt == A_MXFP8 && (K % 128) == 0) bs = BS_MX;
     if (fmt == W_NVFP4 && afmt == A_NVFP4 && (K % 256) == 0) bs = BS_NV;
+    if (fmt == W_FP8 && afmt == A_FP8 && (K % 128) == 0) bs = BS_F8;
   }
   return make_layout(fmt, d->w_group, N, K, bs);
 }

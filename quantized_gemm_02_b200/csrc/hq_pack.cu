@@ -190,7 +190,8 @@ __host__ __device__ inline uint32_t bs_sf_offset(int i, int j) { return (uint32_
 
 // Codes: row-major copy with the rows past N zeroed; 16 bytes per thread.
 __global__ void pack_bs_codes_kernel(Layout L, int E, const uint8_t *codes, uint8_t *packed) {
-  const size_t row16 = (size_t)L.K / 32;  // 16-byte pieces per row (K/2 bytes)
+  const size_t rb = L.bs_row_bytes();
+  const size_t row16 = rb / 16;  // 16-byte pieces per row
   const size_t rows = (size_t)L.NT * TILE_N;
   const size_t total = (size_t)E * rows * row16;
   for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < total;
@@ -200,12 +201,13 @@ __global__ void pack_bs_codes_kernel(Layout L, int E, const uint8_t *codes, uint
     const int r = (int)(rem / row16);
     const size_t c = rem % row16;
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (r < L.N) v = reinterpret_cast<const uint4 *>(codes + ((size_t)e * L.N + r) * (L.K / 2))[c];
-    reinterpret_cast<uint4 *>(packed + (size_t)e * L.stride + L.w_off + (size_t)r * (L.K / 2))[c] = v;
+    if (r < L.N) v = reinterpret_cast<const uint4 *>(codes + ((size_t)e * L.N + r) * rb)[c];
+    reinterpret_cast<uint4 *>(packed + (size_t)e * L.stride + L.w_off + (size_t)r * rb)[c] = v;
   }
 }
 
-// Scales into 512-byte chunks (one thread per scale byte) and the global scale.
+// Scales into 512-byte chunks (one thread per scale byte) and the global
+// scale; FP8: the per-row fp32 scales, zero past N.
 __global__ void pack_bs_side_kernel(Layout L, int E, const uint8_t *scales, const float *global_scale,
                                     uint8_t *packed) {
   const int R = L.NT * TILE_N;
@@ -217,6 +219,11 @@ __global__ void pack_bs_side_kernel(Layout L, int E, const uint8_t *scales, cons
     const int r = rem / L.G, gi = rem % L.G;
     const int nt = r / TILE_N, i = r % TILE_N;
     uint8_t *base = packed + (size_t)e * L.stride;
+    if (L.bs == BS_F8) {
+      reinterpret_cast<float *>(base + L.c_off)[r] =
+          (r < L.N) ? reinterpret_cast<const float *>(scales)[(size_t)e * L.N + r] : 0.f;
+      continue;
+    }
     const uint8_t sv = (r < L.N) ? scales[((size_t)e * L.N + r) * L.G + gi] : (uint8_t)0;
     base[L.s_off + ((size_t)nt * (L.G / 4) + gi / 4) * 512 + bs_sf_offset(i, gi & 3)] = sv;
     if (L.fmt == W_NVFP4 && r == 0 && gi == 0) reinterpret_cast<float *>(base + L.g_off)[0] = global_scale[e];
@@ -225,7 +232,8 @@ __global__ void pack_bs_side_kernel(Layout L, int E, const uint8_t *scales, cons
 
 __global__ void unpack_bs_kernel(Layout L, int E, const uint8_t *packed, uint8_t *codes, uint8_t *scales,
                                  float *global_scale) {
-  const size_t row16 = (size_t)L.K / 32;
+  const size_t rb = L.bs_row_bytes();
+  const size_t row16 = rb / 16;
   const size_t total_c = (size_t)E * L.N * row16;
   const size_t total_s = (size_t)E * L.N * L.G;
   for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < total_c + total_s;
@@ -235,8 +243,8 @@ __global__ void unpack_bs_kernel(Layout L, int E, const uint8_t *packed, uint8_t
       const size_t rem = idx % ((size_t)L.N * row16);
       const int r = (int)(rem / row16);
       const size_t c = rem % row16;
-      reinterpret_cast<uint4 *>(codes + ((size_t)e * L.N + r) * (L.K / 2))[c] =
-          reinterpret_cast<const uint4 *>(packed + (size_t)e * L.stride + L.w_off + (size_t)r * (L.K / 2))[c];
+      reinterpret_cast<uint4 *>(codes + ((size_t)e * L.N + r) * rb)[c] =
+          reinterpret_cast<const uint4 *>(packed + (size_t)e * L.stride + L.w_off + (size_t)r * rb)[c];
     } else {
       const size_t j = idx - total_c;
       const int e = (int)(j / ((size_t)L.N * L.G));
@@ -244,6 +252,10 @@ __global__ void unpack_bs_kernel(Layout L, int E, const uint8_t *packed, uint8_t
       const int r = rem / L.G, gi = rem % L.G;
       const int nt = r / TILE_N, i = r % TILE_N;
       const uint8_t *base = packed + (size_t)e * L.stride;
+      if (L.bs == BS_F8) {
+        reinterpret_cast<float *>(scales)[(size_t)e * L.N + r] = reinterpret_cast<const float *>(base + L.c_off)[r];
+        continue;
+      }
       scales[j] = base[L.s_off + ((size_t)nt * (L.G / 4) + gi / 4) * 512 + bs_sf_offset(i, gi & 3)];
       if (L.fmt == W_NVFP4 && r == 0 && gi == 0) global_scale[e] = reinterpret_cast<const float *>(base + L.g_off)[0];
     }
@@ -260,7 +272,7 @@ static int pack_grid(size_t total, int threads) {
 hq_status launch_pack(const Layout &L, int E, const void *codes, const void *scales, const void *zeros,
                       const float *global_scale, void *packed, cudaStream_t st) {
   if (L.bs != BS_NONE) {
-    const size_t n16 = (size_t)E * L.NT * TILE_N * (L.K / 32);
+    const size_t n16 = (size_t)E * L.NT * TILE_N * (L.bs_row_bytes() / 16);
     pack_bs_codes_kernel<<<pack_grid(n16, 256), 256, 0, st>>>(L, E, (const uint8_t *)codes, (uint8_t *)packed);
     const size_t ns = (size_t)E * L.NT * TILE_N * L.G;
     pack_bs_side_kernel<<<pack_grid(ns, 256), 256, 0, st>>>(L, E, (const uint8_t *)scales, global_scale,
@@ -278,7 +290,7 @@ hq_status launch_pack(const Layout &L, int E, const void *codes, const void *sca
 hq_status launch_unpack(const Layout &L, int E, const void *packed, void *codes, void *scales, void *zeros,
                         float *global_scale, cudaStream_t st) {
   if (L.bs != BS_NONE) {
-    const size_t n = (size_t)E * L.N * (L.K / 32) + (size_t)E * L.N * L.G;
+    const size_t n = (size_t)E * L.N * (L.bs_row_bytes() / 16) + (size_t)E * L.N * L.G;
     unpack_bs_kernel<<<pack_grid(n, 256), 256, 0, st>>>(L, E, (const uint8_t *)packed, (uint8_t *)codes,
                                                          (uint8_t *)scales, global_scale);
     return check_launch();

@@ -78,12 +78,20 @@ def test_gemm_many_token_tiles():
     parity("fp8", "fp8", 2100, 136, 256, seed=7)
 
 
-@pytest.mark.parametrize("wname,aname", [("mxfp4", "mxfp8"), ("nvfp4", "nvfp4")])
+@pytest.mark.parametrize("wname,aname", [("mxfp4", "mxfp8"), ("nvfp4", "nvfp4"), ("fp8", "fp8")])
 @pytest.mark.parametrize("M", [129, 300])
 def test_gemm_block_scaled_many_token_tiles(wname, aname, M):
     # more than 128 tokens: several 128-token tiles of the block-scaled
-    # kernel (scale chunks of each token slot), ragged last tile
+    # kernel (scale chunks of each token slot), ragged last tile; FP8 x FP8
+    # runs 256-token tiles (no scale columns in tensor memory)
     parity(wname, aname, M, 136, 512, seed=20 + M)
+
+
+@pytest.mark.parametrize("M", [16, 300])
+def test_gemm_fp8_fp8_k_not_multiple_of_128(M):
+    # K = 192: the FP8 x FP8 pair keeps the tiled layout and the kernels that
+    # stage the E4M3 weights through tensor memory
+    parity("fp8", "fp8", M, 136, 192, seed=40 + M)
 
 
 def test_config1_full():

@@ -27,10 +27,10 @@ def test_pack_unpack_identity(wname):
         assert np.array_equal(np_bits(out[k]), np_bits(v)), k
 
 
-@pytest.mark.parametrize("wname,aname", [("mxfp4", "mxfp8"), ("nvfp4", "nvfp4")])
+@pytest.mark.parametrize("wname,aname", [("mxfp4", "mxfp8"), ("nvfp4", "nvfp4"), ("fp8", "fp8")])
 def test_pack_unpack_identity_block_scaled(wname, aname):
     # block-scaled layouts (chosen by the activation format): codes row-major,
-    # scales in 512-byte chunks
+    # scales in 512-byte chunks; FP8 x FP8: E4M3 bytes row-major, row scales
     import quantized_gemm_02_b200 as hq
     E, N, K = 2, 80, 512
     w = make_weights(wname, E, N, K, seed=5)
@@ -43,13 +43,14 @@ def test_pack_unpack_identity_block_scaled(wname, aname):
         if v is None:
             continue
         assert np.array_equal(np_bits(out[k]), np_bits(v)), k
-    # the codes sit row-major (two per byte, even k low), padded rows zero
+    # the codes sit row-major (4-bit: two per byte, even k low), padded rows zero
     d = cdesc(wname, aname)
     per_e = hq.hq_packed_weights_bytes(d, 1, N, K)
     p0 = packed[:per_e].cpu().numpy()
     codes = w["codes"][0].numpy() if hasattr(w["codes"], "numpy") else w["codes"][0].cpu().numpy()
-    assert np.array_equal(p0[: N * K // 2].reshape(N, K // 2), codes.reshape(N, K // 2))
-    assert not p0[N * K // 2: 128 * K // 2].any()
+    rb = K if wname == "fp8" else K // 2
+    assert np.array_equal(p0[: N * rb].reshape(N, rb), codes.reshape(N, rb))
+    assert not p0[N * rb: 128 * rb].any()
 
 
 def test_pack_is_deterministic_and_pads_with_zero():

@@ -36,6 +36,7 @@ def _reference_and_bound(wname, aname, w, x, M, N, K):
     ("mxfp4", "bf16", 4, 512, 8192),        # split-K: tile counters at the head of the scratch
     ("nvfp4", "nvfp4", 24, 320, 1024),      # block-scaled MMA, Stream-K tickets in the scratch
     ("nvfp4", "fp8", 24, 320, 1024),        # quantised activations: decoded copy in the scratch
+    ("fp8", "fp8", 24, 320, 1024),          # FP8 MMA straight from TMA, per-token scales in the epilogue
     ("uint4_g128", "bf16", 40, 200, 2048),  # several token tiles
 ])
 def test_noalloc_matches_hq_gemm_twice(wname, aname, M, N, K):
