@@ -806,14 +806,20 @@ TcLaunch plan_tc(int rows_per_tile, int mtiles_bound_moe, int N, int KB, bool mo
   t.bnt = rows_per_tile <= 16 ? 16 : rows_per_tile <= 32 ? 32 : rows_per_tile <= 64 ? 64 : rows_per_tile <= 128 ? 128 : 256;
   t.kind = t.bnt <= 32 ? 1 : 0;
   if (bs != BS_NONE) {
-    // block-scaled kernel: one CTA per SM, a stage is 2 (MX, FP8) or 4 (NV)
-    // 64-k blocks; up to 128 tokens per tile next to the scale columns in
-    // tensor memory, 256 without scales (FP8)
+    // block-scaled kernel: one CTA per SM, a stage is 1 (FP8), 2 (MX) or 4
+    // (NV) 64-k blocks; up to 128 tokens per tile next to the scale columns
+    // in tensor memory, 256 without scales (FP8)
     t.kind = 2;
     if (t.bnt > 128 && bs != BS_F8) t.bnt = 128;
-    KB /= (bs == BS_NV ? 4 : 2);
+    KB /= (bs == BS_NV ? 4 : bs == BS_MX ? 2 : 1);
   }
   t.ntw = (N + TILE_N - 1) / TILE_N;
+  if (t.kind == 2 && t.bnt == 256 && !moe &&
+      (long long)t.ntw * ((rows_per_tile + 255) / 256) < 2LL * sm_count()) {
+    // fewer than two 256-token tiles per SM: 128-token tiles halve the
+    // Stream-K partial sums and split fewer tiles
+    t.bnt = 128;
+  }
   t.mtiles = moe ? mtiles_bound_moe : (rows_per_tile + t.bnt - 1) / t.bnt;
   if (t.mtiles < 1) t.mtiles = 1;
   const long long iters = (long long)t.ntw * t.mtiles * KB;

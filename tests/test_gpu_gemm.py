@@ -87,6 +87,14 @@ def test_gemm_block_scaled_many_token_tiles(wname, aname, M):
     parity(wname, aname, M, 136, 512, seed=20 + M)
 
 
+def test_gemm_fp8_fp8_256_token_tiles():
+    # enough 256-token tiles (2 x 148 weight tiles) for the FP8 kernel to use
+    # them: 300 tokens = one full and one ragged tile; sampled columns
+    N = 148 * 128
+    cols = np.sort(np.random.default_rng(3).choice(N, 256, replace=False))
+    parity("fp8", "fp8", 300, N, 256, seed=44, cols=cols)
+
+
 @pytest.mark.parametrize("M", [16, 300])
 def test_gemm_fp8_fp8_k_not_multiple_of_128(M):
     # K = 192: the FP8 x FP8 pair keeps the tiled layout and the kernels that
