@@ -132,10 +132,11 @@ HQ_API hq_status hq_selftest_wait_timeout(unsigned long long limit_ns, hq_stream
  * The packed layout depends on the whole description, the activation
  *   format included: MXFP4 weights with a_dtype MXFP8 (K a multiple of 128)
  *   and NVFP4 weights with a_dtype NVFP4 (K a multiple of 256) are stored
- *   for the block-scaled tensor-core MMA (codes as they are, scales in the
- *   MMA's chunk order), FP8 weights with a_dtype E4M3 (K a multiple of 128)
- *   as row-major E4M3 bytes with per-row fp32 scales for the FP8 MMA; every
- *   other pair for in-kernel dequantisation.  Pack,
+ *   for the block-scaled tensor-core MMA (each row's codes cut into stage
+ *   chunks stored contiguously per 128-row tile, scales in the MMA's chunk
+ *   order), FP8 weights with a_dtype E4M3 (K a multiple of 128) likewise as
+ *   E4M3 bytes with per-row fp32 scales for the FP8 MMA; every other pair
+ *   for in-kernel dequantisation.  Pack,
  *   unpack, hq_gemm and hq_moe_gemm must be given the same description.
  *   The packed buffer must be 32-byte aligned (cudaMalloc's 256 is).
  * hq_pack_weights: standard-format codes / scales / zeros (device) and, for

@@ -363,12 +363,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     Walk w;
     w.start(beg, end, p.KB);
     int cur_t = -1, wrow = 0, expert = 0;
+    const int nchunk = p.KB;  // stage chunks per weight row (one per stage)
     const uint8_t *sfsrc = nullptr;
     for (int is = 0, s = 0, ph = 0; w.left > 0; ++is, w.next(p.KB)) {
       if (w.t != cur_t) {
         const TileInfo ti = tile_info(w.t);
         expert = ti.expert;
-        wrow = ti.wt * BM;
+        wrow = ti.wt * nchunk * BM;  // first chunk row of the tile
         sfsrc = p.packed + (size_t)ti.expert * p.stride + p.s_off + (size_t)ti.wt * chunks_per_tile * 512;
         cur_t = w.t;
       }
@@ -378,12 +379,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         uint8_t *st = smem + s * C::STAGE;
         // the transaction count of the expanding (MX) copy is the packed bytes read
         mbar_arrive_expect_tx(&full[s], (uint32_t)(C::W_GLOBAL + C::SF_CH * 512));
-        // MX: coordinates in 4-bit elements (expanded to bytes in shared memory); NV, F8: bytes
-        const int x = KIND == BS_MX ? w.ks * C::KSTAGE : w.ks * 128;
+        // the stage's 128 rows are one contiguous chunk block of the tile
         asm volatile(
             "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint "
             "[%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(st)),
-            "l"(&w_map), "r"(x), "r"(wrow), "r"(expert), "r"(smem_u32(&full[s])), "l"(pol)
+            "l"(&w_map), "r"(0), "r"(wrow + w.ks * BM), "r"(expert), "r"(smem_u32(&full[s])), "l"(pol)
             : "memory");
         if constexpr (C::SF_CH > 0)
           bulk_g2s(st + C::SFA_OFF, sfsrc + (size_t)w.ks * C::SF_CH * 512, C::SF_CH * 512, &full[s]);
@@ -562,16 +562,18 @@ __global__ void bs_sf_tiles_kernel(int slots, int bnt, int kst, int sf_ch, int l
 
 // ---- host side -------------------------------------------------------------------
 
-// Weight codes of all experts: rows NT*128 per expert, experts `stride` bytes
-// apart.  MX: 4-bit elements expanded to one byte each in shared memory
-// (box 128 codes x 128 rows); NV, F8: bytes (box 128 bytes x 128 rows).
+// Weight codes of all experts as rows of one stage chunk ([NT][stages][128]
+// rows per expert), experts `stride` bytes apart.  MX: 4-bit elements
+// expanded to one byte each in shared memory (box 128 codes x 128 rows); NV,
+// F8: bytes (box 128 bytes x 128 rows).
 static bool make_bs_weight_map(CUtensorMap *m, const Layout &L, const void *packed, int E) {
   auto fn = encode_fn();
   if (!fn) return false;
   const bool mx = L.bs == BS_MX;
-  const size_t rb = L.bs_row_bytes();
-  cuuint64_t dims[3] = {(cuuint64_t)(mx ? L.K : rb), (cuuint64_t)L.NT * TILE_N, (cuuint64_t)E};
-  cuuint64_t strides[2] = {(cuuint64_t)rb, (cuuint64_t)L.stride};
+  const size_t cb = (size_t)L.bs_chunk_bytes();
+  const size_t rows = (size_t)L.NT * (L.bs_row_bytes() / cb) * TILE_N;
+  cuuint64_t dims[3] = {(cuuint64_t)(mx ? 2 * cb : cb), (cuuint64_t)rows, (cuuint64_t)E};
+  cuuint64_t strides[2] = {(cuuint64_t)cb, (cuuint64_t)L.stride};
   cuuint32_t box[3] = {128u, 128u, 1u};
   cuuint32_t estr[3] = {1u, 1u, 1u};
   const CUresult r = fn(m, mx ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B : CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
@@ -681,7 +683,9 @@ hq_status launch_bs_gemm(const Layout &L, const void *packed, int E, const void 
   p.ntw = t.ntw;
   p.mtiles = t.mtiles;
   p.nctas = t.nctas;
-  p.weights_once = (!moe && t.mtiles == 1) ? 1 : 0;
+  // weights read by one token tile (dense), or by about one per expert (MoE):
+  // stream them past L2 so that the activation tiles stay resident
+  p.weights_once = ((!moe && t.mtiles == 1) || (moe && t.mtiles <= 2 * E)) ? 1 : 0;
   p.a_sf = (const uint8_t *)sf_tiles;
   p.a_sf_ld = 0;
   p.a_rows = a_rows;

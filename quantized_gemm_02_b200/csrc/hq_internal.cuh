@@ -55,8 +55,16 @@ struct Layout {
   size_t w_off, s_off, z_off, c_off, g_off, stride;     // offsets inside an expert region
   __host__ __device__ size_t unit_bytes() const { return (size_t)TILE_N * TILE_K * wbits / 8; }
   __host__ __device__ int chunks() const { return wbits == 4 ? 2 : 4; }
-  // row-major code bytes per weight row of the block-scaled / FP8 layouts
+  // code bytes per weight row of the block-scaled / FP8 layouts
   __host__ __device__ size_t bs_row_bytes() const { return bs == BS_F8 ? (size_t)K : (size_t)K / 2; }
+  // ... stored in chunks of this many bytes per row: one MMA stage (MX: 128
+  // codes = 64 bytes; NV: 256 codes, F8: 128 codes = 128 bytes)
+  __host__ __device__ int bs_chunk_bytes() const { return bs == BS_MX ? 64 : 128; }
+  // byte offset (from w_off) of row r's chunk c: [NT][row_bytes / chunk][128 rows][chunk]
+  __host__ __device__ size_t bs_chunk_off(int r, int c) const {
+    const size_t nc = bs_row_bytes() / bs_chunk_bytes();
+    return (((size_t)(r / TILE_N) * nc + c) * TILE_N + (r % TILE_N)) * bs_chunk_bytes();
+  }
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -111,14 +119,16 @@ inline bool act_format(const hq_quant_desc *d, int *afmt) {
 //    one the tensor core multiplies with block scales itself:
 //      BS_MX  MXFP4 weights x MXFP8 activations (kind::mxf8f6f4, K % 128 == 0)
 //      BS_NV  NVFP4 weights x NVFP4 activations (kind::mxf4nvf4, K % 256 == 0)
-//    codes: row-major [NT*128][K/2] bytes, two E2M1 codes per byte (even k in
-//    the low nibble), rows past N zero; scales: per 128-row tile, chunks of
+//    codes: [NT][stages][128 rows][chunk] bytes, two E2M1 codes per byte
+//    (even k in the low nibble), rows past N zero, chunk = one stage of a row
+//    (MX: 64 bytes, NV: 128 bytes), so that a stage of a tile is one
+//    contiguous 8 / 16 KB piece of HBM; scales: per 128-row tile, chunks of
 //    4 scale columns x 128 rows in the order the tensor-memory copy expects
 //    (row i, scale column j of the chunk at byte (i%32)*16 + (i/32)*4 + j),
 //    [NT][K / (4 * scale group)][512 B]; NVFP4 global scale as fp32.
 //  * BS_F8: FP8 weights x FP8 activations with K % 128 == 0 (kind::f8f6f4,
-//    both operands straight from TMA): codes row-major [NT*128][K] E4M3
-//    bytes, rows past N zero; per-row fp32 scales [NT*128] (zero past N).
+//    both operands straight from TMA): codes [NT][K/128][128 rows][128 B]
+//    E4M3 bytes, rows past N zero; per-row fp32 scales [NT*128] (zero past N).
 inline Layout make_layout(int fmt, int group, int N, int K, int bs = BS_NONE) {
   Layout L{};
   L.fmt = fmt;

@@ -188,7 +188,8 @@ __global__ void unpack_side_kernel(Layout L, int E, const uint8_t *packed, uint8
 // scales of rows i, i + 32, i + 64, i + 96 in four consecutive columns.
 __host__ __device__ inline uint32_t bs_sf_offset(int i, int j) { return (uint32_t)((i & 31) * 16 + (i >> 5) * 4 + j); }
 
-// Codes: row-major copy with the rows past N zeroed; 16 bytes per thread.
+// Codes: each row's bytes cut into stage chunks, [NT][chunk][128 rows][chunk
+// bytes], rows past N zeroed; 16 bytes per thread.
 __global__ void pack_bs_codes_kernel(Layout L, int E, const uint8_t *codes, uint8_t *packed) {
   const size_t rb = L.bs_row_bytes();
   const size_t row16 = rb / 16;  // 16-byte pieces per row
@@ -202,7 +203,9 @@ __global__ void pack_bs_codes_kernel(Layout L, int E, const uint8_t *codes, uint
     const size_t c = rem % row16;
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
     if (r < L.N) v = reinterpret_cast<const uint4 *>(codes + ((size_t)e * L.N + r) * rb)[c];
-    reinterpret_cast<uint4 *>(packed + (size_t)e * L.stride + L.w_off + (size_t)r * rb)[c] = v;
+    const int cb = L.bs_chunk_bytes();
+    *reinterpret_cast<uint4 *>(packed + (size_t)e * L.stride + L.w_off +
+                               L.bs_chunk_off(r, (int)(c * 16 / cb)) + (c * 16) % cb) = v;
   }
 }
 
@@ -243,8 +246,9 @@ __global__ void unpack_bs_kernel(Layout L, int E, const uint8_t *packed, uint8_t
       const size_t rem = idx % ((size_t)L.N * row16);
       const int r = (int)(rem / row16);
       const size_t c = rem % row16;
-      reinterpret_cast<uint4 *>(codes + ((size_t)e * L.N + r) * rb)[c] =
-          reinterpret_cast<const uint4 *>(packed + (size_t)e * L.stride + L.w_off + (size_t)r * rb)[c];
+      const int cb = L.bs_chunk_bytes();
+      reinterpret_cast<uint4 *>(codes + ((size_t)e * L.N + r) * rb)[c] = *reinterpret_cast<const uint4 *>(
+          packed + (size_t)e * L.stride + L.w_off + L.bs_chunk_off(r, (int)(c * 16 / cb)) + (c * 16) % cb);
     } else {
       const size_t j = idx - total_c;
       const int e = (int)(j / ((size_t)L.N * L.G));

@@ -43,14 +43,18 @@ def test_pack_unpack_identity_block_scaled(wname, aname):
         if v is None:
             continue
         assert np.array_equal(np_bits(out[k]), np_bits(v)), k
-    # the codes sit row-major (4-bit: two per byte, even k low), padded rows zero
+    # the codes of each row sit in stage chunks (MXFP4: 64 bytes, else 128),
+    # [chunk][128 rows][chunk bytes] per 128-row tile (4-bit: two per byte,
+    # even k low), padded rows zero
     d = cdesc(wname, aname)
     per_e = hq.hq_packed_weights_bytes(d, 1, N, K)
     p0 = packed[:per_e].cpu().numpy()
     codes = w["codes"][0].numpy() if hasattr(w["codes"], "numpy") else w["codes"][0].cpu().numpy()
     rb = K if wname == "fp8" else K // 2
-    assert np.array_equal(p0[: N * rb].reshape(N, rb), codes.reshape(N, rb))
-    assert not p0[N * rb: 128 * rb].any()
+    cb = 64 if wname == "mxfp4" else 128
+    rows = p0[: 128 * rb].reshape(rb // cb, 128, cb).transpose(1, 0, 2).reshape(128, rb)
+    assert np.array_equal(rows[:N], codes.reshape(N, rb))
+    assert not rows[N:].any()
 
 
 def test_pack_is_deterministic_and_pads_with_zero():
