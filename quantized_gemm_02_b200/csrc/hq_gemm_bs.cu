@@ -168,16 +168,23 @@ __device__ __forceinline__ void epilogue_segment(const Params &p, const TileInfo
   const int n = ti.wt * BM + r;
   float *part = p.partial + ((size_t)cta * 2 + (head ? 0 : 1)) * BNT * BM;
   auto write = [&](int c0, const float *x) {
-    if (n >= p.N) return;
+    // the chunk's output rows (and FP8 per-token scales): one load per lane,
+    // handed to the other lanes by shuffles, so no store waits on a load
+    int orow_l = 0;
+    float rs_l = 1.f;
+    if (c0 + lane < ti.nvalid) {
+      const int pos = ti.base + c0 + lane;
+      orow_l = p.moe ? p.perm[pos] : pos;
+      if (p.row_scale) rs_l = p.row_scale[p.moe ? orow_l / p.a_div : pos];
+    }
 #pragma unroll
     for (int i = 0; i < CW; ++i) {
-      const int m = c0 + i;
-      if (m < ti.nvalid) {
-        const int pos = ti.base + m;
-        const int orow = p.moe ? p.perm[pos] : pos;
+      const int orow = __shfl_sync(0xffffffffu, orow_l, i);
+      const float rs = __shfl_sync(0xffffffffu, rs_l, i);
+      if (c0 + i < ti.nvalid && n < p.N) {
         // FP8: per-token x per-row scales; block-scaled kinds: global scales
         float z = x[i];
-        if (p.row_scale) z *= p.row_scale[p.moe ? orow / p.a_div : pos];
+        if (p.row_scale) z *= rs;
         z *= cs;
         z *= gs;
         p.out[(size_t)orow * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(z));

@@ -222,14 +222,23 @@ __device__ __forceinline__ void decode_bf16(const uint8_t *wpk, const uint8_t *s
 template <int BNT>
 __device__ __forceinline__ void store_rows(const Params &p, const TileInfo &ti, int n, const float (&x)[BNT],
                                            float cs, float gs) {
-  if (n >= p.N) return;
+  // output rows (and per-token scales) of the tile's tokens: one load per
+  // lane, handed to the other lanes by shuffles (whole warp, BNT <= 32)
+  const int lane = threadIdx.x & 31;
+  int orow_l = 0;
+  float rs_l = 1.f;
+  if (lane < BNT && lane < ti.nvalid) {
+    const int pos = ti.base + lane;
+    orow_l = p.moe ? p.perm[pos] : pos;
+    if (p.row_scale) rs_l = p.row_scale[p.moe ? orow_l / p.a_div : pos];
+  }
 #pragma unroll
   for (int m = 0; m < BNT; ++m) {
-    if (m < ti.nvalid) {
-      const int pos = ti.base + m;
-      const int orow = p.moe ? p.perm[pos] : pos;
+    const int orow = __shfl_sync(0xffffffffu, orow_l, m);
+    const float rs = __shfl_sync(0xffffffffu, rs_l, m);
+    if (m < ti.nvalid && n < p.N) {
       float z = x[m];
-      if (p.row_scale) z *= p.row_scale[p.moe ? orow / p.a_div : pos];
+      if (p.row_scale) z *= rs;
       z *= cs;
       z *= gs;
       p.out[(size_t)orow * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(z));

@@ -667,15 +667,23 @@ __global__ void __launch_bounds__(THREADS, (BNT <= 64 ? 2 : 1)) tc_gemm_kernel(c
         if (split_mode) {
 #pragma unroll
           for (int i = 0; i < 16; ++i) __stcg(&part[(size_t)(c0 + i) * BM + r], v[i]);
-        } else if (n < p.N) {
+        } else {
+          // the 16 tokens' output rows (and per-token scales): one load per
+          // lane, handed to the other lanes by shuffles
+          int orow_l = 0;
+          float rs_l = 1.f;
+          if (c0 + (lane & 15) < ti.nvalid) {
+            const int pos = ti.base + c0 + (lane & 15);
+            orow_l = p.moe ? p.perm[pos] : pos;
+            if (p.row_scale) rs_l = p.row_scale[p.moe ? orow_l / p.a_div : pos];
+          }
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const int m = c0 + i;
-            if (m < ti.nvalid) {
-              const int pos = ti.base + m;
-              const int orow = p.moe ? p.perm[pos] : pos;
+            const int orow = __shfl_sync(0xffffffffu, orow_l, i);
+            const float rs = __shfl_sync(0xffffffffu, rs_l, i);
+            if (c0 + i < ti.nvalid && n < p.N) {
               float x = v[i];
-              if (p.row_scale) x *= p.row_scale[p.moe ? orow / p.a_div : pos];
+              if (p.row_scale) x *= rs;
               x *= cs;
               x *= gs;
               p.out[(size_t)orow * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(x));
