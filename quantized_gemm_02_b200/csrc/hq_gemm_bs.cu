@@ -12,7 +12,8 @@
 //     instruction, E2M1 weights expanded to one byte per code in shared
 //     memory by the TMA) or kind::mxf4nvf4.block_scale.scale_vec::4X (NV,
 //     K = 64, both operands packed E2M1); 128 weight rows are operand A,
-//     16..128 tokens operand B, both in shared memory with a 128-byte swizzle;
+//     16..128 tokens operand B (NVFP4 MoE: 192; FP8: up to 256), both in
+//     shared memory with a 128-byte swizzle;
 //   * the scale chunks (128 rows x 4 scales, 512 bytes) go shared memory ->
 //     tensor memory with tcgen05.cp.32x128b.warpx4; the weight scales are
 //     stored in that order by the repack, the activation scales are gathered
@@ -43,8 +44,6 @@ using tc::TileInfo;
 constexpr int WARP_W = 4, WARP_MMA = 5, WARP_ACT = 6;
 constexpr int THREADS = 7 * 32;
 constexpr int TMEM_COLS = 512;
-constexpr int SFA_COL = 256;  // TMEM columns of the weight scales (after two 128-column accumulators)
-constexpr int SFB_COL = 288;  // TMEM columns of the activation scales
 
 // KIND: BS_MX, BS_NV or BS_F8.  A stage is one 128-byte row of each operand:
 // 128 k (MX: E2M1 expanded to bytes / E4M3; F8: E4M3) or 256 k (NV: packed
@@ -57,16 +56,22 @@ struct Cfg {
   static constexpr int W_GLOBAL = KIND == BS_MX ? BM * 64 : BM * 128;  // packed bytes it is read from
   static constexpr int A_SMEM = BNT * 128;
   static constexpr int SFA_OFF = W_SMEM + A_SMEM;
+  // activation scale chunk: 512 bytes per 128 token rows (tiles of more
+  // than 128 tokens: a second 512 bytes for rows 128..255)
+  static constexpr int SFB_HALVES = BNT > 128 ? 2 : 1;
+  static constexpr int SFB_CHB = 512 * SFB_HALVES;  // bytes per activation scale chunk
+  static constexpr int SFB_CPC = 4 * SFB_HALVES;    // TMEM columns per activation scale chunk
   static constexpr int SFB_OFF = SFA_OFF + SF_CH * 512;
-  static constexpr int STAGE = (SFB_OFF + SF_CH * 512 + 1023) / 1024 * 1024;
+  static constexpr int STAGE = (SFB_OFF + SF_CH * SFB_CHB + 1023) / 1024 * 1024;
   static constexpr int NS_FIT = (200 * 1024) / STAGE;
   static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;
   static constexpr int CTRL = 8192;
   static constexpr int BYTES = NS * STAGE + CTRL + 1024;
   static constexpr int ND = 2;
-  // the accumulators fit before the scale columns (FP8 has none)
-  static_assert(SF_CH == 0 ? ND * BNT <= TMEM_COLS : (BNT <= 128 && ND * BNT <= SFA_COL), "TMEM budget");
-  static_assert(SFB_COL + 4 * SF_CH <= TMEM_COLS, "TMEM budget");
+  // TMEM: two accumulators, then the weight and the activation scale columns
+  static constexpr int SFA_COL = ND * BNT;
+  static constexpr int SFB_COL = SFA_COL + 4 * SF_CH;
+  static_assert(SFB_COL + SFB_CPC * SF_CH <= TMEM_COLS, "TMEM budget");
   static_assert(NS >= 3, "stage too large");
 };
 
@@ -408,17 +413,17 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (w.t != cur_t) {
         base = tile_info(w.t).base;
         // scale chunks of this tile's token slot, laid out by bs_sf_tiles_kernel
-        sfsrc = p.a_sf + (size_t)(w.t / p.ntw) * p.KB * (C::SF_CH * 512);
+        sfsrc = p.a_sf + (size_t)(w.t / p.ntw) * p.KB * (C::SF_CH * C::SFB_CHB);
         cur_t = w.t;
       }
       if (is >= NS && !mbar_wait(&sfree[s], ph ^ 1)) { *s_abort = 1; break; }
       if (*(volatile int *)s_abort) break;
       if (lane == 0) {
         uint8_t *st = smem + s * C::STAGE;
-        mbar_arrive_expect_tx(&full[s], (uint32_t)(C::A_SMEM + C::SF_CH * 512));
+        mbar_arrive_expect_tx(&full[s], (uint32_t)(C::A_SMEM + C::SF_CH * C::SFB_CHB));
         tma_load_2d(st + C::W_SMEM, &a_map, w.ks * 128, base, &full[s]);
         if constexpr (C::SF_CH > 0)
-          bulk_g2s(st + C::SFB_OFF, sfsrc + (size_t)w.ks * C::SF_CH * 512, C::SF_CH * 512, &full[s]);
+          bulk_g2s(st + C::SFB_OFF, sfsrc + (size_t)w.ks * C::SF_CH * C::SFB_CHB, C::SF_CH * C::SFB_CHB, &full[s]);
       }
       __syncwarp();
       if (++s == NS) { s = 0; ph ^= 1; }
@@ -447,16 +452,20 @@ __global__ void __launch_bounds__(THREADS, 1)
         // order, so the previous stage's MMAs have read the old scales
 #pragma unroll
         for (int c = 0; c < C::SF_CH; ++c) {
-          sf_copy(tmem + (uint32_t)(SFA_COL + 4 * c), sf_desc(st + C::SFA_OFF + c * 512));
-          sf_copy(tmem + (uint32_t)(SFB_COL + 4 * c), sf_desc(st + C::SFB_OFF + c * 512));
+          sf_copy(tmem + (uint32_t)(C::SFA_COL + 4 * c), sf_desc(st + C::SFA_OFF + c * 512));
+#pragma unroll
+          for (int h = 0; h < C::SFB_HALVES; ++h)
+            sf_copy(tmem + (uint32_t)(C::SFB_COL + C::SFB_CPC * c + 4 * h),
+                    sf_desc(st + C::SFB_OFF + c * C::SFB_CHB + h * 512));
         }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           // MX: one scale per 32 k = byte j of the chunk's column; NV: chunk j, all 4 bytes
           const uint32_t sf_id = KIND == BS_MX ? (uint32_t)j : 0u;
-          const uint32_t col = KIND == BS_MX ? 0u : (uint32_t)(4 * j);
+          const uint32_t cola = KIND == BS_MX ? 0u : (uint32_t)(4 * j);
+          const uint32_t colb = KIND == BS_MX ? 0u : (uint32_t)(C::SFB_CPC * j);
           mma_bs<KIND>(tmem_d, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(2 * j), idesc_bs<KIND, BNT>(sf_id),
-                       (tmem + SFA_COL + col) | (sf_id << 30), (tmem + SFB_COL + col) | (sf_id << 30),
+                       (tmem + C::SFA_COL + cola) | (sf_id << 30), (tmem + C::SFB_COL + colb) | (sf_id << 30),
                        j > 0 ? 1u : acc0);
         }
         tc::mma_commit(&sfree[s]);
@@ -501,9 +510,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 // Activation scales in the order the block-scaled kernel copies them: for
-// token slot q, stage ks and chunk c, 512 bytes with 4 scales of each of the
-// slot's rows n at (n % 32) * 16 + (n / 32) * 4 (rows past the slot's valid
-// rows, and n >= bnt, are zero).  Dense: slot q = rows [q * bnt, q * bnt +
+// token slot q, stage ks and chunk c, 512 bytes per 128 rows (1024 for tiles
+// of more than 128 tokens, rows 128..255 in the second half) with 4 scales of
+// each row n at (n % 32) * 16 + (n / 32 % 4) * 4 of its half (rows past the
+// slot's valid rows, and n >= bnt, are zero).  Dense: slot q = rows [q * bnt, q * bnt +
 // bnt) of the activations.  MoE: slots enumerate the experts' token tiles in
 // expert order (rows offsets[e] + i * bnt, ...) and expert-sorted row r reads
 // caller row perm[r] / div.  One thread per 4-byte word.
@@ -534,11 +544,12 @@ __global__ void bs_sf_tiles_kernel(int slots, int bnt, int kst, int sf_ch, int l
     }
     __syncthreads();
   }
-  const size_t total = (size_t)slots * kst * sf_ch * 128;
+  const int rows = bnt > 128 ? 256 : 128;  // token rows per chunk (512 bytes per 128)
+  const size_t total = (size_t)slots * kst * sf_ch * rows;
   for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < total;
        idx += (size_t)gridDim.x * blockDim.x) {
-    const int n = (int)(idx & 127);
-    const size_t rest = idx >> 7;
+    const int n = (int)(idx % rows);
+    const size_t rest = idx / rows;
     const int c = (int)(rest % sf_ch);
     const size_t rest2 = rest / sf_ch;
     const int ks = (int)(rest2 % kst);
@@ -561,7 +572,7 @@ __global__ void bs_sf_tiles_kernel(int slots, int bnt, int kst, int sf_ch, int l
       }
       if (src >= 0) v = *reinterpret_cast<const uint32_t *>(sf + (size_t)src * ld + ((size_t)ks * sf_ch + c) * 4);
     }
-    out[(((size_t)q * kst + ks) * sf_ch + c) * 128 + (n & 31) * 4 + (n >> 5)] = v;
+    out[(((size_t)q * kst + ks) * sf_ch + c) * rows + (n >> 7) * 128 + (n & 31) * 4 + ((n & 127) >> 5)] = v;
   }
 }
 
@@ -629,6 +640,9 @@ static hq_status bs_launch_kind(const CUtensorMap &wm, const CUtensorMap &am, co
     case 32: return bs_launch_one<KIND, 32>(wm, am, p, t, st);
     case 64: return bs_launch_one<KIND, 64>(wm, am, p, t, st);
     case 128: return bs_launch_one<KIND, 128>(wm, am, p, t, st);
+    case 192:
+      if constexpr (KIND == BS_NV) return bs_launch_one<KIND, 192>(wm, am, p, t, st);
+      return HQ_ERR_UNSUPPORTED;
     default:
       if constexpr (KIND == BS_F8) return bs_launch_one<KIND, 256>(wm, am, p, t, st);
       return HQ_ERR_UNSUPPORTED;
@@ -639,7 +653,7 @@ size_t bs_sf_tiles_bytes(const Layout &L, const TcLaunch &t) {
   if (L.bs == BS_NONE || L.bs == BS_F8) return 0;
   const int kstage = L.bs == BS_MX ? 128 : 256;
   const int sf_ch = L.bs == BS_MX ? 1 : 4;
-  return (size_t)t.mtiles * (L.K / kstage) * sf_ch * 512;
+  return (size_t)t.mtiles * (L.K / kstage) * sf_ch * (t.bnt > 128 ? 1024 : 512);
 }
 
 // a_codes: `a_rows` activation rows (MXFP8, FP8: K E4M3 bytes per row; NVFP4:
@@ -661,7 +675,7 @@ hq_status launch_bs_gemm(const Layout &L, const void *packed, int E, const void 
   if (!make_bs_weight_map(&wm, L, packed, E)) return HQ_ERR_CUDA;
   if (!make_bs_act_map(&am, a_codes, a_rows, row_bytes, t.bnt)) return HQ_ERR_CUDA;
   if (L.bs != BS_F8) {
-    const size_t words = (size_t)t.mtiles * (L.K / kstage) * sf_ch * 128;
+    const size_t words = (size_t)t.mtiles * (L.K / kstage) * sf_ch * (t.bnt > 128 ? 256 : 128);
     size_t blocks = (words + 255) / 256;
     if (blocks > 148 * 8) blocks = 148 * 8;
     bs::bs_sf_tiles_kernel<<<(int)blocks, 256, moe ? (E + 1) * sizeof(int) : 0, st>>>(

@@ -98,6 +98,18 @@ def test_moe_small(wname, aname, a_per_slot):
     assert_close(res[(0, 1)].cpu(), out, bound, rel=8e-3, what="combined")
 
 
+@pytest.mark.parametrize("wname,aname", [("nvfp4", "nvfp4"), ("mxfp4", "mxfp8"), ("fp8", "fp8")])
+def test_moe_block_scaled_wide_token_tiles(wname, aname):
+    # ~150 routed rows per expert: NVFP4 x NVFP4 takes 192-token tiles
+    # (activation scale chunks of two 128-row halves), the other pairs
+    # 128-token tiles; Zipf routing gives some experts more than one tile
+    T, E, k, N, K = 300, 16, 8, 96, 256
+    res, out, bound, Y, B, ids, wts = moe_case(wname, aname, T, E, k, N, K, 0, seed=37, zipf=True)
+    assert torch.equal(res[(0, 0)], res[(1, 0)])
+    assert_close(res[(0, 0)].cpu(), Y, B, what="per-slot Y")
+    assert_close(res[(0, 1)].cpu(), out, bound, rel=8e-3, what="combined")
+
+
 def test_moe_single_expert_top1_equals_dense():
     import quantized_gemm_02_b200 as hq
     T, N, K = 17, 128, 512
