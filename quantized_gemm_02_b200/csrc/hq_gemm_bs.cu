@@ -1,6 +1,7 @@
-// Block-scaled tensor-core GEMM: MXFP4 weights x MXFP8 activations and
-// NVFP4 weights x NVFP4 activations, with the block scales applied by the
-// tensor core itself (no dequantisation anywhere).
+// Tensor-core GEMM with both operands fed straight from TMA: MXFP4 weights x
+// MXFP8 activations and NVFP4 weights x NVFP4 activations, with the block
+// scales applied by the tensor core itself (no dequantisation anywhere), and
+// FP8 weights x per-token FP8 activations.
 //
 // "Announcing Humming", section "Shared CUDA components across formats and
 // architectures": the microscaling formats feed block-scaled MMAs directly on
@@ -10,14 +11,16 @@
 //
 //   * tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale (MX, K = 32 per
 //     instruction, E2M1 weights expanded to one byte per code in shared
-//     memory by the TMA) or kind::mxf4nvf4.block_scale.scale_vec::4X (NV,
-//     K = 64, both operands packed E2M1); 128 weight rows are operand A,
-//     16..128 tokens operand B (NVFP4 MoE: 192; FP8: up to 256), both in
-//     shared memory with a 128-byte swizzle;
+//     memory by the TMA), kind::mxf4nvf4.block_scale.scale_vec::4X (NV,
+//     K = 64, both operands packed E2M1) or kind::f8f6f4 (FP8, K = 32, the
+//     per-row and per-token scales in the epilogue); 128 weight rows are
+//     operand A, 16..128 tokens operand B (NVFP4 MoE: 192; FP8: up to 256),
+//     both in shared memory with a 128-byte swizzle;
+//   * the weight codes are stored per 128-row tile in stage chunks, so one
+//     stage of a tile is one contiguous piece of HBM (one TMA box);
 //   * the scale chunks (128 rows x 4 scales, 512 bytes) go shared memory ->
 //     tensor memory with tcgen05.cp.32x128b.warpx4; the weight scales are
-//     stored in that order by the repack, the activation scales are gathered
-//     into it by the activation producer;
+//     stored in that order by the repack;
 //   * warps: 0..3 epilogue, 4 weight producer (3-D TMA of the codes, bulk copy
 //     of the scale chunks), 5 MMA issuer, 6 activation producer (2-D TMA of
 //     the codes, bulk copy of the scale chunks);
