@@ -51,6 +51,8 @@ WORKLOAD_TITLE = {
     "w4a16_asym_sweep": "dense W4A16 UINT4 asym g128 bf16-scale, (N,K) in {(8192,8192),(28672,8192),(8192,28672)}, "
                         "M in {1,4,16,64,256,1024,4096,8192}",
     "w4a16_dense_m16": "dense W4A16 INT4 sym g128, M=16, N=K=4096",
+    "moe_masked_nvfp4": "masked-layout MoE W4A4 NVFP4 x NVFP4 (activations quantised on the fly), E=256 slabs of "
+                        "256 rows, counts from a softmax top-8 routing of T=4096, H=7168, I=2048, gate-up + down",
 }
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -437,6 +439,60 @@ def workload_moe_nvfp4(hq, gen_seed=0):
     return ops, cfg, [w]
 
 
+def workload_moe_masked_nvfp4(hq, gen_seed=0):
+    """Masked-layout MoE (expert slabs with per-expert valid counts), NVFP4 x
+    NVFP4, config-5 MoE shapes: the counts come from a softmax top-8 routing
+    of T = 4096 tokens over E = 256 experts, slabs of 256 rows, expected_m =
+    the mean count.  Step = gate-up (N = 2I, K = H) + down (N = H, K = I)."""
+    dev = "cuda"
+    E, topk, H, I, T, slab = 256, 8, 7168, 2048, 4096, 256
+    gen = synth.generator(gen_seed, dev)
+    d = desc_of(hq, hq.HQ_E2M1, 16, hq.HQ_UE4M3, 0, 1, hq.HQ_NVFP4)
+    ids, _ = synth.routing_softmax_topk(T, E, topk, gen, device=dev)
+    counts = torch.bincount(ids.flatten().long(), minlength=E).clamp(max=slab).to(torch.int32)
+    touched = int((counts > 0).sum())
+    rows = int(counts.sum())
+    expected_m = max(1, rows // E)
+    parts = {}
+    for part, (N, K) in (("gate_up", (2 * I, H)), ("down", (H, I))):
+        w = synth.nvfp4_weights_random(E, N, K, gen, device=dev)
+        packed = torch.empty(hq.hq_packed_weights_bytes(d, E, N, K), dtype=torch.uint8, device=dev)
+        hq.hq_pack_weights(d, E, N, K, w["codes"], w["scales"], None, w["global"], packed)
+        del w
+        parts[part] = (packed, N, K, N * K // 2 + N * K // 16)
+    pg, Ng, Kg, bg = parts["gate_up"]
+    pd, Nd, Kd, bd = parts["down"]
+    x_gate = synth.bf16_normal((E * slab, Kg), gen, device=dev)
+    x_down = synth.bf16_normal((E * slab, Kd), gen, device=dev)
+    y = torch.empty(E * slab, Ng, dtype=torch.bfloat16, device=dev)
+    out = torch.empty(E * slab, Nd, dtype=torch.bfloat16, device=dev)
+    wsb = max(hq.hq_moe_masked_workspace_bytes(d, E, slab, Ng, Kg, expected_m),
+              hq.hq_moe_masked_workspace_bytes(d, E, slab, Nd, Kd, expected_m))
+    ws = torch.zeros(wsb, dtype=torch.uint8, device=dev)
+    counts_h = counts.cpu().pin_memory()
+    counts_e = torch.empty_like(counts)
+    x_h = x_gate.cpu().pin_memory()
+    out_h = torch.empty(E * slab, Nd, dtype=torch.bfloat16).pin_memory()
+
+    def run():
+        hq.hq_moe_gemm_masked(d, E, slab, Ng, Kg, pg, x_gate, counts, expected_m, y, ws, wsb)
+        hq.hq_moe_gemm_masked(d, E, slab, Nd, Kd, pd, x_down, counts, expected_m, out, ws, wsb)
+
+    def e2e():
+        counts_e.copy_(counts_h, non_blocking=True)
+        x_gate.copy_(x_h, non_blocking=True)
+        run()
+        out_h.copy_(out, non_blocking=True)
+
+    flops = 2.0 * rows * (Ng * Kg + Nd * Kd)
+    io = rows * (Kg // 2 + Ng * 2 + Kd // 2 + Nd * 2)
+    # per GEMM: routing prepare, amax + quantise, gather codes, scale relayout, GEMM
+    op = Op(f"moe_masked_nvfp4_T{T}_slab{slab}", run, flops, touched * (bg + bd), io, 2 * 6,
+            E * slab * Kg * 2 + E * 4, E * slab * Nd * 2, e2e, kernel="bs_gemm_kernel", peak_ratio=4.0)
+    cfg = {"workload": WORKLOAD_TITLE["moe_masked_nvfp4"], "l2": "flushed before every call"}
+    return [op], cfg, [parts, x_gate, x_down, y, out, ws, counts]
+
+
 def workload_dense_quantised(hq, fmt, gen_seed=0, N=7168, K=7168, Ms=(1, 32, 256, 2048, 8192)):
     """Config 5 dense: N = K = 7168, both operands N(0,1) quantised by the
     library's own quantiser (weights per output row), M swept."""
@@ -503,6 +559,7 @@ WORKLOADS = {
     "moe_w4a16_mxfp4": workload_moe_w4a16_mxfp4,
     "moe_w4a8_mxfp8": workload_moe_w4a8_mxfp8,
     "moe_nvfp4": workload_moe_nvfp4,
+    "moe_masked_nvfp4": workload_moe_masked_nvfp4,
     "w4a4_nvfp4": lambda hq: workload_dense_quantised(hq, "nvfp4"),
     "w8a8_fp8": lambda hq: workload_dense_quantised(hq, "fp8"),
 }

@@ -245,6 +245,30 @@ HQ_API hq_status hq_moe_gemm(hq_moe_mode mode, const hq_quant_desc *desc, int T,
                       hq_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Masked MoE expert GEMM (SGLang digest: humming_moe_runner_core_run with
+ * gemm type "grouped_masked", arguments expert_num_tokens and expected_m).
+ * The activations arrive already grouped per expert in fixed-size slabs:
+ *   a_bf16: bf16 [E * slab, K]; expert e owns rows [e * slab, (e + 1) * slab),
+ *       of which the first c_e = clamp(expert_num_tokens[e], 0, slab) are
+ *       valid (the rest may hold anything, NaN included, and are ignored).
+ *   expert_num_tokens: device int32 [E].
+ *   expected_m: the typical c_e (a tiling hint; < 1 means slab).
+ *   out_bf16: bf16 [E * slab, N]; row e * slab + i = a_row . W_e^T for
+ *       i < c_e; the other rows are left as they were.
+ * If desc->a_dtype is not BF16 the valid rows are quantised on the fly with
+ * hq_quant_act's recipe (NVFP4: the tensor scale of the valid rows alone).
+ * The result of a valid row equals hq_moe_gemm's for the same row and expert.
+ * E in [1, 1024], E * slab <= 2^30, K a multiple of 64; `workspace` of
+ * hq_moe_masked_workspace_bytes() bytes, 16-byte aligned.
+ * ---------------------------------------------------------------------- */
+HQ_API size_t hq_moe_masked_workspace_bytes(const hq_quant_desc *desc, int E, int slab, int N, int K,
+                                     int expected_m);
+HQ_API hq_status hq_moe_gemm_masked(const hq_quant_desc *desc, int E, int slab, int N, int K,
+                             const void *packed_w, const void *a_bf16,
+                             const int32_t *expert_num_tokens, int expected_m, void *out_bf16,
+                             void *workspace, size_t ws_bytes, hq_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Fused weighted top-k sum (SGLang digest: moe_fused_mul_sum, and
  * moe_unpermute): out[t, n] = routed_scale * sum_j w[t, j] * y[r(t, j), n]
  * with r(t, j) = inv_perm[t * topk + j] if inv_perm is non-NULL (y in

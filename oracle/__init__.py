@@ -25,6 +25,9 @@ library; citations name the page and its section):
 * MoE ("Announcing Humming", section "Performance"/WnA16 on Indexed and
   Grouped paths; SGLang PR #23754 digest, humming_moe_runner_core_run and
   moe_fused_mul_sum): out[t] = s_r * sum_j w[t, j] * (a[t] . W_{ids[t, j]}^T).
+  The masked layout (same digest, gemm type "grouped_masked" with
+  expert_num_tokens and expected_m): expert e multiplies the first
+  expert_num_tokens[e] rows of its own fixed-size slab of activation rows.
 * Activation quantisers (per-token FP8, MXFP8, NVFP4) use fp32 IEEE
   operations in the stated order with round-to-nearest-even and saturation;
   the pages name the activation formats ("Announcing Humming", sections
@@ -387,3 +390,32 @@ def moe(A_slots: np.ndarray, topk_ids: np.ndarray, topk_weights: np.ndarray, dec
     out = routed_scale * np.einsum("tj,tjn->tn", w, Y.reshape(T, k, N))
     bound = abs(routed_scale) * np.einsum("tj,tjn->tn", np.abs(w), B.reshape(T, k, N))
     return out, bound, Y, B
+
+
+def moe_masked(A_slab: np.ndarray, counts, slab: int, decode_expert, row_scale=None):
+    """Masked-layout MoE expert outputs (SGLang PR #23754 digest:
+    humming_moe_runner_core_run, gemm type "grouped_masked"): ``A_slab`` is
+    [E * slab, K] (fp64, already decoded); expert e's rows are
+    [e * slab, e * slab + c_e) with c_e = clamp(counts[e], 0, slab), and
+    Y[e * slab + i] = a . W_e^T for those rows.  Returns (Y, B, valid) with
+    Y and B NaN on the rows that are not valid, ``valid`` their mask.  The
+    reading that a count outside [0, slab] is clamped is this oracle's (the
+    pages state no rule)."""
+    E = len(counts)
+    R = E * slab
+    Y = None
+    B = None
+    valid = np.zeros(R, dtype=bool)
+    for e in range(E):
+        c = min(max(int(counts[e]), 0), slab)
+        rows = np.arange(e * slab, e * slab + c)
+        valid[rows] = True
+        W, col = decode_expert(e)
+        if Y is None:
+            Y = np.full((R, W.shape[0]), np.nan)
+            B = np.full((R, W.shape[0]), np.nan)
+        if c == 0:
+            continue
+        rs = None if row_scale is None else row_scale[rows]
+        Y[rows], B[rows] = gemm(A_slab[rows], W, rs, col)
+    return Y, B, valid

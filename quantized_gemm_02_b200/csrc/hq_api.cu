@@ -36,6 +36,10 @@ hq_status launch_bs_gemm(const Layout &L, const void *packed, int E, const void 
 size_t bs_sf_tiles_bytes(const Layout &L, const TcLaunch &t);
 hq_status launch_gather_bytes(int R, int row_bytes, const void *a, const int32_t *idx, int div, void *out,
                               cudaStream_t st);
+hq_status launch_quant_act_masked(int afmt, int E, int slab, int K, const void *x, const int32_t *counts,
+                                  void *codes, void *scales, float *global_out, void *workspace, cudaStream_t st);
+hq_status launch_moe_masked_prepare(int E, int slab, const int32_t *counts, int32_t *offsets, int32_t *perm,
+                                    cudaStream_t st);
 
 hq_status check_launch() {
   const cudaError_t e = cudaGetLastError();
@@ -134,6 +138,28 @@ static hq_status plan_moe(const hq_quant_desc *d, int T, int topk, int E, int N,
   return HQ_OK;
 }
 
+// Masked layout plan: E slabs of `slab` rows, of which expected_m are
+// typically valid (the token tile follows it); R = E * slab rows bound the
+// staging and the token tiles (at most ceil(slab / tile) per expert).
+static hq_status plan_moe_masked(const hq_quant_desc *d, int E, int slab, int N, int K, int expected_m,
+                                 MoePlan *pl) {
+  int fmt, afmt;
+  if (!d) return HQ_ERR_INVALID_ARG;
+  if (!weight_format(d, &fmt) || !act_format(d, &afmt)) return HQ_ERR_UNSUPPORTED;
+  if (E < 1 || E > 1024 || slab < 1 || N < 1 || !valid_k(d, K)) return HQ_ERR_INVALID_ARG;
+  if ((long)E * slab > (1L << 30)) return HQ_ERR_INVALID_ARG;
+  pl->L = layout_for(d, fmt, N, K);
+  pl->afmt = afmt;
+  pl->R = E * slab;
+  pl->src_rows = E * slab;
+  const int em = expected_m < 1 ? slab : (expected_m > slab ? slab : expected_m);
+  const int bnt = plan_tc(em, 1, N, pl->L.KB, true, pl->L.bs).bnt;
+  long bound = (long)E * ((slab + bnt - 1) / bnt);
+  if (bound > pl->R) bound = pl->R;
+  pl->s = plan_tc(em, (int)bound, N, pl->L.KB, true, pl->L.bs);
+  return HQ_OK;
+}
+
 struct MoeWs {
   void *split, *y, *a_bf16, *codes, *scales, *glob, *amax;
   void *s_codes, *s_scales;  // block-scaled layouts: expert-sorted codes, scale chunks per token tile
@@ -163,6 +189,64 @@ static size_t moe_ws(const MoePlan &pl, hq_moe_mode mode, int K, int N, int comb
     w->codes = w->scales = w->glob = w->amax = nullptr;
   }
   return c.off;
+}
+
+// The GEMM part of every MoE mode, given the routing (offsets, perm): rows
+// are staged expert-contiguous in the workspace (quantised on the fly when
+// the description asks: `counts` selects the masked layout's quantiser),
+// then the grouped tensor-core GEMM, then the optional weighted combine.
+static hq_status moe_run(const MoePlan &pl, int T, int topk, int E, int N, int K, const void *packed_w,
+                         const void *a_bf16, int div, const int32_t *counts, const int32_t *expert_offsets,
+                         const int32_t *perm, const float *topk_weights, float routed_scale, int combine,
+                         void *out_bf16, const MoeWs &w, cudaStream_t st) {
+  const void *a_use = a_bf16;
+  const float *row_scale = nullptr;
+  const float *a_global = nullptr;
+  // The tensor-core kernel reads activation tiles by TMA from expert-sorted
+  // rows in both modes: the rows are gathered (and, for quantised
+  // activations, quantised on the fly and decoded exactly) into the
+  // workspace first.  Results do not depend on the mode.
+  const int a_indexed = 0;
+  hq_status s = HQ_OK;
+  void *y = combine ? w.y : out_bf16;
+  auto quant = [&]() {
+    if (counts)
+      return launch_quant_act_masked(pl.afmt, E, pl.src_rows / E, K, a_bf16, counts, w.codes, w.scales,
+                                     (float *)w.glob, w.amax, st);
+    return launch_quant_act(pl.afmt, pl.src_rows, K, a_bf16, w.codes, w.scales, (float *)w.glob, nullptr, w.amax,
+                            st);
+  };
+  if (pl.L.bs != BS_NONE) {
+    // quantise the caller rows once, gather codes and scales into expert order
+    s = quant();
+    if (s != HQ_OK) return s;
+    s = launch_gather_bytes(pl.R, (int)act_code_bytes(pl.afmt, K), w.codes, perm, div, w.s_codes, st);
+    if (s != HQ_OK) return s;
+    s = launch_bs_gemm(pl.L, packed_w, E, w.s_codes, pl.R, w.scales, div,
+                       pl.afmt == A_NVFP4 ? (const float *)w.glob : nullptr, 0, 1, expert_offsets, perm, y, pl.s,
+                       w.split, w.s_scales, st);
+    if (s != HQ_OK) return s;
+    if (combine) s = launch_unpermute_sum(T, topk, N, y, nullptr, topk_weights, routed_scale, out_bf16, st);
+    return s;
+  }
+  if (pl.afmt != A_BF16) {
+    s = quant();
+    if (s != HQ_OK) return s;
+    s = launch_act_decode(pl.afmt, pl.R, K, w.codes, w.scales, perm, div, w.a_bf16, st);
+    if (s != HQ_OK) return s;
+    if (pl.afmt == A_FP8) row_scale = (const float *)w.scales;
+    if (pl.afmt == A_NVFP4) a_global = (const float *)w.glob;
+  } else {
+    s = launch_gather_rows(pl.R, K, a_bf16, perm, div, w.a_bf16, st);
+    if (s != HQ_OK) return s;
+  }
+  a_use = w.a_bf16;
+  const int a_rows = (a_indexed ? pl.src_rows : pl.R);
+  s = launch_tc_gemm(pl.L, packed_w, a_use, a_rows, row_scale, a_global, 0, 1, E, expert_offsets, perm, div, a_indexed,
+                     y, pl.s, w.split, st);
+  if (s != HQ_OK) return s;
+  if (combine) s = launch_unpermute_sum(T, topk, N, y, nullptr, topk_weights, routed_scale, out_bf16, st);
+  return s;
 }
 
 }  // namespace hq
@@ -344,49 +428,42 @@ hq_status hq_moe_gemm(hq_moe_mode mode, const hq_quant_desc *desc, int T, int to
   const size_t need = moe_ws(pl, mode, K, N, combine, (uint8_t *)workspace, &w);
   if (!workspace || ws_bytes < need || !aligned16(workspace)) return HQ_ERR_WORKSPACE;
   if (!device_is_sm100()) return HQ_ERR_ARCH;
+  return moe_run(pl, T, topk, E, N, K, packed_w, a_bf16, a_per_slot ? 1 : topk, nullptr, expert_offsets, perm,
+                 topk_weights, routed_scale, combine, out_bf16, w, (cudaStream_t)stream);
+}
+
+size_t hq_moe_masked_workspace_bytes(const hq_quant_desc *desc, int E, int slab, int N, int K, int expected_m) {
+  MoePlan pl;
+  if (plan_moe_masked(desc, E, slab, N, K, expected_m, &pl) != HQ_OK) return 0;
+  MoeWs w;
+  Carver c{nullptr};
+  c.off = moe_ws(pl, HQ_MOE_GROUPED, K, N, 0, nullptr, &w);
+  c.take((size_t)(E + 1) * sizeof(int32_t));
+  c.take((size_t)E * slab * sizeof(int32_t));
+  return c.off;
+}
+
+hq_status hq_moe_gemm_masked(const hq_quant_desc *desc, int E, int slab, int N, int K, const void *packed_w,
+                             const void *a_bf16, const int32_t *expert_num_tokens, int expected_m, void *out_bf16,
+                             void *workspace, size_t ws_bytes, hq_stream_t stream) {
+  MoePlan pl;
+  const hq_status ps = plan_moe_masked(desc, E, slab, N, K, expected_m, &pl);
+  if (ps != HQ_OK) return ps;
+  if (!packed_w || !a_bf16 || !expert_num_tokens || !out_bf16) return HQ_ERR_INVALID_ARG;
+  if (!aligned16(packed_w) || !aligned16(a_bf16) || !aligned16(out_bf16)) return HQ_ERR_INVALID_ARG;
+  MoeWs w;
+  Carver c{(uint8_t *)workspace};
+  c.off = moe_ws(pl, HQ_MOE_GROUPED, K, N, 0, (uint8_t *)workspace, &w);
+  int32_t *offsets = (int32_t *)c.take((size_t)(E + 1) * sizeof(int32_t));
+  int32_t *perm = (int32_t *)c.take((size_t)E * slab * sizeof(int32_t));
+  if (!workspace || ws_bytes < c.off || !aligned16(workspace)) return HQ_ERR_WORKSPACE;
+  if (!device_is_sm100()) return HQ_ERR_ARCH;
   cudaStream_t st = (cudaStream_t)stream;
-  const int div = a_per_slot ? 1 : topk;
-  const void *a_use = a_bf16;
-  const float *row_scale = nullptr;
-  const float *a_global = nullptr;
-  // The tensor-core kernel reads activation tiles by TMA from expert-sorted
-  // rows in both modes: the rows are gathered (and, for quantised
-  // activations, quantised on the fly and decoded exactly) into the
-  // workspace first.  Results do not depend on the mode.
-  const int a_indexed = 0;
-  hq_status s = HQ_OK;
-  void *y = combine ? w.y : out_bf16;
-  if (pl.L.bs != BS_NONE) {
-    // quantise the caller rows once, gather codes and scales into expert order
-    s = launch_quant_act(pl.afmt, pl.src_rows, K, a_bf16, w.codes, w.scales, (float *)w.glob, nullptr, w.amax, st);
-    if (s != HQ_OK) return s;
-    s = launch_gather_bytes(pl.R, (int)act_code_bytes(pl.afmt, K), w.codes, perm, div, w.s_codes, st);
-    if (s != HQ_OK) return s;
-    s = launch_bs_gemm(pl.L, packed_w, E, w.s_codes, pl.R, w.scales, div,
-                       pl.afmt == A_NVFP4 ? (const float *)w.glob : nullptr, 0, 1, expert_offsets, perm, y, pl.s,
-                       w.split, w.s_scales, st);
-    if (s != HQ_OK) return s;
-    if (combine) s = launch_unpermute_sum(T, topk, N, y, nullptr, topk_weights, routed_scale, out_bf16, st);
-    return s;
-  }
-  if (pl.afmt != A_BF16) {
-    s = launch_quant_act(pl.afmt, pl.src_rows, K, a_bf16, w.codes, w.scales, (float *)w.glob, nullptr, w.amax, st);
-    if (s != HQ_OK) return s;
-    s = launch_act_decode(pl.afmt, pl.R, K, w.codes, w.scales, perm, div, w.a_bf16, st);
-    if (s != HQ_OK) return s;
-    if (pl.afmt == A_FP8) row_scale = (const float *)w.scales;
-    if (pl.afmt == A_NVFP4) a_global = (const float *)w.glob;
-  } else {
-    s = launch_gather_rows(pl.R, K, a_bf16, perm, div, w.a_bf16, st);
-    if (s != HQ_OK) return s;
-  }
-  a_use = w.a_bf16;
-  const int a_rows = (a_indexed ? pl.src_rows : pl.R);
-  s = launch_tc_gemm(pl.L, packed_w, a_use, a_rows, row_scale, a_global, 0, 1, E, expert_offsets, perm, div, a_indexed,
-                     y, pl.s, w.split, st);
+  const hq_status s = launch_moe_masked_prepare(E, slab, expert_num_tokens, offsets, perm, st);
   if (s != HQ_OK) return s;
-  if (combine) s = launch_unpermute_sum(T, topk, N, y, nullptr, topk_weights, routed_scale, out_bf16, st);
-  return s;
+  // every valid row is its own slot: one row per slot (div = 1), no combine
+  return moe_run(pl, E * slab, 1, E, N, K, packed_w, a_bf16, 1, expert_num_tokens, offsets, perm, nullptr, 1.f, 0,
+                 out_bf16, w, st);
 }
 
 hq_status hq_moe_unpermute_sum(int T, int topk, int N, const void *y_bf16, const int32_t *inv_perm,

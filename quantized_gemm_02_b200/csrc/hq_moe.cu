@@ -147,6 +147,42 @@ hq_status launch_moe_permute(int T, int topk, int E, const int32_t *ids, int32_t
   return check_launch();
 }
 
+// Masked MoE layout (SGLang digest: humming_moe_runner_core_run, gemm type
+// "grouped_masked"): expert e owns rows [e * slab, e * slab + c_e) of an
+// [E * slab, K] block, c_e = clamp(counts[e], 0, slab).  Writes the grouped
+// path's routing for it: offsets [E + 1], the exclusive prefix of c_e, and
+// perm[offsets[e] + i] = e * slab + i; the positions past the total get row
+// 0 (staged but never multiplied).  One block per expert, each summing the
+// counts before its own; E <= 1024.
+__global__ void moe_masked_prepare_kernel(int E, int slab, const int32_t *__restrict__ counts,
+                                          int32_t *__restrict__ offsets, int32_t *__restrict__ perm) {
+  __shared__ int s_base;
+  const int e = blockIdx.x;
+  if (threadIdx.x < 32) {
+    int sum = 0;
+    for (int j = threadIdx.x; j < e; j += 32) sum += min(max(counts[j], 0), slab);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (threadIdx.x == 0) s_base = sum;
+  }
+  __syncthreads();
+  const int base = s_base;
+  const int c = min(max(counts[e], 0), slab);
+  for (int i = threadIdx.x; i < c; i += blockDim.x) perm[base + i] = e * slab + i;
+  if (threadIdx.x == 0) {
+    offsets[e] = base;
+    if (e == E - 1) offsets[E] = base + c;
+  }
+  if (e == E - 1)
+    for (int r = base + c + threadIdx.x; r < E * slab; r += blockDim.x) perm[r] = 0;
+}
+
+hq_status launch_moe_masked_prepare(int E, int slab, const int32_t *counts, int32_t *offsets, int32_t *perm,
+                                    cudaStream_t st) {
+  moe_masked_prepare_kernel<<<E, 256, 0, st>>>(E, slab, counts, offsets, perm);
+  return check_launch();
+}
+
 hq_status launch_unpermute_sum(int T, int topk, int N, const void *y, const int32_t *inv, const float *w, float rs,
                                void *out, cudaStream_t st) {
   if (T == 0) return HQ_OK;

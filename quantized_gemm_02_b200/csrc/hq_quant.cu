@@ -159,6 +159,27 @@ __global__ void amax_kernel(size_t n8, const uint16_t *__restrict__ x, unsigned 
   if ((threadIdx.x & 31) == 0 && a > 0.f) atomicMax(amax_bits, __float_as_uint(a));
 }
 
+// Pass 1 for the masked MoE layout: the amax over the valid rows only (row i
+// of expert e's slab is valid for i < clamp(counts[e], 0, slab)).
+__global__ void amax_rows_kernel(int slab, int K, size_t n8, const uint16_t *__restrict__ x,
+                                 const int32_t *__restrict__ counts, unsigned int *__restrict__ amax_bits) {
+  const size_t row8 = (size_t)K / 8;
+  float a = 0.f;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8; i += (size_t)gridDim.x * blockDim.x) {
+    const size_t row = i / row8;
+    const int e = (int)(row / slab), r = (int)(row % slab);
+    const int c = min(max(counts[e], 0), slab);
+    if (r >= c) continue;
+    const uint4 v = reinterpret_cast<const uint4 *>(x)[i];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) a = fmaxf(a, fmaxf(fabsf(bf16_lo(w[j])), fabsf(bf16_hi(w[j]))));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+  if ((threadIdx.x & 31) == 0 && a > 0.f) atomicMax(amax_bits, __float_as_uint(a));
+}
+
 __device__ __forceinline__ float nvfp4_global(const unsigned int *amax_bits, const float *static_global) {
   if (static_global) return *static_global;
   const float amax = __uint_as_float(*amax_bits);
@@ -302,6 +323,26 @@ hq_status launch_quant_act(int afmt, int M, int K, const void *x, void *codes, v
     default:
       return HQ_ERR_UNSUPPORTED;
   }
+  return check_launch();
+}
+
+
+// Quantisation of a masked MoE block [E * slab, K]: every row is quantised
+// (the rows past an expert's count are never read by the GEMM), but the NVFP4
+// tensor scale comes from the valid rows alone, so that it is the one the
+// valid rows would get on their own.
+hq_status launch_quant_act_masked(int afmt, int E, int slab, int K, const void *x, const int32_t *counts,
+                                  void *codes, void *scales, float *global_out, void *workspace, cudaStream_t st) {
+  const int M = E * slab;
+  if (afmt != A_NVFP4) return launch_quant_act(afmt, M, K, x, codes, scales, global_out, nullptr, workspace, st);
+  const uint16_t *xb = (const uint16_t *)x;
+  unsigned int *amax = (unsigned int *)workspace;
+  if (cudaMemsetAsync(amax, 0, sizeof(unsigned int), st) != cudaSuccess) return HQ_ERR_CUDA;
+  const size_t n8 = (size_t)M * K / 8;
+  amax_rows_kernel<<<quant_grid(n8, 256), 256, 0, st>>>(slab, K, n8, xb, counts, amax);
+  const size_t nb = (size_t)M * K / 16;
+  quant_nvfp4_kernel<<<quant_grid(nb, 128), 128, 0, st>>>(nb, xb, (uint8_t *)codes, (uint8_t *)scales, amax,
+                                                       nullptr, global_out);
   return check_launch();
 }
 

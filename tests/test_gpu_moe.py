@@ -159,3 +159,48 @@ def test_config3_shapes_gate_up(T):
 
     ref, bound, _, _ = O.moe(np.repeat(A, k, axis=0), ids.numpy(), wts.numpy(), dec, 1.0)
     assert_close(out[0].cpu()[:, torch.as_tensor(cols)], ref, bound, rel=8e-3, what=f"config3 T={T}")
+
+
+@pytest.mark.parametrize("wname,aname", [("mxfp4", "bf16"), ("int4_g128", "bf16"), ("uint4_g64", "bf16"),
+                                         ("mxfp4", "mxfp8"), ("nvfp4", "nvfp4"), ("fp8", "fp8"),
+                                         ("nvfp4", "fp8")])
+def test_moe_masked(wname, aname):
+    # masked layout: E slabs of `slab` rows, expert e uses its first c_e rows;
+    # empty and full slabs, NaN in every unused row, the output's unused rows
+    # keep their contents.  Quantised activations: the oracle quantises the
+    # valid rows alone (NVFP4: their own tensor scale).
+    import quantized_gemm_02_b200 as hq
+    E, slab, N, K = 8, 48, 96, 256
+    counts = np.array([0, 48, 17, 1, 30, 48, 5, 22], dtype=np.int32)
+    g = synth.generator(51)
+    x = synth.bf16_normal((E * slab, K), g)
+    valid = np.concatenate([np.arange(e * slab, e * slab + counts[e]) for e in range(E)])
+    mask = np.zeros(E * slab, dtype=bool)
+    mask[valid] = True
+    x[torch.as_tensor(np.nonzero(~mask)[0])] = float("nan")
+    w = make_weights(wname, E, N, K, seed=52)
+    packed = gpu_pack(wname, w, E, N, K, aname)
+    d = cdesc(wname, aname)
+    wsb = hq.hq_moe_masked_workspace_bytes(d, E, slab, N, K, 24)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+    out = torch.full((E * slab, N), 7.0, dtype=torch.bfloat16, device="cuda")
+    hq.hq_moe_gemm_masked(d, E, slab, N, K, packed, x.cuda(), torch.as_tensor(counts).cuda(), 24, out, ws, wsb)
+    torch.cuda.synchronize()
+    assert hq.hq_device_error() == 0
+    xb = np_bits(x[torch.as_tensor(valid)])
+    if aname == "bf16":
+        A_valid, row_valid = O.decode_act("bf16", len(valid), K, xb)
+    else:
+        q, s, og = oracle_quant(aname, xb)
+        A_valid, row_valid = O.decode_act(aname, len(valid), K, q, s, og)
+    A_slab = np.full((E * slab, K), np.nan)
+    A_slab[valid] = A_valid
+    row_slab = None
+    if row_valid is not None:
+        row_slab = np.full(E * slab, np.nan)
+        row_slab[valid] = row_valid
+    Y, B, vmask = O.moe_masked(A_slab, counts, slab, oracle_decoder(wname, w, N, K), row_scale=row_slab)
+    assert np.array_equal(vmask, mask)
+    got = out.cpu()
+    assert_close(got[torch.as_tensor(valid)], Y[valid], B[valid], what=f"masked {wname}x{aname}")
+    assert torch.all(got[torch.as_tensor(np.nonzero(~mask)[0])].float() == 7.0)

@@ -225,3 +225,36 @@ def test_moe_permute_bruteforce():
     assert np.array_equal(perm[inv], np.arange(T * k))
     # each token's k experts are distinct
     assert all(len(set(r)) == k for r in ids.tolist())
+
+
+def test_moe_masked_matches_routed_top1_and_ignores_invalid_rows():
+    # a top-1 routing laid out as slabs (expert e's tokens in token order,
+    # padded to the slab) gives the routed MoE's per-slot outputs exactly;
+    # NaN in the padding rows reaches no valid row; counts past the slab clamp
+    T, E, N, K, slab = 11, 4, 8, 64, 6
+    ab, af = _a(T, K, seed=6)
+    g = synth.generator(7)
+    w = synth.mxfp4_weights(E, N, K, g)
+    d = O.Desc("e2m1", 32, "e8m0")
+    dec = lambda e: O.decode_weights(d, N, K, w["codes"][e].numpy(), w["scales"][e].numpy())
+    ids = np.array([[2], [0], [2], [3], [2], [0], [2], [2], [0], [3], [2]], dtype=np.int32)
+    Y_routed, B_routed = O.moe_expert_outputs(af, ids, dec)
+    A_slab = np.full((E * slab, K), np.nan)
+    counts = np.zeros(E, dtype=np.int64)
+    where = {}
+    for t in range(T):
+        e = int(ids[t, 0])
+        if counts[e] < slab:
+            where[t] = e * slab + counts[e]
+            A_slab[where[t]] = af[t]
+        counts[e] += 1
+    Y, B, valid = O.moe_masked(A_slab, counts, slab, dec)
+    assert counts[2] == 6 and counts[0] == 3 and counts[1] == 0
+    assert valid.sum() == sum(min(int(c), slab) for c in counts)
+    for t, r in where.items():
+        assert valid[r]
+        assert np.array_equal(Y[r], Y_routed[t]) and np.array_equal(B[r], B_routed[t])
+    assert np.isnan(Y[~valid]).all() and not np.isnan(Y[valid]).any()
+    # a count above the slab takes the slab; a negative count none
+    Y2, _, valid2 = O.moe_masked(A_slab, np.array([3, -4, 99, 2]), slab, dec)
+    assert valid2.sum() == 3 + 0 + slab + 2
