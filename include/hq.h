@@ -269,6 +269,17 @@ HQ_API hq_status hq_moe_gemm_masked(const hq_quant_desc *desc, int E, int slab, 
                              void *workspace, size_t ws_bytes, hq_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * SiLU-and-mul between an MoE layer's gate-up and down GEMMs (the gate-up
+ * GEMM computes N = 2I columns per row: gate then up).  y bf16 [R, 2I],
+ * out bf16 [R, I]: out[r, i] = bf16_rne(silu(g) * u) with g = y[r, i],
+ * u = y[r, I + i], silu(g) = g / (1 + exp(-g)), computed in fp32.  I a
+ * multiple of 8; both buffers 16-byte aligned.  (The pages name no
+ * activation; this is the usual gated-MLP form, an addition of this
+ * library.)
+ * ---------------------------------------------------------------------- */
+HQ_API hq_status hq_silu_and_mul(int R, int I, const void *y_bf16, void *out_bf16, hq_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Fused weighted top-k sum (SGLang digest: moe_fused_mul_sum, and
  * moe_unpermute): out[t, n] = routed_scale * sum_j w[t, j] * y[r(t, j), n]
  * with r(t, j) = inv_perm[t * topk + j] if inv_perm is non-NULL (y in

@@ -419,3 +419,15 @@ def moe_masked(A_slab: np.ndarray, counts, slab: int, decode_expert, row_scale=N
         rs = None if row_scale is None else row_scale[rows]
         Y[rows], B[rows] = gemm(A_slab[rows], W, rs, col)
     return Y, B, valid
+
+
+def silu_and_mul(Y: np.ndarray) -> np.ndarray:
+    """Gated activation between an MoE layer's gate-up and down GEMMs, in
+    fp64: for Y [R, 2I] (gate columns first, then up), out[r, i] =
+    silu(Y[r, i]) * Y[r, I + i] with silu(g) = g / (1 + exp(-g)).  The pages
+    name no activation; this is the usual gated-MLP form (a reading)."""
+    Y = np.asarray(Y, dtype=np.float64)
+    I = Y.shape[1] // 2
+    g, u = Y[:, :I], Y[:, I:]
+    with np.errstate(over="ignore"):
+        return g / (1.0 + np.exp(-g)) * u

@@ -17,7 +17,7 @@ __all__ = [
     "HQ_NVFP4", "HQ_MOE_GROUPED", "HQ_MOE_INDEXED",
     "hq_status_string", "hq_device_error", "hq_packed_weights_bytes", "hq_pack_weights", "hq_unpack_weights",
     "hq_quant_act", "hq_gemm_workspace_bytes", "hq_gemm", "hq_moe_permute", "hq_moe_workspace_bytes",
-    "hq_moe_gemm", "hq_moe_masked_workspace_bytes", "hq_moe_gemm_masked", "hq_moe_unpermute_sum",
+    "hq_moe_gemm", "hq_moe_masked_workspace_bytes", "hq_moe_gemm_masked", "hq_silu_and_mul", "hq_moe_unpermute_sum",
     "hq_gemm_noalloc", "hq_selftest_wait_timeout",
 ]
 
@@ -33,7 +33,7 @@ STATUS = {
 EXPORTS = (
     "hq_status_string", "hq_device_error", "hq_packed_weights_bytes", "hq_pack_weights", "hq_unpack_weights",
     "hq_quant_act", "hq_gemm_workspace_bytes", "hq_gemm", "hq_moe_permute", "hq_moe_workspace_bytes",
-    "hq_moe_gemm", "hq_moe_masked_workspace_bytes", "hq_moe_gemm_masked", "hq_moe_unpermute_sum",
+    "hq_moe_gemm", "hq_moe_masked_workspace_bytes", "hq_moe_gemm_masked", "hq_silu_and_mul", "hq_moe_unpermute_sum",
     "hq_gemm_noalloc", "hq_selftest_wait_timeout",
 )
 
@@ -89,6 +89,7 @@ def _lib() -> ctypes.CDLL:
             "hq_moe_gemm": (I, [I, D, I, I, I, I, I, P, P, I, P, P, P, P, F, I, P, P, Z, P]),
             "hq_moe_masked_workspace_bytes": (Z, [D, I, I, I, I, I]),
             "hq_moe_gemm_masked": (I, [D, I, I, I, I, P, P, P, I, P, P, Z, P]),
+            "hq_silu_and_mul": (I, [I, I, P, P, P]),
             "hq_moe_unpermute_sum": (I, [I, I, I, P, P, P, F, P, P]),
             "hq_gemm_noalloc": (I, [D, I, I, I, P, P, P, P, P, P]),
             "hq_selftest_wait_timeout": (I, [ctypes.c_ulonglong, P]),
@@ -186,6 +187,10 @@ def hq_moe_gemm_masked(desc, E, slab, N, K, packed_w, a, expert_num_tokens, expe
     _check("hq_moe_gemm_masked", _lib().hq_moe_gemm_masked(
         ctypes.byref(desc), E, slab, N, K, _ptr(packed_w), _ptr(a), _ptr(expert_num_tokens), expected_m, _ptr(out),
         _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def hq_silu_and_mul(R, I, y, out, stream=None):
+    _check("hq_silu_and_mul", _lib().hq_silu_and_mul(R, I, _ptr(y), _ptr(out), _stream(stream)))
 
 
 def hq_moe_gemm(mode, desc, T, topk, E, N, K, packed_w, a, a_per_slot, expert_offsets, perm, inv_perm,

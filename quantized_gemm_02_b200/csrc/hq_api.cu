@@ -40,6 +40,7 @@ hq_status launch_quant_act_masked(int afmt, int E, int slab, int K, const void *
                                   void *codes, void *scales, float *global_out, void *workspace, cudaStream_t st);
 hq_status launch_moe_masked_prepare(int E, int slab, const int32_t *counts, int32_t *offsets, int32_t *perm,
                                     cudaStream_t st);
+hq_status launch_silu_and_mul(int R, int I, const void *y, void *out, cudaStream_t st);
 
 hq_status check_launch() {
   const cudaError_t e = cudaGetLastError();
@@ -464,6 +465,14 @@ hq_status hq_moe_gemm_masked(const hq_quant_desc *desc, int E, int slab, int N, 
   // every valid row is its own slot: one row per slot (div = 1), no combine
   return moe_run(pl, E * slab, 1, E, N, K, packed_w, a_bf16, 1, expert_num_tokens, offsets, perm, nullptr, 1.f, 0,
                  out_bf16, w, st);
+}
+
+hq_status hq_silu_and_mul(int R, int I, const void *y_bf16, void *out_bf16, hq_stream_t stream) {
+  if (R < 0 || I < 8 || (I % 8) != 0) return HQ_ERR_INVALID_ARG;
+  if (R == 0) return HQ_OK;
+  if (!y_bf16 || !out_bf16 || !aligned16(y_bf16) || !aligned16(out_bf16)) return HQ_ERR_INVALID_ARG;
+  if (!device_is_sm100()) return HQ_ERR_ARCH;
+  return launch_silu_and_mul(R, I, y_bf16, out_bf16, (cudaStream_t)stream);
 }
 
 hq_status hq_moe_unpermute_sum(int T, int topk, int N, const void *y_bf16, const int32_t *inv_perm,

@@ -183,6 +183,43 @@ hq_status launch_moe_masked_prepare(int E, int slab, const int32_t *counts, int3
   return check_launch();
 }
 
+// SiLU-and-mul between the gate-up and the down GEMM of an MoE layer:
+// out[r, i] = bf16(silu(g) * u), g = y[r, i], u = y[r, I + i], in fp32 with
+// silu(g) = g / (1 + exp(-g)) (expf, IEEE division); 8 columns per thread.
+__global__ void silu_and_mul_kernel(int R, int I, const uint16_t *__restrict__ y, uint16_t *__restrict__ out) {
+  const int per_row = I / 8;
+  const size_t total = (size_t)R * per_row;
+  for (size_t c = blockIdx.x * (size_t)blockDim.x + threadIdx.x; c < total; c += (size_t)gridDim.x * blockDim.x) {
+    const int r = (int)(c / per_row), ch = (int)(c % per_row);
+    const uint4 gv = reinterpret_cast<const uint4 *>(y + (size_t)r * 2 * I)[ch];
+    const uint4 uv = reinterpret_cast<const uint4 *>(y + (size_t)r * 2 * I + I)[ch];
+    const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w}, uw[4] = {uv.x, uv.y, uv.z, uv.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float res[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float g = __uint_as_float(h ? (gw[i] & 0xFFFF0000u) : (gw[i] << 16));
+        const float u = __uint_as_float(h ? (uw[i] & 0xFFFF0000u) : (uw[i] << 16));
+        res[h] = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.f, expf(-g))), u);
+      }
+      o[i] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(res[0])) |
+             ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(res[1])) << 16);
+    }
+    reinterpret_cast<uint4 *>(out + (size_t)r * I)[ch] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+hq_status launch_silu_and_mul(int R, int I, const void *y, void *out, cudaStream_t st) {
+  if (R == 0) return HQ_OK;
+  const size_t total = (size_t)R * (I / 8);
+  size_t blocks = (total + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  silu_and_mul_kernel<<<(int)blocks, 256, 0, st>>>(R, I, (const uint16_t *)y, (uint16_t *)out);
+  return check_launch();
+}
+
 hq_status launch_unpermute_sum(int T, int topk, int N, const void *y, const int32_t *inv, const float *w, float rs,
                                void *out, cudaStream_t st) {
   if (T == 0) return HQ_OK;

@@ -204,3 +204,19 @@ def test_moe_masked(wname, aname):
     got = out.cpu()
     assert_close(got[torch.as_tensor(valid)], Y[valid], B[valid], what=f"masked {wname}x{aname}")
     assert torch.all(got[torch.as_tensor(np.nonzero(~mask)[0])].float() == 7.0)
+
+
+def test_silu_and_mul():
+    # fp32 on the GPU, fp64 in the oracle, both rounded once to bf16: within
+    # one bf16 step (2^-7 relative); extreme gates included
+    import quantized_gemm_02_b200 as hq
+    R, I = 37, 136
+    y = synth.bf16_normal((R, 2 * I), synth.generator(61)) * 3
+    y[0, :8] = torch.tensor([0.0, 100.0, -100.0, 1e-3, -1e-3, 88.0, -90.0, 7.0], dtype=torch.bfloat16)
+    out = torch.empty(R, I, dtype=torch.bfloat16, device="cuda")
+    hq.hq_silu_and_mul(R, I, y.cuda(), out)
+    torch.cuda.synchronize()
+    ref = O.silu_and_mul(y.float().numpy().astype(np.float64))
+    got = out.cpu().float().numpy().astype(np.float64)
+    tol = np.maximum(np.abs(ref) * 2.0 ** -7, 1e-30)
+    assert np.all(np.abs(got - ref) <= tol), float(np.max(np.abs(got - ref) / tol))

@@ -258,3 +258,17 @@ def test_moe_masked_matches_routed_top1_and_ignores_invalid_rows():
     # a count above the slab takes the slab; a negative count none
     Y2, _, valid2 = O.moe_masked(A_slab, np.array([3, -4, 99, 2]), slab, dec)
     assert valid2.sum() == 3 + 0 + slab + 2
+
+
+def test_silu_and_mul_closed_forms():
+    g = np.array([0.0, 1.0, -1.0, 2.5, -2.5, 40.0, -40.0, -800.0])
+    u = np.array([3.0, 1.0, 1.0, -2.0, 0.5, 1.0, 1.0, 2.0])
+    out = O.silu_and_mul(np.concatenate([g, u])[None, :])[0]
+    assert out[0] == 0.0
+    assert out[1] == pytest.approx(0.7310585786300049, abs=1e-15)  # sigma(1) = 1 / (1 + 1/e)
+    # silu(-x) = silu(x) - x (sigma(-x) = 1 - sigma(x)), times the up value
+    assert out[2] == pytest.approx(0.7310585786300049 - 1.0, abs=1e-15)
+    assert out[4] / 0.5 == pytest.approx(out[3] / -2.0 - 2.5, abs=1e-12)
+    # large |g|: silu(g) -> g, silu(-g) -> 0 (no overflow trouble)
+    assert out[5] == pytest.approx(40.0, rel=1e-15)
+    assert abs(out[6]) < 1e-15 and out[7] == 0.0
