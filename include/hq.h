@@ -106,6 +106,23 @@ typedef struct {
 
 typedef enum { HQ_MOE_GROUPED = 0, HQ_MOE_INDEXED = 1 } hq_moe_mode;
 
+/*
+ * Compute options ("Announcing Humming", section "Tuning & JIT per
+ * workload": the compute configuration holds the GEMM type and options such
+ * as batch invariance).  Zero-initialise; unknown fields must stay zero.
+ *   batch_invariant: 1 = every output row is bit-identical whatever the
+ *       number of rows M of the call (and whatever the other rows hold): one
+ *       fixed token tile (64 rows) and no split of K, each tile summed in k
+ *       order by one CTA.  Slower at small M, where splitting K is what keeps
+ *       every SM busy.  (With NVFP4 activations the caller's codes, scales and
+ *       global scale are taken as given; a dynamic global scale computed over
+ *       a batch is itself batch-dependent.)
+ */
+typedef struct {
+  int32_t batch_invariant;
+  int32_t reserved[7];
+} hq_compute_config;
+
 /* Text for a status code (static storage). */
 HQ_API const char *hq_status_string(hq_status s);
 
@@ -197,6 +214,15 @@ HQ_API size_t hq_gemm_workspace_bytes(const hq_quant_desc *desc, int M, int N, i
 HQ_API hq_status hq_gemm(const hq_quant_desc *desc, int M, int N, int K, const void *packed_w,
                   const void *a, const void *a_scales, const float *a_global, void *c_bf16,
                   void *workspace, size_t ws_bytes, hq_stream_t stream);
+
+/* hq_gemm with compute options (cfg may be NULL: the defaults, identical to
+ * hq_gemm).  Same arguments and contract as hq_gemm; size the workspace with
+ * hq_gemm_config_workspace_bytes for the same cfg. */
+HQ_API size_t hq_gemm_config_workspace_bytes(const hq_quant_desc *desc, const hq_compute_config *cfg, int M,
+                                      int N, int K);
+HQ_API hq_status hq_gemm_config(const hq_quant_desc *desc, const hq_compute_config *cfg, int M, int N, int K,
+                         const void *packed_w, const void *a, const void *a_scales, const float *a_global,
+                         void *c_bf16, void *workspace, size_t ws_bytes, hq_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * MoE routing prepare (SGLang digest: moe_permute_prepare /

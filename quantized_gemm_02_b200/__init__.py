@@ -12,11 +12,12 @@ import ctypes
 import os
 
 __all__ = [
-    "HQError", "QuantDesc", "lib", "library_path", "EXPORTS",
+    "HQError", "QuantDesc", "ComputeConfig", "lib", "library_path", "EXPORTS",
     "HQ_BF16", "HQ_FP32", "HQ_INT4", "HQ_UINT4", "HQ_E2M1", "HQ_E4M3", "HQ_E8M0", "HQ_UE4M3", "HQ_MXFP8",
     "HQ_NVFP4", "HQ_MOE_GROUPED", "HQ_MOE_INDEXED",
     "hq_status_string", "hq_device_error", "hq_packed_weights_bytes", "hq_pack_weights", "hq_unpack_weights",
-    "hq_quant_act", "hq_gemm_workspace_bytes", "hq_gemm", "hq_moe_permute", "hq_moe_workspace_bytes",
+    "hq_quant_act", "hq_gemm_workspace_bytes", "hq_gemm", "hq_gemm_config_workspace_bytes",
+    "hq_gemm_config", "hq_moe_permute", "hq_moe_workspace_bytes",
     "hq_moe_gemm", "hq_moe_masked_workspace_bytes", "hq_moe_gemm_masked", "hq_silu_and_mul", "hq_moe_unpermute_sum",
     "hq_gemm_noalloc", "hq_selftest_wait_timeout",
 ]
@@ -32,7 +33,8 @@ STATUS = {
 # Every symbol include/hq.h declares.
 EXPORTS = (
     "hq_status_string", "hq_device_error", "hq_packed_weights_bytes", "hq_pack_weights", "hq_unpack_weights",
-    "hq_quant_act", "hq_gemm_workspace_bytes", "hq_gemm", "hq_moe_permute", "hq_moe_workspace_bytes",
+    "hq_quant_act", "hq_gemm_workspace_bytes", "hq_gemm", "hq_gemm_config_workspace_bytes",
+    "hq_gemm_config", "hq_moe_permute", "hq_moe_workspace_bytes",
     "hq_moe_gemm", "hq_moe_masked_workspace_bytes", "hq_moe_gemm_masked", "hq_silu_and_mul", "hq_moe_unpermute_sum",
     "hq_gemm_noalloc", "hq_selftest_wait_timeout",
 )
@@ -56,6 +58,11 @@ class QuantDesc(ctypes.Structure):
                 % (self.w_dtype, self.w_group, self.w_scale_dtype, self.w_has_zero, self.w_has_global, self.a_dtype))
 
 
+class ComputeConfig(ctypes.Structure):
+    """hq_compute_config: compute options (zero = the defaults)."""
+    _fields_ = [("batch_invariant", ctypes.c_int32), ("reserved", ctypes.c_int32 * 7)]
+
+
 HERE = os.path.dirname(os.path.abspath(__file__))
 
 
@@ -75,6 +82,7 @@ def _lib() -> ctypes.CDLL:
         L = ctypes.CDLL(path)
         P, I, Z, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
         D = ctypes.POINTER(QuantDesc)
+        C = ctypes.POINTER(ComputeConfig)
         sig = {
             "hq_status_string": (ctypes.c_char_p, [I]),
             "hq_device_error": (I, [P]),
@@ -90,6 +98,8 @@ def _lib() -> ctypes.CDLL:
             "hq_moe_masked_workspace_bytes": (Z, [D, I, I, I, I, I]),
             "hq_moe_gemm_masked": (I, [D, I, I, I, I, P, P, P, I, P, P, Z, P]),
             "hq_silu_and_mul": (I, [I, I, P, P, P]),
+            "hq_gemm_config_workspace_bytes": (Z, [D, C, I, I, I]),
+            "hq_gemm_config": (I, [D, C, I, I, I, P, P, P, P, P, P, Z, P]),
             "hq_moe_unpermute_sum": (I, [I, I, I, P, P, P, F, P, P]),
             "hq_gemm_noalloc": (I, [D, I, I, I, P, P, P, P, P, P]),
             "hq_selftest_wait_timeout": (I, [ctypes.c_ulonglong, P]),
@@ -166,6 +176,20 @@ def hq_gemm_workspace_bytes(desc, M, N, K) -> int:
 def hq_gemm(desc, M, N, K, packed_w, a, a_scales, a_global, c, workspace, ws_bytes, stream=None):
     _check("hq_gemm", _lib().hq_gemm(
         ctypes.byref(desc), M, N, K, _ptr(packed_w), _ptr(a), _ptr(a_scales), _ptr(a_global), _ptr(c),
+        _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def _cfg(cfg):
+    return None if cfg is None else ctypes.byref(cfg)
+
+
+def hq_gemm_config_workspace_bytes(desc, cfg, M, N, K) -> int:
+    return _lib().hq_gemm_config_workspace_bytes(ctypes.byref(desc), _cfg(cfg), M, N, K)
+
+
+def hq_gemm_config(desc, cfg, M, N, K, packed_w, a, a_scales, a_global, c, workspace, ws_bytes, stream=None):
+    _check("hq_gemm_config", _lib().hq_gemm_config(
+        ctypes.byref(desc), _cfg(cfg), M, N, K, _ptr(packed_w), _ptr(a), _ptr(a_scales), _ptr(a_global), _ptr(c),
         _ptr(workspace), ws_bytes, _stream(stream)))
 
 

@@ -98,6 +98,43 @@ static hq_status plan_dense(const hq_quant_desc *d, int M, int N, int K, DensePl
   return HQ_OK;
 }
 
+static int device_sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    n = 148;
+  return n > 0 ? n : 148;
+}
+
+// Dense plan with compute options.  Batch invariance: 64-token tiles and no
+// K split, so that each output row is one tile's k-ordered sum whatever M:
+// the multi-stage kernel with at most as many CTAs as tiles (whole tiles
+// round-robin), or the TMA-fed kernel with a CTA count that divides the tile
+// count (its contiguous per-CTA ranges then hold whole tiles).
+static hq_status plan_dense_cfg(const hq_quant_desc *d, const hq_compute_config *cfg, int M, int N, int K,
+                                DensePlan *pl) {
+  const hq_status ps = plan_dense(d, M, N, K, pl);
+  if (ps != HQ_OK || !cfg || !cfg->batch_invariant) return ps;
+  for (int i = 0; i < 7; ++i)
+    if (cfg->reserved[i] != 0) return HQ_ERR_INVALID_ARG;
+  TcLaunch t{};
+  t.bnt = 64;
+  t.ntw = pl->L.NT;
+  t.mtiles = M > 0 ? (M + 63) / 64 : 1;
+  const long tiles = (long)t.ntw * t.mtiles;
+  const int sms = device_sm_count();
+  if (pl->L.bs == BS_NONE) {
+    t.kind = 0;
+    t.nctas = (int)(tiles < 2L * sms ? tiles : 2L * sms);  // two 64-token CTAs per SM
+  } else {
+    t.kind = 2;
+    int n = (int)(tiles < sms ? tiles : sms);
+    while (n > 1 && tiles % n != 0) --n;
+    t.nctas = n;
+  }
+  pl->s = t;
+  return HQ_OK;
+}
+
 // Dense workspace: split-K state; then either the decoded bf16 copy of
 // quantised activations, or (block-scaled MMA) the activation scales in the
 // kernel's chunk order.
@@ -352,18 +389,23 @@ hq_status hq_quant_act(const hq_quant_desc *desc, int M, int K, const void *x_bf
                           (cudaStream_t)stream);
 }
 
-size_t hq_gemm_workspace_bytes(const hq_quant_desc *desc, int M, int N, int K) {
+size_t hq_gemm_config_workspace_bytes(const hq_quant_desc *desc, const hq_compute_config *cfg, int M, int N,
+                                      int K) {
   DensePlan pl;
-  if (plan_dense(desc, M, N, K, &pl) != HQ_OK) return 0;
+  if (plan_dense_cfg(desc, cfg, M, N, K, &pl) != HQ_OK) return 0;
   void *a, *b;
   return dense_ws(pl, M, K, nullptr, &a, &b);
 }
 
-hq_status hq_gemm(const hq_quant_desc *desc, int M, int N, int K, const void *packed_w, const void *a,
-                  const void *a_scales, const float *a_global, void *c_bf16, void *workspace, size_t ws_bytes,
-                  hq_stream_t stream) {
+size_t hq_gemm_workspace_bytes(const hq_quant_desc *desc, int M, int N, int K) {
+  return hq_gemm_config_workspace_bytes(desc, nullptr, M, N, K);
+}
+
+hq_status hq_gemm_config(const hq_quant_desc *desc, const hq_compute_config *cfg, int M, int N, int K,
+                         const void *packed_w, const void *a, const void *a_scales, const float *a_global,
+                         void *c_bf16, void *workspace, size_t ws_bytes, hq_stream_t stream) {
   DensePlan pl;
-  const hq_status ps = plan_dense(desc, M, N, K, &pl);
+  const hq_status ps = plan_dense_cfg(desc, cfg, M, N, K, &pl);
   if (ps != HQ_OK) return ps;
   if (M == 0) return HQ_OK;
   if (!packed_w || !a || !c_bf16 || !aligned16(packed_w) || !aligned16(a)) return HQ_ERR_INVALID_ARG;
@@ -394,6 +436,13 @@ hq_status hq_gemm(const hq_quant_desc *desc, int M, int N, int K, const void *pa
   }
   return launch_tc_gemm(pl.L, packed_w, a_use, M, row_scale, pl.afmt == A_NVFP4 ? a_global : nullptr, M, 0, 1,
                         nullptr, nullptr, 1, 0, c_bf16, pl.s, split_ws, st);
+}
+
+hq_status hq_gemm(const hq_quant_desc *desc, int M, int N, int K, const void *packed_w, const void *a,
+                  const void *a_scales, const float *a_global, void *c_bf16, void *workspace, size_t ws_bytes,
+                  hq_stream_t stream) {
+  return hq_gemm_config(desc, nullptr, M, N, K, packed_w, a, a_scales, a_global, c_bf16, workspace, ws_bytes,
+                        stream);
 }
 
 hq_status hq_moe_permute(int T, int topk, int E, const int32_t *topk_ids, int32_t *expert_offsets, int32_t *perm,

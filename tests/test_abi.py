@@ -82,3 +82,15 @@ def test_host_validation_without_device():
     assert e.value.status == 1  # E > 1024
     # a zero-row GEMM is a no-op that succeeds without a device
     hq.hq_gemm(d, 0, 64, 128, 16, 16, None, None, 16, None, 0, stream=0)
+
+
+def test_compute_config_queries():
+    d = cdesc("uint4_g128")
+    assert hq.hq_gemm_config_workspace_bytes(d, None, 16, 8192, 8192) == hq.hq_gemm_workspace_bytes(d, 16, 8192, 8192)
+    c = hq.ComputeConfig()
+    assert hq.hq_gemm_config_workspace_bytes(d, c, 16, 8192, 8192) == hq.hq_gemm_workspace_bytes(d, 16, 8192, 8192)
+    c.batch_invariant = 1
+    assert hq.hq_gemm_config_workspace_bytes(d, c, 16, 8192, 8192) > 0
+    assert hq.hq_gemm_config_workspace_bytes(cdesc("nvfp4", "nvfp4"), c, 300, 7168, 7168) > 0
+    c.reserved[3] = 1  # unknown options must stay zero
+    assert hq.hq_gemm_config_workspace_bytes(d, c, 16, 8192, 8192) == 0

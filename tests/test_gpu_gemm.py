@@ -162,3 +162,45 @@ def test_split_k_deterministic_and_workspace_reusable():
     torch.cuda.synchronize()
     assert torch.equal(outs[0], outs[1]) and torch.equal(outs[1], outs[2])
     assert hq.hq_device_error() == 0
+
+
+@pytest.mark.parametrize("wname,aname", [("uint4_g128", "bf16"), ("mxfp4", "bf16"), ("mxfp4", "mxfp8"),
+                                         ("nvfp4", "nvfp4"), ("fp8", "fp8"), ("int4_g128", "fp8")])
+def test_batch_invariant_rows_do_not_depend_on_m(wname, aname):
+    # compute option batch_invariant: the first m rows of a 300-row call are
+    # bit-identical to a call with only those m rows (same codes and scales);
+    # the 300-row result also matches the oracle
+    import quantized_gemm_02_b200 as hq
+    N, K, Mmax = 136, 512, 300
+    w = make_weights(wname, 1, N, K, seed=71)
+    packed = gpu_pack(wname, w, 1, N, K, aname)
+    x = synth.bf16_normal((Mmax, K), synth.generator(72))
+    d = cdesc(wname, aname)
+    cfg = hq.ComputeConfig()
+    cfg.batch_invariant = 1
+    if aname == "bf16":
+        codes, scales, g = x.cuda(), None, None
+    else:
+        codes, scales, g = gpu_quant(aname, x.cuda())
+        if aname != "nvfp4":
+            g = None
+    outs = {}
+    for M in (Mmax, 1, 5, 64, 65, 200):
+        wsb = hq.hq_gemm_config_workspace_bytes(d, cfg, M, N, K)
+        ws = torch.zeros(max(wsb, 16), dtype=torch.uint8, device="cuda")
+        c = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+        hq.hq_gemm_config(d, cfg, M, N, K, packed, codes[:M].contiguous(),
+                          None if scales is None else scales[:M].contiguous(), g, c, ws, wsb)
+        outs[M] = c
+    torch.cuda.synchronize()
+    for M, c in outs.items():
+        assert torch.equal(c, outs[Mmax][:M]), M
+    xb = np_bits(x)
+    if aname == "bf16":
+        A, row = O.decode_act("bf16", Mmax, K, xb)
+    else:
+        q, s, og = oracle_quant(aname, xb)
+        A, row = O.decode_act(aname, Mmax, K, q, s, og)
+    W, col = oracle_decoder(wname, w, N, K)(0)
+    ref, bound = O.gemm(A, W, row, col)
+    assert_close(outs[Mmax].cpu(), ref, bound, what=f"batch-invariant {wname}x{aname}")
