@@ -94,3 +94,28 @@ def test_compute_config_queries():
     assert hq.hq_gemm_config_workspace_bytes(cdesc("nvfp4", "nvfp4"), c, 300, 7168, 7168) > 0
     c.reserved[3] = 1  # unknown options must stay zero
     assert hq.hq_gemm_config_workspace_bytes(d, c, 16, 8192, 8192) == 0
+
+
+def test_masked_moe_and_silu_host_validation():
+    d = cdesc("mxfp4")
+    # size query: E slabs of `slab` rows; the routing arrays sit after the MoE workspace
+    n = hq.hq_moe_masked_workspace_bytes(d, 8, 48, 96, 256, 24)
+    assert n >= 8 * 48 * 256 * 2 + 8 * 48 * 4
+    assert hq.hq_moe_masked_workspace_bytes(d, 8, 48, 96, 256, 0) > 0      # expected_m < 1: the slab
+    assert hq.hq_moe_masked_workspace_bytes(d, 0, 48, 96, 256, 24) == 0    # no experts
+    assert hq.hq_moe_masked_workspace_bytes(d, 2000, 48, 96, 256, 24) == 0  # E > 1024
+    assert hq.hq_moe_masked_workspace_bytes(d, 8, 0, 96, 256, 24) == 0     # empty slab
+    assert hq.hq_moe_masked_workspace_bytes(d, 8, 48, 96, 100, 24) == 0    # K not a multiple of 64
+    with pytest.raises(hq.HQError) as e:
+        hq.hq_moe_gemm_masked(d, 8, 48, 96, 256, 16, 16, None, 24, 16, 16, n, stream=0)
+    assert e.value.status == 1  # no expert_num_tokens
+    with pytest.raises(hq.HQError) as e:
+        hq.hq_moe_gemm_masked(d, 8, 48, 96, 256, 16, 16, 16, 24, 16, None, 0, stream=0)
+    assert e.value.status == 3  # no workspace
+    with pytest.raises(hq.HQError) as e:
+        hq.hq_silu_and_mul(4, 12, 16, 16, stream=0)
+    assert e.value.status == 1  # I not a multiple of 8
+    with pytest.raises(hq.HQError) as e:
+        hq.hq_silu_and_mul(4, 16, 17, 32, stream=0)
+    assert e.value.status == 1  # misaligned input
+    hq.hq_silu_and_mul(0, 16, None, None, stream=0)  # zero rows: a no-op without a device
