@@ -569,36 +569,70 @@ WORKLOADS = {
 # CPU oracle baseline (bounded sample)
 # ---------------------------------------------------------------------------
 def cpu_baseline(workload: str, budget_s: float = 15.0):
-    """Times the oracle as it stands on a bounded sample of the workload:
-    decode one (N, K) weight matrix and multiply M rows in fp64."""
+    """Times the oracle as it stands on a bounded sample of the workload: the
+    workload's own weight and activation formats at one of its shapes, i.e.
+    decode one (N, K) weight matrix, quantise and decode M activation rows
+    when the workload quantises them, and multiply in fp64."""
     import oracle as O
     gen = synth.generator(0)
-    if workload == "w4a16_dense_m16":
-        N, K, M, group, asym, wd = 4096, 4096, 16, 128, False, "int4"
+    # (weight kind, activation format, N, K, M)
+    samples = {
+        "w4a16_dense_m16": ("int4", "bf16", 4096, 4096, 16),
+        "w4a16_asym_sweep": ("uint4", "bf16", 8192, 8192, 16),
+        "moe_w4a16_mxfp4": ("mxfp4", "bf16", 4096, 7168, 16),
+        "moe_w4a8_mxfp8": ("mxfp4", "mxfp8", 4096, 7168, 64),
+        "moe_nvfp4": ("nvfp4", "nvfp4", 4096, 7168, 128),
+        "moe_masked_nvfp4": ("nvfp4", "nvfp4", 4096, 7168, 128),
+        "w4a4_nvfp4": ("nvfp4", "nvfp4", 7168, 7168, 32),
+        "w8a8_fp8": ("fp8", "fp8", 7168, 7168, 32),
+    }
+    wk, ak, N, K, M = samples.get(workload, samples["w4a16_asym_sweep"])
+    if wk in ("int4", "uint4"):
+        w = synth.int4_weights(1, N, K, 128, wk == "uint4", gen)
+        desc = O.Desc(wk, 128, "bf16", w_zero=(wk == "uint4"))
+        args = (synth.to_np_bits(w["codes"][0]), synth.to_np_bits(w["scales"][0]),
+                None if w["zeros"] is None else synth.to_np_bits(w["zeros"][0]))
+    elif wk == "mxfp4":
+        w = synth.mxfp4_weights(1, N, K, gen)
+        desc = O.Desc("e2m1", 32, "e8m0")
+        args = (synth.to_np_bits(w["codes"][0]), synth.to_np_bits(w["scales"][0]), None)
+    elif wk == "nvfp4":
+        w = synth.nvfp4_weights_random(1, N, K, gen)
+        desc = O.Desc("e2m1", 16, "ue4m3", w_global=True)
+        args = (synth.to_np_bits(w["codes"][0]), synth.to_np_bits(w["scales"][0]), None,
+                synth.to_np_bits(w["global"])[0])
     else:
-        N, K, M, group, asym, wd = 8192, 8192, 16, 128, True, "uint4"
-    w = synth.int4_weights(1, N, K, group, asym, gen)
+        w = synth.fp8_weights_random(1, N, K, gen)
+        desc = O.Desc("e4m3", 0, "fp32")
+        args = (synth.to_np_bits(w["codes"][0]), synth.to_np_bits(w["scales"][0]), None)
     x = synth.bf16_normal((M, K), gen)
-    desc = O.Desc(wd, group, "bf16", w_zero=asym)
-    codes = synth.to_np_bits(w["codes"][0])
-    scales = synth.to_np_bits(w["scales"][0])
-    zeros = None if w["zeros"] is None else synth.to_np_bits(w["zeros"][0])
     xb = synth.to_np_bits(x)
     flops = 0.0
     t0 = time.perf_counter()
     n = 0
     while True:
-        A, _ = O.decode_act("bf16", M, K, xb)
-        W, col = O.decode_weights(desc, N, K, codes, scales, zeros)
-        O.gemm(A, W, None, col)
+        if ak == "bf16":
+            A, row = O.decode_act("bf16", M, K, xb)
+        elif ak == "fp8":
+            q, sc = O.quant_fp8_per_token(xb)
+            A, row = O.decode_act("fp8", M, K, q, sc)
+        elif ak == "mxfp8":
+            q, sc = O.quant_mxfp8(xb)
+            A, row = O.decode_act("mxfp8", M, K, q, sc)
+        else:
+            q, sc, g = O.quant_nvfp4(xb)
+            A, row = O.decode_act("nvfp4", M, K, q, sc, g)
+        W, col = O.decode_weights(desc, N, K, *args)
+        O.gemm(A, W, row, col)
         flops += 2.0 * M * N * K
         n += 1
         if time.perf_counter() - t0 > budget_s or n >= 50:
             break
     dt = time.perf_counter() - t0
     cores = len(os.sched_getaffinity(0))
+    act = "" if ak == "bf16" else f" + {ak} quantise/decode of A"
     return {"value": flops / dt / 1e12, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
-            "sample": f"{n} x (decode {wd} g{group} W[{N},{K}] + fp64 GEMM M={M}), {dt:.1f} s; numpy BLAS threads",
+            "sample": f"{n} x (decode {wk} W[{N},{K}]{act} + fp64 GEMM M={M}), {dt:.1f} s; numpy BLAS threads",
             "seconds": dt}
 
 
