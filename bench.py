@@ -240,6 +240,26 @@ def dense_op(hq, d, name, M, N, K, packed, w_bytes, gen, a_fmt="bf16", a_bits=No
               kernel=gemm_kernel_name(M))
 
 
+NOMINAL_HBM_GBS = 8000.0  # the nominal B200 figure the targets are quoted against
+
+
+def sweep_entry(op, t_ms, peaks):
+    """One sweep point: time, TFLOPS, weight GB/s and the fractions of the
+    rooflines: HBM (measured copy bandwidth, and the nominal 8 TB/s), tensor
+    (measured bf16 peak x the MMA kind's nominal ratio), and the combined
+    roofline fraction max(bytes / BW, flops / peak) / t with the measured
+    figures."""
+    s = t_ms / 1e3
+    hb = op.bytes / s / 1e9
+    t_bw = op.bytes / (peaks["hbm_gbs"] * 1e9)
+    t_fl = op.flops / (peaks["bf16_tflops"] * op.peak_ratio * 1e12)
+    return {"op": op.name, "us": round(t_ms * 1e3, 2), "tflops": round(op.flops / s / 1e12, 2),
+            "weight_gbs": round(op.w_bytes / s / 1e9, 1), "hbm_frac": round(hb / peaks["hbm_gbs"], 3),
+            "hbm_frac_nominal": round(hb / NOMINAL_HBM_GBS, 3),
+            "tensor_frac": round(op.flops / s / 1e12 / (peaks["bf16_tflops"] * op.peak_ratio), 3),
+            "roofline_frac": round(max(t_bw, t_fl) / s, 3)}
+
+
 def gemm_kernel_name(rows_per_tile):
     """The GEMM kernel the library picks for a token tile of this many rows."""
     return "dec_gemm_kernel" if rows_per_tile <= 32 else "tc_gemm_kernel"
@@ -807,13 +827,7 @@ def main():
         " bf16 x %g (nominal ratio of the MMA kind)" % dom.peak_ratio if roof["bound"] == "tensor" and dom.peak_ratio != 1
         else "")
 
-    sweep = []
-    for op, t in zip(ops, per_op):
-        s = t / 1e3
-        hb = op.bytes / s / 1e9
-        sweep.append({"op": op.name, "us": round(t * 1e3, 2), "tflops": round(op.flops / s / 1e12, 2),
-                      "weight_gbs": round(op.w_bytes / s / 1e9, 1), "hbm_frac": round(hb / peaks["hbm_gbs"], 3),
-                      "tensor_frac": round(op.flops / s / 1e12 / (peaks["bf16_tflops"] * op.peak_ratio), 3)})
+    sweep = [sweep_entry(op, t, peaks) for op, t in zip(ops, per_op)]
     line = {
         "metric": METRIC,
         "value": value, "unit": "TFLOPS", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
