@@ -36,7 +36,11 @@ library; citations name the page and its section):
   listed in the design notes.
 
 Parity pins live in ``tests/test_oracle_*.py``.  Functions without an
-independent pin say "parity unpinned" in their docstring.
+independent pin say "parity unpinned" in their docstring.  The functions of
+the last section (FP6, INT1-3, MXINT4 and block-scaled FP8) serve rows that
+have no GPU path yet; their element values and reductions are pinned, while
+the MXINT4 and INT1-3 code conventions are readings (the pages only name
+those formats).
 """
 from __future__ import annotations
 
@@ -49,7 +53,9 @@ __all__ = [
     "Desc", "e2m1_value", "e4m3_value", "e8m0_value", "E2M1", "E4M3", "E8M0",
     "bf16_to_f64", "e4m3_rn_sat", "e2m1_rn_sat", "unpack_nibbles_i32", "unpack_nibbles_u8",
     "decode_weights", "quant_fp8_per_token", "quant_mxfp8", "quant_nvfp4", "decode_act",
-    "gemm", "moe_permute", "moe", "moe_expert_outputs",
+    "gemm", "moe_permute", "moe", "moe_expert_outputs", "moe_masked", "silu_and_mul",
+    "fp6_value", "E2M3", "E3M2", "decode_int_weights", "decode_fp6_weights", "decode_mxint4_weights",
+    "decode_fp8_block_weights", "quant_fp8_block", "decode_fp8_block_act",
 ]
 
 
@@ -431,3 +437,107 @@ def silu_and_mul(Y: np.ndarray) -> np.ndarray:
     g, u = Y[:, :I], Y[:, I:]
     with np.errstate(over="ignore"):
         return g / (1.0 + np.exp(-g)) * u
+
+
+# ---------------------------------------------------------------------------
+# Formats of the rows that come next (oracle first; no GPU path yet): FP6
+# and INT1/2/3 weights ("Announcing Humming", section "Performance":
+# WnA16 with INT1, INT2, INT3 and FP4 to FP8 weights), MXINT4 weights (same
+# section, MoE on B300), FP8 with block scales (section "W8A8 / W4A8 /
+# W4A4": block-scaled FP8 W8A8 as on Hopper).
+# ---------------------------------------------------------------------------
+
+def fp6_value(code: int, kind: str) -> float:
+    """OCP MX v1.0 FP6.  'e2m3': sign bit 5, exponent bits 4..3 (bias 1),
+    mantissa bits 2..0; 'e3m2': exponent bits 4..2 (bias 3), mantissa bits
+    1..0.  Exponent 0 is subnormal; there are no infinities or NaNs."""
+    s = -1.0 if (code >> 5) & 1 else 1.0
+    if kind == "e2m3":
+        e, m, mb, bias = (code >> 3) & 3, code & 7, 3, 1
+    elif kind == "e3m2":
+        e, m, mb, bias = (code >> 2) & 7, code & 3, 2, 3
+    else:
+        raise ValueError(kind)
+    if e == 0:
+        return s * (m / 2.0 ** mb) * 2.0 ** (1 - bias)
+    return s * (1.0 + m / 2.0 ** mb) * 2.0 ** (e - bias)
+
+
+E2M3 = np.array([fp6_value(c, "e2m3") for c in range(64)], dtype=np.float64)
+E3M2 = np.array([fp6_value(c, "e3m2") for c in range(64)], dtype=np.float64)
+
+
+def decode_int_weights(bits: int, codes, scales, group: int, zeros=None):
+    """b-bit integer weights (b in 1..8) from unpacked codes u [N, K] in
+    [0, 2^b): w = (u - z) * s with z the per-group zero point when given
+    (unsigned codes, as UINT4), else w = q * s with q the b-bit two's
+    complement value of u (signed codes, as INT4); s bf16 bits
+    [N, K / group] (group 0 = per channel).  The code-level form is this
+    oracle's reading: the pages name INT1/2/3 without a packing or a
+    signedness rule, so the INT4 rules are carried over."""
+    u = np.asarray(codes).astype(np.int64)
+    if u.min(initial=0) < 0 or u.max(initial=0) >= (1 << bits):
+        raise ValueError("code out of range")
+    N, K = u.shape
+    g = K if group == 0 else group
+    s = bf16_to_f64(np.asarray(scales).reshape(N, K // g))
+    grp = np.arange(K) // g
+    if zeros is None:
+        q = np.where(u >= (1 << (bits - 1)), u - (1 << bits), u)
+        return q.astype(np.float64) * s[:, grp]
+    z = np.asarray(zeros).astype(np.int64).reshape(N, K // g)
+    return (u - z[:, grp]).astype(np.float64) * s[:, grp]
+
+
+def decode_fp6_weights(kind: str, codes, e8m0_scales):
+    """MXFP6 weights (OCP MX v1.0): FP6 codes [N, K] (one per byte, low 6
+    bits) with an E8M0 scale per 32 along K: w = fp6 * 2^(c - 127)."""
+    c = np.asarray(codes).astype(np.int64)
+    N, K = c.shape
+    table = E2M3 if kind == "e2m3" else E3M2
+    blk = np.arange(K) // 32
+    return table[c & 63] * E8M0[np.asarray(e8m0_scales).reshape(N, K // 32)][:, blk]
+
+
+def decode_mxint4_weights(codes, e8m0_scales, K: int):
+    """MXINT4 weights: packed 4-bit two's complement codes [N, K/2] (low
+    nibble = even k) with an E8M0 scale per 32 along K: w = q * 2^(c - 127).
+    Reading: the pages name MXINT4 only; this is MXFP4's layout with INT4
+    elements and no further element scale."""
+    q = _signed4(unpack_nibbles_u8(codes, K)).astype(np.float64)
+    N = q.shape[0]
+    blk = np.arange(K) // 32
+    return q * E8M0[np.asarray(e8m0_scales).reshape(N, K // 32)][:, blk]
+
+
+def decode_fp8_block_weights(codes, scales, block: int = 128):
+    """FP8 weights with block scales: E4M3 codes [N, K] and fp32 scales
+    [ceil(N / block), K / block], one per block x block tile:
+    w[n, k] = e4m3(code) * s[n // block, k // block]."""
+    c = np.asarray(codes)
+    N, K = c.shape
+    s = np.asarray(scales, dtype=np.float32).astype(np.float64)
+    return E4M3[c] * s[np.arange(N)[:, None] // block, np.arange(K)[None, :] // block]
+
+
+def quant_fp8_block(x_bits: np.ndarray, group: int = 128):
+    """FP8 activations with a scale per token and per `group` along K:
+    s = amax_group / 448 (fp32), q = e4m3(x / s), RNE, saturating; an
+    all-zero group gets s = 1 (the per-token recipe applied to each group).
+    Returns codes [M, K] and fp32 scales [M, K / group]."""
+    x = bf16_to_f32(x_bits)
+    M, K = x.shape
+    xg = x.reshape(M, K // group, group)
+    amax = np.max(np.abs(xg), axis=2).astype(np.float32)
+    s = (amax / np.float32(448.0)).astype(np.float32)
+    s = np.where(amax == 0, np.float32(1.0), s).astype(np.float32)
+    q = e4m3_rn_sat((xg / s[..., None]).astype(np.float32)).reshape(M, K)
+    return q, s
+
+
+def decode_fp8_block_act(codes, scales, group: int = 128):
+    """Decode block-scaled FP8 activations to fp64 [M, K]."""
+    c = np.asarray(codes)
+    M, K = c.shape
+    s = np.asarray(scales, dtype=np.float32).astype(np.float64).reshape(M, K // group)
+    return E4M3[c] * s[:, np.arange(K) // group]
