@@ -215,6 +215,25 @@ HQ_API hq_status hq_gemm(const hq_quant_desc *desc, int M, int N, int K, const v
                   const void *a, const void *a_scales, const float *a_global, void *c_bf16,
                   void *workspace, size_t ws_bytes, hq_stream_t stream);
 
+/* Which kernel and tiling a call would use (host only; no device work).
+ * Filled for hq_gemm / hq_gemm_config (hq_gemm_plan) and for hq_moe_gemm
+ * (hq_moe_plan) with the same arguments; the CTA count follows the current
+ * device's SM count (148 when no device is present). */
+typedef struct {
+  int32_t kernel;       /* 0: multi-stage (dequantised weights in TMEM), 1: decode (<= 32 tokens
+                           per tile), 2: TMA-fed (block-scaled pairs, FP8 x FP8)               */
+  int32_t layout;       /* 0: dequantisation, 1: MXFP4 x MXFP8, 2: NVFP4 x NVFP4, 3: FP8 x FP8  */
+  int32_t token_tile;   /* tokens per tile (the MMA's N)                                       */
+  int32_t weight_tiles; /* 128-row weight tiles                                                */
+  int32_t token_tiles;  /* token tiles (MoE: an upper bound over experts)                      */
+  int32_t ctas;         /* persistent CTAs launched                                            */
+  int32_t reserved[2];
+} hq_plan_info;
+HQ_API hq_status hq_gemm_plan(const hq_quant_desc *desc, const hq_compute_config *cfg, int M, int N, int K,
+                       hq_plan_info *out);
+HQ_API hq_status hq_moe_plan(const hq_quant_desc *desc, int T, int topk, int E, int N, int K, int a_per_slot,
+                      hq_plan_info *out);
+
 /* hq_gemm with compute options (cfg may be NULL: the defaults, identical to
  * hq_gemm).  Same arguments and contract as hq_gemm; size the workspace with
  * hq_gemm_config_workspace_bytes for the same cfg. */

@@ -12,12 +12,12 @@ import ctypes
 import os
 
 __all__ = [
-    "HQError", "QuantDesc", "ComputeConfig", "lib", "library_path", "EXPORTS",
+    "HQError", "QuantDesc", "ComputeConfig", "PlanInfo", "lib", "library_path", "EXPORTS",
     "HQ_BF16", "HQ_FP32", "HQ_INT4", "HQ_UINT4", "HQ_E2M1", "HQ_E4M3", "HQ_E8M0", "HQ_UE4M3", "HQ_MXFP8",
     "HQ_NVFP4", "HQ_MOE_GROUPED", "HQ_MOE_INDEXED",
     "hq_status_string", "hq_device_error", "hq_packed_weights_bytes", "hq_pack_weights", "hq_unpack_weights",
     "hq_quant_act", "hq_gemm_workspace_bytes", "hq_gemm", "hq_gemm_config_workspace_bytes",
-    "hq_gemm_config", "hq_moe_permute", "hq_moe_workspace_bytes",
+    "hq_gemm_config", "hq_gemm_plan", "hq_moe_plan", "hq_moe_permute", "hq_moe_workspace_bytes",
     "hq_moe_gemm", "hq_moe_masked_workspace_bytes", "hq_moe_gemm_masked", "hq_silu_and_mul", "hq_moe_unpermute_sum",
     "hq_gemm_noalloc", "hq_selftest_wait_timeout",
 ]
@@ -34,7 +34,7 @@ STATUS = {
 EXPORTS = (
     "hq_status_string", "hq_device_error", "hq_packed_weights_bytes", "hq_pack_weights", "hq_unpack_weights",
     "hq_quant_act", "hq_gemm_workspace_bytes", "hq_gemm", "hq_gemm_config_workspace_bytes",
-    "hq_gemm_config", "hq_moe_permute", "hq_moe_workspace_bytes",
+    "hq_gemm_config", "hq_gemm_plan", "hq_moe_plan", "hq_moe_permute", "hq_moe_workspace_bytes",
     "hq_moe_gemm", "hq_moe_masked_workspace_bytes", "hq_moe_gemm_masked", "hq_silu_and_mul", "hq_moe_unpermute_sum",
     "hq_gemm_noalloc", "hq_selftest_wait_timeout",
 )
@@ -61,6 +61,17 @@ class QuantDesc(ctypes.Structure):
 class ComputeConfig(ctypes.Structure):
     """hq_compute_config: compute options (zero = the defaults)."""
     _fields_ = [("batch_invariant", ctypes.c_int32), ("reserved", ctypes.c_int32 * 7)]
+
+
+class PlanInfo(ctypes.Structure):
+    """hq_plan_info: the kernel and tiling a call would use."""
+    _fields_ = [("kernel", ctypes.c_int32), ("layout", ctypes.c_int32), ("token_tile", ctypes.c_int32),
+                ("weight_tiles", ctypes.c_int32), ("token_tiles", ctypes.c_int32), ("ctas", ctypes.c_int32),
+                ("reserved", ctypes.c_int32 * 2)]
+
+    def as_dict(self):
+        return {k: getattr(self, k) for k in ("kernel", "layout", "token_tile", "weight_tiles", "token_tiles",
+                                                "ctas")}
 
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -100,6 +111,8 @@ def _lib() -> ctypes.CDLL:
             "hq_silu_and_mul": (I, [I, I, P, P, P]),
             "hq_gemm_config_workspace_bytes": (Z, [D, C, I, I, I]),
             "hq_gemm_config": (I, [D, C, I, I, I, P, P, P, P, P, P, Z, P]),
+            "hq_gemm_plan": (I, [D, C, I, I, I, ctypes.POINTER(PlanInfo)]),
+            "hq_moe_plan": (I, [D, I, I, I, I, I, I, ctypes.POINTER(PlanInfo)]),
             "hq_moe_unpermute_sum": (I, [I, I, I, P, P, P, F, P, P]),
             "hq_gemm_noalloc": (I, [D, I, I, I, P, P, P, P, P, P]),
             "hq_selftest_wait_timeout": (I, [ctypes.c_ulonglong, P]),
@@ -191,6 +204,18 @@ def hq_gemm_config(desc, cfg, M, N, K, packed_w, a, a_scales, a_global, c, works
     _check("hq_gemm_config", _lib().hq_gemm_config(
         ctypes.byref(desc), _cfg(cfg), M, N, K, _ptr(packed_w), _ptr(a), _ptr(a_scales), _ptr(a_global), _ptr(c),
         _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def hq_gemm_plan(desc, cfg, M, N, K) -> dict:
+    info = PlanInfo()
+    _check("hq_gemm_plan", _lib().hq_gemm_plan(ctypes.byref(desc), _cfg(cfg), M, N, K, ctypes.byref(info)))
+    return info.as_dict()
+
+
+def hq_moe_plan(desc, T, topk, E, N, K, a_per_slot) -> dict:
+    info = PlanInfo()
+    _check("hq_moe_plan", _lib().hq_moe_plan(ctypes.byref(desc), T, topk, E, N, K, a_per_slot, ctypes.byref(info)))
+    return info.as_dict()
 
 
 def hq_moe_permute(T, topk, E, topk_ids, expert_offsets, perm, inv_perm, stream=None):

@@ -389,6 +389,36 @@ hq_status hq_quant_act(const hq_quant_desc *desc, int M, int K, const void *x_bf
                           (cudaStream_t)stream);
 }
 
+static void fill_plan(const Layout &L, const TcLaunch &t, hq_plan_info *out) {
+  std::memset(out, 0, sizeof(*out));
+  out->kernel = t.kind;
+  out->layout = L.bs;
+  out->token_tile = t.bnt;
+  out->weight_tiles = t.ntw;
+  out->token_tiles = t.mtiles;
+  out->ctas = t.nctas;
+}
+
+hq_status hq_gemm_plan(const hq_quant_desc *desc, const hq_compute_config *cfg, int M, int N, int K,
+                       hq_plan_info *out) {
+  if (!out) return HQ_ERR_INVALID_ARG;
+  DensePlan pl;
+  const hq_status ps = plan_dense_cfg(desc, cfg, M, N, K, &pl);
+  if (ps != HQ_OK) return ps;
+  fill_plan(pl.L, pl.s, out);
+  return HQ_OK;
+}
+
+hq_status hq_moe_plan(const hq_quant_desc *desc, int T, int topk, int E, int N, int K, int a_per_slot,
+                      hq_plan_info *out) {
+  if (!out) return HQ_ERR_INVALID_ARG;
+  MoePlan pl;
+  const hq_status ps = plan_moe(desc, T, topk, E, N, K, a_per_slot, &pl);
+  if (ps != HQ_OK) return ps;
+  fill_plan(pl.L, pl.s, out);
+  return HQ_OK;
+}
+
 size_t hq_gemm_config_workspace_bytes(const hq_quant_desc *desc, const hq_compute_config *cfg, int M, int N,
                                       int K) {
   DensePlan pl;

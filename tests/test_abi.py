@@ -119,3 +119,38 @@ def test_masked_moe_and_silu_host_validation():
         hq.hq_silu_and_mul(4, 16, 17, 32, stream=0)
     assert e.value.status == 1  # misaligned input
     hq.hq_silu_and_mul(0, 16, None, None, stream=0)  # zero rows: a no-op without a device
+
+
+def test_host_dispatch_plans():
+    # which kernel and tiling each call takes (host only; 148 SMs without a device)
+    p = hq.hq_gemm_plan
+    # W4A16: decode kernel up to 32 tokens, then the multi-stage kernel
+    assert p(cdesc("uint4_g128"), None, 16, 28672, 8192) == {
+        "kernel": 1, "layout": 0, "token_tile": 16, "weight_tiles": 224, "token_tiles": 1, "ctas": 148}
+    assert p(cdesc("uint4_g128"), None, 32, 8192, 8192)["token_tile"] == 32
+    big = p(cdesc("uint4_g128"), None, 8192, 28672, 8192)
+    assert big["kernel"] == 0 and big["token_tile"] == 256 and big["token_tiles"] == 32
+    assert p(cdesc("uint4_g128"), None, 64, 8192, 8192)["token_tile"] == 64
+    # the microscaling pairs take their own layouts and the TMA-fed kernel, at most 128 tokens
+    mx = p(cdesc("mxfp4", "mxfp8"), None, 8192, 7168, 7168)
+    assert (mx["kernel"], mx["layout"], mx["token_tile"]) == (2, 1, 128)
+    nv = p(cdesc("nvfp4", "nvfp4"), None, 1, 7168, 7168)
+    assert (nv["kernel"], nv["layout"], nv["token_tile"]) == (2, 2, 16)
+    # other quantised pairs decode the activations and keep the dequantisation layout
+    assert p(cdesc("nvfp4", "fp8"), None, 8192, 7168, 7168)["layout"] == 0
+    # FP8 x FP8: 256-token tiles only with at least two per SM, else 128; K % 128 != 0 keeps the old layout
+    assert p(cdesc("fp8", "fp8"), None, 8192, 7168, 7168)["token_tile"] == 256
+    assert p(cdesc("fp8", "fp8"), None, 256, 7168, 7168)["token_tile"] == 128
+    assert p(cdesc("fp8", "fp8"), None, 300, 7168, 192)["layout"] == 0
+    # batch invariance: 64-token tiles, no K split (CTAs <= tiles; TMA-fed kernel: CTAs divide tiles)
+    c = hq.ComputeConfig()
+    c.batch_invariant = 1
+    bi = p(cdesc("uint4_g128"), c, 1, 8192, 8192)
+    assert (bi["kernel"], bi["token_tile"], bi["ctas"]) == (0, 64, 64)
+    bi2 = p(cdesc("nvfp4", "nvfp4"), c, 300, 7168, 7168)
+    tiles = bi2["weight_tiles"] * bi2["token_tiles"]
+    assert bi2["token_tile"] == 64 and tiles % bi2["ctas"] == 0 and bi2["ctas"] <= 148
+    # MoE: NVFP4 takes 192-token tiles at ~128 rows per expert, MXFP4 x MXFP8 stays at 128
+    assert hq.hq_moe_plan(cdesc("nvfp4", "nvfp4"), 4096, 8, 256, 4096, 7168, 0)["token_tile"] == 192
+    assert hq.hq_moe_plan(cdesc("mxfp4", "mxfp8"), 4096, 8, 256, 4096, 7168, 0)["token_tile"] == 128
+    assert hq.hq_moe_plan(cdesc("mxfp4"), 1, 8, 256, 4096, 7168, 0)["token_tile"] == 16
