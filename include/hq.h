@@ -339,15 +339,17 @@ HQ_API hq_status hq_moe_unpermute_sum(int T, int topk, int N, const void *y_bf16
  * Dense GEMM for callers that cannot allocate device memory (no counterpart
  * in the pages; an addition of this library).
  *
- * Some callers cannot call cudaMalloc when they run a GEMM: code running
- * inside a CUDA graph capture, embedded runtimes or allocator hooks that own
- * all device memory, and plugins that are given no allocator.  This call
+ * Some callers cannot call cudaMalloc when they run a GEMM: embedded
+ * runtimes or allocator hooks that own all device memory, plugins that are
+ * given no allocator, and code paths that must not allocate.  This call
  * computes exactly what hq_gemm computes, with the same arguments except the
  * workspace: its scratch is one fixed array of 64 MiB inside the library's
  * device image, which every GPU that loads the library holds until the
  * process exits.
  *   - Sizes whose workspace (hq_gemm_workspace_bytes) exceeds 64 MiB are
  *     rejected with HQ_ERR_WORKSPACE before anything is launched.
+ *   - Arguments are checked as hq_gemm checks them; a rejected call
+ *     enqueues nothing.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current and caches it; make
  *     that first call before any stream capture.

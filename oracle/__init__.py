@@ -53,7 +53,7 @@ __all__ = [
     "Desc", "e2m1_value", "e4m3_value", "e8m0_value", "E2M1", "E4M3", "E8M0",
     "bf16_to_f64", "e4m3_rn_sat", "e2m1_rn_sat", "unpack_nibbles_i32", "unpack_nibbles_u8",
     "decode_weights", "quant_fp8_per_token", "quant_mxfp8", "quant_nvfp4", "decode_act",
-    "gemm", "moe_permute", "moe", "moe_expert_outputs", "moe_masked", "silu_and_mul",
+    "gemm", "moe_permute", "moe", "moe_expert_outputs", "moe_masked", "silu_and_mul", "nvfp4_global_scale",
     "fp6_value", "E2M3", "E3M2", "decode_int_weights", "decode_fp6_weights", "decode_mxint4_weights",
     "decode_fp8_block_weights", "quant_fp8_block", "decode_fp8_block_act",
 ]
@@ -286,6 +286,17 @@ def quant_mxfp8(x_bits: np.ndarray):
     return q, (e + 127).astype(np.uint8)
 
 
+def nvfp4_global_scale(x_bits: np.ndarray) -> np.float32:
+    """The NVFP4 tensor (second-level) scale of a bf16 tensor: g = amax / (448
+    * 6) in fp32, 1 for an all-zero tensor.  ``quant_nvfp4`` uses it when no
+    static scale is given; quantising some rows of a tensor with
+    ``global_scale=nvfp4_global_scale(whole tensor)`` gives those rows' codes
+    in the whole tensor's quantisation."""
+    x = bf16_to_f32(x_bits)
+    amax_t = np.float32(np.max(np.abs(x))) if x.size else np.float32(0)
+    return np.float32(amax_t / np.float32(2688.0)) if amax_t > 0 else np.float32(1.0)
+
+
 def quant_nvfp4(x_bits: np.ndarray, global_scale=None):
     """NVFP4: g = amax_tensor / (448 * 6) (fp32; 1 if the tensor is zero)
     unless a static ``global_scale`` is given; per block of 16 along K,
@@ -294,11 +305,7 @@ def quant_nvfp4(x_bits: np.ndarray, global_scale=None):
     [M, K/2] (low nibble = even k), UE4M3 codes [M, K/16] and g."""
     x = bf16_to_f32(x_bits)
     M, K = x.shape
-    if global_scale is None:
-        amax_t = np.float32(np.max(np.abs(x))) if x.size else np.float32(0)
-        g = np.float32(amax_t / np.float32(2688.0)) if amax_t > 0 else np.float32(1.0)
-    else:
-        g = np.float32(global_scale)
+    g = nvfp4_global_scale(x_bits) if global_scale is None else np.float32(global_scale)
     xb = x.reshape(M, K // 16, 16)
     amax_b = np.max(np.abs(xb), axis=2).astype(np.float32)
     sbv = ((amax_b / np.float32(6.0)).astype(np.float32) / g).astype(np.float32)

@@ -135,6 +135,17 @@ static hq_status plan_dense_cfg(const hq_quant_desc *d, const hq_compute_config 
   return HQ_OK;
 }
 
+// Pointer checks of a dense call (shared by every dense entry point, before
+// anything is enqueued).
+static hq_status dense_args(const DensePlan &pl, const void *packed_w, const void *a, const void *a_scales,
+                            const float *a_global, const void *c_bf16) {
+  if (!packed_w || !a || !c_bf16 || !aligned16(packed_w) || !aligned16(a)) return HQ_ERR_INVALID_ARG;
+  if (pl.afmt != A_BF16 && !a_scales) return HQ_ERR_INVALID_ARG;
+  if (pl.afmt == A_NVFP4 && !a_global) return HQ_ERR_INVALID_ARG;
+  if (pl.L.bs != BS_NONE && ((uintptr_t)a_scales & 3u)) return HQ_ERR_INVALID_ARG;
+  return HQ_OK;
+}
+
 // Dense workspace: split-K state; then either the decoded bf16 copy of
 // quantised activations, or (block-scaled MMA) the activation scales in the
 // kernel's chunk order.
@@ -438,9 +449,8 @@ hq_status hq_gemm_config(const hq_quant_desc *desc, const hq_compute_config *cfg
   const hq_status ps = plan_dense_cfg(desc, cfg, M, N, K, &pl);
   if (ps != HQ_OK) return ps;
   if (M == 0) return HQ_OK;
-  if (!packed_w || !a || !c_bf16 || !aligned16(packed_w) || !aligned16(a)) return HQ_ERR_INVALID_ARG;
-  if (pl.afmt != A_BF16 && !a_scales) return HQ_ERR_INVALID_ARG;
-  if (pl.afmt == A_NVFP4 && !a_global) return HQ_ERR_INVALID_ARG;
+  const hq_status as = dense_args(pl, packed_w, a, a_scales, a_global, c_bf16);
+  if (as != HQ_OK) return as;
   void *split_ws, *a_dec;
   const size_t need = dense_ws(pl, M, K, (uint8_t *)workspace, &split_ws, &a_dec);
   if (!workspace || ws_bytes < need || !aligned16(workspace)) return HQ_ERR_WORKSPACE;

@@ -1,12 +1,11 @@
 // hq_gemm_noalloc: the dense GEMM for callers that cannot allocate device
 // memory.
 //
-// Some callers cannot call cudaMalloc at the point where they run a GEMM: code
-// that runs inside a CUDA graph being captured, where an allocation would
-// either be illegal or end up baked into the graph; custom allocator hooks
-// and embedded runtimes that own all device memory and forbid side
-// allocations; and plugins loaded into a host framework that gives them no
-// allocator at all.  hq_gemm needs a caller-supplied workspace (split-K
+// Some callers cannot call cudaMalloc at the point where they run a GEMM:
+// custom allocator hooks and embedded runtimes that own all device memory and
+// forbid side allocations, plugins loaded into a host framework that gives
+// them no allocator at all, and code paths that must not allocate while they
+// run.  hq_gemm needs a caller-supplied workspace (split-K
 // partial sums, tile counters, decoded activations).  This entry point instead
 // uses one fixed scratch array that lives in the library's own device image:
 // a file-scope __device__ array that every GPU loading the library holds
@@ -53,6 +52,9 @@ extern "C" hq_status hq_gemm_noalloc(const hq_quant_desc *desc, int M, int N, in
   void *split_ws, *a_dec;
   const size_t need = dense_ws(pl, M, K, nullptr, &split_ws, &a_dec);
   if (need > NOALLOC_SCRATCH_BYTES) return HQ_ERR_WORKSPACE;
+  // every argument check hq_gemm makes, before anything is enqueued
+  const hq_status as = dense_args(pl, packed_w, a, a_scales, a_global, c_bf16);
+  if (as != HQ_OK) return as;
   if (!device_is_sm100()) return HQ_ERR_ARCH;
   void *scratch = nullptr;
   const hq_status ss = noalloc_scratch(&scratch);

@@ -207,8 +207,9 @@ def test_moe_masked(wname, aname):
 
 
 def test_silu_and_mul():
-    # fp32 on the GPU, fp64 in the oracle, both rounded once to bf16: within
-    # one bf16 step (2^-7 relative); extreme gates included
+    # fp32 on the GPU, rounded once to bf16: within half a bf16 step (2^-9
+    # relative) of the fp64 oracle plus the fp32 steps' own error; the test
+    # allows 2^-8 relative and a tiny absolute term; extreme gates included
     import quantized_gemm_02_b200 as hq
     R, I = 37, 136
     y = synth.bf16_normal((R, 2 * I), synth.generator(61)) * 3
@@ -218,5 +219,5 @@ def test_silu_and_mul():
     torch.cuda.synchronize()
     ref = O.silu_and_mul(y.float().numpy().astype(np.float64))
     got = out.cpu().float().numpy().astype(np.float64)
-    tol = np.maximum(np.abs(ref) * 2.0 ** -7, 1e-30)
+    tol = np.abs(ref) * 2.0 ** -8 + 1e-30
     assert np.all(np.abs(got - ref) <= tol), float(np.max(np.abs(got - ref) / tol))

@@ -1,8 +1,8 @@
 """hq_gemm_noalloc: the dense GEMM for callers that cannot allocate device
-memory (inside a CUDA graph capture, under an allocator that owns all device
-memory, or as a plugin with no allocator).  It must compute what hq_gemm
-computes, using the library's fixed device scratch array instead of a caller
-workspace.
+memory (under an allocator that owns all device memory, as a plugin given no
+allocator, or on a code path that must not allocate).  It must compute what
+hq_gemm computes, using the library's fixed device scratch array instead of
+a caller workspace: each call is compared with hq_gemm and with the oracle.
 
 Collected last on purpose: if it fails, a run that stops at the first failure
 has already run every other test.  It also passes when run alone in a fresh
@@ -62,13 +62,14 @@ def test_noalloc_matches_hq_gemm_twice(wname, aname, M, N, K):
         outs.append(c)
     torch.cuda.synchronize()
     assert hq.hq_device_error() == 0
-    _, bound = _reference_and_bound(wname, aname, w, x, M, N, K)
+    ref, bound = _reference_and_bound(wname, aname, w, x, M, N, K)
     tol = REL * bound + ABS
     r = ref_c.float().cpu().numpy()
     for c in outs:
-        g = c.float().cpu().numpy()
+        g = c.float().cpu().numpy().astype(np.float64)
         assert np.all(np.isfinite(g))
-        assert np.all(np.abs(g - r) <= tol)
+        assert np.all(np.abs(g - r) <= tol)    # against hq_gemm
+        assert np.all(np.abs(g - ref) <= tol)  # against the oracle
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
@@ -80,3 +81,7 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     with pytest.raises(hq.HQError) as e:
         hq.hq_gemm_noalloc(d, 4096, 256, 16384, 16, 16, 16, 16, 16)
     assert e.value.status == 3  # HQ_ERR_WORKSPACE
+    # argument errors are reported as hq_gemm reports them
+    with pytest.raises(hq.HQError) as e:
+        hq.hq_gemm_noalloc(cdesc("uint4_g128"), 16, 256, 1024, 16, None, None, None, 16)
+    assert e.value.status == 1  # HQ_ERR_INVALID_ARG
