@@ -392,10 +392,10 @@ def moe_ops(hq, name, wdesc, E, topk, H, I, Ts, routing, gen, mode_names=("group
             def run(mode=mode, pg=pg, pd=pd, Ng=Ng, Kg=Kg, Nd=Nd, Kd=Kd, ws=ws, y=y, out=out, ids=ids, wts=wts,
                     x_gate=x_gate, x_down=x_down, off=off, perm=perm, inv=inv, T=T, wsg=wsg, wsd=wsd):
                 hq.hq_moe_permute(T, topk, E, ids, off, perm, inv)
-                hq.hq_moe_gemm(mode, wdesc, T, topk, E, Ng, Kg, pg, x_gate, 0, off, perm, inv, wts, 1.0, 0, y, ws,
-                               wsg)
-                hq.hq_moe_gemm(mode, wdesc, T, topk, E, Nd, Kd, pd, x_down, 1, off, perm, inv, wts, 1.0, 1, out,
-                               ws, wsd)
+                hq.hq_moe_gemm(mode, wdesc, T, topk, E, Ng, Kg, pg, x_gate, None, None, 0, None, wts, off, perm, 0,
+                               1.0, y, ws, wsg)
+                hq.hq_moe_gemm(mode, wdesc, T, topk, E, Nd, Kd, pd, x_down, None, None, 1, None, wts, off, perm, 1,
+                               1.0, out, ws, wsd)
 
             def e2e(run=run, ids=ids, ids_e=ids_e, ids_h=ids_h, x_gate=x_gate, x_e=x_e, x_gate_h=x_gate_h,
                     out=out, out_h=out_h):

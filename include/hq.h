@@ -94,6 +94,9 @@ typedef enum {
  *   E2M1  + UE4M3 scales, w_group = 16, w_has_global = 1    (NVFP4)
  *   E4M3  + FP32 per-channel scales, w_group = 0            (FP8)
  * and every one of them with a_dtype in {BF16, E4M3, MXFP8, NVFP4}.
+ * a_group is the activation's scale granularity along K: 0 = the format's
+ * own (E4M3: one fp32 scale per token; MXFP8: 32; NVFP4: 16); MXFP8 also
+ * accepts 32 and NVFP4 16.  Zero-initialise the struct.
  */
 typedef struct {
   int32_t w_dtype;       /* HQ_INT4 | HQ_UINT4 | HQ_E2M1 | HQ_E4M3           */
@@ -102,6 +105,7 @@ typedef struct {
   int32_t w_has_zero;    /* 1: UINT4 zero points, same grouping as scales   */
   int32_t w_has_global;  /* 1: FP32 second-level scale per expert (NVFP4)   */
   int32_t a_dtype;       /* HQ_BF16 | HQ_E4M3 | HQ_MXFP8 | HQ_NVFP4          */
+  int32_t a_group;       /* activation scale group along K (0: the format's) */
 } hq_quant_desc;
 
 typedef enum { HQ_MOE_GROUPED = 0, HQ_MOE_INDEXED = 1 } hq_moe_mode;
@@ -260,33 +264,43 @@ HQ_API hq_status hq_moe_permute(int T, int topk, int E, const int32_t *topk_ids,
 /* ------------------------------------------------------------------------
  * MoE expert GEMM ("Announcing Humming", section "Performance": Indexed and
  * Grouped MoE paths; SGLang digest: humming_moe_runner_core_run with gemm
- * types "indexed" and "grouped_contiguous").
+ * types "indexed" and "grouped_contiguous").  Slot s = t * topk + j of token
+ * t multiplies expert e(s) = topk_ids[t, j]:  Y[s] = a_row(s) . W_e(s)^T.
  *   packed_w: hq_pack_weights output for E experts of N x K.
- *   a_bf16: activations in slot-independent token order: [T, K] when
- *       a_per_slot == 0 (every slot of token t multiplies row t, the
- *       gate-up case) or [T * topk, K] when a_per_slot == 1 (slot s
- *       multiplies row s, the down case).  If desc->a_dtype is not BF16 the
- *       activations are quantised on the fly with hq_quant_act's recipe.
- *   expert_offsets / perm / inv_perm: hq_moe_permute outputs.
- *   mode HQ_MOE_GROUPED: rows are first gathered expert-contiguous into the
- *       workspace, then a grouped GEMM runs over them.
- *   mode HQ_MOE_INDEXED: rows are addressed through the routing index.  In
- *       this version the tensor-core kernel reads both modes' rows from the
- *       expert-contiguous copy in the workspace; the modes give bit-identical
- *       results.
- *   combine == 0: out = Y bf16 [T * topk, N], Y[s] = a_row(s) . W_e(s)^T.
+ *   a: activations in slot-independent token order, a_per_slot == 0: [T, K]
+ *       (every slot of token t multiplies row t, the gate-up case), or
+ *       a_per_slot == 1: [T * topk, K] (slot s multiplies row s, the down
+ *       case).  Either bf16 (a_scales == NULL; quantised on the fly with
+ *       hq_quant_act's recipe when desc->a_dtype is not BF16), or, with
+ *       a_scales != NULL, codes already quantised by the caller in
+ *       hq_quant_act's layout for desc->a_dtype (a_scales 4-byte aligned;
+ *       NVFP4 also a_global, device fp32 [1]).
+ *   Routing: expert_offsets [E + 1] and perm [T * topk] from hq_moe_permute;
+ *       or both NULL and topk_ids (device int32 [T, topk]): the call then
+ *       runs the routing prepare itself into the workspace.
+ *   mode HQ_MOE_GROUPED: the routed rows are first copied expert-contiguous
+ *       into the workspace (quantised codes as they are), and the grouped
+ *       GEMM reads each token tile as one block of rows.
+ *   mode HQ_MOE_INDEXED: no copy; the GEMM reads each token tile's rows
+ *       straight from `a` (or from its quantised or decoded copy, which has
+ *       the caller's T or T * topk rows, not the routed T * topk) through
+ *       the routing index, four rows per tensor-memory-access gather.
+ *   combine == 0: out = Y bf16 [T * topk, N] in slot order.
  *   combine == 1: out bf16 [T, N],
  *       out[t] = routed_scale * sum_j topk_weights[t, j] * Y[t * topk + j]
- *       (fp32 sum over j in increasing j; Y rounded to bf16 first).
- * The result does not depend on the mode.
+ *       (fp32 sum over j in increasing j; Y rounded to bf16 first); N a
+ *       multiple of 8.
+ * Both modes give bit-identical results (the same rows in the same tiles
+ * and k order).  `workspace`: hq_moe_workspace_bytes() bytes (enough for
+ * on-the-fly quantisation and internal routing), 16-byte aligned.
  * ---------------------------------------------------------------------- */
 HQ_API size_t hq_moe_workspace_bytes(hq_moe_mode mode, const hq_quant_desc *desc, int T, int topk, int E,
                               int N, int K, int a_per_slot, int combine);
 HQ_API hq_status hq_moe_gemm(hq_moe_mode mode, const hq_quant_desc *desc, int T, int topk, int E, int N,
-                      int K, const void *packed_w, const void *a_bf16, int a_per_slot,
-                      const int32_t *expert_offsets, const int32_t *perm,
-                      const int32_t *inv_perm, const float *topk_weights, float routed_scale,
-                      int combine, void *out_bf16, void *workspace, size_t ws_bytes,
+                      int K, const void *packed_w, const void *a, const void *a_scales,
+                      const float *a_global, int a_per_slot, const int32_t *topk_ids,
+                      const float *topk_weights, const int32_t *expert_offsets, const int32_t *perm,
+                      int combine, float routed_scale, void *out_bf16, void *workspace, size_t ws_bytes,
                       hq_stream_t stream);
 
 /* ------------------------------------------------------------------------

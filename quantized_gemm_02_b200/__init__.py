@@ -51,11 +51,13 @@ class QuantDesc(ctypes.Structure):
     _fields_ = [
         ("w_dtype", ctypes.c_int32), ("w_group", ctypes.c_int32), ("w_scale_dtype", ctypes.c_int32),
         ("w_has_zero", ctypes.c_int32), ("w_has_global", ctypes.c_int32), ("a_dtype", ctypes.c_int32),
+        ("a_group", ctypes.c_int32),
     ]
 
     def __repr__(self):
-        return ("QuantDesc(w_dtype=%d, w_group=%d, w_scale_dtype=%d, w_has_zero=%d, w_has_global=%d, a_dtype=%d)"
-                % (self.w_dtype, self.w_group, self.w_scale_dtype, self.w_has_zero, self.w_has_global, self.a_dtype))
+        return ("QuantDesc(w_dtype=%d, w_group=%d, w_scale_dtype=%d, w_has_zero=%d, w_has_global=%d, a_dtype=%d, "
+                "a_group=%d)" % (self.w_dtype, self.w_group, self.w_scale_dtype, self.w_has_zero, self.w_has_global,
+                                 self.a_dtype, self.a_group))
 
 
 class ComputeConfig(ctypes.Structure):
@@ -105,7 +107,7 @@ def _lib() -> ctypes.CDLL:
             "hq_gemm": (I, [D, I, I, I, P, P, P, P, P, P, Z, P]),
             "hq_moe_permute": (I, [I, I, I, P, P, P, P, P]),
             "hq_moe_workspace_bytes": (Z, [I, D, I, I, I, I, I, I, I]),
-            "hq_moe_gemm": (I, [I, D, I, I, I, I, I, P, P, I, P, P, P, P, F, I, P, P, Z, P]),
+            "hq_moe_gemm": (I, [I, D, I, I, I, I, I, P, P, P, P, I, P, P, P, P, I, F, P, P, Z, P]),
             "hq_moe_masked_workspace_bytes": (Z, [D, I, I, I, I, I]),
             "hq_moe_gemm_masked": (I, [D, I, I, I, I, P, P, P, I, P, P, Z, P]),
             "hq_silu_and_mul": (I, [I, I, P, P, P]),
@@ -242,12 +244,12 @@ def hq_silu_and_mul(R, I, y, out, stream=None):
     _check("hq_silu_and_mul", _lib().hq_silu_and_mul(R, I, _ptr(y), _ptr(out), _stream(stream)))
 
 
-def hq_moe_gemm(mode, desc, T, topk, E, N, K, packed_w, a, a_per_slot, expert_offsets, perm, inv_perm,
-                topk_weights, routed_scale, combine, out, workspace, ws_bytes, stream=None):
+def hq_moe_gemm(mode, desc, T, topk, E, N, K, packed_w, a, a_scales, a_global, a_per_slot, topk_ids, topk_weights,
+                expert_offsets, perm, combine, routed_scale, out, workspace, ws_bytes, stream=None):
     _check("hq_moe_gemm", _lib().hq_moe_gemm(
-        mode, ctypes.byref(desc), T, topk, E, N, K, _ptr(packed_w), _ptr(a), a_per_slot, _ptr(expert_offsets),
-        _ptr(perm), _ptr(inv_perm), _ptr(topk_weights), float(routed_scale), combine, _ptr(out),
-        _ptr(workspace), ws_bytes, _stream(stream)))
+        mode, ctypes.byref(desc), T, topk, E, N, K, _ptr(packed_w), _ptr(a), _ptr(a_scales), _ptr(a_global),
+        a_per_slot, _ptr(topk_ids), _ptr(topk_weights), _ptr(expert_offsets), _ptr(perm), combine,
+        float(routed_scale), _ptr(out), _ptr(workspace), ws_bytes, _stream(stream)))
 
 
 def hq_moe_unpermute_sum(T, topk, N, y, inv_perm, topk_weights, routed_scale, out, stream=None):

@@ -32,7 +32,7 @@ hq_status launch_tc_gemm(const Layout &L, const void *packed, const void *a_bf16
 hq_status launch_bs_gemm(const Layout &L, const void *packed, int E, const void *a_codes, int a_rows,
                          const void *a_scales, int a_div, const float *a_global, int M, int moe,
                          const int32_t *offsets, const int32_t *perm, void *out, const TcLaunch &t,
-                         void *workspace, void *sf_tiles, cudaStream_t st);
+                         void *workspace, void *sf_tiles, cudaStream_t st, int gather = 0);
 size_t bs_sf_tiles_bytes(const Layout &L, const TcLaunch &t);
 hq_status launch_gather_bytes(int R, int row_bytes, const void *a, const int32_t *idx, int div, void *out,
                               cudaStream_t st);
@@ -212,21 +212,27 @@ static hq_status plan_moe_masked(const hq_quant_desc *d, int E, int slab, int N,
 struct MoeWs {
   void *split, *y, *a_bf16, *codes, *scales, *glob, *amax;
   void *s_codes, *s_scales;  // block-scaled layouts: expert-sorted codes, scale chunks per token tile
+  int32_t *r_off, *r_perm, *r_inv;  // routing prepared by the call itself (from topk_ids)
 };
 
-static size_t moe_ws(const MoePlan &pl, hq_moe_mode mode, int K, int N, int combine, uint8_t *base, MoeWs *w) {
+// Workspace of an MoE call.  Grouped mode stages the R routed rows
+// expert-contiguous (bf16 rows for the dequantisation kernels, quantised
+// codes for the block-scaled MMA); indexed mode stages nothing for bf16
+// activations and only the caller's rows decoded to bf16 for quantised ones
+// on the dequantisation path (src_rows rows, not R).  `route` adds room for
+// the routing prepare of a call given topk_ids alone.
+static size_t moe_ws(const MoePlan &pl, hq_moe_mode mode, int E, int K, int N, int combine, bool route,
+                     uint8_t *base, MoeWs *w) {
   Carver c{base};
+  const bool indexed = (mode == HQ_MOE_INDEXED);
   w->split = c.take(tc_workspace_bytes(pl.s));
   w->y = combine ? c.take((size_t)pl.R * N * 2) : nullptr;
-  // both modes stage the expert-sorted rows (see hq_moe_gemm): bf16 rows, or
-  // for a block-scaled layout the quantised codes and scales as they are
-  (void)mode;
+  w->a_bf16 = w->s_codes = w->s_scales = nullptr;
   if (pl.L.bs == BS_NONE) {
-    w->a_bf16 = c.take((size_t)pl.R * K * 2);
-    w->s_codes = w->s_scales = nullptr;
+    if (!indexed) w->a_bf16 = c.take((size_t)pl.R * K * 2);
+    else if (pl.afmt != A_BF16) w->a_bf16 = c.take((size_t)pl.src_rows * K * 2);
   } else {
-    w->a_bf16 = nullptr;
-    w->s_codes = c.take((size_t)pl.R * act_code_bytes(pl.afmt, K));
+    if (!indexed) w->s_codes = c.take((size_t)pl.R * act_code_bytes(pl.afmt, K));
     w->s_scales = c.take(bs_sf_tiles_bytes(pl.L, pl.s));  // scales in the kernel's chunk order
   }
   if (pl.afmt != A_BF16) {
@@ -237,62 +243,78 @@ static size_t moe_ws(const MoePlan &pl, hq_moe_mode mode, int K, int N, int comb
   } else {
     w->codes = w->scales = w->glob = w->amax = nullptr;
   }
+  w->r_off = w->r_perm = w->r_inv = nullptr;
+  if (route) {
+    w->r_off = (int32_t *)c.take((size_t)(E + 1) * sizeof(int32_t));
+    w->r_perm = (int32_t *)c.take((size_t)pl.R * sizeof(int32_t));
+    w->r_inv = (int32_t *)c.take((size_t)pl.R * sizeof(int32_t));
+  }
   return c.off;
 }
 
-// The GEMM part of every MoE mode, given the routing (offsets, perm): rows
-// are staged expert-contiguous in the workspace (quantised on the fly when
-// the description asks: `counts` selects the masked layout's quantiser),
-// then the grouped tensor-core GEMM, then the optional weighted combine.
-static hq_status moe_run(const MoePlan &pl, int T, int topk, int E, int N, int K, const void *packed_w,
-                         const void *a_bf16, int div, const int32_t *counts, const int32_t *expert_offsets,
-                         const int32_t *perm, const float *topk_weights, float routed_scale, int combine,
-                         void *out_bf16, const MoeWs &w, cudaStream_t st) {
-  const void *a_use = a_bf16;
-  const float *row_scale = nullptr;
-  const float *a_global = nullptr;
-  // The tensor-core kernel reads activation tiles by TMA from expert-sorted
-  // rows in both modes: the rows are gathered (and, for quantised
-  // activations, quantised on the fly and decoded exactly) into the
-  // workspace first.  Results do not depend on the mode.
-  const int a_indexed = 0;
+// The GEMM part of every MoE mode, given the routing (offsets, perm).
+// Activation rows: bf16 `a`, quantised here when the description asks
+// (`counts` selects the masked layout's quantiser), or the caller's codes
+// (`a_scales` non-null).  Grouped mode copies the routed rows
+// expert-contiguous first; indexed mode lets the GEMM gather the caller's
+// rows through the routing index.  Then the optional weighted combine.
+static hq_status moe_run(const MoePlan &pl, hq_moe_mode mode, int T, int topk, int E, int N, int K,
+                         const void *packed_w, const void *a, const void *a_scales, const float *a_global, int div,
+                         const int32_t *counts, const int32_t *expert_offsets, const int32_t *perm,
+                         const float *topk_weights, float routed_scale, int combine, void *out_bf16, const MoeWs &w,
+                         cudaStream_t st) {
+  const bool indexed = (mode == HQ_MOE_INDEXED);
   hq_status s = HQ_OK;
   void *y = combine ? w.y : out_bf16;
-  auto quant = [&]() {
-    if (counts)
-      return launch_quant_act_masked(pl.afmt, E, pl.src_rows / E, K, a_bf16, counts, w.codes, w.scales,
-                                     (float *)w.glob, w.amax, st);
-    return launch_quant_act(pl.afmt, pl.src_rows, K, a_bf16, w.codes, w.scales, (float *)w.glob, nullptr, w.amax,
-                            st);
-  };
+  // quantised activation rows (src_rows of them): the caller's or our own
+  const void *codes = a;
+  const void *scales = a_scales;
+  const float *glob = a_global;
+  if (pl.afmt != A_BF16 && !a_scales) {
+    s = counts ? launch_quant_act_masked(pl.afmt, E, pl.src_rows / E, K, a, counts, w.codes, w.scales,
+                                         (float *)w.glob, w.amax, st)
+               : launch_quant_act(pl.afmt, pl.src_rows, K, a, w.codes, w.scales, (float *)w.glob, nullptr, w.amax,
+                                  st);
+    if (s != HQ_OK) return s;
+    codes = w.codes;
+    scales = w.scales;
+    glob = (const float *)w.glob;
+  }
   if (pl.L.bs != BS_NONE) {
-    // quantise the caller rows once, gather codes and scales into expert order
-    s = quant();
-    if (s != HQ_OK) return s;
-    s = launch_gather_bytes(pl.R, (int)act_code_bytes(pl.afmt, K), w.codes, perm, div, w.s_codes, st);
-    if (s != HQ_OK) return s;
-    s = launch_bs_gemm(pl.L, packed_w, E, w.s_codes, pl.R, w.scales, div,
-                       pl.afmt == A_NVFP4 ? (const float *)w.glob : nullptr, 0, 1, expert_offsets, perm, y, pl.s,
-                       w.split, w.s_scales, st);
-    if (s != HQ_OK) return s;
-    if (combine) s = launch_unpermute_sum(T, topk, N, y, nullptr, topk_weights, routed_scale, out_bf16, st);
-    return s;
-  }
-  if (pl.afmt != A_BF16) {
-    s = quant();
-    if (s != HQ_OK) return s;
-    s = launch_act_decode(pl.afmt, pl.R, K, w.codes, w.scales, perm, div, w.a_bf16, st);
-    if (s != HQ_OK) return s;
-    if (pl.afmt == A_FP8) row_scale = (const float *)w.scales;
-    if (pl.afmt == A_NVFP4) a_global = (const float *)w.glob;
+    // block-scaled MMA: the quantised codes go to the tensor core as they are
+    const void *rows = codes;
+    int a_rows = pl.src_rows;
+    if (!indexed) {
+      s = launch_gather_bytes(pl.R, (int)act_code_bytes(pl.afmt, K), codes, perm, div, w.s_codes, st);
+      if (s != HQ_OK) return s;
+      rows = w.s_codes;
+      a_rows = pl.R;
+    }
+    s = launch_bs_gemm(pl.L, packed_w, E, rows, a_rows, scales, div, pl.afmt == A_NVFP4 ? glob : nullptr, 0, 1,
+                       expert_offsets, perm, y, pl.s, w.split, w.s_scales, st, indexed ? 1 : 0);
   } else {
-    s = launch_gather_rows(pl.R, K, a_bf16, perm, div, w.a_bf16, st);
-    if (s != HQ_OK) return s;
+    const void *a_use = a;
+    int a_rows = pl.src_rows;
+    const float *row_scale = nullptr;
+    const float *a_glob = nullptr;
+    if (pl.afmt != A_BF16) {
+      // decoded exactly to bf16: the caller's rows (indexed) or the routed rows (grouped)
+      s = indexed ? launch_act_decode(pl.afmt, pl.src_rows, K, codes, scales, nullptr, 1, w.a_bf16, st)
+                  : launch_act_decode(pl.afmt, pl.R, K, codes, scales, perm, div, w.a_bf16, st);
+      if (s != HQ_OK) return s;
+      a_use = w.a_bf16;
+      a_rows = indexed ? pl.src_rows : pl.R;
+      if (pl.afmt == A_FP8) row_scale = (const float *)scales;
+      if (pl.afmt == A_NVFP4) a_glob = glob;
+    } else if (!indexed) {
+      s = launch_gather_rows(pl.R, K, a, perm, div, w.a_bf16, st);
+      if (s != HQ_OK) return s;
+      a_use = w.a_bf16;
+      a_rows = pl.R;
+    }
+    s = launch_tc_gemm(pl.L, packed_w, a_use, a_rows, row_scale, a_glob, 0, 1, E, expert_offsets, perm, div,
+                       indexed ? 1 : 0, y, pl.s, w.split, st);
   }
-  a_use = w.a_bf16;
-  const int a_rows = (a_indexed ? pl.src_rows : pl.R);
-  s = launch_tc_gemm(pl.L, packed_w, a_use, a_rows, row_scale, a_global, 0, 1, E, expert_offsets, perm, div, a_indexed,
-                     y, pl.s, w.split, st);
   if (s != HQ_OK) return s;
   if (combine) s = launch_unpermute_sum(T, topk, N, y, nullptr, topk_weights, routed_scale, out_bf16, st);
   return s;
@@ -496,30 +518,44 @@ hq_status hq_moe_permute(int T, int topk, int E, const int32_t *topk_ids, int32_
 size_t hq_moe_workspace_bytes(hq_moe_mode mode, const hq_quant_desc *desc, int T, int topk, int E, int N, int K,
                               int a_per_slot, int combine) {
   MoePlan pl;
+  if (mode != HQ_MOE_GROUPED && mode != HQ_MOE_INDEXED) return 0;
   if (plan_moe(desc, T, topk, E, N, K, a_per_slot, &pl) != HQ_OK) return 0;
   MoeWs w;
-  return moe_ws(pl, mode, K, N, combine, nullptr, &w);
+  return moe_ws(pl, mode, E, K, N, combine, true, nullptr, &w);
 }
 
 hq_status hq_moe_gemm(hq_moe_mode mode, const hq_quant_desc *desc, int T, int topk, int E, int N, int K,
-                      const void *packed_w, const void *a_bf16, int a_per_slot, const int32_t *expert_offsets,
-                      const int32_t *perm, const int32_t *inv_perm, const float *topk_weights, float routed_scale,
-                      int combine, void *out_bf16, void *workspace, size_t ws_bytes, hq_stream_t stream) {
+                      const void *packed_w, const void *a, const void *a_scales, const float *a_global,
+                      int a_per_slot, const int32_t *topk_ids, const float *topk_weights,
+                      const int32_t *expert_offsets, const int32_t *perm, int combine, float routed_scale,
+                      void *out_bf16, void *workspace, size_t ws_bytes, hq_stream_t stream) {
   MoePlan pl;
   if (mode != HQ_MOE_GROUPED && mode != HQ_MOE_INDEXED) return HQ_ERR_INVALID_ARG;
   const hq_status ps = plan_moe(desc, T, topk, E, N, K, a_per_slot, &pl);
   if (ps != HQ_OK) return ps;
   if (T == 0) return HQ_OK;
-  if (!packed_w || !a_bf16 || !expert_offsets || !perm || !out_bf16) return HQ_ERR_INVALID_ARG;
-  if (!aligned16(packed_w) || !aligned16(a_bf16) || !aligned16(out_bf16)) return HQ_ERR_INVALID_ARG;
+  if (!packed_w || !a || !out_bf16) return HQ_ERR_INVALID_ARG;
+  if (!aligned16(packed_w) || !aligned16(a) || !aligned16(out_bf16)) return HQ_ERR_INVALID_ARG;
+  const bool routed = expert_offsets && perm;
+  if (!routed && (expert_offsets || perm || !topk_ids)) return HQ_ERR_INVALID_ARG;
+  if (a_scales) {
+    if (pl.afmt == A_BF16 || ((uintptr_t)a_scales & 3u)) return HQ_ERR_INVALID_ARG;
+    if (pl.afmt == A_NVFP4 && !a_global) return HQ_ERR_INVALID_ARG;
+  }
   if (combine && (!topk_weights || (N % 8) != 0)) return HQ_ERR_INVALID_ARG;
-  (void)inv_perm;
   MoeWs w;
-  const size_t need = moe_ws(pl, mode, K, N, combine, (uint8_t *)workspace, &w);
+  const size_t need = moe_ws(pl, mode, E, K, N, combine, true, (uint8_t *)workspace, &w);
   if (!workspace || ws_bytes < need || !aligned16(workspace)) return HQ_ERR_WORKSPACE;
   if (!device_is_sm100()) return HQ_ERR_ARCH;
-  return moe_run(pl, T, topk, E, N, K, packed_w, a_bf16, a_per_slot ? 1 : topk, nullptr, expert_offsets, perm,
-                 topk_weights, routed_scale, combine, out_bf16, w, (cudaStream_t)stream);
+  cudaStream_t st = (cudaStream_t)stream;
+  if (!routed) {
+    const hq_status s = launch_moe_permute(T, topk, E, topk_ids, w.r_off, w.r_perm, w.r_inv, st);
+    if (s != HQ_OK) return s;
+    expert_offsets = w.r_off;
+    perm = w.r_perm;
+  }
+  return moe_run(pl, mode, T, topk, E, N, K, packed_w, a, a_scales, a_global, a_per_slot ? 1 : topk, nullptr,
+                 expert_offsets, perm, topk_weights, routed_scale, combine, out_bf16, w, st);
 }
 
 size_t hq_moe_masked_workspace_bytes(const hq_quant_desc *desc, int E, int slab, int N, int K, int expected_m) {
@@ -527,7 +563,7 @@ size_t hq_moe_masked_workspace_bytes(const hq_quant_desc *desc, int E, int slab,
   if (plan_moe_masked(desc, E, slab, N, K, expected_m, &pl) != HQ_OK) return 0;
   MoeWs w;
   Carver c{nullptr};
-  c.off = moe_ws(pl, HQ_MOE_GROUPED, K, N, 0, nullptr, &w);
+  c.off = moe_ws(pl, HQ_MOE_GROUPED, E, K, N, 0, false, nullptr, &w);
   c.take((size_t)(E + 1) * sizeof(int32_t));
   c.take((size_t)E * slab * sizeof(int32_t));
   return c.off;
@@ -543,7 +579,7 @@ hq_status hq_moe_gemm_masked(const hq_quant_desc *desc, int E, int slab, int N, 
   if (!aligned16(packed_w) || !aligned16(a_bf16) || !aligned16(out_bf16)) return HQ_ERR_INVALID_ARG;
   MoeWs w;
   Carver c{(uint8_t *)workspace};
-  c.off = moe_ws(pl, HQ_MOE_GROUPED, K, N, 0, (uint8_t *)workspace, &w);
+  c.off = moe_ws(pl, HQ_MOE_GROUPED, E, K, N, 0, false, (uint8_t *)workspace, &w);
   int32_t *offsets = (int32_t *)c.take((size_t)(E + 1) * sizeof(int32_t));
   int32_t *perm = (int32_t *)c.take((size_t)E * slab * sizeof(int32_t));
   if (!workspace || ws_bytes < c.off || !aligned16(workspace)) return HQ_ERR_WORKSPACE;
@@ -552,8 +588,8 @@ hq_status hq_moe_gemm_masked(const hq_quant_desc *desc, int E, int slab, int N, 
   const hq_status s = launch_moe_masked_prepare(E, slab, expert_num_tokens, offsets, perm, st);
   if (s != HQ_OK) return s;
   // every valid row is its own slot: one row per slot (div = 1), no combine
-  return moe_run(pl, E * slab, 1, E, N, K, packed_w, a_bf16, 1, expert_num_tokens, offsets, perm, nullptr, 1.f, 0,
-                 out_bf16, w, st);
+  return moe_run(pl, HQ_MOE_GROUPED, E * slab, 1, E, N, K, packed_w, a_bf16, nullptr, nullptr, 1, expert_num_tokens,
+                 offsets, perm, nullptr, 1.f, 0, out_bf16, w, st);
 }
 
 hq_status hq_silu_and_mul(int R, int I, const void *y_bf16, void *out_bf16, hq_stream_t stream) {

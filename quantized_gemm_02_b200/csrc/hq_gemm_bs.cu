@@ -281,6 +281,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(s_total + 1);
   int *s_abort = reinterpret_cast<int *>(tmem_slot + 1);
   int *s_tpre = s_abort + 1;  // [E+1] MoE: prefix of token tiles per expert
+  int *s_rows = s_tpre + (p.moe ? p.E + 1 : 0);  // [BNT] indexed mode: caller rows of the producer's tile
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int cta = blockIdx.x;
@@ -407,24 +408,41 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (++s == NS) { s = 0; ph ^= 1; }
     }
   } else if (warp == WARP_ACT) {
-    // ================= activation producer: codes (2-D TMA) + scale chunks (bulk) =================
+    // ================= activation producer: codes (2-D TMA, or 4-row gathers =================
+    // ================= in MoE indexed mode) + scale chunks (bulk)            =================
     Walk w;
     w.start(beg, end, p.KB);
-    int cur_t = -1, base = 0;
+    int cur_t = -1, base = 0, nvalid = 0;
     const uint8_t *sfsrc = nullptr;
     for (int is = 0, s = 0, ph = 0; w.left > 0; ++is, w.next(p.KB)) {
       if (w.t != cur_t) {
-        base = tile_info(w.t).base;
+        const TileInfo ti = tile_info(w.t);
+        base = ti.base;
+        nvalid = ti.nvalid;
         // scale chunks of this tile's token slot, laid out by bs_sf_tiles_kernel
         sfsrc = p.a_sf + (size_t)(w.t / p.ntw) * p.KB * (C::SF_CH * C::SFB_CHB);
         cur_t = w.t;
+        if (p.gather) {
+          // the tile's caller rows; positions past the valid rows repeat the
+          // last one (loaded, never written back)
+          for (int i = lane; i < BNT; i += 32) s_rows[i] = p.perm[base + min(i, nvalid - 1)] / p.a_div;
+          __syncwarp();
+        }
       }
       if (is >= NS && !mbar_wait(&sfree[s], ph ^ 1)) { *s_abort = 1; break; }
       if (*(volatile int *)s_abort) break;
       if (lane == 0) {
         uint8_t *st = smem + s * C::STAGE;
-        mbar_arrive_expect_tx(&full[s], (uint32_t)(C::A_SMEM + C::SF_CH * C::SFB_CHB));
-        tma_load_2d(st + C::W_SMEM, &a_map, w.ks * 128, base, &full[s]);
+        if (!p.gather) {
+          mbar_arrive_expect_tx(&full[s], (uint32_t)(C::A_SMEM + C::SF_CH * C::SFB_CHB));
+          tma_load_2d(st + C::W_SMEM, &a_map, w.ks * 128, base, &full[s]);
+        } else {
+          const int ng = (nvalid + 3) >> 2;
+          mbar_arrive_expect_tx(&full[s], (uint32_t)(ng * 4 * 128 + C::SF_CH * C::SFB_CHB));
+          for (int gi = 0; gi < ng; ++gi)
+            tc::tma_gather4(st + C::W_SMEM + gi * 512, &a_map, w.ks * 128, s_rows[4 * gi], s_rows[4 * gi + 1],
+                            s_rows[4 * gi + 2], s_rows[4 * gi + 3], &full[s]);
+        }
         if constexpr (C::SF_CH > 0)
           bulk_g2s(st + C::SFB_OFF, sfsrc + (size_t)w.ks * C::SF_CH * C::SFB_CHB, C::SF_CH * C::SFB_CHB, &full[s]);
       }
@@ -661,14 +679,15 @@ size_t bs_sf_tiles_bytes(const Layout &L, const TcLaunch &t) {
 
 // a_codes: `a_rows` activation rows (MXFP8, FP8: K E4M3 bytes per row; NVFP4:
 // K/2 packed bytes) in the order the tiles read them: dense rows of a, or MoE
-// expert-sorted rows.  a_scales: the caller's scale rows (MXFP8: K/32 E8M0,
+// expert-sorted rows; with `gather` (MoE indexed mode) the caller's rows,
+// expert-sorted row r read from row perm[r] / a_div.  a_scales: the caller's scale rows (MXFP8: K/32 E8M0,
 // NVFP4: K/16 UE4M3, FP8: one fp32 per row), read through perm / div for MoE.
 // Outputs go to row perm[r] for MoE.  sf_tiles: bs_sf_tiles_bytes() of
 // scratch (none for FP8).
 hq_status launch_bs_gemm(const Layout &L, const void *packed, int E, const void *a_codes, int a_rows,
                          const void *a_scales, int a_div, const float *a_global, int M, int moe,
                          const int32_t *offsets, const int32_t *perm, void *out, const TcLaunch &t,
-                         void *workspace, void *sf_tiles, cudaStream_t st) {
+                         void *workspace, void *sf_tiles, cudaStream_t st, int gather) {
   if (L.bs == BS_NONE || t.kind != 2) return HQ_ERR_UNSUPPORTED;
   if (((uintptr_t)packed & 31) != 0 || ((uintptr_t)a_scales & 3) != 0) return HQ_ERR_INVALID_ARG;
   const int kstage = L.bs == BS_NV ? 256 : 128;
@@ -676,7 +695,8 @@ hq_status launch_bs_gemm(const Layout &L, const void *packed, int E, const void 
   const int row_bytes = L.bs == BS_NV ? L.K / 2 : L.K;
   CUtensorMap wm, am;
   if (!make_bs_weight_map(&wm, L, packed, E)) return HQ_ERR_CUDA;
-  if (!make_bs_act_map(&am, a_codes, a_rows, row_bytes, t.bnt)) return HQ_ERR_CUDA;
+  // indexed mode: one-row boxes for the 4-row gathers of caller rows
+  if (!make_bs_act_map(&am, a_codes, a_rows, row_bytes, gather ? 1 : t.bnt)) return HQ_ERR_CUDA;
   if (L.bs != BS_F8) {
     const size_t words = (size_t)t.mtiles * (L.K / kstage) * sf_ch * (t.bnt > 128 ? 256 : 128);
     size_t blocks = (words + 255) / 256;
@@ -702,7 +722,8 @@ hq_status launch_bs_gemm(const Layout &L, const void *packed, int E, const void 
   // FP8: per-token scales in the epilogue, caller row perm[r] / div for MoE;
   // the block scales were laid out per token tile above
   p.row_scale = L.bs == BS_F8 ? (const float *)a_scales : nullptr;
-  p.a_div = L.bs == BS_F8 ? a_div : 1;
+  p.a_div = a_div;
+  p.gather = gather;
   p.out = (uint16_t *)out;
   p.ntw = t.ntw;
   p.mtiles = t.mtiles;

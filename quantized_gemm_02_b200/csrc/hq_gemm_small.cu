@@ -454,23 +454,45 @@ __global__ void __launch_bounds__(THREADS, 1) dec_gemm_kernel(const __grid_const
       __syncwarp();
     }
   } else if (warp == WARP_ACT) {
-    // ================= activation producer: one 3-D TMA per stage =================
+    // ================= activation producer: one 3-D TMA per stage, or =================
+    // ================= (MoE indexed mode) 4-row gathers per 64-k block =================
     Walk w;
     w.start(beg, end, p.KB);
     Ring rs;
     rs.init();
-    int cur_t = -1, base = 0;
+    int cur_t = -1, base = 0, nvalid = 0, my_row = 0;
     for (int is = 0; w.left > 0; ++is, w.next(p.KB), rs.next(NS)) {
       if (w.t != cur_t) {
-        base = tile_info(w.t).base;
+        const TileInfo ti = tile_info(w.t);
+        base = ti.base;
+        nvalid = ti.nvalid;
         cur_t = w.t;
+        // indexed mode: lane i holds the caller row of the tile's row i
+        // (rows past the valid ones repeat the last: loaded, never written back)
+        if (p.gather) my_row = p.perm[base + min(lane, nvalid - 1)] / p.a_div;
       }
       if (is >= NS && !mbar_wait(&sfree[rs.idx], rs.phase ^ 1)) { *s_abort = 1; break; }
       if (*(volatile int *)s_abort) break;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&full[rs.idx], (uint32_t)C::ACT);
-        // box {64 k, BNT rows, KPS blocks}
-        tma_load_3d(smem + rs.idx * C::STAGE, &act_map, 0, base, w.kb, &full[rs.idx]);
+      uint8_t *st = smem + rs.idx * C::STAGE;
+      if (!p.gather) {
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[rs.idx], (uint32_t)C::ACT);
+          // box {64 k, BNT rows, KPS blocks}
+          tma_load_3d(st, &act_map, 0, base, w.kb, &full[rs.idx]);
+        }
+      } else {
+        const int ng = (nvalid + 3) >> 2;  // 4-row gathers per 64-k block
+        if (lane == 0) mbar_arrive_expect_tx(&full[rs.idx], (uint32_t)(w.n * ng * 4 * 128));
+        for (int gi = 0; gi < ng; ++gi) {
+          const int r0 = __shfl_sync(0xffffffffu, my_row, 4 * gi);
+          const int r1 = __shfl_sync(0xffffffffu, my_row, 4 * gi + 1);
+          const int r2 = __shfl_sync(0xffffffffu, my_row, 4 * gi + 2);
+          const int r3 = __shfl_sync(0xffffffffu, my_row, 4 * gi + 3);
+          if (lane == 0)
+            for (int j = 0; j < w.n; ++j)
+              tc::tma_gather4(st + j * C::ACT_KB + gi * 512, &act_map, (w.kb + j) * TILE_K, r0, r1, r2, r3,
+                              &full[rs.idx]);
+        }
       }
       __syncwarp();
     }
@@ -668,7 +690,11 @@ static hq_status dec_launch_wf(const CUtensorMap &map, const tc::Params &p, cons
 hq_status launch_dec_gemm(const Layout &L, const tc::Params &p, const void *a, int a_rows, const TcLaunch &t,
                           cudaStream_t st, bool e4m3_act) {
   CUtensorMap map;
-  if (!make_act_map_3d(&map, a, a_rows, L.K, t.bnt, e4m3_act)) return HQ_ERR_CUDA;
+  // indexed mode: a 2-D map of the caller's rows with one-row boxes for the
+  // 4-row gathers (bf16 only); otherwise the 3-D map of KPS blocks per box
+  if (p.gather ? !make_act_map(&map, a, a_rows, L.K, 1, false)
+               : !make_act_map_3d(&map, a, a_rows, L.K, t.bnt, e4m3_act))
+    return HQ_ERR_CUDA;
   switch (L.fmt) {
     case W_INT4: return dec_launch_wf<W_INT4>(map, p, t, st);
     case W_UINT4: return dec_launch_wf<W_UINT4>(map, p, t, st);

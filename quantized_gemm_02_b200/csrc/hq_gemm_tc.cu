@@ -342,6 +342,7 @@ __global__ void __launch_bounds__(THREADS, (BNT <= 64 ? 2 : 1)) tc_gemm_kernel(c
   int *s_abort = reinterpret_cast<int *>(tmem_slot + 1);
   int *s_last = s_abort + 1;
   int *s_tpre = s_last + 1;  // [E+1] MoE: prefix of token tiles per expert
+  int *s_rows = s_tpre + (p.moe ? p.E + 1 : 0);  // [BNT] indexed mode: caller rows of the producer's tile
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int cta = blockIdx.x;
@@ -451,6 +452,12 @@ __global__ void __launch_bounds__(THREADS, (BNT <= 64 ? 2 : 1)) tc_gemm_kernel(c
       int t, ukb0, ukb1, usp;
       if (!unit_at(sch, cta, p.nctas, p.KB, u, t, ukb0, ukb1, usp)) break;
       const TileInfo ti = tile_info(t);
+      if (p.gather) {
+        // the tile's caller rows, read once per tile; positions past the
+        // valid rows repeat the last one (loaded, never written back)
+        for (int i = lane; i < BNT; i += 32) s_rows[i] = p.perm[ti.base + min(i, ti.nvalid - 1)] / p.a_div;
+        __syncwarp();
+      }
       const int nst = (ukb1 - ukb0 + C::KPS - 1) / C::KPS;
       const int rot = stage_rotation(cta, nst);
       for (int i = 0; i < nst; ++i, ++is) {
@@ -474,13 +481,10 @@ __global__ void __launch_bounds__(THREADS, (BNT <= 64 ? 2 : 1)) tc_gemm_kernel(c
           if (!p.gather) {
             tma_load_2d(st + j * C::ACT_KB, &act_map, kbj * TILE_K, ti.base, &full[s]);
           } else {
-            for (int i = 0; i < ti.nvalid; i += 4) {
-              int r[4];
-#pragma unroll
-              for (int q = 0; q < 4; ++q) r[q] = p.perm[ti.base + min(i + q, ti.nvalid - 1)] / p.a_div;
-              tma_gather4(st + j * C::ACT_KB + i * row_bytes, &act_map, kbj * TILE_K, r[0], r[1], r[2], r[3],
-                          &full[s]);
-            }
+            // four rows per gather, each 64 k (one 128-byte swizzled row of the tile)
+            for (int i = 0; i < ti.nvalid; i += 4)
+              tma_gather4(st + j * C::ACT_KB + i * row_bytes, &act_map, kbj * TILE_K, s_rows[i], s_rows[i + 1],
+                          s_rows[i + 2], s_rows[i + 3], &full[s]);
           }
         }
         bulk_g2s_stream(st + C::ACT, eb + p.w_off + ((size_t)ti.wt * p.KB + kbs) * TR::unit, TR::unit * nblk,
@@ -930,9 +934,10 @@ hq_status launch_tc_gemm(const Layout &L, const void *packed, const void *a_bf16
   p.counters = (int *)workspace;
   p.partial = (float *)((uint8_t *)workspace + tc_counter_bytes(t));
   if (t.kind == 1) {
-    if (gather) return HQ_ERR_UNSUPPORTED;
+    if (gather && e4m3_act) return HQ_ERR_UNSUPPORTED;
     return launch_dec_gemm(L, p, a_bf16, a_rows, t, st, e4m3_act);
   }
+  if (gather && e4m3_act) return HQ_ERR_UNSUPPORTED;
   switch (L.fmt) {
     case W_INT4: return tc_launch_wf<W_INT4>(map, p, t, st);
     case W_UINT4: return tc_launch_wf<W_UINT4>(map, p, t, st);

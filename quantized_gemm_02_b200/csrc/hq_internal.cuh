@@ -103,12 +103,14 @@ inline bool valid_k(const hq_quant_desc *d, int K) {
   return d->w_group == 0 || (K % d->w_group) == 0;
 }
 
+// The activation format of a description; a_group must be 0 (the format's
+// own scale granularity) or that granularity spelled out.
 inline bool act_format(const hq_quant_desc *d, int *afmt) {
   switch (d->a_dtype) {
-    case HQ_BF16: *afmt = A_BF16; return true;
-    case HQ_E4M3: *afmt = A_FP8; return true;
-    case HQ_MXFP8: *afmt = A_MXFP8; return true;
-    case HQ_NVFP4: *afmt = A_NVFP4; return true;
+    case HQ_BF16: *afmt = A_BF16; return d->a_group == 0;
+    case HQ_E4M3: *afmt = A_FP8; return d->a_group == 0;
+    case HQ_MXFP8: *afmt = A_MXFP8; return d->a_group == 0 || d->a_group == 32;
+    case HQ_NVFP4: *afmt = A_NVFP4; return d->a_group == 0 || d->a_group == 16;
     default: return false;
   }
 }

@@ -84,6 +84,47 @@ def test_host_validation_without_device():
     hq.hq_gemm(d, 0, 64, 128, 16, 16, None, None, 16, None, 0, stream=0)
 
 
+def test_moe_gemm_host_validation():
+    d = cdesc("mxfp4")
+    T, k, E, N, K = 4, 2, 8, 128, 256
+    wsb = hq.hq_moe_workspace_bytes(hq.HQ_MOE_INDEXED, d, T, k, E, N, K, 0, 0)
+    assert wsb > 0
+    call = lambda desc, a_s=None, a_g=None, ids=None, off=None, perm=None, ws=16: hq.hq_moe_gemm(
+        hq.HQ_MOE_INDEXED, desc, T, k, E, N, K, 16, 16, a_s, a_g, 0, ids, None, off, perm, 0, 1.0, 16, ws, wsb,
+        stream=0)
+    with pytest.raises(hq.HQError) as e:
+        call(d)  # neither routing arrays nor topk_ids
+    assert e.value.status == 1
+    with pytest.raises(hq.HQError) as e:
+        call(d, off=16)  # offsets without perm
+    assert e.value.status == 1
+    with pytest.raises(hq.HQError) as e:
+        call(d, a_s=16, ids=16)  # scales for bf16 activations
+    assert e.value.status == 1
+    with pytest.raises(hq.HQError) as e:
+        call(cdesc("nvfp4", "nvfp4"), a_s=16, ids=16)  # NVFP4 codes without their tensor scale
+    assert e.value.status == 1
+    with pytest.raises(hq.HQError) as e:
+        call(cdesc("mxfp4", "mxfp8"), a_s=18, ids=16)  # scales not 4-byte aligned
+    assert e.value.status == 1
+    with pytest.raises(hq.HQError) as e:
+        call(d, ids=16, ws=None)
+    assert e.value.status == 3
+    bad = cdesc("mxfp4", "mxfp8")
+    bad.a_group = 16  # MXFP8 scales are per 32
+    with pytest.raises(hq.HQError) as e:
+        call(bad, ids=16)
+    assert e.value.status == 2
+    assert hq.hq_moe_workspace_bytes(hq.HQ_MOE_INDEXED, bad, T, k, E, N, K, 0, 0) == 0
+    ok = cdesc("mxfp4", "mxfp8")
+    ok.a_group = 32
+    assert hq.hq_moe_workspace_bytes(hq.HQ_MOE_INDEXED, ok, T, k, E, N, K, 0, 0) > 0
+    # indexed mode stages no rows for bf16 activations; grouped copies T * topk rows
+    g = hq.hq_moe_workspace_bytes(hq.HQ_MOE_GROUPED, d, 64, 8, 256, 4096, 7168, 0, 0)
+    i = hq.hq_moe_workspace_bytes(hq.HQ_MOE_INDEXED, d, 64, 8, 256, 4096, 7168, 0, 0)
+    assert g - i >= 64 * 8 * 7168 * 2
+
+
 def test_compute_config_queries():
     d = cdesc("uint4_g128")
     assert hq.hq_gemm_config_workspace_bytes(d, None, 16, 8192, 8192) == hq.hq_gemm_workspace_bytes(d, 16, 8192, 8192)

@@ -232,8 +232,8 @@ def _moe_full(wname, aname, T, part, zipf, seed, modes=(0, 1)):
             wsb = hq.hq_moe_workspace_bytes(mode, d, T, K_TOP, E_, N, K, per_slot, combine)
             ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
             out = torch.full(((T if combine else T * K_TOP), N), float("nan"), dtype=torch.bfloat16, device="cuda")
-            hq.hq_moe_gemm(mode, d, T, K_TOP, E_, N, K, packed, x, per_slot, off, perm, inv, wts, 1.0, combine, out,
-                           ws, wsb)
+            hq.hq_moe_gemm(mode, d, T, K_TOP, E_, N, K, packed, x, None, None, per_slot, None, wts, off, perm, combine,
+                           1.0, out, ws, wsb)
             torch.cuda.synchronize()
             assert hq.hq_device_error() == 0
             res[(mode, combine)] = out

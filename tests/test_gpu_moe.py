@@ -44,13 +44,16 @@ def test_permute_rejects_bad_ids():
     assert hq.hq_device_error() == 0  # cleared
 
 
-def run_moe(mode, wname, aname, packed, T, k, E, N, K, a, a_per_slot, off, perm, inv, w, rs, combine):
+def run_moe(mode, wname, aname, packed, T, k, E, N, K, a, a_per_slot, off, perm, inv, w, rs, combine, ids=None,
+            a_scales=None, a_global=None):
+    """One hq_moe_gemm call; with ``ids`` and no off / perm the call routes itself."""
     import quantized_gemm_02_b200 as hq
     d = cdesc(wname, aname)
     wsb = hq.hq_moe_workspace_bytes(mode, d, T, k, E, N, K, a_per_slot, combine)
     ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
     out = torch.empty((T if combine else T * k), N, dtype=torch.bfloat16, device="cuda")
-    hq.hq_moe_gemm(mode, d, T, k, E, N, K, packed, a, a_per_slot, off, perm, inv, w, rs, combine, out, ws, wsb)
+    hq.hq_moe_gemm(mode, d, T, k, E, N, K, packed, a, a_scales, a_global, a_per_slot, ids, w, off, perm, combine, rs,
+                   out, ws, wsb)
     return out
 
 
@@ -108,6 +111,59 @@ def test_moe_block_scaled_wide_token_tiles(wname, aname):
     assert torch.equal(res[(0, 0)], res[(1, 0)])
     assert_close(res[(0, 0)].cpu(), Y, B, what="per-slot Y")
     assert_close(res[(0, 1)].cpu(), out, bound, rel=8e-3, what="combined")
+
+
+@pytest.mark.parametrize("wname,aname,T", [("mxfp4", "bf16", 100), ("mxfp4", "bf16", 300), ("int4_g128", "fp8", 300),
+                                           ("nvfp4", "mxfp8", 100), ("uint4_g64", "nvfp4", 300)])
+def test_moe_indexed_multi_stage_tiles(wname, aname, T):
+    # 50 and 150 rows per expert on average: 64- and 256-token tiles of the
+    # multi-stage kernel; indexed mode gathers the caller's rows (bf16, or
+    # the caller's rows decoded once) with 4-row tensor gathers, grouped mode
+    # copies the routed rows first; both must agree bit for bit
+    E, k, N, K = 16, 8, 96, 256
+    res, out, bound, Y, B, ids, wts = moe_case(wname, aname, T, E, k, N, K, 0, seed=41 + T, zipf=True)
+    assert torch.equal(res[(0, 0)], res[(1, 0)])
+    assert torch.equal(res[(0, 1)], res[(1, 1)])
+    assert_close(res[(1, 0)].cpu(), Y, B, what="indexed per-slot Y")
+    assert_close(res[(1, 1)].cpu(), out, bound, rel=8e-3, what="indexed combined")
+
+
+@pytest.mark.parametrize("wname,aname", [("mxfp4", "mxfp8"), ("nvfp4", "nvfp4"), ("int4_g128", "fp8"), ("fp8", "fp8"),
+                                         ("mxfp4", "bf16")])
+@pytest.mark.parametrize("mode", [0, 1])
+def test_moe_caller_quantised_and_self_routed(wname, aname, mode):
+    # activations quantised by the caller (hq_quant_act) and passed with
+    # their scales, routing from topk_ids alone (the call prepares it):
+    # bit-identical to on-the-fly quantisation with explicit routing, and
+    # within the tolerance of the oracle
+    T, E, k, N, K = 37, 16, 4, 96, 256
+    g = synth.generator(77)
+    x = synth.bf16_normal((T, K), g)
+    ids, wts = synth.routing_softmax_topk(T, E, k, g)
+    w = make_weights(wname, E, N, K, seed=78)
+    packed = gpu_pack(wname, w, E, N, K, aname)
+    off, perm, inv = gpu_permute(ids.cuda(), E)
+    ref = run_moe(mode, wname, aname, packed, T, k, E, N, K, x.cuda(), 0, off, perm, inv, wts.cuda(), 1.5, 1)
+    if aname == "bf16":
+        a, a_s, a_g = x.cuda(), None, None
+    else:
+        a, a_s, a_g = gpu_quant(aname, x.cuda())
+        if aname != "nvfp4":
+            a_g = None
+    got = run_moe(mode, wname, aname, packed, T, k, E, N, K, a, 0, None, None, None, wts.cuda(), 1.5, 1,
+                  ids=ids.cuda(), a_scales=a_s, a_global=a_g)
+    torch.cuda.synchronize()
+    assert torch.equal(got, ref)
+    xb = np_bits(x)
+    if aname == "bf16":
+        A, row = O.decode_act("bf16", T, K, xb)
+    else:
+        q, s, og = oracle_quant(aname, xb)
+        A, row = O.decode_act(aname, T, K, q, s, og)
+    rows = np.repeat(np.arange(T), k)
+    o, b, _, _ = O.moe(A[rows], ids.numpy(), wts.numpy(), oracle_decoder(wname, w, N, K), 1.5,
+                       None if row is None else row[rows])
+    assert_close(got.cpu(), o, b, rel=8e-3, what=f"caller-quantised {wname}x{aname} mode {mode}")
 
 
 def test_moe_single_expert_top1_equals_dense():
