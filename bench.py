@@ -3,27 +3,42 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl hq|reference] [--workload NAME]
                     [--shape M,N,K [--shape-fmt uint4|nvfp4|fp8]] [--eager] [--no-cpu-baseline]
 
-Metric: quantised GEMM TFLOPS (and weight GB/s, % of roofline) versus M.
-Default workload ``w4a16_asym_sweep``: dense W4A16 with UINT4 weights, UINT4
-zero points and bf16 scales per 128-K group, (N, K) in {(8192, 8192),
-(28672, 8192), (8192, 28672)}, M swept over 1, 4, 16, 64, 256, 1024, 4096,
-8192; A bf16 N(0, 1).  One step runs every (shape, M) GEMM once; the L2 is
-flushed (a 512 MiB memset, untimed) before each GEMM and each GEMM is timed
-with CUDA events on its stream.  Each call is captured once in a CUDA graph
+Metric: quantised GEMM TFLOPS (and weight GB/s, % of roofline) versus M,
+dense and MoE.  The default workload ``all`` runs every configuration once
+per step:
+
+  1. dense W4A16 INT4 symmetric g128, M = 16, N = K = 4096;
+  2. dense W4A16 UINT4 + zero points g128, (N, K) in {(8192, 8192),
+     (28672, 8192), (8192, 28672)}, M in {1, 4, 16, 64, 256, 1024, 4096, 8192};
+  3. MoE W4A16 MXFP4, E = 256, top-8 softmax routing, H = 7168, I = 2048,
+     T in {1, 16, 128, 1024, 4096}, grouped and indexed modes;
+  4. MoE W4A8 (MXFP4 weights x MXFP8 activations quantised on the fly),
+     Zipf(1.2) routing, T in {1, 64, 512, 4096}, both modes, fused weighted sum;
+  5. dense W4A4 NVFP4 x NVFP4 and W8A8 FP8 at N = K = 7168, M in {1, 32, 256,
+     2048, 8192} (activation quantisation inside the call), and the NVFP4 MoE
+     at T = 4096 in both modes.
+
+An MoE layer is timed as its library calls: the routing prepare, the
+gate-up GEMM and the down GEMM with the weighted top-k sum.  The L2 is
+flushed (a 512 MiB memset, untimed) before every call and each call is timed
+with CUDA events on its stream; each call is captured once in a CUDA graph
 and replayed (``--eager`` times the plain calls).  ``value`` = total flops of
-a step / summed GEMM time.  Other workloads (``--workload``):
-``w4a16_dense_m16``, ``moe_w4a16_mxfp4``, ``moe_w4a8_mxfp8``, ``moe_nvfp4``,
-``w4a4_nvfp4``, ``w8a8_fp8``.  The roofline object describes the dominant
-call: HBM-bound calls against the measured copy bandwidth, tensor-bound ones
-against the measured bf16 peak times the nominal ratio of the call's MMA kind
-(FP8 and MXFP8 x FP4 weights 2, FP4 x FP4 4); ``traffic`` is the committed ncu
-DRAM figure when the kernel sources still match it.
+a step / summed call time; ``sweep`` lists every call with its roofline
+fractions and ``per_config`` sums them per configuration.  The roofline
+object describes the call that takes the most time: HBM-bound calls against
+the measured copy bandwidth, tensor-bound ones against the measured bf16
+peak times the nominal ratio of the call's MMA kind (FP8 and MXFP8 x FP4
+weights 2, FP4 x FP4 4); ``traffic`` is the committed ncu DRAM figure when
+the kernel sources still match it.  ``--workload`` picks one configuration
+(``w4a16_dense_m16``, ``w4a16_asym_sweep``, ``moe_w4a16_mxfp4``,
+``moe_w4a8_mxfp8``, ``w4a4_nvfp4``, ``w8a8_fp8``, ``moe_nvfp4``) or the
+masked-layout MoE (``moe_masked_nvfp4``).
 
 Multi-GPU (torchrun): replicas only, every rank runs the same workload on
 its own GPU; the timed region is bracketed by a barrier and a synchronise,
 the time is the max over ranks and ``value`` counts every rank's flops.
 ``--impl reference`` times the CPU oracle (the only reference there is) on
-a bounded sample of the same workload, on rank 0 only.
+bounded samples of the same workload, on rank 0 only.
 """
 from __future__ import annotations
 
@@ -45,15 +60,6 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 METRIC = "quantized GEMM TFLOPS and weight GB/s vs M (dense+MoE), % of roofline, 1xB200"
-
-# Workload titles shared by the library arm's config and the reference arm's config.
-WORKLOAD_TITLE = {
-    "w4a16_asym_sweep": "dense W4A16 UINT4 asym g128 bf16-scale, (N,K) in {(8192,8192),(28672,8192),(8192,28672)}, "
-                        "M in {1,4,16,64,256,1024,4096,8192}",
-    "w4a16_dense_m16": "dense W4A16 INT4 sym g128, M=16, N=K=4096",
-    "moe_masked_nvfp4": "masked-layout MoE W4A4 NVFP4 x NVFP4 (activations quantised on the fly), E=256 slabs of "
-                        "256 rows, counts from a softmax top-8 routing of T=4096, H=7168, I=2048, gate-up + down",
-}
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -184,8 +190,9 @@ class Op:
     """One library call of a step, with its algorithmic cost."""
 
     def __init__(self, name, run, flops, w_bytes, io_bytes, kernels, h2d=None, d2h=None, e2e=None, kernel=None,
-                 peak_ratio=1.0):
+                 peak_ratio=1.0, config=0):
         self.name = name
+        self.config = config      # which benchmark configuration (1..5) the call belongs to
         self.kernel = kernel      # the library kernel that dominates the call
         # dense tensor peak of the call's MMA kind relative to bf16 (nominal ratios: FP8 and
         # MXFP8-with-FP4-weights 2, FP4 x FP4 4), applied to the measured bf16 peak
@@ -217,7 +224,7 @@ def desc_of(hq, w_dtype, group, scale_dtype, zero, glob, a_dtype):
     return d
 
 
-def dense_op(hq, d, name, M, N, K, packed, w_bytes, gen, a_fmt="bf16", a_bits=None):
+def dense_op(hq, d, name, M, N, K, packed, w_bytes, gen, config):
     """A dense hq_gemm over resident inputs (bf16 activations)."""
     dev = "cuda"
     A = synth.bf16_normal((M, K), gen, device=dev)
@@ -237,7 +244,7 @@ def dense_op(hq, d, name, M, N, K, packed, w_bytes, gen, a_fmt="bf16", a_bits=No
         C_h.copy_(C, non_blocking=True)
 
     return Op(name, run, 2.0 * M * N * K, w_bytes, M * K * 2 + M * N * 2, 1, M * K * 2, M * N * 2, e2e,
-              kernel=gemm_kernel_name(M))
+              kernel=gemm_kernel_name(M), config=config)
 
 
 NOMINAL_HBM_GBS = 8000.0  # the nominal B200 figure the targets are quoted against
@@ -253,7 +260,8 @@ def sweep_entry(op, t_ms, peaks):
     hb = op.bytes / s / 1e9
     t_bw = op.bytes / (peaks["hbm_gbs"] * 1e9)
     t_fl = op.flops / (peaks["bf16_tflops"] * op.peak_ratio * 1e12)
-    return {"op": op.name, "us": round(t_ms * 1e3, 2), "tflops": round(op.flops / s / 1e12, 2),
+    return {"op": op.name, "config": op.config, "us": round(t_ms * 1e3, 2),
+            "tflops": round(op.flops / s / 1e12, 2),
             "weight_gbs": round(op.w_bytes / s / 1e9, 1), "hbm_frac": round(hb / peaks["hbm_gbs"], 3),
             "hbm_frac_nominal": round(hb / NOMINAL_HBM_GBS, 3),
             "tensor_frac": round(op.flops / s / 1e12 / (peaks["bf16_tflops"] * op.peak_ratio), 3),
@@ -301,13 +309,38 @@ def packed_bytes_int4(N, K, group, zero):
     return N * K // 2 + N * G * 2 + (N * G // 2 if zero else 0)
 
 
-def workload_w4a16_asym_sweep(hq, gen_seed=0):
+CONFIG_TITLES = {
+    1: "dense W4A16 INT4 sym g128, M=16, N=K=4096",
+    2: "dense W4A16 UINT4 asym g128, (N,K) in {(8192,8192),(28672,8192),(8192,28672)}, M in {1,4,16,64,256,1024,"
+       "4096,8192}",
+    3: "MoE W4A16 MXFP4, E=256 top-8 softmax routing, H=7168, I=2048, T in {1,16,128,1024,4096}, grouped + indexed",
+    4: "MoE W4A8 MXFP4 x MXFP8 (quantised on the fly), Zipf(1.2) routing, E=256 top-8, H=7168, I=2048, "
+       "T in {1,64,512,4096}, grouped + indexed, fused weighted sum",
+    5: "dense W4A4 NVFP4 x NVFP4 and W8A8 FP8 (per-channel x per-token), N=K=7168, M in {1,32,256,2048,8192}, "
+       "activation quantisation inside the step; NVFP4 MoE at T=4096, grouped + indexed",
+}
+
+# Workload titles shared by the library arm's config and the reference arm's config.
+WORKLOAD_TITLE = {
+    "all": "all five configurations: " + "; ".join(f"({i}) {t}" for i, t in CONFIG_TITLES.items()),
+    "w4a16_asym_sweep": CONFIG_TITLES[2],
+    "w4a16_dense_m16": CONFIG_TITLES[1],
+    "moe_w4a16_mxfp4": CONFIG_TITLES[3],
+    "moe_w4a8_mxfp8": CONFIG_TITLES[4],
+    "moe_nvfp4": "MoE W4A4 NVFP4 x NVFP4 (activations quantised on the fly), E=256 top-8, H=7168, I=2048, T=4096, "
+                 "grouped + indexed",
+    "w4a4_nvfp4": "dense W4A4 NVFP4 x NVFP4, N=K=7168, M in {1,32,256,2048,8192}",
+    "w8a8_fp8": "dense W8A8 FP8 per-channel x per-token, N=K=7168, M in {1,32,256,2048,8192}",
+    "moe_masked_nvfp4": "masked-layout MoE W4A4 NVFP4 x NVFP4 (activations quantised on the fly), E=256 slabs of "
+                        "256 rows, counts from a softmax top-8 routing of T=4096, H=7168, I=2048, gate-up + down",
+}
+
+
+def ops_w4a16_asym_sweep(hq, gen):
     shapes = [(8192, 8192), (28672, 8192), (8192, 28672)]
     Ms = [1, 4, 16, 64, 256, 1024, 4096, 8192]
     d = desc_of(hq, hq.HQ_UINT4, 128, hq.HQ_BF16, 1, 0, hq.HQ_BF16)
-    gen = synth.generator(gen_seed, "cuda")
-    ops = []
-    keep = []
+    ops, keep = [], []
     for (N, K) in shapes:
         w = synth.int4_weights(1, N, K, 128, True, gen, device="cuda")
         packed = torch.empty(hq.hq_packed_weights_bytes(d, 1, N, K), dtype=torch.uint8, device="cuda")
@@ -315,57 +348,75 @@ def workload_w4a16_asym_sweep(hq, gen_seed=0):
         keep.append(packed)
         wb = packed_bytes_int4(N, K, 128, True)
         for M in Ms:
-            ops.append(dense_op(hq, d, f"N{N}_K{K}_M{M}", M, N, K, packed, wb, gen))
-    cfg = {"workload": WORKLOAD_TITLE["w4a16_asym_sweep"], "shapes": shapes, "M": Ms, "l2": "flushed before every GEMM (512 MiB memset, untimed)"}
-    return ops, cfg, keep
+            ops.append(dense_op(hq, d, f"N{N}_K{K}_M{M}", M, N, K, packed, wb, gen, 2))
+    return ops, keep
 
 
-def workload_w4a16_dense_m16(hq, gen_seed=0):
+def ops_w4a16_dense_m16(hq, gen):
     N = K = 4096
     M = 16
     d = desc_of(hq, hq.HQ_INT4, 128, hq.HQ_BF16, 0, 0, hq.HQ_BF16)
-    gen = synth.generator(gen_seed, "cuda")
     w = synth.int4_weights(1, N, K, 128, False, gen, device="cuda")
     packed = torch.empty(hq.hq_packed_weights_bytes(d, 1, N, K), dtype=torch.uint8, device="cuda")
     hq.hq_pack_weights(d, 1, N, K, w["codes"], w["scales"], None, None, packed)
-    ops = [dense_op(hq, d, "N4096_K4096_M16", M, N, K, packed, packed_bytes_int4(N, K, 128, False), gen)]
-    cfg = {"workload": WORKLOAD_TITLE["w4a16_dense_m16"], "l2": "flushed before every GEMM"}
-    return ops, cfg, [packed]
+    return [dense_op(hq, d, "cfg1_N4096_K4096_M16", M, N, K, packed, packed_bytes_int4(N, K, 128, False), gen,
+                     1)], [packed]
 
 
-def workload_shape(hq, M, N, K, gen_seed=0):
+def ops_shape(hq, M, N, K, gen):
     """One dense W4A16 UINT4-asymmetric GEMM of the given shape (profiling)."""
     d = desc_of(hq, hq.HQ_UINT4, 128, hq.HQ_BF16, 1, 0, hq.HQ_BF16)
-    gen = synth.generator(gen_seed, "cuda")
     w = synth.int4_weights(1, N, K, 128, True, gen, device="cuda")
     packed = torch.empty(hq.hq_packed_weights_bytes(d, 1, N, K), dtype=torch.uint8, device="cuda")
     hq.hq_pack_weights(d, 1, N, K, w["codes"], w["scales"], w["zeros"], None, packed)
-    ops = [dense_op(hq, d, f"N{N}_K{K}_M{M}", M, N, K, packed, packed_bytes_int4(N, K, 128, True), gen)]
-    cfg = {"workload": f"dense W4A16 UINT4 asym g128, M={M}, N={N}, K={K}", "l2": "flushed before every GEMM"}
-    return ops, cfg, [packed]
+    return [dense_op(hq, d, f"N{N}_K{K}_M{M}", M, N, K, packed, packed_bytes_int4(N, K, 128, True), gen, 2)], [packed]
 
 
-def moe_ops(hq, name, wdesc, E, topk, H, I, Ts, routing, gen, mode_names=("grouped", "indexed"), weights=None,
-            a_dtype=None):
-    """MoE gate-up (N = 2I, K = H) and down (N = H, K = I) GEMMs for every T
-    and mode; step time = permute + gate-up + down, as the pages time MoE."""
+def moe_call_kernels(hq, wdesc, a_dtype, mode, combine):
+    """Library kernel launches of one hq_moe_gemm call: on-the-fly
+    quantisation (MXFP8, per-token FP8: one kernel; NVFP4: tensor amax +
+    quantise), the grouped mode's row copy, the block-scaled MMA's scale
+    relayout or the dequantisation path's exact decode, the GEMM, and the
+    weighted combine."""
+    quant = a_dtype not in (None, hq.HQ_BF16)
+    block_scaled = (wdesc.w_dtype == hq.HQ_E2M1 and
+                    ((wdesc.w_scale_dtype == hq.HQ_E8M0 and a_dtype == hq.HQ_MXFP8) or
+                     (wdesc.w_scale_dtype == hq.HQ_UE4M3 and a_dtype == hq.HQ_NVFP4)))
+    n = 1  # the GEMM
+    if quant:
+        n += 2 if a_dtype == hq.HQ_NVFP4 else 1
+        n += 1  # scale relayout (block-scaled) or exact decode to bf16
+        if block_scaled and mode == hq.HQ_MOE_GROUPED:
+            n += 1  # row copy of the codes
+    elif mode == hq.HQ_MOE_GROUPED:
+        n += 1  # row copy
+    return n + (1 if combine else 0), block_scaled
+
+
+def ops_moe(hq, config, name, wdesc, E, topk, H, I, Ts, routing, gen, a_dtype, modes=("grouped", "indexed")):
+    """MoE calls per T: the routing prepare, then per mode the gate-up GEMM
+    (N = 2I, K = H, one activation row per token) and the down GEMM (N = H,
+    K = I, one row per routed slot) with the fused weighted top-k sum; a MoE
+    layer's time is the sum, as the pages time MoE (gate-up + down)."""
     dev = "cuda"
-    if weights is None:
-        weights = {}
-        for part, (N, K) in (("gate_up", (2 * I, H)), ("down", (H, I))):
-            if wdesc.w_dtype == hq.HQ_E2M1 and wdesc.w_scale_dtype == hq.HQ_E8M0:
-                w = synth.mxfp4_weights(E, N, K, gen, device=dev)
-                glob = None
-                bytes_per = N * K // 2 + N * K // 32
-            else:
-                w = synth.nvfp4_weights_random(E, N, K, gen, device=dev)
-                glob = w["global"]
-                bytes_per = N * K // 2 + N * K // 16
-            packed = torch.empty(hq.hq_packed_weights_bytes(wdesc, E, N, K), dtype=torch.uint8, device=dev)
-            hq.hq_pack_weights(wdesc, E, N, K, w["codes"], w["scales"], None, glob, packed)
-            del w
-            weights[part] = (packed, N, K, bytes_per)
-    ops = []
+    weights = {}
+    for part, (N, K) in (("gate_up", (2 * I, H)), ("down", (H, I))):
+        if wdesc.w_dtype == hq.HQ_E2M1 and wdesc.w_scale_dtype == hq.HQ_E8M0:
+            w = synth.mxfp4_weights(E, N, K, gen, device=dev)
+            glob = None
+            bytes_per = N * K // 2 + N * K // 32
+        else:
+            w = synth.nvfp4_weights_random(E, N, K, gen, device=dev)
+            glob = w["global"]
+            bytes_per = N * K // 2 + N * K // 16
+        packed = torch.empty(hq.hq_packed_weights_bytes(wdesc, E, N, K), dtype=torch.uint8, device=dev)
+        hq.hq_pack_weights(wdesc, E, N, K, w["codes"], w["scales"], None, glob, packed)
+        del w
+        weights[part] = (packed, N, K, bytes_per)
+    pg, Ng, Kg, bg = weights["gate_up"]
+    pd, Nd, Kd, bd = weights["down"]
+    ratio = 1.0
+    ops, keep = [], [weights]
     for T in Ts:
         ids, wts = routing(T, gen)
         touched = int(torch.unique(ids).numel())
@@ -376,97 +427,87 @@ def moe_ops(hq, name, wdesc, E, topk, H, I, Ts, routing, gen, mode_names=("group
         inv = torch.empty(T * topk, dtype=torch.int32, device=dev)
         ids_h = ids.cpu().pin_memory()
         x_gate_h = x_gate.cpu().pin_memory()
-        out_h = torch.empty(T, H, dtype=torch.bfloat16).pin_memory()
-        for mode_name in mode_names:
+        x_down_h = x_down.cpu().pin_memory()
+        keep += [ids, wts, x_gate, x_down, off, perm, inv, ids_h, x_gate_h, x_down_h]
+
+        def run_perm(T=T, ids=ids, off=off, perm=perm, inv=inv):
+            hq.hq_moe_permute(T, topk, E, ids, off, perm, inv)
+
+        def e2e_perm(run_perm=run_perm, ids=ids, ids_h=ids_h):
+            ids.copy_(ids_h, non_blocking=True)
+            run_perm()
+
+        ops.append(Op(f"{name}_T{T}_routing", run_perm, 0.0, 0, T * topk * 4 * 3 + (E + 1) * 4, 1, T * topk * 4, 0,
+                      e2e_perm, kernel="moe_permute_kernel", config=config))
+        for mode_name in modes:
             mode = hq.HQ_MOE_GROUPED if mode_name == "grouped" else hq.HQ_MOE_INDEXED
-            pg, Ng, Kg, bg = weights["gate_up"]
-            pd, Nd, Kd, bd = weights["down"]
             wsg = hq.hq_moe_workspace_bytes(mode, wdesc, T, topk, E, Ng, Kg, 0, 0)
             wsd = hq.hq_moe_workspace_bytes(mode, wdesc, T, topk, E, Nd, Kd, 1, 1)
             ws = torch.zeros(max(wsg, wsd), dtype=torch.uint8, device=dev)
             y = torch.empty(T * topk, Ng, dtype=torch.bfloat16, device=dev)
             out = torch.empty(T, Nd, dtype=torch.bfloat16, device=dev)
-            ids_e = torch.empty_like(ids)
-            x_e = torch.empty_like(x_gate)
+            out_h = torch.empty(T, Nd, dtype=torch.bfloat16).pin_memory()
+            keep += [ws, y, out, out_h]
 
-            def run(mode=mode, pg=pg, pd=pd, Ng=Ng, Kg=Kg, Nd=Nd, Kd=Kd, ws=ws, y=y, out=out, ids=ids, wts=wts,
-                    x_gate=x_gate, x_down=x_down, off=off, perm=perm, inv=inv, T=T, wsg=wsg, wsd=wsd):
-                hq.hq_moe_permute(T, topk, E, ids, off, perm, inv)
+            def run_gate(mode=mode, ws=ws, y=y, x_gate=x_gate, wts=wts, off=off, perm=perm, T=T, wsg=wsg):
                 hq.hq_moe_gemm(mode, wdesc, T, topk, E, Ng, Kg, pg, x_gate, None, None, 0, None, wts, off, perm, 0,
                                1.0, y, ws, wsg)
+
+            def e2e_gate(run_gate=run_gate, x_gate=x_gate, x_gate_h=x_gate_h):
+                x_gate.copy_(x_gate_h, non_blocking=True)
+                run_gate()
+
+            def run_down(mode=mode, ws=ws, out=out, x_down=x_down, wts=wts, off=off, perm=perm, T=T, wsd=wsd):
                 hq.hq_moe_gemm(mode, wdesc, T, topk, E, Nd, Kd, pd, x_down, None, None, 1, None, wts, off, perm, 1,
                                1.0, out, ws, wsd)
 
-            def e2e(run=run, ids=ids, ids_e=ids_e, ids_h=ids_h, x_gate=x_gate, x_e=x_e, x_gate_h=x_gate_h,
-                    out=out, out_h=out_h):
-                ids.copy_(ids_h, non_blocking=True)
-                x_gate.copy_(x_gate_h, non_blocking=True)
-                run()
+            def e2e_down(run_down=run_down, x_down=x_down, x_down_h=x_down_h, out=out, out_h=out_h):
+                x_down.copy_(x_down_h, non_blocking=True)
+                run_down()
                 out_h.copy_(out, non_blocking=True)
 
-            flops = 2.0 * T * topk * (Ng * Kg + Nd * Kd)
-            wbytes = touched * (bg + bd)
-            io = T * Kg * 2 + T * topk * Ng * 2 + T * topk * Kd * 2 + T * Nd * 2
-            quant = a_dtype is not None and a_dtype != hq.HQ_BF16
-            block_scaled = (wdesc.w_dtype == hq.HQ_E2M1 and
-                            ((wdesc.w_scale_dtype == hq.HQ_E8M0 and a_dtype == hq.HQ_MXFP8) or
-                             (wdesc.w_scale_dtype == hq.HQ_UE4M3 and a_dtype == hq.HQ_NVFP4)))
-            # kernels: permute; per GEMM: quant + gather codes + scale relayout + GEMM (block-scaled MMA),
-            # quant + decode + GEMM, or gather + GEMM (bf16); combine
-            per_gemm = 4 if block_scaled else (3 if quant else 2)
-            kernels = 1 + per_gemm * 2 + 1
-            ratio = 1.0
-            if block_scaled:
+            kg, bs = moe_call_kernels(hq, wdesc, a_dtype, mode, 0)
+            kd, _ = moe_call_kernels(hq, wdesc, a_dtype, mode, 1)
+            if bs:
                 ratio = 2.0 if wdesc.w_scale_dtype == hq.HQ_E8M0 else 4.0
-            ops.append(Op(f"{name}_T{T}_{mode_name}", run, flops, wbytes, io, kernels,
-                          T * topk * 4 + T * Kg * 2, T * Nd * 2, e2e,
-                          kernel="bs_gemm_kernel" if block_scaled else "MoE GEMM kernels", peak_ratio=ratio))
-    return ops, weights
+            kern = "bs_gemm_kernel" if bs else ("dec_gemm_kernel / tc_gemm_kernel")
+            ops.append(Op(f"{name}_T{T}_{mode_name}_gate_up", run_gate, 2.0 * T * topk * Ng * Kg, touched * bg,
+                          T * Kg * 2 + T * topk * Ng * 2, kg, T * Kg * 2, 0, e2e_gate, kernel=kern, peak_ratio=ratio,
+                          config=config))
+            ops.append(Op(f"{name}_T{T}_{mode_name}_down", run_down, 2.0 * T * topk * Nd * Kd, touched * bd,
+                          T * topk * Kd * 2 + T * Nd * 2, kd, T * topk * Kd * 2, T * Nd * 2, e2e_down, kernel=kern,
+                          peak_ratio=ratio, config=config))
+    return ops, keep
 
 
-def workload_moe_w4a16_mxfp4(hq, gen_seed=0):
-    E, topk, H, I = 256, 8, 7168, 2048
-    gen = synth.generator(gen_seed, "cuda")
+E_MOE, TOPK, H_MOE, I_MOE = 256, 8, 7168, 2048
+
+
+def ops_moe_w4a16_mxfp4(hq, gen, Ts=(1, 16, 128, 1024, 4096)):
     d = desc_of(hq, hq.HQ_E2M1, 32, hq.HQ_E8M0, 0, 0, hq.HQ_BF16)
-    routing = lambda T, g: synth.routing_softmax_topk(T, E, topk, g, device="cuda")
-    ops, w = moe_ops(hq, "moe_w4a16_mxfp4", d, E, topk, H, I, [1, 16, 128, 1024, 4096], routing, gen)
-    cfg = {"workload": "MoE W4A16 MXFP4: E=256 top-8 softmax routing, H=7168, I=2048, T in {1,16,128,1024,4096}, "
-                       "grouped + indexed; step = permute + gate-up + down (+ fused weighted sum)",
-           "l2": "flushed before every call; weights ~6 GB"}
-    return ops, cfg, [w]
+    routing = lambda T, g: synth.routing_softmax_topk(T, E_MOE, TOPK, g, device="cuda")
+    return ops_moe(hq, 3, "cfg3_moe_w4a16", d, E_MOE, TOPK, H_MOE, I_MOE, list(Ts), routing, gen, hq.HQ_BF16)
 
 
-def workload_moe_w4a8_mxfp8(hq, gen_seed=0):
-    E, topk, H, I = 256, 8, 7168, 2048
-    gen = synth.generator(gen_seed, "cuda")
+def ops_moe_w4a8_mxfp8(hq, gen, Ts=(1, 64, 512, 4096)):
     d = desc_of(hq, hq.HQ_E2M1, 32, hq.HQ_E8M0, 0, 0, hq.HQ_MXFP8)
-    routing = lambda T, g: synth.routing_zipf(T, E, topk, 1.2, g, device="cuda")
-    ops, w = moe_ops(hq, "moe_w4a8_mxfp8", d, E, topk, H, I, [1, 64, 512, 4096], routing, gen, a_dtype=hq.HQ_MXFP8)
-    cfg = {"workload": "MoE W4A8: MXFP4 weights x MXFP8 activations quantised on the fly, Zipf(1.2) routing, E=256 "
-                       "top-8, H=7168, I=2048, T in {1,64,512,4096}, grouped + indexed, fused weighted sum",
-           "l2": "flushed before every call"}
-    return ops, cfg, [w]
+    routing = lambda T, g: synth.routing_zipf(T, E_MOE, TOPK, 1.2, g, device="cuda")
+    return ops_moe(hq, 4, "cfg4_moe_w4a8", d, E_MOE, TOPK, H_MOE, I_MOE, list(Ts), routing, gen, hq.HQ_MXFP8)
 
 
-def workload_moe_nvfp4(hq, gen_seed=0):
-    E, topk, H, I = 256, 8, 7168, 2048
-    gen = synth.generator(gen_seed, "cuda")
+def ops_moe_nvfp4(hq, gen, Ts=(4096,)):
     d = desc_of(hq, hq.HQ_E2M1, 16, hq.HQ_UE4M3, 0, 1, hq.HQ_NVFP4)
-    routing = lambda T, g: synth.routing_softmax_topk(T, E, topk, g, device="cuda")
-    ops, w = moe_ops(hq, "moe_nvfp4", d, E, topk, H, I, [4096], routing, gen, a_dtype=hq.HQ_NVFP4)
-    cfg = {"workload": "MoE W4A4 NVFP4 x NVFP4 (activations quantised on the fly), E=256 top-8, H=7168, I=2048, "
-                       "T=4096, grouped + indexed", "l2": "flushed before every call"}
-    return ops, cfg, [w]
+    routing = lambda T, g: synth.routing_softmax_topk(T, E_MOE, TOPK, g, device="cuda")
+    return ops_moe(hq, 5, "cfg5_moe_nvfp4", d, E_MOE, TOPK, H_MOE, I_MOE, list(Ts), routing, gen, hq.HQ_NVFP4)
 
 
-def workload_moe_masked_nvfp4(hq, gen_seed=0):
+def ops_moe_masked_nvfp4(hq, gen):
     """Masked-layout MoE (expert slabs with per-expert valid counts), NVFP4 x
     NVFP4, config-5 MoE shapes: the counts come from a softmax top-8 routing
     of T = 4096 tokens over E = 256 experts, slabs of 256 rows, expected_m =
     the mean count.  Step = gate-up (N = 2I, K = H) + down (N = H, K = I)."""
     dev = "cuda"
-    E, topk, H, I, T, slab = 256, 8, 7168, 2048, 4096, 256
-    gen = synth.generator(gen_seed, dev)
+    E, topk, H, I, T, slab = E_MOE, TOPK, H_MOE, I_MOE, 4096, 256
     d = desc_of(hq, hq.HQ_E2M1, 16, hq.HQ_UE4M3, 0, 1, hq.HQ_NVFP4)
     ids, _ = synth.routing_softmax_topk(T, E, topk, gen, device=dev)
     counts = torch.bincount(ids.flatten().long(), minlength=E).clamp(max=slab).to(torch.int32)
@@ -508,16 +549,15 @@ def workload_moe_masked_nvfp4(hq, gen_seed=0):
     io = rows * (Kg // 2 + Ng * 2 + Kd // 2 + Nd * 2)
     # per GEMM: routing prepare, amax + quantise, gather codes, scale relayout, GEMM
     op = Op(f"moe_masked_nvfp4_T{T}_slab{slab}", run, flops, touched * (bg + bd), io, 2 * 6,
-            E * slab * Kg * 2 + E * 4, E * slab * Nd * 2, e2e, kernel="bs_gemm_kernel", peak_ratio=4.0)
-    cfg = {"workload": WORKLOAD_TITLE["moe_masked_nvfp4"], "l2": "flushed before every call"}
-    return [op], cfg, [parts, x_gate, x_down, y, out, ws, counts]
+            E * slab * Kg * 2 + E * 4, E * slab * Nd * 2, e2e, kernel="bs_gemm_kernel", peak_ratio=4.0, config=5)
+    return [op], [parts, x_gate, x_down, y, out, ws, counts]
 
 
-def workload_dense_quantised(hq, fmt, gen_seed=0, N=7168, K=7168, Ms=(1, 32, 256, 2048, 8192)):
+def ops_dense_quantised(hq, fmt, gen, N=7168, K=7168, Ms=(1, 32, 256, 2048, 8192)):
     """Config 5 dense: N = K = 7168, both operands N(0,1) quantised by the
-    library's own quantiser (weights per output row), M swept."""
+    library's own quantiser (weights per output row), M swept; each call
+    quantises its activations and multiplies."""
     dev = "cuda"
-    gen = synth.generator(gen_seed, dev)
     if fmt == "nvfp4":
         d = desc_of(hq, hq.HQ_E2M1, 16, hq.HQ_UE4M3, 0, 1, hq.HQ_NVFP4)
         wbytes = N * K // 2 + N * K // 16
@@ -543,7 +583,7 @@ def workload_dense_quantised(hq, fmt, gen_seed=0, N=7168, K=7168, Ms=(1, 32, 256
     packed = torch.empty(hq.hq_packed_weights_bytes(d, 1, N, K), dtype=torch.uint8, device=dev)
     hq.hq_pack_weights(d, 1, N, K, wc, wsc, None, wg if fmt == "nvfp4" else None, packed)
     ops = []
-    keep = [packed]
+    keep = [packed, wg]
     for M in Ms:
         x = synth.bf16_normal((M, K), gen, device=dev)
         c, s, g, wq2 = quant(x)
@@ -552,6 +592,7 @@ def workload_dense_quantised(hq, fmt, gen_seed=0, N=7168, K=7168, Ms=(1, 32, 256
         ws = torch.zeros(max(wsb, 256), dtype=torch.uint8, device=dev)
         x_h = x.cpu().pin_memory()
         C_h = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
+        keep += [x, c, s, g, wq2, C, ws, x_h, C_h]
 
         def run(M=M, x=x, c=c, s=s, g=g, wq2=wq2, C=C, ws=ws, wsb=wsb):
             hq.hq_quant_act(d, M, K, x, c, s, g, None, wq2, 64)
@@ -563,50 +604,62 @@ def workload_dense_quantised(hq, fmt, gen_seed=0, N=7168, K=7168, Ms=(1, 32, 256
             C_h.copy_(C, non_blocking=True)
 
         kern = (2 if fmt == "nvfp4" else 1) + (1 if fmt == "fp8" else 2)
-        ops.append(Op(f"{fmt}_N{N}_K{K}_M{M}", run, 2.0 * M * N * K, wbytes, M * K * 2 + M * N * 2, kern,
-                      M * K * 2, M * N * 2, e2e,
-                      kernel="bs_gemm_kernel",
-                      peak_ratio=4.0 if fmt == "nvfp4" else 2.0))
-    cfg = {"workload": f"dense {'W4A4 NVFP4 x NVFP4' if fmt == 'nvfp4' else 'W8A8 FP8 per-channel x per-token'}, "
-                       f"N={N}, K={K}, M in {{{','.join(str(m) for m in Ms)}}}, activation quantisation inside the step",
-           "l2": "flushed before every call"}
-    return ops, cfg, keep
+        ops.append(Op(f"cfg5_{fmt}_N{N}_K{K}_M{M}", run, 2.0 * M * N * K, wbytes, M * K * 2 + M * N * 2, kern,
+                      M * K * 2, M * N * 2, e2e, kernel="bs_gemm_kernel",
+                      peak_ratio=4.0 if fmt == "nvfp4" else 2.0, config=5))
+    return ops, keep
+
+
+def _workload(builders, title):
+    def build(hq, gen_seed=0):
+        gen = synth.generator(gen_seed, "cuda")
+        ops, keep = [], []
+        for b in builders:
+            o, k = b(hq, gen)
+            ops += o
+            keep += k
+        return ops, {"workload": title, "l2": "flushed before every call (512 MiB memset, untimed)"}, keep
+    return build
 
 
 WORKLOADS = {
-    "w4a16_asym_sweep": workload_w4a16_asym_sweep,
-    "w4a16_dense_m16": workload_w4a16_dense_m16,
-    "moe_w4a16_mxfp4": workload_moe_w4a16_mxfp4,
-    "moe_w4a8_mxfp8": workload_moe_w4a8_mxfp8,
-    "moe_nvfp4": workload_moe_nvfp4,
-    "moe_masked_nvfp4": workload_moe_masked_nvfp4,
-    "w4a4_nvfp4": lambda hq: workload_dense_quantised(hq, "nvfp4"),
-    "w8a8_fp8": lambda hq: workload_dense_quantised(hq, "fp8"),
+    "all": _workload([ops_w4a16_dense_m16, ops_w4a16_asym_sweep, ops_moe_w4a16_mxfp4, ops_moe_w4a8_mxfp8,
+                      lambda hq, g: ops_dense_quantised(hq, "nvfp4", g), lambda hq, g: ops_dense_quantised(hq, "fp8", g),
+                      ops_moe_nvfp4], WORKLOAD_TITLE["all"]),
+    "w4a16_asym_sweep": _workload([ops_w4a16_asym_sweep], WORKLOAD_TITLE["w4a16_asym_sweep"]),
+    "w4a16_dense_m16": _workload([ops_w4a16_dense_m16], WORKLOAD_TITLE["w4a16_dense_m16"]),
+    "moe_w4a16_mxfp4": _workload([ops_moe_w4a16_mxfp4], WORKLOAD_TITLE["moe_w4a16_mxfp4"]),
+    "moe_w4a8_mxfp8": _workload([ops_moe_w4a8_mxfp8], WORKLOAD_TITLE["moe_w4a8_mxfp8"]),
+    "moe_nvfp4": _workload([ops_moe_nvfp4], WORKLOAD_TITLE["moe_nvfp4"]),
+    "moe_masked_nvfp4": _workload([ops_moe_masked_nvfp4], WORKLOAD_TITLE["moe_masked_nvfp4"]),
+    "w4a4_nvfp4": _workload([lambda hq, g: ops_dense_quantised(hq, "nvfp4", g)], WORKLOAD_TITLE["w4a4_nvfp4"]),
+    "w8a8_fp8": _workload([lambda hq, g: ops_dense_quantised(hq, "fp8", g)], WORKLOAD_TITLE["w8a8_fp8"]),
+}
+
+# configurations each workload covers (for the CPU samples)
+WORKLOAD_CONFIGS = {"all": (1, 2, 3, 4, 5), "w4a16_asym_sweep": (2,), "w4a16_dense_m16": (1,),
+                    "moe_w4a16_mxfp4": (3,), "moe_w4a8_mxfp8": (4,), "moe_nvfp4": (5,), "moe_masked_nvfp4": (5,),
+                    "w4a4_nvfp4": (5,), "w8a8_fp8": (5,)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline (bounded samples)
+# ---------------------------------------------------------------------------
+# One sample per configuration: (weight kind, activation format, N, K, M):
+# decode one weight matrix of the configuration's format and shape, quantise
+# and decode M activation rows where the configuration quantises them, and
+# multiply in fp64 (the MoE samples are one expert's gate-up matrix).
+CPU_SAMPLES = {
+    1: [("int4", "bf16", 4096, 4096, 16)],
+    2: [("uint4", "bf16", 8192, 8192, 16)],
+    3: [("mxfp4", "bf16", 4096, 7168, 16)],
+    4: [("mxfp4", "mxfp8", 4096, 7168, 64)],
+    5: [("nvfp4", "nvfp4", 7168, 7168, 32), ("fp8", "fp8", 7168, 7168, 32)],
 }
 
 
-# ---------------------------------------------------------------------------
-# CPU oracle baseline (bounded sample)
-# ---------------------------------------------------------------------------
-def cpu_baseline(workload: str, budget_s: float = 15.0):
-    """Times the oracle as it stands on a bounded sample of the workload: the
-    workload's own weight and activation formats at one of its shapes, i.e.
-    decode one (N, K) weight matrix, quantise and decode M activation rows
-    when the workload quantises them, and multiply in fp64."""
-    import oracle as O
-    gen = synth.generator(0)
-    # (weight kind, activation format, N, K, M)
-    samples = {
-        "w4a16_dense_m16": ("int4", "bf16", 4096, 4096, 16),
-        "w4a16_asym_sweep": ("uint4", "bf16", 8192, 8192, 16),
-        "moe_w4a16_mxfp4": ("mxfp4", "bf16", 4096, 7168, 16),
-        "moe_w4a8_mxfp8": ("mxfp4", "mxfp8", 4096, 7168, 64),
-        "moe_nvfp4": ("nvfp4", "nvfp4", 4096, 7168, 128),
-        "moe_masked_nvfp4": ("nvfp4", "nvfp4", 4096, 7168, 128),
-        "w4a4_nvfp4": ("nvfp4", "nvfp4", 7168, 7168, 32),
-        "w8a8_fp8": ("fp8", "fp8", 7168, 7168, 32),
-    }
-    wk, ak, N, K, M = samples.get(workload, samples["w4a16_asym_sweep"])
+def _cpu_sample(O, wk, ak, N, K, M, budget_s, gen):
+    """Times the oracle on one sample until ``budget_s``; returns (flops, s, n)."""
     if wk in ("int4", "uint4"):
         w = synth.int4_weights(1, N, K, 128, wk == "uint4", gen)
         desc = O.Desc(wk, 128, "bf16", w_zero=(wk == "uint4"))
@@ -625,11 +678,9 @@ def cpu_baseline(workload: str, budget_s: float = 15.0):
         w = synth.fp8_weights_random(1, N, K, gen)
         desc = O.Desc("e4m3", 0, "fp32")
         args = (synth.to_np_bits(w["codes"][0]), synth.to_np_bits(w["scales"][0]), None)
-    x = synth.bf16_normal((M, K), gen)
-    xb = synth.to_np_bits(x)
-    flops = 0.0
+    xb = synth.to_np_bits(synth.bf16_normal((M, K), gen))
+    flops, n = 0.0, 0
     t0 = time.perf_counter()
-    n = 0
     while True:
         if ak == "bf16":
             A, row = O.decode_act("bf16", M, K, xb)
@@ -648,12 +699,45 @@ def cpu_baseline(workload: str, budget_s: float = 15.0):
         n += 1
         if time.perf_counter() - t0 > budget_s or n >= 50:
             break
-    dt = time.perf_counter() - t0
+    return flops, time.perf_counter() - t0, n
+
+
+def cpu_baseline(workload: str, budget_s: float = 15.0):
+    """Times the oracle as it stands on bounded samples of the workload, one
+    per configuration it covers (all host threads numpy's BLAS uses), plus
+    the first sample again on one thread.  ``value`` = sampled flops / time."""
+    import oracle as O
+    gen = synth.generator(0)
+    cfgs = WORKLOAD_CONFIGS.get(workload, (2,))
+    samples = [(c, s) for c in cfgs for s in CPU_SAMPLES[c]]
+    per = max(1.0, budget_s / len(samples))
+    tot_f = tot_s = 0.0
+    per_cfg = {}
+    descr = []
+    for c, (wk, ak, N, K, M) in samples:
+        f, s, n = _cpu_sample(O, wk, ak, N, K, M, per, gen)
+        tot_f += f
+        tot_s += s
+        e = per_cfg.setdefault(str(c), {"flops": 0.0, "seconds": 0.0})
+        e["flops"] += f
+        e["seconds"] += s
+        act = "" if ak == "bf16" else f" + {ak} quantise/decode of A"
+        descr.append(f"cfg{c}: {n} x (decode {wk} W[{N},{K}]{act} + fp64 GEMM M={M})")
+    for e in per_cfg.values():
+        e["tflops"] = e["flops"] / e["seconds"] / 1e12
+    one = None
+    try:
+        from threadpoolctl import threadpool_limits
+        c, (wk, ak, N, K, M) = samples[0]
+        with threadpool_limits(limits=1):
+            f, s, n = _cpu_sample(O, wk, ak, N, K, M, min(per, 5.0), gen)
+        one = {"tflops": f / s / 1e12, "cores": 1, "sample": f"cfg{c}: {n} x decode {wk} W[{N},{K}] + GEMM M={M}"}
+    except Exception as exc:  # threadpoolctl unavailable: no 1-thread figure
+        one = {"unavailable": type(exc).__name__}
     cores = len(os.sched_getaffinity(0))
-    act = "" if ak == "bf16" else f" + {ak} quantise/decode of A"
-    return {"value": flops / dt / 1e12, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
-            "sample": f"{n} x (decode {wk} W[{N},{K}]{act} + fp64 GEMM M={M}), {dt:.1f} s; numpy BLAS threads",
-            "seconds": dt}
+    return {"value": tot_f / tot_s / 1e12, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
+            "sample": "; ".join(descr) + f"; {tot_s:.1f} s on numpy BLAS threads", "seconds": tot_s,
+            "per_config": per_cfg, "one_core": one}
 
 
 # ---------------------------------------------------------------------------
@@ -707,9 +791,10 @@ def run_reference(args, ws, rank):
             "ms_per_step": statistics.median([s["seconds"] for s in steps]) * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": WORKLOAD_TITLE.get(args.workload, args.workload), "sample": cb["sample"],
-                       "note": "CPU fp64 oracle on the host cores, a bounded sample of the workload"},
+                       "note": "CPU fp64 oracle on the host cores, bounded samples of the workload"},
             "cpu_baseline": {"value": v, "unit": "TFLOPS", "cores": cb["cores"], "kind": "oracle",
-                             "sample": cb["sample"]},
+                             "sample": cb["sample"], "per_config": cb.get("per_config"),
+                             "one_core": cb.get("one_core")},
             "e2e": {"value": v, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -721,7 +806,7 @@ def main():
     ap.add_argument("--steps", type=int, default=3)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="hq", choices=["hq", "reference"])
-    ap.add_argument("--workload", default="w4a16_asym_sweep", choices=list(WORKLOADS))
+    ap.add_argument("--workload", default="all", choices=list(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time plain calls instead of replayed CUDA graphs")
     ap.add_argument("--shape", default=None, help="M,N,K: one dense GEMM instead of a workload")
@@ -736,10 +821,14 @@ def main():
     peaks = load_peaks()
     if args.shape:
         M, N, K = (int(x) for x in args.shape.split(","))
+        gen = synth.generator(0, "cuda")
         if args.shape_fmt == "uint4":
-            ops, cfg, keep = workload_shape(hq, M, N, K)
+            ops, keep = ops_shape(hq, M, N, K, gen)
+            cfg = {"workload": f"dense W4A16 UINT4 asym g128, M={M}, N={N}, K={K}"}
         else:
-            ops, cfg, keep = workload_dense_quantised(hq, args.shape_fmt, N=N, K=K, Ms=(M,))
+            ops, keep = ops_dense_quantised(hq, args.shape_fmt, gen, N=N, K=K, Ms=(M,))
+            cfg = {"workload": f"dense {args.shape_fmt} x {args.shape_fmt}, M={M}, N={N}, K={K}"}
+        cfg["l2"] = "flushed before every call"
     else:
         ops, cfg, keep = WORKLOADS[args.workload](hq)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
@@ -833,6 +922,22 @@ def main():
         else "")
 
     sweep = [sweep_entry(op, t, peaks) for op, t in zip(ops, per_op)]
+    per_config = {}
+    for op, t, e in zip(ops, per_op, sweep):
+        pc = per_config.setdefault(str(op.config), {"title": CONFIG_TITLES.get(op.config, ""), "calls": 0,
+                                                    "ms": 0.0, "flops": 0.0, "fracs": []})
+        pc["calls"] += 1
+        pc["ms"] += t
+        pc["flops"] += op.flops
+        if op.flops > 0:
+            pc["fracs"].append(e["roofline_frac"])
+    for pc in per_config.values():
+        pc["tflops"] = round(pc["flops"] / (pc["ms"] / 1e3) / 1e12, 2) if pc["ms"] > 0 else 0.0
+        pc["ms"] = round(pc["ms"], 4)
+        fr = pc.pop("fracs")
+        pc["roofline_frac_min"] = min(fr) if fr else None
+        pc["roofline_frac_max"] = max(fr) if fr else None
+        del pc["flops"]
     line = {
         "metric": METRIC,
         "value": value, "unit": "TFLOPS", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
@@ -841,7 +946,7 @@ def main():
         "e2e": {"value": flops_step * ws / (e2e_ms / 1e3) / 1e12, "unit": "TFLOPS",
                 "h2d_bytes_per_step": sum(op.h2d for op in ops), "d2h_bytes_per_step": sum(op.d2h for op in ops)},
         "gpu_launches": sum(op.kernels for op in ops) * args.steps,
-        "roofline": roof, "clocks": clk, "sweep": sweep,
+        "roofline": roof, "clocks": clk, "per_config": per_config, "sweep": sweep,
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.workload)

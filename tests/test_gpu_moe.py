@@ -7,7 +7,7 @@ import torch
 
 import oracle as O
 import synth
-from hqtest import assert_close, cdesc, gpu_pack, make_weights, np_bits, oracle_decoder, oracle_quant
+from hqtest import assert_close, cdesc, gpu_pack, gpu_quant, make_weights, np_bits, oracle_decoder, oracle_quant
 
 pytestmark = pytest.mark.gpu
 
