@@ -318,11 +318,14 @@ CONFIG_TITLES = {
        "T in {1,64,512,4096}, grouped + indexed, fused weighted sum",
     5: "dense W4A4 NVFP4 x NVFP4 and W8A8 FP8 (per-channel x per-token), N=K=7168, M in {1,32,256,2048,8192}, "
        "activation quantisation inside the step; NVFP4 MoE at T=4096, grouped + indexed",
+    "mxint4": "MoE W4A16 MXINT4 (INT4 elements, E8M0 per 32) at the config-3 shapes and routing, T in {16, 4096}, "
+              "grouped + indexed",
 }
 
 # Workload titles shared by the library arm's config and the reference arm's config.
 WORKLOAD_TITLE = {
-    "all": "all five configurations: " + "; ".join(f"({i}) {t}" for i, t in CONFIG_TITLES.items()),
+    "all": "all five configurations and the next-row formats: " +
+           "; ".join(f"({i}) {t}" for i, t in CONFIG_TITLES.items()),
     "w4a16_asym_sweep": CONFIG_TITLES[2],
     "w4a16_dense_m16": CONFIG_TITLES[1],
     "moe_w4a16_mxfp4": CONFIG_TITLES[3],
@@ -331,6 +334,8 @@ WORKLOAD_TITLE = {
                  "grouped + indexed",
     "w4a4_nvfp4": "dense W4A4 NVFP4 x NVFP4, N=K=7168, M in {1,32,256,2048,8192}",
     "w8a8_fp8": "dense W8A8 FP8 per-channel x per-token, N=K=7168, M in {1,32,256,2048,8192}",
+    "moe_w4a16_mxint4": "MoE W4A16 MXINT4 (INT4 elements, E8M0 per 32), config-3 shapes and routing, T in "
+                        "{16, 4096}, grouped + indexed",
     "moe_masked_nvfp4": "masked-layout MoE W4A4 NVFP4 x NVFP4 (activations quantised on the fly), E=256 slabs of "
                         "256 rows, counts from a softmax top-8 routing of T=4096, H=7168, I=2048, gate-up + down",
 }
@@ -403,6 +408,10 @@ def ops_moe(hq, config, name, wdesc, E, topk, H, I, Ts, routing, gen, a_dtype, m
     for part, (N, K) in (("gate_up", (2 * I, H)), ("down", (H, I))):
         if wdesc.w_dtype == hq.HQ_E2M1 and wdesc.w_scale_dtype == hq.HQ_E8M0:
             w = synth.mxfp4_weights(E, N, K, gen, device=dev)
+            glob = None
+            bytes_per = N * K // 2 + N * K // 32
+        elif wdesc.w_dtype == hq.HQ_INT4 and wdesc.w_scale_dtype == hq.HQ_E8M0:
+            w = synth.mxint4_weights(E, N, K, gen, device=dev)
             glob = None
             bytes_per = N * K // 2 + N * K // 32
         else:
@@ -487,6 +496,15 @@ def ops_moe_w4a16_mxfp4(hq, gen, Ts=(1, 16, 128, 1024, 4096)):
     d = desc_of(hq, hq.HQ_E2M1, 32, hq.HQ_E8M0, 0, 0, hq.HQ_BF16)
     routing = lambda T, g: synth.routing_softmax_topk(T, E_MOE, TOPK, g, device="cuda")
     return ops_moe(hq, 3, "cfg3_moe_w4a16", d, E_MOE, TOPK, H_MOE, I_MOE, list(Ts), routing, gen, hq.HQ_BF16)
+
+
+def ops_moe_w4a16_mxint4(hq, gen, Ts=(16, 4096)):
+    """MoE W4A16 with MXINT4 weights (INT4 elements, E8M0 per 32) at the
+    config-3 shapes and routing."""
+    d = desc_of(hq, hq.HQ_INT4, 32, hq.HQ_E8M0, 0, 0, hq.HQ_BF16)
+    routing = lambda T, g: synth.routing_softmax_topk(T, E_MOE, TOPK, g, device="cuda")
+    return ops_moe(hq, "mxint4", "moe_w4a16_mxint4", d, E_MOE, TOPK, H_MOE, I_MOE, list(Ts), routing, gen,
+                   hq.HQ_BF16)
 
 
 def ops_moe_w4a8_mxfp8(hq, gen, Ts=(1, 64, 512, 4096)):
@@ -625,7 +643,8 @@ def _workload(builders, title):
 WORKLOADS = {
     "all": _workload([ops_w4a16_dense_m16, ops_w4a16_asym_sweep, ops_moe_w4a16_mxfp4, ops_moe_w4a8_mxfp8,
                       lambda hq, g: ops_dense_quantised(hq, "nvfp4", g), lambda hq, g: ops_dense_quantised(hq, "fp8", g),
-                      ops_moe_nvfp4], WORKLOAD_TITLE["all"]),
+                      ops_moe_nvfp4, ops_moe_w4a16_mxint4], WORKLOAD_TITLE["all"]),
+    "moe_w4a16_mxint4": _workload([ops_moe_w4a16_mxint4], WORKLOAD_TITLE["moe_w4a16_mxint4"]),
     "w4a16_asym_sweep": _workload([ops_w4a16_asym_sweep], WORKLOAD_TITLE["w4a16_asym_sweep"]),
     "w4a16_dense_m16": _workload([ops_w4a16_dense_m16], WORKLOAD_TITLE["w4a16_dense_m16"]),
     "moe_w4a16_mxfp4": _workload([ops_moe_w4a16_mxfp4], WORKLOAD_TITLE["moe_w4a16_mxfp4"]),
@@ -637,7 +656,7 @@ WORKLOADS = {
 }
 
 # configurations each workload covers (for the CPU samples)
-WORKLOAD_CONFIGS = {"all": (1, 2, 3, 4, 5), "w4a16_asym_sweep": (2,), "w4a16_dense_m16": (1,),
+WORKLOAD_CONFIGS = {"all": (1, 2, 3, 4, 5), "moe_w4a16_mxint4": (3,), "w4a16_asym_sweep": (2,), "w4a16_dense_m16": (1,),
                     "moe_w4a16_mxfp4": (3,), "moe_w4a8_mxfp8": (4,), "moe_nvfp4": (5,), "moe_masked_nvfp4": (5,),
                     "w4a4_nvfp4": (5,), "w8a8_fp8": (5,)}
 

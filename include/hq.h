@@ -34,10 +34,11 @@
  *                         the group axis (G = K / w_group, or 1 per channel).
  *       INT4 scales       bf16  [E, N, G].
  *       E2M1 codes        uint8 [E, N, K/2], low nibble = even k.
- *       E8M0 scales       uint8 [E, N, K/32] (MXFP4).
+ *       E8M0 scales       uint8 [E, N, K/32] (MXFP4, MXINT4).
  *       UE4M3 scales      uint8 [E, N, K/16] (NVFP4) + fp32 global [E].
  *       E4M3 codes        uint8 [E, N, K] + fp32 per-channel scales [E, N].
- *   - Decoded values: INT4 w = (q - z) * s (z = 0 when symmetric);
+ *   - Decoded values: INT4 w = (q - z) * s (z = 0 when symmetric; MXINT4
+ *     s = 2^(c - 127));
  *     MXFP4 w = e2m1 * 2^(c - 127); NVFP4 w = e2m1 * ue4m3 * g;
  *     FP8 w = e4m3 with the channel scale applied to the output.
  *   - Accumulation is fp32; outputs are bf16 (round to nearest even).
@@ -89,6 +90,7 @@ typedef enum {
  * Unified quantisation description ("Announcing Humming", section "Unified
  * quantization representation").  Supported weight descriptions:
  *   INT4  + BF16 scales, w_group in {0 (per channel), 32, 64, 128}
+ *   INT4  + E8M0 scales, w_group = 32                       (MXINT4)
  *   UINT4 + BF16 scales + zero points, w_group in {32, 64, 128}
  *   E2M1  + E8M0 scales, w_group = 32                       (MXFP4)
  *   E2M1  + UE4M3 scales, w_group = 16, w_has_global = 1    (NVFP4)

@@ -219,6 +219,9 @@ def decode_weights(d: Desc, N: int, K: int, codes, scales, zeros=None, global_sc
             s = bf16_to_f64(np.asarray(scales).reshape(N, G))
         elif d.w_scale == "fp32":
             s = np.asarray(scales, dtype=np.float32).reshape(N, G).astype(np.float64)
+        elif d.w_scale == "e8m0" and d.w_dtype == "int4" and g == 32 and not d.w_zero:
+            # MXINT4: the int32 words are the packed bytes (low nibble = even k)
+            return decode_mxint4_weights(np.ascontiguousarray(codes).view(np.uint8), scales, K), None
         else:
             raise ValueError(d.w_scale)
         z = np.zeros((N, G), dtype=np.int64)

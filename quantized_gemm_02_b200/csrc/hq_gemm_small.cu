@@ -168,11 +168,13 @@ __device__ __forceinline__ void decode_bf16(const uint8_t *wpk, const uint8_t *s
       const uint4 v = *reinterpret_cast<const uint4 *>(wpk + c * (BM * 16) + r * 16);
       const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
       const int gt = ((kbase + 32 * c) >> gshift) - g0;  // group of this chunk's first k
-      if constexpr (WF == W_INT4 || WF == W_UINT4) {
+      if constexpr (WF == W_INT4 || WF == W_UINT4 || WF == W_MXINT4) {
         // groups are >= 32 k: one scale (and zero point) per chunk, loaded
-        // again only when the second chunk starts a new group
+        // again only when the second chunk starts a new group (MXINT4: the
+        // E8M0 power of two as a bf16, exact)
         if (c == 0 || gt != (((kbase) >> gshift) - g0)) {
-          s2c = tc::bcast16(reinterpret_cast<const uint16_t *>(sc)[gt * BM + r]);
+          s2c = WF == W_MXINT4 ? tc::bcast16(tc::e8m0_code_to_bf16(sc[gt * BM + r]))
+                               : tc::bcast16(reinterpret_cast<const uint16_t *>(sc)[gt * BM + r]);
           z2c = (WF == W_UINT4) ? tc::bcast16(0x4300u + zp[gt * BM + r]) : 0x43084308u;
         }
         const uint32_t s2 = s2c, z2 = z2c;
@@ -697,6 +699,7 @@ hq_status launch_dec_gemm(const Layout &L, const tc::Params &p, const void *a, i
     return HQ_ERR_CUDA;
   switch (L.fmt) {
     case W_INT4: return dec_launch_wf<W_INT4>(map, p, t, st);
+    case W_MXINT4: return dec_launch_wf<W_MXINT4>(map, p, t, st);
     case W_UINT4: return dec_launch_wf<W_UINT4>(map, p, t, st);
     case W_MXFP4: return dec_launch_wf<W_MXFP4>(map, p, t, st);
     case W_NVFP4: return dec_launch_wf<W_NVFP4>(map, p, t, st);

@@ -547,9 +547,11 @@ __global__ void __launch_bounds__(THREADS, (BNT <= 64 ? 2 : 1)) tc_gemm_kernel(c
           if constexpr (TR::wbits == 4) {
             const uint4 v = *reinterpret_cast<const uint4 *>(wpk_j + half * (BM * 16) + r * 16);
             const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-            if constexpr (WF == W_INT4 || WF == W_UINT4) {
+            if constexpr (WF == W_INT4 || WF == W_UINT4 || WF == W_MXINT4) {
               // groups are >= 32 k: one scale (and zero point) covers the thread's 32 k
-              const uint32_t s2 = bcast16(reinterpret_cast<const uint16_t *>(sc)[gt * BM + r]);
+              // (MXINT4: the E8M0 power of two as a bf16, exact)
+              const uint32_t s2 = WF == W_MXINT4 ? bcast16(e8m0_code_to_bf16(sc[gt * BM + r]))
+                                                 : bcast16(reinterpret_cast<const uint16_t *>(sc)[gt * BM + r]);
               const uint32_t z2 = (WF == W_UINT4) ? bcast16(0x4300u + zp[gt * BM + r]) : 0x43084308u;
   #pragma unroll
               for (int j = 0; j < 4; ++j)
@@ -940,6 +942,7 @@ hq_status launch_tc_gemm(const Layout &L, const void *packed, const void *a_bf16
   if (gather && e4m3_act) return HQ_ERR_UNSUPPORTED;
   switch (L.fmt) {
     case W_INT4: return tc_launch_wf<W_INT4>(map, p, t, st);
+    case W_MXINT4: return tc_launch_wf<W_MXINT4>(map, p, t, st);
     case W_UINT4: return tc_launch_wf<W_UINT4>(map, p, t, st);
     case W_MXFP4: return tc_launch_wf<W_MXFP4>(map, p, t, st);
     case W_NVFP4: return tc_launch_wf<W_NVFP4>(map, p, t, st);

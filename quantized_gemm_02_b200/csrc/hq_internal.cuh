@@ -34,7 +34,9 @@
 namespace hq {
 
 // Internal weight formats.
-enum WFmt : int { W_INT4 = 0, W_UINT4 = 1, W_MXFP4 = 2, W_NVFP4 = 3, W_FP8 = 4, W_NFMT = 5 };
+// W_MXINT4: INT4 codes with an E8M0 scale per 32 along K (the MX layout with
+// integer elements).
+enum WFmt : int { W_INT4 = 0, W_UINT4 = 1, W_MXFP4 = 2, W_NVFP4 = 3, W_FP8 = 4, W_MXINT4 = 5, W_NFMT = 6 };
 // Internal activation formats.
 enum AFmt : int { A_BF16 = 0, A_FP8 = 1, A_MXFP8 = 2, A_NVFP4 = 3 };
 
@@ -74,7 +76,13 @@ inline bool weight_format(const hq_quant_desc *d, int *fmt) {
   if (!d) return false;
   switch (d->w_dtype) {
     case HQ_INT4:
-      if (d->w_scale_dtype != HQ_BF16 || d->w_has_zero || d->w_has_global) return false;
+      if (d->w_has_zero || d->w_has_global) return false;
+      if (d->w_scale_dtype == HQ_E8M0) {
+        if (d->w_group != 32) return false;
+        *fmt = W_MXINT4;
+        return true;
+      }
+      if (d->w_scale_dtype != HQ_BF16) return false;
       if (!(d->w_group == 0 || d->w_group == 32 || d->w_group == 64 || d->w_group == 128)) return false;
       *fmt = W_INT4;
       return true;

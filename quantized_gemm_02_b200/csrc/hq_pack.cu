@@ -66,8 +66,8 @@ __global__ void pack_weights_kernel(Layout L, int E, const uint8_t *codes, uint8
       uint32_t v = 0;
       if (r < L.N) {
         v = std_code(L.fmt, ce, L.K, r, k);
-        if (L.fmt == W_INT4) v ^= 8u;  // two's complement -> biased (q + 8)
-      } else if (L.fmt == W_INT4) {
+        if (L.fmt == W_INT4 || L.fmt == W_MXINT4) v ^= 8u;  // two's complement -> biased (q + 8)
+      } else if (L.fmt == W_INT4 || L.fmt == W_MXINT4) {
         v = 8u;  // padded rows decode to zero
       }
       word |= v << (slot * L.wbits);
@@ -141,7 +141,7 @@ __global__ void unpack_codes_kernel(Layout L, int E, const uint8_t *packed, uint
       const FragPos fp = frag_pos(L.wbits, i_row, kk);
       const size_t unit = (size_t)nt * L.KB + kb;
       uint32_t v = (pw[unit * words_per_unit + fp.word] >> fp.shift) & ((1u << L.wbits) - 1u);
-      if (L.fmt == W_INT4) v ^= 8u;
+      if (L.fmt == W_INT4 || L.fmt == W_MXINT4) v ^= 8u;
       out |= v << (j * L.wbits);
     }
     if (per == 8) reinterpret_cast<uint32_t *>(codes)[idx] = out;

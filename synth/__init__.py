@@ -34,7 +34,7 @@ import numpy as np
 import torch
 
 __all__ = [
-    "generator", "bf16_normal", "random_bytes", "int4_weights", "mxfp4_weights",
+    "generator", "bf16_normal", "random_bytes", "int4_weights", "mxint4_weights", "mxfp4_weights",
     "nvfp4_weights_random", "fp8_weights_random", "routing_softmax_topk", "routing_zipf",
     "pack_nibbles_i32", "pack_nibbles_u8", "to_np_bits",
 ]
@@ -118,6 +118,16 @@ def int4_weights(E: int, N: int, K: int, group: int, asym: bool, gen: torch.Gene
             z[..., -1] &= keep
         zeros = z
     return {"codes": codes, "scales": scales, "zeros": zeros}
+
+
+def mxint4_weights(E: int, N: int, K: int, gen: torch.Generator, exp_lo: int = -8, exp_hi: int = -4,
+                   device: str = "cpu") -> dict:
+    """MXINT4: INT4 codes uniform over all 16 nibbles (int32 words as for
+    INT4); E8M0 scale exponents uniform over the integers [exp_lo, exp_hi]."""
+    codes = random_bytes((E, N, K // 2), gen, device).view(torch.int32)
+    e = torch.randint(exp_lo + 127, exp_hi + 128, (E, N, K // 32), generator=gen,
+                      dtype=torch.int32, device=device)
+    return {"codes": codes, "scales": e.to(torch.uint8)}
 
 
 def mxfp4_weights(E: int, N: int, K: int, gen: torch.Generator, exp_lo: int = -8, exp_hi: int = -4,

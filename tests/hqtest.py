@@ -30,6 +30,8 @@ WFORMATS = {
               dict(w_dtype="e2m1", w_group=16, w_scale="ue4m3", w_global=True)),
     "fp8": (dict(w_dtype=5, w_group=0, w_scale_dtype=1, w_has_zero=0, w_has_global=0),
             dict(w_dtype="e4m3", w_group=0, w_scale="fp32")),
+    "mxint4": (dict(w_dtype=2, w_group=32, w_scale_dtype=6, w_has_zero=0, w_has_global=0),
+               dict(w_dtype="int4", w_group=32, w_scale="e8m0")),
 }
 AFORMATS = {"bf16": 0, "fp8": 5, "mxfp8": 8, "nvfp4": 9}
 
@@ -49,6 +51,9 @@ def make_weights(wname: str, E: int, N: int, K: int, seed: int = 0, device: str 
     """Standard-format weights for E experts (torch tensors on ``device``)."""
     g = synth.generator(seed, device)
     fields, _ = WFORMATS[wname]
+    if wname == "mxint4":
+        w = synth.mxint4_weights(E, N, K, g, device=device)
+        return {"codes": w["codes"], "scales": w["scales"], "zeros": None, "global": None}
     if fields["w_dtype"] in (2, 3):
         w = synth.int4_weights(E, N, K, fields["w_group"], fields["w_dtype"] == 3, g, device)
         return {"codes": w["codes"], "scales": w["scales"], "zeros": w["zeros"], "global": None}

@@ -302,6 +302,12 @@ def test_config4_moe_w4a8_zipf(T, part):
     _moe_full("mxfp4", "mxfp8", T, part, zipf=True, seed=900 + T)
 
 
+@pytest.mark.parametrize("T,part", [(16, "gate_up"), (4096, "gate_up"), (4096, "down")])
+def test_moe_w4a16_mxint4(T, part):
+    # MXINT4 weights (INT4 elements, E8M0 per 32) at the config-3 MoE shapes
+    _moe_full("mxint4", "bf16", T, part, zipf=False, seed=1100 + T)
+
+
 @pytest.mark.parametrize("part", ["gate_up", "down"])
 def test_config5_moe_nvfp4(part):
     _moe_full("nvfp4", "nvfp4", 4096, part, zipf=False, seed=1000)

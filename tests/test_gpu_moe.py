@@ -87,7 +87,7 @@ def moe_case(wname, aname, T, E, k, N, K, a_per_slot, seed, zipf=False, device_w
 
 
 @pytest.mark.parametrize("wname,aname", [("mxfp4", "bf16"), ("int4_g128", "bf16"), ("uint4_g64", "bf16"),
-                                         ("mxfp4", "mxfp8"), ("nvfp4", "nvfp4"), ("fp8", "fp8")])
+                                         ("mxfp4", "mxfp8"), ("nvfp4", "nvfp4"), ("fp8", "fp8"), ("mxint4", "bf16")])
 @pytest.mark.parametrize("a_per_slot", [0, 1])
 def test_moe_small(wname, aname, a_per_slot):
     T, E, k, N, K = 23, 16, 4, 96, 256

@@ -110,3 +110,21 @@ def test_fp8_block_scales_reduce_to_per_channel_and_per_token():
     A = O.decode_fp8_block_act(q, s)
     A2, row = O.decode_act("fp8", 15, 128, q2, s2)
     assert np.array_equal(A, (A2 * row[:, None]).reshape(5, 384))
+
+
+def test_mxint4_through_decode_weights_equals_int4_with_power_of_two_scales():
+    # the unified description routes INT4 + E8M0 per 32 to the MXINT4
+    # decoder, reading the INT4 int32 words as their bytes; with bf16 group
+    # scales equal to the same powers of two (bf16 bits = code << 7) the
+    # plain INT4 g32 decoder gives the same weights
+    N, K = 6, 128
+    g = synth.generator(11)
+    w = synth.mxint4_weights(1, N, K, g, exp_lo=-20, exp_hi=10)
+    codes = w["codes"][0].numpy()
+    sc = w["scales"][0].numpy()
+    Wm, col = O.decode_weights(O.Desc("int4", 32, "e8m0"), N, K, codes, sc)
+    assert col is None
+    assert np.array_equal(Wm, O.decode_mxint4_weights(codes.view(np.uint8), sc, K))
+    bf16_scales = (sc.astype(np.uint16) << 7).astype(np.uint16)
+    Wi, _ = O.decode_weights(O.Desc("int4", 32, "bf16"), N, K, codes, bf16_scales)
+    assert np.array_equal(Wm, Wi)
