@@ -56,6 +56,7 @@ __all__ = [
     "gemm", "moe_permute", "moe", "moe_expert_outputs", "moe_masked", "silu_and_mul", "nvfp4_global_scale",
     "fp6_value", "E2M3", "E3M2", "decode_int_weights", "decode_fp6_weights", "decode_mxint4_weights",
     "decode_fp8_block_weights", "quant_fp8_block", "decode_fp8_block_act",
+    "unpack_bits", "e0m_value", "E0M3", "E0M7", "int_to_e0m", "decode_lowbit_weights",
 ]
 
 
@@ -551,3 +552,68 @@ def decode_fp8_block_act(codes, scales, group: int = 128):
     M, K = c.shape
     s = np.asarray(scales, dtype=np.float32).astype(np.float64).reshape(M, K // group)
     return E4M3[c] * s[:, np.arange(K) // group]
+
+
+# ---------------------------------------------------------------------------
+# Standard format of b-bit weight codes and the zero-exponent float view
+# ("Announcing Humming", section "Quantization support": a float format with
+# no exponent bits whose values are the symmetric integers of its width,
+# e.g. float8e0m7 and INT8 without -128 both hold -127..127; symmetric INT
+# weights that fit are converted to it; section "Performance", WnA16:
+# INT1/2/3 and FP4 to FP8 weights)
+# ---------------------------------------------------------------------------
+
+def unpack_bits(packed, bits: int, K: int) -> np.ndarray:
+    """b-bit codes from a little-endian bit stream per row: element k of a row
+    occupies bits [b*k, b*k + b) of the row's bytes (bit 0 = the least
+    significant bit of byte 0).  For b = 4 this is the INT4 / E2M1 nibble
+    order.  Reading: the pages give no packing for INT1/2/3 or FP6; this is
+    the plain stream."""
+    by = np.asarray(packed, dtype=np.uint8)
+    bitsarr = np.unpackbits(by, axis=-1, bitorder="little")[..., :bits * K]
+    bitsarr = bitsarr.reshape(*by.shape[:-1], K, bits).astype(np.int64)
+    return (bitsarr << np.arange(bits, dtype=np.int64)).sum(axis=-1)
+
+
+def e0m_value(code: int, bits: int) -> float:
+    """Float with zero exponent bits and (bits - 1) mantissa bits
+    (float4e0m3, float8e0m7): the sign bit, then the magnitude m read as an
+    integer; the value is -m or m (code 1 << (bits - 1) is -0)."""
+    m = code & ((1 << (bits - 1)) - 1)
+    return -float(m) if (code >> (bits - 1)) & 1 else float(m)
+
+
+E0M3 = np.array([e0m_value(c, 4) for c in range(16)], dtype=np.float64)
+E0M7 = np.array([e0m_value(c, 8) for c in range(256)], dtype=np.float64)
+
+
+def int_to_e0m(q, bits: int) -> np.ndarray:
+    """Symmetric integers |q| <= 2^(bits - 1) - 1 to their zero-exponent
+    codes (sign bit and magnitude); q = 0 gives +0."""
+    q = np.asarray(q, dtype=np.int64)
+    lim = (1 << (bits - 1)) - 1
+    if np.any(np.abs(q) > lim):
+        raise ValueError("not a symmetric integer of this width")
+    return (np.where(q < 0, 1 << (bits - 1), 0) | np.abs(q)).astype(np.int64)
+
+
+def decode_lowbit_weights(kind: str, packed, scales, K: int, group: int = 0, zeros=None):
+    """Weights of the other WnA16 widths from the standard bit stream
+    (``unpack_bits``) [N, K * b / 8] bytes:
+      'int2' / 'int3': signed b-bit two's complement times bf16 group scales;
+      'uint2' / 'uint3': (u - z) times bf16 group scales, z uint8 [N, K/group];
+      'e0m3': float4e0m3 times bf16 group scales;
+      'e2m3' / 'e3m2': MXFP6 with an E8M0 scale per 32."""
+    if kind in ("int2", "int3", "uint2", "uint3"):
+        b = int(kind[-1])
+        u = unpack_bits(packed, b, K)
+        return decode_int_weights(b, u, scales, group, zeros if kind.startswith("u") else None)
+    if kind == "e0m3":
+        c = unpack_bits(packed, 4, K)
+        N = c.shape[0]
+        g = K if group == 0 else group
+        s = bf16_to_f64(np.asarray(scales).reshape(N, K // g))
+        return E0M3[c] * s[:, np.arange(K) // g]
+    if kind in ("e2m3", "e3m2"):
+        return decode_fp6_weights(kind, unpack_bits(packed, 6, K), scales)
+    raise ValueError(kind)
