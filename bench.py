@@ -318,6 +318,10 @@ CONFIG_TITLES = {
        "T in {1,64,512,4096}, grouped + indexed, fused weighted sum",
     5: "dense W4A4 NVFP4 x NVFP4 and W8A8 FP8 (per-channel x per-token), N=K=7168, M in {1,32,256,2048,8192}, "
        "activation quantisation inside the step; NVFP4 MoE at T=4096, grouped + indexed",
+    "silu": "MoE gate-up GEMM + SiLU-and-mul at the config-3 shapes (MXFP4, bf16 activations, grouped), "
+            "T in {16, 4096}: two calls versus the fused epilogue",
+    "lowbit": "dense WnA16 at the other widths (INT2, INT3 g128; MXFP6 E2M3; float4e0m3 g128), N=28672, "
+              "K=8192, M in {1, 16}",
     "mxint4": "MoE W4A16 MXINT4 (INT4 elements, E8M0 per 32) at the config-3 shapes and routing, T in {16, 4096}, "
               "grouped + indexed",
 }
@@ -334,6 +338,8 @@ WORKLOAD_TITLE = {
                  "grouped + indexed",
     "w4a4_nvfp4": "dense W4A4 NVFP4 x NVFP4, N=K=7168, M in {1,32,256,2048,8192}",
     "w8a8_fp8": "dense W8A8 FP8 per-channel x per-token, N=K=7168, M in {1,32,256,2048,8192}",
+    "moe_silu": "MoE gate-up GEMM + SiLU-and-mul at the config-3 shapes, T in {16, 4096}: unfused and fused",
+    "lowbit": "dense WnA16 INT2, INT3, MXFP6 E2M3, float4e0m3 at N=28672, K=8192, M in {1, 16}",
     "moe_w4a16_mxint4": "MoE W4A16 MXINT4 (INT4 elements, E8M0 per 32), config-3 shapes and routing, T in "
                         "{16, 4096}, grouped + indexed",
     "moe_masked_nvfp4": "masked-layout MoE W4A4 NVFP4 x NVFP4 (activations quantised on the fly), E=256 slabs of "
@@ -375,6 +381,28 @@ def ops_shape(hq, M, N, K, gen):
     packed = torch.empty(hq.hq_packed_weights_bytes(d, 1, N, K), dtype=torch.uint8, device="cuda")
     hq.hq_pack_weights(d, 1, N, K, w["codes"], w["scales"], w["zeros"], None, packed)
     return [dense_op(hq, d, f"N{N}_K{K}_M{M}", M, N, K, packed, packed_bytes_int4(N, K, 128, True), gen, 2)], [packed]
+
+
+def ops_lowbit(hq, gen, N=28672, K=8192, Ms=(1, 16)):
+    """The other WnA16 widths on the largest config-2 shape with bf16
+    activations: INT2 and INT3 (symmetric, bf16 scales per 128), MXFP6
+    (E2M3, E8M0 per 32) and float4e0m3 (the zero-exponent view of symmetric
+    INT4, bf16 scales per 128); weight GB/s at decode sizes."""
+    kinds = [("int2_g128", hq.HQ_INT2, 128, hq.HQ_BF16, 2, False),
+             ("int3_g128", hq.HQ_INT3, 128, hq.HQ_BF16, 3, False),
+             ("mxfp6_e2m3", hq.HQ_E2M3, 32, hq.HQ_E8M0, 6, True),
+             ("e0m3_g128", hq.HQ_E0M3, 128, hq.HQ_BF16, 4, False)]
+    ops, keep = [], []
+    for name, wd, grp, sd, bits, e8 in kinds:
+        d = desc_of(hq, wd, grp, sd, 0, 0, hq.HQ_BF16)
+        w = synth.lowbit_weights(1, N, K, bits, grp, False, e8, gen, device="cuda")
+        packed = torch.empty(hq.hq_packed_weights_bytes(d, 1, N, K), dtype=torch.uint8, device="cuda")
+        hq.hq_pack_weights(d, 1, N, K, w["codes"], w["scales"], None, None, packed)
+        keep.append(packed)
+        wb = N * K * bits // 8 + N * (K // grp) * (1 if e8 else 2)
+        for M in Ms:
+            ops.append(dense_op(hq, d, f"{name}_N{N}_K{K}_M{M}", M, N, K, packed, wb, gen, "lowbit"))
+    return ops, keep
 
 
 def moe_call_kernels(hq, wdesc, a_dtype, mode, combine):
@@ -505,6 +533,61 @@ def ops_moe_w4a16_mxint4(hq, gen, Ts=(16, 4096)):
     routing = lambda T, g: synth.routing_softmax_topk(T, E_MOE, TOPK, g, device="cuda")
     return ops_moe(hq, "mxint4", "moe_w4a16_mxint4", d, E_MOE, TOPK, H_MOE, I_MOE, list(Ts), routing, gen,
                    hq.HQ_BF16)
+
+
+def ops_moe_silu(hq, gen, Ts=(16, 4096)):
+    """The gate-up GEMM followed by SiLU-and-mul at the config-3 shapes
+    (MXFP4 weights, bf16 activations, grouped mode): the two-call form
+    (hq_moe_gemm writing the [T * 8, 2I] gate-up rows, then hq_silu_and_mul)
+    and the fused form (hq_moe_gemm_gated on gate/up-interleaved weights)."""
+    dev = "cuda"
+    E, topk, H, I = E_MOE, TOPK, H_MOE, I_MOE
+    d = desc_of(hq, hq.HQ_E2M1, 32, hq.HQ_E8M0, 0, 0, hq.HQ_BF16)
+    w = synth.mxfp4_weights(E, 2 * I, H, gen, device=dev)
+    nb = hq.hq_packed_weights_bytes(d, E, 2 * I, H)
+    plain = torch.empty(nb, dtype=torch.uint8, device=dev)
+    gated = torch.empty(nb, dtype=torch.uint8, device=dev)
+    hq.hq_pack_weights(d, E, 2 * I, H, w["codes"], w["scales"], None, None, plain)
+    hq.hq_pack_weights_gated(d, E, 2 * I, H, w["codes"], w["scales"], None, None, gated)
+    del w
+    bytes_per = 2 * I * H // 2 + 2 * I * H // 32
+    ops, keep = [], [plain, gated]
+    for T in Ts:
+        ids, wts = synth.routing_softmax_topk(T, E, topk, gen, device=dev)
+        touched = int(torch.unique(ids).numel())
+        x = synth.bf16_normal((T, H), gen, device=dev)
+        off = torch.empty(E + 1, dtype=torch.int32, device=dev)
+        perm = torch.empty(T * topk, dtype=torch.int32, device=dev)
+        inv = torch.empty(T * topk, dtype=torch.int32, device=dev)
+        hq.hq_moe_permute(T, topk, E, ids, off, perm, inv)
+        mode = hq.HQ_MOE_GROUPED
+        wsb = max(hq.hq_moe_workspace_bytes(mode, d, T, topk, E, 2 * I, H, 0, 0),
+                  hq.hq_moe_gated_workspace_bytes(mode, d, T, topk, E, I, H))
+        ws = torch.zeros(wsb, dtype=torch.uint8, device=dev)
+        y = torch.empty(T * topk, 2 * I, dtype=torch.bfloat16, device=dev)
+        h = torch.empty(T * topk, I, dtype=torch.bfloat16, device=dev)
+        x_h = x.cpu().pin_memory()
+        h_h = torch.empty(T * topk, I, dtype=torch.bfloat16).pin_memory()
+        keep += [ids, wts, x, off, perm, inv, ws, y, h, x_h, h_h]
+
+        def run_two(T=T, x=x, off=off, perm=perm, ws=ws, y=y, h=h, wsb=wsb):
+            hq.hq_moe_gemm(mode, d, T, topk, E, 2 * I, H, plain, x, None, None, 0, None, None, off, perm, 0, 1.0, y,
+                           ws, wsb)
+            hq.hq_silu_and_mul(T * topk, I, y, h)
+
+        def run_fused(T=T, x=x, off=off, perm=perm, ws=ws, h=h, wsb=wsb):
+            hq.hq_moe_gemm_gated(mode, d, T, topk, E, I, H, gated, x, None, None, None, off, perm, h, ws, wsb)
+
+        for nm, run, nk in (("gate_up_then_silu", run_two, 3), ("gate_up_silu_fused", run_fused, 2)):
+            def e2e(run=run, x=x, x_h=x_h, h=h, h_h=h_h):
+                x.copy_(x_h, non_blocking=True)
+                run()
+                h_h.copy_(h, non_blocking=True)
+            io = T * H * 2 + T * topk * I * 2 + (2 * T * topk * 2 * I * 2 if nm == "gate_up_then_silu" else 0)
+            ops.append(Op(f"silu_mxfp4_T{T}_{nm}", run, 2.0 * T * topk * 2 * I * H, touched * bytes_per, io, nk,
+                          T * H * 2, T * topk * I * 2, e2e, kernel="dec_gemm_kernel / tc_gemm_kernel",
+                          config="silu"))
+    return ops, keep
 
 
 def ops_moe_w4a8_mxfp8(hq, gen, Ts=(1, 64, 512, 4096)):
@@ -643,7 +726,9 @@ def _workload(builders, title):
 WORKLOADS = {
     "all": _workload([ops_w4a16_dense_m16, ops_w4a16_asym_sweep, ops_moe_w4a16_mxfp4, ops_moe_w4a8_mxfp8,
                       lambda hq, g: ops_dense_quantised(hq, "nvfp4", g), lambda hq, g: ops_dense_quantised(hq, "fp8", g),
-                      ops_moe_nvfp4, ops_moe_w4a16_mxint4], WORKLOAD_TITLE["all"]),
+                      ops_moe_nvfp4, ops_moe_w4a16_mxint4, ops_moe_silu, ops_lowbit], WORKLOAD_TITLE["all"]),
+    "lowbit": _workload([ops_lowbit], WORKLOAD_TITLE["lowbit"]),
+    "moe_silu": _workload([ops_moe_silu], WORKLOAD_TITLE["moe_silu"]),
     "moe_w4a16_mxint4": _workload([ops_moe_w4a16_mxint4], WORKLOAD_TITLE["moe_w4a16_mxint4"]),
     "w4a16_asym_sweep": _workload([ops_w4a16_asym_sweep], WORKLOAD_TITLE["w4a16_asym_sweep"]),
     "w4a16_dense_m16": _workload([ops_w4a16_dense_m16], WORKLOAD_TITLE["w4a16_dense_m16"]),
@@ -656,7 +741,7 @@ WORKLOADS = {
 }
 
 # configurations each workload covers (for the CPU samples)
-WORKLOAD_CONFIGS = {"all": (1, 2, 3, 4, 5), "moe_w4a16_mxint4": (3,), "w4a16_asym_sweep": (2,), "w4a16_dense_m16": (1,),
+WORKLOAD_CONFIGS = {"all": (1, 2, 3, 4, 5), "moe_w4a16_mxint4": (3,), "moe_silu": (3,), "lowbit": (2,), "w4a16_asym_sweep": (2,), "w4a16_dense_m16": (1,),
                     "moe_w4a16_mxfp4": (3,), "moe_w4a8_mxfp8": (4,), "moe_nvfp4": (5,), "moe_masked_nvfp4": (5,),
                     "w4a4_nvfp4": (5,), "w8a8_fp8": (5,)}
 

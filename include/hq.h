@@ -37,6 +37,12 @@
  *       E8M0 scales       uint8 [E, N, K/32] (MXFP4, MXINT4).
  *       UE4M3 scales      uint8 [E, N, K/16] (NVFP4) + fp32 global [E].
  *       E4M3 codes        uint8 [E, N, K] + fp32 per-channel scales [E, N].
+ *       INT2/UINT2/INT3/UINT3/E2M3/E3M2/E0M3 codes (b bits): uint8
+ *                         [E, N, K * b / 8], a little-endian bit stream per
+ *                         row (code k at bits b*k .. b*k + b - 1; for b = 4
+ *                         the INT4 / E2M1 nibble order).  UINT2/UINT3 zero
+ *                         points: uint8 [E, N, G], one per byte.  E0M3 code:
+ *                         bit 3 = sign, bits 0..2 = magnitude.
  *   - Decoded values: INT4 w = (q - z) * s (z = 0 when symmetric; MXINT4
  *     s = 2^(c - 127));
  *     MXFP4 w = e2m1 * 2^(c - 127); NVFP4 w = e2m1 * ue4m3 * g;
@@ -83,7 +89,14 @@ typedef enum {
   HQ_E8M0 = 6,   /* power-of-two scale (OCP MX)                            */
   HQ_UE4M3 = 7,  /* unsigned E4M3 block scale (NVFP4)                      */
   HQ_MXFP8 = 8,  /* activation: E4M3 codes + E8M0 scale per 32 along K     */
-  HQ_NVFP4 = 9   /* activation: E2M1 codes + UE4M3 per 16 + fp32 global    */
+  HQ_NVFP4 = 9,  /* activation: E2M1 codes + UE4M3 per 16 + fp32 global    */
+  HQ_INT2 = 10,  /* signed 2-bit, two's complement                         */
+  HQ_UINT2 = 11, /* unsigned 2-bit (with zero points)                      */
+  HQ_INT3 = 12,  /* signed 3-bit, two's complement                         */
+  HQ_UINT3 = 13, /* unsigned 3-bit (with zero points)                      */
+  HQ_E2M3 = 14,  /* FP6 (OCP MX), with E8M0 scales: MXFP6                  */
+  HQ_E3M2 = 15,  /* FP6 (OCP MX), with E8M0 scales: MXFP6                  */
+  HQ_E0M3 = 16   /* float4e0m3: sign + 3-bit magnitude, no exponent bits   */
 } hq_dtype;
 
 /*
@@ -95,7 +108,13 @@ typedef enum {
  *   E2M1  + E8M0 scales, w_group = 32                       (MXFP4)
  *   E2M1  + UE4M3 scales, w_group = 16, w_has_global = 1    (NVFP4)
  *   E4M3  + FP32 per-channel scales, w_group = 0            (FP8)
- * and every one of them with a_dtype in {BF16, E4M3, MXFP8, NVFP4}.
+ *   INT2, INT3, E0M3 + BF16 scales, w_group in {0, 32, 64, 128}
+ *   UINT2, UINT3 + BF16 scales + zero points, w_group in {32, 64, 128}
+ *   E2M3, E3M2 + E8M0 scales, w_group = 32                  (MXFP6)
+ * and every one of them with a_dtype in {BF16, E4M3, MXFP8, NVFP4}.  E0M3
+ * ("Announcing Humming", section "Quantization support": a float with no
+ * exponent bits, whose values are the symmetric integers -7..7) is the
+ * zero-exponent view of symmetric INT4 and computes as INT4.
  * a_group is the activation's scale granularity along K: 0 = the format's
  * own (E4M3: one fp32 scale per token; MXFP8: 32; NVFP4: 16); MXFP8 also
  * accepts 32 and NVFP4 16.  Zero-initialise the struct.
@@ -304,6 +323,38 @@ HQ_API hq_status hq_moe_gemm(hq_moe_mode mode, const hq_quant_desc *desc, int T,
                       const float *topk_weights, const int32_t *expert_offsets, const int32_t *perm,
                       int combine, float routed_scale, void *out_bf16, void *workspace, size_t ws_bytes,
                       hq_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Gate-up GEMM with SiLU-and-mul fused into its epilogue (an addition of this
+ * library; the pages name no activation, and the gated-MLP form is the
+ * usual one).  For an MoE layer's gate-up weights, N2 = 2I rows per expert
+ * (standard format: gate rows 0..I-1, then up rows I..2I-1), I a multiple of
+ * 64:
+ *   hq_pack_weights_gated / hq_unpack_weights_gated: as hq_pack_weights /
+ *       hq_unpack_weights (same arguments, same hq_packed_weights_bytes), but
+ *       the gate and the up row of each output column are stored side by
+ *       side in the packed tiles.  Only hq_moe_gemm_gated reads this form.
+ *   hq_moe_gemm_gated: hq_moe_gemm's gate-up call (one activation row per
+ *       token, a_per_slot = 0; modes, activation formats, routing and
+ *       workspace rules as there, hq_moe_gated_workspace_bytes) whose
+ *       epilogue writes out bf16 [T * topk, I] in slot order:
+ *       out[s, i] = bf16_rne(silu(g) * u), g = Y[s, i], u = Y[s, I + i] in
+ *       fp32 (Y unrounded), silu(g) = g / (1 + exp(-g)).  The up-and-gate
+ *       bf16 tensor [T * topk, 2I] of the unfused path never reaches HBM.
+ * ---------------------------------------------------------------------- */
+HQ_API hq_status hq_pack_weights_gated(const hq_quant_desc *desc, int E, int N2, int K, const void *codes,
+                                       const void *scales, const void *zeros, const float *global_scale,
+                                       void *packed, hq_stream_t stream);
+HQ_API hq_status hq_unpack_weights_gated(const hq_quant_desc *desc, int E, int N2, int K, const void *packed,
+                                         void *codes, void *scales, void *zeros, float *global_scale,
+                                         hq_stream_t stream);
+HQ_API size_t hq_moe_gated_workspace_bytes(hq_moe_mode mode, const hq_quant_desc *desc, int T, int topk, int E,
+                                           int I, int K);
+HQ_API hq_status hq_moe_gemm_gated(hq_moe_mode mode, const hq_quant_desc *desc, int T, int topk, int E, int I,
+                                   int K, const void *packed_w, const void *a, const void *a_scales,
+                                   const float *a_global, const int32_t *topk_ids, const int32_t *expert_offsets,
+                                   const int32_t *perm, void *out_bf16, void *workspace, size_t ws_bytes,
+                                   hq_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * Masked MoE expert GEMM (SGLang digest: humming_moe_runner_core_run with

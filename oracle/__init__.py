@@ -211,6 +211,10 @@ def decode_weights(d: Desc, N: int, K: int, codes, scales, zeros=None, global_sc
     scales are folded into W).
     """
     col = None
+    if d.w_dtype in ("int2", "uint2", "int3", "uint3", "e0m3", "e2m3", "e3m2"):
+        # the other widths, from the standard b-bit code stream
+        z = None if zeros is None else np.asarray(zeros).reshape(N, -1)
+        return decode_lowbit_weights(d.w_dtype, np.asarray(codes).reshape(N, -1), scales, K, d.w_group, z), None
     if d.w_dtype in ("int4", "uint4"):
         q = unpack_nibbles_i32(codes, K)
         q = _signed4(q) if d.w_dtype == "int4" else q.astype(np.int64)

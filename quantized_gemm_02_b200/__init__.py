@@ -14,15 +14,18 @@ import os
 __all__ = [
     "HQError", "QuantDesc", "ComputeConfig", "PlanInfo", "lib", "library_path", "EXPORTS",
     "HQ_BF16", "HQ_FP32", "HQ_INT4", "HQ_UINT4", "HQ_E2M1", "HQ_E4M3", "HQ_E8M0", "HQ_UE4M3", "HQ_MXFP8",
-    "HQ_NVFP4", "HQ_MOE_GROUPED", "HQ_MOE_INDEXED",
+    "HQ_NVFP4", "HQ_INT2", "HQ_UINT2", "HQ_INT3", "HQ_UINT3", "HQ_E2M3", "HQ_E3M2", "HQ_E0M3",
+    "HQ_MOE_GROUPED", "HQ_MOE_INDEXED",
     "hq_status_string", "hq_device_error", "hq_packed_weights_bytes", "hq_pack_weights", "hq_unpack_weights",
     "hq_quant_act", "hq_gemm_workspace_bytes", "hq_gemm", "hq_gemm_config_workspace_bytes",
     "hq_gemm_config", "hq_gemm_plan", "hq_moe_plan", "hq_moe_permute", "hq_moe_workspace_bytes",
     "hq_moe_gemm", "hq_moe_masked_workspace_bytes", "hq_moe_gemm_masked", "hq_silu_and_mul", "hq_moe_unpermute_sum",
-    "hq_gemm_noalloc", "hq_selftest_wait_timeout",
+    "hq_gemm_noalloc", "hq_selftest_wait_timeout", "hq_pack_weights_gated", "hq_unpack_weights_gated",
+    "hq_moe_gated_workspace_bytes", "hq_moe_gemm_gated",
 ]
 
 HQ_BF16, HQ_FP32, HQ_INT4, HQ_UINT4, HQ_E2M1, HQ_E4M3, HQ_E8M0, HQ_UE4M3, HQ_MXFP8, HQ_NVFP4 = range(10)
+HQ_INT2, HQ_UINT2, HQ_INT3, HQ_UINT3, HQ_E2M3, HQ_E3M2, HQ_E0M3 = range(10, 17)
 HQ_MOE_GROUPED, HQ_MOE_INDEXED = 0, 1
 
 STATUS = {
@@ -36,7 +39,8 @@ EXPORTS = (
     "hq_quant_act", "hq_gemm_workspace_bytes", "hq_gemm", "hq_gemm_config_workspace_bytes",
     "hq_gemm_config", "hq_gemm_plan", "hq_moe_plan", "hq_moe_permute", "hq_moe_workspace_bytes",
     "hq_moe_gemm", "hq_moe_masked_workspace_bytes", "hq_moe_gemm_masked", "hq_silu_and_mul", "hq_moe_unpermute_sum",
-    "hq_gemm_noalloc", "hq_selftest_wait_timeout",
+    "hq_gemm_noalloc", "hq_selftest_wait_timeout", "hq_pack_weights_gated", "hq_unpack_weights_gated",
+    "hq_moe_gated_workspace_bytes", "hq_moe_gemm_gated",
 )
 
 
@@ -118,6 +122,10 @@ def _lib() -> ctypes.CDLL:
             "hq_moe_unpermute_sum": (I, [I, I, I, P, P, P, F, P, P]),
             "hq_gemm_noalloc": (I, [D, I, I, I, P, P, P, P, P, P]),
             "hq_selftest_wait_timeout": (I, [ctypes.c_ulonglong, P]),
+            "hq_pack_weights_gated": (I, [D, I, I, I, P, P, P, P, P, P]),
+            "hq_unpack_weights_gated": (I, [D, I, I, I, P, P, P, P, P, P]),
+            "hq_moe_gated_workspace_bytes": (Z, [I, D, I, I, I, I, I]),
+            "hq_moe_gemm_gated": (I, [I, D, I, I, I, I, I, P, P, P, P, P, P, P, P, P, Z, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -271,3 +279,28 @@ def hq_selftest_wait_timeout(limit_ns: int, stream=None):
     limit_ns); afterwards hq_device_error() reports HQ_ERR_TIMEOUT."""
     _check("hq_selftest_wait_timeout", _lib().hq_selftest_wait_timeout(int(limit_ns), _stream(stream)))
 
+
+
+def hq_pack_weights_gated(desc, E, N2, K, codes, scales, zeros, global_scale, packed, stream=None):
+    """hq_pack_weights for gate-up weights read by hq_moe_gemm_gated."""
+    _check("hq_pack_weights_gated", _lib().hq_pack_weights_gated(
+        ctypes.byref(desc), E, N2, K, _ptr(codes), _ptr(scales), _ptr(zeros), _ptr(global_scale), _ptr(packed),
+        _stream(stream)))
+
+
+def hq_unpack_weights_gated(desc, E, N2, K, packed, codes, scales, zeros, global_scale, stream=None):
+    _check("hq_unpack_weights_gated", _lib().hq_unpack_weights_gated(
+        ctypes.byref(desc), E, N2, K, _ptr(packed), _ptr(codes), _ptr(scales), _ptr(zeros), _ptr(global_scale),
+        _stream(stream)))
+
+
+def hq_moe_gated_workspace_bytes(mode, desc, T, topk, E, I, K) -> int:
+    return _lib().hq_moe_gated_workspace_bytes(mode, ctypes.byref(desc), T, topk, E, I, K)
+
+
+def hq_moe_gemm_gated(mode, desc, T, topk, E, I, K, packed_w, a, a_scales, a_global, topk_ids, expert_offsets, perm,
+                      out, workspace, ws_bytes, stream=None):
+    """Gate-up MoE GEMM with SiLU-and-mul in its epilogue: out [T * topk, I]."""
+    _check("hq_moe_gemm_gated", _lib().hq_moe_gemm_gated(
+        mode, ctypes.byref(desc), T, topk, E, I, K, _ptr(packed_w), _ptr(a), _ptr(a_scales), _ptr(a_global),
+        _ptr(topk_ids), _ptr(expert_offsets), _ptr(perm), _ptr(out), _ptr(workspace), ws_bytes, _stream(stream)))

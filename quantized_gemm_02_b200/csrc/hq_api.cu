@@ -374,33 +374,60 @@ size_t hq_packed_weights_bytes(const hq_quant_desc *desc, int E, int N, int K) {
   return layout_for(desc, fmt, N, K).stride * (size_t)E;
 }
 
-hq_status hq_pack_weights(const hq_quant_desc *desc, int E, int N, int K, const void *codes, const void *scales,
-                          const void *zeros, const float *global_scale, void *packed, hq_stream_t stream) {
+// Pack / unpack with the plain or the gated (gate/up rows side by side) row order.
+static hq_status pack_impl(const hq_quant_desc *desc, int E, int N, int K, const void *codes, const void *scales,
+                           const void *zeros, const float *global_scale, void *packed, hq_stream_t stream,
+                           bool gated) {
   int fmt;
   if (!desc) return HQ_ERR_INVALID_ARG;
   if (!weight_format(desc, &fmt)) return HQ_ERR_UNSUPPORTED;
   if (E < 1 || N < 1 || !valid_k(desc, K)) return HQ_ERR_INVALID_ARG;
+  if (gated && (N % TILE_N) != 0) return HQ_ERR_INVALID_ARG;
   if (!codes || !scales || !packed) return HQ_ERR_INVALID_ARG;
   if ((fmt == W_UINT4) != (zeros != nullptr)) return HQ_ERR_INVALID_ARG;
   if ((fmt == W_NVFP4) != (global_scale != nullptr)) return HQ_ERR_INVALID_ARG;
   if (!aligned16(codes) || !aligned16(packed) || ((uintptr_t)scales & 3u)) return HQ_ERR_INVALID_ARG;
   if (!device_is_sm100()) return HQ_ERR_ARCH;
-  const Layout L = layout_for(desc, fmt, N, K);
+  Layout L = layout_for(desc, fmt, N, K);
+  L.gated = gated ? 1 : 0;
   return launch_pack(L, E, codes, scales, zeros, global_scale, packed, (cudaStream_t)stream);
 }
 
-hq_status hq_unpack_weights(const hq_quant_desc *desc, int E, int N, int K, const void *packed, void *codes,
-                            void *scales, void *zeros, float *global_scale, hq_stream_t stream) {
+static hq_status unpack_impl(const hq_quant_desc *desc, int E, int N, int K, const void *packed, void *codes,
+                             void *scales, void *zeros, float *global_scale, hq_stream_t stream, bool gated) {
   int fmt;
   if (!desc) return HQ_ERR_INVALID_ARG;
   if (!weight_format(desc, &fmt)) return HQ_ERR_UNSUPPORTED;
   if (E < 1 || N < 1 || !valid_k(desc, K)) return HQ_ERR_INVALID_ARG;
+  if (gated && (N % TILE_N) != 0) return HQ_ERR_INVALID_ARG;
   if (!codes || !scales || !packed) return HQ_ERR_INVALID_ARG;
   if ((fmt == W_UINT4) != (zeros != nullptr)) return HQ_ERR_INVALID_ARG;
   if ((fmt == W_NVFP4) != (global_scale != nullptr)) return HQ_ERR_INVALID_ARG;
   if (!device_is_sm100()) return HQ_ERR_ARCH;
-  const Layout L = layout_for(desc, fmt, N, K);
+  Layout L = layout_for(desc, fmt, N, K);
+  L.gated = gated ? 1 : 0;
   return launch_unpack(L, E, packed, codes, scales, zeros, global_scale, (cudaStream_t)stream);
+}
+
+hq_status hq_pack_weights(const hq_quant_desc *desc, int E, int N, int K, const void *codes, const void *scales,
+                          const void *zeros, const float *global_scale, void *packed, hq_stream_t stream) {
+  return pack_impl(desc, E, N, K, codes, scales, zeros, global_scale, packed, stream, false);
+}
+
+hq_status hq_unpack_weights(const hq_quant_desc *desc, int E, int N, int K, const void *packed, void *codes,
+                            void *scales, void *zeros, float *global_scale, hq_stream_t stream) {
+  return unpack_impl(desc, E, N, K, packed, codes, scales, zeros, global_scale, stream, false);
+}
+
+hq_status hq_pack_weights_gated(const hq_quant_desc *desc, int E, int N2, int K, const void *codes,
+                                const void *scales, const void *zeros, const float *global_scale, void *packed,
+                                hq_stream_t stream) {
+  return pack_impl(desc, E, N2, K, codes, scales, zeros, global_scale, packed, stream, true);
+}
+
+hq_status hq_unpack_weights_gated(const hq_quant_desc *desc, int E, int N2, int K, const void *packed, void *codes,
+                                  void *scales, void *zeros, float *global_scale, hq_stream_t stream) {
+  return unpack_impl(desc, E, N2, K, packed, codes, scales, zeros, global_scale, stream, true);
 }
 
 hq_status hq_quant_act(const hq_quant_desc *desc, int M, int K, const void *x_bf16, void *codes, void *scales,
@@ -556,6 +583,47 @@ hq_status hq_moe_gemm(hq_moe_mode mode, const hq_quant_desc *desc, int T, int to
   }
   return moe_run(pl, mode, T, topk, E, N, K, packed_w, a, a_scales, a_global, a_per_slot ? 1 : topk, nullptr,
                  expert_offsets, perm, topk_weights, routed_scale, combine, out_bf16, w, st);
+}
+
+size_t hq_moe_gated_workspace_bytes(hq_moe_mode mode, const hq_quant_desc *desc, int T, int topk, int E, int I,
+                                    int K) {
+  if (I < 1 || (I % (TILE_N / 2)) != 0 || I > (1 << 29)) return 0;
+  return hq_moe_workspace_bytes(mode, desc, T, topk, E, 2 * I, K, 0, 0);
+}
+
+hq_status hq_moe_gemm_gated(hq_moe_mode mode, const hq_quant_desc *desc, int T, int topk, int E, int I, int K,
+                            const void *packed_w, const void *a, const void *a_scales, const float *a_global,
+                            const int32_t *topk_ids, const int32_t *expert_offsets, const int32_t *perm,
+                            void *out_bf16, void *workspace, size_t ws_bytes, hq_stream_t stream) {
+  MoePlan pl;
+  if (mode != HQ_MOE_GROUPED && mode != HQ_MOE_INDEXED) return HQ_ERR_INVALID_ARG;
+  if (I < 1 || (I % (TILE_N / 2)) != 0 || I > (1 << 29)) return HQ_ERR_INVALID_ARG;
+  const int N = 2 * I;
+  const hq_status ps = plan_moe(desc, T, topk, E, N, K, 0, &pl);
+  if (ps != HQ_OK) return ps;
+  pl.L.gated = 1;  // weights from hq_pack_weights_gated; the epilogue writes silu(gate) * up
+  if (T == 0) return HQ_OK;
+  if (!packed_w || !a || !out_bf16) return HQ_ERR_INVALID_ARG;
+  if (!aligned16(packed_w) || !aligned16(a) || !aligned16(out_bf16)) return HQ_ERR_INVALID_ARG;
+  const bool routed = expert_offsets && perm;
+  if (!routed && (expert_offsets || perm || !topk_ids)) return HQ_ERR_INVALID_ARG;
+  if (a_scales) {
+    if (pl.afmt == A_BF16 || ((uintptr_t)a_scales & 3u)) return HQ_ERR_INVALID_ARG;
+    if (pl.afmt == A_NVFP4 && !a_global) return HQ_ERR_INVALID_ARG;
+  }
+  MoeWs w;
+  const size_t need = moe_ws(pl, mode, E, K, N, 0, true, (uint8_t *)workspace, &w);
+  if (!workspace || ws_bytes < need || !aligned16(workspace)) return HQ_ERR_WORKSPACE;
+  if (!device_is_sm100()) return HQ_ERR_ARCH;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (!routed) {
+    const hq_status s = launch_moe_permute(T, topk, E, topk_ids, w.r_off, w.r_perm, w.r_inv, st);
+    if (s != HQ_OK) return s;
+    expert_offsets = w.r_off;
+    perm = w.r_perm;
+  }
+  return moe_run(pl, mode, T, topk, E, N, K, packed_w, a, a_scales, a_global, topk, nullptr, expert_offsets, perm,
+                 nullptr, 1.f, 0, out_bf16, w, st);
 }
 
 size_t hq_moe_masked_workspace_bytes(const hq_quant_desc *desc, int E, int slab, int N, int K, int expected_m) {

@@ -189,14 +189,12 @@ __device__ __forceinline__ void epilogue_segment(const Params &p, const TileInfo
     for (int i = 0; i < CW; ++i) {
       const int orow = __shfl_sync(0xffffffffu, orow_l, i);
       const float rs = __shfl_sync(0xffffffffu, rs_l, i);
-      if (c0 + i < ti.nvalid && n < p.N) {
-        // FP8: per-token x per-row scales; block-scaled kinds: global scales
-        float z = x[i];
-        if (p.row_scale) z *= rs;
-        z *= cs;
-        z *= gs;
-        p.out[(size_t)orow * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(z));
-      }
+      // FP8: per-token x per-row scales; block-scaled kinds: global scales
+      float z = x[i];
+      if (p.row_scale) z *= rs;
+      z *= cs;
+      z *= gs;
+      tc::put_out(p, orow, n, z, c0 + i < ti.nvalid && n < p.N);
     }
   };
 #pragma unroll 1
@@ -714,6 +712,7 @@ hq_status launch_bs_gemm(const Layout &L, const void *packed, int E, const void 
   p.N = L.N; p.K = L.K; p.NT = L.NT; p.G = L.G; p.group = L.group;
   p.KB = L.K / kstage;  // iterations (stages) per tile
   p.a_global = a_global;
+  p.gated = L.gated;
   p.M = M;
   p.moe = moe;
   p.E = E;

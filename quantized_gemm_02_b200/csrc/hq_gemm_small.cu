@@ -161,7 +161,15 @@ template <int WF>
 __device__ __forceinline__ void decode_bf16(const uint8_t *wpk, const uint8_t *sc, const uint8_t *zp, int r,
                                             int kbase, int g0, int gshift, uint32_t (&rg)[32]) {
   using TR = Traits<WF>;
-  if constexpr (TR::wbits == 4) {
+  if constexpr (fmt_lowbit(WF)) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int gt = ((kbase + 32 * h) >> gshift) - g0;
+      uint32_t s2, z2;
+      tc::lowbit_scale_zero<WF>(sc, zp, gt, r, s2, z2);
+      tc::decode_half_lowbit<WF>(wpk, s2, z2, r, h, rg + 16 * h);
+    }
+  } else if constexpr (TR::wbits == 4) {
     uint32_t s2c = 0, z2c = 0;  // INT4 / UINT4: scale and zero point of the previous chunk
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
@@ -238,13 +246,11 @@ __device__ __forceinline__ void store_rows(const Params &p, const TileInfo &ti, 
   for (int m = 0; m < BNT; ++m) {
     const int orow = __shfl_sync(0xffffffffu, orow_l, m);
     const float rs = __shfl_sync(0xffffffffu, rs_l, m);
-    if (m < ti.nvalid && n < p.N) {
-      float z = x[m];
-      if (p.row_scale) z *= rs;
-      z *= cs;
-      z *= gs;
-      p.out[(size_t)orow * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(z));
-    }
+    float z = x[m];
+    if (p.row_scale) z *= rs;
+    z *= cs;
+    z *= gs;
+    tc::put_out(p, orow, n, z, m < ti.nvalid && n < p.N);
   }
 }
 
@@ -699,7 +705,14 @@ hq_status launch_dec_gemm(const Layout &L, const tc::Params &p, const void *a, i
     return HQ_ERR_CUDA;
   switch (L.fmt) {
     case W_INT4: return dec_launch_wf<W_INT4>(map, p, t, st);
+    case W_E0M3: return dec_launch_wf<W_INT4>(map, p, t, st);  // packed as INT4
     case W_MXINT4: return dec_launch_wf<W_MXINT4>(map, p, t, st);
+    case W_INT2: return dec_launch_wf<W_INT2>(map, p, t, st);
+    case W_UINT2: return dec_launch_wf<W_UINT2>(map, p, t, st);
+    case W_INT3: return dec_launch_wf<W_INT3>(map, p, t, st);
+    case W_UINT3: return dec_launch_wf<W_UINT3>(map, p, t, st);
+    case W_E2M3: return dec_launch_wf<W_E2M3>(map, p, t, st);
+    case W_E3M2: return dec_launch_wf<W_E3M2>(map, p, t, st);
     case W_UINT4: return dec_launch_wf<W_UINT4>(map, p, t, st);
     case W_MXFP4: return dec_launch_wf<W_MXFP4>(map, p, t, st);
     case W_NVFP4: return dec_launch_wf<W_NVFP4>(map, p, t, st);

@@ -48,12 +48,12 @@ constexpr int WARP_PRODUCER = 4, WARP_MMA = 5, WARP_DQ0 = 6, NDQ = 8;
 
 template <int WF>
 struct Traits {
-  static constexpr int wbits = (WF == W_FP8) ? 8 : 4;
+  static constexpr int wbits = fmt_bits(WF);
   static constexpr int unit = BM * TILE_K * wbits / 8;  // packed bytes per (tile, k-block)
-  static constexpr int sbytes = (WF == W_INT4 || WF == W_UINT4) ? 2 : 1;
+  static constexpr int sbytes = fmt_bf16_scales(WF) ? 2 : 1;
   static constexpr int max_groups_kb = (WF == W_NVFP4) ? 4 : 2;  // scale groups per k-block (upper bound)
   static constexpr bool has_scales = (WF != W_FP8);
-  static constexpr bool has_zero = (WF == W_UINT4);
+  static constexpr bool has_zero = fmt_zero(WF);
 };
 
 // F8: both operands E4M3 (kind::f8f6f4, weights copied into TMEM unchanged);
@@ -97,6 +97,7 @@ struct Params {
   int gshift;              // k >> gshift = scale group (31 for one group per row)
   const float *row_scale;  // per caller row (FP8 per-token) or null
   const float *a_global;   // NVFP4 activation global scale or null
+  int gated;               // fused SiLU-and-mul: out[row, n / 2] = silu(gate) * up (packed rows 2j, 2j + 1)
   int M;                   // dense rows
   int moe, E;
   const int32_t *offsets, *perm;
@@ -220,6 +221,27 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// ---- output ---------------------------------------------------------------------
+// silu(g) * u in fp32 (CUDA expf, IEEE division), as hq_silu_and_mul computes it.
+__device__ __forceinline__ float silu_mul(float g, float u) {
+  return __fmul_rn(__fdiv_rn(g, __fadd_rn(1.f, expf(-g))), u);
+}
+
+// One scaled output value of weight row n for output row `orow`.  Plain: bf16
+// at column n.  Gated (gate-up weights packed gate/up side by side): lanes of
+// rows 2j and 2j + 1 exchange their values and the even lane writes
+// silu(gate) * up at column n / 2 of an N / 2-wide row.  All 32 lanes of the
+// warp call it together (consecutive lanes = consecutive weight rows).
+__device__ __forceinline__ void put_out(const Params &p, int orow, int n, float z, bool ok) {
+  if (!p.gated) {
+    if (ok) p.out[(size_t)orow * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(z));
+    return;
+  }
+  const float u = __shfl_xor_sync(0xffffffffu, z, 1);
+  if (ok && !(n & 1))
+    p.out[(size_t)orow * (p.N >> 1) + (n >> 1)] = __bfloat16_as_ushort(__float2bfloat16_rn(silu_mul(z, u)));
+}
+
 // ---- bf16 pair arithmetic and decoders ---------------------------------------
 __device__ __forceinline__ uint32_t bsub2(uint32_t a, uint32_t b) {
   __nv_bfloat162 r = __hsub2(*reinterpret_cast<__nv_bfloat162 *>(&a), *reinterpret_cast<__nv_bfloat162 *>(&b));
@@ -244,6 +266,61 @@ __device__ __forceinline__ uint32_t e2m1_pair(uint32_t x) {
 // E4M3 pair (codes at bits 0..7 and 16..23) -> bf16 pair carrying value * 2^-120
 __device__ __forceinline__ uint32_t e4m3_pair(uint32_t x) {
   return ((x & 0x007F007Fu) << 4) | ((x & 0x00800080u) << 8);
+}
+
+// Low-bit units (2-, 3- and 6-bit codes; planes as in hq_internal.cuh): the
+// 32 k of half h (k 32h .. 32h + 31 of the 64-k block) of weight row r as 16
+// bf16 pairs in k order (pair q = k 32h + 2q, 32h + 2q + 1).  Integer codes:
+// ((u | 128) - (128 + z)) * s, the subtraction exact and the product the
+// one rounding; MXFP6: the code's exponent and mantissa bits placed in the
+// bf16 fields (the value times 2^-126 for E2M3, 2^-124 for E3M2, exact for
+// subnormal codes too), scaled back, then by the E8M0 scale s2.
+template <int WF>
+__device__ __forceinline__ void decode_half_lowbit(const uint8_t *unit, uint32_t s2, uint32_t z2, int r, int h,
+                                                   uint32_t *rg) {
+  constexpr int b = fmt_bits(WF);
+  const uint2 v2 = *reinterpret_cast<const uint2 *>(unit + plane2_off(WF) + r * 16 + h * 8);
+  const uint32_t w2[2] = {v2.x, v2.y};
+  uint32_t c[16];
+#pragma unroll
+  for (int a = 0; a < 2; ++a)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) c[8 * a + i] = (w2[a] >> (2 * i)) & 0x00030003u;
+  if constexpr (b == 3) {
+    const uint32_t w1 = *reinterpret_cast<const uint32_t *>(unit + plane1_off(WF) + r * 8 + h * 4);
+#pragma unroll
+    for (int q = 0; q < 16; ++q) c[q] |= ((w1 >> q) & 0x00010001u) << 2;
+  }
+  if constexpr (b == 6) {
+    const uint4 v4 = *reinterpret_cast<const uint4 *>(unit + h * (BM * 16) + r * 16);
+    const uint32_t w4[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+    for (int q = 0; q < 16; ++q) c[q] = (c[q] << 4) | ((w4[q >> 2] >> (4 * (q & 3))) & 0x000F000Fu);
+  }
+#pragma unroll
+  for (int q = 0; q < 16; ++q) {
+    if constexpr (WF == W_E2M3) {
+      const uint32_t x = ((c[q] & 0x001F001Fu) << 4) | ((c[q] & 0x00200020u) << 10);
+      rg[q] = bmul2(bmul2(x, 0x7E807E80u), s2);  // x 2^126
+    } else if constexpr (WF == W_E3M2) {
+      const uint32_t x = ((c[q] & 0x001F001Fu) << 5) | ((c[q] & 0x00200020u) << 10);
+      rg[q] = bmul2(bmul2(x, 0x7D807D80u), s2);  // x 2^124
+    } else {
+      rg[q] = bmul2(bsub2(c[q] | 0x43004300u, z2), s2);
+    }
+  }
+}
+
+// Scale and zero-point pairs of a low-bit row's group: bf16 scale (integer
+// codes) or the E8M0 power of two (MXFP6); zero point 128 + z (unsigned
+// codes) or 128 + 2^(b-1) (signed codes, stored biased).
+template <int WF>
+__device__ __forceinline__ void lowbit_scale_zero(const uint8_t *sc, const uint8_t *zp, int gt, int r, uint32_t &s2,
+                                                  uint32_t &z2) {
+  if constexpr (fmt_bf16_scales(WF)) s2 = bcast16(reinterpret_cast<const uint16_t *>(sc)[gt * BM + r]);
+  else s2 = bcast16(e8m0_code_to_bf16(sc[gt * BM + r]));
+  if constexpr (fmt_zero(WF)) z2 = bcast16(0x4300u + zp[gt * BM + r]);
+  else z2 = bcast16(0x4300u + (1u << (fmt_bits(WF) - 1)));
 }
 
 // ---- the kernel ----------------------------------------------------------------
@@ -544,7 +621,11 @@ __global__ void __launch_bounds__(THREADS, (BNT <= 64 ? 2 : 1)) tc_gemm_kernel(c
           tmem_st8(t_row + (uint32_t)(a * C::A_COLS + half * 8), rg8);
         } else {
           uint32_t rg[16];
-          if constexpr (TR::wbits == 4) {
+          if constexpr (fmt_lowbit(WF)) {
+            uint32_t s2, z2;
+            lowbit_scale_zero<WF>(sc, zp, gt, r, s2, z2);
+            decode_half_lowbit<WF>(wpk_j, s2, z2, r, half, rg);
+          } else if constexpr (TR::wbits == 4) {
             const uint4 v = *reinterpret_cast<const uint4 *>(wpk_j + half * (BM * 16) + r * 16);
             const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
             if constexpr (WF == W_INT4 || WF == W_UINT4 || WF == W_MXINT4) {
@@ -687,13 +768,11 @@ __global__ void __launch_bounds__(THREADS, (BNT <= 64 ? 2 : 1)) tc_gemm_kernel(c
           for (int i = 0; i < 16; ++i) {
             const int orow = __shfl_sync(0xffffffffu, orow_l, i);
             const float rs = __shfl_sync(0xffffffffu, rs_l, i);
-            if (c0 + i < ti.nvalid && n < p.N) {
-              float x = v[i];
-              if (p.row_scale) x *= rs;
-              x *= cs;
-              x *= gs;
-              p.out[(size_t)orow * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(x));
-            }
+            float x = v[i];
+            if (p.row_scale) x *= rs;
+            x *= cs;
+            x *= gs;
+            put_out(p, orow, n, x, c0 + i < ti.nvalid && n < p.N);
           }
         }
       }
@@ -752,15 +831,28 @@ __global__ void __launch_bounds__(THREADS, (BNT <= 64 ? 2 : 1)) tc_gemm_kernel(c
       const int orow = p.moe ? p.perm[pos] : pos;
       const float rs = p.row_scale ? p.row_scale[p.moe ? orow / p.a_div : pos] : 1.f;
       const float a4[4] = {acc.x, acc.y, acc.z, acc.w};
+      float xs[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int n = ti.wt * BM + r4 * 4 + j;
+        xs[j] = 0.f;
         if (n < p.N) {
           float x = a4[j];
           if (p.row_scale) x *= rs;
           if (WF == W_FP8) x *= reinterpret_cast<const float *>(eb + p.c_off)[n];
           x *= gs;
-          p.out[(size_t)orow * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(x));
+          xs[j] = x;
+          if (!p.gated) p.out[(size_t)orow * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(x));
+        }
+      }
+      if (p.gated) {
+        // the thread's four rows are two gate/up pairs
+#pragma unroll
+        for (int j = 0; j < 4; j += 2) {
+          const int n = ti.wt * BM + r4 * 4 + j;
+          if (n < p.N)
+            p.out[(size_t)orow * (p.N >> 1) + (n >> 1)] =
+                __bfloat16_as_ushort(__float2bfloat16_rn(silu_mul(xs[j], xs[j + 1])));
         }
       }
     }
@@ -913,6 +1005,7 @@ hq_status launch_tc_gemm(const Layout &L, const void *packed, const void *a_bf16
   p.gshift = ((L.group & (L.group - 1)) == 0) ? __builtin_ctz((unsigned)L.group) : 31;
   p.row_scale = row_scale;
   p.a_global = a_global;
+  p.gated = L.gated;
   p.M = M;
   p.moe = moe;
   p.E = E;
@@ -942,7 +1035,14 @@ hq_status launch_tc_gemm(const Layout &L, const void *packed, const void *a_bf16
   if (gather && e4m3_act) return HQ_ERR_UNSUPPORTED;
   switch (L.fmt) {
     case W_INT4: return tc_launch_wf<W_INT4>(map, p, t, st);
+    case W_E0M3: return tc_launch_wf<W_INT4>(map, p, t, st);  // packed as INT4
     case W_MXINT4: return tc_launch_wf<W_MXINT4>(map, p, t, st);
+    case W_INT2: return tc_launch_wf<W_INT2>(map, p, t, st);
+    case W_UINT2: return tc_launch_wf<W_UINT2>(map, p, t, st);
+    case W_INT3: return tc_launch_wf<W_INT3>(map, p, t, st);
+    case W_UINT3: return tc_launch_wf<W_UINT3>(map, p, t, st);
+    case W_E2M3: return tc_launch_wf<W_E2M3>(map, p, t, st);
+    case W_E3M2: return tc_launch_wf<W_E3M2>(map, p, t, st);
     case W_UINT4: return tc_launch_wf<W_UINT4>(map, p, t, st);
     case W_MXFP4: return tc_launch_wf<W_MXFP4>(map, p, t, st);
     case W_NVFP4: return tc_launch_wf<W_NVFP4>(map, p, t, st);

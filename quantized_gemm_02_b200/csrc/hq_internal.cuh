@@ -35,8 +35,36 @@ namespace hq {
 
 // Internal weight formats.
 // W_MXINT4: INT4 codes with an E8M0 scale per 32 along K (the MX layout with
-// integer elements).
-enum WFmt : int { W_INT4 = 0, W_UINT4 = 1, W_MXFP4 = 2, W_NVFP4 = 3, W_FP8 = 4, W_MXINT4 = 5, W_NFMT = 6 };
+// integer elements).  Low-bit WnA16 widths: W_INT2 / W_INT3 (signed, stored
+// biased like INT4), W_UINT2 / W_UINT3 (with zero points), W_E2M3 / W_E3M2
+// (MXFP6, E8M0 per 32).  W_E0M3 (float4e0m3, the zero-exponent view of
+// symmetric INT4) is converted by the repack into the INT4 layout; the GEMM
+// kernels see INT4.
+enum WFmt : int {
+  W_INT4 = 0, W_UINT4 = 1, W_MXFP4 = 2, W_NVFP4 = 3, W_FP8 = 4, W_MXINT4 = 5,
+  W_INT2 = 6, W_UINT2 = 7, W_INT3 = 8, W_UINT3 = 9, W_E2M3 = 10, W_E3M2 = 11, W_E0M3 = 12, W_NFMT = 13
+};
+
+// Bits per stored weight code of a format.
+__host__ __device__ constexpr int fmt_bits(int fmt) {
+  return fmt == W_FP8 ? 8 : (fmt == W_INT2 || fmt == W_UINT2) ? 2 : (fmt == W_INT3 || fmt == W_UINT3) ? 3
+         : (fmt == W_E2M3 || fmt == W_E3M2) ? 6 : 4;
+}
+__host__ __device__ constexpr bool fmt_lowbit(int fmt) { return fmt >= W_INT2 && fmt <= W_E3M2; }
+__host__ __device__ constexpr bool fmt_zero(int fmt) { return fmt == W_UINT4 || fmt == W_UINT2 || fmt == W_UINT3; }
+__host__ __device__ constexpr bool fmt_bf16_scales(int fmt) {
+  return fmt == W_INT4 || fmt == W_UINT4 || fmt == W_INT2 || fmt == W_UINT2 || fmt == W_INT3 || fmt == W_UINT3 ||
+         fmt == W_E0M3;
+}
+// Unit planes of the low-bit layouts (byte offsets inside a 128-row x 64-k
+// unit): a 4-bit plane (the INT4 unit's order, 4 KiB; 6-bit codes' low
+// nibbles), a 2-bit plane ([128 rows][16 B]: word j of a row holds k
+// 16j..16j+15, even k in bits 0..15 and odd k in bits 16..31, two bits
+// each; the low two bits of 2- and 3-bit codes, the high two of 6-bit
+// ones) and a 1-bit plane ([128 rows][8 B]: word j holds k 32j..32j+31,
+// even k in bits 0..15, odd in 16..31; the high bit of 3-bit codes).
+__host__ __device__ constexpr int plane2_off(int fmt) { return (fmt == W_E2M3 || fmt == W_E3M2) ? 4096 : 0; }
+__host__ __device__ constexpr int plane1_off(int fmt) { return (fmt == W_INT3 || fmt == W_UINT3) ? 2048 : 0; }
 // Internal activation formats.
 enum AFmt : int { A_BF16 = 0, A_FP8 = 1, A_MXFP8 = 2, A_NVFP4 = 3 };
 
@@ -50,12 +78,28 @@ enum { BS_NONE = 0, BS_MX = 1, BS_NV = 2, BS_F8 = 3 };
 struct Layout {
   int fmt;
   int bs;                      // BS_*: block-scaled MMA layout, or the dequantisation layout
+  int gated;                   // gate-up weights for the fused SiLU-and-mul epilogue (see std_row)
   int N, K, NT, KB, G, group;  // group = k per scale group (K for per-channel)
   int wbits;                   // 4 or 8
   int sbytes;                  // bytes per scale element (per-group scales)
   size_t w_bytes, s_bytes, z_bytes, c_bytes, g_bytes;  // per expert
   size_t w_off, s_off, z_off, c_off, g_off, stride;     // offsets inside an expert region
   __host__ __device__ size_t unit_bytes() const { return (size_t)TILE_N * TILE_K * wbits / 8; }
+  // Gate-up weights (N = 2I rows: gate rows 0..I-1, then up rows) are packed
+  // with the gate and the up row of output column j side by side: rows 2i
+  // and 2i + 1 of 128-row tile t hold gate and up rows of column 64 t + i,
+  // so one tile's epilogue has both values of 64 columns.  std_row maps a
+  // packed row to its standard-format row, packed_row the other way.
+  __host__ __device__ int std_row(int p) const {
+    if (!gated) return p;
+    const int i = p % TILE_N;
+    return (p / TILE_N) * (TILE_N / 2) + (i >> 1) + ((i & 1) ? N / 2 : 0);
+  }
+  __host__ __device__ int packed_row(int r) const {
+    if (!gated) return r;
+    const int h = r >= N / 2 ? 1 : 0, j = h ? r - N / 2 : r;
+    return (j / (TILE_N / 2)) * TILE_N + (j % (TILE_N / 2)) * 2 + h;
+  }
   __host__ __device__ int chunks() const { return wbits == 4 ? 2 : 4; }
   // code bytes per weight row of the block-scaled / FP8 layouts
   __host__ __device__ size_t bs_row_bytes() const { return bs == BS_F8 ? (size_t)K : (size_t)K / 2; }
@@ -99,6 +143,24 @@ inline bool weight_format(const hq_quant_desc *d, int *fmt) {
     case HQ_E4M3:
       if (d->w_scale_dtype != HQ_FP32 || d->w_group != 0 || d->w_has_zero || d->w_has_global) return false;
       *fmt = W_FP8;
+      return true;
+    case HQ_INT2:
+    case HQ_INT3:
+    case HQ_E0M3:
+      if (d->w_scale_dtype != HQ_BF16 || d->w_has_zero || d->w_has_global) return false;
+      if (!(d->w_group == 0 || d->w_group == 32 || d->w_group == 64 || d->w_group == 128)) return false;
+      *fmt = d->w_dtype == HQ_INT2 ? W_INT2 : d->w_dtype == HQ_INT3 ? W_INT3 : W_E0M3;
+      return true;
+    case HQ_UINT2:
+    case HQ_UINT3:
+      if (d->w_scale_dtype != HQ_BF16 || !d->w_has_zero || d->w_has_global) return false;
+      if (!(d->w_group == 32 || d->w_group == 64 || d->w_group == 128)) return false;
+      *fmt = d->w_dtype == HQ_UINT2 ? W_UINT2 : W_UINT3;
+      return true;
+    case HQ_E2M3:
+    case HQ_E3M2:
+      if (d->w_scale_dtype != HQ_E8M0 || d->w_group != 32 || d->w_has_zero || d->w_has_global) return false;
+      *fmt = d->w_dtype == HQ_E2M3 ? W_E2M3 : W_E3M2;
       return true;
     default:
       return false;
@@ -149,11 +211,11 @@ inline Layout make_layout(int fmt, int group, int N, int K, int bs = BS_NONE) {
   L.KB = K / TILE_K;
   L.group = (group == 0) ? K : group;
   L.G = K / L.group;
-  L.wbits = (fmt == W_FP8) ? 8 : 4;
-  L.sbytes = (fmt == W_INT4 || fmt == W_UINT4) ? 2 : 1;
+  L.wbits = fmt_bits(fmt);
+  L.sbytes = fmt_bf16_scales(fmt) ? 2 : 1;
   L.w_bytes = (size_t)L.NT * L.KB * L.unit_bytes();
   L.s_bytes = (fmt == W_FP8) ? 0 : (size_t)L.NT * L.G * TILE_N * L.sbytes;
-  L.z_bytes = (fmt == W_UINT4) ? (size_t)L.NT * L.G * TILE_N : 0;
+  L.z_bytes = fmt_zero(fmt) ? (size_t)L.NT * L.G * TILE_N : 0;
   L.c_bytes = (fmt == W_FP8) ? (size_t)L.NT * TILE_N * 4 : 0;
   L.g_bytes = (fmt == W_NVFP4) ? 16 : 0;
   if (bs != BS_NONE) {

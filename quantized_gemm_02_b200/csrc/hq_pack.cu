@@ -32,7 +32,7 @@ __host__ __device__ inline FragPos frag_pos(int wbits, int i_row, int kk) {
 // Raw code (nibble or byte) of the standard-format element (r, k).
 __device__ inline uint32_t std_code(int fmt, const uint8_t *codes, int K, int r, int k) {
   if (fmt == W_FP8) return codes[(size_t)r * K + k];
-  if (fmt == W_MXFP4 || fmt == W_NVFP4) {
+  if (fmt == W_MXFP4 || fmt == W_NVFP4 || fmt == W_E0M3) {
     const uint8_t b = codes[(size_t)r * (K / 2) + (k >> 1)];
     return (k & 1) ? (b >> 4) : (b & 15);
   }
@@ -65,9 +65,11 @@ __global__ void pack_weights_kernel(Layout L, int E, const uint8_t *codes, uint8
       const int k = kb * TILE_K + kk;
       uint32_t v = 0;
       if (r < L.N) {
-        v = std_code(L.fmt, ce, L.K, r, k);
+        v = std_code(L.fmt, ce, L.K, L.std_row(r), k);
         if (L.fmt == W_INT4 || L.fmt == W_MXINT4) v ^= 8u;  // two's complement -> biased (q + 8)
-      } else if (L.fmt == W_INT4 || L.fmt == W_MXINT4) {
+        // float4e0m3 (sign, magnitude m) is the symmetric integer +-m: biased 8 +- m
+        if (L.fmt == W_E0M3) v = (v & 8u) ? 8u - (v & 7u) : 8u + v;
+      } else if (L.fmt == W_INT4 || L.fmt == W_MXINT4 || L.fmt == W_E0M3) {
         v = 8u;  // padded rows decode to zero
       }
       word |= v << (slot * L.wbits);
@@ -89,29 +91,32 @@ __global__ void pack_side_kernel(Layout L, int E, const uint8_t *scales, const u
     const int nt = r / TILE_N, i = r % TILE_N;
     uint8_t *base = packed + (size_t)e * L.stride;
     const size_t dst = ((size_t)nt * L.G + gi) * TILE_N + i;
+    const int sr = L.std_row(r);  // standard-format row of packed row r
     if (L.fmt == W_FP8) {
       if (gi == 0) {
         float c = 0.f;
-        if (r < L.N) c = reinterpret_cast<const float *>(scales)[(size_t)e * L.N + r];
+        if (r < L.N) c = reinterpret_cast<const float *>(scales)[(size_t)e * L.N + sr];
         reinterpret_cast<float *>(base + L.c_off)[(size_t)nt * TILE_N + i] = c;
       }
     } else if (L.sbytes == 2) {
       uint16_t s = 0;
-      if (r < L.N) s = reinterpret_cast<const uint16_t *>(scales)[((size_t)e * L.N + r) * L.G + gi];
+      if (r < L.N) s = reinterpret_cast<const uint16_t *>(scales)[((size_t)e * L.N + sr) * L.G + gi];
       reinterpret_cast<uint16_t *>(base + L.s_off)[dst] = s;
     } else {
       uint8_t s = 0;
-      if (r < L.N) s = scales[((size_t)e * L.N + r) * L.G + gi];
+      if (r < L.N) s = scales[((size_t)e * L.N + sr) * L.G + gi];
       (base + L.s_off)[dst] = s;
     }
     if (L.fmt == W_UINT4) {
       uint8_t z = 0;
       if (r < L.N) {
         const int zw = (L.G + 7) / 8;
-        const uint32_t w = reinterpret_cast<const uint32_t *>(zeros)[((size_t)e * L.N + r) * zw + gi / 8];
+        const uint32_t w = reinterpret_cast<const uint32_t *>(zeros)[((size_t)e * L.N + sr) * zw + gi / 8];
         z = (uint8_t)((w >> (4 * (gi % 8))) & 15u);
       }
       (base + L.z_off)[dst] = z;
+    } else if (L.fmt == W_UINT2 || L.fmt == W_UINT3) {
+      (base + L.z_off)[dst] = (r < L.N) ? zeros[((size_t)e * L.N + sr) * L.G + gi] : (uint8_t)0;
     }
     if (L.fmt == W_NVFP4 && r == 0 && gi == 0) {
       reinterpret_cast<float *>(base + L.g_off)[0] = global_scale[e];
@@ -122,7 +127,7 @@ __global__ void pack_side_kernel(Layout L, int E, const uint8_t *scales, const u
 // Inverse: one thread per standard-format code word/byte.
 __global__ void unpack_codes_kernel(Layout L, int E, const uint8_t *packed, uint8_t *codes) {
   // elements per standard-format storage unit
-  const int per = (L.fmt == W_FP8) ? 1 : (L.fmt == W_MXFP4 || L.fmt == W_NVFP4) ? 2 : 8;
+  const int per = (L.fmt == W_FP8) ? 1 : (L.fmt == W_MXFP4 || L.fmt == W_NVFP4 || L.fmt == W_E0M3) ? 2 : 8;
   const size_t units_per_row = (size_t)L.K / per;
   const size_t total = (size_t)E * L.N * units_per_row;
   const size_t words_per_unit = L.unit_bytes() / 4;
@@ -133,7 +138,8 @@ __global__ void unpack_codes_kernel(Layout L, int E, const uint8_t *packed, uint
     const int r = (int)(rem / units_per_row);
     const int u = (int)(rem % units_per_row);
     const uint32_t *pw = reinterpret_cast<const uint32_t *>(packed + (size_t)e * L.stride + L.w_off);
-    const int nt = r / TILE_N, i_row = r % TILE_N;
+    const int pr = L.packed_row(r);
+    const int nt = pr / TILE_N, i_row = pr % TILE_N;
     uint32_t out = 0;
     for (int j = 0; j < per; ++j) {
       const int k = u * per + j;
@@ -142,6 +148,7 @@ __global__ void unpack_codes_kernel(Layout L, int E, const uint8_t *packed, uint
       const size_t unit = (size_t)nt * L.KB + kb;
       uint32_t v = (pw[unit * words_per_unit + fp.word] >> fp.shift) & ((1u << L.wbits) - 1u);
       if (L.fmt == W_INT4 || L.fmt == W_MXINT4) v ^= 8u;
+      if (L.fmt == W_E0M3) v = v >= 8u ? v - 8u : (8u | (8u - v));  // back to sign and magnitude (0 is +0)
       out |= v << (j * L.wbits);
     }
     if (per == 8) reinterpret_cast<uint32_t *>(codes)[idx] = out;
@@ -157,7 +164,8 @@ __global__ void unpack_side_kernel(Layout L, int E, const uint8_t *packed, uint8
     const int e = (int)(idx / ((size_t)L.N * L.G));
     const int rem = (int)(idx % ((size_t)L.N * L.G));
     const int r = rem / L.G, gi = rem % L.G;
-    const int nt = r / TILE_N, i = r % TILE_N;
+    const int pr = L.packed_row(r);
+    const int nt = pr / TILE_N, i = pr % TILE_N;
     const uint8_t *base = packed + (size_t)e * L.stride;
     const size_t src = ((size_t)nt * L.G + gi) * TILE_N + i;
     if (L.fmt == W_FP8) {
@@ -169,6 +177,7 @@ __global__ void unpack_side_kernel(Layout L, int E, const uint8_t *packed, uint8
     } else {
       scales[idx] = (base + L.s_off)[src];
     }
+    if ((L.fmt == W_UINT2 || L.fmt == W_UINT3)) zeros[((size_t)e * L.N + r) * L.G + gi] = (base + L.z_off)[src];
     if (L.fmt == W_UINT4 && (gi % 8) == 0) {
       const int zw = (L.G + 7) / 8;
       uint32_t w = 0;
@@ -202,7 +211,7 @@ __global__ void pack_bs_codes_kernel(Layout L, int E, const uint8_t *codes, uint
     const int r = (int)(rem / row16);
     const size_t c = rem % row16;
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (r < L.N) v = reinterpret_cast<const uint4 *>(codes + ((size_t)e * L.N + r) * rb)[c];
+    if (r < L.N) v = reinterpret_cast<const uint4 *>(codes + ((size_t)e * L.N + L.std_row(r)) * rb)[c];
     const int cb = L.bs_chunk_bytes();
     *reinterpret_cast<uint4 *>(packed + (size_t)e * L.stride + L.w_off +
                                L.bs_chunk_off(r, (int)(c * 16 / cb)) + (c * 16) % cb) = v;
@@ -224,10 +233,10 @@ __global__ void pack_bs_side_kernel(Layout L, int E, const uint8_t *scales, cons
     uint8_t *base = packed + (size_t)e * L.stride;
     if (L.bs == BS_F8) {
       reinterpret_cast<float *>(base + L.c_off)[r] =
-          (r < L.N) ? reinterpret_cast<const float *>(scales)[(size_t)e * L.N + r] : 0.f;
+          (r < L.N) ? reinterpret_cast<const float *>(scales)[(size_t)e * L.N + L.std_row(r)] : 0.f;
       continue;
     }
-    const uint8_t sv = (r < L.N) ? scales[((size_t)e * L.N + r) * L.G + gi] : (uint8_t)0;
+    const uint8_t sv = (r < L.N) ? scales[((size_t)e * L.N + L.std_row(r)) * L.G + gi] : (uint8_t)0;
     base[L.s_off + ((size_t)nt * (L.G / 4) + gi / 4) * 512 + bs_sf_offset(i, gi & 3)] = sv;
     if (L.fmt == W_NVFP4 && r == 0 && gi == 0) reinterpret_cast<float *>(base + L.g_off)[0] = global_scale[e];
   }
@@ -248,21 +257,133 @@ __global__ void unpack_bs_kernel(Layout L, int E, const uint8_t *packed, uint8_t
       const size_t c = rem % row16;
       const int cb = L.bs_chunk_bytes();
       reinterpret_cast<uint4 *>(codes + ((size_t)e * L.N + r) * rb)[c] = *reinterpret_cast<const uint4 *>(
-          packed + (size_t)e * L.stride + L.w_off + L.bs_chunk_off(r, (int)(c * 16 / cb)) + (c * 16) % cb);
+          packed + (size_t)e * L.stride + L.w_off + L.bs_chunk_off(L.packed_row(r), (int)(c * 16 / cb)) +
+          (c * 16) % cb);
     } else {
       const size_t j = idx - total_c;
       const int e = (int)(j / ((size_t)L.N * L.G));
       const int rem = (int)(j % ((size_t)L.N * L.G));
       const int r = rem / L.G, gi = rem % L.G;
-      const int nt = r / TILE_N, i = r % TILE_N;
+      const int pr = L.packed_row(r);
+      const int nt = pr / TILE_N, i = pr % TILE_N;
       const uint8_t *base = packed + (size_t)e * L.stride;
       if (L.bs == BS_F8) {
-        reinterpret_cast<float *>(scales)[(size_t)e * L.N + r] = reinterpret_cast<const float *>(base + L.c_off)[r];
+        reinterpret_cast<float *>(scales)[(size_t)e * L.N + r] = reinterpret_cast<const float *>(base + L.c_off)[pr];
         continue;
       }
       scales[j] = base[L.s_off + ((size_t)nt * (L.G / 4) + gi / 4) * 512 + bs_sf_offset(i, gi & 3)];
       if (L.fmt == W_NVFP4 && r == 0 && gi == 0) global_scale[e] = reinterpret_cast<const float *>(base + L.g_off)[0];
     }
+  }
+}
+
+// ---- low-bit layouts (2-, 3- and 6-bit codes) ---------------------------------------
+// Code k of row r of a b-bit little-endian code stream (row_bytes per row).
+__device__ inline uint32_t stream_code(const uint8_t *codes, size_t row_bytes, int r, int k, int b) {
+  const uint8_t *row = codes + (size_t)r * row_bytes;
+  const int bit = b * k, byte = bit >> 3, off = bit & 7;
+  uint32_t v = row[byte];
+  if (off + b > 8) v |= (uint32_t)row[byte + 1] << 8;
+  return (v >> off) & ((1u << b) - 1u);
+}
+
+// Signed codes are stored biased (two's complement -> + 2^(b-1)), so every
+// integer format decodes as (u - z).
+__device__ inline bool lowbit_signed(int fmt) { return fmt == W_INT2 || fmt == W_INT3; }
+
+// The stored (biased) code of packed row p (of the tile order), k of the
+// matrix; padded rows decode to zero.
+__device__ inline uint32_t lowbit_stored(const Layout &L, const uint8_t *ce, size_t rb, int p, int k) {
+  const int b = L.wbits;
+  if (p >= L.N) return lowbit_signed(L.fmt) ? (1u << (b - 1)) : 0u;
+  uint32_t c = stream_code(ce, rb, L.std_row(p), k, b);
+  if (lowbit_signed(L.fmt)) c ^= 1u << (b - 1);
+  return c;
+}
+
+// One thread per packed 32-bit word of the planes (see plane2_off /
+// plane1_off in hq_internal.cuh).
+__global__ void pack_lowbit_kernel(Layout L, int E, const uint8_t *codes, uint8_t *packed) {
+  const int b = L.wbits;
+  const size_t rb = (size_t)L.K * b / 8;
+  const size_t wpu = L.unit_bytes() / 4;
+  const int p4w = (b == 6) ? 1024 : 0;  // words of the 4-bit plane
+  const size_t total = (size_t)E * L.NT * L.KB * wpu;
+  for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < total;
+       idx += (size_t)gridDim.x * blockDim.x) {
+    const int e = (int)(idx / ((size_t)L.NT * L.KB * wpu));
+    const size_t rem = idx % ((size_t)L.NT * L.KB * wpu);
+    const size_t unit = rem / wpu;
+    const int wi = (int)(rem % wpu);
+    const int nt = (int)(unit / L.KB), kb = (int)(unit % L.KB);
+    const uint8_t *ce = codes + (size_t)e * L.N * rb;
+    uint32_t word = 0;
+    if (wi < p4w) {
+      // low nibbles of 6-bit codes, in the INT4 unit order
+      const int chunk = wi / (TILE_N * 4), i_row = (wi / 4) % TILE_N, j = wi % 4;
+      for (int slot = 0; slot < 8; ++slot) {
+        const int kk = chunk * 32 + j * 8 + 2 * (slot & 3) + (slot >> 2);
+        word |= (lowbit_stored(L, ce, rb, nt * TILE_N + i_row, kb * TILE_K + kk) & 15u) << (4 * slot);
+      }
+    } else if (wi < p4w + 512) {
+      // 2-bit plane: low two bits (2-, 3-bit codes) or high two (6-bit)
+      const int w = wi - p4w, i_row = w / 4, j = w % 4;
+      const int sh = (b == 6) ? 4 : 0;
+      for (int p = 0; p < 16; ++p) {
+        const int kk = 16 * j + (p < 8 ? 2 * p : 2 * (p - 8) + 1);
+        word |= ((lowbit_stored(L, ce, rb, nt * TILE_N + i_row, kb * TILE_K + kk) >> sh) & 3u) << (2 * p);
+      }
+    } else {
+      // 1-bit plane: the high bit of 3-bit codes
+      const int w = wi - p4w - 512, i_row = w / 2, j = w % 2;
+      for (int p = 0; p < 32; ++p) {
+        const int kk = 32 * j + (p < 16 ? 2 * p : 2 * (p - 16) + 1);
+        word |= ((lowbit_stored(L, ce, rb, nt * TILE_N + i_row, kb * TILE_K + kk) >> 2) & 1u) << p;
+      }
+    }
+    reinterpret_cast<uint32_t *>(packed + (size_t)e * L.stride + L.w_off)[unit * wpu + wi] = word;
+  }
+}
+
+// Inverse: one thread per 8 codes of a standard row (b bytes of the stream).
+__global__ void unpack_lowbit_kernel(Layout L, int E, const uint8_t *packed, uint8_t *codes) {
+  const int b = L.wbits;
+  const size_t rb = (size_t)L.K * b / 8;
+  const size_t wpu = L.unit_bytes() / 4;
+  const int p4w = (b == 6) ? 1024 : 0;
+  const size_t per_row = (size_t)L.K / 8;
+  const size_t total = (size_t)E * L.N * per_row;
+  for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < total;
+       idx += (size_t)gridDim.x * blockDim.x) {
+    const int e = (int)(idx / ((size_t)L.N * per_row));
+    const size_t rem = idx % ((size_t)L.N * per_row);
+    const int r = (int)(rem / per_row), g8 = (int)(rem % per_row);
+    const int pr = L.packed_row(r);
+    const int nt = pr / TILE_N, i_row = pr % TILE_N;
+    const uint32_t *pw = reinterpret_cast<const uint32_t *>(packed + (size_t)e * L.stride + L.w_off);
+    uint64_t bitsacc = 0;
+    for (int q = 0; q < 8; ++q) {
+      const int k = g8 * 8 + q, kb = k / TILE_K, kk = k % TILE_K;
+      const uint32_t *u = pw + ((size_t)nt * L.KB + kb) * wpu;
+      uint32_t c = 0;
+      if (b == 6) {
+        const int ko = kk & 7, slot = (ko & 1) * 4 + (ko >> 1);
+        c = (u[((kk >> 5) * TILE_N + i_row) * 4 + ((kk & 31) >> 3)] >> (4 * slot)) & 15u;
+      }
+      {
+        const int ko = kk & 15, p = (ko & 1) ? 8 + (ko >> 1) : (ko >> 1);
+        const uint32_t f = (u[p4w + i_row * 4 + (kk >> 4)] >> (2 * p)) & 3u;
+        c |= (b == 6) ? (f << 4) : f;
+      }
+      if (b == 3) {
+        const int ko = kk & 31, p = (ko & 1) ? 16 + (ko >> 1) : (ko >> 1);
+        c |= ((u[p4w + 512 + i_row * 2 + (kk >> 5)] >> p) & 1u) << 2;
+      }
+      if (lowbit_signed(L.fmt)) c ^= 1u << (b - 1);
+      bitsacc |= (uint64_t)c << (b * q);
+    }
+    uint8_t *dst = codes + ((size_t)e * L.N + r) * rb + (size_t)g8 * b;
+    for (int i = 0; i < b; ++i) dst[i] = (uint8_t)(bitsacc >> (8 * i));
   }
 }
 
@@ -284,7 +405,10 @@ hq_status launch_pack(const Layout &L, int E, const void *codes, const void *sca
     return check_launch();
   }
   const size_t words = (size_t)E * L.NT * L.KB * (L.unit_bytes() / 4);
-  pack_weights_kernel<<<pack_grid(words, 256), 256, 0, st>>>(L, E, (const uint8_t *)codes, (uint8_t *)packed);
+  if (fmt_lowbit(L.fmt))
+    pack_lowbit_kernel<<<pack_grid(words, 256), 256, 0, st>>>(L, E, (const uint8_t *)codes, (uint8_t *)packed);
+  else
+    pack_weights_kernel<<<pack_grid(words, 256), 256, 0, st>>>(L, E, (const uint8_t *)codes, (uint8_t *)packed);
   const size_t side = (size_t)E * L.NT * TILE_N * L.G;
   pack_side_kernel<<<pack_grid(side, 256), 256, 0, st>>>(L, E, (const uint8_t *)scales, (const uint8_t *)zeros,
                                                         global_scale, (uint8_t *)packed);
@@ -299,9 +423,14 @@ hq_status launch_unpack(const Layout &L, int E, const void *packed, void *codes,
                                                          (uint8_t *)scales, global_scale);
     return check_launch();
   }
-  const int per = (L.fmt == W_FP8) ? 1 : (L.fmt == W_MXFP4 || L.fmt == W_NVFP4) ? 2 : 8;
-  const size_t n = (size_t)E * L.N * (L.K / per);
-  unpack_codes_kernel<<<pack_grid(n, 256), 256, 0, st>>>(L, E, (const uint8_t *)packed, (uint8_t *)codes);
+  if (fmt_lowbit(L.fmt)) {
+    const size_t n8 = (size_t)E * L.N * (L.K / 8);
+    unpack_lowbit_kernel<<<pack_grid(n8, 256), 256, 0, st>>>(L, E, (const uint8_t *)packed, (uint8_t *)codes);
+  } else {
+    const int per = (L.fmt == W_FP8) ? 1 : (L.fmt == W_MXFP4 || L.fmt == W_NVFP4 || L.fmt == W_E0M3) ? 2 : 8;
+    const size_t n = (size_t)E * L.N * (L.K / per);
+    unpack_codes_kernel<<<pack_grid(n, 256), 256, 0, st>>>(L, E, (const uint8_t *)packed, (uint8_t *)codes);
+  }
   const size_t side = (size_t)E * L.N * L.G;
   unpack_side_kernel<<<pack_grid(side, 256), 256, 0, st>>>(L, E, (const uint8_t *)packed, (uint8_t *)scales,
                                                           (uint8_t *)zeros, global_scale);

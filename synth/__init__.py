@@ -34,7 +34,8 @@ import numpy as np
 import torch
 
 __all__ = [
-    "generator", "bf16_normal", "random_bytes", "int4_weights", "mxint4_weights", "mxfp4_weights",
+    "generator", "bf16_normal", "random_bytes", "int4_weights", "lowbit_weights", "mxint4_weights",
+    "mxfp4_weights",
     "nvfp4_weights_random", "fp8_weights_random", "routing_softmax_topk", "routing_zipf",
     "pack_nibbles_i32", "pack_nibbles_u8", "to_np_bits",
 ]
@@ -117,6 +118,26 @@ def int4_weights(E: int, N: int, K: int, group: int, asym: bool, gen: torch.Gene
             keep = (1 << (4 * (G % 8))) - 1
             z[..., -1] &= keep
         zeros = z
+    return {"codes": codes, "scales": scales, "zeros": zeros}
+
+
+def lowbit_weights(E: int, N: int, K: int, bits: int, group: int, zero: bool, e8m0: bool, gen: torch.Generator,
+                   device: str = "cpu") -> dict:
+    """b-bit codes (b = 2, 3, 6, or 4 for float4e0m3) as the standard
+    little-endian bit stream: uniform random bytes are uniform codes.
+    Scales: bf16 |N(0, 0.02)| + 1e-3 per group, or (e8m0) E8M0 exponents
+    uniform over [-8, -4] per 32; zero points uint8 uniform in [0, 2^b)."""
+    codes = random_bytes((E, N, K * bits // 8), gen, device)
+    G = 1 if group == 0 else K // group
+    if e8m0:
+        scales = torch.randint(119, 124, (E, N, K // 32), generator=gen, dtype=torch.int32, device=device)
+        scales = scales.to(torch.uint8)
+    else:
+        scales = _scales_bf16((E, N, G), gen, device)
+    zeros = None
+    if zero:
+        zeros = torch.randint(0, 1 << bits, (E, N, G), generator=gen, dtype=torch.int32, device=device)
+        zeros = zeros.to(torch.uint8)
     return {"codes": codes, "scales": scales, "zeros": zeros}
 
 

@@ -32,7 +32,22 @@ WFORMATS = {
             dict(w_dtype="e4m3", w_group=0, w_scale="fp32")),
     "mxint4": (dict(w_dtype=2, w_group=32, w_scale_dtype=6, w_has_zero=0, w_has_global=0),
                dict(w_dtype="int4", w_group=32, w_scale="e8m0")),
+    "int2_g64": (dict(w_dtype=10, w_group=64, w_scale_dtype=0, w_has_zero=0, w_has_global=0),
+                 dict(w_dtype="int2", w_group=64, w_scale="bf16")),
+    "uint2_g32": (dict(w_dtype=11, w_group=32, w_scale_dtype=0, w_has_zero=1, w_has_global=0),
+                  dict(w_dtype="uint2", w_group=32, w_scale="bf16", w_zero=True)),
+    "int3_g128": (dict(w_dtype=12, w_group=128, w_scale_dtype=0, w_has_zero=0, w_has_global=0),
+                  dict(w_dtype="int3", w_group=128, w_scale="bf16")),
+    "uint3_g64": (dict(w_dtype=13, w_group=64, w_scale_dtype=0, w_has_zero=1, w_has_global=0),
+                  dict(w_dtype="uint3", w_group=64, w_scale="bf16", w_zero=True)),
+    "e2m3": (dict(w_dtype=14, w_group=32, w_scale_dtype=6, w_has_zero=0, w_has_global=0),
+             dict(w_dtype="e2m3", w_group=32, w_scale="e8m0")),
+    "e3m2": (dict(w_dtype=15, w_group=32, w_scale_dtype=6, w_has_zero=0, w_has_global=0),
+             dict(w_dtype="e3m2", w_group=32, w_scale="e8m0")),
+    "e0m3_g128": (dict(w_dtype=16, w_group=128, w_scale_dtype=0, w_has_zero=0, w_has_global=0),
+                  dict(w_dtype="e0m3", w_group=128, w_scale="bf16")),
 }
+LOWBIT = {"int2_g64": 2, "uint2_g32": 2, "int3_g128": 3, "uint3_g64": 3, "e2m3": 6, "e3m2": 6, "e0m3_g128": 4}
 AFORMATS = {"bf16": 0, "fp8": 5, "mxfp8": 8, "nvfp4": 9}
 
 
@@ -54,6 +69,10 @@ def make_weights(wname: str, E: int, N: int, K: int, seed: int = 0, device: str 
     if wname == "mxint4":
         w = synth.mxint4_weights(E, N, K, g, device=device)
         return {"codes": w["codes"], "scales": w["scales"], "zeros": None, "global": None}
+    if wname in LOWBIT:
+        w = synth.lowbit_weights(E, N, K, LOWBIT[wname], fields["w_group"], bool(fields["w_has_zero"]),
+                                 fields["w_scale_dtype"] == 6, g, device)
+        return {"codes": w["codes"], "scales": w["scales"], "zeros": w["zeros"], "global": None}
     if fields["w_dtype"] in (2, 3):
         w = synth.int4_weights(E, N, K, fields["w_group"], fields["w_dtype"] == 3, g, device)
         return {"codes": w["codes"], "scales": w["scales"], "zeros": w["zeros"], "global": None}

@@ -61,6 +61,7 @@ def test_gemm_bf16_acts_small(wname, M):
 @pytest.mark.parametrize("wname,aname", [
     ("mxfp4", "mxfp8"), ("nvfp4", "nvfp4"), ("fp8", "fp8"), ("int4_g128", "fp8"),
     ("uint4_g128", "mxfp8"), ("mxfp4", "nvfp4"), ("fp8", "mxfp8"), ("nvfp4", "fp8"), ("mxint4", "mxfp8"),
+    ("int3_g128", "fp8"), ("e2m3", "mxfp8"), ("uint2_g32", "nvfp4"), ("e0m3_g128", "fp8"),
 ])
 @pytest.mark.parametrize("M", [1, 16, 40])
 def test_gemm_quantised_acts_small(wname, aname, M):

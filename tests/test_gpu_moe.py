@@ -277,3 +277,75 @@ def test_silu_and_mul():
     got = out.cpu().float().numpy().astype(np.float64)
     tol = np.abs(ref) * 2.0 ** -8 + 1e-30
     assert np.all(np.abs(got - ref) <= tol), float(np.max(np.abs(got - ref) / tol))
+
+
+def _gated_pack(wname, aname, w, E, N2, K):
+    import quantized_gemm_02_b200 as hq
+    d = cdesc(wname, aname)
+    packed = torch.empty(hq.hq_packed_weights_bytes(d, E, N2, K), dtype=torch.uint8, device="cuda")
+    cu = {kk: (None if v is None else v.cuda()) for kk, v in w.items()}
+    hq.hq_pack_weights_gated(d, E, N2, K, cu["codes"], cu["scales"], cu["zeros"], cu["global"], packed)
+    return packed
+
+
+@pytest.mark.parametrize("wname,aname", [("uint4_g64", "bf16"), ("mxfp4", "bf16"), ("fp8", "bf16"),
+                                         ("mxfp4", "mxfp8"), ("nvfp4", "nvfp4"), ("fp8", "fp8")])
+def test_pack_unpack_gated_identity(wname, aname):
+    # the gated row order (gate and up rows side by side) round-trips
+    import quantized_gemm_02_b200 as hq
+    E, N2, K = 2, 256, 256
+    w = make_weights(wname, E, N2, K, seed=90)
+    packed = _gated_pack(wname, aname, w, E, N2, K)
+    plain = gpu_pack(wname, w, E, N2, K, aname)
+    assert not torch.equal(packed, plain)  # the row order differs
+    out = {kk: (None if v is None else torch.zeros_like(v, device="cuda")) for kk, v in w.items()}
+    hq.hq_unpack_weights_gated(cdesc(wname, aname), E, N2, K, packed, out["codes"], out["scales"], out["zeros"],
+                               out["global"])
+    torch.cuda.synchronize()
+    for kk, v in w.items():
+        if v is not None:
+            assert np.array_equal(np_bits(out[kk]), np_bits(v)), kk
+
+
+@pytest.mark.parametrize("wname,aname,T", [("mxfp4", "bf16", 5), ("mxfp4", "bf16", 300), ("int4_g128", "bf16", 40),
+                                           ("uint4_g64", "fp8", 300), ("mxfp4", "mxfp8", 37), ("mxfp4", "mxfp8", 300),
+                                           ("nvfp4", "nvfp4", 300), ("fp8", "fp8", 37), ("mxint4", "bf16", 23)])
+@pytest.mark.parametrize("mode", [0, 1])
+def test_moe_gate_up_with_fused_silu(wname, aname, T, mode):
+    # SiLU-and-mul in the gate-up epilogue against the oracle's
+    # silu_and_mul of its expert outputs.  Tolerance: the GEMM bound carried
+    # through silu(g) * u (|silu'| <= 1.1), plus one bf16 rounding (2^-8
+    # relative allows the fp32 steps too).  Decode, multi-stage (split and
+    # whole tiles) and block-scaled kernels, both modes.
+    import quantized_gemm_02_b200 as hq
+    E, k, I, K = 16, 4, 128, 256
+    N2 = 2 * I
+    g = synth.generator(95 + T)
+    x = synth.bf16_normal((T, K), g)
+    ids, wts = synth.routing_zipf(T, E, k, 1.2, g)
+    w = make_weights(wname, E, N2, K, seed=96)
+    packed = _gated_pack(wname, aname, w, E, N2, K)
+    d = cdesc(wname, aname)
+    wsb = hq.hq_moe_gated_workspace_bytes(mode, d, T, k, E, I, K)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+    out = torch.full((T * k, I), float("nan"), dtype=torch.bfloat16, device="cuda")
+    hq.hq_moe_gemm_gated(mode, d, T, k, E, I, K, packed, x.cuda(), None, None, ids.cuda(), None, None, out, ws, wsb)
+    torch.cuda.synchronize()
+    assert hq.hq_device_error() == 0
+    xb = np_bits(x)
+    if aname == "bf16":
+        A, row = O.decode_act("bf16", T, K, xb)
+    else:
+        q, s, og = oracle_quant(aname, xb)
+        A, row = O.decode_act(aname, T, K, q, s, og)
+    rows = np.repeat(np.arange(T), k)
+    Y, B = O.moe_expert_outputs(A[rows], ids.numpy(), oracle_decoder(wname, w, N2, K),
+                                None if row is None else row[rows])
+    ref = O.silu_and_mul(Y)
+    gg, uu = Y[:, :I], Y[:, I:]
+    sig = 1.0 / (1.0 + np.exp(-gg))
+    dsilu = np.abs(sig * (1.0 + gg * (1.0 - sig)))
+    tol = 4e-3 * (dsilu * B[:, :I] * np.abs(uu) + np.abs(gg * sig) * B[:, I:]) + 2.0 ** -8 * np.abs(ref) + 1e-5
+    got = out.float().cpu().numpy().astype(np.float64)
+    err = np.abs(got - ref)
+    assert np.all(err <= tol), float(np.max(err / tol))

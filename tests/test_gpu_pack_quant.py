@@ -24,7 +24,13 @@ def test_pack_unpack_identity(wname):
     for k, v in w.items():
         if v is None:
             continue
-        assert np.array_equal(np_bits(out[k]), np_bits(v)), k
+        want = np_bits(v)
+        if wname.startswith("e0m3") and k == "codes":
+            # float4e0m3 is stored as the symmetric integer it is: -0 comes back as +0
+            want = want.copy()
+            want[(want & 0x0F) == 0x08] &= 0xF0
+            want[(want & 0xF0) == 0x80] &= 0x0F
+        assert np.array_equal(np_bits(out[k]), want), k
 
 
 @pytest.mark.parametrize("wname,aname", [("mxfp4", "mxfp8"), ("nvfp4", "nvfp4"), ("fp8", "fp8")])
