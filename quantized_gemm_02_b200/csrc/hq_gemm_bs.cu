@@ -429,17 +429,26 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       if (is >= NS && !mbar_wait(&sfree[s], ph ^ 1)) { *s_abort = 1; break; }
       if (*(volatile int *)s_abort) break;
+      if (p.gather) {
+        // indexed mode: the tile's rows of the stage (128 bytes each) from the
+        // caller's codes, 16 bytes per copy into the swizzled tile, all lanes;
+        // the copies arrive on the stage barrier
+        uint8_t *st = smem + s * C::STAGE;
+        for (int it = lane; it < nvalid * 8; it += 32) {
+          const int ii = it >> 3, c = it & 7;
+          cp_async16(st + C::W_SMEM + sw128_offset(ii, c),
+                     p.a_src + (size_t)s_rows[ii] * p.a_ld + (size_t)w.ks * 128 + c * 16);
+        }
+        cp_async_arrive(&full[s]);
+        __syncwarp();
+      }
       if (lane == 0) {
         uint8_t *st = smem + s * C::STAGE;
         if (!p.gather) {
           mbar_arrive_expect_tx(&full[s], (uint32_t)(C::A_SMEM + C::SF_CH * C::SFB_CHB));
           tma_load_2d(st + C::W_SMEM, &a_map, w.ks * 128, base, &full[s]);
         } else {
-          const int ng = (nvalid + 3) >> 2;
-          mbar_arrive_expect_tx(&full[s], (uint32_t)(ng * 4 * 128 + C::SF_CH * C::SFB_CHB));
-          for (int gi = 0; gi < ng; ++gi)
-            tc::tma_gather4(st + C::W_SMEM + gi * 512, &a_map, w.ks * 128, s_rows[4 * gi], s_rows[4 * gi + 1],
-                            s_rows[4 * gi + 2], s_rows[4 * gi + 3], &full[s]);
+          mbar_arrive_expect_tx(&full[s], (uint32_t)(C::SF_CH * C::SFB_CHB));
         }
         if constexpr (C::SF_CH > 0)
           bulk_g2s(st + C::SFB_OFF, sfsrc + (size_t)w.ks * C::SF_CH * C::SFB_CHB, C::SF_CH * C::SFB_CHB, &full[s]);
@@ -460,6 +469,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       if (!mbar_wait(&full[s], ph)) { *s_abort = 1; break; }
       if (*(volatile int *)s_abort) break;
+      if (p.gather) fence_proxy_async_smem();  // cp.async rows -> tensor-core reads
       tc::tc_fence_after();
       const uint32_t st = smem_u32(smem + s * C::STAGE);
       const uint64_t adesc = tc::sw128_desc(st);
@@ -693,8 +703,7 @@ hq_status launch_bs_gemm(const Layout &L, const void *packed, int E, const void 
   const int row_bytes = L.bs == BS_NV ? L.K / 2 : L.K;
   CUtensorMap wm, am;
   if (!make_bs_weight_map(&wm, L, packed, E)) return HQ_ERR_CUDA;
-  // indexed mode: one-row boxes for the 4-row gathers of caller rows
-  if (!make_bs_act_map(&am, a_codes, a_rows, row_bytes, gather ? 1 : t.bnt)) return HQ_ERR_CUDA;
+  if (!make_bs_act_map(&am, a_codes, a_rows, row_bytes, t.bnt)) return HQ_ERR_CUDA;
   if (L.bs != BS_F8) {
     const size_t words = (size_t)t.mtiles * (L.K / kstage) * sf_ch * (t.bnt > 128 ? 256 : 128);
     size_t blocks = (words + 255) / 256;
@@ -723,6 +732,8 @@ hq_status launch_bs_gemm(const Layout &L, const void *packed, int E, const void 
   p.row_scale = L.bs == BS_F8 ? (const float *)a_scales : nullptr;
   p.a_div = a_div;
   p.gather = gather;
+  p.a_src = (const uint8_t *)a_codes;
+  p.a_ld = row_bytes;
   p.out = (uint16_t *)out;
   p.ntw = t.ntw;
   p.mtiles = t.mtiles;

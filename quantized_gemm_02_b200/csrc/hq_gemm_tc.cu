@@ -16,8 +16,10 @@
 //                    TMEM lanes 32w..32w+31), fp32 scales, bf16 out or fp32
 //                    split-K partials with a deterministic last-split fixup;
 //       warp 4       producer: TMA of the activation tile (bf16, 128-byte
-//                    swizzle; a 4-row gather for MoE indexed mode), 1-D bulk
-//                    copies of the packed weight unit, scales, zero points;
+//                    swizzle; for MoE indexed mode the tile's rows gathered
+//                    through the routing index by 16-byte cp.async copies
+//                    into the same swizzled layout), 1-D bulk copies of the
+//                    packed weight unit, scales, zero points;
 //       warp 5       MMA issuer: tcgen05.mma.cta_group::1.kind::f16 with A
 //                    from TMEM and B from a shared-memory descriptor;
 //       warps 6..13  dequant: thread = weight row, decodes 32 k of its row per
@@ -103,6 +105,8 @@ struct Params {
   const int32_t *offsets, *perm;
   int a_div;
   int gather;              // MoE indexed mode: activation rows gathered by index
+  const uint8_t *a_src;    // indexed mode: the activation rows (a_ld bytes apart)
+  int a_ld;
   uint16_t *out;
   int ntw;                 // 128-row weight tiles
   int mtiles;              // token tiles (dense: exact; MoE: upper bound)
@@ -182,15 +186,6 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
       "[%4];" ::"r"(smem_u32(dst)),
       "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ void tma_gather4(void *dst, const CUtensorMap *map, int x, int r0, int r1, int r2, int r3,
-                                            uint64_t *bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
-      "%3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
-      "l"(map), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(smem_u32(bar))
       : "memory");
 }
 
@@ -543,6 +538,19 @@ __global__ void __launch_bounds__(THREADS, (BNT <= 64 ? 2 : 1)) tc_gemm_kernel(c
       const int s = is % NS;
       if (is >= NS && !mbar_wait(&sfree[s], ((is / NS) - 1) & 1)) { *s_abort = 1; stop = true; break; }
       if (*(volatile int *)s_abort) { stop = true; break; }
+      if (p.gather) {
+        // indexed mode: the tile's rows from the caller's activations, 16 bytes
+        // per copy, all lanes; the copies arrive on the stage barrier
+        uint8_t *st = smem + s * C::STAGE;
+        const int items = ti.nvalid * nblk * 8;
+        for (int it = lane; it < items; it += 32) {
+          const int ii = it / (nblk * 8), rem = it - ii * (nblk * 8), j = rem >> 3, c = rem & 7;
+          cp_async16(st + j * C::ACT_KB + sw128_offset(ii, c),
+                     p.a_src + (size_t)s_rows[ii] * p.a_ld + (size_t)(kbs + j) * 128 + c * 16);
+        }
+        cp_async_arrive(&full[s]);
+        __syncwarp();
+      }
       if (lane == 0) {
         const uint8_t *eb = p.packed + (size_t)ti.expert * p.stride;
         uint8_t *st = smem + s * C::STAGE;
@@ -550,20 +558,10 @@ __global__ void __launch_bounds__(THREADS, (BNT <= 64 ? 2 : 1)) tc_gemm_kernel(c
         const int g1 = (((kbs + nblk) * TILE_K - 1) >> p.gshift) + 1;
         const uint32_t sb = TR::has_scales ? (uint32_t)((g1 - g0) * BM * TR::sbytes) : 0u;
         const uint32_t zb = TR::has_zero ? (uint32_t)((g1 - g0) * BM) : 0u;
-        constexpr uint32_t row_bytes = F8 ? 64u : 128u;
-        const uint32_t ab = p.gather ? (uint32_t)(((ti.nvalid + 3) / 4) * 4 * row_bytes) : (uint32_t)C::ACT_KB;
+        const uint32_t ab = p.gather ? 0u : (uint32_t)C::ACT_KB;
         mbar_arrive_expect_tx(&full[s], ab * nblk + TR::unit * nblk + sb + zb);
-        for (int j = 0; j < nblk; ++j) {
-          const int kbj = kbs + j;
-          if (!p.gather) {
-            tma_load_2d(st + j * C::ACT_KB, &act_map, kbj * TILE_K, ti.base, &full[s]);
-          } else {
-            // four rows per gather, each 64 k (one 128-byte swizzled row of the tile)
-            for (int i = 0; i < ti.nvalid; i += 4)
-              tma_gather4(st + j * C::ACT_KB + i * row_bytes, &act_map, kbj * TILE_K, s_rows[i], s_rows[i + 1],
-                          s_rows[i + 2], s_rows[i + 3], &full[s]);
-          }
-        }
+        if (!p.gather)
+          for (int j = 0; j < nblk; ++j) tma_load_2d(st + j * C::ACT_KB, &act_map, (kbs + j) * TILE_K, ti.base, &full[s]);
         bulk_g2s_stream(st + C::ACT, eb + p.w_off + ((size_t)ti.wt * p.KB + kbs) * TR::unit, TR::unit * nblk,
                         &full[s], pol);
         if (TR::has_scales)
@@ -696,6 +694,7 @@ __global__ void __launch_bounds__(THREADS, (BNT <= 64 ? 2 : 1)) tc_gemm_kernel(c
         const int nblk = min(C::KPS, ukb1 - kbs);
         const int s = is % NS;
         if (!mbar_wait(&full[s], (is / NS) & 1)) { *s_abort = 1; stop = true; break; }
+        if (p.gather) fence_proxy_async_smem();  // cp.async rows -> tensor-core reads
         for (int j = 0; j < nblk; ++j, ++ia) {
           const int a = ia % NA;
           const bool first = (i == 0 && j == 0);
@@ -996,7 +995,7 @@ hq_status launch_tc_gemm(const Layout &L, const void *packed, const void *a_bf16
                          bool e4m3_act) {
   if (e4m3_act && L.fmt != W_FP8) return HQ_ERR_UNSUPPORTED;
   CUtensorMap map;
-  if (!make_act_map(&map, a_bf16, a_rows, L.K, gather ? 1 : t.bnt, e4m3_act)) return HQ_ERR_CUDA;
+  if (!make_act_map(&map, a_bf16, a_rows, L.K, t.bnt, e4m3_act)) return HQ_ERR_CUDA;
   tc::Params p{};
   p.packed = (const uint8_t *)packed;
   p.stride = L.stride;
@@ -1013,6 +1012,8 @@ hq_status launch_tc_gemm(const Layout &L, const void *packed, const void *a_bf16
   p.perm = perm;
   p.a_div = a_div;
   p.gather = gather;
+  p.a_src = (const uint8_t *)a_bf16;
+  p.a_ld = L.K * 2;
   p.out = (uint16_t *)out;
   p.ntw = t.ntw;
   p.mtiles = t.mtiles;
