@@ -322,6 +322,8 @@ CONFIG_TITLES = {
             "T in {16, 4096}: two calls versus the fused epilogue",
     "lowbit": "dense WnA16 at the other widths (INT2, INT3 g128; MXFP6 E2M3; float4e0m3 g128), N=28672, "
               "K=8192, M in {1, 16}",
+    "fp8b": "block-scaled FP8 W8A8 (128 x 128 weight blocks, per token and 128 k activation scales): dense "
+            "N=K=7168, M in {1,32,256,2048,8192}; MoE at the config-3 shapes, T in {64, 4096}, grouped + indexed",
     "mxint4": "MoE W4A16 MXINT4 (INT4 elements, E8M0 per 32) at the config-3 shapes and routing, T in {16, 4096}, "
               "grouped + indexed",
 }
@@ -340,6 +342,8 @@ WORKLOAD_TITLE = {
     "w8a8_fp8": "dense W8A8 FP8 per-channel x per-token, N=K=7168, M in {1,32,256,2048,8192}",
     "moe_silu": "MoE gate-up GEMM + SiLU-and-mul at the config-3 shapes, T in {16, 4096}: unfused and fused",
     "lowbit": "dense WnA16 INT2, INT3, MXFP6 E2M3, float4e0m3 at N=28672, K=8192, M in {1, 16}",
+    "w8a8_fp8_block": "block-scaled FP8 W8A8: dense N=K=7168, M in {1,32,256,2048,8192}, and MoE at the config-3 "
+                      "shapes, T in {64, 4096}, grouped + indexed",
     "moe_w4a16_mxint4": "MoE W4A16 MXINT4 (INT4 elements, E8M0 per 32), config-3 shapes and routing, T in "
                         "{16, 4096}, grouped + indexed",
     "moe_masked_nvfp4": "masked-layout MoE W4A4 NVFP4 x NVFP4 (activations quantised on the fly), E=256 slabs of "
@@ -412,9 +416,10 @@ def moe_call_kernels(hq, wdesc, a_dtype, mode, combine):
     relayout or the dequantisation path's exact decode, the GEMM, and the
     weighted combine."""
     quant = a_dtype not in (None, hq.HQ_BF16)
-    block_scaled = (wdesc.w_dtype == hq.HQ_E2M1 and
-                    ((wdesc.w_scale_dtype == hq.HQ_E8M0 and a_dtype == hq.HQ_MXFP8) or
-                     (wdesc.w_scale_dtype == hq.HQ_UE4M3 and a_dtype == hq.HQ_NVFP4)))
+    block_scaled = ((wdesc.w_dtype == hq.HQ_E2M1 and
+                     ((wdesc.w_scale_dtype == hq.HQ_E8M0 and a_dtype == hq.HQ_MXFP8) or
+                      (wdesc.w_scale_dtype == hq.HQ_UE4M3 and a_dtype == hq.HQ_NVFP4))) or
+                    (wdesc.w_dtype == hq.HQ_E4M3 and wdesc.w_group == 128))
     n = 1  # the GEMM
     if quant:
         n += 2 if a_dtype == hq.HQ_NVFP4 else 1
@@ -442,6 +447,10 @@ def ops_moe(hq, config, name, wdesc, E, topk, H, I, Ts, routing, gen, a_dtype, m
             w = synth.mxint4_weights(E, N, K, gen, device=dev)
             glob = None
             bytes_per = N * K // 2 + N * K // 32
+        elif wdesc.w_dtype == hq.HQ_E4M3 and wdesc.w_group == 128:
+            w = synth.fp8_block_weights(E, N, K, gen, device=dev)
+            glob = None
+            bytes_per = N * K + ((N + 127) // 128) * (K // 128) * 4
         else:
             w = synth.nvfp4_weights_random(E, N, K, gen, device=dev)
             glob = w["global"]
@@ -506,7 +515,7 @@ def ops_moe(hq, config, name, wdesc, E, topk, H, I, Ts, routing, gen, a_dtype, m
             kg, bs = moe_call_kernels(hq, wdesc, a_dtype, mode, 0)
             kd, _ = moe_call_kernels(hq, wdesc, a_dtype, mode, 1)
             if bs:
-                ratio = 2.0 if wdesc.w_scale_dtype == hq.HQ_E8M0 else 4.0
+                ratio = 4.0 if wdesc.w_scale_dtype == hq.HQ_UE4M3 else 2.0
             kern = "bs_gemm_kernel" if bs else ("dec_gemm_kernel / tc_gemm_kernel")
             ops.append(Op(f"{name}_T{T}_{mode_name}_gate_up", run_gate, 2.0 * T * topk * Ng * Kg, touched * bg,
                           T * Kg * 2 + T * topk * Ng * 2, kg, T * Kg * 2, 0, e2e_gate, kernel=kern, peak_ratio=ratio,
@@ -590,6 +599,16 @@ def ops_moe_silu(hq, gen, Ts=(16, 4096)):
     return ops, keep
 
 
+def ops_moe_fp8_block(hq, gen, Ts=(64, 4096)):
+    """Block-scaled FP8 W8A8 MoE (128 x 128 weight blocks, per token and 128
+    k activation scales quantised on the fly) at the config-3 shapes."""
+    d = desc_of(hq, hq.HQ_E4M3, 128, hq.HQ_FP32, 0, 0, hq.HQ_E4M3)
+    d.a_group = 128
+    routing = lambda T, g: synth.routing_softmax_topk(T, E_MOE, TOPK, g, device="cuda")
+    return ops_moe(hq, "fp8b", "moe_w8a8_fp8_block", d, E_MOE, TOPK, H_MOE, I_MOE, list(Ts), routing, gen,
+                   hq.HQ_E4M3)
+
+
 def ops_moe_w4a8_mxfp8(hq, gen, Ts=(1, 64, 512, 4096)):
     d = desc_of(hq, hq.HQ_E2M1, 32, hq.HQ_E8M0, 0, 0, hq.HQ_MXFP8)
     routing = lambda T, g: synth.routing_zipf(T, E_MOE, TOPK, 1.2, g, device="cuda")
@@ -662,6 +681,10 @@ def ops_dense_quantised(hq, fmt, gen, N=7168, K=7168, Ms=(1, 32, 256, 2048, 8192
     if fmt == "nvfp4":
         d = desc_of(hq, hq.HQ_E2M1, 16, hq.HQ_UE4M3, 0, 1, hq.HQ_NVFP4)
         wbytes = N * K // 2 + N * K // 16
+    elif fmt == "fp8b":
+        d = desc_of(hq, hq.HQ_E4M3, 128, hq.HQ_FP32, 0, 0, hq.HQ_E4M3)
+        d.a_group = 128
+        wbytes = N * K + ((N + 127) // 128) * (K // 128) * 4
     else:
         d = desc_of(hq, hq.HQ_E4M3, 0, hq.HQ_FP32, 0, 0, hq.HQ_E4M3)
         wbytes = N * K + N * 4
@@ -672,6 +695,9 @@ def ops_dense_quantised(hq, fmt, gen, N=7168, K=7168, Ms=(1, 32, 256, 2048, 8192
         if fmt == "nvfp4":
             c = torch.empty(M, K // 2, dtype=torch.uint8, device=dev)
             s = torch.empty(M, K // 16, dtype=torch.uint8, device=dev)
+        elif fmt == "fp8b":
+            c = torch.empty(M, K, dtype=torch.uint8, device=dev)
+            s = torch.empty(M, K // 128, dtype=torch.float32, device=dev)
         else:
             c = torch.empty(M, K, dtype=torch.uint8, device=dev)
             s = torch.empty(M, dtype=torch.float32, device=dev)
@@ -679,10 +705,16 @@ def ops_dense_quantised(hq, fmt, gen, N=7168, K=7168, Ms=(1, 32, 256, 2048, 8192
         wsq = torch.zeros(64, dtype=torch.uint8, device=dev)
         return c, s, g, wsq
 
-    wc, wsc, wg, wq = quant(Wf)
-    hq.hq_quant_act(d, N, K, Wf, wc, wsc, wg, None, wq, 64)
     packed = torch.empty(hq.hq_packed_weights_bytes(d, 1, N, K), dtype=torch.uint8, device=dev)
-    hq.hq_pack_weights(d, 1, N, K, wc, wsc, None, wg if fmt == "nvfp4" else None, packed)
+    if fmt == "fp8b":
+        # random E4M3 codes with 128 x 128 block scales (no weight quantiser for blocks)
+        wb = synth.fp8_block_weights(1, N, K, gen, device=dev)
+        hq.hq_pack_weights(d, 1, N, K, wb["codes"], wb["scales"], None, None, packed)
+        wg = None
+    else:
+        wc, wsc, wg, wq = quant(Wf)
+        hq.hq_quant_act(d, N, K, Wf, wc, wsc, wg, None, wq, 64)
+        hq.hq_pack_weights(d, 1, N, K, wc, wsc, None, wg if fmt == "nvfp4" else None, packed)
     ops = []
     keep = [packed, wg]
     for M in Ms:
@@ -705,9 +737,11 @@ def ops_dense_quantised(hq, fmt, gen, N=7168, K=7168, Ms=(1, 32, 256, 2048, 8192
             C_h.copy_(C, non_blocking=True)
 
         kern = (2 if fmt == "nvfp4" else 1) + (1 if fmt == "fp8" else 2)
-        ops.append(Op(f"cfg5_{fmt}_N{N}_K{K}_M{M}", run, 2.0 * M * N * K, wbytes, M * K * 2 + M * N * 2, kern,
-                      M * K * 2, M * N * 2, e2e, kernel="bs_gemm_kernel",
-                      peak_ratio=4.0 if fmt == "nvfp4" else 2.0, config=5))
+        tag = 5 if fmt != "fp8b" else "fp8b"
+        ops.append(Op(f"{'cfg5_' if tag == 5 else ''}{fmt}_N{N}_K{K}_M{M}", run, 2.0 * M * N * K, wbytes,
+                      M * K * 2 + M * N * 2, kern, M * K * 2, M * N * 2, e2e,
+                      kernel="bsf_gemm_kernel" if fmt == "fp8b" else "bs_gemm_kernel",
+                      peak_ratio=4.0 if fmt == "nvfp4" else 2.0, config=tag))
     return ops, keep
 
 
@@ -726,7 +760,10 @@ def _workload(builders, title):
 WORKLOADS = {
     "all": _workload([ops_w4a16_dense_m16, ops_w4a16_asym_sweep, ops_moe_w4a16_mxfp4, ops_moe_w4a8_mxfp8,
                       lambda hq, g: ops_dense_quantised(hq, "nvfp4", g), lambda hq, g: ops_dense_quantised(hq, "fp8", g),
-                      ops_moe_nvfp4, ops_moe_w4a16_mxint4, ops_moe_silu, ops_lowbit], WORKLOAD_TITLE["all"]),
+                      ops_moe_nvfp4, ops_moe_w4a16_mxint4, ops_moe_silu, ops_lowbit,
+                      lambda hq, g: ops_dense_quantised(hq, "fp8b", g), ops_moe_fp8_block], WORKLOAD_TITLE["all"]),
+    "w8a8_fp8_block": _workload([lambda hq, g: ops_dense_quantised(hq, "fp8b", g), ops_moe_fp8_block],
+                                WORKLOAD_TITLE["w8a8_fp8_block"]),
     "lowbit": _workload([ops_lowbit], WORKLOAD_TITLE["lowbit"]),
     "moe_silu": _workload([ops_moe_silu], WORKLOAD_TITLE["moe_silu"]),
     "moe_w4a16_mxint4": _workload([ops_moe_w4a16_mxint4], WORKLOAD_TITLE["moe_w4a16_mxint4"]),
@@ -741,7 +778,7 @@ WORKLOADS = {
 }
 
 # configurations each workload covers (for the CPU samples)
-WORKLOAD_CONFIGS = {"all": (1, 2, 3, 4, 5), "moe_w4a16_mxint4": (3,), "moe_silu": (3,), "lowbit": (2,), "w4a16_asym_sweep": (2,), "w4a16_dense_m16": (1,),
+WORKLOAD_CONFIGS = {"all": (1, 2, 3, 4, 5), "w8a8_fp8_block": (5,), "moe_w4a16_mxint4": (3,), "moe_silu": (3,), "lowbit": (2,), "w4a16_asym_sweep": (2,), "w4a16_dense_m16": (1,),
                     "moe_w4a16_mxfp4": (3,), "moe_w4a8_mxfp8": (4,), "moe_nvfp4": (5,), "moe_masked_nvfp4": (5,),
                     "w4a4_nvfp4": (5,), "w8a8_fp8": (5,)}
 

@@ -36,7 +36,8 @@
  *       E2M1 codes        uint8 [E, N, K/2], low nibble = even k.
  *       E8M0 scales       uint8 [E, N, K/32] (MXFP4, MXINT4).
  *       UE4M3 scales      uint8 [E, N, K/16] (NVFP4) + fp32 global [E].
- *       E4M3 codes        uint8 [E, N, K] + fp32 per-channel scales [E, N].
+ *       E4M3 codes        uint8 [E, N, K] + fp32 per-channel scales [E, N]
+ *                         (block-scaled: fp32 [E, ceil(N / 128), K / 128]).
  *       INT2/UINT2/INT3/UINT3/E2M3/E3M2/E0M3 codes (b bits): uint8
  *                         [E, N, K * b / 8], a little-endian bit stream per
  *                         row (code k at bits b*k .. b*k + b - 1; for b = 4
@@ -108,6 +109,8 @@ typedef enum {
  *   E2M1  + E8M0 scales, w_group = 32                       (MXFP4)
  *   E2M1  + UE4M3 scales, w_group = 16, w_has_global = 1    (NVFP4)
  *   E4M3  + FP32 per-channel scales, w_group = 0            (FP8)
+ *   E4M3  + FP32 scales per 128 x 128 block, w_group = 128  (block-scaled
+ *         FP8, only with a_dtype E4M3 and a_group 128, K a multiple of 128)
  *   INT2, INT3, E0M3 + BF16 scales, w_group in {0, 32, 64, 128}
  *   UINT2, UINT3 + BF16 scales + zero points, w_group in {32, 64, 128}
  *   E2M3, E3M2 + E8M0 scales, w_group = 32                  (MXFP6)
@@ -117,7 +120,9 @@ typedef enum {
  * zero-exponent view of symmetric INT4 and computes as INT4.
  * a_group is the activation's scale granularity along K: 0 = the format's
  * own (E4M3: one fp32 scale per token; MXFP8: 32; NVFP4: 16); MXFP8 also
- * accepts 32 and NVFP4 16.  Zero-initialise the struct.
+ * accepts 32 and NVFP4 16; E4M3 with a_group 128 has one fp32 scale per
+ * token and 128 k (the activations of block-scaled FP8, which take no
+ * other weight format).  Zero-initialise the struct.
  */
 typedef struct {
   int32_t w_dtype;       /* HQ_INT4 | HQ_UINT4 | HQ_E2M1 | HQ_E4M3           */
@@ -201,6 +206,8 @@ HQ_API hq_status hq_unpack_weights(const hq_quant_desc *desc, int E, int N, int 
  * FP8, MXFP8, NVFP4 activations).  x: bf16 [M, K], K a multiple of 32.
  *   a_dtype == HQ_E4M3: codes uint8 [M, K], scales fp32 [M];
  *       s = amax_row / 448, q = e4m3(x / s) (s = 1 for an all-zero row).
+ *       With a_group == 128: scales fp32 [M, K / 128], the same recipe on
+ *       each 128-k group of a row (K a multiple of 128).
  *   a_dtype == HQ_MXFP8: codes uint8 [M, K], scales uint8 E8M0 [M, K/32];
  *       e = floor(log2(amax_blk)) - 8 clamped to [-127, 127], code e + 127,
  *       q = e4m3(x * 2^-e) (code 127 and q = 0 for an all-zero block).
@@ -221,7 +228,10 @@ HQ_API hq_status hq_quant_act(const hq_quant_desc *desc, int M, int K, const voi
  * Dense GEMM: C[M, N] (bf16) = A[M, K] . W[N, K]^T with W the packed
  * weights of one expert (E = 1) and A in desc->a_dtype:
  *   BF16:  a = bf16 [M, K], a_scales = NULL
- *   E4M3:  a = uint8 [M, K], a_scales = fp32 [M] (per token)
+ *   E4M3:  a = uint8 [M, K], a_scales = fp32 [M] (per token), or with
+ *          a_group 128 fp32 [M, K / 128] (block-scaled FP8 weights: each
+ *          128-k stage is multiplied in the tensor core and added in fp32
+ *          with both scales)
  *   MXFP8: a = uint8 [M, K], a_scales = uint8 [M, K/32]
  *   NVFP4: a = uint8 [M, K/2], a_scales = uint8 [M, K/16], a_global = fp32 [1]
  * M >= 0 (M == 0 is a no-op), N >= 1, K a multiple of 64.

@@ -247,6 +247,9 @@ def decode_weights(d: Desc, N: int, K: int, codes, scales, zeros=None, global_sc
                 W = W * float(np.float32(global_scale))
         else:
             raise ValueError(d.w_scale)
+    elif d.w_dtype == "e4m3" and d.w_group == 128:
+        # block-scaled FP8: scales [ceil(N / 128), K / 128]
+        W = decode_fp8_block_weights(np.asarray(codes).reshape(N, K), np.asarray(scales).reshape(-1, K // 128))
     elif d.w_dtype == "e4m3":
         W = E4M3[np.asarray(codes).reshape(N, K)]
         col = np.asarray(scales, dtype=np.float32).reshape(N).astype(np.float64)
@@ -338,6 +341,9 @@ def decode_act(a_dtype: str, M: int, K: int, a, scales=None, global_scale=None):
     elif a_dtype == "mxfp8":
         blk = np.arange(K) // 32
         A = E4M3[np.asarray(a).reshape(M, K)] * E8M0[np.asarray(scales).reshape(M, K // 32)][:, blk]
+    elif a_dtype == "fp8g":
+        # E4M3 with an fp32 scale per token and 128 k (quant_fp8_block)
+        A = decode_fp8_block_act(np.asarray(a).reshape(M, K), np.asarray(scales).reshape(M, K // 128))
     elif a_dtype == "nvfp4":
         blk = np.arange(K) // 16
         c = unpack_nibbles_u8(np.asarray(a).reshape(M, K // 2), K)
@@ -525,14 +531,18 @@ def decode_mxint4_weights(codes, e8m0_scales, K: int):
     return q * E8M0[np.asarray(e8m0_scales).reshape(N, K // 32)][:, blk]
 
 
-def decode_fp8_block_weights(codes, scales, block: int = 128):
+def decode_fp8_block_weights(codes, scales, block: int = 128, row_block=None):
     """FP8 weights with block scales: E4M3 codes [N, K] and fp32 scales
-    [ceil(N / block), K / block], one per block x block tile:
-    w[n, k] = e4m3(code) * s[n // block, k // block]."""
+    [ceil(N / row_block), K / block], one per row_block x block tile
+    (row_block defaults to block: square blocks):
+    w[n, k] = e4m3(code) * s[n // row_block, k // block].  row_block = 1
+    takes one scale row per weight row (a block's scale row repeated), for
+    decoding some rows of a matrix."""
     c = np.asarray(codes)
     N, K = c.shape
+    rb = block if row_block is None else row_block
     s = np.asarray(scales, dtype=np.float32).astype(np.float64)
-    return E4M3[c] * s[np.arange(N)[:, None] // block, np.arange(K)[None, :] // block]
+    return E4M3[c] * s[np.arange(N)[:, None] // rb, np.arange(K)[None, :] // block]
 
 
 def quant_fp8_block(x_bits: np.ndarray, group: int = 128):

@@ -63,6 +63,7 @@ static size_t act_code_bytes(int afmt, int K) { return afmt == A_NVFP4 ? (size_t
 static size_t act_scale_bytes(int afmt, int K) {
   switch (afmt) {
     case A_FP8: return 4;
+    case A_FP8G: return (size_t)K / 128 * 4;
     case A_MXFP8: return (size_t)K / 32;
     case A_NVFP4: return (size_t)K / 16;
     default: return 0;
@@ -94,6 +95,7 @@ static hq_status plan_dense(const hq_quant_desc *d, int M, int N, int K, DensePl
   if (M < 0 || N < 1 || !valid_k(d, K)) return HQ_ERR_INVALID_ARG;
   pl->L = layout_for(d, fmt, N, K);
   pl->afmt = afmt;
+  if (!pair_supported(pl->L, afmt)) return HQ_ERR_UNSUPPORTED;
   pl->s = plan_tc(M > 0 ? M : 1, 0, N, pl->L.KB, false, pl->L.bs);
   return HQ_OK;
 }
@@ -175,6 +177,7 @@ static hq_status plan_moe(const hq_quant_desc *d, int T, int topk, int E, int N,
   if ((long)T * topk > (1L << 30)) return HQ_ERR_INVALID_ARG;
   pl->L = layout_for(d, fmt, N, K);
   pl->afmt = afmt;
+  if (!pair_supported(pl->L, afmt)) return HQ_ERR_UNSUPPORTED;
   pl->R = T * topk;
   pl->src_rows = a_per_slot ? pl->R : T;
   const int R = pl->R > 0 ? pl->R : 1;
@@ -199,6 +202,7 @@ static hq_status plan_moe_masked(const hq_quant_desc *d, int E, int slab, int N,
   if ((long)E * slab > (1L << 30)) return HQ_ERR_INVALID_ARG;
   pl->L = layout_for(d, fmt, N, K);
   pl->afmt = afmt;
+  if (!pair_supported(pl->L, afmt)) return HQ_ERR_UNSUPPORTED;
   pl->R = E * slab;
   pl->src_rows = E * slab;
   const int em = expected_m < 1 ? slab : (expected_m > slab ? slab : expected_m);
@@ -369,9 +373,11 @@ hq_status hq_device_error(hq_stream_t stream) {
 }
 
 size_t hq_packed_weights_bytes(const hq_quant_desc *desc, int E, int N, int K) {
-  int fmt;
+  int fmt, afmt;
   if (!weight_format(desc, &fmt) || E < 1 || N < 1 || !valid_k(desc, K)) return 0;
-  return layout_for(desc, fmt, N, K).stride * (size_t)E;
+  const Layout L = layout_for(desc, fmt, N, K);
+  if (!act_format(desc, &afmt) || !pair_supported(L, afmt)) return 0;
+  return L.stride * (size_t)E;
 }
 
 // Pack / unpack with the plain or the gated (gate/up rows side by side) row order.
@@ -387,8 +393,11 @@ static hq_status pack_impl(const hq_quant_desc *desc, int E, int N, int K, const
   if ((fmt == W_UINT4) != (zeros != nullptr)) return HQ_ERR_INVALID_ARG;
   if ((fmt == W_NVFP4) != (global_scale != nullptr)) return HQ_ERR_INVALID_ARG;
   if (!aligned16(codes) || !aligned16(packed) || ((uintptr_t)scales & 3u)) return HQ_ERR_INVALID_ARG;
-  if (!device_is_sm100()) return HQ_ERR_ARCH;
   Layout L = layout_for(desc, fmt, N, K);
+  int afmt;
+  if (!act_format(desc, &afmt) || !pair_supported(L, afmt)) return HQ_ERR_UNSUPPORTED;
+  if (gated && L.bs == BS_F8B) return HQ_ERR_UNSUPPORTED;  // a tile would span two scale blocks
+  if (!device_is_sm100()) return HQ_ERR_ARCH;
   L.gated = gated ? 1 : 0;
   return launch_pack(L, E, codes, scales, zeros, global_scale, packed, (cudaStream_t)stream);
 }
@@ -403,8 +412,11 @@ static hq_status unpack_impl(const hq_quant_desc *desc, int E, int N, int K, con
   if (!codes || !scales || !packed) return HQ_ERR_INVALID_ARG;
   if ((fmt == W_UINT4) != (zeros != nullptr)) return HQ_ERR_INVALID_ARG;
   if ((fmt == W_NVFP4) != (global_scale != nullptr)) return HQ_ERR_INVALID_ARG;
-  if (!device_is_sm100()) return HQ_ERR_ARCH;
   Layout L = layout_for(desc, fmt, N, K);
+  int afmt;
+  if (!act_format(desc, &afmt) || !pair_supported(L, afmt)) return HQ_ERR_UNSUPPORTED;
+  if (gated && L.bs == BS_F8B) return HQ_ERR_UNSUPPORTED;
+  if (!device_is_sm100()) return HQ_ERR_ARCH;
   L.gated = gated ? 1 : 0;
   return launch_unpack(L, E, packed, codes, scales, zeros, global_scale, (cudaStream_t)stream);
 }
@@ -438,6 +450,7 @@ hq_status hq_quant_act(const hq_quant_desc *desc, int M, int K, const void *x_bf
   if (!act_format(desc, &afmt)) return HQ_ERR_UNSUPPORTED;
   if (afmt == A_BF16) return HQ_ERR_INVALID_ARG;
   if (M < 0 || K < 32 || (K % 32) != 0) return HQ_ERR_INVALID_ARG;
+  if (afmt == A_FP8G && (K % 128) != 0) return HQ_ERR_INVALID_ARG;
   if (M == 0) return HQ_OK;
   if (!x_bf16 || !codes || !scales || !aligned16(x_bf16) || !aligned16(codes)) return HQ_ERR_INVALID_ARG;
   if (afmt == A_NVFP4) {

@@ -605,6 +605,400 @@ __global__ void bs_sf_tiles_kernel(int slots, int bnt, int kst, int sf_ch, int l
   }
 }
 
+
+// ---- FP8 with 128 x 128 block weight scales and per-(token, 128 k) activation
+// scales.  The tensor core cannot apply arbitrary fp32 block scales, so each
+// 128-k stage is multiplied into its own TMEM accumulator (a ring of NP) and
+// the epilogue warps promote it into fp32 registers:
+//     acc[m] += P[m] * (s_w[tile, stage] * s_a[m, stage]),
+// the product summed per stage in the tensor core's fp32 and the stages in
+// k order.  Warps: 0..3 promotion + output (thread = weight row, BNT
+// accumulators in registers), 4 weight producer, 5 MMA issuer, 6 activation
+// producer (codes by TMA or, indexed mode, cp.async gathers; the stage's
+// activation scales by a bulk copy from their per-token-tile relayout).
+template <int BNT>
+struct CfgF8B {
+  static constexpr int W_SMEM = BM * 128;
+  static constexpr int A_SMEM = BNT * 128;
+  static constexpr int SA_OFF = W_SMEM + A_SMEM;
+  static constexpr int STAGE = (SA_OFF + BNT * 4 + 1023) / 1024 * 1024;
+  static constexpr int NS_FIT = (200 * 1024) / STAGE;
+  static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;
+  static constexpr int CTRL = 8192;
+  static constexpr int BYTES = NS * STAGE + CTRL + 1024;
+  static constexpr int NP = (512 / BNT) > 4 ? 4 : (512 / BNT);  // stage accumulators in TMEM
+  static constexpr int TMEM_COLS = NP * BNT < 32 ? 32 : NP * BNT;
+  static_assert(NS >= 3 && NP >= 2, "budget");
+  static_assert((TMEM_COLS & (TMEM_COLS - 1)) == 0, "TMEM allocation is a power of two");
+};
+
+// Output of one promoted segment (thread = weight row n): whole tiles are
+// written; a Stream-K piece is stored as fp32 partials, and the last of the
+// CTAs sharing the tile sums the parts in k order (32 columns at a time).
+template <int BNT>
+__device__ __forceinline__ void f8b_finish(const Params &p, const TileInfo &ti, int t, bool whole, bool head,
+                                           const float (&acc)[BNT], int cta, int warp, int lane, long long total) {
+  constexpr int CW = BNT < 32 ? BNT : 32;
+  const int r = warp * 32 + lane;
+  const int n = ti.wt * BM + r;
+  auto write = [&](int c0, const float *x) {
+    int orow_l = 0;
+    if (c0 + lane < ti.nvalid) {
+      const int pos = ti.base + c0 + lane;
+      orow_l = p.moe ? p.perm[pos] : pos;
+    }
+#pragma unroll
+    for (int i = 0; i < CW; ++i) {
+      const int orow = __shfl_sync(0xffffffffu, orow_l, i);
+      tc::put_out(p, orow, n, x[i], c0 + i < ti.nvalid && n < p.N);
+    }
+  };
+  if (whole) {
+#pragma unroll
+    for (int c0 = 0; c0 < BNT; c0 += CW) write(c0, acc + c0);
+    return;
+  }
+  float *part = p.partial + ((size_t)cta * 2 + (head ? 0 : 1)) * BNT * BM;
+#pragma unroll
+  for (int m = 0; m < BNT; ++m) __stcg(&part[(size_t)m * BM + r], acc[m]);
+  __threadfence();
+  __syncwarp();
+  const long long t_first = (long long)t * p.KB;
+  const int c_first = dec::cta_of(t_first, total, p.nctas);
+  const int c_last = dec::cta_of(t_first + p.KB - 1, total, p.nctas);
+  int last = 0;
+  if (lane == 0) {
+    int *ctr = p.counters + (size_t)t * 4 + warp;
+    last = (atomicAdd(ctr, 1) == c_last - c_first);
+    if (last) *ctr = 0;  // ready for the next call
+  }
+  last = __shfl_sync(0xffffffffu, last, 0);
+  if (!last) return;
+  __threadfence();
+#pragma unroll 1
+  for (int c0 = 0; c0 < BNT; c0 += CW) {
+    float x[CW];
+#pragma unroll
+    for (int i = 0; i < CW; ++i) x[i] = 0.f;
+    for (int c = c_first; c <= c_last; ++c) {
+      const float *pc = p.partial + ((size_t)c * 2 + (c == c_first ? 1 : 0)) * BNT * BM + (size_t)c0 * BM + r;
+#pragma unroll
+      for (int i = 0; i < CW; ++i) x[i] += __ldcg(pc + (size_t)i * BM);
+    }
+    write(c0, x);
+  }
+}
+
+template <int BNT>
+__global__ void __launch_bounds__(THREADS, 1)
+    bsf_gemm_kernel(const __grid_constant__ CUtensorMap w_map, const __grid_constant__ CUtensorMap a_map,
+                    const Params p) {
+  using C = CfgF8B<BNT>;
+  constexpr int NS = C::NS, NP = C::NP;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t *ctrl = smem + NS * C::STAGE;
+  uint64_t *full = reinterpret_cast<uint64_t *>(ctrl);  // [NS] codes + activation scales landed
+  uint64_t *sfree = full + NS;                           // [NS] MMAs done and the stage's scales read
+  uint64_t *pfull = sfree + NS;                          // [NP] stage accumulator complete
+  uint64_t *pempty = pfull + NP;                         // [NP] stage accumulator promoted
+  long long *s_total = reinterpret_cast<long long *>(pempty + NP);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(s_total + 1);
+  int *s_abort = reinterpret_cast<int *>(tmem_slot + 1);
+  int *s_tpre = s_abort + 1;                      // [E+1] MoE: prefix of token tiles per expert
+  int *s_rows = s_tpre + (p.moe ? p.E + 1 : 0);  // [BNT] indexed mode: caller rows of the producer's tile
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int cta = blockIdx.x;
+  if (warp == 0) {
+    int tvalid = 0;
+    if (!p.moe) {
+      tvalid = (p.M + BNT - 1) / BNT;
+    } else if (p.offsets[p.E] >= 0) {
+      int running = 0;
+      for (int e0 = 0; e0 < p.E; e0 += 32) {
+        const int e = e0 + lane;
+        int tiles = 0;
+        if (e < p.E) tiles = (p.offsets[e + 1] - p.offsets[e] + BNT - 1) / BNT;
+        int incl = tiles;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        if (e < p.E) s_tpre[e + 1] = running + incl;
+        running += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      if (lane == 0) s_tpre[0] = 0;
+      tvalid = running;
+    }
+    if (tvalid > p.mtiles) tvalid = p.mtiles;
+    if (lane == 0) {
+      *s_total = (long long)tvalid * p.ntw * p.KB;  // (tile, stage) iterations
+      *s_abort = 0;
+    }
+  }
+  if (tid == 32) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 2);      // weight producer and activation producer
+      mbar_init(&sfree[s], 1 + 4);  // MMA commit and the four promotion warps
+    }
+    for (int q = 0; q < NP; ++q) {
+      mbar_init(&pfull[q], 1);
+      mbar_init(&pempty[q], 4);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const long long total = __shfl_sync(0xffffffffu, *s_total, 0);
+  const long long beg = dec::range_begin(cta, total, p.nctas);
+  const long long end = dec::range_begin(cta + 1, total, p.nctas);
+  if (beg >= end) return;
+
+  auto tile_info = [&](int t) {
+    TileInfo ti;
+    const int slot = t / p.ntw;
+    ti.wt = t - slot * p.ntw;
+    if (!p.moe) {
+      ti.expert = 0;
+      ti.base = slot * BNT;
+      ti.nvalid = min(BNT, p.M - ti.base);
+    } else {
+      int lo = 0, hi = p.E;
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (s_tpre[mid] <= slot) lo = mid;
+        else hi = mid;
+      }
+      ti.expert = lo;
+      ti.base = p.offsets[lo] + (slot - s_tpre[lo]) * BNT;
+      ti.nvalid = min(BNT, p.offsets[lo + 1] - ti.base);
+    }
+    return ti;
+  };
+
+  const bool producer = (warp == WARP_W || warp == WARP_ACT);
+  uint32_t tmem = 0;
+  if (producer) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&w_map) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&a_map) : "memory");
+  } else {
+    if (warp == 0) {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                   "r"(C::TMEM_COLS));
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc::tc_fence_before();
+    asm volatile("bar.sync 1, %0;" ::"r"(THREADS - 64) : "memory");
+    tc::tc_fence_after();
+    tmem = __shfl_sync(0xffffffffu, *tmem_slot, 0);
+  }
+
+  if (warp == WARP_W) {
+    // ================= weight producer: one 3-D TMA of the stage's codes =================
+    const uint64_t pol = p.weights_once ? policy_evict_first() : policy_evict_normal();
+    Walk w;
+    w.start(beg, end, p.KB);
+    int cur_t = -1, wrow = 0, expert = 0;
+    for (int is = 0, s = 0, ph = 0; w.left > 0; ++is, w.next(p.KB)) {
+      if (w.t != cur_t) {
+        const TileInfo ti = tile_info(w.t);
+        expert = ti.expert;
+        wrow = ti.wt * p.KB * BM;
+        cur_t = w.t;
+      }
+      if (is >= NS && !mbar_wait(&sfree[s], ph ^ 1)) { *s_abort = 1; break; }
+      if (*(volatile int *)s_abort) break;
+      if (lane == 0) {
+        uint8_t *st = smem + s * C::STAGE;
+        mbar_arrive_expect_tx(&full[s], (uint32_t)C::W_SMEM);
+        asm volatile(
+            "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint "
+            "[%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(st)),
+            "l"(&w_map), "r"(0), "r"(wrow + w.ks * BM), "r"(expert), "r"(smem_u32(&full[s])), "l"(pol)
+            : "memory");
+      }
+      __syncwarp();
+      if (++s == NS) { s = 0; ph ^= 1; }
+    }
+  } else if (warp == WARP_ACT) {
+    // ================= activation producer: codes + the stage's scales =================
+    Walk w;
+    w.start(beg, end, p.KB);
+    int cur_t = -1, base = 0, nvalid = 0;
+    const uint8_t *sasrc = nullptr;
+    for (int is = 0, s = 0, ph = 0; w.left > 0; ++is, w.next(p.KB)) {
+      if (w.t != cur_t) {
+        const TileInfo ti = tile_info(w.t);
+        base = ti.base;
+        nvalid = ti.nvalid;
+        // activation scales of this tile's token slot: [KB][BNT] fp32
+        sasrc = p.a_sf + (size_t)(w.t / p.ntw) * p.KB * BNT * 4;
+        cur_t = w.t;
+        if (p.gather) {
+          for (int i = lane; i < BNT; i += 32) s_rows[i] = p.perm[base + min(i, nvalid - 1)] / p.a_div;
+          __syncwarp();
+        }
+      }
+      if (is >= NS && !mbar_wait(&sfree[s], ph ^ 1)) { *s_abort = 1; break; }
+      if (*(volatile int *)s_abort) break;
+      uint8_t *st = smem + s * C::STAGE;
+      if (p.gather) {
+        for (int it = lane; it < nvalid * 8; it += 32) {
+          const int ii = it >> 3, c = it & 7;
+          cp_async16(st + C::W_SMEM + sw128_offset(ii, c),
+                     p.a_src + (size_t)s_rows[ii] * p.a_ld + (size_t)w.ks * 128 + c * 16);
+        }
+        cp_async_arrive(&full[s]);
+        __syncwarp();
+      }
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&full[s], (uint32_t)((p.gather ? 0 : C::A_SMEM) + BNT * 4));
+        if (!p.gather) tma_load_2d(st + C::W_SMEM, &a_map, w.ks * 128, base, &full[s]);
+        bulk_g2s(st + C::SA_OFF, sasrc + (size_t)w.ks * BNT * 4, (uint32_t)(BNT * 4), &full[s]);
+      }
+      __syncwarp();
+      if (++s == NS) { s = 0; ph ^= 1; }
+    }
+  } else if (warp == WARP_MMA) {
+    // ================= MMA issuer: each stage into its own accumulator =================
+    constexpr uint32_t idesc = tc::idesc_e4m3<BNT>();
+    Walk w;
+    w.start(beg, end, p.KB);
+    for (int is = 0, s = 0, ph = 0, q = 0, qph = 0; w.left > 0; ++is, w.next(p.KB)) {
+      if (!mbar_wait(&full[s], ph)) { *s_abort = 1; break; }
+      if (is >= NP && !mbar_wait(&pempty[q], qph ^ 1)) { *s_abort = 1; break; }
+      if (*(volatile int *)s_abort) break;
+      if (p.gather) fence_proxy_async_smem();  // cp.async rows -> tensor-core reads
+      tc::tc_fence_after();
+      const uint32_t st = smem_u32(smem + s * C::STAGE);
+      const uint64_t adesc = tc::sw128_desc(st);
+      const uint64_t bdesc = tc::sw128_desc(st + C::W_SMEM);
+      if (dec::elect_one()) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          mma_bs<BS_F8>(tmem + (uint32_t)(q * BNT), adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(2 * j), idesc, 0u,
+                        0u, j > 0 ? 1u : 0u);
+        tc::mma_commit(&pfull[q]);
+        tc::mma_commit(&sfree[s]);
+      }
+      __syncwarp();
+      if (++s == NS) { s = 0; ph ^= 1; }
+      if (++q == NP) { q = 0; qph ^= 1; }
+    }
+  } else if (warp < 4) {
+    // ================= promotion: warps 0..3, thread = weight row =================
+    float acc[BNT];
+    Walk w;
+    w.start(beg, end, p.KB);
+    int t0 = w.t, ks0 = w.ks;  // where the current segment started
+    for (int is = 0, s = 0, ph = 0, q = 0, qph = 0; w.left > 0; ++is, w.next(p.KB)) {
+      if (w.seg_first) {
+#pragma unroll
+        for (int m = 0; m < BNT; ++m) acc[m] = 0.f;
+        t0 = w.t;
+        ks0 = w.ks;
+      }
+      const TileInfo ti = tile_info(w.t);
+      const float sw = __ldg(reinterpret_cast<const float *>(p.packed + (size_t)ti.expert * p.stride + p.c_off) +
+                             (size_t)ti.wt * p.KB + w.ks);
+      // the stage (its activation scales) has landed, and its MMAs are done
+      const bool ok = mbar_wait(&full[s], ph) && mbar_wait(&pfull[q], qph);
+      tc::tc_fence_after();
+      if (!ok || *(volatile int *)s_abort) break;
+      const float *sa = reinterpret_cast<const float *>(smem + s * C::STAGE + C::SA_OFF);
+#pragma unroll
+      for (int c0 = 0; c0 < BNT; c0 += 16) {
+        float v[16];
+        tc::tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(q * BNT + c0), v);
+#pragma unroll
+        for (int i = 0; i < 16; i += 4) {
+          const float4 a4 = *reinterpret_cast<const float4 *>(sa + c0 + i);
+          acc[c0 + i] = fmaf(v[i], __fmul_rn(sw, a4.x), acc[c0 + i]);
+          acc[c0 + i + 1] = fmaf(v[i + 1], __fmul_rn(sw, a4.y), acc[c0 + i + 1]);
+          acc[c0 + i + 2] = fmaf(v[i + 2], __fmul_rn(sw, a4.z), acc[c0 + i + 2]);
+          acc[c0 + i + 3] = fmaf(v[i + 3], __fmul_rn(sw, a4.w), acc[c0 + i + 3]);
+        }
+      }
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&pempty[q]);
+        mbar_arrive(&sfree[s]);
+      }
+      if (w.seg_last) {
+        const bool whole = (ks0 == 0) && (w.ks == p.KB - 1);
+        f8b_finish<BNT>(p, tile_info(t0), t0, whole, ks0 > 0, acc, cta, warp, lane, total);
+      }
+      if (++s == NS) { s = 0; ph ^= 1; }
+      if (++q == NP) { q = 0; qph ^= 1; }
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc::tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS));
+  }
+}
+
+// Activation scales per token tile for the block-scaled FP8 kernel: out
+// [slots][kst][bnt] fp32 with out[q][ks][n] = the scale of the tile's row n
+// for stage ks (0 past the slot's valid rows).  Dense: slot q = rows
+// [q * bnt, q * bnt + bnt); MoE: as bs_sf_tiles_kernel, expert-sorted row r
+// reads caller row perm[r] / div.  One thread per output value.
+__global__ void f8b_sa_tiles_kernel(int slots, int bnt, int kst, const float *__restrict__ sa, int M, int moe, int E,
+                                    const int32_t *__restrict__ offsets, const int32_t *__restrict__ perm, int div,
+                                    float *__restrict__ out) {
+  extern __shared__ int tpre[];
+  bool routed_ok = true;
+  if (moe) {
+    routed_ok = offsets[E] >= 0;
+    if (threadIdx.x < 32) {
+      const int lane = threadIdx.x;
+      int running = 0;
+      for (int e0 = 0; e0 < E; e0 += 32) {
+        const int e = e0 + lane;
+        int tiles = 0;
+        if (e < E && routed_ok) tiles = (offsets[e + 1] - offsets[e] + bnt - 1) / bnt;
+        int incl = tiles;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        if (e < E) tpre[e + 1] = running + incl;
+        running += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      if (lane == 0) tpre[0] = 0;
+    }
+    __syncthreads();
+  }
+  const size_t total = (size_t)slots * kst * bnt;
+  for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < total;
+       idx += (size_t)gridDim.x * blockDim.x) {
+    const int n = (int)(idx % bnt);
+    const size_t rest = idx / bnt;
+    const int ks = (int)(rest % kst);
+    const int q = (int)(rest / kst);
+    int src = -1;
+    if (!moe) {
+      const int row = q * bnt + n;
+      if (row < M) src = row;
+    } else if (routed_ok && q < tpre[E]) {
+      int lo = 0, hi = E;
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (tpre[mid] <= q) lo = mid;
+        else hi = mid;
+      }
+      const int row = offsets[lo] + (q - tpre[lo]) * bnt + n;
+      if (row < offsets[lo + 1]) src = perm[row] / div;
+    }
+    out[idx] = src >= 0 ? sa[(size_t)src * kst + ks] : 0.f;
+  }
+}
+
 }  // namespace bs
 
 // ---- host side -------------------------------------------------------------------
@@ -661,6 +1055,23 @@ static hq_status bs_launch_one(const CUtensorMap &wm, const CUtensorMap &am, con
   return check_launch();
 }
 
+template <int BNT>
+static hq_status bsf_launch_one(const CUtensorMap &wm, const CUtensorMap &am, const tc::Params &p, const TcLaunch &t,
+                                cudaStream_t st) {
+  using C = bs::CfgF8B<BNT>;
+  auto kern = bs::bsf_gemm_kernel<BNT>;
+  static unsigned configured = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return HQ_ERR_CUDA;
+  if (dev >= 32 || !(configured & (1u << dev))) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::BYTES) != cudaSuccess)
+      return HQ_ERR_CUDA;
+    if (dev < 32) configured |= 1u << dev;
+  }
+  kern<<<t.nctas, bs::THREADS, C::BYTES, st>>>(wm, am, p);
+  return check_launch();
+}
+
 template <int KIND>
 static hq_status bs_launch_kind(const CUtensorMap &wm, const CUtensorMap &am, const tc::Params &p,
                                 const TcLaunch &t, cudaStream_t st) {
@@ -680,6 +1091,7 @@ static hq_status bs_launch_kind(const CUtensorMap &wm, const CUtensorMap &am, co
 
 size_t bs_sf_tiles_bytes(const Layout &L, const TcLaunch &t) {
   if (L.bs == BS_NONE || L.bs == BS_F8) return 0;
+  if (L.bs == BS_F8B) return (size_t)t.mtiles * (L.K / 128) * t.bnt * 4;
   const int kstage = L.bs == BS_MX ? 128 : 256;
   const int sf_ch = L.bs == BS_MX ? 1 : 4;
   return (size_t)t.mtiles * (L.K / kstage) * sf_ch * (t.bnt > 128 ? 1024 : 512);
@@ -704,7 +1116,16 @@ hq_status launch_bs_gemm(const Layout &L, const void *packed, int E, const void 
   CUtensorMap wm, am;
   if (!make_bs_weight_map(&wm, L, packed, E)) return HQ_ERR_CUDA;
   if (!make_bs_act_map(&am, a_codes, a_rows, row_bytes, t.bnt)) return HQ_ERR_CUDA;
-  if (L.bs != BS_F8) {
+  if (L.bs == BS_F8B) {
+    // activation scales per token tile and stage: [mtiles][K / 128][bnt] fp32
+    const size_t n = (size_t)t.mtiles * (L.K / 128) * t.bnt;
+    size_t blocks = (n + 255) / 256;
+    if (blocks > 148 * 8) blocks = 148 * 8;
+    bs::f8b_sa_tiles_kernel<<<(int)blocks, 256, moe ? (E + 1) * sizeof(int) : 0, st>>>(
+        t.mtiles, t.bnt, L.K / 128, (const float *)a_scales, M, moe, E, offsets, perm, a_div, (float *)sf_tiles);
+    const hq_status s = check_launch();
+    if (s != HQ_OK) return s;
+  } else if (L.bs != BS_F8) {
     const size_t words = (size_t)t.mtiles * (L.K / kstage) * sf_ch * (t.bnt > 128 ? 256 : 128);
     size_t blocks = (words + 255) / 256;
     if (blocks > 148 * 8) blocks = 148 * 8;
@@ -748,6 +1169,15 @@ hq_status launch_bs_gemm(const Layout &L, const void *packed, int E, const void 
   p.partial = (float *)((uint8_t *)workspace + tc_counter_bytes(t));
   if (L.bs == BS_MX) return bs_launch_kind<BS_MX>(wm, am, p, t, st);
   if (L.bs == BS_F8) return bs_launch_kind<BS_F8>(wm, am, p, t, st);
+  if (L.bs == BS_F8B) {
+    switch (t.bnt) {
+      case 16: return bsf_launch_one<16>(wm, am, p, t, st);
+      case 32: return bsf_launch_one<32>(wm, am, p, t, st);
+      case 64: return bsf_launch_one<64>(wm, am, p, t, st);
+      case 128: return bsf_launch_one<128>(wm, am, p, t, st);
+      default: return HQ_ERR_UNSUPPORTED;
+    }
+  }
   return bs_launch_kind<BS_NV>(wm, am, p, t, st);
 }
 

@@ -42,12 +42,14 @@ namespace hq {
 // kernels see INT4.
 enum WFmt : int {
   W_INT4 = 0, W_UINT4 = 1, W_MXFP4 = 2, W_NVFP4 = 3, W_FP8 = 4, W_MXINT4 = 5,
-  W_INT2 = 6, W_UINT2 = 7, W_INT3 = 8, W_UINT3 = 9, W_E2M3 = 10, W_E3M2 = 11, W_E0M3 = 12, W_NFMT = 13
+  W_INT2 = 6, W_UINT2 = 7, W_INT3 = 8, W_UINT3 = 9, W_E2M3 = 10, W_E3M2 = 11, W_E0M3 = 12,
+  W_FP8B = 13,  // E4M3 with one fp32 scale per 128 x 128 block (rows x k)
+  W_NFMT = 14
 };
 
 // Bits per stored weight code of a format.
 __host__ __device__ constexpr int fmt_bits(int fmt) {
-  return fmt == W_FP8 ? 8 : (fmt == W_INT2 || fmt == W_UINT2) ? 2 : (fmt == W_INT3 || fmt == W_UINT3) ? 3
+  return (fmt == W_FP8 || fmt == W_FP8B) ? 8 : (fmt == W_INT2 || fmt == W_UINT2) ? 2 : (fmt == W_INT3 || fmt == W_UINT3) ? 3
          : (fmt == W_E2M3 || fmt == W_E3M2) ? 6 : 4;
 }
 __host__ __device__ constexpr bool fmt_lowbit(int fmt) { return fmt >= W_INT2 && fmt <= W_E3M2; }
@@ -65,15 +67,16 @@ __host__ __device__ constexpr bool fmt_bf16_scales(int fmt) {
 // even k in bits 0..15, odd in 16..31; the high bit of 3-bit codes).
 __host__ __device__ constexpr int plane2_off(int fmt) { return (fmt == W_E2M3 || fmt == W_E3M2) ? 4096 : 0; }
 __host__ __device__ constexpr int plane1_off(int fmt) { return (fmt == W_INT3 || fmt == W_UINT3) ? 2048 : 0; }
-// Internal activation formats.
-enum AFmt : int { A_BF16 = 0, A_FP8 = 1, A_MXFP8 = 2, A_NVFP4 = 3 };
+// Internal activation formats (A_FP8G: E4M3 with an fp32 scale per token and
+// 128 k).
+enum AFmt : int { A_BF16 = 0, A_FP8 = 1, A_MXFP8 = 2, A_NVFP4 = 3, A_FP8G = 4 };
 
 constexpr int TILE_N = 128;  // rows of W per tile (the MMA M dimension)
 constexpr int TILE_K = 64;   // k per k-block
 
 // Block-scaled layouts: weights that the tensor core consumes as they are
 // (no dequantisation), with the block scales next to them.
-enum { BS_NONE = 0, BS_MX = 1, BS_NV = 2, BS_F8 = 3 };
+enum { BS_NONE = 0, BS_MX = 1, BS_NV = 2, BS_F8 = 3, BS_F8B = 4 };
 
 struct Layout {
   int fmt;
@@ -102,7 +105,7 @@ struct Layout {
   }
   __host__ __device__ int chunks() const { return wbits == 4 ? 2 : 4; }
   // code bytes per weight row of the block-scaled / FP8 layouts
-  __host__ __device__ size_t bs_row_bytes() const { return bs == BS_F8 ? (size_t)K : (size_t)K / 2; }
+  __host__ __device__ size_t bs_row_bytes() const { return (bs == BS_F8 || bs == BS_F8B) ? (size_t)K : (size_t)K / 2; }
   // ... stored in chunks of this many bytes per row: one MMA stage (MX: 128
   // codes = 64 bytes; NV: 256 codes, F8: 128 codes = 128 bytes)
   __host__ __device__ int bs_chunk_bytes() const { return bs == BS_MX ? 64 : 128; }
@@ -141,7 +144,9 @@ inline bool weight_format(const hq_quant_desc *d, int *fmt) {
       if (d->w_scale_dtype == HQ_UE4M3 && d->w_group == 16 && d->w_has_global) { *fmt = W_NVFP4; return true; }
       return false;
     case HQ_E4M3:
-      if (d->w_scale_dtype != HQ_FP32 || d->w_group != 0 || d->w_has_zero || d->w_has_global) return false;
+      if (d->w_scale_dtype != HQ_FP32 || d->w_has_zero || d->w_has_global) return false;
+      if (d->w_group == 128) { *fmt = W_FP8B; return true; }  // 128 x 128 blocks
+      if (d->w_group != 0) return false;
       *fmt = W_FP8;
       return true;
     case HQ_INT2:
@@ -178,7 +183,9 @@ inline bool valid_k(const hq_quant_desc *d, int K) {
 inline bool act_format(const hq_quant_desc *d, int *afmt) {
   switch (d->a_dtype) {
     case HQ_BF16: *afmt = A_BF16; return d->a_group == 0;
-    case HQ_E4M3: *afmt = A_FP8; return d->a_group == 0;
+    case HQ_E4M3:
+      *afmt = d->a_group == 128 ? A_FP8G : A_FP8;
+      return d->a_group == 0 || d->a_group == 128;
     case HQ_MXFP8: *afmt = A_MXFP8; return d->a_group == 0 || d->a_group == 32;
     case HQ_NVFP4: *afmt = A_NVFP4; return d->a_group == 0 || d->a_group == 16;
     default: return false;
@@ -216,13 +223,14 @@ inline Layout make_layout(int fmt, int group, int N, int K, int bs = BS_NONE) {
   L.w_bytes = (size_t)L.NT * L.KB * L.unit_bytes();
   L.s_bytes = (fmt == W_FP8) ? 0 : (size_t)L.NT * L.G * TILE_N * L.sbytes;
   L.z_bytes = fmt_zero(fmt) ? (size_t)L.NT * L.G * TILE_N : 0;
+  if (fmt == W_FP8B) L.s_bytes = 0;
   L.c_bytes = (fmt == W_FP8) ? (size_t)L.NT * TILE_N * 4 : 0;
   L.g_bytes = (fmt == W_NVFP4) ? 16 : 0;
   if (bs != BS_NONE) {
     L.w_bytes = (size_t)L.NT * TILE_N * L.bs_row_bytes();
-    L.s_bytes = bs == BS_F8 ? 0 : (size_t)L.NT * (K / (4 * L.group)) * 512;
+    L.s_bytes = (bs == BS_F8 || bs == BS_F8B) ? 0 : (size_t)L.NT * (K / (4 * L.group)) * 512;
     L.z_bytes = 0;
-    L.c_bytes = bs == BS_F8 ? (size_t)L.NT * TILE_N * 4 : 0;
+    L.c_bytes = bs == BS_F8 ? (size_t)L.NT * TILE_N * 4 : bs == BS_F8B ? (size_t)L.NT * (K / 128) * 4 : 0;
   }
   size_t off = 0;
   L.w_off = off; off = align_up(off + L.w_bytes, 256);
@@ -243,8 +251,17 @@ inline Layout layout_for(const hq_quant_desc *d, int fmt, int N, int K) {
     if (fmt == W_MXFP4 && afmt == A_MXFP8 && (K % 128) == 0) bs = BS_MX;
     if (fmt == W_NVFP4 && afmt == A_NVFP4 && (K % 256) == 0) bs = BS_NV;
     if (fmt == W_FP8 && afmt == A_FP8 && (K % 128) == 0) bs = BS_F8;
+    if (fmt == W_FP8B && afmt == A_FP8G && (K % 128) == 0) bs = BS_F8B;
   }
   return make_layout(fmt, d->w_group, N, K, bs);
+}
+
+// Formats that exist only as a pair: block-scaled FP8 weights with per-128
+// FP8 activations (the block-scaled W8A8 of DeepGEMM-style MoE), on the
+// TMA-fed kernel.
+inline bool pair_supported(const Layout &L, int afmt) {
+  if (L.fmt == W_FP8B || afmt == A_FP8G) return L.bs == BS_F8B;
+  return true;
 }
 
 // Device-side error word (one per device, module scope).  The library is

@@ -236,6 +236,13 @@ __global__ void pack_bs_side_kernel(Layout L, int E, const uint8_t *scales, cons
           (r < L.N) ? reinterpret_cast<const float *>(scales)[(size_t)e * L.N + L.std_row(r)] : 0.f;
       continue;
     }
+    if (L.bs == BS_F8B) {
+      // one fp32 scale per (128-row tile, 128 k): standard [E][NT][K / 128]
+      if (i == 0)
+        reinterpret_cast<float *>(base + L.c_off)[(size_t)nt * L.G + gi] =
+            reinterpret_cast<const float *>(scales)[((size_t)e * L.NT + nt) * L.G + gi];
+      continue;
+    }
     const uint8_t sv = (r < L.N) ? scales[((size_t)e * L.N + L.std_row(r)) * L.G + gi] : (uint8_t)0;
     base[L.s_off + ((size_t)nt * (L.G / 4) + gi / 4) * 512 + bs_sf_offset(i, gi & 3)] = sv;
     if (L.fmt == W_NVFP4 && r == 0 && gi == 0) reinterpret_cast<float *>(base + L.g_off)[0] = global_scale[e];
@@ -269,6 +276,12 @@ __global__ void unpack_bs_kernel(Layout L, int E, const uint8_t *packed, uint8_t
       const uint8_t *base = packed + (size_t)e * L.stride;
       if (L.bs == BS_F8) {
         reinterpret_cast<float *>(scales)[(size_t)e * L.N + r] = reinterpret_cast<const float *>(base + L.c_off)[pr];
+        continue;
+      }
+      if (L.bs == BS_F8B) {
+        if ((r % TILE_N) == 0)
+          reinterpret_cast<float *>(scales)[((size_t)e * L.NT + r / TILE_N) * L.G + gi] =
+              reinterpret_cast<const float *>(base + L.c_off)[(size_t)(r / TILE_N) * L.G + gi];
         continue;
       }
       scales[j] = base[L.s_off + ((size_t)nt * (L.G / 4) + gi / 4) * 512 + bs_sf_offset(i, gi & 3)];

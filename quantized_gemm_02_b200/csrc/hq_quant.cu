@@ -107,6 +107,27 @@ __global__ void quant_fp8_token_kernel(int M, int K, const uint16_t *__restrict_
   }
 }
 
+// ---- FP8 per token and 128 k ------------------------------------------------
+// One warp per (row, 128-k group), 4 values per lane: s = amax / 448 (1 for
+// an all-zero group), q = e4m3(x / s), as the per-token recipe on each group.
+__global__ void quant_fp8_group_kernel(size_t ngroups, const uint16_t *__restrict__ x, uint8_t *__restrict__ q,
+                                       float *__restrict__ scales) {
+  const int lane = threadIdx.x & 31;
+  const size_t warps = (size_t)gridDim.x * (blockDim.x >> 5);
+  for (size_t g = blockIdx.x * (size_t)(blockDim.x >> 5) + (threadIdx.x >> 5); g < ngroups; g += warps) {
+    const uint2 v = reinterpret_cast<const uint2 *>(x + g * 128)[lane];
+    const float f[4] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y)};
+    float amax = fmaxf(fmaxf(fabsf(f[0]), fabsf(f[1])), fmaxf(fabsf(f[2]), fabsf(f[3])));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float s = (amax == 0.f) ? 1.f : __fdiv_rn(amax, 448.f);
+    const uint32_t a = f32x2_to_e4m3x2(__fdiv_rn(f[0], s), __fdiv_rn(f[1], s));
+    const uint32_t b = f32x2_to_e4m3x2(__fdiv_rn(f[2], s), __fdiv_rn(f[3], s));
+    reinterpret_cast<uint32_t *>(q + g * 128)[lane] = a | (b << 16);
+    if (lane == 0) scales[g] = s;
+  }
+}
+
 // ---- MXFP8 -----------------------------------------------------------------
 // One thread per 32-element block.
 __global__ void quant_mxfp8_kernel(size_t nblocks, const uint16_t *__restrict__ x, uint8_t *__restrict__ q,
@@ -303,6 +324,11 @@ hq_status launch_quant_act(int afmt, int M, int K, const void *x, void *codes, v
     case A_FP8:
       quant_fp8_token_kernel<<<M, 256, 0, st>>>(M, K, xb, (uint8_t *)codes, (float *)scales);
       break;
+    case A_FP8G: {
+      const size_t ng = (size_t)M * K / 128;
+      quant_fp8_group_kernel<<<quant_grid(ng * 32, 256), 256, 0, st>>>(ng, xb, (uint8_t *)codes, (float *)scales);
+      break;
+    }
     case A_MXFP8: {
       const size_t nb = (size_t)M * K / 32;
       quant_mxfp8_kernel<<<quant_grid(nb, 128), 128, 0, st>>>(nb, xb, (uint8_t *)codes, (uint8_t *)scales);

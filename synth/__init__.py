@@ -36,7 +36,7 @@ import torch
 __all__ = [
     "generator", "bf16_normal", "random_bytes", "int4_weights", "lowbit_weights", "mxint4_weights",
     "mxfp4_weights",
-    "nvfp4_weights_random", "fp8_weights_random", "routing_softmax_topk", "routing_zipf",
+    "nvfp4_weights_random", "fp8_weights_random", "fp8_block_weights", "routing_softmax_topk", "routing_zipf",
     "pack_nibbles_i32", "pack_nibbles_u8", "to_np_bits",
 ]
 
@@ -178,6 +178,15 @@ def fp8_weights_random(E: int, N: int, K: int, gen: torch.Generator, device: str
     codes = (r + (r >= 0x7F).to(torch.int32)).to(torch.uint8)
     sc = torch.randn(E, N, generator=gen, dtype=torch.float32, device=device).abs() * 0.01 + 1e-3
     return {"codes": codes, "scales": sc}
+
+
+def fp8_block_weights(E: int, N: int, K: int, gen: torch.Generator, device: str = "cpu") -> dict:
+    """E4M3 codes uniform over the 254 finite codes; one fp32 scale per 128
+    rows x 128 k, |N(0, 0.01)| + 1e-3: scales [E, ceil(N / 128), K / 128]."""
+    r = torch.randint(0, 254, (E, N, K), generator=gen, dtype=torch.int32, device=device)
+    codes = (r + (r >= 0x7F).to(torch.int32)).to(torch.uint8)
+    sc = torch.randn(E, (N + 127) // 128, K // 128, generator=gen, dtype=torch.float32, device=device).abs() * 0.01
+    return {"codes": codes, "scales": sc + 1e-3}
 
 
 def routing_softmax_topk(T: int, E: int, k: int, gen: torch.Generator, device: str = "cpu"):

@@ -46,15 +46,21 @@ WFORMATS = {
              dict(w_dtype="e3m2", w_group=32, w_scale="e8m0")),
     "e0m3_g128": (dict(w_dtype=16, w_group=128, w_scale_dtype=0, w_has_zero=0, w_has_global=0),
                   dict(w_dtype="e0m3", w_group=128, w_scale="bf16")),
+    # block-scaled FP8 (128 x 128 weight blocks); only with "fp8g" activations
+    "fp8b": (dict(w_dtype=5, w_group=128, w_scale_dtype=1, w_has_zero=0, w_has_global=0),
+             dict(w_dtype="e4m3", w_group=128, w_scale="fp32")),
 }
+PAIR_ONLY = {"fp8b": "fp8g"}  # weight formats that exist with one activation format only
 LOWBIT = {"int2_g64": 2, "uint2_g32": 2, "int3_g128": 3, "uint3_g64": 3, "e2m3": 6, "e3m2": 6, "e0m3_g128": 4}
-AFORMATS = {"bf16": 0, "fp8": 5, "mxfp8": 8, "nvfp4": 9}
+AFORMATS = {"bf16": 0, "fp8": 5, "mxfp8": 8, "nvfp4": 9, "fp8g": 5}
+AGROUP = {"fp8g": 128}  # E4M3 with an fp32 scale per token and 128 k
 
 
 def cdesc(wname: str, aname: str = "bf16"):
     import quantized_gemm_02_b200 as hq
     d = hq.QuantDesc(**WFORMATS[wname][0])
     d.a_dtype = AFORMATS[aname]
+    d.a_group = AGROUP.get(aname, 0)
     return d
 
 
@@ -68,6 +74,9 @@ def make_weights(wname: str, E: int, N: int, K: int, seed: int = 0, device: str 
     fields, _ = WFORMATS[wname]
     if wname == "mxint4":
         w = synth.mxint4_weights(E, N, K, g, device=device)
+        return {"codes": w["codes"], "scales": w["scales"], "zeros": None, "global": None}
+    if wname == "fp8b":
+        w = synth.fp8_block_weights(E, N, K, g, device)
         return {"codes": w["codes"], "scales": w["scales"], "zeros": None, "global": None}
     if wname in LOWBIT:
         w = synth.lowbit_weights(E, N, K, LOWBIT[wname], fields["w_group"], bool(fields["w_has_zero"]),
@@ -99,6 +108,10 @@ def oracle_decoder(wname: str, w: dict, N: int, K: int):
     glob = np_bits(w["global"])
 
     def dec(e, rows=None):
+        if wname == "fp8b":
+            # block scales: the rows' own scale rows
+            rr = np.arange(N) if rows is None else np.asarray(rows)
+            return O.decode_fp8_block_weights(codes[e][rr], scales[e][rr // 128], 128, row_block=1), None
         c, s = codes[e], scales[e]
         z = None if zeros is None else zeros[e]
         if rows is not None:
@@ -126,6 +139,9 @@ def gpu_pack(wname: str, w: dict, E: int, N: int, K: int, aname: str = "bf16"):
 
 def act_storage(aname: str, M: int, K: int, device="cuda"):
     """Empty code / scale tensors for a quantised activation format."""
+    if aname == "fp8g":
+        return (torch.empty(M, K, dtype=torch.uint8, device=device),
+                torch.empty(M, K // 128, dtype=torch.float32, device=device))
     if aname == "fp8":
         return (torch.empty(M, K, dtype=torch.uint8, device=device), torch.empty(M, dtype=torch.float32, device=device))
     if aname == "mxfp8":
@@ -147,6 +163,9 @@ def gpu_quant(aname: str, x: torch.Tensor, static_global=None):
 
 
 def oracle_quant(aname: str, x_bits: np.ndarray):
+    if aname == "fp8g":
+        q, s = O.quant_fp8_block(x_bits)
+        return q, s, None
     if aname == "fp8":
         q, s = O.quant_fp8_per_token(x_bits)
         return q, s, None

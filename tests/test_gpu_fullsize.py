@@ -50,6 +50,10 @@ def _weight_rows(wname, w, rows, K):
     standard-format tensors (which may live on the GPU)."""
     idx = torch.as_tensor(np.asarray(rows), device=w["codes"].device)
     c = np_bits(w["codes"][0][idx])
+    if wname == "fp8b":
+        # block scales: each row's own 128-row block scale row
+        s = np_bits(w["scales"][0][idx // 128])
+        return O.decode_fp8_block_weights(c, s, 128, row_block=1), None
     s = np_bits(w["scales"][0][idx])
     z = None if w["zeros"] is None else np_bits(w["zeros"][0][idx])
     g = None if w["global"] is None else np_bits(w["global"])[0]
@@ -172,6 +176,19 @@ def test_config5_large_m(aname, M):
     _check_dense(wname, aname, w, x, C, M, N, K, seed=M, glob=glob)
 
 
+@pytest.mark.parametrize("M", [32, 2048])
+def test_fp8_block_scaled_dense(M):
+    # block-scaled FP8 W8A8 at N = K = 7168 (128 x 128 weight blocks, per
+    # token and 128 k activation scales quantised on the GPU)
+    N = K = 7168
+    w = make_weights("fp8b", 1, N, K, seed=750 + M, device="cuda")
+    packed = gpu_pack("fp8b", w, 1, N, K, "fp8g")
+    x = synth.bf16_normal((M, K), synth.generator(751 + M, "cuda"), device="cuda")
+    ac, asc, _ = gpu_quant("fp8g", x)
+    C = _run_dense("fp8b", "fp8g", packed, ac, asc, None, M, N, K)
+    _check_dense("fp8b", "fp8g", w, x, C, M, N, K, seed=M)
+
+
 @pytest.mark.parametrize("M", [2048, 8192])
 def test_mxfp4_mxfp8_dense_large_m(M):
     # MXFP4 weights x MXFP8 activations on the block-scaled MMA at N = K = 7168
@@ -215,8 +232,9 @@ def _moe_full(wname, aname, T, part, zipf, seed, modes=(0, 1)):
         if v is None:
             sub[key] = (None, None, None)
             continue
-        sub[key] = (np_bits(v[:, torch.as_tensor(cols, device="cuda")]),
-                    np_bits(v[:, torch.as_tensor(cols2, device="cuda")]),
+        div = 128 if (wname == "fp8b" and key == "scales") else 1  # block scales: one row per 128
+        sub[key] = (np_bits(v[:, torch.as_tensor(cols // div, device="cuda")]),
+                    np_bits(v[:, torch.as_tensor(cols2 // div, device="cuda")]),
                     {int(e): np_bits(v[int(e)]) for e in full_experts})
     glob = None if w["global"] is None else np_bits(w["global"])
     del w
@@ -253,6 +271,8 @@ def _moe_full(wname, aname, T, part, zipf, seed, modes=(0, 1)):
     def dec_from(which, e, n):
         # which: 0 = the sampled columns, 1 = the element columns, 2 = whole experts
         c, s, z = (sub["codes"][which], sub["scales"][which], sub["zeros"][which])
+        if wname == "fp8b" and which != 2:
+            return O.decode_fp8_block_weights(c[e], s[e], 128, row_block=1), None
         return O.decode_weights(od, n, K, c[e], s[e], None if z is None else z[e], None if glob is None else glob[e])
 
     out_c, bound_c, Y, B = O.moe(A_slots, ids_np, wts.cpu().numpy(), lambda e: dec_from(0, e, len(cols)), 1.0,
@@ -306,6 +326,12 @@ def test_config4_moe_w4a8_zipf(T, part):
 def test_moe_w4a16_mxint4(T, part):
     # MXINT4 weights (INT4 elements, E8M0 per 32) at the config-3 MoE shapes
     _moe_full("mxint4", "bf16", T, part, zipf=False, seed=1100 + T)
+
+
+def test_moe_fp8_block_scaled():
+    # block-scaled FP8 W8A8 MoE (the DeepGEMM-style layout) at the config-3
+    # gate-up shape, T = 1024
+    _moe_full("fp8b", "fp8g", 1024, "gate_up", zipf=False, seed=1200)
 
 
 @pytest.mark.parametrize("part", ["gate_up", "down"])

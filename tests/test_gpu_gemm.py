@@ -10,7 +10,7 @@ import torch
 
 import oracle as O
 import synth
-from hqtest import (WFORMATS, assert_close, cdesc, gpu_pack, gpu_quant, make_weights, np_bits, odesc,
+from hqtest import (PAIR_ONLY, WFORMATS, assert_close, cdesc, gpu_pack, gpu_quant, make_weights, np_bits, odesc,
                     oracle_decoder, oracle_quant)
 
 pytestmark = pytest.mark.gpu
@@ -52,7 +52,7 @@ def parity(wname, aname, M, N, K, seed=0, cols=None, rows=None):
     return assert_close(got, ref, bound, what=f"{wname}x{aname} M={M} N={N} K={K}")
 
 
-@pytest.mark.parametrize("wname", list(WFORMATS))
+@pytest.mark.parametrize("wname", [w for w in WFORMATS if w not in PAIR_ONLY])
 @pytest.mark.parametrize("M", [1, 7, 16, 33])
 def test_gemm_bf16_acts_small(wname, M):
     parity(wname, "bf16", M, 200, 512, seed=M)
@@ -66,6 +66,15 @@ def test_gemm_bf16_acts_small(wname, M):
 @pytest.mark.parametrize("M", [1, 16, 40])
 def test_gemm_quantised_acts_small(wname, aname, M):
     parity(wname, aname, M, 136, 256, seed=10 + M)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 200, 512), (16, 200, 512), (40, 136, 1024), (300, 200, 512),
+                                   (129, 2048, 384), (5, 512, 8192)])
+def test_gemm_fp8_block_scaled(M, N, K):
+    # FP8 weights with 128 x 128 block scales x FP8 activations with per-(token,
+    # 128 k) scales: per-stage accumulators promoted with both scales in fp32;
+    # whole tiles, Stream-K pieces and the fixup (5 x 512 x 8192: many pieces)
+    parity("fp8b", "fp8g", M, N, K, seed=80 + M)
 
 
 def test_gemm_large_token_count():

@@ -87,7 +87,8 @@ def moe_case(wname, aname, T, E, k, N, K, a_per_slot, seed, zipf=False, device_w
 
 
 @pytest.mark.parametrize("wname,aname", [("mxfp4", "bf16"), ("int4_g128", "bf16"), ("uint4_g64", "bf16"),
-                                         ("mxfp4", "mxfp8"), ("nvfp4", "nvfp4"), ("fp8", "fp8"), ("mxint4", "bf16")])
+                                         ("mxfp4", "mxfp8"), ("nvfp4", "nvfp4"), ("fp8", "fp8"), ("mxint4", "bf16"),
+                                         ("fp8b", "fp8g"), ("int3_g128", "bf16"), ("e3m2", "bf16")])
 @pytest.mark.parametrize("a_per_slot", [0, 1])
 def test_moe_small(wname, aname, a_per_slot):
     T, E, k, N, K = 23, 16, 4, 96, 256
@@ -101,7 +102,7 @@ def test_moe_small(wname, aname, a_per_slot):
     assert_close(res[(0, 1)].cpu(), out, bound, rel=8e-3, what="combined")
 
 
-@pytest.mark.parametrize("wname,aname", [("nvfp4", "nvfp4"), ("mxfp4", "mxfp8"), ("fp8", "fp8")])
+@pytest.mark.parametrize("wname,aname", [("nvfp4", "nvfp4"), ("mxfp4", "mxfp8"), ("fp8", "fp8"), ("fp8b", "fp8g")])
 def test_moe_block_scaled_wide_token_tiles(wname, aname):
     # ~150 routed rows per expert: NVFP4 x NVFP4 takes 192-token tiles
     # (activation scale chunks of two 128-row halves), the other pairs
@@ -129,7 +130,7 @@ def test_moe_indexed_multi_stage_tiles(wname, aname, T):
 
 
 @pytest.mark.parametrize("wname,aname", [("mxfp4", "mxfp8"), ("nvfp4", "nvfp4"), ("int4_g128", "fp8"), ("fp8", "fp8"),
-                                         ("mxfp4", "bf16")])
+                                         ("mxfp4", "bf16"), ("fp8b", "fp8g")])
 @pytest.mark.parametrize("mode", [0, 1])
 def test_moe_caller_quantised_and_self_routed(wname, aname, mode):
     # activations quantised by the caller (hq_quant_act) and passed with

@@ -5,12 +5,12 @@ import torch
 
 import oracle as O
 import synth
-from hqtest import WFORMATS, cdesc, gpu_pack, gpu_quant, make_weights, np_bits, oracle_quant
+from hqtest import PAIR_ONLY, WFORMATS, cdesc, gpu_pack, gpu_quant, make_weights, np_bits, oracle_quant
 
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("wname", list(WFORMATS))
+@pytest.mark.parametrize("wname", [w for w in WFORMATS if w not in PAIR_ONLY])
 def test_pack_unpack_identity(wname):
     import quantized_gemm_02_b200 as hq
     E, N, K = 2, 80, 384  # ragged N (pads to 128 rows), 6 k-blocks
@@ -33,7 +33,7 @@ def test_pack_unpack_identity(wname):
         assert np.array_equal(np_bits(out[k]), want), k
 
 
-@pytest.mark.parametrize("wname,aname", [("mxfp4", "mxfp8"), ("nvfp4", "nvfp4"), ("fp8", "fp8")])
+@pytest.mark.parametrize("wname,aname", [("mxfp4", "mxfp8"), ("nvfp4", "nvfp4"), ("fp8", "fp8"), ("fp8b", "fp8g")])
 def test_pack_unpack_identity_block_scaled(wname, aname):
     # block-scaled layouts (chosen by the activation format): codes row-major,
     # scales in 512-byte chunks; FP8 x FP8: E4M3 bytes row-major, row scales
@@ -56,7 +56,7 @@ def test_pack_unpack_identity_block_scaled(wname, aname):
     per_e = hq.hq_packed_weights_bytes(d, 1, N, K)
     p0 = packed[:per_e].cpu().numpy()
     codes = w["codes"][0].numpy() if hasattr(w["codes"], "numpy") else w["codes"][0].cpu().numpy()
-    rb = K if wname == "fp8" else K // 2
+    rb = K if wname in ("fp8", "fp8b") else K // 2
     cb = 64 if wname == "mxfp4" else 128
     rows = p0[: 128 * rb].reshape(rb // cb, 128, cb).transpose(1, 0, 2).reshape(128, rb)
     assert np.array_equal(rows[:N], codes.reshape(N, rb))
@@ -81,7 +81,7 @@ def _acts(M, K, seed):
     return x
 
 
-@pytest.mark.parametrize("aname", ["fp8", "mxfp8", "nvfp4"])
+@pytest.mark.parametrize("aname", ["fp8", "mxfp8", "nvfp4", "fp8g"])
 @pytest.mark.parametrize("shape", [(37, 512), (5, 7168)])
 def test_quant_act_bit_exact(aname, shape):
     M, K = shape
@@ -90,7 +90,7 @@ def test_quant_act_bit_exact(aname, shape):
     torch.cuda.synchronize()
     q, s, og = oracle_quant(aname, np_bits(x))
     assert np.array_equal(codes.cpu().numpy(), q)
-    if aname == "fp8":
+    if aname in ("fp8", "fp8g"):
         assert np.array_equal(scales.cpu().numpy().view(np.uint32), s.view(np.uint32))
     else:
         assert np.array_equal(scales.cpu().numpy(), s)

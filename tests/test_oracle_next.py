@@ -128,3 +128,21 @@ def test_mxint4_through_decode_weights_equals_int4_with_power_of_two_scales():
     bf16_scales = (sc.astype(np.uint16) << 7).astype(np.uint16)
     Wi, _ = O.decode_weights(O.Desc("int4", 32, "bf16"), N, K, codes, bf16_scales)
     assert np.array_equal(Wm, Wi)
+
+
+def test_fp8_block_weights_by_rows_and_through_decode_weights():
+    # decoding chosen rows with their own block-scale rows (row_block = 1)
+    # gives those rows of the whole-matrix decode; the unified description
+    # (E4M3, group 128, fp32 scales) routes to the block decoder
+    N, K = 300, 256
+    g = synth.generator(12)
+    w = synth.fp8_block_weights(1, N, K, g)
+    c, s = w["codes"][0].numpy(), w["scales"][0].numpy()
+    assert s.shape == (3, 2)
+    full = O.decode_fp8_block_weights(c, s)
+    rows = np.array([0, 127, 128, 299])
+    part = O.decode_fp8_block_weights(c[rows], s[rows // 128], 128, row_block=1)
+    assert np.array_equal(part, full[rows])
+    Wd, col = O.decode_weights(O.Desc("e4m3", 128, "fp32"), N, K, c, s)
+    assert col is None and np.array_equal(Wd, full)
+    assert full[200, 130] == O.E4M3[c[200, 130]] * float(s[1, 1])
