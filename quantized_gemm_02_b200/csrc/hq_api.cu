@@ -390,7 +390,7 @@ static hq_status pack_impl(const hq_quant_desc *desc, int E, int N, int K, const
   if (E < 1 || N < 1 || !valid_k(desc, K)) return HQ_ERR_INVALID_ARG;
   if (gated && (N % TILE_N) != 0) return HQ_ERR_INVALID_ARG;
   if (!codes || !scales || !packed) return HQ_ERR_INVALID_ARG;
-  if ((fmt == W_UINT4) != (zeros != nullptr)) return HQ_ERR_INVALID_ARG;
+  if (fmt_zero(fmt) != (zeros != nullptr)) return HQ_ERR_INVALID_ARG;
   if ((fmt == W_NVFP4) != (global_scale != nullptr)) return HQ_ERR_INVALID_ARG;
   if (!aligned16(codes) || !aligned16(packed) || ((uintptr_t)scales & 3u)) return HQ_ERR_INVALID_ARG;
   Layout L = layout_for(desc, fmt, N, K);
@@ -410,7 +410,7 @@ static hq_status unpack_impl(const hq_quant_desc *desc, int E, int N, int K, con
   if (E < 1 || N < 1 || !valid_k(desc, K)) return HQ_ERR_INVALID_ARG;
   if (gated && (N % TILE_N) != 0) return HQ_ERR_INVALID_ARG;
   if (!codes || !scales || !packed) return HQ_ERR_INVALID_ARG;
-  if ((fmt == W_UINT4) != (zeros != nullptr)) return HQ_ERR_INVALID_ARG;
+  if (fmt_zero(fmt) != (zeros != nullptr)) return HQ_ERR_INVALID_ARG;
   if ((fmt == W_NVFP4) != (global_scale != nullptr)) return HQ_ERR_INVALID_ARG;
   Layout L = layout_for(desc, fmt, N, K);
   int afmt;
