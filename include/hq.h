@@ -38,10 +38,10 @@
  *       UE4M3 scales      uint8 [E, N, K/16] (NVFP4) + fp32 global [E].
  *       E4M3 codes        uint8 [E, N, K] + fp32 per-channel scales [E, N]
  *                         (block-scaled: fp32 [E, ceil(N / 128), K / 128]).
- *       INT2/UINT2/INT3/UINT3/E2M3/E3M2/E0M3 codes (b bits): uint8
+ *       INT1/UINT1/INT2/UINT2/INT3/UINT3/E2M3/E3M2/E0M3 codes (b bits): uint8
  *                         [E, N, K * b / 8], a little-endian bit stream per
  *                         row (code k at bits b*k .. b*k + b - 1; for b = 4
- *                         the INT4 / E2M1 nibble order).  UINT2/UINT3 zero
+ *                         the INT4 / E2M1 nibble order).  UINT1/2/3 zero
  *                         points: uint8 [E, N, G], one per byte.  E0M3 code:
  *                         bit 3 = sign, bits 0..2 = magnitude.
  *   - Decoded values: INT4 w = (q - z) * s (z = 0 when symmetric; MXINT4
@@ -97,7 +97,9 @@ typedef enum {
   HQ_UINT3 = 13, /* unsigned 3-bit (with zero points)                      */
   HQ_E2M3 = 14,  /* FP6 (OCP MX), with E8M0 scales: MXFP6                  */
   HQ_E3M2 = 15,  /* FP6 (OCP MX), with E8M0 scales: MXFP6                  */
-  HQ_E0M3 = 16   /* float4e0m3: sign + 3-bit magnitude, no exponent bits   */
+  HQ_E0M3 = 16,  /* float4e0m3: sign + 3-bit magnitude, no exponent bits   */
+  HQ_INT1 = 17,  /* signed 1-bit, two's complement (codes 0, -1)           */
+  HQ_UINT1 = 18  /* unsigned 1-bit (with zero points)                      */
 } hq_dtype;
 
 /*
@@ -111,8 +113,8 @@ typedef enum {
  *   E4M3  + FP32 per-channel scales, w_group = 0            (FP8)
  *   E4M3  + FP32 scales per 128 x 128 block, w_group = 128  (block-scaled
  *         FP8, only with a_dtype E4M3 and a_group 128, K a multiple of 128)
- *   INT2, INT3, E0M3 + BF16 scales, w_group in {0, 32, 64, 128}
- *   UINT2, UINT3 + BF16 scales + zero points, w_group in {32, 64, 128}
+ *   INT1, INT2, INT3, E0M3 + BF16 scales, w_group in {0, 32, 64, 128}
+ *   UINT1, UINT2, UINT3 + BF16 scales + zero points, w_group in {32, 64, 128}
  *   E2M3, E3M2 + E8M0 scales, w_group = 32                  (MXFP6)
  * and every one of them with a_dtype in {BF16, E4M3, MXFP8, NVFP4}.  E0M3
  * ("Announcing Humming", section "Quantization support": a float with no

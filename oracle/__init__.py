@@ -211,7 +211,7 @@ def decode_weights(d: Desc, N: int, K: int, codes, scales, zeros=None, global_sc
     scales are folded into W).
     """
     col = None
-    if d.w_dtype in ("int2", "uint2", "int3", "uint3", "e0m3", "e2m3", "e3m2"):
+    if d.w_dtype in ("int1", "uint1", "int2", "uint2", "int3", "uint3", "e0m3", "e2m3", "e3m2"):
         # the other widths, from the standard b-bit code stream
         z = None if zeros is None else np.asarray(zeros).reshape(N, -1)
         return decode_lowbit_weights(d.w_dtype, np.asarray(codes).reshape(N, -1), scales, K, d.w_group, z), None
@@ -614,11 +614,13 @@ def int_to_e0m(q, bits: int) -> np.ndarray:
 def decode_lowbit_weights(kind: str, packed, scales, K: int, group: int = 0, zeros=None):
     """Weights of the other WnA16 widths from the standard bit stream
     (``unpack_bits``) [N, K * b / 8] bytes:
-      'int2' / 'int3': signed b-bit two's complement times bf16 group scales;
-      'uint2' / 'uint3': (u - z) times bf16 group scales, z uint8 [N, K/group];
+      'int1' / 'int2' / 'int3': signed b-bit two's complement times bf16
+          group scales (INT1: codes 0 and -1);
+      'uint1' / 'uint2' / 'uint3': (u - z) times bf16 group scales, z uint8
+          [N, K/group];
       'e0m3': float4e0m3 times bf16 group scales;
       'e2m3' / 'e3m2': MXFP6 with an E8M0 scale per 32."""
-    if kind in ("int2", "int3", "uint2", "uint3"):
+    if kind in ("int1", "uint1", "int2", "int3", "uint2", "uint3"):
         b = int(kind[-1])
         u = unpack_bits(packed, b, K)
         return decode_int_weights(b, u, scales, group, zeros if kind.startswith("u") else None)

@@ -14,7 +14,7 @@ import os
 __all__ = [
     "HQError", "QuantDesc", "ComputeConfig", "PlanInfo", "lib", "library_path", "EXPORTS",
     "HQ_BF16", "HQ_FP32", "HQ_INT4", "HQ_UINT4", "HQ_E2M1", "HQ_E4M3", "HQ_E8M0", "HQ_UE4M3", "HQ_MXFP8",
-    "HQ_NVFP4", "HQ_INT2", "HQ_UINT2", "HQ_INT3", "HQ_UINT3", "HQ_E2M3", "HQ_E3M2", "HQ_E0M3",
+    "HQ_NVFP4", "HQ_INT2", "HQ_UINT2", "HQ_INT3", "HQ_UINT3", "HQ_E2M3", "HQ_E3M2", "HQ_E0M3", "HQ_INT1", "HQ_UINT1",
     "HQ_MOE_GROUPED", "HQ_MOE_INDEXED",
     "hq_status_string", "hq_device_error", "hq_packed_weights_bytes", "hq_pack_weights", "hq_unpack_weights",
     "hq_quant_act", "hq_gemm_workspace_bytes", "hq_gemm", "hq_gemm_config_workspace_bytes",
@@ -25,7 +25,7 @@ __all__ = [
 ]
 
 HQ_BF16, HQ_FP32, HQ_INT4, HQ_UINT4, HQ_E2M1, HQ_E4M3, HQ_E8M0, HQ_UE4M3, HQ_MXFP8, HQ_NVFP4 = range(10)
-HQ_INT2, HQ_UINT2, HQ_INT3, HQ_UINT3, HQ_E2M3, HQ_E3M2, HQ_E0M3 = range(10, 17)
+HQ_INT2, HQ_UINT2, HQ_INT3, HQ_UINT3, HQ_E2M3, HQ_E3M2, HQ_E0M3, HQ_INT1, HQ_UINT1 = range(10, 19)
 HQ_MOE_GROUPED, HQ_MOE_INDEXED = 0, 1
 
 STATUS = {

@@ -709,6 +709,8 @@ hq_status launch_dec_gemm(const Layout &L, const tc::Params &p, const void *a, i
     case W_INT4: return dec_launch_wf<W_INT4>(map, p, t, st);
     case W_E0M3: return dec_launch_wf<W_INT4>(map, p, t, st);  // packed as INT4
     case W_MXINT4: return dec_launch_wf<W_MXINT4>(map, p, t, st);
+    case W_INT1: return dec_launch_wf<W_INT1>(map, p, t, st);
+    case W_UINT1: return dec_launch_wf<W_UINT1>(map, p, t, st);
     case W_INT2: return dec_launch_wf<W_INT2>(map, p, t, st);
     case W_UINT2: return dec_launch_wf<W_UINT2>(map, p, t, st);
     case W_INT3: return dec_launch_wf<W_INT3>(map, p, t, st);

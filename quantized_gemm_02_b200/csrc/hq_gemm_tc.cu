@@ -274,13 +274,19 @@ template <int WF>
 __device__ __forceinline__ void decode_half_lowbit(const uint8_t *unit, uint32_t s2, uint32_t z2, int r, int h,
                                                    uint32_t *rg) {
   constexpr int b = fmt_bits(WF);
-  const uint2 v2 = *reinterpret_cast<const uint2 *>(unit + plane2_off(WF) + r * 16 + h * 8);
-  const uint32_t w2[2] = {v2.x, v2.y};
   uint32_t c[16];
+  if constexpr (b == 1) {
+    const uint32_t w1 = *reinterpret_cast<const uint32_t *>(unit + plane1_off(WF) + r * 8 + h * 4);
 #pragma unroll
-  for (int a = 0; a < 2; ++a)
+    for (int q = 0; q < 16; ++q) c[q] = (w1 >> q) & 0x00010001u;
+  } else {
+    const uint2 v2 = *reinterpret_cast<const uint2 *>(unit + plane2_off(WF) + r * 16 + h * 8);
+    const uint32_t w2[2] = {v2.x, v2.y};
 #pragma unroll
-    for (int i = 0; i < 8; ++i) c[8 * a + i] = (w2[a] >> (2 * i)) & 0x00030003u;
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) c[8 * a + i] = (w2[a] >> (2 * i)) & 0x00030003u;
+  }
   if constexpr (b == 3) {
     const uint32_t w1 = *reinterpret_cast<const uint32_t *>(unit + plane1_off(WF) + r * 8 + h * 4);
 #pragma unroll
@@ -1038,6 +1044,8 @@ hq_status launch_tc_gemm(const Layout &L, const void *packed, const void *a_bf16
     case W_INT4: return tc_launch_wf<W_INT4>(map, p, t, st);
     case W_E0M3: return tc_launch_wf<W_INT4>(map, p, t, st);  // packed as INT4
     case W_MXINT4: return tc_launch_wf<W_MXINT4>(map, p, t, st);
+    case W_INT1: return tc_launch_wf<W_INT1>(map, p, t, st);
+    case W_UINT1: return tc_launch_wf<W_UINT1>(map, p, t, st);
     case W_INT2: return tc_launch_wf<W_INT2>(map, p, t, st);
     case W_UINT2: return tc_launch_wf<W_UINT2>(map, p, t, st);
     case W_INT3: return tc_launch_wf<W_INT3>(map, p, t, st);

@@ -44,19 +44,24 @@ enum WFmt : int {
   W_INT4 = 0, W_UINT4 = 1, W_MXFP4 = 2, W_NVFP4 = 3, W_FP8 = 4, W_MXINT4 = 5,
   W_INT2 = 6, W_UINT2 = 7, W_INT3 = 8, W_UINT3 = 9, W_E2M3 = 10, W_E3M2 = 11, W_E0M3 = 12,
   W_FP8B = 13,  // E4M3 with one fp32 scale per 128 x 128 block (rows x k)
-  W_NFMT = 14
+  W_INT1 = 14, W_UINT1 = 15,
+  W_NFMT = 16
 };
 
 // Bits per stored weight code of a format.
 __host__ __device__ constexpr int fmt_bits(int fmt) {
   return (fmt == W_FP8 || fmt == W_FP8B) ? 8 : (fmt == W_INT2 || fmt == W_UINT2) ? 2 : (fmt == W_INT3 || fmt == W_UINT3) ? 3
-         : (fmt == W_E2M3 || fmt == W_E3M2) ? 6 : 4;
+         : (fmt == W_E2M3 || fmt == W_E3M2) ? 6 : (fmt == W_INT1 || fmt == W_UINT1) ? 1 : 4;
 }
-__host__ __device__ constexpr bool fmt_lowbit(int fmt) { return fmt >= W_INT2 && fmt <= W_E3M2; }
-__host__ __device__ constexpr bool fmt_zero(int fmt) { return fmt == W_UINT4 || fmt == W_UINT2 || fmt == W_UINT3; }
+__host__ __device__ constexpr bool fmt_lowbit(int fmt) {
+  return (fmt >= W_INT2 && fmt <= W_E3M2) || fmt == W_INT1 || fmt == W_UINT1;
+}
+__host__ __device__ constexpr bool fmt_zero(int fmt) {
+  return fmt == W_UINT4 || fmt == W_UINT2 || fmt == W_UINT3 || fmt == W_UINT1;
+}
 __host__ __device__ constexpr bool fmt_bf16_scales(int fmt) {
   return fmt == W_INT4 || fmt == W_UINT4 || fmt == W_INT2 || fmt == W_UINT2 || fmt == W_INT3 || fmt == W_UINT3 ||
-         fmt == W_E0M3;
+         fmt == W_E0M3 || fmt == W_INT1 || fmt == W_UINT1;
 }
 // Unit planes of the low-bit layouts (byte offsets inside a 128-row x 64-k
 // unit): a 4-bit plane (the INT4 unit's order, 4 KiB; 6-bit codes' low
@@ -64,7 +69,8 @@ __host__ __device__ constexpr bool fmt_bf16_scales(int fmt) {
 // 16j..16j+15, even k in bits 0..15 and odd k in bits 16..31, two bits
 // each; the low two bits of 2- and 3-bit codes, the high two of 6-bit
 // ones) and a 1-bit plane ([128 rows][8 B]: word j holds k 32j..32j+31,
-// even k in bits 0..15, odd in 16..31; the high bit of 3-bit codes).
+// even k in bits 0..15, odd in 16..31; the high bit of 3-bit codes, or the
+// 1-bit codes themselves).
 __host__ __device__ constexpr int plane2_off(int fmt) { return (fmt == W_E2M3 || fmt == W_E3M2) ? 4096 : 0; }
 __host__ __device__ constexpr int plane1_off(int fmt) { return (fmt == W_INT3 || fmt == W_UINT3) ? 2048 : 0; }
 // Internal activation formats (A_FP8G: E4M3 with an fp32 scale per token and
@@ -149,18 +155,20 @@ inline bool weight_format(const hq_quant_desc *d, int *fmt) {
       if (d->w_group != 0) return false;
       *fmt = W_FP8;
       return true;
+    case HQ_INT1:
     case HQ_INT2:
     case HQ_INT3:
     case HQ_E0M3:
       if (d->w_scale_dtype != HQ_BF16 || d->w_has_zero || d->w_has_global) return false;
       if (!(d->w_group == 0 || d->w_group == 32 || d->w_group == 64 || d->w_group == 128)) return false;
-      *fmt = d->w_dtype == HQ_INT2 ? W_INT2 : d->w_dtype == HQ_INT3 ? W_INT3 : W_E0M3;
+      *fmt = d->w_dtype == HQ_INT1 ? W_INT1 : d->w_dtype == HQ_INT2 ? W_INT2 : d->w_dtype == HQ_INT3 ? W_INT3 : W_E0M3;
       return true;
+    case HQ_UINT1:
     case HQ_UINT2:
     case HQ_UINT3:
       if (d->w_scale_dtype != HQ_BF16 || !d->w_has_zero || d->w_has_global) return false;
       if (!(d->w_group == 32 || d->w_group == 64 || d->w_group == 128)) return false;
-      *fmt = d->w_dtype == HQ_UINT2 ? W_UINT2 : W_UINT3;
+      *fmt = d->w_dtype == HQ_UINT1 ? W_UINT1 : d->w_dtype == HQ_UINT2 ? W_UINT2 : W_UINT3;
       return true;
     case HQ_E2M3:
     case HQ_E3M2:

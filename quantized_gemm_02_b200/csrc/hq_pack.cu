@@ -302,7 +302,7 @@ __device__ inline uint32_t stream_code(const uint8_t *codes, size_t row_bytes, i
 
 // Signed codes are stored biased (two's complement -> + 2^(b-1)), so every
 // integer format decodes as (u - z).
-__device__ inline bool lowbit_signed(int fmt) { return fmt == W_INT2 || fmt == W_INT3; }
+__device__ inline bool lowbit_signed(int fmt) { return fmt == W_INT1 || fmt == W_INT2 || fmt == W_INT3; }
 
 // The stored (biased) code of packed row p (of the tile order), k of the
 // matrix; padded rows decode to zero.
@@ -321,6 +321,7 @@ __global__ void pack_lowbit_kernel(Layout L, int E, const uint8_t *codes, uint8_
   const size_t rb = (size_t)L.K * b / 8;
   const size_t wpu = L.unit_bytes() / 4;
   const int p4w = (b == 6) ? 1024 : 0;  // words of the 4-bit plane
+  const int p2w = (b == 1) ? 0 : 512;   // words of the 2-bit plane
   const size_t total = (size_t)E * L.NT * L.KB * wpu;
   for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < total;
        idx += (size_t)gridDim.x * blockDim.x) {
@@ -338,7 +339,7 @@ __global__ void pack_lowbit_kernel(Layout L, int E, const uint8_t *codes, uint8_
         const int kk = chunk * 32 + j * 8 + 2 * (slot & 3) + (slot >> 2);
         word |= (lowbit_stored(L, ce, rb, nt * TILE_N + i_row, kb * TILE_K + kk) & 15u) << (4 * slot);
       }
-    } else if (wi < p4w + 512) {
+    } else if (wi < p4w + p2w) {
       // 2-bit plane: low two bits (2-, 3-bit codes) or high two (6-bit)
       const int w = wi - p4w, i_row = w / 4, j = w % 4;
       const int sh = (b == 6) ? 4 : 0;
@@ -347,11 +348,12 @@ __global__ void pack_lowbit_kernel(Layout L, int E, const uint8_t *codes, uint8_
         word |= ((lowbit_stored(L, ce, rb, nt * TILE_N + i_row, kb * TILE_K + kk) >> sh) & 3u) << (2 * p);
       }
     } else {
-      // 1-bit plane: the high bit of 3-bit codes
-      const int w = wi - p4w - 512, i_row = w / 2, j = w % 2;
+      // 1-bit plane: the high bit of 3-bit codes, or 1-bit codes
+      const int w = wi - p4w - p2w, i_row = w / 2, j = w % 2;
+      const int sh = (b == 3) ? 2 : 0;
       for (int p = 0; p < 32; ++p) {
         const int kk = 32 * j + (p < 16 ? 2 * p : 2 * (p - 16) + 1);
-        word |= ((lowbit_stored(L, ce, rb, nt * TILE_N + i_row, kb * TILE_K + kk) >> 2) & 1u) << p;
+        word |= ((lowbit_stored(L, ce, rb, nt * TILE_N + i_row, kb * TILE_K + kk) >> sh) & 1u) << p;
       }
     }
     reinterpret_cast<uint32_t *>(packed + (size_t)e * L.stride + L.w_off)[unit * wpu + wi] = word;
@@ -364,6 +366,7 @@ __global__ void unpack_lowbit_kernel(Layout L, int E, const uint8_t *packed, uin
   const size_t rb = (size_t)L.K * b / 8;
   const size_t wpu = L.unit_bytes() / 4;
   const int p4w = (b == 6) ? 1024 : 0;
+  const int p2w = (b == 1) ? 0 : 512;
   const size_t per_row = (size_t)L.K / 8;
   const size_t total = (size_t)E * L.N * per_row;
   for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < total;
@@ -383,14 +386,14 @@ __global__ void unpack_lowbit_kernel(Layout L, int E, const uint8_t *packed, uin
         const int ko = kk & 7, slot = (ko & 1) * 4 + (ko >> 1);
         c = (u[((kk >> 5) * TILE_N + i_row) * 4 + ((kk & 31) >> 3)] >> (4 * slot)) & 15u;
       }
-      {
+      if (b != 1) {
         const int ko = kk & 15, p = (ko & 1) ? 8 + (ko >> 1) : (ko >> 1);
         const uint32_t f = (u[p4w + i_row * 4 + (kk >> 4)] >> (2 * p)) & 3u;
         c |= (b == 6) ? (f << 4) : f;
       }
-      if (b == 3) {
+      if (b == 3 || b == 1) {
         const int ko = kk & 31, p = (ko & 1) ? 16 + (ko >> 1) : (ko >> 1);
-        c |= ((u[p4w + 512 + i_row * 2 + (kk >> 5)] >> p) & 1u) << 2;
+        c |= ((u[p4w + p2w + i_row * 2 + (kk >> 5)] >> p) & 1u) << (b == 3 ? 2 : 0);
       }
       if (lowbit_signed(L.fmt)) c ^= 1u << (b - 1);
       bitsacc |= (uint64_t)c << (b * q);

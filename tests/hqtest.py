@@ -32,6 +32,10 @@ WFORMATS = {
             dict(w_dtype="e4m3", w_group=0, w_scale="fp32")),
     "mxint4": (dict(w_dtype=2, w_group=32, w_scale_dtype=6, w_has_zero=0, w_has_global=0),
                dict(w_dtype="int4", w_group=32, w_scale="e8m0")),
+    "int1_g128": (dict(w_dtype=17, w_group=128, w_scale_dtype=0, w_has_zero=0, w_has_global=0),
+                  dict(w_dtype="int1", w_group=128, w_scale="bf16")),
+    "uint1_g64": (dict(w_dtype=18, w_group=64, w_scale_dtype=0, w_has_zero=1, w_has_global=0),
+                  dict(w_dtype="uint1", w_group=64, w_scale="bf16", w_zero=True)),
     "int2_g64": (dict(w_dtype=10, w_group=64, w_scale_dtype=0, w_has_zero=0, w_has_global=0),
                  dict(w_dtype="int2", w_group=64, w_scale="bf16")),
     "uint2_g32": (dict(w_dtype=11, w_group=32, w_scale_dtype=0, w_has_zero=1, w_has_global=0),
@@ -51,7 +55,7 @@ WFORMATS = {
              dict(w_dtype="e4m3", w_group=128, w_scale="fp32")),
 }
 PAIR_ONLY = {"fp8b": "fp8g"}  # weight formats that exist with one activation format only
-LOWBIT = {"int2_g64": 2, "uint2_g32": 2, "int3_g128": 3, "uint3_g64": 3, "e2m3": 6, "e3m2": 6, "e0m3_g128": 4}
+LOWBIT = {"int1_g128": 1, "uint1_g64": 1, "int2_g64": 2, "uint2_g32": 2, "int3_g128": 3, "uint3_g64": 3, "e2m3": 6, "e3m2": 6, "e0m3_g128": 4}
 AFORMATS = {"bf16": 0, "fp8": 5, "mxfp8": 8, "nvfp4": 9, "fp8g": 5}
 AGROUP = {"fp8g": 128}  # E4M3 with an fp32 scale per token and 128 k
 

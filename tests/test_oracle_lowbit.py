@@ -110,7 +110,8 @@ def test_symmetric_int4_view_as_e0m3_keeps_the_weights():
     assert np.array_equal(W_int, W_e0)
 
 
-@pytest.mark.parametrize("kind,bits", [("int2", 2), ("int3", 3), ("uint2", 2), ("uint3", 3)])
+@pytest.mark.parametrize("kind,bits", [("int1", 1), ("int2", 2), ("int3", 3), ("uint1", 1), ("uint2", 2),
+                                       ("uint3", 3)])
 def test_lowbit_integers_from_the_stream(kind, bits):
     N, K, G = 4, 128, 64
     rng = np.random.default_rng(bits)
