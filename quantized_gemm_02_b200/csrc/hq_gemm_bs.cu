@@ -379,13 +379,21 @@ __global__ void __launch_bounds__(THREADS, 1)
     int cur_t = -1, wrow = 0, expert = 0;
     const int nchunk = p.KB;  // stage chunks per weight row (one per stage)
     const uint8_t *sfsrc = nullptr;
+    const uint8_t *wtile = nullptr;  // the tile's first stage chunk (stage chunks are contiguous)
+    // the codes of the tile's stages are prefetched into L2 about 128 KB ahead
+    constexpr int PF = (128 * 1024) / C::W_GLOBAL;
     for (int is = 0, s = 0, ph = 0; w.left > 0; ++is, w.next(p.KB)) {
       if (w.t != cur_t) {
         const TileInfo ti = tile_info(w.t);
         expert = ti.expert;
         wrow = ti.wt * nchunk * BM;  // first chunk row of the tile
         sfsrc = p.packed + (size_t)ti.expert * p.stride + p.s_off + (size_t)ti.wt * chunks_per_tile * 512;
+        wtile = p.packed + (size_t)ti.expert * p.stride + p.w_off + (size_t)ti.wt * nchunk * C::W_GLOBAL;
+        if (lane == 0)
+          for (int q = 1; q <= PF && w.ks + q < p.KB; ++q) prefetch_l2(wtile + (size_t)(w.ks + q) * C::W_GLOBAL, C::W_GLOBAL);
         cur_t = w.t;
+      } else if (lane == 0 && w.ks + PF < p.KB) {
+        prefetch_l2(wtile + (size_t)(w.ks + PF) * C::W_GLOBAL, C::W_GLOBAL);
       }
       if (is >= NS && !mbar_wait(&sfree[s], ph ^ 1)) { *s_abort = 1; break; }
       if (*(volatile int *)s_abort) break;
@@ -800,12 +808,19 @@ __global__ void __launch_bounds__(THREADS, 1)
     Walk w;
     w.start(beg, end, p.KB);
     int cur_t = -1, wrow = 0, expert = 0;
+    const uint8_t *wtile = nullptr;
+    constexpr int PF = (128 * 1024) / C::W_SMEM;  // stages of codes prefetched into L2 ahead
     for (int is = 0, s = 0, ph = 0; w.left > 0; ++is, w.next(p.KB)) {
       if (w.t != cur_t) {
         const TileInfo ti = tile_info(w.t);
         expert = ti.expert;
         wrow = ti.wt * p.KB * BM;
+        wtile = p.packed + (size_t)ti.expert * p.stride + p.w_off + (size_t)ti.wt * p.KB * C::W_SMEM;
+        if (lane == 0)
+          for (int q = 1; q <= PF && w.ks + q < p.KB; ++q) prefetch_l2(wtile + (size_t)(w.ks + q) * C::W_SMEM, C::W_SMEM);
         cur_t = w.t;
+      } else if (lane == 0 && w.ks + PF < p.KB) {
+        prefetch_l2(wtile + (size_t)(w.ks + PF) * C::W_SMEM, C::W_SMEM);
       }
       if (is >= NS && !mbar_wait(&sfree[s], ph ^ 1)) { *s_abort = 1; break; }
       if (*(volatile int *)s_abort) break;

@@ -524,12 +524,25 @@ __global__ void __launch_bounds__(THREADS, (BNT <= 64 ? 2 : 1)) tc_gemm_kernel(c
   if (warp == WARP_PRODUCER) {
     // ================= producer (whole warp in step, lane 0 issues) =================
     const uint64_t pol = p.weights_once ? policy_evict_first() : policy_evict_normal();
+    // weights are prefetched into L2 about 64 KB ahead of the copies (within
+    // the unit; the next unit's first blocks near its end)
+    constexpr int PF = (64 * 1024) / (C::KPS * TR::unit) > 1 ? (64 * 1024) / (C::KPS * TR::unit) : 1;
     int is = 0;
     bool stop = false;
     for (int u = 0; !stop; ++u) {
       int t, ukb0, ukb1, usp;
       if (!unit_at(sch, cta, p.nctas, p.KB, u, t, ukb0, ukb1, usp)) break;
       const TileInfo ti = tile_info(t);
+      int tn, nkb0, nkb1, nsp;  // the next unit, for the prefetch across units
+      const bool has_next = unit_at(sch, cta, p.nctas, p.KB, u + 1, tn, nkb0, nkb1, nsp);
+      const uint8_t *wnext = nullptr;  // the next unit's weight tile
+      int nst_next = 0, rot_next = 0;
+      if (has_next) {
+        const TileInfo tin = tile_info(tn);
+        wnext = p.packed + (size_t)tin.expert * p.stride + p.w_off + (size_t)tin.wt * p.KB * TR::unit;
+        nst_next = (nkb1 - nkb0 + C::KPS - 1) / C::KPS;
+        rot_next = stage_rotation(cta, nst_next);
+      }
       if (p.gather) {
         // the tile's caller rows, read once per tile; positions past the
         // valid rows repeat the last one (loaded, never written back)
@@ -570,6 +583,20 @@ __global__ void __launch_bounds__(THREADS, (BNT <= 64 ? 2 : 1)) tc_gemm_kernel(c
           for (int j = 0; j < nblk; ++j) tma_load_2d(st + j * C::ACT_KB, &act_map, (kbs + j) * TILE_K, ti.base, &full[s]);
         bulk_g2s_stream(st + C::ACT, eb + p.w_off + ((size_t)ti.wt * p.KB + kbs) * TR::unit, TR::unit * nblk,
                         &full[s], pol);
+        if (i == 0) {
+          // the first PF stages of the unit, then one stage per stage
+          for (int q = 1; q <= PF && q < nst; ++q) {
+            const int kq = ukb0 + stage_of(q, rot, nst) * C::KPS;
+            prefetch_l2(eb + p.w_off + ((size_t)ti.wt * p.KB + kq) * TR::unit, TR::unit * min(C::KPS, ukb1 - kq));
+          }
+        } else if (i + PF < nst) {
+          const int kq = ukb0 + stage_of(i + PF, rot, nst) * C::KPS;
+          prefetch_l2(eb + p.w_off + ((size_t)ti.wt * p.KB + kq) * TR::unit, TR::unit * min(C::KPS, ukb1 - kq));
+        } else if (wnext && i + PF - nst < nst_next) {
+          // the next unit's first stages, in the order it will take them
+          const int kq = nkb0 + stage_of(i + PF - nst, rot_next, nst_next) * C::KPS;
+          prefetch_l2(wnext + (size_t)kq * TR::unit, TR::unit * min(C::KPS, nkb1 - kq));
+        }
         if (TR::has_scales)
           bulk_g2s(st + C::ACT + C::WPK, eb + p.s_off + ((size_t)ti.wt * p.G + g0) * BM * TR::sbytes, sb,
                    &full[s]);

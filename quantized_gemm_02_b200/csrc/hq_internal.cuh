@@ -389,6 +389,14 @@ __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.p
 // map's SWIZZLE_128B loads produce and the MMA descriptors read.
 __device__ __forceinline__ uint32_t sw128_offset(int i, int c) { return (uint32_t)(i * 128 + ((c ^ (i & 7)) << 4)); }
 
+// Prefetch of a global range into L2 (16-byte aligned address, size a
+// multiple of 16): the weight producers issue it some stages ahead, so that
+// their bulk copies find the weights in L2 instead of waiting a DRAM round
+// trip with only the ring's few stages in flight.
+__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
