@@ -341,6 +341,8 @@ WORKLOAD_TITLE = {
     "w4a4_nvfp4": "dense W4A4 NVFP4 x NVFP4, N=K=7168, M in {1,32,256,2048,8192}",
     "w8a8_fp8": "dense W8A8 FP8 per-channel x per-token, N=K=7168, M in {1,32,256,2048,8192}",
     "moe_silu": "MoE gate-up GEMM + SiLU-and-mul at the config-3 shapes, T in {16, 4096}: unfused and fused",
+    "moe_profile_e64": "MoE W4A16 MXFP4 at the config-3 expert shapes with E=64, T=1024 (about 128 rows per "
+                       "expert), grouped + indexed: a small case of the T=4096 calls for profiling",
     "lowbit": "dense WnA16 INT2, INT3, MXFP6 E2M3, float4e0m3 at N=28672, K=8192, M in {1, 16}",
     "w8a8_fp8_block": "block-scaled FP8 W8A8: dense N=K=7168, M in {1,32,256,2048,8192}, and MoE at the config-3 "
                       "shapes, T in {64, 4096}, grouped + indexed",
@@ -609,6 +611,15 @@ def ops_moe_fp8_block(hq, gen, Ts=(64, 4096)):
                    hq.HQ_E4M3)
 
 
+def ops_moe_profile_e64(hq, gen):
+    """A profiling case of the config-3 MoE calls at a quarter of the experts:
+    E = 64, T = 1024, top-8 (about 128 routed rows per expert, as at T = 4096
+    with 256 experts), MXFP4 W4A16, grouped and indexed; 1.4 GB of weights."""
+    d = desc_of(hq, hq.HQ_E2M1, 32, hq.HQ_E8M0, 0, 0, hq.HQ_BF16)
+    routing = lambda T, g: synth.routing_softmax_topk(T, 64, TOPK, g, device="cuda")
+    return ops_moe(hq, 3, "moe_w4a16_e64", d, 64, TOPK, H_MOE, I_MOE, [1024], routing, gen, hq.HQ_BF16)
+
+
 def ops_moe_w4a8_mxfp8(hq, gen, Ts=(1, 64, 512, 4096)):
     d = desc_of(hq, hq.HQ_E2M1, 32, hq.HQ_E8M0, 0, 0, hq.HQ_MXFP8)
     routing = lambda T, g: synth.routing_zipf(T, E_MOE, TOPK, 1.2, g, device="cuda")
@@ -766,6 +777,7 @@ WORKLOADS = {
                                 WORKLOAD_TITLE["w8a8_fp8_block"]),
     "lowbit": _workload([ops_lowbit], WORKLOAD_TITLE["lowbit"]),
     "moe_silu": _workload([ops_moe_silu], WORKLOAD_TITLE["moe_silu"]),
+    "moe_profile_e64": _workload([ops_moe_profile_e64], WORKLOAD_TITLE["moe_profile_e64"]),
     "moe_w4a16_mxint4": _workload([ops_moe_w4a16_mxint4], WORKLOAD_TITLE["moe_w4a16_mxint4"]),
     "w4a16_asym_sweep": _workload([ops_w4a16_asym_sweep], WORKLOAD_TITLE["w4a16_asym_sweep"]),
     "w4a16_dense_m16": _workload([ops_w4a16_dense_m16], WORKLOAD_TITLE["w4a16_dense_m16"]),
@@ -778,7 +790,7 @@ WORKLOADS = {
 }
 
 # configurations each workload covers (for the CPU samples)
-WORKLOAD_CONFIGS = {"all": (1, 2, 3, 4, 5), "w8a8_fp8_block": (5,), "moe_w4a16_mxint4": (3,), "moe_silu": (3,), "lowbit": (2,), "w4a16_asym_sweep": (2,), "w4a16_dense_m16": (1,),
+WORKLOAD_CONFIGS = {"all": (1, 2, 3, 4, 5), "moe_profile_e64": (3,), "w8a8_fp8_block": (5,), "moe_w4a16_mxint4": (3,), "moe_silu": (3,), "lowbit": (2,), "w4a16_asym_sweep": (2,), "w4a16_dense_m16": (1,),
                     "moe_w4a16_mxfp4": (3,), "moe_w4a8_mxfp8": (4,), "moe_nvfp4": (5,), "moe_masked_nvfp4": (5,),
                     "w4a4_nvfp4": (5,), "w8a8_fp8": (5,)}
 

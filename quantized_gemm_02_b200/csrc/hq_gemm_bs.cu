@@ -379,21 +379,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     int cur_t = -1, wrow = 0, expert = 0;
     const int nchunk = p.KB;  // stage chunks per weight row (one per stage)
     const uint8_t *sfsrc = nullptr;
-    const uint8_t *wtile = nullptr;  // the tile's first stage chunk (stage chunks are contiguous)
-    // the codes of the tile's stages are prefetched into L2 about 128 KB ahead
-    constexpr int PF = (128 * 1024) / C::W_GLOBAL;
     for (int is = 0, s = 0, ph = 0; w.left > 0; ++is, w.next(p.KB)) {
       if (w.t != cur_t) {
         const TileInfo ti = tile_info(w.t);
         expert = ti.expert;
         wrow = ti.wt * nchunk * BM;  // first chunk row of the tile
         sfsrc = p.packed + (size_t)ti.expert * p.stride + p.s_off + (size_t)ti.wt * chunks_per_tile * 512;
-        wtile = p.packed + (size_t)ti.expert * p.stride + p.w_off + (size_t)ti.wt * nchunk * C::W_GLOBAL;
-        if (lane == 0)
-          for (int q = 1; q <= PF && w.ks + q < p.KB; ++q) prefetch_l2(wtile + (size_t)(w.ks + q) * C::W_GLOBAL, C::W_GLOBAL);
         cur_t = w.t;
-      } else if (lane == 0 && w.ks + PF < p.KB) {
-        prefetch_l2(wtile + (size_t)(w.ks + PF) * C::W_GLOBAL, C::W_GLOBAL);
       }
       if (is >= NS && !mbar_wait(&sfree[s], ph ^ 1)) { *s_abort = 1; break; }
       if (*(volatile int *)s_abort) break;
@@ -437,26 +429,18 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       if (is >= NS && !mbar_wait(&sfree[s], ph ^ 1)) { *s_abort = 1; break; }
       if (*(volatile int *)s_abort) break;
-      if (p.gather) {
-        // indexed mode: the tile's rows of the stage (128 bytes each) from the
-        // caller's codes, 16 bytes per copy into the swizzled tile, all lanes;
-        // the copies arrive on the stage barrier
-        uint8_t *st = smem + s * C::STAGE;
-        for (int it = lane; it < nvalid * 8; it += 32) {
-          const int ii = it >> 3, c = it & 7;
-          cp_async16(st + C::W_SMEM + sw128_offset(ii, c),
-                     p.a_src + (size_t)s_rows[ii] * p.a_ld + (size_t)w.ks * 128 + c * 16);
-        }
-        cp_async_arrive(&full[s]);
-        __syncwarp();
-      }
       if (lane == 0) {
         uint8_t *st = smem + s * C::STAGE;
         if (!p.gather) {
           mbar_arrive_expect_tx(&full[s], (uint32_t)(C::A_SMEM + C::SF_CH * C::SFB_CHB));
           tma_load_2d(st + C::W_SMEM, &a_map, w.ks * 128, base, &full[s]);
         } else {
-          mbar_arrive_expect_tx(&full[s], (uint32_t)(C::SF_CH * C::SFB_CHB));
+          // indexed mode: the tile's caller rows, four 128-byte rows per gather
+          const int ng = (nvalid + 3) >> 2;
+          mbar_arrive_expect_tx(&full[s], (uint32_t)(ng * 4 * 128 + C::SF_CH * C::SFB_CHB));
+          for (int gi = 0; gi < ng; ++gi)
+            tc::tma_gather4(st + C::W_SMEM + gi * 512, &a_map, w.ks * 128, s_rows[4 * gi], s_rows[4 * gi + 1],
+                            s_rows[4 * gi + 2], s_rows[4 * gi + 3], &full[s]);
         }
         if constexpr (C::SF_CH > 0)
           bulk_g2s(st + C::SFB_OFF, sfsrc + (size_t)w.ks * C::SF_CH * C::SFB_CHB, C::SF_CH * C::SFB_CHB, &full[s]);
@@ -477,7 +461,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       if (!mbar_wait(&full[s], ph)) { *s_abort = 1; break; }
       if (*(volatile int *)s_abort) break;
-      if (p.gather) fence_proxy_async_smem();  // cp.async rows -> tensor-core reads
       tc::tc_fence_after();
       const uint32_t st = smem_u32(smem + s * C::STAGE);
       const uint64_t adesc = tc::sw128_desc(st);
@@ -808,19 +791,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     Walk w;
     w.start(beg, end, p.KB);
     int cur_t = -1, wrow = 0, expert = 0;
-    const uint8_t *wtile = nullptr;
-    constexpr int PF = (128 * 1024) / C::W_SMEM;  // stages of codes prefetched into L2 ahead
     for (int is = 0, s = 0, ph = 0; w.left > 0; ++is, w.next(p.KB)) {
       if (w.t != cur_t) {
         const TileInfo ti = tile_info(w.t);
         expert = ti.expert;
         wrow = ti.wt * p.KB * BM;
-        wtile = p.packed + (size_t)ti.expert * p.stride + p.w_off + (size_t)ti.wt * p.KB * C::W_SMEM;
-        if (lane == 0)
-          for (int q = 1; q <= PF && w.ks + q < p.KB; ++q) prefetch_l2(wtile + (size_t)(w.ks + q) * C::W_SMEM, C::W_SMEM);
         cur_t = w.t;
-      } else if (lane == 0 && w.ks + PF < p.KB) {
-        prefetch_l2(wtile + (size_t)(w.ks + PF) * C::W_SMEM, C::W_SMEM);
       }
       if (is >= NS && !mbar_wait(&sfree[s], ph ^ 1)) { *s_abort = 1; break; }
       if (*(volatile int *)s_abort) break;
@@ -858,18 +834,16 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (is >= NS && !mbar_wait(&sfree[s], ph ^ 1)) { *s_abort = 1; break; }
       if (*(volatile int *)s_abort) break;
       uint8_t *st = smem + s * C::STAGE;
-      if (p.gather) {
-        for (int it = lane; it < nvalid * 8; it += 32) {
-          const int ii = it >> 3, c = it & 7;
-          cp_async16(st + C::W_SMEM + sw128_offset(ii, c),
-                     p.a_src + (size_t)s_rows[ii] * p.a_ld + (size_t)w.ks * 128 + c * 16);
-        }
-        cp_async_arrive(&full[s]);
-        __syncwarp();
-      }
       if (lane == 0) {
-        mbar_arrive_expect_tx(&full[s], (uint32_t)((p.gather ? 0 : C::A_SMEM) + BNT * 4));
-        if (!p.gather) tma_load_2d(st + C::W_SMEM, &a_map, w.ks * 128, base, &full[s]);
+        const int ng = (nvalid + 3) >> 2;  // indexed mode: four 128-byte rows per gather
+        mbar_arrive_expect_tx(&full[s], (uint32_t)((p.gather ? ng * 4 * 128 : C::A_SMEM) + BNT * 4));
+        if (!p.gather) {
+          tma_load_2d(st + C::W_SMEM, &a_map, w.ks * 128, base, &full[s]);
+        } else {
+          for (int gi = 0; gi < ng; ++gi)
+            tc::tma_gather4(st + C::W_SMEM + gi * 512, &a_map, w.ks * 128, s_rows[4 * gi], s_rows[4 * gi + 1],
+                            s_rows[4 * gi + 2], s_rows[4 * gi + 3], &full[s]);
+        }
         bulk_g2s(st + C::SA_OFF, sasrc + (size_t)w.ks * BNT * 4, (uint32_t)(BNT * 4), &full[s]);
       }
       __syncwarp();
@@ -884,7 +858,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!mbar_wait(&full[s], ph)) { *s_abort = 1; break; }
       if (is >= NP && !mbar_wait(&pempty[q], qph ^ 1)) { *s_abort = 1; break; }
       if (*(volatile int *)s_abort) break;
-      if (p.gather) fence_proxy_async_smem();  // cp.async rows -> tensor-core reads
       tc::tc_fence_after();
       const uint32_t st = smem_u32(smem + s * C::STAGE);
       const uint64_t adesc = tc::sw128_desc(st);
@@ -1130,7 +1103,8 @@ hq_status launch_bs_gemm(const Layout &L, const void *packed, int E, const void 
   const int row_bytes = L.bs == BS_NV ? L.K / 2 : L.K;
   CUtensorMap wm, am;
   if (!make_bs_weight_map(&wm, L, packed, E)) return HQ_ERR_CUDA;
-  if (!make_bs_act_map(&am, a_codes, a_rows, row_bytes, t.bnt)) return HQ_ERR_CUDA;
+  // indexed mode: one-row boxes for the 4-row gathers of caller rows
+  if (!make_bs_act_map(&am, a_codes, a_rows, row_bytes, gather ? 1 : t.bnt)) return HQ_ERR_CUDA;
   if (L.bs == BS_F8B) {
     // activation scales per token tile and stage: [mtiles][K / 128][bnt] fp32
     const size_t n = (size_t)t.mtiles * (L.K / 128) * t.bnt;
@@ -1168,8 +1142,6 @@ hq_status launch_bs_gemm(const Layout &L, const void *packed, int E, const void 
   p.row_scale = L.bs == BS_F8 ? (const float *)a_scales : nullptr;
   p.a_div = a_div;
   p.gather = gather;
-  p.a_src = (const uint8_t *)a_codes;
-  p.a_ld = row_bytes;
   p.out = (uint16_t *)out;
   p.ntw = t.ntw;
   p.mtiles = t.mtiles;

@@ -489,23 +489,18 @@ __global__ void __launch_bounds__(THREADS, 1) dec_gemm_kernel(const __grid_const
           tma_load_3d(st, &act_map, 0, base, w.kb, &full[rs.idx]);
         }
       } else {
-        // the valid rows' 128-byte pieces of the stage's blocks, 16 bytes per
-        // copy into the swizzled tile; the copies arrive on the stage barrier
-        const int per_row = w.n * 8;
-        const int items = nvalid * per_row;
-        for (int b0 = 0; b0 < items; b0 += 32) {
-          const int it = b0 + lane;
-          const int ii = it / per_row;
-          const int row = __shfl_sync(0xffffffffu, my_row, ii & 31);
-          if (it < items) {
-            const int rem = it - ii * per_row, j = rem >> 3, c = rem & 7;
-            cp_async16(st + j * C::ACT_KB + sw128_offset(ii, c),
-                       p.a_src + (size_t)row * p.a_ld + (size_t)(w.kb + j) * 128 + c * 16);
-          }
+        const int ng = (nvalid + 3) >> 2;  // 4-row gathers per 64-k block
+        if (lane == 0) mbar_arrive_expect_tx(&full[rs.idx], (uint32_t)(w.n * ng * 4 * 128));
+        for (int gi = 0; gi < ng; ++gi) {
+          const int r0 = __shfl_sync(0xffffffffu, my_row, 4 * gi);
+          const int r1 = __shfl_sync(0xffffffffu, my_row, 4 * gi + 1);
+          const int r2 = __shfl_sync(0xffffffffu, my_row, 4 * gi + 2);
+          const int r3 = __shfl_sync(0xffffffffu, my_row, 4 * gi + 3);
+          if (lane == 0)
+            for (int j = 0; j < w.n; ++j)
+              tc::tma_gather4(st + j * C::ACT_KB + gi * 512, &act_map, (w.kb + j) * TILE_K, r0, r1, r2, r3,
+                              &full[rs.idx]);
         }
-        cp_async_arrive(&full[rs.idx]);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&full[rs.idx]);
       }
       __syncwarp();
     }
@@ -577,7 +572,6 @@ __global__ void __launch_bounds__(THREADS, 1) dec_gemm_kernel(const __grid_const
       if (!mbar_wait(&full[rs.idx], rs.phase)) { *s_abort = 1; break; }
       if (!mbar_wait(&afull[ra.idx], ra.phase)) { *s_abort = 1; break; }
       if (*(volatile int *)s_abort) break;
-      if (p.gather) fence_proxy_async_smem();  // cp.async rows -> tensor-core reads
       tc::tc_fence_after();
       // operands are warp-uniform (they live in uniform registers); one
       // elected lane issues the stage's MMAs back to back
@@ -704,7 +698,11 @@ static hq_status dec_launch_wf(const CUtensorMap &map, const tc::Params &p, cons
 hq_status launch_dec_gemm(const Layout &L, const tc::Params &p, const void *a, int a_rows, const TcLaunch &t,
                           cudaStream_t st, bool e4m3_act) {
   CUtensorMap map;
-  if (!make_act_map_3d(&map, a, a_rows, L.K, t.bnt, e4m3_act)) return HQ_ERR_CUDA;
+  // indexed mode: a 2-D map of the caller's rows with one-row boxes for the
+  // 4-row gathers (bf16 only); otherwise the 3-D map of KPS blocks per box
+  if (p.gather ? !make_act_map(&map, a, a_rows, L.K, 1, false)
+               : !make_act_map_3d(&map, a, a_rows, L.K, t.bnt, e4m3_act))
+    return HQ_ERR_CUDA;
   switch (L.fmt) {
     case W_INT4: return dec_launch_wf<W_INT4>(map, p, t, st);
     case W_E0M3: return dec_launch_wf<W_INT4>(map, p, t, st);  // packed as INT4

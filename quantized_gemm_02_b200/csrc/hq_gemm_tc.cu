@@ -16,10 +16,9 @@
 //                    TMEM lanes 32w..32w+31), fp32 scales, bf16 out or fp32
 //                    split-K partials with a deterministic last-split fixup;
 //       warp 4       producer: TMA of the activation tile (bf16, 128-byte
-//                    swizzle; for MoE indexed mode the tile's rows gathered
-//                    through the routing index by 16-byte cp.async copies
-//                    into the same swizzled layout), 1-D bulk copies of the
-//                    packed weight unit, scales, zero points;
+//                    swizzle; for MoE indexed mode 4-row gathers of the
+//                    caller's rows through the routing index), 1-D bulk
+//                    copies of the packed weight unit, scales, zero points;
 //       warp 5       MMA issuer: tcgen05.mma.cta_group::1.kind::f16 with A
 //                    from TMEM and B from a shared-memory descriptor;
 //       warps 6..13  dequant: thread = weight row, decodes 32 k of its row per
@@ -105,8 +104,6 @@ struct Params {
   const int32_t *offsets, *perm;
   int a_div;
   int gather;              // MoE indexed mode: activation rows gathered by index
-  const uint8_t *a_src;    // indexed mode: the activation rows (a_ld bytes apart)
-  int a_ld;
   uint16_t *out;
   int ntw;                 // 128-row weight tiles
   int mtiles;              // token tiles (dense: exact; MoE: upper bound)
@@ -186,6 +183,17 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
       "[%4];" ::"r"(smem_u32(dst)),
       "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Four rows (given by index) of one box column of a 2-D tensor map with
+// one-row boxes, landing as consecutive box rows in shared memory.
+__device__ __forceinline__ void tma_gather4(void *dst, const CUtensorMap *map, int x, int r0, int r1, int r2, int r3,
+                                            uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(smem_u32(bar))
       : "memory");
 }
 
@@ -524,25 +532,12 @@ __global__ void __launch_bounds__(THREADS, (BNT <= 64 ? 2 : 1)) tc_gemm_kernel(c
   if (warp == WARP_PRODUCER) {
     // ================= producer (whole warp in step, lane 0 issues) =================
     const uint64_t pol = p.weights_once ? policy_evict_first() : policy_evict_normal();
-    // weights are prefetched into L2 about 64 KB ahead of the copies (within
-    // the unit; the next unit's first blocks near its end)
-    constexpr int PF = (64 * 1024) / (C::KPS * TR::unit) > 1 ? (64 * 1024) / (C::KPS * TR::unit) : 1;
     int is = 0;
     bool stop = false;
     for (int u = 0; !stop; ++u) {
       int t, ukb0, ukb1, usp;
       if (!unit_at(sch, cta, p.nctas, p.KB, u, t, ukb0, ukb1, usp)) break;
       const TileInfo ti = tile_info(t);
-      int tn, nkb0, nkb1, nsp;  // the next unit, for the prefetch across units
-      const bool has_next = unit_at(sch, cta, p.nctas, p.KB, u + 1, tn, nkb0, nkb1, nsp);
-      const uint8_t *wnext = nullptr;  // the next unit's weight tile
-      int nst_next = 0, rot_next = 0;
-      if (has_next) {
-        const TileInfo tin = tile_info(tn);
-        wnext = p.packed + (size_t)tin.expert * p.stride + p.w_off + (size_t)tin.wt * p.KB * TR::unit;
-        nst_next = (nkb1 - nkb0 + C::KPS - 1) / C::KPS;
-        rot_next = stage_rotation(cta, nst_next);
-      }
       if (p.gather) {
         // the tile's caller rows, read once per tile; positions past the
         // valid rows repeat the last one (loaded, never written back)
@@ -557,19 +552,6 @@ __global__ void __launch_bounds__(THREADS, (BNT <= 64 ? 2 : 1)) tc_gemm_kernel(c
       const int s = is % NS;
       if (is >= NS && !mbar_wait(&sfree[s], ((is / NS) - 1) & 1)) { *s_abort = 1; stop = true; break; }
       if (*(volatile int *)s_abort) { stop = true; break; }
-      if (p.gather) {
-        // indexed mode: the tile's rows from the caller's activations, 16 bytes
-        // per copy, all lanes; the copies arrive on the stage barrier
-        uint8_t *st = smem + s * C::STAGE;
-        const int items = ti.nvalid * nblk * 8;
-        for (int it = lane; it < items; it += 32) {
-          const int ii = it / (nblk * 8), rem = it - ii * (nblk * 8), j = rem >> 3, c = rem & 7;
-          cp_async16(st + j * C::ACT_KB + sw128_offset(ii, c),
-                     p.a_src + (size_t)s_rows[ii] * p.a_ld + (size_t)(kbs + j) * 128 + c * 16);
-        }
-        cp_async_arrive(&full[s]);
-        __syncwarp();
-      }
       if (lane == 0) {
         const uint8_t *eb = p.packed + (size_t)ti.expert * p.stride;
         uint8_t *st = smem + s * C::STAGE;
@@ -577,26 +559,20 @@ __global__ void __launch_bounds__(THREADS, (BNT <= 64 ? 2 : 1)) tc_gemm_kernel(c
         const int g1 = (((kbs + nblk) * TILE_K - 1) >> p.gshift) + 1;
         const uint32_t sb = TR::has_scales ? (uint32_t)((g1 - g0) * BM * TR::sbytes) : 0u;
         const uint32_t zb = TR::has_zero ? (uint32_t)((g1 - g0) * BM) : 0u;
-        const uint32_t ab = p.gather ? 0u : (uint32_t)C::ACT_KB;
+        // indexed mode: ceil(nvalid / 4) gathers of four 128-byte rows per 64-k block
+        const uint32_t ab = p.gather ? (uint32_t)(((ti.nvalid + 3) / 4) * 4 * 128) : (uint32_t)C::ACT_KB;
         mbar_arrive_expect_tx(&full[s], ab * nblk + TR::unit * nblk + sb + zb);
-        if (!p.gather)
-          for (int j = 0; j < nblk; ++j) tma_load_2d(st + j * C::ACT_KB, &act_map, (kbs + j) * TILE_K, ti.base, &full[s]);
+        for (int j = 0; j < nblk; ++j) {
+          if (!p.gather) {
+            tma_load_2d(st + j * C::ACT_KB, &act_map, (kbs + j) * TILE_K, ti.base, &full[s]);
+          } else {
+            for (int i = 0; i < ti.nvalid; i += 4)
+              tma_gather4(st + j * C::ACT_KB + i * 128, &act_map, (kbs + j) * TILE_K, s_rows[i], s_rows[i + 1],
+                          s_rows[i + 2], s_rows[i + 3], &full[s]);
+          }
+        }
         bulk_g2s_stream(st + C::ACT, eb + p.w_off + ((size_t)ti.wt * p.KB + kbs) * TR::unit, TR::unit * nblk,
                         &full[s], pol);
-        if (i == 0) {
-          // the first PF stages of the unit, then one stage per stage
-          for (int q = 1; q <= PF && q < nst; ++q) {
-            const int kq = ukb0 + stage_of(q, rot, nst) * C::KPS;
-            prefetch_l2(eb + p.w_off + ((size_t)ti.wt * p.KB + kq) * TR::unit, TR::unit * min(C::KPS, ukb1 - kq));
-          }
-        } else if (i + PF < nst) {
-          const int kq = ukb0 + stage_of(i + PF, rot, nst) * C::KPS;
-          prefetch_l2(eb + p.w_off + ((size_t)ti.wt * p.KB + kq) * TR::unit, TR::unit * min(C::KPS, ukb1 - kq));
-        } else if (wnext && i + PF - nst < nst_next) {
-          // the next unit's first stages, in the order it will take them
-          const int kq = nkb0 + stage_of(i + PF - nst, rot_next, nst_next) * C::KPS;
-          prefetch_l2(wnext + (size_t)kq * TR::unit, TR::unit * min(C::KPS, nkb1 - kq));
-        }
         if (TR::has_scales)
           bulk_g2s(st + C::ACT + C::WPK, eb + p.s_off + ((size_t)ti.wt * p.G + g0) * BM * TR::sbytes, sb,
                    &full[s]);
@@ -727,7 +703,6 @@ __global__ void __launch_bounds__(THREADS, (BNT <= 64 ? 2 : 1)) tc_gemm_kernel(c
         const int nblk = min(C::KPS, ukb1 - kbs);
         const int s = is % NS;
         if (!mbar_wait(&full[s], (is / NS) & 1)) { *s_abort = 1; stop = true; break; }
-        if (p.gather) fence_proxy_async_smem();  // cp.async rows -> tensor-core reads
         for (int j = 0; j < nblk; ++j, ++ia) {
           const int a = ia % NA;
           const bool first = (i == 0 && j == 0);
@@ -1028,7 +1003,8 @@ hq_status launch_tc_gemm(const Layout &L, const void *packed, const void *a_bf16
                          bool e4m3_act) {
   if (e4m3_act && L.fmt != W_FP8) return HQ_ERR_UNSUPPORTED;
   CUtensorMap map;
-  if (!make_act_map(&map, a_bf16, a_rows, L.K, t.bnt, e4m3_act)) return HQ_ERR_CUDA;
+  // indexed mode: one-row boxes for the 4-row gathers
+  if (!make_act_map(&map, a_bf16, a_rows, L.K, gather ? 1 : t.bnt, e4m3_act)) return HQ_ERR_CUDA;
   tc::Params p{};
   p.packed = (const uint8_t *)packed;
   p.stride = L.stride;
@@ -1045,8 +1021,6 @@ hq_status launch_tc_gemm(const Layout &L, const void *packed, const void *a_bf16
   p.perm = perm;
   p.a_div = a_div;
   p.gather = gather;
-  p.a_src = (const uint8_t *)a_bf16;
-  p.a_ld = L.K * 2;
   p.out = (uint16_t *)out;
   p.ntw = t.ntw;
   p.mtiles = t.mtiles;

@@ -371,32 +371,6 @@ __device__ __forceinline__ void bulk_g2s_stream(void *dst, const void *src, uint
       : "memory");
 }
 
-// 16-byte asynchronous global -> shared copy (L2 only), and the arrive-on of
-// an mbarrier once every earlier one of this thread has landed (the arrival
-// is self-balanced: the barrier's expected count does not include it).
-// Shared memory written this way is read by the tensor core only after the
-// consumer's fence_proxy_async_smem().
-__device__ __forceinline__ void cp_async16(void *dst_smem, const void *src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst_smem)), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
-  asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-
-// Byte offset of 16-byte chunk c of row i in a tile of 128-byte rows stored
-// with the 128-byte swizzle (tile 1024-byte aligned): the layout the tensor
-// map's SWIZZLE_128B loads produce and the MMA descriptors read.
-__device__ __forceinline__ uint32_t sw128_offset(int i, int c) { return (uint32_t)(i * 128 + ((c ^ (i & 7)) << 4)); }
-
-// Prefetch of a global range into L2 (16-byte aligned address, size a
-// multiple of 16): the weight producers issue it some stages ahead, so that
-// their bulk copies find the weights in L2 instead of waiting a DRAM round
-// trip with only the ring's few stages in flight.
-__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
-
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));

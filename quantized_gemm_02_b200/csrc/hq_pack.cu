@@ -115,7 +115,7 @@ __global__ void pack_side_kernel(Layout L, int E, const uint8_t *scales, const u
         z = (uint8_t)((w >> (4 * (gi % 8))) & 15u);
       }
       (base + L.z_off)[dst] = z;
-    } else if (L.fmt == W_UINT2 || L.fmt == W_UINT3) {
+    } else if (L.fmt == W_UINT1 || L.fmt == W_UINT2 || L.fmt == W_UINT3) {
       (base + L.z_off)[dst] = (r < L.N) ? zeros[((size_t)e * L.N + sr) * L.G + gi] : (uint8_t)0;
     }
     if (L.fmt == W_NVFP4 && r == 0 && gi == 0) {
@@ -177,7 +177,7 @@ __global__ void unpack_side_kernel(Layout L, int E, const uint8_t *packed, uint8
     } else {
       scales[idx] = (base + L.s_off)[src];
     }
-    if ((L.fmt == W_UINT2 || L.fmt == W_UINT3)) zeros[((size_t)e * L.N + r) * L.G + gi] = (base + L.z_off)[src];
+    if ((L.fmt == W_UINT1 || L.fmt == W_UINT2 || L.fmt == W_UINT3)) zeros[((size_t)e * L.N + r) * L.G + gi] = (base + L.z_off)[src];
     if (L.fmt == W_UINT4 && (gi % 8) == 0) {
       const int zw = (L.G + 7) / 8;
       uint32_t w = 0;
