@@ -20,7 +20,9 @@ per step:
 
 An MoE layer is timed as its library calls: the routing prepare, the
 gate-up GEMM and the down GEMM with the weighted top-k sum.  The L2 is
-flushed (a 512 MiB memset, untimed) before every call and each call is timed
+flushed before every call (untimed: a 512 MiB memset, then one read of that
+buffer, so that the timed call finds no line of its inputs in L2 and no dirty
+line whose write-back it would pay for) and each call is timed
 with CUDA events on its stream; each call is captured once in a CUDA graph
 and replayed (``--eager`` times the plain calls).  ``value`` = total flops of
 a step / summed call time; ``sweep`` lists every call with its roofline
@@ -246,6 +248,9 @@ def dense_op(hq, d, name, M, N, K, packed, w_bytes, gen, config):
     return Op(name, run, 2.0 * M * N * K, w_bytes, M * K * 2 + M * N * 2, 1, M * K * 2, M * N * 2, e2e,
               kernel=gemm_kernel_name(M), config=config)
 
+
+L2_NOTE = ("flushed before every call (512 MiB memset, then one read of that buffer so that no dirty line is "
+           "left in L2; untimed)")
 
 NOMINAL_HBM_GBS = 8000.0  # the nominal B200 figure the targets are quoted against
 
@@ -764,7 +769,7 @@ def _workload(builders, title):
             o, k = b(hq, gen)
             ops += o
             keep += k
-        return ops, {"workload": title, "l2": "flushed before every call (512 MiB memset, untimed)"}, keep
+        return ops, {"workload": title, "l2": L2_NOTE}, keep
     return build
 
 
@@ -981,10 +986,11 @@ def main():
         else:
             ops, keep = ops_dense_quantised(hq, args.shape_fmt, gen, N=N, K=K, Ms=(M,))
             cfg = {"workload": f"dense {args.shape_fmt} x {args.shape_fmt}, M={M}, N={N}, K={K}"}
-        cfg["l2"] = "flushed before every call"
+        cfg["l2"] = L2_NOTE
     else:
         ops, cfg, keep = WORKLOADS[args.workload](hq)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    flush_sink = torch.empty((), dtype=torch.int64, device="cuda")
     stream = torch.cuda.current_stream()
     n_ops = len(ops)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in ops]
@@ -1015,6 +1021,7 @@ def main():
         times = []
         for i, op in enumerate(ops):
             flush.zero_()
+            flush_sink.copy_(flush.view(torch.int64).sum())  # leaves the L2 holding clean lines only
             a, b = ev[i]
             a.record(stream)
             if e2e:

@@ -430,8 +430,8 @@ HQ_API hq_status hq_moe_unpermute_sum(int T, int topk, int N, const void *y_bf16
  *   - Arguments are checked as hq_gemm checks them; a rejected call
  *     enqueues nothing.
  *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current and caches it; make
- *     that first call before any stream capture.
+ *     (cudaGetSymbolAddress, a synchronous runtime query) with that device
+ *     current and caches it; later calls reuse the cached address.
  *   - The call allocates nothing; it clears the part of the array that must
  *     start at zero (split-K tile counters) with cudaMemsetAsync on `stream`.
  *   - Every call shares the one array and it keeps the last call's contents:
