@@ -346,6 +346,8 @@ WORKLOAD_TITLE = {
     "w4a4_nvfp4": "dense W4A4 NVFP4 x NVFP4, N=K=7168, M in {1,32,256,2048,8192}",
     "w8a8_fp8": "dense W8A8 FP8 per-channel x per-token, N=K=7168, M in {1,32,256,2048,8192}",
     "moe_silu": "MoE gate-up GEMM + SiLU-and-mul at the config-3 shapes, T in {16, 4096}: unfused and fused",
+    "moe_nvfp4_down_profile": "MoE NVFP4 x NVFP4 down GEMM alone (config-5 MoE: E=256, top-8 softmax routing, "
+                              "T=4096, N=7168, K=2048, grouped), only the down weights resident",
     "moe_profile_e64": "MoE W4A16 MXFP4 at the config-3 expert shapes with E=64, T=1024 (about 128 rows per "
                        "expert), grouped + indexed: a small case of the T=4096 calls for profiling",
     "lowbit": "dense WnA16 INT2, INT3, MXFP6 E2M3, float4e0m3 at N=28672, K=8192, M in {1, 16}",
@@ -438,7 +440,8 @@ def moe_call_kernels(hq, wdesc, a_dtype, mode, combine):
     return n + (1 if combine else 0), block_scaled
 
 
-def ops_moe(hq, config, name, wdesc, E, topk, H, I, Ts, routing, gen, a_dtype, modes=("grouped", "indexed")):
+def ops_moe(hq, config, name, wdesc, E, topk, H, I, Ts, routing, gen, a_dtype, modes=("grouped", "indexed"),
+            parts=("gate_up", "down")):
     """MoE calls per T: the routing prepare, then per mode the gate-up GEMM
     (N = 2I, K = H, one activation row per token) and the down GEMM (N = H,
     K = I, one row per routed slot) with the fused weighted top-k sum; a MoE
@@ -446,6 +449,9 @@ def ops_moe(hq, config, name, wdesc, E, topk, H, I, Ts, routing, gen, a_dtype, m
     dev = "cuda"
     weights = {}
     for part, (N, K) in (("gate_up", (2 * I, H)), ("down", (H, I))):
+        if part not in parts:
+            weights[part] = (None, N, K, 0)
+            continue
         if wdesc.w_dtype == hq.HQ_E2M1 and wdesc.w_scale_dtype == hq.HQ_E8M0:
             w = synth.mxfp4_weights(E, N, K, gen, device=dev)
             glob = None
@@ -524,12 +530,14 @@ def ops_moe(hq, config, name, wdesc, E, topk, H, I, Ts, routing, gen, a_dtype, m
             if bs:
                 ratio = 4.0 if wdesc.w_scale_dtype == hq.HQ_UE4M3 else 2.0
             kern = "bs_gemm_kernel" if bs else ("dec_gemm_kernel / tc_gemm_kernel")
-            ops.append(Op(f"{name}_T{T}_{mode_name}_gate_up", run_gate, 2.0 * T * topk * Ng * Kg, touched * bg,
-                          T * Kg * 2 + T * topk * Ng * 2, kg, T * Kg * 2, 0, e2e_gate, kernel=kern, peak_ratio=ratio,
-                          config=config))
-            ops.append(Op(f"{name}_T{T}_{mode_name}_down", run_down, 2.0 * T * topk * Nd * Kd, touched * bd,
-                          T * topk * Kd * 2 + T * Nd * 2, kd, T * topk * Kd * 2, T * Nd * 2, e2e_down, kernel=kern,
-                          peak_ratio=ratio, config=config))
+            if "gate_up" in parts:
+                ops.append(Op(f"{name}_T{T}_{mode_name}_gate_up", run_gate, 2.0 * T * topk * Ng * Kg, touched * bg,
+                              T * Kg * 2 + T * topk * Ng * 2, kg, T * Kg * 2, 0, e2e_gate, kernel=kern,
+                              peak_ratio=ratio, config=config))
+            if "down" in parts:
+                ops.append(Op(f"{name}_T{T}_{mode_name}_down", run_down, 2.0 * T * topk * Nd * Kd, touched * bd,
+                              T * topk * Kd * 2 + T * Nd * 2, kd, T * topk * Kd * 2, T * Nd * 2, e2e_down,
+                              kernel=kern, peak_ratio=ratio, config=config))
     return ops, keep
 
 
@@ -635,6 +643,17 @@ def ops_moe_nvfp4(hq, gen, Ts=(4096,)):
     d = desc_of(hq, hq.HQ_E2M1, 16, hq.HQ_UE4M3, 0, 1, hq.HQ_NVFP4)
     routing = lambda T, g: synth.routing_softmax_topk(T, E_MOE, TOPK, g, device="cuda")
     return ops_moe(hq, 5, "cfg5_moe_nvfp4", d, E_MOE, TOPK, H_MOE, I_MOE, list(Ts), routing, gen, hq.HQ_NVFP4)
+
+
+def ops_moe_nvfp4_down_profile(hq, gen):
+    """A profiling case: the config-5 NVFP4 MoE down GEMM alone (E = 256,
+    top-8 softmax routing of T = 4096 tokens, N = 7168, K = 2048, grouped,
+    with the weighted top-k sum), only the down weights on the device
+    (1.9 GB)."""
+    d = desc_of(hq, hq.HQ_E2M1, 16, hq.HQ_UE4M3, 0, 1, hq.HQ_NVFP4)
+    routing = lambda T, g: synth.routing_softmax_topk(T, E_MOE, TOPK, g, device="cuda")
+    return ops_moe(hq, 5, "moe_nvfp4_down", d, E_MOE, TOPK, H_MOE, I_MOE, [4096], routing, gen, hq.HQ_NVFP4,
+                   modes=("grouped",), parts=("down",))
 
 
 def ops_moe_masked_nvfp4(hq, gen):
@@ -783,6 +802,7 @@ WORKLOADS = {
     "lowbit": _workload([ops_lowbit], WORKLOAD_TITLE["lowbit"]),
     "moe_silu": _workload([ops_moe_silu], WORKLOAD_TITLE["moe_silu"]),
     "moe_profile_e64": _workload([ops_moe_profile_e64], WORKLOAD_TITLE["moe_profile_e64"]),
+    "moe_nvfp4_down_profile": _workload([ops_moe_nvfp4_down_profile], WORKLOAD_TITLE["moe_nvfp4_down_profile"]),
     "moe_w4a16_mxint4": _workload([ops_moe_w4a16_mxint4], WORKLOAD_TITLE["moe_w4a16_mxint4"]),
     "w4a16_asym_sweep": _workload([ops_w4a16_asym_sweep], WORKLOAD_TITLE["w4a16_asym_sweep"]),
     "w4a16_dense_m16": _workload([ops_w4a16_dense_m16], WORKLOAD_TITLE["w4a16_dense_m16"]),
@@ -795,7 +815,7 @@ WORKLOADS = {
 }
 
 # configurations each workload covers (for the CPU samples)
-WORKLOAD_CONFIGS = {"all": (1, 2, 3, 4, 5), "moe_profile_e64": (3,), "w8a8_fp8_block": (5,), "moe_w4a16_mxint4": (3,), "moe_silu": (3,), "lowbit": (2,), "w4a16_asym_sweep": (2,), "w4a16_dense_m16": (1,),
+WORKLOAD_CONFIGS = {"all": (1, 2, 3, 4, 5), "moe_profile_e64": (3,), "moe_nvfp4_down_profile": (5,), "w8a8_fp8_block": (5,), "moe_w4a16_mxint4": (3,), "moe_silu": (3,), "lowbit": (2,), "w4a16_asym_sweep": (2,), "w4a16_dense_m16": (1,),
                     "moe_w4a16_mxfp4": (3,), "moe_w4a8_mxfp8": (4,), "moe_nvfp4": (5,), "moe_masked_nvfp4": (5,),
                     "w4a4_nvfp4": (5,), "w8a8_fp8": (5,)}
 

@@ -180,10 +180,11 @@ __device__ __forceinline__ void decode_bf16(const uint8_t *wpk, const uint8_t *s
         // groups are >= 32 k: one scale (and zero point) per chunk, loaded
         // again only when the second chunk starts a new group (MXINT4: the
         // E8M0 power of two as a bf16, exact)
-        if (c == 0 || gt != (((kbase) >> gshift) - g0)) {
+        if (c == 0 || (gshift < 6 && gt != ((kbase >> gshift) - g0))) {
           s2c = WF == W_MXINT4 ? tc::bcast16(tc::e8m0_code_to_bf16(sc[gt * BM + r]))
                                : tc::bcast16(reinterpret_cast<const uint16_t *>(sc)[gt * BM + r]);
-          z2c = (WF == W_UINT4) ? tc::bcast16(0x4300u + zp[gt * BM + r]) : 0x43084308u;
+          // bf16 pair 128 + z in both halves, one multiply-add
+          z2c = (WF == W_UINT4) ? 0x43004300u + (uint32_t)zp[gt * BM + r] * 0x10001u : 0x43084308u;
         }
         const uint32_t s2 = s2c, z2 = z2c;
 #pragma unroll

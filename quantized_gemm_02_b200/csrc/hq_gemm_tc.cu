@@ -254,7 +254,7 @@ __device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b) {
   __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162 *>(&a), *reinterpret_cast<__nv_bfloat162 *>(&b));
   return *reinterpret_cast<uint32_t *>(&r);
 }
-__device__ __forceinline__ uint32_t bcast16(uint32_t h) { return (h & 0xFFFFu) | (h << 16); }
+__device__ __forceinline__ uint32_t bcast16(uint32_t h) { return (h & 0xFFFFu) * 0x10001u; }
 // bf16 bits of an E4M3 / UE4M3 code's value (exact: <= 4 significant bits)
 __device__ __forceinline__ uint32_t e4m3_code_to_bf16(uint32_t c) {
   const float mag = __uint_as_float((c & 0x7Fu) << 20) * 1.329227995784916e36f;  // 2^120
