@@ -185,17 +185,21 @@ __device__ __forceinline__ void epilogue_segment(const Params &p, const TileInfo
       orow_l = p.moe ? p.perm[pos] : pos;
       if (p.row_scale) rs_l = p.row_scale[p.moe ? orow_l / p.a_div : pos];
     }
+    auto stores = [&](auto gated) {
 #pragma unroll
-    for (int i = 0; i < CW; ++i) {
-      const int orow = __shfl_sync(0xffffffffu, orow_l, i);
-      const float rs = __shfl_sync(0xffffffffu, rs_l, i);
-      // FP8: per-token x per-row scales; block-scaled kinds: global scales
-      float z = x[i];
-      if (p.row_scale) z *= rs;
-      z *= cs;
-      z *= gs;
-      tc::put_out(p, orow, n, z, c0 + i < ti.nvalid && n < p.N);
-    }
+      for (int i = 0; i < CW; ++i) {
+        const int orow = __shfl_sync(0xffffffffu, orow_l, i);
+        const float rs = __shfl_sync(0xffffffffu, rs_l, i);
+        // FP8: per-token x per-row scales; block-scaled kinds: global scales
+        float z = x[i];
+        if (p.row_scale) z *= rs;
+        z *= cs;
+        z *= gs;
+        tc::put_out<decltype(gated)::value>(p, orow, n, z, c0 + i < ti.nvalid && n < p.N);
+      }
+    };
+    if (p.gated) stores(tc::GatedTag<true>{});
+    else stores(tc::GatedTag<false>{});
   };
 #pragma unroll 1
   for (int c0 = 0; c0 < BNT; c0 += CW) {
@@ -638,11 +642,15 @@ __device__ __forceinline__ void f8b_finish(const Params &p, const TileInfo &ti, 
       const int pos = ti.base + c0 + lane;
       orow_l = p.moe ? p.perm[pos] : pos;
     }
+    auto stores = [&](auto gated) {
 #pragma unroll
-    for (int i = 0; i < CW; ++i) {
-      const int orow = __shfl_sync(0xffffffffu, orow_l, i);
-      tc::put_out(p, orow, n, x[i], c0 + i < ti.nvalid && n < p.N);
-    }
+      for (int i = 0; i < CW; ++i) {
+        const int orow = __shfl_sync(0xffffffffu, orow_l, i);
+        tc::put_out<decltype(gated)::value>(p, orow, n, x[i], c0 + i < ti.nvalid && n < p.N);
+      }
+    };
+    if (p.gated) stores(tc::GatedTag<true>{});
+    else stores(tc::GatedTag<false>{});
   };
   if (whole) {
 #pragma unroll

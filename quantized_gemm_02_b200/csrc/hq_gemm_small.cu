@@ -243,16 +243,20 @@ __device__ __forceinline__ void store_rows(const Params &p, const TileInfo &ti, 
     orow_l = p.moe ? p.perm[pos] : pos;
     if (p.row_scale) rs_l = p.row_scale[p.moe ? orow_l / p.a_div : pos];
   }
+  auto stores = [&](auto gated) {
 #pragma unroll
-  for (int m = 0; m < BNT; ++m) {
-    const int orow = __shfl_sync(0xffffffffu, orow_l, m);
-    const float rs = __shfl_sync(0xffffffffu, rs_l, m);
-    float z = x[m];
-    if (p.row_scale) z *= rs;
-    z *= cs;
-    z *= gs;
-    tc::put_out(p, orow, n, z, m < ti.nvalid && n < p.N);
-  }
+    for (int m = 0; m < BNT; ++m) {
+      const int orow = __shfl_sync(0xffffffffu, orow_l, m);
+      const float rs = __shfl_sync(0xffffffffu, rs_l, m);
+      float z = x[m];
+      if (p.row_scale) z *= rs;
+      z *= cs;
+      z *= gs;
+      tc::put_out<decltype(gated)::value>(p, orow, n, z, m < ti.nvalid && n < p.N);
+    }
+  };
+  if (p.gated) stores(tc::GatedTag<true>{});
+  else stores(tc::GatedTag<false>{});
 }
 
 template <int BNT>

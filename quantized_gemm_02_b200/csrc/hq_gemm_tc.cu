@@ -235,14 +235,21 @@ __device__ __forceinline__ float silu_mul(float g, float u) {
 // rows 2j and 2j + 1 exchange their values and the even lane writes
 // silu(gate) * up at column n / 2 of an N / 2-wide row.  All 32 lanes of the
 // warp call it together (consecutive lanes = consecutive weight rows).
+// The epilogues pick the form once per block of stores (GatedTag<p.gated>),
+// so that the plain stores of a block issue back to back.
+template <bool G>
+struct GatedTag {
+  static constexpr bool value = G;
+};
+template <bool G>
 __device__ __forceinline__ void put_out(const Params &p, int orow, int n, float z, bool ok) {
-  if (!p.gated) {
+  if constexpr (!G) {
     if (ok) p.out[(size_t)orow * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(z));
-    return;
+  } else {
+    const float u = __shfl_xor_sync(0xffffffffu, z, 1);
+    if (ok && !(n & 1))
+      p.out[(size_t)orow * (p.N >> 1) + (n >> 1)] = __bfloat16_as_ushort(__float2bfloat16_rn(silu_mul(z, u)));
   }
-  const float u = __shfl_xor_sync(0xffffffffu, z, 1);
-  if (ok && !(n & 1))
-    p.out[(size_t)orow * (p.N >> 1) + (n >> 1)] = __bfloat16_as_ushort(__float2bfloat16_rn(silu_mul(z, u)));
 }
 
 // ---- bf16 pair arithmetic and decoders ---------------------------------------
@@ -771,16 +778,20 @@ __global__ void __launch_bounds__(THREADS, (BNT <= 64 ? 2 : 1)) tc_gemm_kernel(c
             orow_l = p.moe ? p.perm[pos] : pos;
             if (p.row_scale) rs_l = p.row_scale[p.moe ? orow_l / p.a_div : pos];
           }
+          auto stores = [&](auto gated) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int orow = __shfl_sync(0xffffffffu, orow_l, i);
-            const float rs = __shfl_sync(0xffffffffu, rs_l, i);
-            float x = v[i];
-            if (p.row_scale) x *= rs;
-            x *= cs;
-            x *= gs;
-            put_out(p, orow, n, x, c0 + i < ti.nvalid && n < p.N);
-          }
+            for (int i = 0; i < 16; ++i) {
+              const int orow = __shfl_sync(0xffffffffu, orow_l, i);
+              const float rs = __shfl_sync(0xffffffffu, rs_l, i);
+              float x = v[i];
+              if (p.row_scale) x *= rs;
+              x *= cs;
+              x *= gs;
+              put_out<decltype(gated)::value>(p, orow, n, x, c0 + i < ti.nvalid && n < p.N);
+            }
+          };
+          if (p.gated) stores(GatedTag<true>{});
+          else stores(GatedTag<false>{});
         }
       }
       if (split_mode) __threadfence();  // partial visible before the tile ticket
