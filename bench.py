@@ -346,6 +346,8 @@ WORKLOAD_TITLE = {
     "w4a4_nvfp4": "dense W4A4 NVFP4 x NVFP4, N=K=7168, M in {1,32,256,2048,8192}",
     "w8a8_fp8": "dense W8A8 FP8 per-channel x per-token, N=K=7168, M in {1,32,256,2048,8192}",
     "moe_silu": "MoE gate-up GEMM + SiLU-and-mul at the config-3 shapes, T in {16, 4096}: unfused and fused",
+    "moe_indexed_gate_up_profile": "MoE W4A16 MXFP4 gate-up GEMM alone, indexed mode (config-3 MoE: E=256, top-8 "
+                                   "softmax routing, T=4096, N=4096, K=7168), only the gate-up weights resident",
     "moe_nvfp4_down_profile": "MoE NVFP4 x NVFP4 down GEMM alone (config-5 MoE: E=256, top-8 softmax routing, "
                               "T=4096, N=7168, K=2048, grouped), only the down weights resident",
     "moe_profile_e64": "MoE W4A16 MXFP4 at the config-3 expert shapes with E=64, T=1024 (about 128 rows per "
@@ -656,6 +658,16 @@ def ops_moe_nvfp4_down_profile(hq, gen):
                    modes=("grouped",), parts=("down",))
 
 
+def ops_moe_w4a16_indexed_gate_up_profile(hq, gen):
+    """A profiling case: the config-3 MoE W4A16 MXFP4 gate-up GEMM alone in
+    indexed mode at T = 4096 (E = 256, top-8 softmax routing, N = 4096,
+    K = 7168), only the gate-up weights on the device (3.8 GB)."""
+    d = desc_of(hq, hq.HQ_E2M1, 32, hq.HQ_E8M0, 0, 0, hq.HQ_BF16)
+    routing = lambda T, g: synth.routing_softmax_topk(T, E_MOE, TOPK, g, device="cuda")
+    return ops_moe(hq, 3, "cfg3_moe_w4a16", d, E_MOE, TOPK, H_MOE, I_MOE, [4096], routing, gen, hq.HQ_BF16,
+                   modes=("indexed",), parts=("gate_up",))
+
+
 def ops_moe_masked_nvfp4(hq, gen):
     """Masked-layout MoE (expert slabs with per-expert valid counts), NVFP4 x
     NVFP4, config-5 MoE shapes: the counts come from a softmax top-8 routing
@@ -803,6 +815,8 @@ WORKLOADS = {
     "moe_silu": _workload([ops_moe_silu], WORKLOAD_TITLE["moe_silu"]),
     "moe_profile_e64": _workload([ops_moe_profile_e64], WORKLOAD_TITLE["moe_profile_e64"]),
     "moe_nvfp4_down_profile": _workload([ops_moe_nvfp4_down_profile], WORKLOAD_TITLE["moe_nvfp4_down_profile"]),
+    "moe_indexed_gate_up_profile": _workload([ops_moe_w4a16_indexed_gate_up_profile],
+                                             WORKLOAD_TITLE["moe_indexed_gate_up_profile"]),
     "moe_w4a16_mxint4": _workload([ops_moe_w4a16_mxint4], WORKLOAD_TITLE["moe_w4a16_mxint4"]),
     "w4a16_asym_sweep": _workload([ops_w4a16_asym_sweep], WORKLOAD_TITLE["w4a16_asym_sweep"]),
     "w4a16_dense_m16": _workload([ops_w4a16_dense_m16], WORKLOAD_TITLE["w4a16_dense_m16"]),
@@ -815,7 +829,7 @@ WORKLOADS = {
 }
 
 # configurations each workload covers (for the CPU samples)
-WORKLOAD_CONFIGS = {"all": (1, 2, 3, 4, 5), "moe_profile_e64": (3,), "moe_nvfp4_down_profile": (5,), "w8a8_fp8_block": (5,), "moe_w4a16_mxint4": (3,), "moe_silu": (3,), "lowbit": (2,), "w4a16_asym_sweep": (2,), "w4a16_dense_m16": (1,),
+WORKLOAD_CONFIGS = {"all": (1, 2, 3, 4, 5), "moe_profile_e64": (3,), "moe_nvfp4_down_profile": (5,), "moe_indexed_gate_up_profile": (3,), "w8a8_fp8_block": (5,), "moe_w4a16_mxint4": (3,), "moe_silu": (3,), "lowbit": (2,), "w4a16_asym_sweep": (2,), "w4a16_dense_m16": (1,),
                     "moe_w4a16_mxfp4": (3,), "moe_w4a8_mxfp8": (4,), "moe_nvfp4": (5,), "moe_masked_nvfp4": (5,),
                     "w4a4_nvfp4": (5,), "w8a8_fp8": (5,)}
 

@@ -433,21 +433,25 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       if (is >= NS && !mbar_wait(&sfree[s], ph ^ 1)) { *s_abort = 1; break; }
       if (*(volatile int *)s_abort) break;
+      const int ng = (nvalid + 3) >> 2;  // indexed mode: four 128-byte rows per gather
       if (lane == 0) {
         uint8_t *st = smem + s * C::STAGE;
         if (!p.gather) {
           mbar_arrive_expect_tx(&full[s], (uint32_t)(C::A_SMEM + C::SF_CH * C::SFB_CHB));
           tma_load_2d(st + C::W_SMEM, &a_map, w.ks * 128, base, &full[s]);
         } else {
-          // indexed mode: the tile's caller rows, four 128-byte rows per gather
-          const int ng = (nvalid + 3) >> 2;
           mbar_arrive_expect_tx(&full[s], (uint32_t)(ng * 4 * 128 + C::SF_CH * C::SFB_CHB));
-          for (int gi = 0; gi < ng; ++gi)
-            tc::tma_gather4(st + C::W_SMEM + gi * 512, &a_map, w.ks * 128, s_rows[4 * gi], s_rows[4 * gi + 1],
-                            s_rows[4 * gi + 2], s_rows[4 * gi + 3], &full[s]);
         }
         if constexpr (C::SF_CH > 0)
           bulk_g2s(st + C::SFB_OFF, sfsrc + (size_t)w.ks * C::SF_CH * C::SFB_CHB, C::SF_CH * C::SFB_CHB, &full[s]);
+      }
+      if (p.gather) {
+        // the tile's caller rows, one 4-row gather per lane at a time
+        __syncwarp();
+        uint8_t *st = smem + s * C::STAGE;
+        for (int gi = lane; gi < ng; gi += 32)
+          tc::tma_gather4(st + C::W_SMEM + gi * 512, &a_map, w.ks * 128, s_rows[4 * gi], s_rows[4 * gi + 1],
+                          s_rows[4 * gi + 2], s_rows[4 * gi + 3], &full[s]);
       }
       __syncwarp();
       if (++s == NS) { s = 0; ph ^= 1; }
@@ -842,17 +846,18 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (is >= NS && !mbar_wait(&sfree[s], ph ^ 1)) { *s_abort = 1; break; }
       if (*(volatile int *)s_abort) break;
       uint8_t *st = smem + s * C::STAGE;
+      const int ng = (nvalid + 3) >> 2;  // indexed mode: four 128-byte rows per gather
       if (lane == 0) {
-        const int ng = (nvalid + 3) >> 2;  // indexed mode: four 128-byte rows per gather
         mbar_arrive_expect_tx(&full[s], (uint32_t)((p.gather ? ng * 4 * 128 : C::A_SMEM) + BNT * 4));
-        if (!p.gather) {
-          tma_load_2d(st + C::W_SMEM, &a_map, w.ks * 128, base, &full[s]);
-        } else {
-          for (int gi = 0; gi < ng; ++gi)
-            tc::tma_gather4(st + C::W_SMEM + gi * 512, &a_map, w.ks * 128, s_rows[4 * gi], s_rows[4 * gi + 1],
-                            s_rows[4 * gi + 2], s_rows[4 * gi + 3], &full[s]);
-        }
+        if (!p.gather) tma_load_2d(st + C::W_SMEM, &a_map, w.ks * 128, base, &full[s]);
         bulk_g2s(st + C::SA_OFF, sasrc + (size_t)w.ks * BNT * 4, (uint32_t)(BNT * 4), &full[s]);
+      }
+      if (p.gather) {
+        // one 4-row gather per lane at a time
+        __syncwarp();
+        for (int gi = lane; gi < ng; gi += 32)
+          tc::tma_gather4(st + C::W_SMEM + gi * 512, &a_map, w.ks * 128, s_rows[4 * gi], s_rows[4 * gi + 1],
+                          s_rows[4 * gi + 2], s_rows[4 * gi + 3], &full[s]);
       }
       __syncwarp();
       if (++s == NS) { s = 0; ph ^= 1; }

@@ -496,16 +496,17 @@ __global__ void __launch_bounds__(THREADS, 1) dec_gemm_kernel(const __grid_const
       } else {
         const int ng = (nvalid + 3) >> 2;  // 4-row gathers per 64-k block
         if (lane == 0) mbar_arrive_expect_tx(&full[rs.idx], (uint32_t)(w.n * ng * 4 * 128));
-        for (int gi = 0; gi < ng; ++gi) {
-          const int r0 = __shfl_sync(0xffffffffu, my_row, 4 * gi);
-          const int r1 = __shfl_sync(0xffffffffu, my_row, 4 * gi + 1);
-          const int r2 = __shfl_sync(0xffffffffu, my_row, 4 * gi + 2);
-          const int r3 = __shfl_sync(0xffffffffu, my_row, 4 * gi + 3);
-          if (lane == 0)
-            for (int j = 0; j < w.n; ++j)
-              tc::tma_gather4(st + j * C::ACT_KB + gi * 512, &act_map, (w.kb + j) * TILE_K, r0, r1, r2, r3,
-                              &full[rs.idx]);
-        }
+        __syncwarp();
+        // lane 4 * gi + j issues the gather of rows 4gi..4gi+3 for block j
+        // (BNT <= 32: at most 8 groups x 4 blocks), all lanes at once
+        const int gi = lane >> 2, j = lane & 3;
+        const int r0 = __shfl_sync(0xffffffffu, my_row, (4 * gi) & 31);
+        const int r1 = __shfl_sync(0xffffffffu, my_row, (4 * gi + 1) & 31);
+        const int r2 = __shfl_sync(0xffffffffu, my_row, (4 * gi + 2) & 31);
+        const int r3 = __shfl_sync(0xffffffffu, my_row, (4 * gi + 3) & 31);
+        if (gi < ng && j < w.n)
+          tc::tma_gather4(st + j * C::ACT_KB + gi * 512, &act_map, (w.kb + j) * TILE_K, r0, r1, r2, r3,
+                          &full[rs.idx]);
       }
       __syncwarp();
     }

@@ -63,7 +63,7 @@ struct Traits {
 // otherwise weights are dequantised to bf16 (kind::f16).
 template <int WF, int BNT, bool F8>
 struct Cfg {
-  static constexpr int KPS = BNT <= 16 ? 4 : BNT <= 64 ? 2 : 1;               // 64-k blocks per stage
+  static constexpr int KPS = BNT <= 16 ? 4 : BNT <= 64 ? 2 : BNT <= 128 ? 3 : 1;  // 64-k blocks per stage
   static constexpr int A_COLS = F8 ? 16 : 32;                                  // TMEM columns per 64-k block
   static constexpr int ACT_KB = BNT * (F8 ? 64 : 128);                         // one block of activations
   static constexpr int ACT = KPS * ACT_KB;                                     // [KPS][BNT][64], swizzled
@@ -569,15 +569,9 @@ __global__ void __launch_bounds__(THREADS, (BNT <= 64 ? 2 : 1)) tc_gemm_kernel(c
         // indexed mode: ceil(nvalid / 4) gathers of four 128-byte rows per 64-k block
         const uint32_t ab = p.gather ? (uint32_t)(((ti.nvalid + 3) / 4) * 4 * 128) : (uint32_t)C::ACT_KB;
         mbar_arrive_expect_tx(&full[s], ab * nblk + TR::unit * nblk + sb + zb);
-        for (int j = 0; j < nblk; ++j) {
-          if (!p.gather) {
+        if (!p.gather)
+          for (int j = 0; j < nblk; ++j)
             tma_load_2d(st + j * C::ACT_KB, &act_map, (kbs + j) * TILE_K, ti.base, &full[s]);
-          } else {
-            for (int i = 0; i < ti.nvalid; i += 4)
-              tma_gather4(st + j * C::ACT_KB + i * 128, &act_map, (kbs + j) * TILE_K, s_rows[i], s_rows[i + 1],
-                          s_rows[i + 2], s_rows[i + 3], &full[s]);
-          }
-        }
         bulk_g2s_stream(st + C::ACT, eb + p.w_off + ((size_t)ti.wt * p.KB + kbs) * TR::unit, TR::unit * nblk,
                         &full[s], pol);
         if (TR::has_scales)
@@ -587,6 +581,16 @@ __global__ void __launch_bounds__(THREADS, (BNT <= 64 ? 2 : 1)) tc_gemm_kernel(c
           bulk_g2s(st + C::ACT + C::WPK + C::SC, eb + p.z_off + ((size_t)ti.wt * p.G + g0) * BM, zb, &full[s]);
       }
       __syncwarp();
+      if (p.gather) {
+        // indexed mode: the stage's 4-row gathers, one group of rows per lane
+        // (issued by all lanes at once: from one lane they are ~25 % slower)
+        uint8_t *st = smem + s * C::STAGE;
+        for (int j = 0; j < nblk; ++j)
+          for (int i = 4 * lane; i < ti.nvalid; i += 128)
+            tma_gather4(st + j * C::ACT_KB + i * 128, &act_map, (kbs + j) * TILE_K, s_rows[i], s_rows[i + 1],
+                        s_rows[i + 2], s_rows[i + 3], &full[s]);
+        __syncwarp();
+      }
       }
     }
   } else if (warp >= WARP_DQ0) {
