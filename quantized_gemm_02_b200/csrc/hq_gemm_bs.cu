@@ -893,6 +893,20 @@ __global__ void __launch_bounds__(THREADS, 1)
     Walk w;
     w.start(beg, end, p.KB);
     int t0 = w.t, ks0 = w.ks;  // where the current segment started
+    // the weight block scale of a stage, loaded one stage ahead so that its
+    // latency is off the promotion's path (tile lookups only when the tile changes)
+    int sw_t = -1;
+    const float *sw_row = nullptr;
+    auto sw_of = [&](int t, int ks) {
+      if (t != sw_t) {
+        const TileInfo ti = tile_info(t);
+        sw_row = reinterpret_cast<const float *>(p.packed + (size_t)ti.expert * p.stride + p.c_off) +
+                 (size_t)ti.wt * p.KB;
+        sw_t = t;
+      }
+      return __ldg(sw_row + ks);
+    };
+    float sw_next = sw_of(w.t, w.ks);
     for (int is = 0, s = 0, ph = 0, q = 0, qph = 0; w.left > 0; ++is, w.next(p.KB)) {
       if (w.seg_first) {
 #pragma unroll
@@ -900,9 +914,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         t0 = w.t;
         ks0 = w.ks;
       }
-      const TileInfo ti = tile_info(w.t);
-      const float sw = __ldg(reinterpret_cast<const float *>(p.packed + (size_t)ti.expert * p.stride + p.c_off) +
-                             (size_t)ti.wt * p.KB + w.ks);
+      const float sw = sw_next;
+      if (w.left > 1) {
+        Walk wn = w;
+        wn.next(p.KB);
+        sw_next = sw_of(wn.t, wn.ks);
+      }
       // the stage (its activation scales) has landed, and its MMAs are done
       const bool ok = mbar_wait(&full[s], ph) && mbar_wait(&pfull[q], qph);
       tc::tc_fence_after();
