@@ -131,6 +131,25 @@ __device__ __forceinline__ void mma_bs(uint32_t tmem_d, uint64_t adesc, uint64_t
   }
 }
 
+// 32 fp32 accumulator columns of this warp's TMEM lanes: the load and its
+// wait in one statement, so that no use of the registers can be scheduled
+// before the data has arrived.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
+      "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
@@ -204,12 +223,16 @@ __device__ __forceinline__ void epilogue_segment(const Params &p, const TileInfo
 #pragma unroll 1
   for (int c0 = 0; c0 < BNT; c0 += CW) {
     float v[CW];
+    if constexpr (CW == 32) {
+      tmem_ld32(tacc + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
+    } else {
 #pragma unroll
-    for (int h = 0; h < CW; h += 16) {
-      float v16[16];
-      tc::tmem_ld16(tacc + ((uint32_t)(warp * 32) << 16) + (uint32_t)(c0 + h), v16);
+      for (int h = 0; h < CW; h += 16) {
+        float v16[16];
+        tc::tmem_ld16(tacc + ((uint32_t)(warp * 32) << 16) + (uint32_t)(c0 + h), v16);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) v[h + i] = v16[i];
+        for (int i = 0; i < 16; ++i) v[h + i] = v16[i];
+      }
     }
     if (whole) {
       write(c0, v);
@@ -925,12 +948,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc::tc_fence_after();
       if (!ok || *(volatile int *)s_abort) break;
       const float *sa = reinterpret_cast<const float *>(smem + s * C::STAGE + C::SA_OFF);
+      constexpr int CL = BNT < 32 ? 16 : 32;  // columns per TMEM load (one wait each)
 #pragma unroll
-      for (int c0 = 0; c0 < BNT; c0 += 16) {
-        float v[16];
-        tc::tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(q * BNT + c0), v);
+      for (int c0 = 0; c0 < BNT; c0 += CL) {
+        float v[CL];
+        if constexpr (CL == 32) tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(q * BNT + c0), v);
+        else tc::tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(q * BNT + c0), v);
 #pragma unroll
-        for (int i = 0; i < 16; i += 4) {
+        for (int i = 0; i < CL; i += 4) {
           const float4 a4 = *reinterpret_cast<const float4 *>(sa + c0 + i);
           acc[c0 + i] = fmaf(v[i], __fmul_rn(sw, a4.x), acc[c0 + i]);
           acc[c0 + i + 1] = fmaf(v[i + 1], __fmul_rn(sw, a4.y), acc[c0 + i + 1]);

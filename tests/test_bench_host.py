@@ -21,3 +21,27 @@ def test_sweep_entry_roofline_fractions():
     e2 = bench.sweep_entry(op2, 0.43, peaks)
     assert abs(e2["tensor_frac"] - op2.flops / 0.43e-3 / 1e12 / (4 * 1648.3)) < 1e-3
     assert e2["roofline_frac"] == e2["tensor_frac"]
+
+
+def test_every_workload_has_a_title_and_its_configs():
+    for name in bench.WORKLOADS:
+        assert name in bench.WORKLOAD_CONFIGS, name
+        if name != "all":
+            assert name in bench.WORKLOAD_TITLE, name
+
+
+def test_measured_traffic_follows_the_kernel_source_digest(tmp_path, monkeypatch):
+    digest = bench.kernel_source_digest()
+    assert len(digest) == 16 and int(digest, 16) >= 0
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (prof / "traffic.md").write_text(
+        "| op | kernel | read | write | traffic | digest |\n|---|---|---|---|---|---|\n"
+        f"| op_a | k | 1 | 2 | 3 | {digest} |\n"
+        "| op_b | k | 1 | 2 | 5 | 0000000000000000 |\n")
+    # the digest is taken of the real kernel sources, the table from the temporary root
+    monkeypatch.setattr(bench, "kernel_source_digest", lambda: digest)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.measured_traffic("op_a") == 3.0
+    assert bench.measured_traffic("op_b") is None  # captured on other sources
+    assert bench.measured_traffic("op_c") is None
