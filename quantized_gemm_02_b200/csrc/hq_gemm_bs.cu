@@ -650,6 +650,12 @@ struct CfgF8B {
   static constexpr int BYTES = NS * STAGE + CTRL + 1024;
   static constexpr int NP = (512 / BNT) > 4 ? 4 : (512 / BNT);  // stage accumulators in TMEM
   static constexpr int TMEM_COLS = NP * BNT < 32 ? 32 : NP * BNT;
+  // promotion groups of four warps (one per TMEM lane quadrant), each taking
+  // BNT / PG token columns of every stage: warps 0..3 and, with two groups,
+  // warps 7..10 (after the producers and the MMA issuer)
+  static constexpr int PG = BNT >= 64 ? 2 : 1;
+  static constexpr int PCOLS = BNT / PG;
+  static constexpr int THREADS = (7 + 4 * (PG - 1)) * 32;
   static_assert(NS >= 3 && NP >= 2, "budget");
   static_assert((TMEM_COLS & (TMEM_COLS - 1)) == 0, "TMEM allocation is a power of two");
 };
@@ -657,11 +663,14 @@ struct CfgF8B {
 // Output of one promoted segment (thread = weight row n): whole tiles are
 // written; a Stream-K piece is stored as fp32 partials, and the last of the
 // CTAs sharing the tile sums the parts in k order (32 columns at a time).
-template <int BNT>
+template <int BNT, int PG>
 __device__ __forceinline__ void f8b_finish(const Params &p, const TileInfo &ti, int t, bool whole, bool head,
-                                           const float (&acc)[BNT], int cta, int warp, int lane, long long total) {
+                                           const float (&acc)[BNT / PG], int cbeg, int cta, int quad, int lane,
+                                           long long total) {
+  constexpr int PCOLS = BNT / PG;
   constexpr int CW = BNT < 32 ? BNT : 32;
-  const int r = warp * 32 + lane;
+  constexpr int CWP = PCOLS < 32 ? PCOLS : 32;
+  const int r = quad * 32 + lane;
   const int n = ti.wt * BM + r;
   auto write = [&](int c0, const float *x) {
     int orow_l = 0;
@@ -680,13 +689,15 @@ __device__ __forceinline__ void f8b_finish(const Params &p, const TileInfo &ti, 
     else stores(tc::GatedTag<false>{});
   };
   if (whole) {
+    // this group's columns [cbeg, cbeg + PCOLS)
+    static_assert(CWP == CW, "a group writes whole column chunks");
 #pragma unroll
-    for (int c0 = 0; c0 < BNT; c0 += CW) write(c0, acc + c0);
+    for (int c0 = 0; c0 < PCOLS; c0 += CW) write(cbeg + c0, acc + c0);
     return;
   }
   float *part = p.partial + ((size_t)cta * 2 + (head ? 0 : 1)) * BNT * BM;
 #pragma unroll
-  for (int m = 0; m < BNT; ++m) __stcg(&part[(size_t)m * BM + r], acc[m]);
+  for (int m = 0; m < PCOLS; ++m) __stcg(&part[(size_t)(cbeg + m) * BM + r], acc[m]);
   __threadfence();
   __syncwarp();
   const long long t_first = (long long)t * p.KB;
@@ -694,8 +705,10 @@ __device__ __forceinline__ void f8b_finish(const Params &p, const TileInfo &ti, 
   const int c_last = dec::cta_of(t_first + p.KB - 1, total, p.nctas);
   int last = 0;
   if (lane == 0) {
-    int *ctr = p.counters + (size_t)t * 4 + warp;
-    last = (atomicAdd(ctr, 1) == c_last - c_first);
+    // one ticket per lane quadrant: every group of every contributing CTA
+    // takes one; the last sums all BNT columns of the quadrant's rows
+    int *ctr = p.counters + (size_t)t * 4 + quad;
+    last = (atomicAdd(ctr, 1) == PG * (c_last - c_first + 1) - 1);
     if (last) *ctr = 0;  // ready for the next call
   }
   last = __shfl_sync(0xffffffffu, last, 0);
@@ -716,7 +729,7 @@ __device__ __forceinline__ void f8b_finish(const Params &p, const TileInfo &ti, 
 }
 
 template <int BNT>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(CfgF8B<BNT>::THREADS, 1)
     bsf_gemm_kernel(const __grid_constant__ CUtensorMap w_map, const __grid_constant__ CUtensorMap a_map,
                     const Params p) {
   using C = CfgF8B<BNT>;
@@ -767,11 +780,11 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (tid == 32) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 2);      // weight producer and activation producer
-      mbar_init(&sfree[s], 1 + 4);  // MMA commit and the four promotion warps
+      mbar_init(&sfree[s], 1 + 4 * C::PG);  // MMA commit and the promotion warps
     }
     for (int q = 0; q < NP; ++q) {
       mbar_init(&pfull[q], 1);
-      mbar_init(&pempty[q], 4);
+      mbar_init(&pempty[q], 4 * C::PG);
     }
     fence_barrier_init();
   }
@@ -815,7 +828,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     tc::tc_fence_before();
-    asm volatile("bar.sync 1, %0;" ::"r"(THREADS - 64) : "memory");
+    asm volatile("bar.sync 1, %0;" ::"r"(C::THREADS - 64) : "memory");
     tc::tc_fence_after();
     tmem = __shfl_sync(0xffffffffu, *tmem_slot, 0);
   }
@@ -910,9 +923,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (++s == NS) { s = 0; ph ^= 1; }
       if (++q == NP) { q = 0; qph ^= 1; }
     }
-  } else if (warp < 4) {
-    // ================= promotion: warps 0..3, thread = weight row =================
-    float acc[BNT];
+  } else if (warp < 4 || warp >= 7) {
+    // ================= promotion: thread = weight row of lane quadrant warp & 3, =================
+    // ================= token columns [cb, cb + PCOLS) (group 0: warps 0..3, 1: 7..10) =================
+    constexpr int PCOLS = C::PCOLS;
+    const int quad = warp & 3;
+    const int cb = warp >= 7 ? PCOLS : 0;
+    float acc[PCOLS];
     Walk w;
     w.start(beg, end, p.KB);
     int t0 = w.t, ks0 = w.ks;  // where the current segment started
@@ -933,7 +950,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int is = 0, s = 0, ph = 0, q = 0, qph = 0; w.left > 0; ++is, w.next(p.KB)) {
       if (w.seg_first) {
 #pragma unroll
-        for (int m = 0; m < BNT; ++m) acc[m] = 0.f;
+        for (int m = 0; m < PCOLS; ++m) acc[m] = 0.f;
         t0 = w.t;
         ks0 = w.ks;
       }
@@ -948,15 +965,16 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc::tc_fence_after();
       if (!ok || *(volatile int *)s_abort) break;
       const float *sa = reinterpret_cast<const float *>(smem + s * C::STAGE + C::SA_OFF);
-      constexpr int CL = BNT < 32 ? 16 : 32;  // columns per TMEM load (one wait each)
+      constexpr int CL = PCOLS < 32 ? 16 : 32;  // columns per TMEM load (one wait each)
+      const uint32_t tq = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(q * BNT + cb);
 #pragma unroll
-      for (int c0 = 0; c0 < BNT; c0 += CL) {
+      for (int c0 = 0; c0 < PCOLS; c0 += CL) {
         float v[CL];
-        if constexpr (CL == 32) tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(q * BNT + c0), v);
-        else tc::tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(q * BNT + c0), v);
+        if constexpr (CL == 32) tmem_ld32(tq + (uint32_t)c0, v);
+        else tc::tmem_ld16(tq + (uint32_t)c0, v);
 #pragma unroll
         for (int i = 0; i < CL; i += 4) {
-          const float4 a4 = *reinterpret_cast<const float4 *>(sa + c0 + i);
+          const float4 a4 = *reinterpret_cast<const float4 *>(sa + cb + c0 + i);
           acc[c0 + i] = fmaf(v[i], __fmul_rn(sw, a4.x), acc[c0 + i]);
           acc[c0 + i + 1] = fmaf(v[i + 1], __fmul_rn(sw, a4.y), acc[c0 + i + 1]);
           acc[c0 + i + 2] = fmaf(v[i + 2], __fmul_rn(sw, a4.z), acc[c0 + i + 2]);
@@ -971,7 +989,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       if (w.seg_last) {
         const bool whole = (ks0 == 0) && (w.ks == p.KB - 1);
-        f8b_finish<BNT>(p, tile_info(t0), t0, whole, ks0 > 0, acc, cta, warp, lane, total);
+        f8b_finish<BNT, C::PG>(p, tile_info(t0), t0, whole, ks0 > 0, acc, cb, cta, quad, lane, total);
       }
       if (++s == NS) { s = 0; ph ^= 1; }
       if (++q == NP) { q = 0; qph ^= 1; }
@@ -1111,7 +1129,7 @@ static hq_status bsf_launch_one(const CUtensorMap &wm, const CUtensorMap &am, co
       return HQ_ERR_CUDA;
     if (dev < 32) configured |= 1u << dev;
   }
-  kern<<<t.nctas, bs::THREADS, C::BYTES, st>>>(wm, am, p);
+  kern<<<t.nctas, C::THREADS, C::BYTES, st>>>(wm, am, p);
   return check_launch();
 }
 
