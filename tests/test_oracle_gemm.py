@@ -227,6 +227,21 @@ def test_moe_permute_bruteforce():
     assert all(len(set(r)) == k for r in ids.tolist())
 
 
+@pytest.mark.parametrize("T", [64, 512, 4096])
+def test_zipf_routing_spans_empty_to_more_than_an_eighth(T):
+    # the config-4 input recipe: Zipf(1.2) popularity over 256 experts, top-8
+    # distinct per token; per-expert counts must reach from 0 (T = 64) to more
+    # than T / 8, so the MoE tests and bench see both empty and crowded experts
+    g = synth.generator(900 + T)
+    ids, wts = synth.routing_zipf(T, 256, 8, 1.2, g)
+    counts = np.bincount(ids.numpy().reshape(-1), minlength=256)
+    assert counts.sum() == T * 8
+    assert counts.max() > T // 8
+    if T <= 512:
+        assert counts.min() == 0
+    assert np.allclose(wts.sum(dim=-1).numpy(), 1.0, atol=1e-6)
+
+
 def test_moe_masked_matches_routed_top1_and_ignores_invalid_rows():
     # a top-1 routing laid out as slabs (expert e's tokens in token order,
     # padded to the slab) gives the routed MoE's per-slot outputs exactly;
