@@ -944,6 +944,10 @@ TcLaunch plan_tc(int rows_per_tile, int mtiles_bound_moe, int N, int KB, bool mo
     // read once (measured slower for MXFP4 x MXFP8, whose MMA runs at half
     // the NVFP4 rate)
     if (moe && bs == BS_NV && rows_per_tile > 96 && rows_per_tile <= 160) t.bnt = 192;
+    // dense NVFP4 from 1024 rows: 192-token tiles (1.5 x the MMA work per
+    // stage for 1.25 x the operand bytes; M = 8192 at N = K = 7168: 383 ->
+    // 344 us; at 256 rows the ragged second tile made it slower)
+    if (!moe && bs == BS_NV && rows_per_tile >= 1024) t.bnt = 192;
     KB /= (bs == BS_NV ? 4 : bs == BS_MX ? 2 : 1);
   }
   t.ntw = (N + TILE_N - 1) / TILE_N;

@@ -177,6 +177,10 @@ def test_host_dispatch_plans():
     assert (mx["kernel"], mx["layout"], mx["token_tile"]) == (2, 1, 128)
     nv = p(cdesc("nvfp4", "nvfp4"), None, 1, 7168, 7168)
     assert (nv["kernel"], nv["layout"], nv["token_tile"]) == (2, 2, 16)
+    # dense NVFP4 from 1024 rows: 192-token tiles (a ragged last one at M = 8192)
+    nv8k = p(cdesc("nvfp4", "nvfp4"), None, 8192, 7168, 7168)
+    assert (nv8k["token_tile"], nv8k["token_tiles"]) == (192, 43)
+    assert p(cdesc("nvfp4", "nvfp4"), None, 256, 7168, 7168)["token_tile"] == 128
     # other quantised pairs decode the activations and keep the dequantisation layout
     assert p(cdesc("nvfp4", "fp8"), None, 8192, 7168, 7168)["layout"] == 0
     # FP8 x FP8: 256-token tiles only with at least two per SM, else 128; K % 128 != 0 keeps the old layout
