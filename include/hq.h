@@ -317,7 +317,8 @@ HQ_API hq_status hq_moe_permute(int T, int topk, int E, const int32_t *topk_ids,
  *   mode HQ_MOE_INDEXED: no copy; the GEMM reads each token tile's rows
  *       straight from `a` (or from its quantised or decoded copy, which has
  *       the caller's T or T * topk rows, not the routed T * topk) through
- *       the routing index, four rows per tensor-memory-access gather.
+ *       the routing index, four rows per TMA (tensor memory accelerator)
+ *       gather instruction.
  *   combine == 0: out = Y bf16 [T * topk, N] in slot order.
  *   combine == 1: out bf16 [T, N],
  *       out[t] = routed_scale * sum_j topk_weights[t, j] * Y[t * topk + j]
